@@ -1,0 +1,432 @@
+/*
+ * q4_oracle.c -- plain, slow, scalar CPU oracle for 4-bit block-scaled
+ * quantization, first-order Sigma-Delta requantization and the W4A4 GEMM.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the parity reference that the CUDA
+ * path is checked against.  Only the test-suite, the smoke check and the CPU
+ * baseline leg of the benchmark load it.  The product library never links,
+ * calls or falls back to it, and it shares no code, header, table or constant
+ * generator with the CUDA sources.
+ *
+ * Arithmetic rules: every floating-point step is a single IEEE-754 binary32
+ * operation in round-to-nearest-even, in the order written, compiled with
+ * -ffp-contract=off and without fast-math (x86-64 SSE arithmetic).  The GEMM is
+ * a triple loop in binary64 over exactly decoded operands.  Codecs are written
+ * as brute-force searches over every code, so that "nearest" is checked by eye.
+ *
+ * Sources (web pages, cited by title and section):
+ *  [LT]  "Looped Transformer quantization: error propagation, NVFP4 and
+ *        Sigma-Delta modulation" (mer.dev/posts/loopquant-fp4):
+ *        sec. 0.2 (NVFP4 precision split: E2M1 grid, two-level scaling),
+ *        sec. 2.1 (first-order Sigma-Delta recursion), sec. 2.2 (residue bound,
+ *        4/6 block scale rounded up, s_tensor = max|W|/(6*256)), sec. 2.5
+ *        (implementation details: block_scale_46, x = W/s, r = 0, v = x + r,
+ *        q = e2m1_round(v), r = v - q).
+ *  [GDN] "Why Gated DeltaNet Survives 4-Bit Quantization: NVFP4 W4A4 for the
+ *        Recurrent Half of a Hybrid 27B LLM", prerequisites "NVFP4 and W4A4
+ *        quantization" (16-element blocks, E4M3 scale = block max / 6, FP32
+ *        per-tensor scale, GEMM on native 4-bit tensor cores).
+ *  [MQ]  "MACaQ: Fast, Model Agnostic Calibrated Quantization for Low-Precision
+ *        Weights and Activations", prerequisites "MXFP4 microscaling format"
+ *        (B = 32, shared E8M0 power-of-two scale, E2M1 elements) and "basis
+ *        transform quantization"; core method steps (i) per-channel balancing
+ *        scale and (ii) block Hadamard rotation of size 32, y = [(x.t)B] W'^T.
+ *
+ * Readings where the pages are silent (each one listed in the design notes):
+ *  R1 E2M1 rounding ties go to the code with an even mantissa bit; magnitudes
+ *     above 6 (and +-inf) saturate to 6; the sign bit is the sign bit of the
+ *     input, so a negative value that rounds to zero gives code 0x8.
+ *  R2 NVFP4 block scale: sbf = amax / (6 * s_t), two binary32 operations in
+ *     that order, then E4M3 with round-to-nearest-even (mode RN) or round-up
+ *     (mode RU, the "rounded up" candidate of [LT] sec. 2.2), saturating at 448.
+ *  R3 Elements are normalised by one reciprocal per block: S = dec(sb) * s_t,
+ *     inv = 1 / S, v = x * inv.  If S is 0, or inv is not finite, or s_t is not
+ *     a positive finite number, the block is degenerate and its normalised
+ *     values are taken as +0.
+ *  R4 MXFP4 shared exponent (mode RN): e = floor(log2(amax)) - 2, the OCP rule
+ *     (emax of E2M1 is 2), clamped to [-127, 127]; mode RU takes the smallest e
+ *     with amax <= 6 * 2^e, so that nothing saturates (needed by Sigma-Delta).
+ *     amax = 0 gives byte 0x00.
+ *  R5 Optional MXFP4 transforms in this order: y = x * c (binary32), then the
+ *     unnormalised Walsh-Hadamard butterflies over each 32-block in Sylvester
+ *     order (strides 1, 2, 4, 8, 16; (a, b) -> (a + b, a - b)), then a
+ *     multiplication by binary32(1/sqrt(32)).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stddef.h>
+#include <string.h>
+
+#define Q4O_NVFP4 0
+#define Q4O_MXFP4 1
+
+/* ------------------------------------------------------------------------ */
+/* E2M1 element code ([LT] sec. 0.2; [GDN] prerequisites; [MQ] MXFP4 format) */
+/* 1 sign bit, 2 exponent bits, 1 mantissa bit.  Positive magnitudes, in code */
+/* order 0..7: 0, 0.5, 1, 1.5, 2, 3, 4, 6.                                   */
+/* ------------------------------------------------------------------------ */
+static const double E2M1_MAG[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+double q4o_e2m1_decode(uint8_t code)
+{
+    double m = E2M1_MAG[code & 7u];
+    return (code & 8u) ? -m : m;
+}
+
+/* Nearest magnitude by exhaustive search (R1).  Two grid points can only tie
+ * when they are neighbours, and neighbours differ in mantissa parity, so "on a
+ * tie take the even code" picks the even-mantissa neighbour. */
+uint8_t q4o_e2m1_encode(float v)
+{
+    int neg = signbit(v) ? 1 : 0;
+    double a = fabs((double)v);
+    int best = 0;
+    if (!(a <= 6.0)) {            /* > 6, +inf: saturate */
+        best = 7;
+    } else {
+        double bestd = a;
+        for (int c = 1; c < 8; ++c) {
+            double d = fabs(a - E2M1_MAG[c]);
+            if (d < bestd || (d == bestd && (c & 1) == 0)) { best = c; bestd = d; }
+        }
+    }
+    return (uint8_t)((neg << 3) | best);
+}
+
+/* ------------------------------------------------------------------------ */
+/* E4M3 (finite-only "fn" variant): bias 7, no infinities, 0x7F/0xFF NaN,    */
+/* largest finite 448, subnormals down to 2^-9.  Block-scale type of NVFP4.  */
+/* ------------------------------------------------------------------------ */
+double q4o_e4m3_decode(uint8_t b)
+{
+    int s = (b >> 7) & 1, e = (b >> 3) & 15, m = b & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m, -9);            /* m/8 * 2^-6 */
+    else v = ldexp(1.0 + m / 8.0, e - 7);
+    return s ? -v : v;
+}
+
+/* Encode a non-negative binary32 scale (R2).  round_up = 0: nearest, ties to
+ * even code; round_up = 1: smallest code whose value is >= v.  Both saturate
+ * at 448 (code 0x7E); v <= 0 gives 0x00. */
+uint8_t q4o_e4m3_encode(float v, int round_up)
+{
+    double a = (double)v;
+    if (!(a > 0.0)) return 0x00;
+    if (!(a < 448.0)) return 0x7E;
+    int best = 0;
+    if (round_up) {
+        for (int c = 0; c <= 0x7E; ++c)
+            if (q4o_e4m3_decode((uint8_t)c) >= a) { best = c; break; }
+    } else {
+        double bestd = a;
+        for (int c = 1; c <= 0x7E; ++c) {
+            double d = fabs(a - q4o_e4m3_decode((uint8_t)c));
+            if (d < bestd || (d == bestd && (c & 1) == 0)) { best = c; bestd = d; }
+        }
+    }
+    return (uint8_t)best;
+}
+
+/* ------------------------------------------------------------------------ */
+/* E8M0: unsigned power-of-two scale, value 2^(byte - 127), 0xFF is NaN.     */
+/* ([MQ] prerequisites, MXFP4 microscaling format.)                          */
+/* ------------------------------------------------------------------------ */
+double q4o_e8m0_decode(uint8_t b)
+{
+    if (b == 0xFF) return NAN;
+    return ldexp(1.0, (int)b - 127);
+}
+
+/* Shared exponent of a 32-block (R4).  Returns e; the stored byte is e+127. */
+int q4o_mx_exponent(float amax, int round_up)
+{
+    if (!(amax > 0.0f)) return -127;
+    int ex;
+    (void)frexpf(amax, &ex);          /* amax = f * 2^ex, f in [0.5, 1) */
+    int e = (ex - 1) - 2;             /* floor(log2 amax) - emax(E2M1)  */
+    if (round_up && ldexp((double)amax, -e) > 6.0) e += 1;
+    if (e < -127) e = -127;
+    if (e > 127) e = 127;
+    return e;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Tensor amax and per-tensor FP32 scale ([LT] sec. 2.2: s_tensor =         */
+/* max|W| / (6*256) for looped weights; the activation recipe uses           */
+/* amax / (6*448)).  denom is the product written as one binary32 constant.  */
+/* ------------------------------------------------------------------------ */
+float q4o_amax(const float* x, int64_t n)
+{
+    float m = 0.0f;
+    for (int64_t i = 0; i < n; ++i) {
+        float a = fabsf(x[i]);
+        if (a > m) m = a;
+    }
+    return m;
+}
+
+float q4o_tensor_scale(float amax, float denom)
+{
+    return amax / denom;
+}
+
+/* ------------------------------------------------------------------------ */
+/* NVFP4 two-level block quantization ([LT] sec. 0.2; [GDN] prerequisites): */
+/* 16 contiguous elements along a row share one E4M3 scale of about block    */
+/* max / 6, under the FP32 tensor scale s_t.  Codes are packed two per byte, */
+/* element 2i in the low nibble.  Scales are written row-major [rows, cols/16]. */
+/* Returns 0, or -1 for an invalid shape.                                    */
+/* ------------------------------------------------------------------------ */
+static int block_is_degenerate(float S, float inv, float s_t)
+{
+    return !(s_t > 0.0f) || !isfinite(s_t) || S == 0.0f || !isfinite(inv);
+}
+
+int q4o_nvfp4_quantize(const float* x, int64_t rows, int64_t cols, float s_t,
+                       int round_up, uint8_t* codes, uint8_t* scales)
+{
+    if (rows < 0 || cols < 0 || cols % 16 != 0) return -1;
+    const int64_t nb = cols / 16;
+    for (int64_t i = 0; i < rows; ++i) {
+        const float* xr = x + i * cols;
+        for (int64_t b = 0; b < nb; ++b) {
+            const float* xb = xr + b * 16;
+            float amax = 0.0f;
+            for (int j = 0; j < 16; ++j) {
+                float a = fabsf(xb[j]);
+                if (a > amax) amax = a;
+            }
+            uint8_t sb = 0;
+            if (s_t > 0.0f && isfinite(s_t)) {
+                float denom = 6.0f * s_t;              /* R2, first op  */
+                float sbf = amax / denom;              /* R2, second op */
+                sb = q4o_e4m3_encode(sbf, round_up);
+            }
+            float S = (float)q4o_e4m3_decode(sb) * s_t;  /* R3 */
+            float inv = 1.0f / S;
+            int degenerate = block_is_degenerate(S, inv, s_t);
+            scales[i * nb + b] = sb;
+            for (int j = 0; j < 16; ++j) {
+                float v = degenerate ? 0.0f : xb[j] * inv;
+                uint8_t c = q4o_e2m1_encode(v);
+                int64_t k = b * 16 + j;
+                uint8_t* dst = codes + i * (cols / 2) + k / 2;
+                if ((k & 1) == 0) *dst = (uint8_t)((*dst & 0xF0u) | c);
+                else *dst = (uint8_t)((*dst & 0x0Fu) | (uint8_t)(c << 4));
+            }
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* 32-point Walsh-Hadamard transform, Sylvester order, unnormalised (R5).    */
+/* ([MQ] basis transform quantization; step (ii) block Hadamard of size 32.) */
+/* ------------------------------------------------------------------------ */
+void q4o_fwht32(float* v)
+{
+    for (int h = 1; h < 32; h *= 2) {
+        for (int i = 0; i < 32; i += 2 * h) {
+            for (int j = i; j < i + h; ++j) {
+                float a = v[j], b = v[j + h];
+                v[j] = a + b;
+                v[j + h] = a - b;
+            }
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* MXFP4 block quantization ([MQ] MXFP4 format; core method (i), (ii)):      */
+/* per 32-block, optional per-channel multiplier c (t for activations, 1/t   */
+/* for weights), optional block Hadamard, shared E8M0 exponent (R4), E2M1.   */
+/* Scales row-major [rows, cols/32] as E8M0 bytes.                           */
+/* ------------------------------------------------------------------------ */
+/* Transform one 32-block before quantization (R5): y = x * c, then the
+ * normalised block Hadamard.  chan points at the block's 32 multipliers or is
+ * NULL; hadamard = 0 skips the rotation. */
+void q4o_mx_transform(const float* x, const float* chan, int hadamard, float* y)
+{
+    const float inv_sqrt32 = (float)(1.0 / sqrt(32.0));   /* binary32 RN */
+    for (int j = 0; j < 32; ++j) y[j] = chan ? x[j] * chan[j] : x[j];
+    if (hadamard) {
+        q4o_fwht32(y);
+        for (int j = 0; j < 32; ++j) y[j] = y[j] * inv_sqrt32;
+    }
+}
+
+int q4o_mxfp4_quantize(const float* x, int64_t rows, int64_t cols,
+                       const float* chan, int hadamard, int round_up,
+                       uint8_t* codes, uint8_t* scales)
+{
+    if (rows < 0 || cols < 0 || cols % 32 != 0) return -1;
+    const int64_t nb = cols / 32;
+    for (int64_t i = 0; i < rows; ++i) {
+        for (int64_t b = 0; b < nb; ++b) {
+            float y[32];
+            q4o_mx_transform(x + i * cols + b * 32, chan ? chan + b * 32 : NULL, hadamard, y);
+            float amax = 0.0f;
+            for (int j = 0; j < 32; ++j) {
+                float a = fabsf(y[j]);
+                if (a > amax) amax = a;
+            }
+            int e = q4o_mx_exponent(amax, round_up);
+            scales[i * nb + b] = (uint8_t)(e + 127);
+            float mult = ldexpf(1.0f, -e);        /* exact power of two */
+            for (int j = 0; j < 32; ++j) {
+                float v = y[j] * mult;
+                uint8_t c = q4o_e2m1_encode(v);
+                int64_t k = b * 32 + j;
+                uint8_t* dst = codes + i * (cols / 2) + k / 2;
+                if ((k & 1) == 0) *dst = (uint8_t)((*dst & 0xF0u) | c);
+                else *dst = (uint8_t)((*dst & 0x0Fu) | (uint8_t)(c << 4));
+            }
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Tensor-core scale-factor layout.  Rows are padded to a multiple of 128    */
+/* and scale columns to a multiple of 4.  The padded matrix is cut into      */
+/* 128 x 4 atoms of 512 bytes, stored atom-row-major; inside an atom, scale  */
+/* (r, c) sits at byte (r % 32) * 16 + (r / 32) * 4 + c.  Padding is zero.    */
+/* ------------------------------------------------------------------------ */
+int64_t q4o_tc_scale_bytes(int64_t rows, int64_t scols)
+{
+    int64_t rp = (rows + 127) / 128 * 128;
+    int64_t cp = (scols + 3) / 4 * 4;
+    return rp * cp;
+}
+
+int64_t q4o_tc_scale_offset(int64_t r, int64_t c, int64_t scols)
+{
+    int64_t catoms = (scols + 3) / 4;
+    int64_t atom = (r / 128) * catoms + (c / 4);
+    int64_t rr = r % 128, cc = c % 4;
+    return atom * 512 + (rr % 32) * 16 + (rr / 32) * 4 + cc;
+}
+
+void q4o_scales_to_tc(const uint8_t* rowmajor, int64_t rows, int64_t scols, uint8_t* out)
+{
+    memset(out, 0, (size_t)q4o_tc_scale_bytes(rows, scols));
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < scols; ++c)
+            out[q4o_tc_scale_offset(r, c, scols)] = rowmajor[r * scols + c];
+}
+
+void q4o_scales_from_tc(const uint8_t* tc, int64_t rows, int64_t scols, uint8_t* rowmajor)
+{
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < scols; ++c)
+            rowmajor[r * scols + c] = tc[q4o_tc_scale_offset(r, c, scols)];
+}
+
+/* ------------------------------------------------------------------------ */
+/* Decoded value of one element: code * block scale (* tensor scale).       */
+/* ------------------------------------------------------------------------ */
+static double block_scale_value(int format, uint8_t sb)
+{
+    return format == Q4O_NVFP4 ? q4o_e4m3_decode(sb) : q4o_e8m0_decode(sb);
+}
+
+static uint8_t code_at(const uint8_t* codes, int64_t cols, int64_t i, int64_t k)
+{
+    uint8_t byte = codes[i * (cols / 2) + k / 2];
+    return (k & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 0x0F);
+}
+
+/* Fake quantization ([GDN] quantize-then-dequantize): out = code * s_b * s_t
+ * in binary64 (exact).  s_t is ignored for MXFP4. */
+int q4o_dequantize(int format, const uint8_t* codes, const uint8_t* scales,
+                   float s_t, int64_t rows, int64_t cols, double* out)
+{
+    int blk = format == Q4O_NVFP4 ? 16 : 32;
+    if (cols % blk != 0) return -1;
+    int64_t nb = cols / blk;
+    for (int64_t i = 0; i < rows; ++i)
+        for (int64_t k = 0; k < cols; ++k) {
+            double v = q4o_e2m1_decode(code_at(codes, cols, i, k))
+                     * block_scale_value(format, scales[i * nb + k / blk]);
+            if (format == Q4O_NVFP4) v *= (double)s_t;
+            out[i * cols + k] = v;
+        }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* One loop visit of first-order Sigma-Delta requantization ([LT] sec. 2.1  */
+/* and the code of sec. 2.5): with the block scale fixed, x = W / s,         */
+/* v_k = x + r_{k-1}, q_k = Q(v_k) (nearest E2M1, saturating), r_k = v_k - q_k.*/
+/* The caller zeroes r before the first visit (r_0 = 0).  x is formed with   */
+/* the per-block reciprocal of R3.  Scales row-major; s_t ignored for MXFP4. */
+/* ------------------------------------------------------------------------ */
+int q4o_sigma_delta_step(int format, const float* w, int64_t rows, int64_t cols,
+                         const uint8_t* scales, float s_t, float* r, uint8_t* codes)
+{
+    int blk = format == Q4O_NVFP4 ? 16 : 32;
+    if (cols % blk != 0) return -1;
+    int64_t nb = cols / blk;
+    for (int64_t i = 0; i < rows; ++i) {
+        for (int64_t b = 0; b < nb; ++b) {
+            uint8_t sb = scales[i * nb + b];
+            float inv;
+            int degenerate;
+            if (format == Q4O_NVFP4) {
+                float S = (float)q4o_e4m3_decode(sb) * s_t;
+                inv = 1.0f / S;
+                degenerate = block_is_degenerate(S, inv, s_t);
+            } else {
+                inv = ldexpf(1.0f, 127 - (int)sb);   /* 2^-e, exact */
+                degenerate = 0;
+            }
+            for (int j = 0; j < blk; ++j) {
+                int64_t k = b * blk + j;
+                int64_t idx = i * cols + k;
+                float x = degenerate ? 0.0f : w[idx] * inv;
+                float v = x + r[idx];
+                uint8_t c = q4o_e2m1_encode(v);
+                r[idx] = v - (float)q4o_e2m1_decode(c);
+                uint8_t* dst = codes + i * (cols / 2) + k / 2;
+                if ((k & 1) == 0) *dst = (uint8_t)((*dst & 0xF0u) | c);
+                else *dst = (uint8_t)((*dst & 0x0Fu) | (uint8_t)(c << 4));
+            }
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* W4A4 GEMM Y = X W^T over decoded operands ([GDN] prerequisites: W4A4 GEMM */
+/* on 4-bit operands; [MQ] inference layer y = x_q W_q^T).  Triple loop in   */
+/* binary64; alpha = s_tA * s_tB for NVFP4 and 1 for MXFP4.  If row_idx is   */
+/* non-NULL only those n_rows rows of Y are computed (Y is n_rows x N).      */
+/* ------------------------------------------------------------------------ */
+int q4o_gemm(int format, int64_t M, int64_t N, int64_t K,
+             const uint8_t* a_codes, const uint8_t* a_scales, float a_st,
+             const uint8_t* b_codes, const uint8_t* b_scales, float b_st,
+             const int64_t* row_idx, int64_t n_rows, double* y)
+{
+    int blk = format == Q4O_NVFP4 ? 16 : 32;
+    if (K % blk != 0) return -1;
+    int64_t nb = K / blk;
+    double alpha = format == Q4O_NVFP4 ? (double)a_st * (double)b_st : 1.0;
+    int64_t nr = row_idx ? n_rows : M;
+    for (int64_t ii = 0; ii < nr; ++ii) {
+        int64_t i = row_idx ? row_idx[ii] : ii;
+        for (int64_t j = 0; j < N; ++j) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                double a = q4o_e2m1_decode(code_at(a_codes, K, i, k))
+                         * block_scale_value(format, a_scales[i * nb + k / blk]);
+                double b = q4o_e2m1_decode(code_at(b_codes, K, j, k))
+                         * block_scale_value(format, b_scales[j * nb + k / blk]);
+                acc += a * b;
+            }
+            y[ii * N + j] = alpha * acc;
+        }
+    }
+    return 0;
+}
