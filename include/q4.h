@@ -1,0 +1,216 @@
+/*
+ * q4.h -- C ABI of libq4: 4-bit block-scaled quantization (NVFP4, MXFP4),
+ * first-order Sigma-Delta requantization and the block-scaled W4A4 GEMM on
+ * NVIDIA B200 (sm_100a).
+ *
+ * Conventions shared by every entry point
+ *   - Pointers named d_* and every tensor argument are DEVICE pointers on the
+ *     current CUDA device.  The caller owns all memory; the library allocates
+ *     nothing persistent and keeps no pointer after a call returns.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Work is enqueued asynchronously on it; nothing synchronises
+ *     the host except q4_get_device_error().
+ *   - Every tensor pointer must be 16-byte aligned.  Matrices are row-major.
+ *   - Inputs must be finite (no NaN, no inf); results for non-finite inputs
+ *     are unspecified.
+ *   - Argument errors are detected on the host before any launch and
+ *     returned as a q4_status; no launch happens then.  A CUDA launch error is
+ *     returned as Q4_ERR_CUDA (q4_last_error() gives the CUDA message).
+ *     Device-side faults of the library's own bounded waits are recorded in a
+ *     device error word and reported by q4_get_device_error().
+ *
+ * Formats (element codes are E2M1: 1 sign, 2 exponent, 1 mantissa bit;
+ * magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6):
+ *   Q4_NVFP4: blocks of 16 consecutive elements along a row share an E4M3
+ *             block scale of about block-max / 6, times one FP32 tensor scale
+ *             s_t ("Looped Transformer quantization", sec. 0.2 "NVFP4
+ *             precision split"; "Why Gated DeltaNet Survives 4-Bit
+ *             Quantization", prerequisites "NVFP4 and W4A4 quantization").
+ *   Q4_MXFP4: blocks of 32 share an E8M0 power-of-two scale, no tensor scale
+ *             ("MACaQ", prerequisites "MXFP4 microscaling format").
+ *
+ * Packed codes: [rows, cols/2] bytes, element 2i in the low nibble of byte i
+ * of its row, element 2i+1 in the high nibble.
+ *
+ * Scale layouts (flag bit Q4_LAYOUT_TC):
+ *   row-major : [rows, cols/block] bytes.
+ *   Q4_LAYOUT_TC (tensor-core layout): rows padded to a multiple of 128,
+ *       scale columns to a multiple of 4; the padded matrix is cut into
+ *       128 x 4 atoms of 512 bytes stored atom-row-major (all atoms of rows
+ *       0..127 first); inside an atom scale (r, c) is byte
+ *       (r % 32) * 16 + ((r / 32) % 4) * 4 + (c % 4).  Padding bytes are 0.
+ *       This is the layout the GEMM reads.  q4_scale_bytes() gives the size.
+ */
+#ifndef Q4_H_
+#define Q4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define Q4_API __attribute__((visibility("default")))
+#else
+#define Q4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { Q4_NVFP4 = 0, Q4_MXFP4 = 1 } q4_format;
+typedef enum { Q4_F32 = 0, Q4_BF16 = 1 } q4_dtype;
+
+typedef enum {
+    Q4_OK = 0,
+    Q4_ERR_ARG = 1,          /* NULL pointer, bad enum, negative size        */
+    Q4_ERR_ALIGN = 2,        /* pointer or row stride not 16-byte aligned     */
+    Q4_ERR_SHAPE = 3,        /* size not a multiple the operation needs       */
+    Q4_ERR_UNSUPPORTED = 4,  /* valid request this build does not implement   */
+    Q4_ERR_CUDA = 5,         /* a CUDA call failed (see q4_last_error)        */
+    Q4_ERR_TIMEOUT = 6,      /* a bounded device wait ran out                 */
+    Q4_ERR_WORKSPACE = 7     /* workspace missing or too small                */
+} q4_status;
+
+/* Flag bits for quantize / dequantize / sigma-delta. */
+enum {
+    Q4_SCALE_RU = 1,     /* round block scales up (NVFP4: E4M3 toward +inf;
+                            MXFP4: smallest exponent with block max <= 6*2^e) */
+    Q4_LAYOUT_TC = 2,    /* scales in the tensor-core layout (else row-major) */
+    Q4_HADAMARD32 = 4    /* MXFP4 only: block Hadamard-32 before quantizing   */
+};
+
+/* Kinds of GEMM left operand. */
+enum {
+    Q4_A_QUANTIZED = 0,  /* a = packed codes [M, K/2], a_scales in TC layout  */
+    Q4_A_BF16 = 1        /* a = bf16 [M, K]; quantized inside the call with
+                            the tensor scale *d_a_gscale (NVFP4 only)         */
+};
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+Q4_API int q4_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+Q4_API const char* q4_status_string(q4_status s);
+
+/* Message of the last CUDA error seen by this thread's calls (static, never NULL). */
+Q4_API const char* q4_last_error(void);
+
+/* Bytes of the scale array of a rows x cols tensor in `format` with the given
+ * layout flags (only Q4_LAYOUT_TC matters).  0 for invalid sizes. */
+Q4_API size_t q4_scale_bytes(q4_format format, int64_t rows, int64_t cols, int flags);
+
+/*
+ * q4_amax -- tensor maximum magnitude and FP32 tensor scale.
+ *   Computes d_out[0] = max_i |x_i| (exact) and d_out[1] = d_out[0] / denom
+ *   (one binary32 division, round-to-nearest).  denom = 6*448 = 2688 gives the
+ *   activation tensor scale; 6*256 = 1536 the looped-weight scale of
+ *   "Looped Transformer quantization", sec. 2.2 (s_tensor = max|W|/(6*256)).
+ *   x: device, n elements of dtype dt, 16-byte aligned.  d_out: device, 2 floats.
+ *   n = 0 gives 0 and 0.  denom must be finite and > 0.
+ */
+Q4_API q4_status q4_amax(q4_dtype dt, const void* x, int64_t n, float denom, float* d_out,
+                  void* stream);
+
+/*
+ * q4_quantize -- block quantization of a rows x cols matrix.
+ *   NVFP4 ("Looped Transformer quantization", sec. 0.2; "Why Gated DeltaNet
+ *   Survives 4-Bit Quantization", prerequisites): per 16-block,
+ *     amax = max|x|,  s_b = E4M3(amax / (6 * s_t))   [RN, or RU with Q4_SCALE_RU],
+ *     S = s_b * s_t,  inv = 1 / S,  code_i = E2M1(x_i * inv)  (nearest, ties to
+ *     even mantissa, saturating at +-6, sign kept for values that round to 0);
+ *     a block whose S is 0 or whose inv is not finite, and every block when s_t
+ *     is not a positive finite number, gets code 0.
+ *   MXFP4 ("MACaQ", prerequisites "MXFP4 microscaling format" and core method
+ *   steps (i)-(ii), y = [(x . t) B]_MXFP4): per 32-block,
+ *     y_j = x_j * c_j (if d_chan), then if Q4_HADAMARD32 the Sylvester-order
+ *     Walsh-Hadamard butterflies (strides 1,2,4,8,16) times fp32(1/sqrt(32)),
+ *     amax = max|y|,  e = floor(log2 amax) - 2 (RN) or the smallest e with
+ *     amax <= 6 * 2^e (RU), clamped to [-127, 127];  byte = e + 127 (0 if
+ *     amax = 0);  code_j = E2M1(y_j * 2^-e).
+ *   block: 16 for NVFP4, 32 for MXFP4 (anything else -> Q4_ERR_UNSUPPORTED).
+ *   in_dt: Q4_BF16 or Q4_F32.  x: device [rows, ld] elements, ld >= cols,
+ *   ld * elem_size a multiple of 16.  cols % block == 0.
+ *   d_gscale: device pointer to s_t (NVFP4, required); must be NULL for MXFP4.
+ *   d_chan: device float[cols] multipliers c (MXFP4 only, optional, NULL = 1).
+ *   codes: device [rows, cols/2] bytes.  scales: device, q4_scale_bytes() bytes.
+ *   flags: Q4_SCALE_RU | Q4_LAYOUT_TC | Q4_HADAMARD32.
+ */
+Q4_API q4_status q4_quantize(q4_format format, int block, q4_dtype in_dt, const void* x,
+                      int64_t rows, int64_t cols, int64_t ld,
+                      const float* d_gscale, const float* d_chan,
+                      uint8_t* codes, uint8_t* scales, int flags, void* stream);
+
+/*
+ * q4_dequantize -- fake quantization, the inverse map ("Why Gated DeltaNet
+ *   Survives 4-Bit Quantization", quantize-then-dequantize probes):
+ *   out = code * s_b * s_t (NVFP4) or code * 2^e (MXFP4), formed in binary32
+ *   (one rounding) and, for Q4_BF16 output, then rounded to bf16.
+ *   codes/scales as written by q4_quantize with the same flags (only
+ *   Q4_LAYOUT_TC matters).  out: device [rows, cols] of out_dt.
+ */
+Q4_API q4_status q4_dequantize(q4_format format, int block, const uint8_t* codes,
+                        const uint8_t* scales, const float* d_gscale,
+                        int64_t rows, int64_t cols, int flags,
+                        q4_dtype out_dt, void* out, void* stream);
+
+/*
+ * q4_sigma_delta_step -- one loop visit of first-order Sigma-Delta
+ *   requantization ("Looped Transformer quantization", sec. 2.1, and the code
+ *   of sec. 2.5): with the block scales fixed,
+ *     x = w * inv (inv = 1/(s_b*s_t) per NVFP4 block, 2^-e per MXFP4 block),
+ *     v = x + r,  q = E2M1(v),  r <- v - q,  codes <- q.
+ *   Start a chain by zeroing r (r_0 = 0).  Scales normally come from
+ *   q4_quantize with Q4_SCALE_RU and s_t = max|W| / (6*256), which keeps
+ *   |x| <= 6 and hence |r| <= 1 (sec. 2.2).
+ *   w: device float [rows, cols] (dense).  scales: device, layout per flags
+ *   (Q4_LAYOUT_TC or row-major).  d_gscale: s_t (NVFP4) or NULL (MXFP4).
+ *   residue: device float [rows, cols], read and written.  codes: device
+ *   [rows, cols/2].  cols % block == 0.
+ */
+Q4_API q4_status q4_sigma_delta_step(q4_format format, int block, const float* w,
+                              int64_t rows, int64_t cols, const uint8_t* scales,
+                              const float* d_gscale, float* residue, uint8_t* codes,
+                              int flags, void* stream);
+
+/*
+ * q4_gemm -- block-scaled FP4 GEMM  Y = alpha * dec(A) dec(B)^T  on the
+ *   tcgen05 tensor cores ("Why Gated DeltaNet Survives 4-Bit Quantization",
+ *   prerequisites: W4A4 runs the GEMM on native 4-bit tensor cores; "MACaQ",
+ *   core method: y = x_q W_q^T).  FP32 accumulation; alpha = s_tA * s_tB for
+ *   NVFP4 and 1 for MXFP4.
+ *   A (M x K): a_kind = Q4_A_QUANTIZED: `a` = codes [M, K/2], a_scales in TC
+ *     layout, d_a_gscale = s_tA (NVFP4) or NULL.  a_kind = Q4_A_BF16 (NVFP4
+ *     only): `a` = bf16 [M, K]; the call quantizes A exactly as q4_quantize
+ *     (RN scales) with s_t = *d_a_gscale; a_scales must be NULL.
+ *   B (N x K, the weight W): b_codes [N, K/2], b_scales in TC layout,
+ *     d_b_gscale = s_tB (NVFP4) or NULL.
+ *   Y: device [M, N] row-major, out_dt Q4_BF16 or Q4_F32.
+ *   K % 64 == 0 (K = 0 writes zeros); N % 8 == 0; M, N >= 0 arbitrary otherwise.
+ *   workspace: device scratch of ws_bytes >= q4_gemm_workspace_size(...)
+ *     (0 bytes for Q4_A_QUANTIZED); its contents on entry do not matter.
+ */
+Q4_API q4_status q4_gemm(q4_format format, int block, int64_t M, int64_t N, int64_t K,
+                  int a_kind, const void* a, const uint8_t* a_scales,
+                  const float* d_a_gscale,
+                  const uint8_t* b_codes, const uint8_t* b_scales,
+                  const float* d_b_gscale,
+                  q4_dtype out_dt, void* y, void* workspace, size_t ws_bytes,
+                  void* stream);
+
+/* Scratch bytes q4_gemm needs for these arguments (0 when none). */
+Q4_API size_t q4_gemm_workspace_size(q4_format format, int64_t M, int64_t N, int64_t K,
+                              int a_kind);
+
+/*
+ * q4_get_device_error -- synchronises `stream`, then reads and clears the
+ *   library's device error word.  Returns Q4_ERR_TIMEOUT if a bounded wait
+ *   inside a GEMM kernel gave up since the last call, Q4_ERR_CUDA if the
+ *   synchronisation itself failed, else Q4_OK.
+ */
+Q4_API q4_status q4_get_device_error(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* Q4_H_ */

@@ -1,0 +1,201 @@
+"""mxfp4_w4a4_block_b200 -- 4-bit block-scaled quantization and the W4A4 GEMM
+on B200 (sm_100a).
+
+This module is a thin ctypes binding of the C-ABI library ``libq4.so``
+(declared in ``include/q4.h``): it marshals torch tensors (device memory and
+the current CUDA stream) into pointers and sizes and checks the returned
+status.  Every step of the computation runs in the library's CUDA kernels;
+there is no CPU fallback, and importing fails loudly if the library has not
+been built (``python -m mxfp4_w4a4_block_b200.build``).
+
+Function names mirror the C entry points: q4_amax, q4_quantize,
+q4_dequantize, q4_sigma_delta_step, q4_gemm, q4_gemm_workspace_size,
+q4_get_device_error, q4_scale_bytes.
+"""
+from __future__ import annotations
+
+import ctypes
+from pathlib import Path
+
+import torch
+
+NVFP4 = 0
+MXFP4 = 1
+F32 = 0
+BF16 = 1
+
+SCALE_RU = 1
+LAYOUT_TC = 2
+HADAMARD32 = 4
+
+A_QUANTIZED = 0
+A_BF16 = 1
+
+BLOCK = {NVFP4: 16, MXFP4: 32}
+
+STATUS = {0: "ok", 1: "invalid argument", 2: "alignment", 3: "shape", 4: "unsupported",
+          5: "CUDA error", 6: "device wait timed out", 7: "workspace"}
+
+LIB_PATH = Path(__file__).resolve().parent / "libq4.so"
+
+# ctypes signatures of include/q4.h
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_I = ctypes.c_int
+_F = ctypes.c_float
+_SZ = ctypes.c_size_t
+SIGNATURES = {
+    "q4_version": (_I, []),
+    "q4_status_string": (ctypes.c_char_p, [_I]),
+    "q4_last_error": (ctypes.c_char_p, []),
+    "q4_scale_bytes": (_SZ, [_I, _I64, _I64, _I]),
+    "q4_amax": (_I, [_I, _P, _I64, _F, _P, _P]),
+    "q4_quantize": (_I, [_I, _I, _I, _P, _I64, _I64, _I64, _P, _P, _P, _P, _I, _P]),
+    "q4_dequantize": (_I, [_I, _I, _P, _P, _P, _I64, _I64, _I, _I, _P, _P]),
+    "q4_sigma_delta_step": (_I, [_I, _I, _P, _I64, _I64, _P, _P, _P, _P, _I, _P]),
+    "q4_gemm": (_I, [_I, _I, _I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _P, _I, _P, _P, _SZ, _P]),
+    "q4_gemm_workspace_size": (_SZ, [_I, _I64, _I64, _I64, _I]),
+    "q4_get_device_error": (_I, [_P]),
+}
+
+_lib = None
+
+
+class Q4Error(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        msg = STATUS.get(status, str(status))
+        if status == 5 and _lib is not None:
+            msg += ": " + _lib.q4_last_error().decode()
+        super().__init__(f"{fn} failed: {msg}")
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C-ABI library; raises if it is missing (there is no fallback)."""
+    global _lib
+    if _lib is None:
+        if not LIB_PATH.exists():
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m mxfp4_w4a4_block_b200.build`")
+        L = ctypes.CDLL(str(LIB_PATH))
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(fn: str, status: int) -> None:
+    if status != 0:
+        raise Q4Error(fn, status)
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+# ------------------------------------------------------------------ sizes
+def q4_scale_bytes(fmt: int, rows: int, cols: int, flags: int = LAYOUT_TC) -> int:
+    return int(lib().q4_scale_bytes(fmt, rows, cols, flags))
+
+
+def q4_gemm_workspace_size(fmt: int, M: int, N: int, K: int, a_kind: int) -> int:
+    return int(lib().q4_gemm_workspace_size(fmt, M, N, K, a_kind))
+
+
+# ------------------------------------------------------------------ ops
+def q4_amax(x: torch.Tensor, denom: float, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """out[0] = max|x|, out[1] = out[0] / denom (device float32[2])."""
+    if out is None:
+        out = torch.empty(2, dtype=torch.float32, device=x.device)
+    _check("q4_amax", lib().q4_amax(_dtype_code(x), _ptr(x), x.numel(), float(denom), _ptr(out),
+                                    _stream(stream)))
+    return out
+
+
+def q4_quantize(fmt: int, x: torch.Tensor, gscale: torch.Tensor | None = None,
+                chan: torch.Tensor | None = None, flags: int = LAYOUT_TC,
+                codes: torch.Tensor | None = None, scales: torch.Tensor | None = None,
+                stream=None, block: int | None = None):
+    """Quantize a 2-D bf16/fp32 tensor; returns (codes, scales)."""
+    rows, cols = x.shape
+    ld = x.stride(0) if x.dim() == 2 and x.stride(1) == 1 else cols
+    if codes is None:
+        codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(max(q4_scale_bytes(fmt, rows, cols, flags), 1), dtype=torch.uint8,
+                             device=x.device)
+    blk = BLOCK[fmt] if block is None else block
+    st = lib().q4_quantize(fmt, blk, _dtype_code(x), _ptr(x), rows, cols, ld, _ptr(gscale), _ptr(chan),
+                           _ptr(codes), _ptr(scales), flags, _stream(stream))
+    _check("q4_quantize", st)
+    return codes, scales
+
+
+def q4_dequantize(fmt: int, codes: torch.Tensor, scales: torch.Tensor, rows: int, cols: int,
+                  gscale: torch.Tensor | None = None, flags: int = LAYOUT_TC,
+                  out_dtype=torch.float32, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    if out is None:
+        out = torch.empty((rows, cols), dtype=out_dtype, device=codes.device)
+    st = lib().q4_dequantize(fmt, BLOCK[fmt], _ptr(codes), _ptr(scales), _ptr(gscale), rows, cols, flags,
+                             _dtype_code(out), _ptr(out), _stream(stream))
+    _check("q4_dequantize", st)
+    return out
+
+
+def q4_sigma_delta_step(fmt: int, w: torch.Tensor, scales: torch.Tensor, residue: torch.Tensor,
+                        gscale: torch.Tensor | None = None, flags: int = LAYOUT_TC,
+                        codes: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """One loop visit: updates `residue` in place and returns the visit's codes."""
+    rows, cols = w.shape
+    if codes is None:
+        codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=w.device)
+    st = lib().q4_sigma_delta_step(fmt, BLOCK[fmt], _ptr(w), rows, cols, _ptr(scales), _ptr(gscale),
+                                   _ptr(residue), _ptr(codes), flags, _stream(stream))
+    _check("q4_sigma_delta_step", st)
+    return codes
+
+
+def q4_gemm(fmt: int, M: int, N: int, K: int, a: torch.Tensor, a_scales, a_gscale,
+            b_codes: torch.Tensor, b_scales: torch.Tensor, b_gscale,
+            out_dtype=torch.bfloat16, a_kind: int = A_QUANTIZED, y: torch.Tensor | None = None,
+            workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Y[M, N] = alpha * dec(A) dec(B)^T on the tensor cores."""
+    dev = b_codes.device
+    if y is None:
+        y = torch.empty((M, N), dtype=out_dtype, device=dev)
+    ws_need = q4_gemm_workspace_size(fmt, M, N, K, a_kind)
+    if workspace is None and ws_need > 0:
+        workspace = torch.empty(ws_need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().q4_gemm(fmt, BLOCK[fmt], M, N, K, a_kind, _ptr(a), _ptr(a_scales), _ptr(a_gscale),
+                       _ptr(b_codes), _ptr(b_scales), _ptr(b_gscale), _dtype_code(y), _ptr(y),
+                       _ptr(workspace), ws_bytes, _stream(stream))
+    _check("q4_gemm", st)
+    return y
+
+
+def q4_get_device_error(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device error status."""
+    return int(lib().q4_get_device_error(_stream(stream)))

@@ -1,0 +1,209 @@
+// q4_api.cu -- the extern "C" entry points declared in include/q4.h: argument
+// validation on the host, then one or more kernel launches on the caller's
+// stream.  No entry point allocates device memory.
+#include <cstdint>
+#include <cstring>
+#include <cuda_runtime.h>
+
+#include "../../include/q4.h"
+#include "q4_internal.h"
+
+
+namespace {
+
+thread_local char g_last_error[256] = "no error";
+
+q4_status cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return Q4_OK;
+    std::strncpy(g_last_error, cudaGetErrorString(e), sizeof(g_last_error) - 1);
+    g_last_error[sizeof(g_last_error) - 1] = '\0';
+    return Q4_ERR_CUDA;
+}
+
+int num_sms() {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int block_of(q4_format f) { return f == Q4_NVFP4 ? 16 : 32; }
+
+bool valid_format(int f) { return f == Q4_NVFP4 || f == Q4_MXFP4; }
+bool valid_dtype(int d) { return d == Q4_F32 || d == Q4_BF16; }
+
+int64_t catoms_of(int64_t cols, int blk) { return ((cols / blk) + 3) / 4; }
+
+}  // namespace
+
+extern "C" {
+
+int q4_version(void) { return 100; }
+
+const char* q4_status_string(q4_status s) {
+    switch (s) {
+        case Q4_OK: return "ok";
+        case Q4_ERR_ARG: return "invalid argument";
+        case Q4_ERR_ALIGN: return "pointer or stride not 16-byte aligned";
+        case Q4_ERR_SHAPE: return "unsupported shape";
+        case Q4_ERR_UNSUPPORTED: return "unsupported request";
+        case Q4_ERR_CUDA: return "CUDA error";
+        case Q4_ERR_TIMEOUT: return "device wait timed out";
+        case Q4_ERR_WORKSPACE: return "workspace missing or too small";
+    }
+    return "unknown status";
+}
+
+const char* q4_last_error(void) { return g_last_error; }
+
+size_t q4_scale_bytes(q4_format format, int64_t rows, int64_t cols, int flags) {
+    if (!valid_format(format) || rows < 0 || cols < 0) return 0;
+    const int blk = block_of(format);
+    if (cols % blk) return 0;
+    const int64_t scols = cols / blk;
+    if (flags & Q4_LAYOUT_TC) return (size_t)(((rows + 127) / 128) * 128 * ((scols + 3) / 4) * 4);
+    return (size_t)(rows * scols);
+}
+
+q4_status q4_amax(q4_dtype dt, const void* x, int64_t n, float denom, float* d_out, void* stream) {
+    if (!valid_dtype(dt) || n < 0 || !d_out || (n > 0 && !x)) return Q4_ERR_ARG;
+    if (!(denom > 0.0f) || !(denom < 3.0e38f)) return Q4_ERR_ARG;
+    if ((x && !aligned16(x)) || (reinterpret_cast<uintptr_t>(d_out) & 3u)) return Q4_ERR_ALIGN;
+    return cuda_status(q4::launch_amax(x, n, dt == Q4_BF16, denom, d_out, (cudaStream_t)stream, num_sms()));
+}
+
+q4_status q4_quantize(q4_format format, int block, q4_dtype in_dt, const void* x, int64_t rows, int64_t cols,
+                      int64_t ld, const float* d_gscale, const float* d_chan, uint8_t* codes, uint8_t* scales,
+                      int flags, void* stream) {
+    if (!valid_format(format) || !valid_dtype(in_dt) || rows < 0 || cols < 0 || ld < cols) return Q4_ERR_ARG;
+    if (block != block_of(format)) return Q4_ERR_UNSUPPORTED;
+    if (flags & ~(Q4_SCALE_RU | Q4_LAYOUT_TC | Q4_HADAMARD32)) return Q4_ERR_ARG;
+    if (format == Q4_NVFP4 && ((flags & Q4_HADAMARD32) || d_chan)) return Q4_ERR_UNSUPPORTED;
+    if (format == Q4_NVFP4 && !d_gscale) return Q4_ERR_ARG;
+    if (format == Q4_MXFP4 && d_gscale) return Q4_ERR_ARG;
+    if (cols % block) return Q4_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return Q4_OK;
+    if (!x || !codes || !scales) return Q4_ERR_ARG;
+    const int esz = in_dt == Q4_BF16 ? 2 : 4;
+    if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || (ld * esz) % 16) return Q4_ERR_ALIGN;
+    if (d_chan && !aligned16(d_chan)) return Q4_ERR_ALIGN;
+    q4::QuantParams p;
+    p.x = x; p.rows = rows; p.cols = cols; p.ld = ld;
+    p.gscale = d_gscale; p.chan = d_chan; p.codes = codes; p.scales = scales;
+    p.scols = cols / block; p.catoms = catoms_of(cols, block);
+    return cuda_status(q4::launch_quantize(p, block, in_dt == Q4_BF16, (flags & Q4_LAYOUT_TC) != 0,
+                                           (flags & Q4_SCALE_RU) != 0, (flags & Q4_HADAMARD32) != 0,
+                                           d_chan != nullptr, (cudaStream_t)stream, num_sms()));
+}
+
+q4_status q4_dequantize(q4_format format, int block, const uint8_t* codes, const uint8_t* scales,
+                        const float* d_gscale, int64_t rows, int64_t cols, int flags, q4_dtype out_dt, void* out,
+                        void* stream) {
+    if (!valid_format(format) || !valid_dtype(out_dt) || rows < 0 || cols < 0) return Q4_ERR_ARG;
+    if (block != block_of(format)) return Q4_ERR_UNSUPPORTED;
+    if (format == Q4_NVFP4 && !d_gscale) return Q4_ERR_ARG;
+    if (cols % block) return Q4_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return Q4_OK;
+    if (!codes || !scales || !out) return Q4_ERR_ARG;
+    if (!aligned16(codes) || !aligned16(out)) return Q4_ERR_ALIGN;
+    q4::DequantParams p;
+    p.codes = codes; p.scales = scales; p.gscale = d_gscale; p.rows = rows; p.cols = cols; p.out = out;
+    p.scols = cols / block; p.catoms = catoms_of(cols, block);
+    return cuda_status(q4::launch_dequantize(p, block, (flags & Q4_LAYOUT_TC) != 0, out_dt == Q4_BF16,
+                                             (cudaStream_t)stream, num_sms()));
+}
+
+q4_status q4_sigma_delta_step(q4_format format, int block, const float* w, int64_t rows, int64_t cols,
+                              const uint8_t* scales, const float* d_gscale, float* residue, uint8_t* codes,
+                              int flags, void* stream) {
+    if (!valid_format(format) || rows < 0 || cols < 0) return Q4_ERR_ARG;
+    if (block != block_of(format)) return Q4_ERR_UNSUPPORTED;
+    if (flags & ~(Q4_LAYOUT_TC)) return Q4_ERR_ARG;
+    if (format == Q4_NVFP4 && !d_gscale) return Q4_ERR_ARG;
+    if (format == Q4_MXFP4 && d_gscale) return Q4_ERR_ARG;
+    if (cols % block) return Q4_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return Q4_OK;
+    if (!w || !scales || !residue || !codes) return Q4_ERR_ARG;
+    if (!aligned16(w) || !aligned16(residue) || !aligned16(codes)) return Q4_ERR_ALIGN;
+    q4::SigmaDeltaParams p;
+    p.w = w; p.rows = rows; p.cols = cols; p.scales = scales; p.gscale = d_gscale;
+    p.residue = residue; p.codes = codes; p.scols = cols / block; p.catoms = catoms_of(cols, block);
+    return cuda_status(q4::launch_sigma_delta(p, block, (flags & Q4_LAYOUT_TC) != 0, (cudaStream_t)stream,
+                                              num_sms()));
+}
+
+size_t q4_gemm_workspace_size(q4_format format, int64_t M, int64_t N, int64_t K, int a_kind) {
+    (void)N;
+    if (a_kind != Q4_A_BF16 || format != Q4_NVFP4 || M <= 0 || K <= 0 || K % 64) return 0;
+    if (q4::fused_decode_supported(M, K)) return 0;
+    // quantize-once: codes [M, K/2] then tensor-core scales, 256-byte aligned
+    const size_t codes = (size_t)M * (size_t)(K / 2);
+    const size_t codes_al = (codes + 255) / 256 * 256;
+    return codes_al + q4_scale_bytes(Q4_NVFP4, M, K, Q4_LAYOUT_TC);
+}
+
+q4_status q4_gemm(q4_format format, int block, int64_t M, int64_t N, int64_t K, int a_kind, const void* a,
+                  const uint8_t* a_scales, const float* d_a_gscale, const uint8_t* b_codes,
+                  const uint8_t* b_scales, const float* d_b_gscale, q4_dtype out_dt, void* y, void* workspace,
+                  size_t ws_bytes, void* stream) {
+    if (!valid_format(format) || !valid_dtype(out_dt) || M < 0 || N < 0 || K < 0) return Q4_ERR_ARG;
+    if (block != block_of(format)) return Q4_ERR_UNSUPPORTED;
+    if (a_kind != Q4_A_QUANTIZED && a_kind != Q4_A_BF16) return Q4_ERR_ARG;
+    if (a_kind == Q4_A_BF16 && format != Q4_NVFP4) return Q4_ERR_UNSUPPORTED;
+    if (format == Q4_NVFP4 && (!d_a_gscale || !d_b_gscale)) return Q4_ERR_ARG;
+    if (format == Q4_MXFP4 && (d_a_gscale || d_b_gscale)) return Q4_ERR_ARG;
+    if (a_kind == Q4_A_BF16 && a_scales) return Q4_ERR_ARG;
+    if (K % 64 || N % 8) return Q4_ERR_SHAPE;
+    if (K > ((int64_t)1 << 30) || M > ((int64_t)1 << 31) || N > ((int64_t)1 << 31)) return Q4_ERR_SHAPE;
+    if (M == 0 || N == 0) return Q4_OK;
+    if (!y) return Q4_ERR_ARG;
+    if (!aligned16(y)) return Q4_ERR_ALIGN;
+    cudaStream_t st = (cudaStream_t)stream;
+    const size_t ysz = (size_t)M * (size_t)N * (out_dt == Q4_BF16 ? 2 : 4);
+    if (K == 0) return cuda_status(cudaMemsetAsync(y, 0, ysz, st));
+    if (!a || !b_codes || !b_scales || (a_kind == Q4_A_QUANTIZED && !a_scales)) return Q4_ERR_ARG;
+    if (!aligned16(a) || !aligned16(b_codes) || !aligned16(b_scales) || (a_scales && !aligned16(a_scales)))
+        return Q4_ERR_ALIGN;
+
+    const uint8_t* a_codes = static_cast<const uint8_t*>(a);
+    if (a_kind == Q4_A_BF16) {
+        if (q4::fused_decode_supported(M, K)) {
+            q4::FusedDecodeParams f;
+            f.M = M; f.N = N; f.K = K; f.a_bf16 = static_cast<const uint16_t*>(a); f.a_gscale = d_a_gscale;
+            f.b_codes = b_codes; f.b_scales = b_scales; f.b_gscale = d_b_gscale; f.y = y;
+            f.out_bf16 = out_dt == Q4_BF16;
+            return cuda_status(q4::launch_fused_decode(f, st, num_sms()));
+        }
+        // larger M: quantize the activations once into the workspace, then the GEMM
+        const size_t need = q4_gemm_workspace_size(format, M, N, K, a_kind);
+        if (!workspace || ws_bytes < need) return Q4_ERR_WORKSPACE;
+        if (!aligned16(workspace)) return Q4_ERR_ALIGN;
+        uint8_t* ws = static_cast<uint8_t*>(workspace);
+        const size_t codes_al = ((size_t)M * (size_t)(K / 2) + 255) / 256 * 256;
+        q4::QuantParams qp;
+        qp.x = a; qp.rows = M; qp.cols = K; qp.ld = K; qp.gscale = d_a_gscale; qp.chan = nullptr;
+        qp.codes = ws; qp.scales = ws + codes_al; qp.scols = K / 16; qp.catoms = catoms_of(K, 16);
+        cudaError_t e = q4::launch_quantize(qp, 16, true, true, false, false, false, st, num_sms());
+        if (e != cudaSuccess) return cuda_status(e);
+        a_codes = ws;
+        a_scales = ws + codes_al;
+    }
+    q4::GemmParams p;
+    p.M = M; p.N = N; p.K = K;
+    p.a_codes = a_codes; p.a_scales = a_scales; p.a_gscale = d_a_gscale;
+    p.b_codes = b_codes; p.b_scales = b_scales; p.b_gscale = d_b_gscale;
+    p.y = y; p.out_bf16 = out_dt == Q4_BF16; p.mxfp4 = format == Q4_MXFP4;
+    return cuda_status(q4::launch_gemm(p, st, num_sms()));
+}
+
+q4_status q4_get_device_error(void* stream) {
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_status(e);
+    unsigned int word = 0;
+    e = q4::read_clear_device_error(&word);
+    if (e != cudaSuccess) return cuda_status(e);
+    return word ? Q4_ERR_TIMEOUT : Q4_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,143 @@
+// q4_codec.cuh -- device-side number formats: E2M1 element codes, E4M3 and
+// E8M0 block scales, and the per-block scale rules of NVFP4 and MXFP4.
+//
+// Every floating-point step uses an explicitly rounded intrinsic (_rn) so the
+// compiler cannot contract or reorder it; the sequences follow the operation
+// order documented in q4.h.
+#pragma once
+#include <cstdint>
+#include <cuda_bf16.h>
+
+namespace q4 {
+
+// Eight E2M1 codes from eight floats: round to nearest, ties to even
+// mantissa, saturating at +-6.  Element 0 lands in the low nibble.
+__device__ __forceinline__ uint32_t e2m1_pack8(const float (&v)[8]) {
+    uint32_t out;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(out)
+        : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+    return out;
+}
+
+// The conversion above may return +0 for a negative input that rounds to
+// zero; the format keeps the input's sign bit there (code 0x8), so copy the
+// sign into every nibble whose magnitude bits are zero.
+__device__ __forceinline__ uint32_t e2m1_fix_signed_zero(uint32_t codes, const float (&v)[8]) {
+    uint32_t signs = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) signs |= (__float_as_uint(v[i]) >> 31) << (4 * i + 3);
+    // nibbles whose low three bits are zero
+    uint32_t mag = codes & 0x77777777u;
+    uint32_t nz = (mag | (mag >> 1) | (mag >> 2)) & 0x11111111u;  // bit 4i set if magnitude != 0
+    uint32_t zero_mask = (~nz & 0x11111111u) * 0x8u;               // bit 4i+3 set if magnitude == 0
+    return (codes & ~zero_mask) | (signs & zero_mask);
+}
+
+// Magnitude of an E2M1 code (low three bits) as float: 0, .5, 1, 1.5, 2, 3, 4, 6.
+__device__ __forceinline__ float e2m1_value(uint32_t code) {
+    // twice the magnitudes, one nibble each: 0,1,2,3,4,6,8,12
+    const uint32_t twice = 0xC8643210u;
+    float m = (float)((twice >> (4 * (code & 7u))) & 0xFu) * 0.5f;
+    return (code & 8u) ? -m : m;
+}
+
+// E4M3 (finite variant) byte -> value, for non-negative codes 0x00..0x7E.
+__device__ __forceinline__ float e4m3_value(uint32_t b) {
+    uint32_t e = (b >> 3) & 15u, m = b & 7u;
+    if (e == 0) return (float)m * 0.001953125f;             // m * 2^-9, exact
+    return __uint_as_float(((e + 120u) << 23) | (m << 20));  // (1 + m/8) * 2^(e-7)
+}
+
+// Non-negative float -> E4M3 byte, round to nearest even, saturating at 448.
+__device__ __forceinline__ uint32_t e4m3_rn(float v) {
+    v = fminf(v, 448.0f);
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(v));
+    return r & 0xFFu;
+}
+
+// Smallest E4M3 byte whose value is >= v (v >= 0), saturating at 448.
+__device__ __forceinline__ uint32_t e4m3_ru(float v) {
+    uint32_t b = e4m3_rn(v);
+    if (b < 0x7Eu && e4m3_value(b) < v) b += 1;
+    return b;
+}
+
+// Shared MXFP4 exponent of a block with maximum magnitude amax >= 0:
+// floor(log2 amax) - 2, or with round_up the smallest e with amax <= 6 * 2^e,
+// clamped to [-127, 127]; amax = 0 gives -127.
+__device__ __forceinline__ int mx_exponent(float amax, bool round_up) {
+    uint32_t bits = __float_as_uint(amax);
+    if (bits == 0) return -127;
+    int fl;
+    uint32_t m23;
+    uint32_t biased = bits >> 23;
+    if (biased != 0) {
+        fl = (int)biased - 127;
+        m23 = bits & 0x7FFFFFu;
+    } else {
+        int p = 31 - __clz(bits);          // leading bit of the subnormal mantissa
+        fl = p - 149;
+        m23 = (bits << (23 - p)) & 0x7FFFFFu;
+    }
+    int e = fl - 2;
+    if (round_up && m23 > 0x400000u) e += 1;  // significand above 1.5: 4*sig > 6
+    return e < -127 ? -127 : (e > 127 ? 127 : e);
+}
+
+// 2^k as a float for k in [-127, 127] (exact; 2^-127 is subnormal).
+__device__ __forceinline__ float exp2_int(int k) {
+    if (k >= -126) return __uint_as_float((uint32_t)(k + 127) << 23);
+    return __uint_as_float(0x00400000u);
+}
+
+// Per-block normalisation factor of NVFP4 (see q4.h): inv = 1 / (s_b * s_t),
+// or 0 with *degenerate set when the block has no usable scale.
+struct NvScale {
+    uint32_t byte;
+    float inv;
+    bool degenerate;
+};
+
+__device__ __forceinline__ bool st_valid(float s_t) {
+    return s_t > 0.0f && isfinite(s_t);
+}
+
+__device__ __forceinline__ NvScale nv_scale_from_amax(float amax, float s_t, bool round_up) {
+    NvScale r;
+    r.byte = 0;
+    if (st_valid(s_t)) {
+        float denom = __fmul_rn(6.0f, s_t);
+        float sbf = __fdiv_rn(amax, denom);
+        r.byte = round_up ? e4m3_ru(sbf) : e4m3_rn(sbf);
+    }
+    float S = __fmul_rn(e4m3_value(r.byte), s_t);
+    r.inv = __frcp_rn(S);
+    r.degenerate = !st_valid(s_t) || S == 0.0f || !isfinite(r.inv);
+    return r;
+}
+
+__device__ __forceinline__ NvScale nv_scale_from_byte(uint32_t byte, float s_t) {
+    NvScale r;
+    r.byte = byte;
+    float S = __fmul_rn(e4m3_value(byte), s_t);
+    r.inv = __frcp_rn(S);
+    r.degenerate = !st_valid(s_t) || S == 0.0f || !isfinite(r.inv);
+    return r;
+}
+
+// Offset of scale (r, c) in the tensor-core scale layout (see q4.h).
+__host__ __device__ __forceinline__ int64_t tc_scale_offset(int64_t r, int64_t c, int64_t catoms) {
+    return ((r >> 7) * catoms + (c >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (c & 3);
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+}  // namespace q4

@@ -1,0 +1,570 @@
+// q4_gemm.cu -- block-scaled FP4 GEMM  Y = alpha * dec(A) dec(B)^T  on the
+// sm_100a tensor cores (tcgen05.mma kind::mxf4nvf4), persistent and warp
+// specialised:
+//   warp 0      TMA producer: A and B code tiles (128-byte swizzle) by tiled
+//               tensor copies, scale atoms by contiguous bulk copies, into a
+//               STAGES-deep ring guarded by full/empty mbarriers;
+//   warp 1      allocates TMEM, and one elected lane issues per k-block the
+//               scale copies shared memory -> TMEM (tcgen05.cp) and the
+//               block-scaled MMAs into an FP32 accumulator in TMEM;
+//   warps 2..5  epilogue: TMEM -> registers (tcgen05.ld), times alpha,
+//               convert, store Y.
+// CTA tile 128 x 256, k-block 256 elements (128 bytes of codes per row).
+// Every mbarrier wait is bounded; on time-out the kernel records an error and
+// winds down, waiting (bounded) for its own copies and MMAs before freeing TMEM.
+#include <cstdint>
+#include <cstdio>
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include "q4_codec.cuh"
+#include "q4_internal.h"
+#include "q4_ptx.cuh"
+
+namespace q4 {
+
+namespace gemm {
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int KB_BYTES = 128;            // bytes of codes per row per k-block
+constexpr int KB_ELEMS = 256;
+constexpr int STAGES = 4;
+constexpr int A_STAGE = BM * KB_BYTES;   // 16 KB
+constexpr int B_STAGE = BN * KB_BYTES;   // 32 KB
+constexpr int SFA_STAGE = 4 * 512;       // up to 4 scale atoms
+constexpr int SFB_STAGE = 2 * 4 * 512;   // 2 row bands of 128
+constexpr int OFF_B = STAGES * A_STAGE;
+constexpr int OFF_SFA = OFF_B + STAGES * B_STAGE;
+constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_STAGE;
+constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_STAGE;
+constexpr int BAR_BYTES = 256;
+constexpr int SMEM_BYTES = OFF_BAR + BAR_BYTES + 1024;   // + alignment slack
+constexpr int THREADS = 192;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t ACC_COL = 0;          // 256 fp32 columns
+constexpr uint32_t SFA_COL = 256;        // 4 columns per scale atom
+constexpr uint32_t SFB_COL = 272;        // 8 columns per scale atom pair (two bands)
+}  // namespace gemm
+
+struct GemmDev {
+    int64_t M, N, K;
+    const uint8_t* a_scales;
+    const uint8_t* b_scales;
+    const float* a_gscale;
+    const float* b_gscale;
+    void* y;
+    int64_t catoms;      // scale atom-columns per 128-row band (same for A and B)
+    int out_bf16;
+};
+
+// Store 32 consecutive fp32 results of one output row (columns col0..col0+31,
+// only those < N), scaled by alpha.
+__device__ __forceinline__ void store_row32(void* y, int64_t N, int64_t row, int64_t col0, const uint32_t (&r)[32],
+                                            float alpha, bool out_bf16) {
+    if (out_bf16) {
+        uint16_t* yp = reinterpret_cast<uint16_t*>(y) + row * N + col0;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            if (col0 + g * 8 >= N) break;
+            uint32_t w[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[g * 8 + 2 * j]) * alpha,
+                                                         __uint_as_float(r[g * 8 + 2 * j + 1]) * alpha);
+                w[j] = *reinterpret_cast<uint32_t*>(&h);
+            }
+            *reinterpret_cast<uint4*>(yp + g * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+    } else {
+        float* yp = reinterpret_cast<float*>(y) + row * N + col0;
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+            if (col0 + g * 4 >= N) break;
+            *reinterpret_cast<float4*>(yp + g * 4) =
+                make_float4(__uint_as_float(r[g * 4]) * alpha, __uint_as_float(r[g * 4 + 1]) * alpha,
+                            __uint_as_float(r[g * 4 + 2]) * alpha, __uint_as_float(r[g * 4 + 3]) * alpha);
+        }
+    }
+}
+
+template <bool MX>
+__global__ void __launch_bounds__(gemm::THREADS, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmDev p) {
+    using namespace gemm;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+    uint64_t* empty = full + STAGES;
+    uint64_t* tmem_full = empty + STAGES;
+    uint64_t* tmem_empty = tmem_full + 1;
+    uint64_t* mma_done = tmem_empty + 1;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(tmem_full, 1);
+        mbar_init(tmem_empty, 128);
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, TMEM_COLS);
+        tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    const int64_t tiles_m = (p.M + BM - 1) / BM;
+    const int64_t tiles_n = (p.N + BN - 1) / BN;
+    const int64_t tiles = tiles_m * tiles_n;
+    const int nkb = (int)((p.K + KB_ELEMS - 1) / KB_ELEMS);
+    const int mma_per_atom = MX ? 2 : 1;
+    const int atoms_per_kb = 4 / mma_per_atom;
+    const int64_t bands_n = (p.N + 127) / 128;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t last_phase[STAGES];
+            bool issued[STAGES];
+            for (int s = 0; s < STAGES; ++s) issued[s] = false, last_phase[s] = 0;
+            for (int64_t t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x) {
+                const int64_t mt = t % tiles_m, nt = t / tiles_m;
+                const int nbands = (nt * 2 + 1 < bands_n) ? 2 : 1;
+                for (int kb = 0; kb < nkb; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1)) { *abort_flag = 1; break; }
+                    const int64_t krem = p.K - (int64_t)kb * KB_ELEMS;
+                    const int kel = krem < KB_ELEMS ? (int)krem : KB_ELEMS;
+                    const int nmma = kel / 64;
+                    const int na = (nmma + mma_per_atom - 1) / mma_per_atom;
+                    const uint32_t bytes = A_STAGE + B_STAGE + (uint32_t)na * 512u * (1u + (uint32_t)nbands);
+                    mbar_arrive_expect_tx(&full[stage], bytes);
+                    tma_load_2d(smem + stage * A_STAGE, &tmA, &full[stage], kb * KB_BYTES, (int32_t)(mt * BM));
+                    tma_load_2d(smem + OFF_B + stage * B_STAGE, &tmB, &full[stage], kb * KB_BYTES, (int32_t)(nt * BN));
+                    const int64_t acol = (int64_t)kb * atoms_per_kb;
+                    bulk_load(smem + OFF_SFA + stage * SFA_STAGE, p.a_scales + (mt * p.catoms + acol) * 512,
+                              (uint32_t)na * 512u, &full[stage]);
+                    for (int b = 0; b < nbands; ++b)
+                        bulk_load(smem + OFF_SFB + stage * SFB_STAGE + b * 2048,
+                                  p.b_scales + ((nt * 2 + b) * p.catoms + acol) * 512, (uint32_t)na * 512u,
+                                  &full[stage]);
+                    issued[stage] = true;
+                    last_phase[stage] = phase;
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                }
+            }
+            // never leave a copy in flight into shared memory we are about to release
+            for (int s = 0; s < STAGES; ++s)
+                if (issued[s]) mbar_wait(&full[s], last_phase[s]);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc0 = idesc_mxf4(BM, BN, MX);
+            int stage = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            for (int64_t t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x) {
+                if (!mbar_wait(tmem_empty, acc_phase ^ 1)) { *abort_flag = 1; break; }
+                tc_fence_after();
+                for (int kb = 0; kb < nkb; ++kb) {
+                    if (!mbar_wait(&full[stage], phase)) { *abort_flag = 1; break; }
+                    tc_fence_after();
+                    const int64_t krem = p.K - (int64_t)kb * KB_ELEMS;
+                    const int kel = krem < KB_ELEMS ? (int)krem : KB_ELEMS;
+                    const int nmma = kel / 64;
+                    const int na = (nmma + mma_per_atom - 1) / mma_per_atom;
+                    const uint32_t sfa_s = smem_u32(smem + OFF_SFA + stage * SFA_STAGE);
+                    const uint32_t sfb_s = smem_u32(smem + OFF_SFB + stage * SFB_STAGE);
+                    for (int a = 0; a < na; ++a) {
+                        tmem_cp_sf(tmem + SFA_COL + a * 4, smem_desc(sfa_s + a * 512, 0, 128, 0));
+                        tmem_cp_sf(tmem + SFB_COL + a * 8, smem_desc(sfb_s + a * 512, 0, 128, 0));
+                        tmem_cp_sf(tmem + SFB_COL + a * 8 + 4, smem_desc(sfb_s + 2048 + a * 512, 0, 128, 0));
+                    }
+                    const uint64_t adesc = smem_desc(smem_u32(smem + stage * A_STAGE), 16, 1024, 2);
+                    const uint64_t bdesc = smem_desc(smem_u32(smem + OFF_B + stage * B_STAGE), 16, 1024, 2);
+                    for (int kk = 0; kk < nmma; ++kk) {
+                        const int atom = kk / mma_per_atom;
+                        const uint32_t sfid = MX ? (uint32_t)(kk % 2) * 2u : 0u;
+                        const uint32_t idesc = idesc_with_sf_id(idesc0, sfid, sfid);
+                        const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
+                        if (MX)
+                            mma_mxf4(tmem + ACC_COL, adesc + 2 * kk, bdesc + 2 * kk, idesc,
+                                     tmem + SFA_COL + atom * 4, tmem + SFB_COL + atom * 8, acc);
+                        else
+                            mma_nvf4(tmem + ACC_COL, adesc + 2 * kk, bdesc + 2 * kk, idesc,
+                                     tmem + SFA_COL + atom * 4, tmem + SFB_COL + atom * 8, acc);
+                    }
+                    tc_commit(&empty[stage]);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                }
+                if (*abort_flag) break;
+                tc_commit(tmem_full);
+                acc_phase ^= 1;
+            }
+            // all MMAs of this thread are complete before TMEM is released
+            tc_commit(mma_done);
+            mbar_wait(mma_done, 0);
+        }
+    } else {
+        const int quad = warp & 3;                 // TMEM lane quadrant this warp may access
+        const int row_in_tile = quad * 32 + lane;
+        const float alpha = MX ? 1.0f : __fmul_rn(*p.a_gscale, *p.b_gscale);
+        uint32_t acc_phase = 0;
+        for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
+            if (!mbar_wait(tmem_full, acc_phase)) { *abort_flag = 1; break; }
+            tc_fence_after();
+            const int64_t mt = t % tiles_m, nt = t / tiles_m;
+            const int64_t row = mt * BM + row_in_tile;
+            for (int c = 0; c < BN / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + ACC_COL + c * 32, r);
+                tmem_ld_wait();
+                const int64_t col0 = nt * BN + c * 32;
+                if (row < p.M && col0 < p.N) store_row32(p.y, p.N, row, col0, r, alpha, p.out_bf16 != 0);
+            }
+            tc_fence_before();
+            mbar_arrive(tmem_empty);
+            acc_phase ^= 1;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
+}
+
+// ------------------------------------------------------------------ host side
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// 2-D byte tensor [rows, row_bytes] with a box of 128 bytes x box_rows and
+// 128-byte swizzle (the operand layout the MMA descriptors describe).
+static bool make_code_map(CUtensorMap* map, const void* base, int64_t rows, int64_t row_bytes, int box_rows) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+    cuuint32_t box[2] = {128u, (cuuint32_t)box_rows};
+    cuuint32_t es[2] = {1u, 1u};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+cudaError_t launch_gemm(const GemmParams& p, cudaStream_t st, int num_sms) {
+    using namespace gemm;
+    if (p.M == 0 || p.N == 0) return cudaSuccess;
+    CUtensorMap ma, mb;
+    if (!make_code_map(&ma, p.a_codes, p.M, p.K / 2, BM)) return cudaErrorInvalidValue;
+    if (!make_code_map(&mb, p.b_codes, p.N, p.K / 2, BN)) return cudaErrorInvalidValue;
+    GemmDev d;
+    d.M = p.M; d.N = p.N; d.K = p.K;
+    d.a_scales = p.a_scales; d.b_scales = p.b_scales;
+    d.a_gscale = p.a_gscale; d.b_gscale = p.b_gscale;
+    d.y = p.y;
+    const int blk = p.mxfp4 ? 32 : 16;
+    d.catoms = ((p.K / blk) + 3) / 4;
+    d.out_bf16 = p.out_bf16 ? 1 : 0;
+    const int64_t tiles = ((p.M + BM - 1) / BM) * ((p.N + BN - 1) / BN);
+    const int grid = (int)(tiles < num_sms ? tiles : num_sms);
+    cudaError_t e;
+    if (p.mxfp4) {
+        e = cudaFuncSetAttribute(gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        gemm_kernel<true><<<grid, THREADS, SMEM_BYTES, st>>>(ma, mb, d);
+    } else {
+        e = cudaFuncSetAttribute(gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        gemm_kernel<false><<<grid, THREADS, SMEM_BYTES, st>>>(ma, mb, d);
+    }
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ fused decode
+// Small-M GEMM with the activation quantization inside the kernel (no bf16
+// activation round trip, no workspace).  Operands are swapped so the weight
+// fills the MMA's 128-row side: D^T[n, m] = sum_k W[n, k] X[m, k].  Each CTA
+// owns 128 weight rows; warps 2..5 first quantize all of X (M <= 128 rows) into
+// shared memory -- codes in the 128-byte-swizzled K-major operand layout, scales
+// in tensor-core atoms -- while warp 0 already streams weight tiles by TMA.
+namespace dec {
+constexpr int THREADS = 192;
+constexpr int W_STAGE = 128 * 128;       // 16 KB of weight codes per k-block
+constexpr int SFW_STAGE = 4 * 512;
+constexpr uint32_t TMEM_COLS = 256;
+constexpr uint32_t ACC_COL = 0;          // up to 128 fp32 columns
+constexpr uint32_t SFA_COL = 192;        // weight scales, 4 atoms x 4 columns
+constexpr uint32_t SFB_COL = 224;        // activation scales, 4 atoms x 4 columns
+constexpr int MAX_SMEM = 232448;         // 227 KB opt-in limit per CTA
+}  // namespace dec
+
+struct DecodeDev {
+    int64_t M, N, K;
+    const uint16_t* x;
+    const float* a_gscale;
+    const uint8_t* w_scales;
+    const float* b_gscale;
+    void* y;
+    int64_t catoms;
+    int np;           // MMA N: M rounded up to 16
+    int nkb;          // k-blocks of 256
+    int stages;
+    int out_bf16;
+};
+
+__device__ __forceinline__ uint32_t sw128_offset(int row, int byte_in_row) {
+    return (uint32_t)((row >> 3) * 1024 + (row & 7) * 128 + ((((byte_in_row >> 4) ^ (row & 7)) & 7) << 4) +
+                      (byte_in_row & 15));
+}
+
+__global__ void __launch_bounds__(dec::THREADS, 1)
+    fused_decode_kernel(const __grid_constant__ CUtensorMap tmW, DecodeDev p) {
+    using namespace dec;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int np = p.np, nkb = p.nkb, S = p.stages;
+    const int xslab = np * 128;                              // bytes of X codes per k-block
+    uint8_t* sx = smem;                                      // nkb slabs
+    uint8_t* sxf = sx + (size_t)nkb * xslab;                 // nkb x 2 KB of X scale atoms
+    uint8_t* sw = sxf + (size_t)nkb * 2048;                  // S weight stages (1024-aligned)
+    uint8_t* swf = sw + (size_t)S * W_STAGE;                 // S x 2 KB weight scale atoms
+    uint64_t* full = reinterpret_cast<uint64_t*>(swf + (size_t)S * SFW_STAGE);
+    uint64_t* empty = full + S;
+    uint64_t* x_ready = empty + S;
+    uint64_t* tmem_full = x_ready + 1;
+    uint64_t* tmem_empty = tmem_full + 1;
+    uint64_t* mma_done = tmem_empty + 1;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+        mbar_init(x_ready, 128);
+        mbar_init(tmem_full, 1);
+        mbar_init(tmem_empty, 128);
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) { tmem_alloc(tmem_holder, TMEM_COLS); tmem_relinquish(); }
+    if (warp == 0 && lane == 0) tma_prefetch_desc(&tmW);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+    const int64_t tiles = (p.N + 127) / 128;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t last_phase[16];
+            bool issued[16];
+            for (int s = 0; s < S; ++s) issued[s] = false, last_phase[s] = 0;
+            for (int64_t t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x) {
+                for (int kb = 0; kb < nkb; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1)) { *abort_flag = 1; break; }
+                    const int64_t krem = p.K - (int64_t)kb * 256;
+                    const int nmma = (krem < 256 ? (int)krem : 256) / 64;
+                    mbar_arrive_expect_tx(&full[stage], W_STAGE + nmma * 512);
+                    tma_load_2d(sw + stage * W_STAGE, &tmW, &full[stage], kb * 128, (int32_t)(t * 128));
+                    bulk_load(swf + stage * SFW_STAGE, p.w_scales + (t * p.catoms + (int64_t)kb * 4) * 512,
+                              (uint32_t)nmma * 512u, &full[stage]);
+                    issued[stage] = true;
+                    last_phase[stage] = phase;
+                    if (++stage == S) { stage = 0; phase ^= 1; }
+                }
+            }
+            for (int s = 0; s < S; ++s)
+                if (issued[s]) mbar_wait(&full[s], last_phase[s]);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc = idesc_mxf4(128, np, false);
+            int stage = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            bool ok = mbar_wait(x_ready, 0);
+            if (!ok) *abort_flag = 1;
+            tc_fence_after();
+            for (int64_t t = blockIdx.x; ok && t < tiles && !*abort_flag; t += gridDim.x) {
+                if (!mbar_wait(tmem_empty, acc_phase ^ 1)) { *abort_flag = 1; break; }
+                tc_fence_after();
+                for (int kb = 0; kb < nkb; ++kb) {
+                    if (!mbar_wait(&full[stage], phase)) { *abort_flag = 1; break; }
+                    tc_fence_after();
+                    const int64_t krem = p.K - (int64_t)kb * 256;
+                    const int nmma = (krem < 256 ? (int)krem : 256) / 64;
+                    const uint32_t wf = smem_u32(swf + stage * SFW_STAGE);
+                    const uint32_t xf = smem_u32(sxf + kb * 2048);
+                    for (int a = 0; a < nmma; ++a) {
+                        tmem_cp_sf(tmem + SFA_COL + a * 4, smem_desc(wf + a * 512, 0, 128, 0));
+                        tmem_cp_sf(tmem + SFB_COL + a * 4, smem_desc(xf + a * 512, 0, 128, 0));
+                    }
+                    const uint64_t adesc = smem_desc(smem_u32(sw + stage * W_STAGE), 16, 1024, 2);
+                    const uint64_t bdesc = smem_desc(smem_u32(sx + kb * xslab), 16, 1024, 2);
+                    for (int kk = 0; kk < nmma; ++kk)
+                        mma_nvf4(tmem + ACC_COL, adesc + 2 * kk, bdesc + 2 * kk, idesc, tmem + SFA_COL + kk * 4,
+                                 tmem + SFB_COL + kk * 4, (kb > 0 || kk > 0) ? 1u : 0u);
+                    tc_commit(&empty[stage]);
+                    if (++stage == S) { stage = 0; phase ^= 1; }
+                }
+                if (*abort_flag) break;
+                tc_commit(tmem_full);
+                acc_phase ^= 1;
+            }
+            tc_commit(mma_done);
+            mbar_wait(mma_done, 0);
+        }
+    } else {
+        // ---- quantize X into shared memory (128 threads)
+        const int qt = threadIdx.x - 64;
+        const float s_t = *p.a_gscale;
+        for (int i = qt; i < nkb * 512; i += 128) reinterpret_cast<uint32_t*>(sxf)[i] = 0u;
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        const int64_t cpr = p.K / 8;                         // chunks per row
+        const int64_t total = (int64_t)np * cpr;
+        for (int64_t q = qt; q < total; q += 128) {
+            const int r = (int)(q / cpr);
+            const int64_t ch = q % cpr;
+            float v[8];
+            if (r < p.M) {
+                uint4 raw = __ldg(reinterpret_cast<const uint4*>(p.x + (int64_t)r * p.K + ch * 8));
+                v[0] = bf16_lo(raw.x); v[1] = bf16_hi(raw.x); v[2] = bf16_lo(raw.y); v[3] = bf16_hi(raw.y);
+                v[4] = bf16_lo(raw.z); v[5] = bf16_hi(raw.z); v[6] = bf16_lo(raw.w); v[7] = bf16_hi(raw.w);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) v[i] = 0.0f;
+            }
+            float amax = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+            // the two halves of a 16-block are neighbouring q, hence neighbouring lanes
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+            NvScale sc = nv_scale_from_amax(amax, s_t, false);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] = sc.degenerate ? 0.0f : __fmul_rn(v[i], sc.inv);
+            const uint32_t codes = e2m1_fix_signed_zero(e2m1_pack8(v), v);
+            const int64_t k = ch * 8;
+            const int kb = (int)(k >> 8);
+            const int byte_in_row = (int)((k & 255) >> 1);
+            *reinterpret_cast<uint32_t*>(sx + (size_t)kb * xslab + sw128_offset(r, byte_in_row)) = codes;
+            if ((ch & 1) == 0) {
+                const int64_t c = k >> 4;                         // scale column
+                const int cin = (int)(c & 15);                    // within the k-block
+                sxf[(size_t)kb * 2048 + (cin >> 2) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (cin & 3)] =
+                    (uint8_t)sc.byte;
+            }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(x_ready);
+
+        // ---- epilogue: thread = one weight row = one output column
+        const int quad = warp & 3;
+        const float alpha = __fmul_rn(*p.a_gscale, *p.b_gscale);
+        uint32_t acc_phase = 0;
+        for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
+            if (!mbar_wait(tmem_full, acc_phase)) { *abort_flag = 1; break; }
+            tc_fence_after();
+            const int64_t n = t * 128 + quad * 32 + lane;
+            for (int c0 = 0; c0 < np; c0 += 32) {
+                uint32_t r[32];
+                tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + ACC_COL + c0, r);
+                tmem_ld_wait();
+                if (n < p.N) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int64_t m = c0 + j;
+                        if (m < p.M) {
+                            const float val = __uint_as_float(r[j]) * alpha;
+                            if (p.out_bf16)
+                                reinterpret_cast<__nv_bfloat16*>(p.y)[m * p.N + n] = __float2bfloat16_rn(val);
+                            else
+                                reinterpret_cast<float*>(p.y)[m * p.N + n] = val;
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(tmem_empty);
+            acc_phase ^= 1;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
+}
+
+static int decode_smem_bytes(int np, int nkb, int stages) {
+    return 1024 + nkb * (np * 128 + 2048) + stages * (dec::W_STAGE + dec::SFW_STAGE) + (2 * stages + 8) * 8 + 64;
+}
+
+static int decode_stages(int64_t M, int64_t K) {
+    if (M <= 0 || M > 128 || K <= 0 || K > (1 << 20)) return 0;
+    const int np = (int)((M + 15) / 16 * 16);
+    const int nkb = (int)((K + 255) / 256);
+    int stages = 8;
+    while (stages >= 2 && decode_smem_bytes(np, nkb, stages) > dec::MAX_SMEM) --stages;
+    return stages >= 2 ? stages : 0;
+}
+
+bool fused_decode_supported(int64_t M, int64_t K) { return decode_stages(M, K) > 0; }
+
+cudaError_t launch_fused_decode(const FusedDecodeParams& p, cudaStream_t st, int num_sms) {
+    using namespace dec;
+    if (p.M == 0 || p.N == 0) return cudaSuccess;
+    const int np = (int)((p.M + 15) / 16 * 16);
+    const int nkb = (int)((p.K + 255) / 256);
+    const int stages = decode_stages(p.M, p.K);
+    if (stages == 0) return cudaErrorNotSupported;
+    CUtensorMap mw;
+    if (!make_code_map(&mw, p.b_codes, p.N, p.K / 2, 128)) return cudaErrorInvalidValue;
+    DecodeDev d;
+    d.M = p.M; d.N = p.N; d.K = p.K; d.x = p.a_bf16; d.a_gscale = p.a_gscale;
+    d.w_scales = p.b_scales; d.b_gscale = p.b_gscale; d.y = p.y;
+    d.catoms = ((p.K / 16) + 3) / 4;
+    d.np = np; d.nkb = nkb; d.stages = stages; d.out_bf16 = p.out_bf16 ? 1 : 0;
+    const int smem = decode_smem_bytes(np, nkb, stages);
+    cudaError_t e = cudaFuncSetAttribute(fused_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    const int64_t tiles = (p.N + 127) / 128;
+    const int grid = (int)(tiles < num_sms ? tiles : num_sms);
+    fused_decode_kernel<<<grid, THREADS, smem, st>>>(mw, d);
+    return cudaGetLastError();
+}
+
+cudaError_t read_clear_device_error(unsigned int* word) {
+    cudaError_t e = cudaMemcpyFromSymbol(word, g_device_error, sizeof(unsigned int));
+    if (e != cudaSuccess || *word == 0) return e;
+    const unsigned int zero = 0;
+    return cudaMemcpyToSymbol(g_device_error, &zero, sizeof(unsigned int));
+}
+
+}  // namespace q4

@@ -1,0 +1,80 @@
+// q4_internal.h -- parameter blocks and launcher declarations shared by the
+// kernel files and the C-ABI layer.  Not part of the public interface.
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace q4 {
+
+struct QuantParams {
+    const void* x;        // [rows, ld] bf16 or fp32
+    int64_t rows, cols, ld;
+    const float* gscale;  // NVFP4 tensor scale (device), else unused
+    const float* chan;    // MXFP4 per-column multiplier or nullptr
+    uint8_t* codes;       // [rows, cols/2]
+    uint8_t* scales;      // tensor-core layout or row-major
+    int64_t scols;        // cols / block
+    int64_t catoms;       // ceil(scols / 4)
+};
+
+struct SigmaDeltaParams {
+    const float* w;       // [rows, cols]
+    int64_t rows, cols;
+    const uint8_t* scales;
+    const float* gscale;
+    float* residue;       // [rows, cols], in/out
+    uint8_t* codes;       // [rows, cols/2]
+    int64_t scols, catoms;
+};
+
+struct DequantParams {
+    const uint8_t* codes;
+    const uint8_t* scales;
+    const float* gscale;
+    int64_t rows, cols;
+    void* out;
+    int64_t scols, catoms;
+};
+
+struct GemmParams {
+    int64_t M, N, K;
+    const uint8_t* a_codes;   // [M, K/2]
+    const uint8_t* a_scales;  // tensor-core layout
+    const float* a_gscale;    // NVFP4 s_tA or nullptr
+    const uint8_t* b_codes;   // [N, K/2]
+    const uint8_t* b_scales;
+    const float* b_gscale;
+    void* y;                  // [M, N]
+    bool out_bf16;
+    bool mxfp4;
+};
+
+struct FusedDecodeParams {
+    int64_t M, N, K;
+    const uint16_t* a_bf16;   // [M, K] bf16 activations
+    const float* a_gscale;    // activation tensor scale
+    const uint8_t* b_codes;
+    const uint8_t* b_scales;
+    const float* b_gscale;
+    void* y;
+    bool out_bf16;
+};
+
+cudaError_t launch_amax(const void* x, int64_t n, bool bf16, float denom, float* d_out,
+                        cudaStream_t st, int num_sms);
+cudaError_t launch_quantize(const QuantParams& p, int blk, bool bf16, bool tc, bool ru, bool had,
+                            bool chan, cudaStream_t st, int num_sms);
+cudaError_t launch_sigma_delta(const SigmaDeltaParams& p, int blk, bool tc, cudaStream_t st, int num_sms);
+cudaError_t launch_dequantize(const DequantParams& p, int blk, bool tc, bool out_bf16, cudaStream_t st,
+                              int num_sms);
+cudaError_t launch_gemm(const GemmParams& p, cudaStream_t st, int num_sms);
+cudaError_t launch_fused_decode(const FusedDecodeParams& p, cudaStream_t st, int num_sms);
+
+// Reads and clears the device error word (bit 0: a bounded wait ran out).
+cudaError_t read_clear_device_error(unsigned int* word);
+
+// Whether the fused-activation small-M GEMM takes this shape (M <= 128 and
+// the quantized activations fit in shared memory next to >= 2 weight stages).
+bool fused_decode_supported(int64_t M, int64_t K);
+
+}  // namespace q4

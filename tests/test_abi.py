@@ -1,0 +1,89 @@
+"""The C-ABI library loads, exports every entry point include/*.h declares,
+and rejects invalid arguments on the host before any launch (no GPU needed:
+validation fails before the first CUDA call)."""
+import ctypes
+import re
+from pathlib import Path
+
+import pytest
+
+ROOT = Path(__file__).resolve().parent.parent
+
+
+def declared_symbols():
+    names = set()
+    for h in (ROOT / "include").glob("*.h"):
+        text = h.read_text()
+        names |= set(re.findall(r"^Q4_API\s+[\w\s\*]+?\b(q4_\w+)\s*\(", text, flags=re.M))
+    return sorted(names)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from mxfp4_w4a4_block_b200 import build
+    build.build()
+    import mxfp4_w4a4_block_b200 as q4
+    return q4.lib()
+
+
+def test_header_declares_the_entry_points():
+    names = declared_symbols()
+    for n in ["q4_amax", "q4_quantize", "q4_dequantize", "q4_sigma_delta_step", "q4_gemm",
+              "q4_gemm_workspace_size", "q4_get_device_error", "q4_status_string", "q4_scale_bytes"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    raw = ctypes.CDLL(str(ROOT / "mxfp4_w4a4_block_b200" / "libq4.so"))
+    for n in declared_symbols():
+        assert hasattr(raw, n), n
+
+
+def test_status_strings_and_version(lib):
+    assert lib.q4_version() >= 100
+    for s in range(8):
+        assert lib.q4_status_string(s)
+
+
+def test_scale_bytes(lib):
+    import mxfp4_w4a4_block_b200 as q4
+    assert q4.q4_scale_bytes(q4.NVFP4, 200, 336, q4.LAYOUT_TC) == 256 * 24
+    assert q4.q4_scale_bytes(q4.NVFP4, 200, 336, 0) == 200 * 21
+    assert q4.q4_scale_bytes(q4.MXFP4, 3, 352, q4.LAYOUT_TC) == 128 * 12
+    assert q4.q4_scale_bytes(q4.NVFP4, 10, 17, 0) == 0
+
+
+def test_workspace_size(lib):
+    import mxfp4_w4a4_block_b200 as q4
+    assert q4.q4_gemm_workspace_size(q4.NVFP4, 16, 17408, 5120, q4.A_BF16) == 0
+    assert q4.q4_gemm_workspace_size(q4.NVFP4, 8192, 5120, 5120, q4.A_QUANTIZED) == 0
+    ws = q4.q4_gemm_workspace_size(q4.NVFP4, 8192, 5120, 5120, q4.A_BF16)
+    assert ws == 8192 * 2560 + 8192 * 320
+
+
+def test_host_validation_without_launch(lib):
+    import mxfp4_w4a4_block_b200 as q4
+    P = 1 << 20                   # a fake, 16-byte aligned "device" address; never dereferenced
+    g = P + 4096
+    # block size must match the format
+    assert lib.q4_quantize(q4.NVFP4, 32, q4.BF16, P, 4, 64, 64, g, None, P, P, 0, None) == 4
+    # NVFP4 needs a tensor scale; MXFP4 must not get one
+    assert lib.q4_quantize(q4.NVFP4, 16, q4.BF16, P, 4, 64, 64, None, None, P, P, 0, None) == 1
+    assert lib.q4_quantize(q4.MXFP4, 32, q4.BF16, P, 4, 64, 64, g, None, P, P, 0, None) == 1
+    # columns must be whole blocks
+    assert lib.q4_quantize(q4.NVFP4, 16, q4.BF16, P, 4, 40, 40, g, None, P, P, 0, None) == 3
+    # misaligned pointer / row stride
+    assert lib.q4_quantize(q4.NVFP4, 16, q4.BF16, P + 2, 4, 64, 64, g, None, P, P, 0, None) == 2
+    assert lib.q4_quantize(q4.NVFP4, 16, q4.BF16, P, 4, 64, 68, g, None, P, P, 0, None) == 2
+    # Hadamard is MXFP4-only
+    assert lib.q4_quantize(q4.NVFP4, 16, q4.BF16, P, 4, 64, 64, g, None, P, P, q4.HADAMARD32, None) == 4
+    # empty tensors are a no-op
+    assert lib.q4_quantize(q4.NVFP4, 16, q4.BF16, None, 0, 64, 64, g, None, None, None, 0, None) == 0
+    # GEMM: K must be a multiple of 64, N of 8
+    assert lib.q4_gemm(q4.NVFP4, 16, 4, 8, 96, 0, P, P, g, P, P, g, q4.BF16, P, None, 0, None) == 3
+    assert lib.q4_gemm(q4.NVFP4, 16, 4, 12, 64, 0, P, P, g, P, P, g, q4.BF16, P, None, 0, None) == 3
+    # GEMM: missing workspace for the quantize-once path
+    assert lib.q4_gemm(q4.NVFP4, 16, 4096, 64, 64, q4.A_BF16, P, None, g, P, P, g, q4.BF16, P,
+                       None, 0, None) == 7
+    # Sigma-Delta: NVFP4 needs s_t
+    assert lib.q4_sigma_delta_step(q4.NVFP4, 16, P, 4, 64, P, None, P, P, 0, None) == 1

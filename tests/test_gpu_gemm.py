@@ -1,0 +1,184 @@
+"""GPU parity of the block-scaled FP4 GEMM (tcgen05) against the binary64 oracle
+on the same decoded operands, through the C-ABI library.
+
+Operands are quantized on both sides from the same synthetic inputs (the
+quantizers agree bit for bit, checked here again); the oracle GEMM only ever
+sees oracle-made codes and scales."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+import mxfp4_w4a4_block_b200 as q4
+from gpu_util import DEV, GEMM_BF16_TOL, GEMM_F32_TOL, dev, gscale_dev, host, rel_fro
+
+pytestmark = pytest.mark.gpu
+
+
+class Operand:
+    """One GEMM operand quantized on the GPU and by the oracle."""
+
+    def __init__(self, fmt, x32, x_t=None, chan=None, had=False, denom=2688.0):
+        self.fmt = fmt
+        self.rows, self.cols = x32.shape
+        x_t = dev(x32) if x_t is None else x_t
+        if fmt == q4.NVFP4:
+            self.s_t = oracle.tensor_scale(oracle.amax(x32), denom)
+            self.g_t = gscale_dev(self.s_t)
+            self.codes, self.scales = q4.q4_quantize(fmt, x_t, gscale=self.g_t, flags=q4.LAYOUT_TC)
+            self.o_codes, self.o_scales = oracle.nvfp4_quantize(x32, self.s_t)
+        else:
+            self.s_t, self.g_t = np.float32(0), None
+            flags = q4.LAYOUT_TC | (q4.HADAMARD32 if had else 0)
+            self.codes, self.scales = q4.q4_quantize(fmt, x_t, chan=None if chan is None else dev(chan),
+                                                     flags=flags)
+            self.o_codes, self.o_scales = oracle.mxfp4_quantize(x32, chan, hadamard=had)
+        assert np.array_equal(host(self.codes), self.o_codes)
+
+    def rows_subset(self, idx):
+        return np.ascontiguousarray(self.o_codes[idx]), np.ascontiguousarray(self.o_scales[idx])
+
+
+def run_gemm(A: Operand, B: Operand, out_dtype):
+    M, K = A.rows, A.cols
+    N = B.rows
+    return q4.q4_gemm(A.fmt, M, N, K, A.codes, A.scales, A.g_t, B.codes, B.scales, B.g_t, out_dtype=out_dtype)
+
+
+def oracle_gemm(A: Operand, B: Operand, rows=None, cols=None):
+    M, K = A.rows, A.cols
+    if cols is None:
+        bc, bs, N = B.o_codes, B.o_scales, B.rows
+    else:
+        bc, bs = B.rows_subset(cols)
+        N = len(cols)
+    return oracle.gemm(A.fmt, A.o_codes, A.o_scales, A.s_t, bc, bs, B.s_t, M, N, K, rows=rows)
+
+
+def check(y: torch.Tensor, ref: np.ndarray, out_dtype):
+    got = host(y.float())
+    if out_dtype == torch.float32:
+        assert rel_fro(got, ref) <= GEMM_F32_TOL
+    else:
+        assert rel_fro(got, ref) <= GEMM_BF16_TOL
+    assert np.all(np.isfinite(got))
+
+
+@pytest.mark.parametrize("fmt", [q4.NVFP4, q4.MXFP4])
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("mnk", [(128, 256, 256), (64, 512, 512), (200, 328, 320), (384, 768, 1024),
+                                 (1, 8, 64), (130, 264, 576)])
+def test_gemm_parity_small(fmt, out_dtype, mnk):
+    M, N, K = mnk
+    x = synth.small_like("heavy", M + K, M, K)
+    w = synth.small_like("weight", N + K, N, K)
+    A, B = Operand(fmt, x), Operand(fmt, w)
+    y = run_gemm(A, B, out_dtype)
+    check(y, oracle_gemm(A, B), out_dtype)
+
+
+def test_gemm_tiny_linear_config():
+    """X 64x512 and W 512x512 fp32 (1% x50 outliers), s_t = amax/(6*448), BF16 out."""
+    d = synth.tiny()
+    A, B = Operand(q4.NVFP4, d["x"]), Operand(q4.NVFP4, d["w"])
+    for od in (torch.float32, torch.bfloat16):
+        check(run_gemm(A, B, od), oracle_gemm(A, B), od)
+
+
+def test_gemm_closed_form_integer_case():
+    """All scales 1 and every element 1.0 x 0.5: every output is K/2 exactly."""
+    M, N, K = 130, 264, 512
+    a = np.ones((M, K), np.float32)
+    b = np.full((N, K), 0.5, np.float32)
+    A = Operand(q4.MXFP4, a)
+    B = Operand(q4.MXFP4, b)
+    y = host(run_gemm(A, B, torch.float32))
+    assert np.all(y == K * 0.5)
+
+
+@pytest.mark.parametrize("M", [1, 16, 33, 128])
+def test_fused_activation_quant_decode_small(M):
+    """a_kind = A_BF16 for small M: the kernel quantizes the bf16 activations itself."""
+    N, K = 392, 1088
+    x = synth.to_bf16(synth.small_like("heavy", M, M, K))
+    x32 = synth.bf16_to_f32(x)
+    w = synth.small_like("weight", 9, N, K)
+    A = Operand(q4.NVFP4, x32, x_t=dev(x))
+    B = Operand(q4.NVFP4, w)
+    for od in (torch.float32, torch.bfloat16):
+        y = q4.q4_gemm(q4.NVFP4, M, N, K, dev(x), None, A.g_t, B.codes, B.scales, B.g_t, out_dtype=od,
+                       a_kind=q4.A_BF16)
+        check(y, oracle_gemm(A, B), od)
+
+
+def test_fused_activation_quant_prefill_path():
+    """a_kind = A_BF16 with M above the fused limit: quantize-once into the workspace."""
+    M, N, K = 300, 264, 640
+    x = synth.to_bf16(synth.small_like("heavy", 1, M, K))
+    x32 = synth.bf16_to_f32(x)
+    w = synth.small_like("weight", 2, N, K)
+    A = Operand(q4.NVFP4, x32, x_t=dev(x))
+    B = Operand(q4.NVFP4, w)
+    assert q4.q4_gemm_workspace_size(q4.NVFP4, M, N, K, q4.A_BF16) > 0
+    y = q4.q4_gemm(q4.NVFP4, M, N, K, dev(x), None, A.g_t, B.codes, B.scales, B.g_t,
+                   out_dtype=torch.float32, a_kind=q4.A_BF16)
+    check(y, oracle_gemm(A, B), torch.float32)
+
+
+def test_decode_config_full_size_sampled_columns():
+    """Decode shape 16 x 17408 x 5120 with the fused activation quantizer; the
+    oracle computes 1024 sampled output columns (all 16 rows)."""
+    d = synth.decode()
+    x32 = synth.bf16_to_f32(d["x"])
+    A = Operand(q4.NVFP4, x32, x_t=dev(d["x"]))
+    B = Operand(q4.NVFP4, d["w"])
+    M, N, K = 16, 17408, 5120
+    y = q4.q4_gemm(q4.NVFP4, M, N, K, dev(d["x"]), None, A.g_t, B.codes, B.scales, B.g_t,
+                   out_dtype=torch.float32, a_kind=q4.A_BF16)
+    cols = np.sort(np.random.default_rng(0).choice(N, 1024, replace=False))
+    ref = oracle_gemm(A, B, cols=cols)
+    check_sub = host(y)[:, cols]
+    assert rel_fro(check_sub, ref) <= GEMM_F32_TOL
+
+
+@pytest.mark.parametrize("n", [5120, 17408])
+def test_prefill_config_full_size_sampled(n):
+    """Prefill 8192 x n x 5120 (quantized A); oracle on 2 rows per 128-row tile
+    and 1024 sampled columns."""
+    d = synth.prefill(n_list=(n,))
+    x32 = synth.bf16_to_f32(d["x"])
+    A = Operand(q4.NVFP4, x32, x_t=dev(d["x"]))
+    B = Operand(q4.NVFP4, d["w"][0])
+    y = run_gemm(A, B, torch.bfloat16)
+    rng = np.random.default_rng(n)
+    rows = np.array([t * 128 + r for t in range(64) for r in sorted(rng.choice(128, 2, replace=False))])
+    cols = np.sort(rng.choice(n, 1024, replace=False))
+    ref = oracle_gemm(A, B, rows=rows, cols=cols)
+    got = host(y.float())[np.ix_(rows, cols)]
+    assert rel_fro(got, ref) <= GEMM_BF16_TOL
+
+
+def test_mxfp4_config_full_size_sampled():
+    """MXFP4 4096 x 14336 x 4096 with t and Hadamard-32 on both operands."""
+    d = synth.mxfp4()
+    x32 = synth.bf16_to_f32(d["x"])
+    A = Operand(q4.MXFP4, x32, x_t=dev(d["x"]), chan=d["t"], had=True)
+    B = Operand(q4.MXFP4, d["w"], chan=d["inv_t"], had=True)
+    y = run_gemm(A, B, torch.float32)
+    rng = np.random.default_rng(1)
+    rows = np.sort(rng.choice(4096, 64, replace=False))
+    cols = np.sort(rng.choice(14336, 1024, replace=False))
+    ref = oracle_gemm(A, B, rows=rows, cols=cols)
+    got = host(y)[np.ix_(rows, cols)]
+    assert rel_fro(got, ref) <= GEMM_F32_TOL
+
+
+def test_gemm_k_zero_and_empty():
+    B = Operand(q4.NVFP4, synth.small_like("weight", 1, 64, 64))
+    y = torch.full((4, 64), 7.0, device=DEV)
+    a = torch.zeros((4, 32), dtype=torch.uint8, device=DEV)
+    q4.q4_gemm(q4.NVFP4, 4, 64, 0, a, B.scales, B.g_t, B.codes, B.scales, B.g_t, out_dtype=torch.float32, y=y)
+    assert float(y.abs().max()) == 0.0
+    q4.q4_gemm(q4.NVFP4, 0, 64, 64, a, B.scales, B.g_t, B.codes, B.scales, B.g_t, out_dtype=torch.float32)
+    assert q4.q4_get_device_error() == 0

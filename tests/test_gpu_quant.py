@@ -1,0 +1,171 @@
+"""GPU parity: amax, NVFP4 / MXFP4 quantize, dequantize -- bit for bit against
+the CPU oracle, through the C-ABI library."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+import mxfp4_w4a4_block_b200 as q4
+from gpu_util import DEV, dev, gscale_dev, host
+
+pytestmark = pytest.mark.gpu
+
+
+def gpu_nvfp4(x_t, s_t, flags):
+    codes, scales = q4.q4_quantize(q4.NVFP4, x_t, gscale=gscale_dev(s_t), flags=flags)
+    return host(codes), host(scales)
+
+
+def check_nvfp4(x32: np.ndarray, x_t: torch.Tensor, s_t, ru: bool, tc: bool):
+    rows, cols = x32.shape
+    flags = (q4.SCALE_RU if ru else 0) | (q4.LAYOUT_TC if tc else 0)
+    gc, gs = gpu_nvfp4(x_t, s_t, flags)
+    oc, os_ = oracle.nvfp4_quantize(x32, s_t, round_up=ru)
+    assert np.array_equal(gc, oc)
+    if tc:
+        assert np.array_equal(gs, oracle.scales_to_tc(os_))
+    else:
+        assert np.array_equal(gs.reshape(os_.shape), os_)
+
+
+def test_e2m1_decisions_exhaustive_near_grid():
+    """Every binary32 value in [-6, 6] with its 8 low mantissa bits clear, plus
+    every neighbourhood of a rounding midpoint, through the NVFP4 kernel with
+    block scale exactly 1 (each 16-block starts with 6.0 and s_t = 1)."""
+    pos = np.arange(0, 0x40C00001, 256, dtype=np.uint32).view(np.float32)   # 0 .. 6
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0], np.float32)
+    near = np.concatenate([np.nextafter(np.repeat(mids, 1), np.float32(np.inf)),
+                           np.nextafter(mids, np.float32(0)), mids])
+    vals = np.concatenate([pos, -pos, near, -near, np.array([0.0, -0.0, 1e-30, -1e-30], np.float32)])
+    vals = vals[np.abs(vals) <= 6.0]
+    pad = (-len(vals)) % 15
+    vals = np.concatenate([vals, np.zeros(pad, np.float32)]).reshape(-1, 15)
+    blocks = np.concatenate([np.full((vals.shape[0], 1), 6.0, np.float32), vals], axis=1)
+    nblk = blocks.shape[0]
+    cols = 16 * 64
+    nrows = (nblk + 63) // 64
+    x = np.zeros((nrows * 64, 16), np.float32)
+    x[:nblk] = blocks
+    x[nblk:, 0] = 6.0
+    x = x.reshape(nrows, cols)
+    check_nvfp4(x, dev(x), 1.0, ru=False, tc=True)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("ru", [False, True])
+@pytest.mark.parametrize("tc", [False, True])
+@pytest.mark.parametrize("shape", [(200, 336), (128, 64), (1, 16), (257, 1040)])
+def test_nvfp4_quantize_parity(dtype, ru, tc, shape):
+    rows, cols = shape
+    x = synth.small_like("heavy", rows * 7 + cols, rows, cols)
+    if dtype == "bf16":
+        xt = synth.to_bf16(x)
+        x32 = synth.bf16_to_f32(xt)
+        x_t = dev(xt)
+    else:
+        x32 = x
+        x_t = dev(x)
+    s_t = oracle.tensor_scale(oracle.amax(x32), 1536.0 if ru else 2688.0)
+    check_nvfp4(x32, x_t, s_t, ru, tc)
+
+
+def test_nvfp4_degenerate_and_saturating_blocks():
+    x = np.zeros((4, 64), np.float32)
+    x[1, :16] = 6.35          # RN scale 1.0 -> 6.35 saturates to 6
+    x[1, 16:32] = -6.35
+    x[2, 0] = -1e-3           # negative values that round to zero keep the sign
+    x[2, 1] = 3.0
+    x[3, :] = -0.0
+    check_nvfp4(x, dev(x), 1.0, ru=False, tc=True)
+    # zero tensor scale: every block degenerate
+    check_nvfp4(x, dev(x), 0.0, ru=False, tc=True)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("had,chan,ru", [(False, False, False), (True, False, False),
+                                         (True, True, False), (False, True, True), (True, True, True)])
+@pytest.mark.parametrize("shape", [(200, 352), (128, 128), (3, 32)])
+def test_mxfp4_quantize_parity(dtype, had, chan, ru, shape):
+    rows, cols = shape
+    x = synth.small_like("outlier", rows + 3 * cols, rows, cols)
+    if dtype == "bf16":
+        xt = synth.to_bf16(x)
+        x32 = synth.bf16_to_f32(xt)
+        x_t = dev(xt)
+    else:
+        x32 = x
+        x_t = dev(x)
+    c = np.exp(np.random.default_rng(cols).uniform(-2, 2, cols)).astype(np.float32) if chan else None
+    flags = q4.LAYOUT_TC | (q4.HADAMARD32 if had else 0) | (q4.SCALE_RU if ru else 0)
+    gc, gs = q4.q4_quantize(q4.MXFP4, x_t, chan=None if c is None else dev(c), flags=flags)
+    oc, os_ = oracle.mxfp4_quantize(x32, c, hadamard=had, round_up=ru)
+    assert np.array_equal(host(gc), oc)
+    assert np.array_equal(host(gs), oracle.scales_to_tc(os_))
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("n", [0, 1, 7, 8, 1000, 123457])
+def test_amax_parity(dtype, n):
+    x = synth.small_like("heavy", n + 1, 1, max(n, 1) * 1).reshape(-1)[:n] if n else np.zeros(0, np.float32)
+    if dtype == "bf16":
+        xt = synth.to_bf16(x)
+        x32 = synth.bf16_to_f32(xt)
+        x_t = dev(xt) if n else torch.zeros(8, dtype=torch.bfloat16, device=DEV)[:0]
+    else:
+        x32 = x
+        x_t = dev(x) if n else torch.zeros(8, dtype=torch.float32, device=DEV)[:0]
+    out = host(q4.q4_amax(x_t, 2688.0))
+    am = oracle.amax(x32) if n else np.float32(0)
+    assert out[0] == am
+    assert out[1] == oracle.tensor_scale(am, 2688.0)
+
+
+@pytest.mark.parametrize("fmt", [q4.NVFP4, q4.MXFP4])
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("tc", [False, True])
+def test_dequantize_parity(fmt, out_dtype, tc):
+    rows, cols = 130, 224
+    x = synth.small_like("heavy", 5, rows, cols)
+    flags = q4.LAYOUT_TC if tc else 0
+    if fmt == q4.NVFP4:
+        s_t = oracle.tensor_scale(oracle.amax(x), 2688.0)
+        gs_t = gscale_dev(s_t)
+        codes, scales = q4.q4_quantize(fmt, dev(x), gscale=gs_t, flags=flags)
+        oc, os_ = oracle.nvfp4_quantize(x, s_t)
+    else:
+        s_t, gs_t = 0.0, None
+        codes, scales = q4.q4_quantize(fmt, dev(x), flags=flags)
+        oc, os_ = oracle.mxfp4_quantize(x)
+    out = host(q4.q4_dequantize(fmt, codes, scales, rows, cols, gscale=gs_t, flags=flags,
+                                out_dtype=out_dtype).float())
+    ref = oracle.dequantize(fmt, oc, os_, s_t, rows, cols)
+    ref_t = torch.from_numpy(ref).float()
+    if out_dtype == torch.bfloat16:
+        ref_t = ref_t.bfloat16().float()
+    assert np.array_equal(out, ref_t.numpy())
+
+
+def test_prefill_activation_quantize_full_size():
+    """The prefill activation (8192 x 5120 bf16) quantized in full, bit for bit."""
+    d = synth.prefill(n_list=())
+    x32 = synth.bf16_to_f32(d["x"])
+    am = host(q4.q4_amax(dev(d["x"]), 2688.0))
+    assert am[0] == oracle.amax(x32)
+    s_t = oracle.tensor_scale(oracle.amax(x32), 2688.0)
+    assert am[1] == s_t
+    gc, gs = q4.q4_quantize(q4.NVFP4, dev(d["x"]), gscale=torch.tensor(am[1:2], device=DEV), flags=q4.LAYOUT_TC)
+    oc, os_ = oracle.nvfp4_quantize(x32, s_t)
+    assert np.array_equal(host(gc), oc)
+    assert np.array_equal(host(gs), oracle.scales_to_tc(os_))
+
+
+def test_mxfp4_activation_quantize_full_size():
+    """The MXFP4 activation (4096 x 4096 bf16) with t and Hadamard-32, bit for bit."""
+    d = synth.mxfp4(n=256)
+    x32 = synth.bf16_to_f32(d["x"])
+    flags = q4.LAYOUT_TC | q4.HADAMARD32
+    gc, gs = q4.q4_quantize(q4.MXFP4, dev(d["x"]), chan=dev(d["t"]), flags=flags)
+    oc, os_ = oracle.mxfp4_quantize(x32, d["t"], hadamard=True)
+    assert np.array_equal(host(gc), oc)
+    assert np.array_equal(host(gs), oracle.scales_to_tc(os_))
