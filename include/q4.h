@@ -202,6 +202,38 @@ Q4_API size_t q4_gemm_workspace_size(q4_format format, int64_t M, int64_t N, int
                               int a_kind);
 
 /*
+ * q4_gemm_a_bf16_noalloc -- the NVFP4 GEMM with bf16 activations
+ *   (q4_gemm with a_kind = Q4_A_BF16) for callers that cannot allocate device
+ *   memory when they call it: code embedded in an application that owns every
+ *   device buffer through its own fixed pool, or that has to keep its device
+ *   footprint constant after start-up, and so cannot pass q4_gemm the scratch
+ *   workspace it needs for larger M.  No counterpart on the source pages: it is
+ *   a packaging variant, not part of the method.
+ *   Same arithmetic as q4_gemm: the activations are quantized exactly as
+ *   q4_quantize (NVFP4, RN scales, tensor scale *d_a_gscale) and multiplied with
+ *   the quantized weight on the tensor cores.  Allocates nothing: the quantized
+ *   activations go to a fixed array of Q4_NOALLOC_SCRATCH_BYTES inside the
+ *   library, which every GPU that loads the library keeps until the process
+ *   exits.  Codes [M, K/2] (rounded up to 256 bytes) plus the tensor-core scales
+ *   must fit in it (M * K / 2 + scales <= 32 MiB, e.g. M = 8192, K = 5120);
+ *   larger sizes return Q4_ERR_WORKSPACE before any launch.
+ *   All calls share that one array: calls whose work overlaps on the GPU (other
+ *   streams, other host threads) race on it and must be serialised by the
+ *   caller.  Each call overwrites every part of the array it reads, so nothing
+ *   has to be cleared between calls.  The first call on a device looks up the
+ *   array's device address (once per device, with that device current); make
+ *   that first call before any stream capture.  A CUDA failure returns
+ *   Q4_ERR_CUDA without updating q4_last_error().
+ *   Arguments as q4_gemm: a_bf16 bf16 [M, K]; b_codes/b_scales/d_b_gscale the
+ *   NVFP4 weight; y [M, N] of out_dt; K % 64 == 0, N % 8 == 0.
+ */
+#define Q4_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+Q4_API q4_status q4_gemm_a_bf16_noalloc(int64_t M, int64_t N, int64_t K, const void* a_bf16,
+                                        const float* d_a_gscale, const uint8_t* b_codes,
+                                        const uint8_t* b_scales, const float* d_b_gscale,
+                                        q4_dtype out_dt, void* y, void* stream);
+
+/*
  * q4_get_device_error -- synchronises `stream`, then reads and clears the
  *   library's device error word.  Returns Q4_ERR_TIMEOUT if a bounded wait
  *   inside a GEMM kernel gave up since the last call, Q4_ERR_CUDA if the

@@ -56,6 +56,7 @@ SIGNATURES = {
     "q4_gemm": (_I, [_I, _I, _I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _P, _I, _P, _P, _SZ, _P]),
     "q4_gemm_workspace_size": (_SZ, [_I, _I64, _I64, _I64, _I]),
     "q4_get_device_error": (_I, [_P]),
+    "q4_gemm_a_bf16_noalloc": (_I, [_I64, _I64, _I64, _P, _P, _P, _P, _P, _I, _P, _P]),
 }
 
 _lib = None
@@ -193,6 +194,19 @@ def q4_gemm(fmt: int, M: int, N: int, K: int, a: torch.Tensor, a_scales, a_gscal
                        _ptr(b_codes), _ptr(b_scales), _ptr(b_gscale), _dtype_code(y), _ptr(y),
                        _ptr(workspace), ws_bytes, _stream(stream))
     _check("q4_gemm", st)
+    return y
+
+
+def q4_gemm_a_bf16_noalloc(M: int, N: int, K: int, a: torch.Tensor, a_gscale, b_codes: torch.Tensor,
+                           b_scales: torch.Tensor, b_gscale, out_dtype=torch.bfloat16,
+                           y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """q4_gemm with bf16 activations using the library's fixed scratch array
+    instead of a workspace (for callers that cannot allocate at call time)."""
+    if y is None:
+        y = torch.empty((M, N), dtype=out_dtype, device=b_codes.device)
+    st = lib().q4_gemm_a_bf16_noalloc(M, N, K, _ptr(a), _ptr(a_gscale), _ptr(b_codes), _ptr(b_scales),
+                                      _ptr(b_gscale), _dtype_code(y), _ptr(y), _stream(stream))
+    _check("q4_gemm_a_bf16_noalloc", st)
     return y
 
 

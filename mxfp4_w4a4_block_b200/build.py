@@ -15,7 +15,7 @@ PKG = Path(__file__).resolve().parent
 CSRC = PKG / "csrc"
 INCLUDE = PKG.parent / "include"
 LIB = PKG / "libq4.so"
-SOURCES = ["q4_api.cu", "q4_quant.cu", "q4_gemm.cu"]
+SOURCES = ["q4_api.cu", "q4_quant.cu", "q4_gemm.cu", "q4_noalloc.cu"]
 HEADERS = ["q4_internal.h", "q4_codec.cuh", "q4_ptx.cuh"]
 
 NVCC_FLAGS = [
