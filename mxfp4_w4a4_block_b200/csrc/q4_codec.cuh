@@ -11,7 +11,8 @@
 namespace q4 {
 
 // Eight E2M1 codes from eight floats: round to nearest, ties to even
-// mantissa, saturating at +-6.  Element 0 lands in the low nibble.
+// mantissa, saturating at +-6, keeping the sign bit of values that round to
+// zero (-0.1 -> 0x8).  Element 0 lands in the low nibble.
 __device__ __forceinline__ uint32_t e2m1_pack8(const float (&v)[8]) {
     uint32_t out;
     asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
@@ -23,20 +24,6 @@ __device__ __forceinline__ uint32_t e2m1_pack8(const float (&v)[8]) {
         : "=r"(out)
         : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
     return out;
-}
-
-// The conversion above may return +0 for a negative input that rounds to
-// zero; the format keeps the input's sign bit there (code 0x8), so copy the
-// sign into every nibble whose magnitude bits are zero.
-__device__ __forceinline__ uint32_t e2m1_fix_signed_zero(uint32_t codes, const float (&v)[8]) {
-    uint32_t signs = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) signs |= (__float_as_uint(v[i]) >> 31) << (4 * i + 3);
-    // nibbles whose low three bits are zero
-    uint32_t mag = codes & 0x77777777u;
-    uint32_t nz = (mag | (mag >> 1) | (mag >> 2)) & 0x11111111u;  // bit 4i set if magnitude != 0
-    uint32_t zero_mask = (~nz & 0x11111111u) * 0x8u;               // bit 4i+3 set if magnitude == 0
-    return (codes & ~zero_mask) | (signs & zero_mask);
 }
 
 // Magnitude of an E2M1 code (low three bits) as float: 0, .5, 1, 1.5, 2, 3, 4, 6.

@@ -4,12 +4,17 @@
 //   warp 0      TMA producer: A and B code tiles (128-byte swizzle) by tiled
 //               tensor copies, scale atoms by contiguous bulk copies, into a
 //               STAGES-deep ring guarded by full/empty mbarriers;
-//   warp 1      allocates TMEM, and one elected lane issues per k-block the
-//               scale copies shared memory -> TMEM (tcgen05.cp) and the
-//               block-scaled MMAs into an FP32 accumulator in TMEM;
-//   warps 2..5  epilogue: TMEM -> registers (tcgen05.ld), times alpha,
-//               convert, store Y.
-// CTA tile 128 x 256, k-block 256 elements (128 bytes of codes per row).
+//   warp 1      allocates TMEM, and one lane issues per k-block the scale
+//               copies shared memory -> TMEM (tcgen05.cp) interleaved with
+//               the block-scaled MMAs into an FP32 accumulator in TMEM, from
+//               an unrolled loop over precomputed descriptors (the issue rate
+//               of this one thread bounds the tensor pipe);
+//   warps 2..9  epilogue: two warps per TMEM lane quarter each drain 128
+//               accumulator columns into registers (tcgen05.ld), release the
+//               accumulator to the next tile's MMAs, then scale, convert and
+//               store Y while those MMAs run.
+// CTA tile 128 x 256, k-block 256 elements (128 bytes of codes per row); the
+// scale columns in TMEM are double-buffered by k-block parity.
 // Every mbarrier wait is bounded; on time-out the kernel records an error and
 // winds down, waiting (bounded) for its own copies and MMAs before freeing TMEM.
 #include <cstdint>
@@ -40,11 +45,13 @@ constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_STAGE;
 constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_STAGE;
 constexpr int BAR_BYTES = 256;
 constexpr int SMEM_BYTES = OFF_BAR + BAR_BYTES + 1024;   // + alignment slack
-constexpr int THREADS = 192;
+constexpr int EPI_WARPS = 8;
+constexpr int THREADS = 64 + 32 * EPI_WARPS;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;          // 256 fp32 columns
-constexpr uint32_t SFA_COL = 256;        // 4 columns per scale atom
-constexpr uint32_t SFB_COL = 272;        // 8 columns per scale atom pair (two bands)
+constexpr uint32_t SF_COL = 256;         // two buffers of 48 columns (k-block parity)
+constexpr uint32_t SF_BUF = 48;          // per buffer: SFA 4 atoms x 4 columns, then SFB 4 atoms x 8
+constexpr uint32_t SFB_OFF = 16;
 }  // namespace gemm
 
 struct GemmDev {
@@ -111,7 +118,7 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
             mbar_init(&empty[s], 1);
         }
         mbar_init(tmem_full, 1);
-        mbar_init(tmem_empty, 128);
+        mbar_init(tmem_empty, 32 * EPI_WARPS);
         mbar_init(mma_done, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -135,6 +142,7 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
     const int nkb = (int)((p.K + KB_ELEMS - 1) / KB_ELEMS);
     const int mma_per_atom = MX ? 2 : 1;
     const int atoms_per_kb = 4 / mma_per_atom;
+    (void)lane;
     const int64_t bands_n = (p.N + 127) / 128;
 
     if (warp == 0) {
@@ -176,8 +184,14 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
     } else if (warp == 1) {
         if (lane == 0) {
             const uint32_t idesc0 = idesc_mxf4(BM, BN, MX);
+            const uint32_t idesc_hi = idesc_with_sf_id(idesc0, 2, 2);   // MXFP4: second MMA of an atom
+            // descriptor bases of stage 0; stage s adds s * stage bytes >> 4
+            const uint64_t adesc0 = smem_desc(smem_u32(smem), 16, 1024, 2);
+            const uint64_t bdesc0 = smem_desc(smem_u32(smem + OFF_B), 16, 1024, 2);
+            const uint64_t sfa0 = smem_desc(smem_u32(smem + OFF_SFA), 0, 128, 0);
+            const uint64_t sfb0 = smem_desc(smem_u32(smem + OFF_SFB), 0, 128, 0);
             int stage = 0;
-            uint32_t phase = 0, acc_phase = 0;
+            uint32_t phase = 0, acc_phase = 0, kpar = 0;
             for (int64_t t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x) {
                 if (!mbar_wait(tmem_empty, acc_phase ^ 1)) { *abort_flag = 1; break; }
                 tc_fence_after();
@@ -185,31 +199,51 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
                     if (!mbar_wait(&full[stage], phase)) { *abort_flag = 1; break; }
                     tc_fence_after();
                     const int64_t krem = p.K - (int64_t)kb * KB_ELEMS;
-                    const int kel = krem < KB_ELEMS ? (int)krem : KB_ELEMS;
-                    const int nmma = kel / 64;
-                    const int na = (nmma + mma_per_atom - 1) / mma_per_atom;
-                    const uint32_t sfa_s = smem_u32(smem + OFF_SFA + stage * SFA_STAGE);
-                    const uint32_t sfb_s = smem_u32(smem + OFF_SFB + stage * SFB_STAGE);
-                    for (int a = 0; a < na; ++a) {
-                        tmem_cp_sf(tmem + SFA_COL + a * 4, smem_desc(sfa_s + a * 512, 0, 128, 0));
-                        tmem_cp_sf(tmem + SFB_COL + a * 8, smem_desc(sfb_s + a * 512, 0, 128, 0));
-                        tmem_cp_sf(tmem + SFB_COL + a * 8 + 4, smem_desc(sfb_s + 2048 + a * 512, 0, 128, 0));
-                    }
-                    const uint64_t adesc = smem_desc(smem_u32(smem + stage * A_STAGE), 16, 1024, 2);
-                    const uint64_t bdesc = smem_desc(smem_u32(smem + OFF_B + stage * B_STAGE), 16, 1024, 2);
-                    for (int kk = 0; kk < nmma; ++kk) {
-                        const int atom = kk / mma_per_atom;
-                        const uint32_t sfid = MX ? (uint32_t)(kk % 2) * 2u : 0u;
-                        const uint32_t idesc = idesc_with_sf_id(idesc0, sfid, sfid);
-                        const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
-                        if (MX)
-                            mma_mxf4(tmem + ACC_COL, adesc + 2 * kk, bdesc + 2 * kk, idesc,
-                                     tmem + SFA_COL + atom * 4, tmem + SFB_COL + atom * 8, acc);
-                        else
-                            mma_nvf4(tmem + ACC_COL, adesc + 2 * kk, bdesc + 2 * kk, idesc,
-                                     tmem + SFA_COL + atom * 4, tmem + SFB_COL + atom * 8, acc);
+                    const int nmma = krem < KB_ELEMS ? (int)(krem / 64) : 4;
+                    const uint64_t ad = adesc0 + (uint64_t)(stage * (A_STAGE >> 4));
+                    const uint64_t bd = bdesc0 + (uint64_t)(stage * (B_STAGE >> 4));
+                    const uint64_t fa = sfa0 + (uint64_t)(stage * (SFA_STAGE >> 4));
+                    const uint64_t fb = sfb0 + (uint64_t)(stage * (SFB_STAGE >> 4));
+                    const uint32_t sfa = tmem + SF_COL + kpar * SF_BUF;
+                    const uint32_t sfb = sfa + SFB_OFF;
+                    uint32_t accf = kb > 0 ? 1u : 0u;
+                    if (nmma == 4) {
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const int atom = MX ? kk / 2 : kk;
+                            if (!MX || (kk & 1) == 0) {
+                                tmem_cp_sf(sfa + atom * 4, fa + atom * 32);
+                                tmem_cp_sf(sfb + atom * 8, fb + atom * 32);
+                                tmem_cp_sf(sfb + atom * 8 + 4, fb + 128 + atom * 32);
+                            }
+                            if (MX)
+                                mma_mxf4(tmem + ACC_COL, ad + 2 * kk, bd + 2 * kk, (kk & 1) ? idesc_hi : idesc0,
+                                         sfa + atom * 4, sfb + atom * 8, accf);
+                            else
+                                mma_nvf4(tmem + ACC_COL, ad + 2 * kk, bd + 2 * kk, idesc0, sfa + atom * 4,
+                                         sfb + atom * 8, accf);
+                            accf = 1u;
+                        }
+                    } else {
+                        // last, partial k-block (K % 256 != 0)
+                        for (int kk = 0; kk < nmma; ++kk) {
+                            const int atom = MX ? kk / 2 : kk;
+                            if (!MX || (kk & 1) == 0) {
+                                tmem_cp_sf(sfa + atom * 4, fa + atom * 32);
+                                tmem_cp_sf(sfb + atom * 8, fb + atom * 32);
+                                tmem_cp_sf(sfb + atom * 8 + 4, fb + 128 + atom * 32);
+                            }
+                            if (MX)
+                                mma_mxf4(tmem + ACC_COL, ad + 2 * kk, bd + 2 * kk, (kk & 1) ? idesc_hi : idesc0,
+                                         sfa + atom * 4, sfb + atom * 8, accf);
+                            else
+                                mma_nvf4(tmem + ACC_COL, ad + 2 * kk, bd + 2 * kk, idesc0, sfa + atom * 4,
+                                         sfb + atom * 8, accf);
+                            accf = 1u;
+                        }
                     }
                     tc_commit(&empty[stage]);
+                    kpar ^= 1u;
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
                 if (*abort_flag) break;
@@ -221,25 +255,32 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
             mbar_wait(mma_done, 0);
         }
     } else {
-        const int quad = warp & 3;                 // TMEM lane quadrant this warp may access
+        const int quad = warp & 3;                 // TMEM lane quarter this warp may access
+        const int half = (warp - 2) >> 2;          // which 128 accumulator columns
         const int row_in_tile = quad * 32 + lane;
         const float alpha = MX ? 1.0f : __fmul_rn(*p.a_gscale, *p.b_gscale);
+        const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + ACC_COL + half * 128;
         uint32_t acc_phase = 0;
         for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
             if (!mbar_wait(tmem_full, acc_phase)) { *abort_flag = 1; break; }
             tc_fence_after();
-            const int64_t mt = t % tiles_m, nt = t / tiles_m;
-            const int64_t row = mt * BM + row_in_tile;
-            for (int c = 0; c < BN / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + ACC_COL + c * 32, r);
-                tmem_ld_wait();
-                const int64_t col0 = nt * BN + c * 32;
-                if (row < p.M && col0 < p.N) store_row32(p.y, p.N, row, col0, r, alpha, p.out_bf16 != 0);
-            }
+            uint32_t r[4][32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld32(taddr + c * 32, r[c]);
+            tmem_ld_wait();
+            // the accumulator is in registers: let the next tile's MMAs start
             tc_fence_before();
             mbar_arrive(tmem_empty);
             acc_phase ^= 1;
+            const int64_t mt = t % tiles_m, nt = t / tiles_m;
+            const int64_t row = mt * BM + row_in_tile;
+            if (row < p.M) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int64_t col0 = nt * BN + half * 128 + c * 32;
+                    if (col0 < p.N) store_row32(p.y, p.N, row, col0, r[c], alpha, p.out_bf16 != 0);
+                }
+            }
         }
     }
 
@@ -470,7 +511,7 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
             NvScale sc = nv_scale_from_amax(amax, s_t, false);
 #pragma unroll
             for (int i = 0; i < 8; ++i) v[i] = sc.degenerate ? 0.0f : __fmul_rn(v[i], sc.inv);
-            const uint32_t codes = e2m1_fix_signed_zero(e2m1_pack8(v), v);
+            const uint32_t codes = e2m1_pack8(v);
             const int64_t k = ch * 8;
             const int kb = (int)(k >> 8);
             const int byte_in_row = (int)((k & 255) >> 1);

@@ -221,7 +221,7 @@ __global__ void __launch_bounds__(256) quantize_kernel(QuantParams p) {
 #pragma unroll
                 for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(v[i], mult);
             }
-            uint32_t codes = e2m1_fix_signed_zero(e2m1_pack8(v), v);
+            uint32_t codes = e2m1_pack8(v);
             if (valid[it])
                 *reinterpret_cast<uint32_t*>(p.codes + row * (p.cols / 2) + col / 2) = codes;
             if (lib == 0) {
@@ -300,7 +300,7 @@ __global__ void __launch_bounds__(256) sigma_delta_kernel(SigmaDeltaParams p) {
                 float x = degenerate ? 0.0f : __fmul_rn(wv[i], inv);
                 v[i] = __fadd_rn(x, rv[i]);
             }
-            uint32_t codes = e2m1_fix_signed_zero(e2m1_pack8(v), v);
+            uint32_t codes = e2m1_pack8(v);
 #pragma unroll
             for (int i = 0; i < 8; ++i) rv[i] = __fsub_rn(v[i], e2m1_value((codes >> (4 * i)) & 15u));
             const int64_t off = row * p.cols + col;
@@ -359,34 +359,52 @@ static int grid_for(int64_t tiles, int num_sms, int per_sm) {
     return (int)(tiles < cap ? tiles : cap);
 }
 
+// Grid of exactly the CTAs that fit on the GPU at once (a persistent
+// grid-stride launch), so the last wave is never partial.
+template <typename K>
+static int resident_grid(K kernel, int64_t tiles, int num_sms) {
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, 256, 0) != cudaSuccess || per_sm < 1)
+        per_sm = 4;
+    return grid_for(tiles, num_sms, per_sm);
+}
+
+template <int BLK, bool BF16, bool TC, bool RU, bool HAD, bool CHAN>
+static void launch_quant_one(const QuantParams& p, int64_t tiles, int num_sms, cudaStream_t st) {
+    auto k = quantize_kernel<BLK, BF16, TC, RU, HAD, CHAN>;
+    k<<<resident_grid(k, tiles, num_sms), 256, 0, st>>>(p);
+}
+
 template <int BLK, bool BF16, bool TC, bool RU>
-static void launch_quant_mx_variants(const QuantParams& p, bool had, bool chan, int grid, cudaStream_t st) {
-    if (had && chan) quantize_kernel<BLK, BF16, TC, RU, true, true><<<grid, 256, 0, st>>>(p);
-    else if (had) quantize_kernel<BLK, BF16, TC, RU, true, false><<<grid, 256, 0, st>>>(p);
-    else if (chan) quantize_kernel<BLK, BF16, TC, RU, false, true><<<grid, 256, 0, st>>>(p);
-    else quantize_kernel<BLK, BF16, TC, RU, false, false><<<grid, 256, 0, st>>>(p);
+static void launch_quant_mx_variants(const QuantParams& p, bool had, bool chan, int64_t tiles, int num_sms,
+                                     cudaStream_t st) {
+    if (had && chan) launch_quant_one<BLK, BF16, TC, RU, true, true>(p, tiles, num_sms, st);
+    else if (had) launch_quant_one<BLK, BF16, TC, RU, true, false>(p, tiles, num_sms, st);
+    else if (chan) launch_quant_one<BLK, BF16, TC, RU, false, true>(p, tiles, num_sms, st);
+    else launch_quant_one<BLK, BF16, TC, RU, false, false>(p, tiles, num_sms, st);
 }
 
 template <int BLK, bool BF16, bool TC>
-static void launch_quant_ru(const QuantParams& p, bool ru, bool had, bool chan, int grid, cudaStream_t st) {
+static void launch_quant_ru(const QuantParams& p, bool ru, bool had, bool chan, int64_t tiles, int num_sms,
+                            cudaStream_t st) {
     if constexpr (BLK == 16) {
-        if (ru) quantize_kernel<BLK, BF16, TC, true, false, false><<<grid, 256, 0, st>>>(p);
-        else quantize_kernel<BLK, BF16, TC, false, false, false><<<grid, 256, 0, st>>>(p);
+        if (ru) launch_quant_one<BLK, BF16, TC, true, false, false>(p, tiles, num_sms, st);
+        else launch_quant_one<BLK, BF16, TC, false, false, false>(p, tiles, num_sms, st);
     } else {
-        if (ru) launch_quant_mx_variants<BLK, BF16, TC, true>(p, had, chan, grid, st);
-        else launch_quant_mx_variants<BLK, BF16, TC, false>(p, had, chan, grid, st);
+        if (ru) launch_quant_mx_variants<BLK, BF16, TC, true>(p, had, chan, tiles, num_sms, st);
+        else launch_quant_mx_variants<BLK, BF16, TC, false>(p, had, chan, tiles, num_sms, st);
     }
 }
 
 template <int BLK>
 static void launch_quant_blk(const QuantParams& p, bool bf16, bool tc, bool ru, bool had, bool chan,
-                             int grid, cudaStream_t st) {
+                             int64_t tiles, int num_sms, cudaStream_t st) {
     if (bf16) {
-        if (tc) launch_quant_ru<BLK, true, true>(p, ru, had, chan, grid, st);
-        else launch_quant_ru<BLK, true, false>(p, ru, had, chan, grid, st);
+        if (tc) launch_quant_ru<BLK, true, true>(p, ru, had, chan, tiles, num_sms, st);
+        else launch_quant_ru<BLK, true, false>(p, ru, had, chan, tiles, num_sms, st);
     } else {
-        if (tc) launch_quant_ru<BLK, false, true>(p, ru, had, chan, grid, st);
-        else launch_quant_ru<BLK, false, false>(p, ru, had, chan, grid, st);
+        if (tc) launch_quant_ru<BLK, false, true>(p, ru, had, chan, tiles, num_sms, st);
+        else launch_quant_ru<BLK, false, false>(p, ru, had, chan, tiles, num_sms, st);
     }
 }
 
@@ -395,9 +413,8 @@ cudaError_t launch_quantize(const QuantParams& p, int blk, bool bf16, bool tc, b
     if (p.rows == 0 || p.cols == 0) return cudaSuccess;
     const int64_t tile_c = 4 * blk;
     const int64_t tiles = ((p.rows + 127) / 128) * ((p.cols + tile_c - 1) / tile_c);
-    const int grid = grid_for(tiles, num_sms, 8);
-    if (blk == 16) launch_quant_blk<16>(p, bf16, tc, ru, had, chan, grid, st);
-    else launch_quant_blk<32>(p, bf16, tc, ru, had, chan, grid, st);
+    if (blk == 16) launch_quant_blk<16>(p, bf16, tc, ru, had, chan, tiles, num_sms, st);
+    else launch_quant_blk<32>(p, bf16, tc, ru, had, chan, tiles, num_sms, st);
     return cudaGetLastError();
 }
 
@@ -405,14 +422,13 @@ cudaError_t launch_sigma_delta(const SigmaDeltaParams& p, int blk, bool tc, cuda
     if (p.rows == 0 || p.cols == 0) return cudaSuccess;
     const int64_t tile_c = 4 * blk;
     const int64_t tiles = ((p.rows + 127) / 128) * ((p.cols + tile_c - 1) / tile_c);
-    const int grid = grid_for(tiles, num_sms, 8);
+#define Q4_SD(B, T) { auto k = sigma_delta_kernel<B, T>; k<<<resident_grid(k, tiles, num_sms), 256, 0, st>>>(p); }
     if (blk == 16) {
-        if (tc) sigma_delta_kernel<16, true><<<grid, 256, 0, st>>>(p);
-        else sigma_delta_kernel<16, false><<<grid, 256, 0, st>>>(p);
+        if (tc) Q4_SD(16, true) else Q4_SD(16, false)
     } else {
-        if (tc) sigma_delta_kernel<32, true><<<grid, 256, 0, st>>>(p);
-        else sigma_delta_kernel<32, false><<<grid, 256, 0, st>>>(p);
+        if (tc) Q4_SD(32, true) else Q4_SD(32, false)
     }
+#undef Q4_SD
     return cudaGetLastError();
 }
 
