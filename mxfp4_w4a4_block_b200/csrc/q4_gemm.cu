@@ -4,12 +4,16 @@
 //   warp 0      TMA producer: A and B code tiles (128-byte swizzle) by tiled
 //               tensor copies, scale atoms by contiguous bulk copies, into a
 //               STAGES-deep ring guarded by full/empty mbarriers;
-//   warp 1      allocates TMEM, and one lane issues per k-block the scale
-//               copies shared memory -> TMEM (tcgen05.cp) interleaved with
-//               the block-scaled MMAs into an FP32 accumulator in TMEM, from
-//               an unrolled loop over precomputed descriptors (the issue rate
-//               of this one thread bounds the tensor pipe);
-//   warps 2..9  epilogue: two warps per TMEM lane quarter each drain 128
+//   warp 1      allocates TMEM, and one lane issues per k-block the copies of
+//               the A scale atoms shared memory -> TMEM (tcgen05.cp)
+//               interleaved with the block-scaled MMAs into an FP32
+//               accumulator in TMEM, from an unrolled loop over precomputed
+//               descriptors;
+//   warp 2      copies the B scale atoms into TMEM on its own, concurrently
+//               with the MMA stream (copies issued by the MMA thread would
+//               serialise with its MMAs), double-buffered by k-block parity
+//               and handed over through mbarriers;
+//   warps 3..10 epilogue: two warps per TMEM lane quarter each drain 128
 //               accumulator columns into registers (tcgen05.ld), release the
 //               accumulator to the next tile's MMAs, then scale, convert and
 //               store Y while those MMAs run.
@@ -43,10 +47,11 @@ constexpr int OFF_B = STAGES * A_STAGE;
 constexpr int OFF_SFA = OFF_B + STAGES * B_STAGE;
 constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_STAGE;
 constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_STAGE;
-constexpr int BAR_BYTES = 256;
+constexpr int BAR_BYTES = 512;
 constexpr int SMEM_BYTES = OFF_BAR + BAR_BYTES + 1024;   // + alignment slack
 constexpr int EPI_WARPS = 8;
-constexpr int THREADS = 64 + 32 * EPI_WARPS;
+constexpr int FIRST_EPI_WARP = 3;
+constexpr int THREADS = 32 * FIRST_EPI_WARP + 32 * EPI_WARPS;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;          // 256 fp32 columns
 constexpr uint32_t SF_COL = 256;         // two buffers of 48 columns (k-block parity)
@@ -106,7 +111,10 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
     uint64_t* tmem_full = empty + STAGES;
     uint64_t* tmem_empty = tmem_full + 1;
     uint64_t* mma_done = tmem_empty + 1;
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
+    uint64_t* sfb_full = mma_done + 1;       // [2] B scales of a k-block are in TMEM
+    uint64_t* sfb_empty = sfb_full + 2;      // [2] the MMAs reading a B-scale buffer are done
+    uint64_t* sf_done = sfb_empty + 2;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sf_done + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5;
@@ -120,6 +128,8 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
         mbar_init(tmem_full, 1);
         mbar_init(tmem_empty, 32 * EPI_WARPS);
         mbar_init(mma_done, 1);
+        for (int b = 0; b < 2; ++b) { mbar_init(&sfb_full[b], 1); mbar_init(&sfb_empty[b], 1); }
+        mbar_init(sf_done, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -189,21 +199,20 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
             const uint64_t adesc0 = smem_desc(smem_u32(smem), 16, 1024, 2);
             const uint64_t bdesc0 = smem_desc(smem_u32(smem + OFF_B), 16, 1024, 2);
             const uint64_t sfa0 = smem_desc(smem_u32(smem + OFF_SFA), 0, 128, 0);
-            const uint64_t sfb0 = smem_desc(smem_u32(smem + OFF_SFB), 0, 128, 0);
             int stage = 0;
-            uint32_t phase = 0, acc_phase = 0, kpar = 0;
+            uint32_t phase = 0, acc_phase = 0, kpar = 0, kcount = 0;
             for (int64_t t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x) {
                 if (!mbar_wait(tmem_empty, acc_phase ^ 1)) { *abort_flag = 1; break; }
                 tc_fence_after();
                 for (int kb = 0; kb < nkb; ++kb) {
                     if (!mbar_wait(&full[stage], phase)) { *abort_flag = 1; break; }
+                    if (!mbar_wait(&sfb_full[kpar], (kcount >> 1) & 1)) { *abort_flag = 1; break; }
                     tc_fence_after();
                     const int64_t krem = p.K - (int64_t)kb * KB_ELEMS;
                     const int nmma = krem < KB_ELEMS ? (int)(krem / 64) : 4;
                     const uint64_t ad = adesc0 + (uint64_t)(stage * (A_STAGE >> 4));
                     const uint64_t bd = bdesc0 + (uint64_t)(stage * (B_STAGE >> 4));
                     const uint64_t fa = sfa0 + (uint64_t)(stage * (SFA_STAGE >> 4));
-                    const uint64_t fb = sfb0 + (uint64_t)(stage * (SFB_STAGE >> 4));
                     const uint32_t sfa = tmem + SF_COL + kpar * SF_BUF;
                     const uint32_t sfb = sfa + SFB_OFF;
                     uint32_t accf = kb > 0 ? 1u : 0u;
@@ -211,11 +220,7 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk) {
                             const int atom = MX ? kk / 2 : kk;
-                            if (!MX || (kk & 1) == 0) {
-                                tmem_cp_sf(sfa + atom * 4, fa + atom * 32);
-                                tmem_cp_sf(sfb + atom * 8, fb + atom * 32);
-                                tmem_cp_sf(sfb + atom * 8 + 4, fb + 128 + atom * 32);
-                            }
+                            if (!MX || (kk & 1) == 0) tmem_cp_sf(sfa + atom * 4, fa + atom * 32);
                             if (MX)
                                 mma_mxf4(tmem + ACC_COL, ad + 2 * kk, bd + 2 * kk, (kk & 1) ? idesc_hi : idesc0,
                                          sfa + atom * 4, sfb + atom * 8, accf);
@@ -228,11 +233,7 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
                         // last, partial k-block (K % 256 != 0)
                         for (int kk = 0; kk < nmma; ++kk) {
                             const int atom = MX ? kk / 2 : kk;
-                            if (!MX || (kk & 1) == 0) {
-                                tmem_cp_sf(sfa + atom * 4, fa + atom * 32);
-                                tmem_cp_sf(sfb + atom * 8, fb + atom * 32);
-                                tmem_cp_sf(sfb + atom * 8 + 4, fb + 128 + atom * 32);
-                            }
+                            if (!MX || (kk & 1) == 0) tmem_cp_sf(sfa + atom * 4, fa + atom * 32);
                             if (MX)
                                 mma_mxf4(tmem + ACC_COL, ad + 2 * kk, bd + 2 * kk, (kk & 1) ? idesc_hi : idesc0,
                                          sfa + atom * 4, sfb + atom * 8, accf);
@@ -243,7 +244,9 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
                         }
                     }
                     tc_commit(&empty[stage]);
+                    tc_commit(&sfb_empty[kpar]);
                     kpar ^= 1u;
+                    ++kcount;
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
                 if (*abort_flag) break;
@@ -254,9 +257,38 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
             tc_commit(mma_done);
             mbar_wait(mma_done, 0);
         }
+    } else if (warp == 2) {
+        if (lane == 0) {
+            const uint64_t sfb0 = smem_desc(smem_u32(smem + OFF_SFB), 0, 128, 0);
+            int stage = 0;
+            uint32_t phase = 0, kpar = 0, kcount = 0;
+            for (int64_t t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x) {
+                for (int kb = 0; kb < nkb; ++kb) {
+                    if (!mbar_wait(&full[stage], phase)) { *abort_flag = 1; break; }
+                    // the MMAs that read this buffer two k-blocks ago are done
+                    if (!mbar_wait(&sfb_empty[kpar], ((kcount >> 1) & 1) ^ 1)) { *abort_flag = 1; break; }
+                    tc_fence_after();
+                    const int64_t krem = p.K - (int64_t)kb * KB_ELEMS;
+                    const int nmma = krem < KB_ELEMS ? (int)(krem / 64) : 4;
+                    const int na = (nmma + mma_per_atom - 1) / mma_per_atom;
+                    const uint64_t fb = sfb0 + (uint64_t)(stage * (SFB_STAGE >> 4));
+                    const uint32_t sfb = tmem + SF_COL + kpar * SF_BUF + SFB_OFF;
+                    for (int a = 0; a < na; ++a) {
+                        tmem_cp_sf(sfb + a * 8, fb + a * 32);
+                        tmem_cp_sf(sfb + a * 8 + 4, fb + 128 + a * 32);
+                    }
+                    tc_commit(&sfb_full[kpar]);
+                    kpar ^= 1u;
+                    ++kcount;
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                }
+            }
+            tc_commit(sf_done);
+            mbar_wait(sf_done, 0);
+        }
     } else {
         const int quad = warp & 3;                 // TMEM lane quarter this warp may access
-        const int half = (warp - 2) >> 2;          // which 128 accumulator columns
+        const int half = (warp - FIRST_EPI_WARP) >> 2;   // which 128 accumulator columns
         const int row_in_tile = quad * 32 + lane;
         const float alpha = MX ? 1.0f : __fmul_rn(*p.a_gscale, *p.b_gscale);
         const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + ACC_COL + half * 128;
