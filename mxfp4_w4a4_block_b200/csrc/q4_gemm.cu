@@ -23,6 +23,7 @@
 // winds down, waiting (bounded) for its own copies and MMAs before freeing TMEM.
 #include <cstdint>
 #include <cstdio>
+#include <cstring>
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -46,11 +47,14 @@ constexpr int SFB_STAGE = 2 * 4 * 512;   // 2 row bands of 128
 constexpr int OFF_B = STAGES * A_STAGE;
 constexpr int OFF_SFA = OFF_B + STAGES * B_STAGE;
 constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_STAGE;
-constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_STAGE;
+constexpr int OFF_EPI = OFF_SFB + STAGES * SFB_STAGE;   // 8 KB: one warp's 32 x 128 bf16 block
+constexpr int EPI_BYTES = 8192;
+constexpr int OFF_BAR = OFF_EPI + EPI_BYTES;
 constexpr int BAR_BYTES = 512;
 constexpr int SMEM_BYTES = OFF_BAR + BAR_BYTES + 1024;   // + alignment slack
+constexpr int SF_WARPS = 4;             // warps 2..5 stage scales, one per TMEM lane quarter
 constexpr int EPI_WARPS = 8;
-constexpr int FIRST_EPI_WARP = 3;
+constexpr int FIRST_EPI_WARP = 2 + SF_WARPS;
 constexpr int THREADS = 32 * FIRST_EPI_WARP + 32 * EPI_WARPS;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;          // 256 fp32 columns
@@ -100,9 +104,41 @@ __device__ __forceinline__ void store_row32(void* y, int64_t N, int64_t row, int
     }
 }
 
+// Scale atoms of one k-block from shared memory into TMEM by tcgen05.st.
+// Called by the four scale warps; warp w writes its TMEM lane quarter w % 4,
+// and every quarter receives the whole atom (the layout the block-scaled MMA
+// reads: lane 32q + r, column j of an atom holds row 32j + r's four scales).
+// Staging through registers keeps these writes out of the tensor pipe that
+// executes the MMAs (a tcgen05.cp would serialise with them).
+__device__ __forceinline__ void stage_scales(uint32_t quarter_taddr, const uint8_t* sfa_smem, const uint8_t* sfb_smem,
+                                             int na, int lane) {
+    for (int a = 0; a < na; ++a) {
+        const uint4 va = *reinterpret_cast<const uint4*>(sfa_smem + a * 512 + lane * 16);
+        const uint4 vb0 = *reinterpret_cast<const uint4*>(sfb_smem + a * 512 + lane * 16);
+        const uint4 vb1 = *reinterpret_cast<const uint4*>(sfb_smem + 2048 + a * 512 + lane * 16);
+        tmem_st4(quarter_taddr + a * 4, va.x, va.y, va.z, va.w);
+        tmem_st4(quarter_taddr + 16 + a * 8, vb0.x, vb0.y, vb0.z, vb0.w);
+        tmem_st4(quarter_taddr + 16 + a * 8 + 4, vb1.x, vb1.y, vb1.z, vb1.w);
+    }
+}
+
+// Store 64 bf16 results (already scaled and packed in pairs) of one row,
+// columns col0..col0+63 that are < N.
+__device__ __forceinline__ void store_row32_bf16(void* y, int64_t N, int64_t row, int64_t col0, const uint32_t (&a)[32],
+                                                 const uint32_t (&b)[32]) {
+    uint16_t* yp = reinterpret_cast<uint16_t*>(y) + row * N + col0;
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {
+        if (col0 + g * 8 >= N) break;
+        const uint32_t* src = g < 4 ? &a[4 * g] : &b[4 * (g - 4)];
+        *reinterpret_cast<uint4*>(yp + g * 8) = make_uint4(src[0], src[1], src[2], src[3]);
+    }
+}
+
 template <bool MX>
 __global__ void __launch_bounds__(gemm::THREADS, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmDev p) {
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const __grid_constant__ CUtensorMap tmY, GemmDev p) {
     using namespace gemm;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -111,10 +147,10 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
     uint64_t* tmem_full = empty + STAGES;
     uint64_t* tmem_empty = tmem_full + 1;
     uint64_t* mma_done = tmem_empty + 1;
-    uint64_t* sfb_full = mma_done + 1;       // [2] B scales of a k-block are in TMEM
-    uint64_t* sfb_empty = sfb_full + 2;      // [2] the MMAs reading a B-scale buffer are done
-    uint64_t* sf_done = sfb_empty + 2;
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sf_done + 1);
+    uint64_t* sf_ready = mma_done + 1;       // [2] a k-block's scales are in TMEM buffer b
+    uint64_t* sf_free = sf_ready + 2;        // [2] the MMAs reading scale buffer b are done
+    uint64_t* epi_turn = sf_free + 2;        // [EPI_WARPS] whose turn it is to use the store buffer
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(epi_turn + EPI_WARPS);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5;
@@ -128,8 +164,8 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
         mbar_init(tmem_full, 1);
         mbar_init(tmem_empty, 32 * EPI_WARPS);
         mbar_init(mma_done, 1);
-        for (int b = 0; b < 2; ++b) { mbar_init(&sfb_full[b], 1); mbar_init(&sfb_empty[b], 1); }
-        mbar_init(sf_done, 1);
+        for (int b = 0; b < 2; ++b) { mbar_init(&sf_ready[b], 32 * SF_WARPS); mbar_init(&sf_free[b], 1); }
+        for (int w = 0; w < EPI_WARPS; ++w) mbar_init(&epi_turn[w], 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -140,6 +176,7 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+        if (p.out_bf16) tma_prefetch_desc(&tmY);
     }
     tc_fence_before();
     __syncthreads();
@@ -152,7 +189,6 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
     const int nkb = (int)((p.K + KB_ELEMS - 1) / KB_ELEMS);
     const int mma_per_atom = MX ? 2 : 1;
     const int atoms_per_kb = 4 / mma_per_atom;
-    (void)lane;
     const int64_t bands_n = (p.N + 127) / 128;
 
     if (warp == 0) {
@@ -195,10 +231,8 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
         if (lane == 0) {
             const uint32_t idesc0 = idesc_mxf4(BM, BN, MX);
             const uint32_t idesc_hi = idesc_with_sf_id(idesc0, 2, 2);   // MXFP4: second MMA of an atom
-            // descriptor bases of stage 0; stage s adds s * stage bytes >> 4
             const uint64_t adesc0 = smem_desc(smem_u32(smem), 16, 1024, 2);
             const uint64_t bdesc0 = smem_desc(smem_u32(smem + OFF_B), 16, 1024, 2);
-            const uint64_t sfa0 = smem_desc(smem_u32(smem + OFF_SFA), 0, 128, 0);
             int stage = 0;
             uint32_t phase = 0, acc_phase = 0, kpar = 0, kcount = 0;
             for (int64_t t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x) {
@@ -206,13 +240,12 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
                 tc_fence_after();
                 for (int kb = 0; kb < nkb; ++kb) {
                     if (!mbar_wait(&full[stage], phase)) { *abort_flag = 1; break; }
-                    if (!mbar_wait(&sfb_full[kpar], (kcount >> 1) & 1)) { *abort_flag = 1; break; }
+                    if (!mbar_wait(&sf_ready[kpar], (kcount >> 1) & 1)) { *abort_flag = 1; break; }
                     tc_fence_after();
                     const int64_t krem = p.K - (int64_t)kb * KB_ELEMS;
                     const int nmma = krem < KB_ELEMS ? (int)(krem / 64) : 4;
                     const uint64_t ad = adesc0 + (uint64_t)(stage * (A_STAGE >> 4));
                     const uint64_t bd = bdesc0 + (uint64_t)(stage * (B_STAGE >> 4));
-                    const uint64_t fa = sfa0 + (uint64_t)(stage * (SFA_STAGE >> 4));
                     const uint32_t sfa = tmem + SF_COL + kpar * SF_BUF;
                     const uint32_t sfb = sfa + SFB_OFF;
                     uint32_t accf = kb > 0 ? 1u : 0u;
@@ -220,7 +253,6 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk) {
                             const int atom = MX ? kk / 2 : kk;
-                            if (!MX || (kk & 1) == 0) tmem_cp_sf(sfa + atom * 4, fa + atom * 32);
                             if (MX)
                                 mma_mxf4(tmem + ACC_COL, ad + 2 * kk, bd + 2 * kk, (kk & 1) ? idesc_hi : idesc0,
                                          sfa + atom * 4, sfb + atom * 8, accf);
@@ -230,10 +262,8 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
                             accf = 1u;
                         }
                     } else {
-                        // last, partial k-block (K % 256 != 0)
                         for (int kk = 0; kk < nmma; ++kk) {
                             const int atom = MX ? kk / 2 : kk;
-                            if (!MX || (kk & 1) == 0) tmem_cp_sf(sfa + atom * 4, fa + atom * 32);
                             if (MX)
                                 mma_mxf4(tmem + ACC_COL, ad + 2 * kk, bd + 2 * kk, (kk & 1) ? idesc_hi : idesc0,
                                          sfa + atom * 4, sfb + atom * 8, accf);
@@ -244,7 +274,7 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
                         }
                     }
                     tc_commit(&empty[stage]);
-                    tc_commit(&sfb_empty[kpar]);
+                    tc_commit(&sf_free[kpar]);
                     kpar ^= 1u;
                     ++kcount;
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -257,34 +287,29 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
             tc_commit(mma_done);
             mbar_wait(mma_done, 0);
         }
-    } else if (warp == 2) {
-        if (lane == 0) {
-            const uint64_t sfb0 = smem_desc(smem_u32(smem + OFF_SFB), 0, 128, 0);
-            int stage = 0;
-            uint32_t phase = 0, kpar = 0, kcount = 0;
-            for (int64_t t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x) {
-                for (int kb = 0; kb < nkb; ++kb) {
-                    if (!mbar_wait(&full[stage], phase)) { *abort_flag = 1; break; }
-                    // the MMAs that read this buffer two k-blocks ago are done
-                    if (!mbar_wait(&sfb_empty[kpar], ((kcount >> 1) & 1) ^ 1)) { *abort_flag = 1; break; }
-                    tc_fence_after();
-                    const int64_t krem = p.K - (int64_t)kb * KB_ELEMS;
-                    const int nmma = krem < KB_ELEMS ? (int)(krem / 64) : 4;
-                    const int na = (nmma + mma_per_atom - 1) / mma_per_atom;
-                    const uint64_t fb = sfb0 + (uint64_t)(stage * (SFB_STAGE >> 4));
-                    const uint32_t sfb = tmem + SF_COL + kpar * SF_BUF + SFB_OFF;
-                    for (int a = 0; a < na; ++a) {
-                        tmem_cp_sf(sfb + a * 8, fb + a * 32);
-                        tmem_cp_sf(sfb + a * 8 + 4, fb + 128 + a * 32);
-                    }
-                    tc_commit(&sfb_full[kpar]);
-                    kpar ^= 1u;
-                    ++kcount;
-                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
-                }
+    } else if (warp < FIRST_EPI_WARP) {
+        // scale warps: stage each k-block's scale atoms into a TMEM buffer
+        const uint32_t quarter = (uint32_t)(warp & 3) * 32u;
+        int stage = 0;
+        uint32_t phase = 0, kpar = 0, kcount = 0;
+        for (int64_t t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x) {
+            for (int kb = 0; kb < nkb; ++kb) {
+                if (!mbar_wait(&full[stage], phase)) { *abort_flag = 1; break; }
+                // the MMAs that read this buffer two k-blocks ago are done
+                if (!mbar_wait(&sf_free[kpar], ((kcount >> 1) & 1) ^ 1)) { *abort_flag = 1; break; }
+                tc_fence_after();
+                const int64_t krem = p.K - (int64_t)kb * KB_ELEMS;
+                const int nmma = krem < KB_ELEMS ? (int)(krem / 64) : 4;
+                const int na = (nmma + mma_per_atom - 1) / mma_per_atom;
+                stage_scales(tmem + (quarter << 16) + SF_COL + kpar * SF_BUF, smem + OFF_SFA + stage * SFA_STAGE,
+                             smem + OFF_SFB + stage * SFB_STAGE, na, lane);
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(&sf_ready[kpar]);
+                kpar ^= 1u;
+                ++kcount;
+                if (++stage == STAGES) { stage = 0; phase ^= 1; }
             }
-            tc_commit(sf_done);
-            mbar_wait(sf_done, 0);
         }
     } else {
         const int quad = warp & 3;                 // TMEM lane quarter this warp may access
@@ -292,28 +317,66 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
         const int row_in_tile = quad * 32 + lane;
         const float alpha = MX ? 1.0f : __fmul_rn(*p.a_gscale, *p.b_gscale);
         const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + ACC_COL + half * 128;
-        uint32_t acc_phase = 0;
-        for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
+        const bool out_bf16 = p.out_bf16 != 0;
+        const int order = warp - FIRST_EPI_WARP;          // position in the store-buffer turn chain
+        uint8_t* buf = smem + OFF_EPI;
+        uint32_t acc_phase = 0, iter = 0;
+        for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++iter) {
             if (!mbar_wait(tmem_full, acc_phase)) { *abort_flag = 1; break; }
             tc_fence_after();
-            uint32_t r[4][32];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32(taddr + c * 32, r[c]);
-            tmem_ld_wait();
-            // the accumulator is in registers: let the next tile's MMAs start
-            tc_fence_before();
-            mbar_arrive(tmem_empty);
-            acc_phase ^= 1;
             const int64_t mt = t % tiles_m, nt = t / tiles_m;
             const int64_t row = mt * BM + row_in_tile;
-            if (row < p.M) {
+            const int64_t col_base = nt * BN + half * 128;
+            uint32_t pk[2][32];          // bf16 pairs: [0] columns 0..63, [1] columns 64..127
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const int64_t col0 = nt * BN + half * 128 + c * 32;
-                    if (col0 < p.N) store_row32(p.y, p.N, row, col0, r[c], alpha, p.out_bf16 != 0);
+            for (int round = 0; round < 4; ++round) {
+                uint32_t r[32];
+                tmem_ld32(taddr + round * 32, r);
+                tmem_ld_wait();
+                if (round == 3) {
+                    // the whole accumulator slice is in registers: let the next tile's MMAs start
+                    tc_fence_before();
+                    mbar_arrive(tmem_empty);
+                }
+                if (out_bf16) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[2 * j]) * alpha,
+                                                                 __uint_as_float(r[2 * j + 1]) * alpha);
+                        pk[round >> 1][(round & 1) * 16 + j] = *reinterpret_cast<uint32_t*>(&h);
+                    }
+                } else if (row < p.M) {
+                    store_row32(p.y, p.N, row, col_base + round * 32, r, alpha, false);
                 }
             }
+            if (out_bf16) {
+                // Turn in the chain of epilogue warps sharing the 8 KB buffer: the
+                // warp's 32 rows x 128 columns go out as two 32 x 64 TMA boxes in
+                // the 128-byte-swizzled layout (conflict-free writes, coalesced
+                // stores; rows and columns outside Y are clipped by the TMA).
+                const bool first = order == 0;
+                if (!mbar_wait(&epi_turn[order], first ? ((iter & 1) ^ 1) : (iter & 1))) { *abort_flag = 1; break; }
+#pragma unroll
+                for (int b = 0; b < 2; ++b)
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        *reinterpret_cast<uint4*>(buf + b * 4096 + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                            make_uint4(pk[b][4 * c], pk[b][4 * c + 1], pk[b][4 * c + 2], pk[b][4 * c + 3]);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    const int32_t r0 = (int32_t)(mt * BM + quad * 32);
+                    tma_store_2d(&tmY, buf, (int32_t)col_base, r0);
+                    tma_store_2d(&tmY, buf + 4096, (int32_t)(col_base + 64), r0);
+                    bulk_commit_group();
+                    bulk_wait_read_all();
+                    mbar_arrive(&epi_turn[(order + 1) % EPI_WARPS]);
+                }
+                __syncwarp();
+            }
+            acc_phase ^= 1;
         }
+        if (lane == 0) bulk_wait_all();
     }
 
     tc_fence_before();
@@ -350,12 +413,333 @@ static bool make_code_map(CUtensorMap* map, const void* base, int64_t rows, int6
     return r == CUDA_SUCCESS;
 }
 
+// ------------------------------------------------------------------ CTA-pair GEMM
+// The same GEMM on CTA pairs (clusters of two CTAs on two SMs) with the
+// 2-SM MMA: a pair owns a 256 x 256 output tile, each CTA stages its own 128
+// rows of A, its own 128 rows of the 256-row B tile and the B scales of both
+// halves; the leader CTA issues one 256 x 256 x 64 MMA per K step for both
+// SMs, so per unit of work the issue, scale-copy and barrier overheads and
+// the per-SM shared-memory traffic for B are halved.  Both CTAs' TMA loads
+// complete on the leader's `full` barriers; the leader's commits are
+// multicast to both CTAs' `empty` and `tmem_full` barriers; both CTAs'
+// epilogue warps release the accumulators on the leader's `tmem_empty`.
+namespace pair {
+constexpr int BM = 128;                  // rows of A per CTA (pair tile 256)
+constexpr int BN = 256;                  // columns per pair tile (128 rows of B per CTA)
+constexpr int KB_BYTES = 128;
+constexpr int KB_ELEMS = 256;
+constexpr int STAGES = 5;
+constexpr int A_STAGE = BM * KB_BYTES;          // 16 KB
+constexpr int B_STAGE = (BN / 2) * KB_BYTES;    // 16 KB
+constexpr int SFA_STAGE = 2048;
+constexpr int SFB_STAGE = 4096;                 // band 0 at +0, band 1 at +2048
+constexpr int OFF_B = STAGES * A_STAGE;
+constexpr int OFF_SFA = OFF_B + STAGES * B_STAGE;
+constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_STAGE;
+constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_STAGE;
+constexpr int BAR_BYTES = 512;
+constexpr int SMEM_BYTES = OFF_BAR + BAR_BYTES + 1024;
+constexpr int EPI_WARPS = 8;
+constexpr int FIRST_EPI_WARP = 3;
+constexpr int THREADS = 32 * FIRST_EPI_WARP + 32 * EPI_WARPS;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t ACC_COL = 0;
+constexpr uint32_t SF_COL = 256;
+constexpr uint32_t SF_BUF = 48;
+constexpr uint32_t SFB_OFF = 16;
+}  // namespace pair
+
+template <bool MX>
+__global__ void __launch_bounds__(pair::THREADS, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB, GemmDev p) {
+    using namespace pair;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+    uint64_t* empty = full + STAGES;
+    uint64_t* tmem_full = empty + STAGES;
+    uint64_t* tmem_empty = tmem_full + 1;
+    uint64_t* mma_done = tmem_empty + 1;
+    uint64_t* sfb_full = mma_done + 1;
+    uint64_t* sfb_empty = sfb_full + 2;
+    uint64_t* sf_done = sfb_empty + 2;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sf_done + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(tmem_full, 1);
+        mbar_init(tmem_empty, 2 * 32 * EPI_WARPS);
+        mbar_init(mma_done, 1);
+        for (int b = 0; b < 2; ++b) { mbar_init(&sfb_full[b], 1); mbar_init(&sfb_empty[b], 1); }
+        mbar_init(sf_done, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc2(tmem_holder, TMEM_COLS);
+        tmem_relinquish2();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA); tma_prefetch_desc(&tmB);
+        tma_prefetch_desc(&tmSA); tma_prefetch_desc(&tmSB);
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();          // barriers and TMEM allocation are visible to the peer
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    const int64_t tiles_m = (p.M + 2 * BM - 1) / (2 * BM);
+    const int64_t tiles_n = (p.N + BN - 1) / BN;
+    const int64_t tiles = tiles_m * tiles_n;
+    const int64_t pair_id = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+    const int nkb = (int)((p.K + KB_ELEMS - 1) / KB_ELEMS);
+    const int mma_per_atom = MX ? 2 : 1;
+    const int atoms_per_kb = 4 / mma_per_atom;
+    const uint32_t sf_bytes = 512u * (uint32_t)atoms_per_kb;       // one band's scales per k-block
+    const uint32_t cta_bytes = A_STAGE + B_STAGE + 3u * sf_bytes;  // one CTA's loads per k-block
+
+    if (warp == 0) {
+        if (lane == 0) {
+            const uint32_t leader_full = mapa_shared(smem_u32(full), 0);
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t last_phase[STAGES];
+            bool issued[STAGES];
+            for (int s = 0; s < STAGES; ++s) issued[s] = false, last_phase[s] = 0;
+            for (int64_t t = pair_id; t < tiles && !*abort_flag; t += npairs) {
+                const int64_t mt = t % tiles_m, nt = t / tiles_m;
+                for (int kb = 0; kb < nkb; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1)) { *abort_flag = 1; break; }
+                    if (leader) mbar_arrive_expect_tx(&full[stage], 2u * cta_bytes);
+                    const uint32_t fb = leader_full + 8u * (uint32_t)stage;
+                    const int32_t krow = (int32_t)(2 * kb * atoms_per_kb);
+                    tma_load_2d_pair(smem + stage * A_STAGE, &tmA, fb, kb * KB_BYTES, (int32_t)(mt * 2 * BM + rank * BM));
+                    tma_load_2d_pair(smem + OFF_B + stage * B_STAGE, &tmB, fb, kb * KB_BYTES,
+                                     (int32_t)(nt * BN + rank * (BN / 2)));
+                    tma_load_2d_pair(smem + OFF_SFA + stage * SFA_STAGE, &tmSA, fb, 0,
+                                     (int32_t)(2 * (mt * 2 + rank) * p.catoms) + krow);
+                    tma_load_2d_pair(smem + OFF_SFB + stage * SFB_STAGE, &tmSB, fb, 0,
+                                     (int32_t)(2 * (nt * 2) * p.catoms) + krow);
+                    tma_load_2d_pair(smem + OFF_SFB + stage * SFB_STAGE + 2048, &tmSB, fb, 0,
+                                     (int32_t)(2 * (nt * 2 + 1) * p.catoms) + krow);
+                    issued[stage] = true;
+                    last_phase[stage] = phase;
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                }
+            }
+            // the leader's barriers count both CTAs' copies: wait for the last ones
+            if (leader)
+                for (int s = 0; s < STAGES; ++s)
+                    if (issued[s]) mbar_wait(&full[s], last_phase[s]);
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && leader) {
+            const uint32_t idesc0 = idesc_mxf4(2 * BM, BN, MX);
+            const uint32_t idesc_hi = idesc_with_sf_id(idesc0, 2, 2);
+            const uint64_t adesc0 = smem_desc(smem_u32(smem), 16, 1024, 2);
+            const uint64_t bdesc0 = smem_desc(smem_u32(smem + OFF_B), 16, 1024, 2);
+            const uint64_t sfa0 = smem_desc(smem_u32(smem + OFF_SFA), 0, 128, 0);
+            int stage = 0;
+            uint32_t phase = 0, acc_phase = 0, kpar = 0, kcount = 0;
+            for (int64_t t = pair_id; t < tiles && !*abort_flag; t += npairs) {
+                if (!mbar_wait(tmem_empty, acc_phase ^ 1)) { *abort_flag = 1; break; }
+                tc_fence_after();
+                for (int kb = 0; kb < nkb; ++kb) {
+                    if (!mbar_wait(&full[stage], phase)) { *abort_flag = 1; break; }
+                    if (!mbar_wait(&sfb_full[kpar], (kcount >> 1) & 1)) { *abort_flag = 1; break; }
+                    tc_fence_after();
+                    const int64_t krem = p.K - (int64_t)kb * KB_ELEMS;
+                    const int nmma = krem < KB_ELEMS ? (int)(krem / 64) : 4;
+                    const uint64_t ad = adesc0 + (uint64_t)(stage * (A_STAGE >> 4));
+                    const uint64_t bd = bdesc0 + (uint64_t)(stage * (B_STAGE >> 4));
+                    const uint64_t fa = sfa0 + (uint64_t)(stage * (SFA_STAGE >> 4));
+                    const uint32_t sfa = tmem + SF_COL + kpar * SF_BUF;
+                    const uint32_t sfb = sfa + SFB_OFF;
+                    uint32_t accf = kb > 0 ? 1u : 0u;
+                    for (int kk = 0; kk < nmma; ++kk) {
+                        const int atom = MX ? kk / 2 : kk;
+                        if (!MX || (kk & 1) == 0) tmem_cp_sf_pair(sfa + atom * 4, fa + atom * 32);
+                        if (MX)
+                            mma_mxf4_pair(tmem + ACC_COL, ad + 2 * kk, bd + 2 * kk, (kk & 1) ? idesc_hi : idesc0,
+                                          sfa + atom * 4, sfb + atom * 8, accf);
+                        else
+                            mma_nvf4_pair(tmem + ACC_COL, ad + 2 * kk, bd + 2 * kk, idesc0, sfa + atom * 4,
+                                          sfb + atom * 8, accf);
+                        accf = 1u;
+                    }
+                    tc_commit_pair_mc(&empty[stage], 0x3);
+                    tc_commit_pair(&sfb_empty[kpar]);
+                    kpar ^= 1u;
+                    ++kcount;
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                }
+                if (*abort_flag) break;
+                tc_commit_pair_mc(tmem_full, 0x3);
+                acc_phase ^= 1;
+            }
+            tc_commit_pair(mma_done);
+            mbar_wait(mma_done, 0);
+        }
+    } else if (warp == 2) {
+        if (lane == 0 && leader) {
+            const uint64_t sfb0 = smem_desc(smem_u32(smem + OFF_SFB), 0, 128, 0);
+            int stage = 0;
+            uint32_t phase = 0, kpar = 0, kcount = 0;
+            for (int64_t t = pair_id; t < tiles && !*abort_flag; t += npairs) {
+                for (int kb = 0; kb < nkb; ++kb) {
+                    if (!mbar_wait(&full[stage], phase)) { *abort_flag = 1; break; }
+                    if (!mbar_wait(&sfb_empty[kpar], ((kcount >> 1) & 1) ^ 1)) { *abort_flag = 1; break; }
+                    tc_fence_after();
+                    const int64_t krem = p.K - (int64_t)kb * KB_ELEMS;
+                    const int nmma = krem < KB_ELEMS ? (int)(krem / 64) : 4;
+                    const int na = (nmma + mma_per_atom - 1) / mma_per_atom;
+                    const uint64_t fb = sfb0 + (uint64_t)(stage * (SFB_STAGE >> 4));
+                    const uint32_t sfb = tmem + SF_COL + kpar * SF_BUF + SFB_OFF;
+                    for (int a = 0; a < na; ++a) {
+                        tmem_cp_sf_pair(sfb + a * 8, fb + a * 32);
+                        tmem_cp_sf_pair(sfb + a * 8 + 4, fb + 128 + a * 32);
+                    }
+                    tc_commit_pair(&sfb_full[kpar]);
+                    kpar ^= 1u;
+                    ++kcount;
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                }
+            }
+            tc_commit_pair(sf_done);
+            mbar_wait(sf_done, 0);
+        }
+    } else {
+        const int quad = warp & 3;
+        const int half = (warp - FIRST_EPI_WARP) >> 2;
+        const int row_in_tile = quad * 32 + lane;
+        const float alpha = MX ? 1.0f : __fmul_rn(*p.a_gscale, *p.b_gscale);
+        const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + ACC_COL + half * 128;
+        const uint32_t leader_tmem_empty = mapa_shared(smem_u32(tmem_empty), 0);
+        uint32_t acc_phase = 0;
+        for (int64_t t = pair_id; t < tiles; t += npairs) {
+            if (!mbar_wait(tmem_full, acc_phase)) { *abort_flag = 1; break; }
+            tc_fence_after();
+            uint32_t r[4][32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld32(taddr + c * 32, r[c]);
+            tmem_ld_wait();
+            tc_fence_before();
+            mbar_arrive_cluster(leader_tmem_empty);
+            acc_phase ^= 1;
+            const int64_t mt = t % tiles_m, nt = t / tiles_m;
+            const int64_t row = mt * 2 * BM + (int64_t)rank * BM + row_in_tile;
+            if (row < p.M) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int64_t col0 = nt * BN + half * 128 + c * 32;
+                    if (col0 < p.N) store_row32(p.y, p.N, row, col0, r[c], alpha, p.out_bf16 != 0);
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();          // both CTAs are done with the pair's barriers and TMEM
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc2(tmem, TMEM_COLS);
+    __syncthreads();
+    cluster_sync();
+}
+
+// The scale tensor (tensor-core layout) as rows of 256 bytes: a k-block's
+// atoms of one 128-row band are 2 * atoms_per_kb consecutive rows.
+static bool make_scale_map(CUtensorMap* map, const void* base, int64_t bytes, int box_rows) {
+    auto enc = tensor_map_encoder();
+    if (!enc || bytes % 256) return false;
+    cuuint64_t dims[2] = {256u, (cuuint64_t)(bytes / 256)};
+    cuuint64_t strides[1] = {256u};
+    cuuint32_t box[2] = {256u, (cuuint32_t)box_rows};
+    cuuint32_t es[2] = {1u, 1u};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// CTA-pair kernel for M >= 256 (off: the 1-CTA kernel with register-staged
+// scales is faster on the shapes measured so far).
+constexpr bool kUsePairKernel = false;
+
+static cudaError_t launch_gemm_pair(const GemmParams& p, const GemmDev& d, cudaStream_t st, int num_sms) {
+    using namespace pair;
+    CUtensorMap ma, mb, msa, msb;
+    const int blk = p.mxfp4 ? 32 : 16;
+    const int box_rows = 2 * (p.mxfp4 ? 2 : 4);
+    const int64_t sa_bytes = ((p.M + 127) / 128) * 128 * d.catoms * 4;
+    const int64_t sb_bytes = ((p.N + 127) / 128) * 128 * d.catoms * 4;
+    (void)blk;
+    if (!make_code_map(&ma, p.a_codes, p.M, p.K / 2, BM)) return cudaErrorInvalidValue;
+    if (!make_code_map(&mb, p.b_codes, p.N, p.K / 2, BN / 2)) return cudaErrorInvalidValue;
+    if (!make_scale_map(&msa, p.a_scales, sa_bytes, box_rows)) return cudaErrorInvalidValue;
+    if (!make_scale_map(&msb, p.b_scales, sb_bytes, box_rows)) return cudaErrorInvalidValue;
+    const int64_t tiles = ((p.M + 2 * BM - 1) / (2 * BM)) * ((p.N + BN - 1) / BN);
+    int pairs = num_sms / 2;
+    if (tiles < pairs) pairs = (int)tiles;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * pairs, 1, 1);
+    cfg.blockDim = dim3(THREADS, 1, 1);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e;
+    if (p.mxfp4) {
+        e = cudaFuncSetAttribute(gemm_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel<true>, ma, mb, msa, msb, d);
+    } else {
+        e = cudaFuncSetAttribute(gemm_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel<false>, ma, mb, msa, msb, d);
+    }
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+// Output Y [M, N] bf16 for TMA stores of 32-row x 64-column boxes, 128-byte swizzle.
+static bool make_out_map(CUtensorMap* map, void* y, int64_t M, int64_t N) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
+    cuuint64_t strides[1] = {(cuuint64_t)(N * 2)};
+    cuuint32_t box[2] = {64u, 32u};
+    cuuint32_t es[2] = {1u, 1u};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, y, dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 cudaError_t launch_gemm(const GemmParams& p, cudaStream_t st, int num_sms) {
     using namespace gemm;
     if (p.M == 0 || p.N == 0) return cudaSuccess;
-    CUtensorMap ma, mb;
+    CUtensorMap ma, mb, my;
     if (!make_code_map(&ma, p.a_codes, p.M, p.K / 2, BM)) return cudaErrorInvalidValue;
     if (!make_code_map(&mb, p.b_codes, p.N, p.K / 2, BN)) return cudaErrorInvalidValue;
+    std::memset(&my, 0, sizeof(my));
+    if (p.out_bf16 && !make_out_map(&my, p.y, p.M, p.N)) return cudaErrorInvalidValue;
     GemmDev d;
     d.M = p.M; d.N = p.N; d.K = p.K;
     d.a_scales = p.a_scales; d.b_scales = p.b_scales;
@@ -364,17 +748,18 @@ cudaError_t launch_gemm(const GemmParams& p, cudaStream_t st, int num_sms) {
     const int blk = p.mxfp4 ? 32 : 16;
     d.catoms = ((p.K / blk) + 3) / 4;
     d.out_bf16 = p.out_bf16 ? 1 : 0;
+    if (kUsePairKernel && p.M >= 2 * BM && num_sms >= 2) return launch_gemm_pair(p, d, st, num_sms);
     const int64_t tiles = ((p.M + BM - 1) / BM) * ((p.N + BN - 1) / BN);
     const int grid = (int)(tiles < num_sms ? tiles : num_sms);
     cudaError_t e;
     if (p.mxfp4) {
         e = cudaFuncSetAttribute(gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
         if (e != cudaSuccess) return e;
-        gemm_kernel<true><<<grid, THREADS, SMEM_BYTES, st>>>(ma, mb, d);
+        gemm_kernel<true><<<grid, THREADS, SMEM_BYTES, st>>>(ma, mb, my, d);
     } else {
         e = cudaFuncSetAttribute(gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
         if (e != cudaSuccess) return e;
-        gemm_kernel<false><<<grid, THREADS, SMEM_BYTES, st>>>(ma, mb, d);
+        gemm_kernel<false><<<grid, THREADS, SMEM_BYTES, st>>>(ma, mb, my, d);
     }
     return cudaGetLastError();
 }
@@ -386,8 +771,12 @@ cudaError_t launch_gemm(const GemmParams& p, cudaStream_t st, int num_sms) {
 // owns 128 weight rows; warps 2..5 first quantize all of X (M <= 128 rows) into
 // shared memory -- codes in the 128-byte-swizzled K-major operand layout, scales
 // in tensor-core atoms -- while warp 0 already streams weight tiles by TMA.
+// The activation loads are batched (QBATCH per thread in flight) because the
+// quantize phase is a chain of L2 round trips.
 namespace dec {
-constexpr int THREADS = 192;
+constexpr int QUANT_WARPS = 8;           // warps 2..9 quantize X; warps 2..5 also run the epilogue
+constexpr int THREADS = 64 + 32 * QUANT_WARPS;
+constexpr int QBATCH = 8;                // 16-byte activation loads in flight per thread
 constexpr int W_STAGE = 128 * 128;       // 16 KB of weight codes per k-block
 constexpr int SFW_STAGE = 4 * 512;
 constexpr uint32_t TMEM_COLS = 256;
@@ -439,7 +828,7 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-        mbar_init(x_ready, 128);
+        mbar_init(x_ready, 32 * QUANT_WARPS);
         mbar_init(tmem_full, 1);
         mbar_init(tmem_empty, 128);
         mbar_init(mma_done, 1);
@@ -516,47 +905,53 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
             mbar_wait(mma_done, 0);
         }
     } else {
-        // ---- quantize X into shared memory (128 threads)
+        // ---- quantize X into shared memory (warps 2..9)
         const int qt = threadIdx.x - 64;
+        constexpr int QT = 32 * QUANT_WARPS;
         const float s_t = *p.a_gscale;
-        for (int i = qt; i < nkb * 512; i += 128) reinterpret_cast<uint32_t*>(sxf)[i] = 0u;
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        const int64_t cpr = p.K / 8;                         // chunks per row
-        const int64_t total = (int64_t)np * cpr;
-        for (int64_t q = qt; q < total; q += 128) {
-            const int r = (int)(q / cpr);
-            const int64_t ch = q % cpr;
-            float v[8];
-            if (r < p.M) {
-                uint4 raw = __ldg(reinterpret_cast<const uint4*>(p.x + (int64_t)r * p.K + ch * 8));
-                v[0] = bf16_lo(raw.x); v[1] = bf16_hi(raw.x); v[2] = bf16_lo(raw.y); v[3] = bf16_hi(raw.y);
-                v[4] = bf16_lo(raw.z); v[5] = bf16_hi(raw.z); v[6] = bf16_lo(raw.w); v[7] = bf16_hi(raw.w);
-            } else {
+        for (int i = qt; i < nkb * 512; i += QT) reinterpret_cast<uint32_t*>(sxf)[i] = 0u;
+        asm volatile("bar.sync 1, %0;" ::"n"(QT) : "memory");
+        // thread -> (chunk ch of every row); the two halves of a 16-block are
+        // chunks ch and ch ^ 1, i.e. neighbouring lanes (cpr is a multiple of 8)
+        const int cpr = (int)(p.K / 8);
+        const int mrows = (int)p.M;
+        for (int ch = qt; ch < cpr; ch += QT) {
+            const unsigned mask = __activemask();
+            const int kb = ch >> 5;                        // 32 chunks of 8 per k-block
+            const int byte_in_row = (ch & 31) * 4;
+            for (int r0 = 0; r0 < np; r0 += QBATCH) {
+                uint4 raw[QBATCH];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) v[i] = 0.0f;
-            }
-            float amax = 0.0f;
+                for (int j = 0; j < QBATCH; ++j) {
+                    const int r = r0 + j;
+                    raw[j] = make_uint4(0u, 0u, 0u, 0u);
+                    if (r < mrows) raw[j] = __ldg(reinterpret_cast<const uint4*>(p.x + (int64_t)r * p.K + ch * 8));
+                }
 #pragma unroll
-            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
-            // the two halves of a 16-block are neighbouring q, hence neighbouring lanes
-            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-            NvScale sc = nv_scale_from_amax(amax, s_t, false);
+                for (int j = 0; j < QBATCH; ++j) {
+                    const int r = r0 + j;
+                    float v[8] = {bf16_lo(raw[j].x), bf16_hi(raw[j].x), bf16_lo(raw[j].y), bf16_hi(raw[j].y),
+                                  bf16_lo(raw[j].z), bf16_hi(raw[j].z), bf16_lo(raw[j].w), bf16_hi(raw[j].w)};
+                    float amax = 0.0f;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) v[i] = sc.degenerate ? 0.0f : __fmul_rn(v[i], sc.inv);
-            const uint32_t codes = e2m1_pack8(v);
-            const int64_t k = ch * 8;
-            const int kb = (int)(k >> 8);
-            const int byte_in_row = (int)((k & 255) >> 1);
-            *reinterpret_cast<uint32_t*>(sx + (size_t)kb * xslab + sw128_offset(r, byte_in_row)) = codes;
-            if ((ch & 1) == 0) {
-                const int64_t c = k >> 4;                         // scale column
-                const int cin = (int)(c & 15);                    // within the k-block
-                sxf[(size_t)kb * 2048 + (cin >> 2) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (cin & 3)] =
-                    (uint8_t)sc.byte;
+                    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+                    amax = fmaxf(amax, __shfl_xor_sync(mask, amax, 1));
+                    const NvScale sc = nv_scale_from_amax(amax, s_t, false);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) v[i] = sc.degenerate ? 0.0f : __fmul_rn(v[i], sc.inv);
+                    *reinterpret_cast<uint32_t*>(sx + (size_t)kb * xslab + sw128_offset(r, byte_in_row)) =
+                        e2m1_pack8(v);
+                    if ((ch & 1) == 0) {
+                        const int cin = (ch >> 1) & 15;            // scale column within the k-block
+                        sxf[(size_t)kb * 2048 + (cin >> 2) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (cin & 3)] =
+                            (uint8_t)sc.byte;
+                    }
+                }
             }
         }
         fence_proxy_async_smem();
         mbar_arrive(x_ready);
+        if (warp >= 6) goto decode_done;                     // warps 6..9 only quantize
 
         // ---- epilogue: thread = one weight row = one output column
         const int quad = warp & 3;
@@ -589,6 +984,7 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
             acc_phase ^= 1;
         }
     }
+decode_done:
     tc_fence_before();
     __syncthreads();
     tc_fence_after();

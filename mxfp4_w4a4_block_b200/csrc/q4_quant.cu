@@ -3,16 +3,10 @@
 // Hadamard-32 of MACaQ fused in), dequantization and the first-order
 // Sigma-Delta step of "Looped Transformer quantization", sec. 2.1.
 //
-// Work decomposition shared by quantize and Sigma-Delta: a CTA of 256 threads
-// owns a tile of 128 rows x (4 * block) columns, i.e. exactly one 512-byte
-// atom of the tensor-core scale layout.  Each thread owns 8 consecutive
-// elements of a row (one 16-byte bf16 load, two for fp32); the 2 (NVFP4) or 4
-// (MXFP4) threads of a block are neighbouring lanes and combine their amax
-// (and the Hadamard stages 8 and 16) with warp shuffles.  A warp reads whole
-// 128- or 256-byte row segments, so loads are fully coalesced; codes leave as
-// one 32-bit store per thread (32 contiguous bytes per row per 8 lanes) and
-// the scale atom is staged in shared memory and written as 512 contiguous
-// bytes.  All loads of a tile are issued before any arithmetic.
+// The quantizer gives each thread whole blocks (the scale rule, the Hadamard
+// rotation and the code packing stay in registers) and each CTA one scale
+// atom's worth of blocks, so the scales leave as 512 contiguous bytes.  The
+// Sigma-Delta step only reads scales and is a plain elementwise stream.
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -82,77 +76,51 @@ cudaError_t launch_amax(const void* x, int64_t n, bool bf16, float denom, float*
 }
 
 // ------------------------------------------------------------------ helpers
-// Eight inputs of one chunk as floats.
-template <bool BF16>
-struct Chunk;
+// Load one 16-byte chunk: 8 bf16 or 4 fp32 values (two chunks make 8 fp32).
+__device__ __forceinline__ void load_bf16x8(const void* src, float* v) {
+    const uint4 raw = __ldg(reinterpret_cast<const uint4*>(src));
+    v[0] = bf16_lo(raw.x); v[1] = bf16_hi(raw.x); v[2] = bf16_lo(raw.y); v[3] = bf16_hi(raw.y);
+    v[4] = bf16_lo(raw.z); v[5] = bf16_hi(raw.z); v[6] = bf16_lo(raw.w); v[7] = bf16_hi(raw.w);
+}
+__device__ __forceinline__ void load_f32x4(const void* src, float* v) {
+    const float4 f = __ldg(reinterpret_cast<const float4*>(src));
+    v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+}
 
-template <>
-struct Chunk<true> {
-    uint4 raw;
-    __device__ __forceinline__ void load(const void* base) { raw = __ldcs(reinterpret_cast<const uint4*>(base)); }
-    __device__ __forceinline__ void zero() { raw = make_uint4(0, 0, 0, 0); }
-    __device__ __forceinline__ void to_float(float (&v)[8]) const {
-        v[0] = bf16_lo(raw.x); v[1] = bf16_hi(raw.x); v[2] = bf16_lo(raw.y); v[3] = bf16_hi(raw.y);
-        v[4] = bf16_lo(raw.z); v[5] = bf16_hi(raw.z); v[6] = bf16_lo(raw.w); v[7] = bf16_hi(raw.w);
-    }
-};
-
-template <>
-struct Chunk<false> {
-    float4 a, b;
-    __device__ __forceinline__ void load(const void* base) {
-        const float4* p = reinterpret_cast<const float4*>(base);
-        a = __ldcs(p);
-        b = __ldcs(p + 1);
-    }
-    __device__ __forceinline__ void zero() { a = b = make_float4(0.f, 0.f, 0.f, 0.f); }
-    __device__ __forceinline__ void to_float(float (&v)[8]) const {
-        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-    }
-};
-
-// In-register stages (strides 1, 2, 4) of the Sylvester Walsh-Hadamard
-// transform over 8 consecutive elements, then the cross-lane stages 8 and 16
-// with the partner lanes of the same 32-block.  `lib` is the lane's index
-// inside its block (0..3).  All lanes of the warp must call this.
-__device__ __forceinline__ void fwht32_warp(float (&v)[8], int lib) {
+// Sylvester-order Walsh-Hadamard butterflies over 32 values held by one
+// thread (strides 1, 2, 4, 8, 16; (a, b) -> (a + b, a - b)), unnormalised.
+__device__ __forceinline__ void fwht32_reg(float (&v)[32]) {
 #pragma unroll
-    for (int h = 1; h < 8; h <<= 1) {
+    for (int h = 1; h < 32; h <<= 1) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < 32; ++i) {
             if ((i & h) == 0) {
-                float a = v[i], b = v[i + h];
+                const float a = v[i], b = v[i + h];
                 v[i] = __fadd_rn(a, b);
                 v[i + h] = __fsub_rn(a, b);
             }
         }
     }
-#pragma unroll
-    for (int lm = 1; lm <= 2; lm <<= 1) {
-        const bool upper = (lib & lm) != 0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            float p = __shfl_xor_sync(0xffffffffu, v[i], lm);
-            // lower element: a + b (a = own value); upper element: a - b with
-            // a = the lower partner's value and b = own value
-            v[i] = upper ? __fsub_rn(p, v[i]) : __fadd_rn(v[i], p);
-        }
-    }
 }
 
 // ------------------------------------------------------------------ quantize
+// One thread per block.  A CTA of 256 threads owns a tile of 128 rows x 4
+// blocks -- exactly one 512-byte atom of the tensor-core scale layout -- so
+// each thread quantizes 2 blocks per tile.  Lanes 4k..4k+3 of a warp take the
+// 4 consecutive blocks of one row, so a warp's loads cover 8 whole row
+// segments (128 or 256 bytes each of bf16); the first 16-byte load of a block
+// brings its lines into L1 for the rest.  All loads of a tile are issued
+// before any arithmetic.
 template <int BLK, bool BF16, bool TC, bool RU, bool HAD, bool CHAN>
 __global__ void __launch_bounds__(256) quantize_kernel(QuantParams p) {
     constexpr int TILE_C = 4 * BLK;          // columns per tile (one scale atom)
-    constexpr int CPR = TILE_C / 8;          // 8-element chunks per tile row
-    constexpr int ITER = 128 * CPR / 256;    // chunks per thread per tile
-    constexpr int TPB = BLK / 8;             // threads per block
+    constexpr int BPT = 2;                   // blocks per thread per tile
     constexpr int ESZ = BF16 ? 2 : 4;
+    constexpr int LOADS = BLK * ESZ / 16;    // 16-byte loads per block
+    constexpr int PER_LOAD = 16 / ESZ;       // values per load
     __shared__ __align__(16) uint8_t sf_atom[512];
 
     const int tid = threadIdx.x;
-    const int lane = tid & 31;
-    const int lib = lane & (TPB - 1);
     const int64_t tiles_c = (p.cols + TILE_C - 1) / TILE_C;
     const int64_t tiles = ((p.rows + 127) / 128) * tiles_c;
     const float s_t = (BLK == 16) ? *p.gscale : 0.0f;
@@ -163,78 +131,80 @@ __global__ void __launch_bounds__(256) quantize_kernel(QuantParams p) {
         const int64_t tr = t / tiles_c, tc = t % tiles_c;
         const int64_t row0 = tr * 128, col0 = tc * TILE_C;
 
-        Chunk<BF16> ch[ITER];
-        bool valid[ITER];
+        float v[BPT][BLK];
+        bool valid[BPT];
 #pragma unroll
-        for (int it = 0; it < ITER; ++it) {
-            const int q = it * 256 + tid;
-            const int64_t row = row0 + q / CPR;
-            const int64_t col = col0 + (q % CPR) * 8;
+        for (int it = 0; it < BPT; ++it) {
+            const int bt = it * 256 + tid;            // block inside the tile
+            const int64_t row = row0 + (bt >> 2);
+            const int64_t col = col0 + (bt & 3) * BLK;
             valid[it] = row < p.rows && col < p.cols;
-            if (valid[it]) ch[it].load(xb + (row * p.ld + col) * ESZ);
-            else ch[it].zero();
+            if (valid[it]) {
+                const char* src = xb + (row * p.ld + col) * ESZ;
+#pragma unroll
+                for (int l = 0; l < LOADS; ++l) {
+                    if (BF16) load_bf16x8(src + 16 * l, &v[it][PER_LOAD * l]);
+                    else load_f32x4(src + 16 * l, &v[it][PER_LOAD * l]);
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < BLK; ++i) v[it][i] = 0.0f;
+            }
         }
 #pragma unroll
-        for (int it = 0; it < ITER; ++it) {
-            const int q = it * 256 + tid;
-            const int rt = q / CPR;                   // row inside the tile
-            const int cq = q % CPR;                   // chunk inside the row
+        for (int it = 0; it < BPT; ++it) {
+            const int bt = it * 256 + tid;
+            const int rt = bt >> 2, cb = bt & 3;
             const int64_t row = row0 + rt;
-            const int64_t col = col0 + cq * 8;
-            float v[8];
-            ch[it].to_float(v);
-            if (CHAN) {
-                float c[8];
-                if (valid[it]) {
-                    const float4* cp = reinterpret_cast<const float4*>(p.chan + col);
-                    float4 c0 = __ldg(cp), c1 = __ldg(cp + 1);
-                    c[0] = c0.x; c[1] = c0.y; c[2] = c0.z; c[3] = c0.w;
-                    c[4] = c1.x; c[5] = c1.y; c[6] = c1.z; c[7] = c1.w;
-                } else {
+            const int64_t col = col0 + cb * BLK;
+            if (CHAN && valid[it]) {
+                const float4* cp = reinterpret_cast<const float4*>(p.chan + col);
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) c[i] = 0.0f;
+                for (int q = 0; q < BLK / 4; ++q) {
+                    const float4 c = __ldg(cp + q);
+                    v[it][4 * q] = __fmul_rn(v[it][4 * q], c.x);
+                    v[it][4 * q + 1] = __fmul_rn(v[it][4 * q + 1], c.y);
+                    v[it][4 * q + 2] = __fmul_rn(v[it][4 * q + 2], c.z);
+                    v[it][4 * q + 3] = __fmul_rn(v[it][4 * q + 3], c.w);
                 }
-#pragma unroll
-                for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(v[i], c[i]);
             }
-            if (HAD) {
-                fwht32_warp(v, lib);
+            if constexpr (HAD) {
+                fwht32_reg(*reinterpret_cast<float(*)[32]>(&v[it][0]));
 #pragma unroll
-                for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(v[i], inv_sqrt32);
+                for (int i = 0; i < BLK; ++i) v[it][i] = __fmul_rn(v[it][i], inv_sqrt32);
             }
             float amax = 0.0f;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
-#pragma unroll
-            for (int o = 1; o < TPB; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-
+            for (int i = 0; i < BLK; ++i) amax = fmaxf(amax, fabsf(v[it][i]));
             uint32_t byte;
-            if (BLK == 16) {
-                NvScale s = nv_scale_from_amax(amax, s_t, RU);
-                byte = s.byte;
+            if constexpr (BLK == 16) {
+                const NvScale sc = nv_scale_from_amax(amax, s_t, RU);
+                byte = sc.byte;
 #pragma unroll
-                for (int i = 0; i < 8; ++i) v[i] = s.degenerate ? 0.0f : __fmul_rn(v[i], s.inv);
+                for (int i = 0; i < BLK; ++i) v[it][i] = sc.degenerate ? 0.0f : __fmul_rn(v[it][i], sc.inv);
             } else {
-                int e = mx_exponent(amax, RU);
+                const int e = mx_exponent(amax, RU);
                 byte = (uint32_t)(e + 127);
-                float mult = exp2_int(-e);
+                const float mult = exp2_int(-e);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(v[i], mult);
+                for (int i = 0; i < BLK; ++i) v[it][i] = __fmul_rn(v[it][i], mult);
             }
-            uint32_t codes = e2m1_pack8(v);
-            if (valid[it])
-                *reinterpret_cast<uint32_t*>(p.codes + row * (p.cols / 2) + col / 2) = codes;
-            if (lib == 0) {
-                const int cb = cq / TPB;              // block inside the tile (0..3)
-                if (TC) sf_atom[(rt & 31) * 16 + (rt >> 5) * 4 + cb] = (uint8_t)byte;
-                else if (valid[it]) p.scales[row * p.scols + tc * 4 + cb] = (uint8_t)byte;
+            uint32_t w[BLK / 8];
+#pragma unroll
+            for (int g = 0; g < BLK / 8; ++g) w[g] = e2m1_pack8(*reinterpret_cast<float(*)[8]>(&v[it][8 * g]));
+            if (valid[it]) {
+                uint8_t* dst = p.codes + row * (p.cols / 2) + col / 2;
+                if constexpr (BLK == 16) *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
+                else *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
             }
+            if (TC) sf_atom[(rt & 31) * 16 + (rt >> 5) * 4 + cb] = (uint8_t)byte;
+            else if (valid[it]) p.scales[row * p.scols + tc * 4 + cb] = (uint8_t)byte;
         }
         if (TC) {
             __syncthreads();
             if (tid < 32) {
-                uint4 w = reinterpret_cast<const uint4*>(sf_atom)[tid];
-                reinterpret_cast<uint4*>(p.scales + (tr * p.catoms + tc) * 512)[tid] = w;
+                const uint4 a = reinterpret_cast<const uint4*>(sf_atom)[tid];
+                reinterpret_cast<uint4*>(p.scales + (tr * p.catoms + tc) * 512)[tid] = a;
             }
             __syncthreads();
         }
@@ -242,73 +212,63 @@ __global__ void __launch_bounds__(256) quantize_kernel(QuantParams p) {
 }
 
 // ------------------------------------------------------------------ sigma-delta
+// Elementwise over 8-weight chunks (grid-stride, two chunks per thread in
+// flight): it reads the fixed block scales and streams w, r in, r out, codes.
+template <int BLK, bool TC>
+__device__ __forceinline__ void sigma_delta_chunk(const SigmaDeltaParams& p, float s_t, int64_t row, int64_t col,
+                                                  const float4& w0, const float4& w1, const float4& r0,
+                                                  const float4& r1, uint32_t sb) {
+    float inv;
+    bool degenerate;
+    if (BLK == 16) {
+        const NvScale s = nv_scale_from_byte(sb, s_t);
+        inv = s.inv;
+        degenerate = s.degenerate;
+    } else {
+        inv = exp2_int(127 - (int)sb);
+        degenerate = false;
+    }
+    const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+    float rv[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float x = degenerate ? 0.0f : __fmul_rn(wv[i], inv);
+        v[i] = __fadd_rn(x, rv[i]);
+    }
+    const uint32_t codes = e2m1_pack8(v);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) rv[i] = __fsub_rn(v[i], e2m1_value((codes >> (4 * i)) & 15u));
+    const int64_t off = row * p.cols + col;
+    float4* rp = reinterpret_cast<float4*>(p.residue + off);
+    rp[0] = make_float4(rv[0], rv[1], rv[2], rv[3]);
+    rp[1] = make_float4(rv[4], rv[5], rv[6], rv[7]);
+    *reinterpret_cast<uint32_t*>(p.codes + row * (p.cols / 2) + col / 2) = codes;
+}
+
 template <int BLK, bool TC>
 __global__ void __launch_bounds__(256) sigma_delta_kernel(SigmaDeltaParams p) {
-    constexpr int TILE_C = 4 * BLK;
-    constexpr int CPR = TILE_C / 8;
-    constexpr int ITER = 128 * CPR / 256;
-    const int tid = threadIdx.x;
-    const int64_t tiles_c = (p.cols + TILE_C - 1) / TILE_C;
-    const int64_t tiles = ((p.rows + 127) / 128) * tiles_c;
+    const int64_t cpr = p.cols / 8;
+    const int64_t total = p.rows * cpr;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     const float s_t = (BLK == 16) ? *p.gscale : 0.0f;
-
-    for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
-        const int64_t tr = t / tiles_c, tc = t % tiles_c;
-        const int64_t row0 = tr * 128, col0 = tc * TILE_C;
-        float4 w[ITER][2], r[ITER][2];
-        uint32_t sb[ITER];
-        bool valid[ITER];
-#pragma unroll
-        for (int it = 0; it < ITER; ++it) {
-            const int q = it * 256 + tid;
-            const int64_t row = row0 + q / CPR;
-            const int64_t col = col0 + (q % CPR) * 8;
-            valid[it] = row < p.rows && col < p.cols;
-            if (valid[it]) {
-                const int64_t off = row * p.cols + col;
-                const float4* wp = reinterpret_cast<const float4*>(p.w + off);
-                const float4* rp = reinterpret_cast<const float4*>(p.residue + off);
-                w[it][0] = __ldcs(wp); w[it][1] = __ldcs(wp + 1);
-                r[it][0] = __ldcs(rp); r[it][1] = __ldcs(rp + 1);
-                const int64_t c = col / BLK;
-                sb[it] = TC ? p.scales[tc_scale_offset(row, c, p.catoms)] : p.scales[row * p.scols + c];
-            }
-        }
-#pragma unroll
-        for (int it = 0; it < ITER; ++it) {
-            if (!valid[it]) continue;
-            const int q = it * 256 + tid;
-            const int64_t row = row0 + q / CPR;
-            const int64_t col = col0 + (q % CPR) * 8;
-            float inv;
-            bool degenerate;
-            if (BLK == 16) {
-                NvScale s = nv_scale_from_byte(sb[it], s_t);
-                inv = s.inv;
-                degenerate = s.degenerate;
-            } else {
-                inv = exp2_int(127 - (int)sb[it]);
-                degenerate = false;
-            }
-            float wv[8] = {w[it][0].x, w[it][0].y, w[it][0].z, w[it][0].w,
-                           w[it][1].x, w[it][1].y, w[it][1].z, w[it][1].w};
-            float rv[8] = {r[it][0].x, r[it][0].y, r[it][0].z, r[it][0].w,
-                           r[it][1].x, r[it][1].y, r[it][1].z, r[it][1].w};
-            float v[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                float x = degenerate ? 0.0f : __fmul_rn(wv[i], inv);
-                v[i] = __fadd_rn(x, rv[i]);
-            }
-            uint32_t codes = e2m1_pack8(v);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) rv[i] = __fsub_rn(v[i], e2m1_value((codes >> (4 * i)) & 15u));
-            const int64_t off = row * p.cols + col;
-            float4* rp = reinterpret_cast<float4*>(p.residue + off);
-            rp[0] = make_float4(rv[0], rv[1], rv[2], rv[3]);
-            rp[1] = make_float4(rv[4], rv[5], rv[6], rv[7]);
-            *reinterpret_cast<uint32_t*>(p.codes + row * (p.cols / 2) + col / 2) = codes;
-        }
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += 2 * stride) {
+        const int64_t j = i + stride;
+        const bool has2 = j < total;
+        const int64_t row_a = i / cpr, col_a = (i % cpr) * 8;
+        const int64_t row_b = has2 ? j / cpr : row_a, col_b = has2 ? (j % cpr) * 8 : col_a;
+        const float4* wa = reinterpret_cast<const float4*>(p.w + row_a * p.cols + col_a);
+        const float4* ra = reinterpret_cast<const float4*>(p.residue + row_a * p.cols + col_a);
+        const float4* wb = reinterpret_cast<const float4*>(p.w + row_b * p.cols + col_b);
+        const float4* rb = reinterpret_cast<const float4*>(p.residue + row_b * p.cols + col_b);
+        const float4 wa0 = __ldcs(wa), wa1 = __ldcs(wa + 1), ra0 = __ldcs(ra), ra1 = __ldcs(ra + 1);
+        float4 wb0 = wa0, wb1 = wa1, rb0 = ra0, rb1 = ra1;
+        if (has2) { wb0 = __ldcs(wb); wb1 = __ldcs(wb + 1); rb0 = __ldcs(rb); rb1 = __ldcs(rb + 1); }
+        const int64_t ca = col_a / BLK, cbk = col_b / BLK;
+        const uint32_t sa = TC ? p.scales[tc_scale_offset(row_a, ca, p.catoms)] : p.scales[row_a * p.scols + ca];
+        const uint32_t sbb = TC ? p.scales[tc_scale_offset(row_b, cbk, p.catoms)] : p.scales[row_b * p.scols + cbk];
+        sigma_delta_chunk<BLK, TC>(p, s_t, row_a, col_a, wa0, wa1, ra0, ra1, sa);
+        if (has2) sigma_delta_chunk<BLK, TC>(p, s_t, row_b, col_b, wb0, wb1, rb0, rb1, sbb);
     }
 }
 
@@ -420,8 +380,7 @@ cudaError_t launch_quantize(const QuantParams& p, int blk, bool bf16, bool tc, b
 
 cudaError_t launch_sigma_delta(const SigmaDeltaParams& p, int blk, bool tc, cudaStream_t st, int num_sms) {
     if (p.rows == 0 || p.cols == 0) return cudaSuccess;
-    const int64_t tile_c = 4 * blk;
-    const int64_t tiles = ((p.rows + 127) / 128) * ((p.cols + tile_c - 1) / tile_c);
+    const int64_t tiles = (p.rows * (p.cols / 8) + 511) / 512;   // CTAs of 256 threads, 2 chunks each
 #define Q4_SD(B, T) { auto k = sigma_delta_kernel<B, T>; k<<<resident_grid(k, tiles, num_sms), 256, 0, st>>>(p); }
     if (blk == 16) {
         if (tc) Q4_SD(16, true) else Q4_SD(16, false)
