@@ -58,7 +58,8 @@ constexpr int FIRST_EPI_WARP = 2 + SF_WARPS;
 constexpr int THREADS = 32 * FIRST_EPI_WARP + 32 * EPI_WARPS;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;          // 256 fp32 columns
-constexpr uint32_t SF_COL = 256;         // two buffers of 48 columns (k-block parity)
+constexpr uint32_t SF_COL = 256;         // SF_NBUF buffers of 48 columns, one per k-block in flight
+constexpr int SF_NBUF = 4;
 constexpr uint32_t SF_BUF = 48;          // per buffer: SFA 4 atoms x 4 columns, then SFB 4 atoms x 8
 constexpr uint32_t SFB_OFF = 16;
 }  // namespace gemm
@@ -147,9 +148,9 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
     uint64_t* tmem_full = empty + STAGES;
     uint64_t* tmem_empty = tmem_full + 1;
     uint64_t* mma_done = tmem_empty + 1;
-    uint64_t* sf_ready = mma_done + 1;       // [2] a k-block's scales are in TMEM buffer b
-    uint64_t* sf_free = sf_ready + 2;        // [2] the MMAs reading scale buffer b are done
-    uint64_t* epi_turn = sf_free + 2;        // [EPI_WARPS] whose turn it is to use the store buffer
+    uint64_t* sf_ready = mma_done + 1;       // [SF_NBUF] a k-block's scales are in TMEM buffer b
+    uint64_t* sf_free = sf_ready + SF_NBUF;  // [SF_NBUF] the MMAs reading scale buffer b are done
+    uint64_t* epi_turn = sf_free + SF_NBUF;  // [EPI_WARPS] whose turn it is to use the store buffer
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(epi_turn + EPI_WARPS);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
@@ -162,9 +163,9 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
             mbar_init(&empty[s], 1);
         }
         mbar_init(tmem_full, 1);
-        mbar_init(tmem_empty, 32 * EPI_WARPS);
+        mbar_init(tmem_empty, EPI_WARPS);               // one arrival per epilogue warp
         mbar_init(mma_done, 1);
-        for (int b = 0; b < 2; ++b) { mbar_init(&sf_ready[b], 32 * SF_WARPS); mbar_init(&sf_free[b], 1); }
+        for (int b = 0; b < SF_NBUF; ++b) { mbar_init(&sf_ready[b], SF_WARPS); mbar_init(&sf_free[b], 1); }
         for (int w = 0; w < EPI_WARPS; ++w) mbar_init(&epi_turn[w], 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -240,7 +241,7 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
                 tc_fence_after();
                 for (int kb = 0; kb < nkb; ++kb) {
                     if (!mbar_wait(&full[stage], phase)) { *abort_flag = 1; break; }
-                    if (!mbar_wait(&sf_ready[kpar], (kcount >> 1) & 1)) { *abort_flag = 1; break; }
+                    if (!mbar_wait(&sf_ready[kpar], (kcount / SF_NBUF) & 1)) { *abort_flag = 1; break; }
                     tc_fence_after();
                     const int64_t krem = p.K - (int64_t)kb * KB_ELEMS;
                     const int nmma = krem < KB_ELEMS ? (int)(krem / 64) : 4;
@@ -275,8 +276,8 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
                     }
                     tc_commit(&empty[stage]);
                     tc_commit(&sf_free[kpar]);
-                    kpar ^= 1u;
                     ++kcount;
+                    kpar = kcount % SF_NBUF;
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
                 if (*abort_flag) break;
@@ -296,7 +297,7 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
             for (int kb = 0; kb < nkb; ++kb) {
                 if (!mbar_wait(&full[stage], phase)) { *abort_flag = 1; break; }
                 // the MMAs that read this buffer two k-blocks ago are done
-                if (!mbar_wait(&sf_free[kpar], ((kcount >> 1) & 1) ^ 1)) { *abort_flag = 1; break; }
+                if (!mbar_wait(&sf_free[kpar], ((kcount / SF_NBUF) & 1) ^ 1)) { *abort_flag = 1; break; }
                 tc_fence_after();
                 const int64_t krem = p.K - (int64_t)kb * KB_ELEMS;
                 const int nmma = krem < KB_ELEMS ? (int)(krem / 64) : 4;
@@ -305,9 +306,10 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
                              smem + OFF_SFB + stage * SFB_STAGE, na, lane);
                 tmem_st_wait();
                 tc_fence_before();
-                mbar_arrive(&sf_ready[kpar]);
-                kpar ^= 1u;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sf_ready[kpar]);
                 ++kcount;
+                kpar = kcount % SF_NBUF;
                 if (++stage == STAGES) { stage = 0; phase ^= 1; }
             }
         }
@@ -336,7 +338,8 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
                 if (round == 3) {
                     // the whole accumulator slice is in registers: let the next tile's MMAs start
                     tc_fence_before();
-                    mbar_arrive(tmem_empty);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(tmem_empty);
                 }
                 if (out_bf16) {
 #pragma unroll
@@ -413,16 +416,33 @@ static bool make_code_map(CUtensorMap* map, const void* base, int64_t rows, int6
     return r == CUDA_SUCCESS;
 }
 
+// Output Y [M, N] bf16 for TMA stores of 32-row x 64-column boxes, 128-byte swizzle.
+static bool make_out_map(CUtensorMap* map, void* y, int64_t M, int64_t N) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
+    cuuint64_t strides[1] = {(cuuint64_t)(N * 2)};
+    cuuint32_t box[2] = {64u, 32u};
+    cuuint32_t es[2] = {1u, 1u};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, y, dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+
 // ------------------------------------------------------------------ CTA-pair GEMM
 // The same GEMM on CTA pairs (clusters of two CTAs on two SMs) with the
 // 2-SM MMA: a pair owns a 256 x 256 output tile, each CTA stages its own 128
-// rows of A, its own 128 rows of the 256-row B tile and the B scales of both
-// halves; the leader CTA issues one 256 x 256 x 64 MMA per K step for both
-// SMs, so per unit of work the issue, scale-copy and barrier overheads and
-// the per-SM shared-memory traffic for B are halved.  Both CTAs' TMA loads
-// complete on the leader's `full` barriers; the leader's commits are
-// multicast to both CTAs' `empty` and `tmem_full` barriers; both CTAs'
-// epilogue warps release the accumulators on the leader's `tmem_empty`.
+// rows of A and its own 128 rows of the 256-row B tile; the leader CTA issues
+// one 256 x 256 x 64 MMA per K step for both SMs, which halves the per-SM
+// shared-memory and L2 traffic for B.  Both CTAs' A/B TMA loads complete on
+// the leader's `full` barriers; each CTA's scale warps stage its own A scales
+// and the whole B-scale tile into its own TMEM (its scale loads complete on a
+// local barrier) and release them to the leader's `sf_ready`; the leader's
+// commits are multicast to both CTAs' `empty`, `sf_free` and `tmem_full`;
+// both CTAs' epilogue warps release the accumulators on the leader's
+// `tmem_empty` and store their own 128 rows.
 namespace pair {
 constexpr int BM = 128;                  // rows of A per CTA (pair tile 256)
 constexpr int BN = 256;                  // columns per pair tile (128 rows of B per CTA)
@@ -436,35 +456,41 @@ constexpr int SFB_STAGE = 4096;                 // band 0 at +0, band 1 at +2048
 constexpr int OFF_B = STAGES * A_STAGE;
 constexpr int OFF_SFA = OFF_B + STAGES * B_STAGE;
 constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_STAGE;
-constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_STAGE;
+constexpr int OFF_EPI = OFF_SFB + STAGES * SFB_STAGE;
+constexpr int EPI_BYTES = 8192;
+constexpr int OFF_BAR = OFF_EPI + EPI_BYTES;
 constexpr int BAR_BYTES = 512;
 constexpr int SMEM_BYTES = OFF_BAR + BAR_BYTES + 1024;
+constexpr int SF_WARPS = 4;
 constexpr int EPI_WARPS = 8;
-constexpr int FIRST_EPI_WARP = 3;
+constexpr int FIRST_EPI_WARP = 2 + SF_WARPS;
 constexpr int THREADS = 32 * FIRST_EPI_WARP + 32 * EPI_WARPS;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;
 constexpr uint32_t SF_COL = 256;
 constexpr uint32_t SF_BUF = 48;
 constexpr uint32_t SFB_OFF = 16;
+constexpr int SF_NBUF = 4;               // scale buffers in TMEM (the hand-off crosses CTAs)
 }  // namespace pair
 
 template <bool MX>
 __global__ void __launch_bounds__(pair::THREADS, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB, GemmDev p) {
+                     const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
+                     const __grid_constant__ CUtensorMap tmY, GemmDev p) {
     using namespace pair;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
-    uint64_t* empty = full + STAGES;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);   // [S] A/B of both CTAs (leader's)
+    uint64_t* sf_full = full + STAGES;                              // [S] this CTA's scale loads
+    uint64_t* empty = sf_full + STAGES;                             // [S]
     uint64_t* tmem_full = empty + STAGES;
-    uint64_t* tmem_empty = tmem_full + 1;
+    uint64_t* tmem_empty = tmem_full + 1;                           // leader's: both CTAs' epilogues
     uint64_t* mma_done = tmem_empty + 1;
-    uint64_t* sfb_full = mma_done + 1;
-    uint64_t* sfb_empty = sfb_full + 2;
-    uint64_t* sf_done = sfb_empty + 2;
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sf_done + 1);
+    uint64_t* sf_ready = mma_done + 1;                              // [SF_NBUF] leader's: both CTAs' scale warps
+    uint64_t* sf_free = sf_ready + SF_NBUF;                         // [SF_NBUF]
+    uint64_t* epi_turn = sf_free + SF_NBUF;                         // [EPI_WARPS]
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(epi_turn + EPI_WARPS);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5;
@@ -475,13 +501,14 @@ __global__ void __launch_bounds__(pair::THREADS, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
+            mbar_init(&sf_full[s], 1);
             mbar_init(&empty[s], 1);
         }
         mbar_init(tmem_full, 1);
-        mbar_init(tmem_empty, 2 * 32 * EPI_WARPS);
+        mbar_init(tmem_empty, 2 * EPI_WARPS);           // one arrival per epilogue warp of either CTA
         mbar_init(mma_done, 1);
-        for (int b = 0; b < 2; ++b) { mbar_init(&sfb_full[b], 1); mbar_init(&sfb_empty[b], 1); }
-        mbar_init(sf_done, 1);
+        for (int b = 0; b < SF_NBUF; ++b) { mbar_init(&sf_ready[b], 2 * SF_WARPS); mbar_init(&sf_free[b], 1); }
+        for (int w = 0; w < EPI_WARPS; ++w) mbar_init(&epi_turn[w], 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -492,6 +519,7 @@ __global__ void __launch_bounds__(pair::THREADS, 1)
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmA); tma_prefetch_desc(&tmB);
         tma_prefetch_desc(&tmSA); tma_prefetch_desc(&tmSB);
+        if (p.out_bf16) tma_prefetch_desc(&tmY);
     }
     tc_fence_before();
     __syncthreads();
@@ -507,7 +535,7 @@ __global__ void __launch_bounds__(pair::THREADS, 1)
     const int mma_per_atom = MX ? 2 : 1;
     const int atoms_per_kb = 4 / mma_per_atom;
     const uint32_t sf_bytes = 512u * (uint32_t)atoms_per_kb;       // one band's scales per k-block
-    const uint32_t cta_bytes = A_STAGE + B_STAGE + 3u * sf_bytes;  // one CTA's loads per k-block
+    const uint32_t ab_bytes = A_STAGE + B_STAGE;                    // one CTA's A/B loads per k-block
 
     if (warp == 0) {
         if (lane == 0) {
@@ -521,27 +549,30 @@ __global__ void __launch_bounds__(pair::THREADS, 1)
                 const int64_t mt = t % tiles_m, nt = t / tiles_m;
                 for (int kb = 0; kb < nkb; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1)) { *abort_flag = 1; break; }
-                    if (leader) mbar_arrive_expect_tx(&full[stage], 2u * cta_bytes);
+                    if (leader) mbar_arrive_expect_tx(&full[stage], 2u * ab_bytes);
+                    mbar_arrive_expect_tx(&sf_full[stage], 3u * sf_bytes);
                     const uint32_t fb = leader_full + 8u * (uint32_t)stage;
                     const int32_t krow = (int32_t)(2 * kb * atoms_per_kb);
                     tma_load_2d_pair(smem + stage * A_STAGE, &tmA, fb, kb * KB_BYTES, (int32_t)(mt * 2 * BM + rank * BM));
                     tma_load_2d_pair(smem + OFF_B + stage * B_STAGE, &tmB, fb, kb * KB_BYTES,
                                      (int32_t)(nt * BN + rank * (BN / 2)));
-                    tma_load_2d_pair(smem + OFF_SFA + stage * SFA_STAGE, &tmSA, fb, 0,
-                                     (int32_t)(2 * (mt * 2 + rank) * p.catoms) + krow);
-                    tma_load_2d_pair(smem + OFF_SFB + stage * SFB_STAGE, &tmSB, fb, 0,
-                                     (int32_t)(2 * (nt * 2) * p.catoms) + krow);
-                    tma_load_2d_pair(smem + OFF_SFB + stage * SFB_STAGE + 2048, &tmSB, fb, 0,
-                                     (int32_t)(2 * (nt * 2 + 1) * p.catoms) + krow);
+                    tma_load_2d(smem + OFF_SFA + stage * SFA_STAGE, &tmSA, &sf_full[stage], 0,
+                                (int32_t)(2 * (mt * 2 + rank) * p.catoms) + krow);
+                    tma_load_2d(smem + OFF_SFB + stage * SFB_STAGE, &tmSB, &sf_full[stage], 0,
+                                (int32_t)(2 * (nt * 2) * p.catoms) + krow);
+                    tma_load_2d(smem + OFF_SFB + stage * SFB_STAGE + 2048, &tmSB, &sf_full[stage], 0,
+                                (int32_t)(2 * (nt * 2 + 1) * p.catoms) + krow);
                     issued[stage] = true;
                     last_phase[stage] = phase;
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
             }
-            // the leader's barriers count both CTAs' copies: wait for the last ones
-            if (leader)
-                for (int s = 0; s < STAGES; ++s)
-                    if (issued[s]) mbar_wait(&full[s], last_phase[s]);
+            // never leave a copy in flight into shared memory we are about to release
+            for (int s = 0; s < STAGES; ++s)
+                if (issued[s]) {
+                    mbar_wait(&sf_full[s], last_phase[s]);
+                    if (leader) mbar_wait(&full[s], last_phase[s]);
+                }
         }
     } else if (warp == 1) {
         if (lane == 0 && leader) {
@@ -549,7 +580,6 @@ __global__ void __launch_bounds__(pair::THREADS, 1)
             const uint32_t idesc_hi = idesc_with_sf_id(idesc0, 2, 2);
             const uint64_t adesc0 = smem_desc(smem_u32(smem), 16, 1024, 2);
             const uint64_t bdesc0 = smem_desc(smem_u32(smem + OFF_B), 16, 1024, 2);
-            const uint64_t sfa0 = smem_desc(smem_u32(smem + OFF_SFA), 0, 128, 0);
             int stage = 0;
             uint32_t phase = 0, acc_phase = 0, kpar = 0, kcount = 0;
             for (int64_t t = pair_id; t < tiles && !*abort_flag; t += npairs) {
@@ -557,19 +587,17 @@ __global__ void __launch_bounds__(pair::THREADS, 1)
                 tc_fence_after();
                 for (int kb = 0; kb < nkb; ++kb) {
                     if (!mbar_wait(&full[stage], phase)) { *abort_flag = 1; break; }
-                    if (!mbar_wait(&sfb_full[kpar], (kcount >> 1) & 1)) { *abort_flag = 1; break; }
+                    if (!mbar_wait(&sf_ready[kpar], (kcount / SF_NBUF) & 1)) { *abort_flag = 1; break; }
                     tc_fence_after();
                     const int64_t krem = p.K - (int64_t)kb * KB_ELEMS;
                     const int nmma = krem < KB_ELEMS ? (int)(krem / 64) : 4;
                     const uint64_t ad = adesc0 + (uint64_t)(stage * (A_STAGE >> 4));
                     const uint64_t bd = bdesc0 + (uint64_t)(stage * (B_STAGE >> 4));
-                    const uint64_t fa = sfa0 + (uint64_t)(stage * (SFA_STAGE >> 4));
                     const uint32_t sfa = tmem + SF_COL + kpar * SF_BUF;
                     const uint32_t sfb = sfa + SFB_OFF;
                     uint32_t accf = kb > 0 ? 1u : 0u;
                     for (int kk = 0; kk < nmma; ++kk) {
                         const int atom = MX ? kk / 2 : kk;
-                        if (!MX || (kk & 1) == 0) tmem_cp_sf_pair(sfa + atom * 4, fa + atom * 32);
                         if (MX)
                             mma_mxf4_pair(tmem + ACC_COL, ad + 2 * kk, bd + 2 * kk, (kk & 1) ? idesc_hi : idesc0,
                                           sfa + atom * 4, sfb + atom * 8, accf);
@@ -579,9 +607,9 @@ __global__ void __launch_bounds__(pair::THREADS, 1)
                         accf = 1u;
                     }
                     tc_commit_pair_mc(&empty[stage], 0x3);
-                    tc_commit_pair(&sfb_empty[kpar]);
-                    kpar ^= 1u;
+                    tc_commit_pair_mc(&sf_free[kpar], 0x3);
                     ++kcount;
+                    kpar = kcount % SF_NBUF;
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
                 if (*abort_flag) break;
@@ -591,62 +619,92 @@ __global__ void __launch_bounds__(pair::THREADS, 1)
             tc_commit_pair(mma_done);
             mbar_wait(mma_done, 0);
         }
-    } else if (warp == 2) {
-        if (lane == 0 && leader) {
-            const uint64_t sfb0 = smem_desc(smem_u32(smem + OFF_SFB), 0, 128, 0);
-            int stage = 0;
-            uint32_t phase = 0, kpar = 0, kcount = 0;
-            for (int64_t t = pair_id; t < tiles && !*abort_flag; t += npairs) {
-                for (int kb = 0; kb < nkb; ++kb) {
-                    if (!mbar_wait(&full[stage], phase)) { *abort_flag = 1; break; }
-                    if (!mbar_wait(&sfb_empty[kpar], ((kcount >> 1) & 1) ^ 1)) { *abort_flag = 1; break; }
-                    tc_fence_after();
-                    const int64_t krem = p.K - (int64_t)kb * KB_ELEMS;
-                    const int nmma = krem < KB_ELEMS ? (int)(krem / 64) : 4;
-                    const int na = (nmma + mma_per_atom - 1) / mma_per_atom;
-                    const uint64_t fb = sfb0 + (uint64_t)(stage * (SFB_STAGE >> 4));
-                    const uint32_t sfb = tmem + SF_COL + kpar * SF_BUF + SFB_OFF;
-                    for (int a = 0; a < na; ++a) {
-                        tmem_cp_sf_pair(sfb + a * 8, fb + a * 32);
-                        tmem_cp_sf_pair(sfb + a * 8 + 4, fb + 128 + a * 32);
-                    }
-                    tc_commit_pair(&sfb_full[kpar]);
-                    kpar ^= 1u;
-                    ++kcount;
-                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
-                }
+    } else if (warp < FIRST_EPI_WARP) {
+        const uint32_t quarter = (uint32_t)(warp & 3) * 32u;
+        const uint32_t leader_sf_ready = mapa_shared(smem_u32(sf_ready), 0);
+        int stage = 0;
+        uint32_t phase = 0, kpar = 0, kcount = 0;
+        for (int64_t t = pair_id; t < tiles && !*abort_flag; t += npairs) {
+            for (int kb = 0; kb < nkb; ++kb) {
+                if (!mbar_wait(&sf_full[stage], phase)) { *abort_flag = 1; break; }
+                if (!mbar_wait(&sf_free[kpar], ((kcount / SF_NBUF) & 1) ^ 1)) { *abort_flag = 1; break; }
+                tc_fence_after();
+                const int64_t krem = p.K - (int64_t)kb * KB_ELEMS;
+                const int nmma = krem < KB_ELEMS ? (int)(krem / 64) : 4;
+                const int na = (nmma + mma_per_atom - 1) / mma_per_atom;
+                stage_scales(tmem + (quarter << 16) + SF_COL + kpar * SF_BUF, smem + OFF_SFA + stage * SFA_STAGE,
+                             smem + OFF_SFB + stage * SFB_STAGE, na, lane);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(leader_sf_ready + 8u * kpar);
+                ++kcount;
+                kpar = kcount % SF_NBUF;
+                if (++stage == STAGES) { stage = 0; phase ^= 1; }
             }
-            tc_commit_pair(sf_done);
-            mbar_wait(sf_done, 0);
         }
     } else {
         const int quad = warp & 3;
         const int half = (warp - FIRST_EPI_WARP) >> 2;
-        const int row_in_tile = quad * 32 + lane;
+        const int order = warp - FIRST_EPI_WARP;
         const float alpha = MX ? 1.0f : __fmul_rn(*p.a_gscale, *p.b_gscale);
         const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + ACC_COL + half * 128;
         const uint32_t leader_tmem_empty = mapa_shared(smem_u32(tmem_empty), 0);
-        uint32_t acc_phase = 0;
-        for (int64_t t = pair_id; t < tiles; t += npairs) {
+        const bool out_bf16 = p.out_bf16 != 0;
+        uint8_t* buf = smem + OFF_EPI;
+        uint32_t acc_phase = 0, iter = 0;
+        for (int64_t t = pair_id; t < tiles; t += npairs, ++iter) {
             if (!mbar_wait(tmem_full, acc_phase)) { *abort_flag = 1; break; }
             tc_fence_after();
-            uint32_t r[4][32];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32(taddr + c * 32, r[c]);
-            tmem_ld_wait();
-            tc_fence_before();
-            mbar_arrive_cluster(leader_tmem_empty);
-            acc_phase ^= 1;
             const int64_t mt = t % tiles_m, nt = t / tiles_m;
-            const int64_t row = mt * 2 * BM + (int64_t)rank * BM + row_in_tile;
-            if (row < p.M) {
+            const int64_t row0 = mt * 2 * BM + (int64_t)rank * BM + quad * 32;
+            const int64_t row = row0 + lane;
+            const int64_t col_base = nt * BN + half * 128;
+            uint32_t pk[2][32];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const int64_t col0 = nt * BN + half * 128 + c * 32;
-                    if (col0 < p.N) store_row32(p.y, p.N, row, col0, r[c], alpha, p.out_bf16 != 0);
+            for (int round = 0; round < 4; ++round) {
+                uint32_t r[32];
+                tmem_ld32(taddr + round * 32, r);
+                tmem_ld_wait();
+                if (round == 3) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_cluster(leader_tmem_empty);
+                }
+                if (out_bf16) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[2 * j]) * alpha,
+                                                                 __uint_as_float(r[2 * j + 1]) * alpha);
+                        pk[round >> 1][(round & 1) * 16 + j] = *reinterpret_cast<uint32_t*>(&h);
+                    }
+                } else if (row < p.M) {
+                    store_row32(p.y, p.N, row, col_base + round * 32, r, alpha, false);
                 }
             }
+            if (out_bf16) {
+                const bool first = order == 0;
+                if (!mbar_wait(&epi_turn[order], first ? ((iter & 1) ^ 1) : (iter & 1))) { *abort_flag = 1; break; }
+#pragma unroll
+                for (int b = 0; b < 2; ++b)
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        *reinterpret_cast<uint4*>(buf + b * 4096 + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                            make_uint4(pk[b][4 * c], pk[b][4 * c + 1], pk[b][4 * c + 2], pk[b][4 * c + 3]);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&tmY, buf, (int32_t)col_base, (int32_t)row0);
+                    tma_store_2d(&tmY, buf + 4096, (int32_t)(col_base + 64), (int32_t)row0);
+                    bulk_commit_group();
+                    bulk_wait_read_all();
+                    mbar_arrive(&epi_turn[(order + 1) % EPI_WARPS]);
+                }
+                __syncwarp();
+            }
+            acc_phase ^= 1;
         }
+        if (lane == 0) bulk_wait_all();
     }
 
     tc_fence_before();
@@ -679,7 +737,7 @@ constexpr bool kUsePairKernel = false;
 
 static cudaError_t launch_gemm_pair(const GemmParams& p, const GemmDev& d, cudaStream_t st, int num_sms) {
     using namespace pair;
-    CUtensorMap ma, mb, msa, msb;
+    CUtensorMap ma, mb, msa, msb, my;
     const int blk = p.mxfp4 ? 32 : 16;
     const int box_rows = 2 * (p.mxfp4 ? 2 : 4);
     const int64_t sa_bytes = ((p.M + 127) / 128) * 128 * d.catoms * 4;
@@ -689,6 +747,8 @@ static cudaError_t launch_gemm_pair(const GemmParams& p, const GemmDev& d, cudaS
     if (!make_code_map(&mb, p.b_codes, p.N, p.K / 2, BN / 2)) return cudaErrorInvalidValue;
     if (!make_scale_map(&msa, p.a_scales, sa_bytes, box_rows)) return cudaErrorInvalidValue;
     if (!make_scale_map(&msb, p.b_scales, sb_bytes, box_rows)) return cudaErrorInvalidValue;
+    std::memset(&my, 0, sizeof(my));
+    if (p.out_bf16 && !make_out_map(&my, p.y, p.M, p.N)) return cudaErrorInvalidValue;
     const int64_t tiles = ((p.M + 2 * BM - 1) / (2 * BM)) * ((p.N + BN - 1) / BN);
     int pairs = num_sms / 2;
     if (tiles < pairs) pairs = (int)tiles;
@@ -708,28 +768,14 @@ static cudaError_t launch_gemm_pair(const GemmParams& p, const GemmDev& d, cudaS
     if (p.mxfp4) {
         e = cudaFuncSetAttribute(gemm_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
         if (e != cudaSuccess) return e;
-        e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel<true>, ma, mb, msa, msb, d);
+        e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel<true>, ma, mb, msa, msb, my, d);
     } else {
         e = cudaFuncSetAttribute(gemm_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
         if (e != cudaSuccess) return e;
-        e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel<false>, ma, mb, msa, msb, d);
+        e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel<false>, ma, mb, msa, msb, my, d);
     }
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
-}
-
-// Output Y [M, N] bf16 for TMA stores of 32-row x 64-column boxes, 128-byte swizzle.
-static bool make_out_map(CUtensorMap* map, void* y, int64_t M, int64_t N) {
-    auto enc = tensor_map_encoder();
-    if (!enc) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
-    cuuint64_t strides[1] = {(cuuint64_t)(N * 2)};
-    cuuint32_t box[2] = {64u, 32u};
-    cuuint32_t es[2] = {1u, 1u};
-    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, y, dims, strides, box, es,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
 }
 
 cudaError_t launch_gemm(const GemmParams& p, cudaStream_t st, int num_sms) {
