@@ -119,6 +119,60 @@ __device__ __forceinline__ NvScale nv_scale_from_byte(uint32_t byte, float s_t) 
     return r;
 }
 
+// E4M3 byte (round to nearest even, saturating) of the binary32 quotient
+// RN(amax / denom), for amax >= 0 and denom > 0, given rden = RN(1 / denom)
+// normal and finite.  q0 = RN(amax * rden) carries two roundings of relative
+// size <= 2^-24 each, so RN(amax / denom) lies within two units in the last
+// place of q0 (four bit-pattern steps below a power of two).  E4M3 rounding
+// is monotone, so when the bytes of q0 -/+ four steps agree that byte is the
+// answer; otherwise (next to an E4M3 rounding boundary) the quotient is
+// formed by the correctly rounded division.
+__device__ __forceinline__ uint32_t e4m3_rn_of_quotient(float amax, float denom, float rden) {
+    const uint32_t b = __float_as_uint(__fmul_rn(amax, rden));
+    const float lo = __uint_as_float(b >= 4u ? b - 4u : 0u);
+    const float hi = __uint_as_float(b + 4u);
+    uint16_t pr;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(pr) : "f"(fminf(hi, 448.0f)), "f"(fminf(lo, 448.0f)));
+    if ((pr & 0xFFu) == (uint32_t)(pr >> 8)) return pr & 0xFFu;
+    return e4m3_rn(__fdiv_rn(amax, denom));
+}
+
+// ---- pairs of binary32 values on the f32x2 ALU: each lane is rounded to
+// nearest exactly as the scalar __fmul_rn / __fadd_rn / __fsub_rn.
+__device__ __forceinline__ float2 mul2_rn(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "mul.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 add2_rn(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "add.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 sub2_rn(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "sub.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
+// Values of the two E2M1 codes in one byte (element 0 = low nibble -> .x),
+// through the hardware E2M1 -> f16 conversion (every E2M1 value is exact in
+// f16 and in binary32).
+__device__ __forceinline__ float2 e2m1x2_value(uint32_t byte) {
+    uint32_t h;
+    asm("{\n\t.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}" : "=r"(h) : "r"(byte));
+    float lo, hi;
+    asm("{\n\t.reg .b16 l, u;\n\tmov.b32 {l, u}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, u;\n\t}"
+        : "=f"(lo), "=f"(hi) : "r"(h));
+    return make_float2(lo, hi);
+}
+
 // Offset of scale (r, c) in the tensor-core scale layout (see q4.h).
 __host__ __device__ __forceinline__ int64_t tc_scale_offset(int64_t r, int64_t c, int64_t catoms) {
     return ((r >> 7) * catoms + (c >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (c & 3);

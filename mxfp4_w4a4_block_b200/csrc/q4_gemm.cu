@@ -401,6 +401,19 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
+bool encode_map_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+                   uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
+    cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t es[2] = {1u, 1u};
+    CUresult r = enc(map, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // 2-D byte tensor [rows, row_bytes] with a box of 128 bytes x box_rows and
 // 128-byte swizzle (the operand layout the MMA descriptors describe).
 static bool make_code_map(CUtensorMap* map, const void* base, int64_t rows, int64_t row_bytes, int box_rows) {
@@ -1076,10 +1089,11 @@ cudaError_t launch_fused_decode(const FusedDecodeParams& p, cudaStream_t st, int
 }
 
 cudaError_t read_clear_device_error(unsigned int* word) {
-    cudaError_t e = cudaMemcpyFromSymbol(word, g_device_error, sizeof(unsigned int));
-    if (e != cudaSuccess || *word == 0) return e;
-    const unsigned int zero = 0;
-    return cudaMemcpyToSymbol(g_device_error, &zero, sizeof(unsigned int));
+    unsigned int a = 0, b = 0;
+    cudaError_t e = read_clear_module_error(&a);
+    if (e == cudaSuccess) e = read_clear_quant_error(&b);
+    *word = a | b;
+    return e;
 }
 
 }  // namespace q4

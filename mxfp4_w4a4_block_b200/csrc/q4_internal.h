@@ -2,6 +2,7 @@
 // kernel files and the C-ABI layer.  Not part of the public interface.
 #pragma once
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 namespace q4 {
@@ -70,8 +71,16 @@ cudaError_t launch_dequantize(const DequantParams& p, int blk, bool tc, bool out
 cudaError_t launch_gemm(const GemmParams& p, cudaStream_t st, int num_sms);
 cudaError_t launch_fused_decode(const FusedDecodeParams& p, cudaStream_t st, int num_sms);
 
-// Reads and clears the device error word (bit 0: a bounded wait ran out).
+// Reads and clears the device error words of all kernel files (bit 0: a
+// bounded wait ran out); read_clear_quant_error covers the quantize file only.
 cudaError_t read_clear_device_error(unsigned int* word);
+cudaError_t read_clear_quant_error(unsigned int* word);
+
+// 2-D tiled tensor map over a row-major [outer, inner] array of `dt`
+// elements with rows `row_bytes` apart; out-of-range box parts read as zero
+// and are not written by stores.  False if the encoder rejects it.
+bool encode_map_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+                   uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle);
 
 // Whether the fused-activation small-M GEMM takes this shape (M <= 128 and
 // the quantized activations fit in shared memory next to >= 2 weight stages).

@@ -5,14 +5,23 @@
 #pragma once
 #include <cstdint>
 #include <cuda.h>
+#include <cuda_runtime.h>
 
 namespace q4 {
 
-// Device error word (defined by the one translation unit that includes this
-// header): bit 0 = a bounded wait ran out.  Read and cleared by
-// q4_get_device_error().
-__device__ unsigned int g_device_error = 0;
+// Device error word: bit 0 = a bounded wait ran out.  Every kernel file that
+// includes this header has its own copy (the files are separate device
+// modules); q4_get_device_error() reads and clears all of them.
+static __device__ unsigned int g_device_error = 0;
 constexpr unsigned kErrTimeout = 1u;
+
+// Reads this file's error word into *word and clears it.
+static inline cudaError_t read_clear_module_error(unsigned int* word) {
+    cudaError_t e = cudaMemcpyFromSymbol(word, g_device_error, sizeof(unsigned int));
+    if (e != cudaSuccess || *word == 0) return e;
+    const unsigned int zero = 0;
+    return cudaMemcpyToSymbol(g_device_error, &zero, sizeof(unsigned int));
+}
 
 // A bounded wait gives up after about this many SM clock cycles (~1 s at the
 // B200's clocks), records kErrTimeout and lets the kernel wind down.
@@ -127,6 +136,21 @@ __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bul
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 // Wait until every committed bulk store of this thread has completed.
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Contiguous bulk copy shared -> global (size and both addresses 16-byte
+// aligned), tracked by the issuing thread's bulk async-group.
+__device__ __forceinline__ void bulk_store(void* dst, const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+                 ::"l"(dst), "r"(smem_u32(src)), "r"(bytes) : "memory");
+}
+// Wait until all but the most recent committed bulk group of this thread have
+// finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+
+// Barrier over the first `nthreads` threads that use barrier `id` (1..15).
+__device__ __forceinline__ void named_barrier(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
 
 // Contiguous bulk copy global -> shared (size and both addresses 16-byte aligned).
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {

@@ -3,15 +3,17 @@
 // Hadamard-32 of MACaQ fused in), dequantization and the first-order
 // Sigma-Delta step of "Looped Transformer quantization", sec. 2.1.
 //
-// The quantizer gives each thread whole blocks (the scale rule, the Hadamard
-// rotation and the code packing stay in registers) and each CTA one scale
-// atom's worth of blocks, so the scales leave as 512 contiguous bytes.  The
-// Sigma-Delta step only reads scales and is a plain elementwise stream.
+// The quantizer and the Sigma-Delta step are persistent producer/consumer
+// kernels: one thread streams tiles into shared memory by TMA, sixteen warps
+// compute, and the results leave by TMA stores (see each kernel).  amax and
+// dequantize are plain grid-stride streams.
 #include <cstdint>
+#include <cstring>
 #include <cuda_runtime.h>
 
 #include "q4_codec.cuh"
 #include "q4_internal.h"
+#include "q4_ptx.cuh"
 
 namespace q4 {
 
@@ -24,8 +26,21 @@ __global__ void __launch_bounds__(256) amax_kernel(const void* __restrict__ x, i
     if (bf16) {
         const uint4* v = reinterpret_cast<const uint4*>(x);
         const int64_t nv = n / 8;
-        for (int64_t i = tid; i < nv; i += nthreads) {
-            uint4 w = __ldcs(v + i);
+        int64_t i = tid;
+        // four independent 16-byte loads in flight per thread
+        for (; i + 3 * nthreads < nv; i += 4 * nthreads) {
+            uint4 w[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) w[u] = __ldg(v + i + u * nthreads);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const uint32_t ws[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) m = fmaxf(m, fmaxf(fabsf(bf16_lo(ws[j])), fabsf(bf16_hi(ws[j]))));
+            }
+        }
+        for (; i < nv; i += nthreads) {
+            uint4 w = __ldg(v + i);
             uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
             for (int j = 0; j < 4; ++j) m = fmaxf(m, fmaxf(fabsf(bf16_lo(ws[j])), fabsf(bf16_hi(ws[j]))));
@@ -36,8 +51,17 @@ __global__ void __launch_bounds__(256) amax_kernel(const void* __restrict__ x, i
     } else {
         const float4* v = reinterpret_cast<const float4*>(x);
         const int64_t nv = n / 4;
-        for (int64_t i = tid; i < nv; i += nthreads) {
-            float4 w = __ldcs(v + i);
+        int64_t i = tid;
+        for (; i + 3 * nthreads < nv; i += 4 * nthreads) {
+            float4 w[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) w[u] = __ldg(v + i + u * nthreads);
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                m = fmaxf(m, fmaxf(fmaxf(fabsf(w[u].x), fabsf(w[u].y)), fmaxf(fabsf(w[u].z), fabsf(w[u].w))));
+        }
+        for (; i < nv; i += nthreads) {
+            float4 w = __ldg(v + i);
             m = fmaxf(m, fmaxf(fmaxf(fabsf(w.x), fabsf(w.y)), fmaxf(fabsf(w.z), fabsf(w.w))));
         }
         const float* s = reinterpret_cast<const float*>(x);
@@ -76,200 +100,490 @@ cudaError_t launch_amax(const void* x, int64_t n, bool bf16, float denom, float*
 }
 
 // ------------------------------------------------------------------ helpers
-// Load one 16-byte chunk: 8 bf16 or 4 fp32 values (two chunks make 8 fp32).
-__device__ __forceinline__ void load_bf16x8(const void* src, float* v) {
-    const uint4 raw = __ldg(reinterpret_cast<const uint4*>(src));
-    v[0] = bf16_lo(raw.x); v[1] = bf16_hi(raw.x); v[2] = bf16_lo(raw.y); v[3] = bf16_hi(raw.y);
-    v[4] = bf16_lo(raw.z); v[5] = bf16_hi(raw.z); v[6] = bf16_lo(raw.w); v[7] = bf16_hi(raw.w);
-}
-__device__ __forceinline__ void load_f32x4(const void* src, float* v) {
-    const float4 f = __ldg(reinterpret_cast<const float4*>(src));
-    v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+// ------------------------------------------------------------------ quantize
+// Persistent, one CTA per SM.  A tile is ROWS rows x one scale-atom column
+// (4 blocks along the row), so the tile's scales are whole 512-byte atoms of
+// the tensor-core layout.  One producer thread streams tiles into a ring of
+// shared-memory stages with TMA (128-byte-wide boxes, 128-byte swizzle, zero
+// fill outside the tensor); 16 consumer warps give each thread whole blocks
+// (the scale rule, the Hadamard rotation and the code packing stay in
+// registers), a warp taking 32 consecutive rows of one block column so its
+// swizzled shared-memory reads are conflict-free.  Codes and scale atoms are
+// staged in shared memory and leave by TMA / bulk stores (three staging
+// buffers, so the stores overlap the next tiles).
+namespace qz {
+constexpr int CONSUMER_WARPS = 16;
+constexpr int CONSUMERS = 32 * CONSUMER_WARPS;
+constexpr int THREADS = CONSUMERS + 32;          // + the producer warp
+constexpr int IN_BYTES = 160 * 1024;             // input stages
+constexpr int NBUF = 3;                          // output staging buffers
+}  // namespace qz
+
+template <int BLK, bool BF16>
+struct QzGeom {
+    static constexpr int ESZ = BF16 ? 2 : 4;
+    static constexpr int ACOL = 4 * BLK * ESZ;                 // input bytes of one atom column per row
+    static constexpr int NBOX = ACOL / 128;                    // 128-byte TMA boxes per row
+    static constexpr int ROWS = (32768 / ACOL) < 128 ? 128 : 32768 / ACOL;
+    static constexpr int STAGE = ROWS * ACOL;
+    static constexpr int NSTAGE = qz::IN_BYTES / STAGE;
+    static constexpr int CODE_TILE = ROWS * 2 * BLK;            // codes of a tile, [ROWS][2*BLK] bytes
+    static constexpr int SF_TILE = ROWS * 4;                    // ROWS/128 scale atoms
+    static constexpr int BPT = ROWS * 4 / qz::CONSUMERS;        // blocks per consumer thread
+    static constexpr int CHUNKS = BLK * ESZ / 16;               // 16-byte chunks per block
+    static constexpr int PER = 16 / ESZ;                        // values per chunk
+    static constexpr int TAB_OFF = NSTAGE * STAGE + qz::NBUF * (CODE_TILE + SF_TILE);
+    static constexpr int BAR_OFF = TAB_OFF + 512;               // after the 128-entry reciprocal table
+    static constexpr int SMEM = BAR_OFF + 256 + 1024;           // + barriers, alignment slack
+    static_assert(BPT >= 1 && ROWS % 128 == 0 && ROWS <= 256, "tile geometry");
+};
+
+// NVFP4 per-launch context: the tensor scale, 6 * s_t and its reciprocal,
+// whether the fast RN scale path applies, and the shared-memory table of
+// 1 / (dec(s_b) * s_t) for every E4M3 byte 0..127 (NaN marks a degenerate
+// scale: zero, or a reciprocal that is not finite).
+struct NvCtx {
+    float s_t, denom, rden;
+    bool st_ok, fast;
+    const float* tab;
+};
+
+__device__ __forceinline__ NvCtx nv_ctx(float s_t, const float* tab) {
+    NvCtx c;
+    c.s_t = s_t;
+    c.st_ok = st_valid(s_t);
+    c.denom = __fmul_rn(6.0f, s_t);
+    c.rden = __frcp_rn(c.denom);
+    c.fast = c.st_ok && isfinite(c.rden) && c.rden >= 0x1p-126f && c.denom >= 0x1p-126f;
+    c.tab = tab;
+    return c;
 }
 
-// Sylvester-order Walsh-Hadamard butterflies over 32 values held by one
-// thread (strides 1, 2, 4, 8, 16; (a, b) -> (a + b, a - b)), unnormalised.
-__device__ __forceinline__ void fwht32_reg(float (&v)[32]) {
-#pragma unroll
-    for (int h = 1; h < 32; h <<= 1) {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            if ((i & h) == 0) {
-                const float a = v[i], b = v[i + h];
-                v[i] = __fadd_rn(a, b);
-                v[i + h] = __fsub_rn(a, b);
-            }
-        }
+__device__ __forceinline__ void nv_fill_table(float s_t, float* tab, int tid, int nthreads) {
+    for (int b = tid; b < 128; b += nthreads) {
+        const NvScale r = nv_scale_from_byte((uint32_t)b, s_t);
+        tab[b] = r.degenerate ? __uint_as_float(0x7FC00000u) : r.inv;
     }
 }
 
-// ------------------------------------------------------------------ quantize
-// One thread per block.  A CTA of 256 threads owns a tile of 128 rows x 4
-// blocks -- exactly one 512-byte atom of the tensor-core scale layout -- so
-// each thread quantizes 2 blocks per tile.  Lanes 4k..4k+3 of a warp take the
-// 4 consecutive blocks of one row, so a warp's loads cover 8 whole row
-// segments (128 or 256 bytes each of bf16); the first 16-byte load of a block
-// brings its lines into L1 for the rest.  All loads of a tile are issued
-// before any arithmetic.
-template <int BLK, bool BF16, bool TC, bool RU, bool HAD, bool CHAN>
-__global__ void __launch_bounds__(256) quantize_kernel(QuantParams p) {
-    constexpr int TILE_C = 4 * BLK;          // columns per tile (one scale atom)
-    constexpr int BPT = 2;                   // blocks per thread per tile
-    constexpr int ESZ = BF16 ? 2 : 4;
-    constexpr int LOADS = BLK * ESZ / 16;    // 16-byte loads per block
-    constexpr int PER_LOAD = 16 / ESZ;       // values per load
-    __shared__ __align__(16) uint8_t sf_atom[512];
-
-    const int tid = threadIdx.x;
-    const int64_t tiles_c = (p.cols + TILE_C - 1) / TILE_C;
-    const int64_t tiles = ((p.rows + 127) / 128) * tiles_c;
-    const float s_t = (BLK == 16) ? *p.gscale : 0.0f;
-    const float inv_sqrt32 = 0x1.6a09e6p-3f;   // binary32 nearest to 1/sqrt(32)
-    const char* xb = reinterpret_cast<const char*>(p.x);
-
-    for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
-        const int64_t tr = t / tiles_c, tc = t % tiles_c;
-        const int64_t row0 = tr * 128, col0 = tc * TILE_C;
-
-        float v[BPT][BLK];
-        bool valid[BPT];
+// One NVFP4 block: amax, E4M3 scale byte (RN or RU of amax / (6 s_t)),
+// codes of x * inv (all zero for a degenerate scale).
+template <bool RU>
+__device__ __forceinline__ void nv_block(const float (&v)[16], const NvCtx& c, uint32_t& byte, uint32_t (&w)[2]) {
+    float amax = 0.0f;
 #pragma unroll
-        for (int it = 0; it < BPT; ++it) {
-            const int bt = it * 256 + tid;            // block inside the tile
-            const int64_t row = row0 + (bt >> 2);
-            const int64_t col = col0 + (bt & 3) * BLK;
-            valid[it] = row < p.rows && col < p.cols;
-            if (valid[it]) {
-                const char* src = xb + (row * p.ld + col) * ESZ;
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    if (!c.st_ok) byte = 0;
+    else if (!RU && c.fast) byte = e4m3_rn_of_quotient(amax, c.denom, c.rden);
+    else byte = RU ? e4m3_ru(__fdiv_rn(amax, c.denom)) : e4m3_rn(__fdiv_rn(amax, c.denom));
+    const float inv = c.tab[byte];
+    if (inv != inv) {
+        w[0] = w[1] = 0u;
+        return;
+    }
+    const float2 iv = make_float2(inv, inv);
 #pragma unroll
-                for (int l = 0; l < LOADS; ++l) {
-                    if (BF16) load_bf16x8(src + 16 * l, &v[it][PER_LOAD * l]);
-                    else load_f32x4(src + 16 * l, &v[it][PER_LOAD * l]);
+    for (int g = 0; g < 2; ++g) {
+        float q[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 m = mul2_rn(make_float2(v[8 * g + 2 * i], v[8 * g + 2 * i + 1]), iv);
+            q[2 * i] = m.x;
+            q[2 * i + 1] = m.y;
+        }
+        w[g] = e2m1_pack8(q);
+    }
+}
+
+// One MXFP4 block of 32 with the optional per-column multiplier and block
+// Hadamard-32.  Values are held as pairs P_j = (v_j, v_{j+16}), so the
+// butterflies of strides 1, 2, 4 and 8 (pairs j, j+h with both j, j+h < 16)
+// are packed f32x2 operations; stride 16 pairs the two halves of each P_j.
+template <bool RU, bool HAD>
+__device__ __forceinline__ void mx_block(const float (&v)[32], const float* chan, uint32_t& byte, uint32_t (&w)[4]) {
+    float2 P[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) P[j] = make_float2(v[j], v[j + 16]);
+    if (chan != nullptr) {
+        const float4* cp = reinterpret_cast<const float4*>(chan);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float4 lo = __ldg(cp + q), hi = __ldg(cp + 4 + q);
+            P[4 * q] = mul2_rn(P[4 * q], make_float2(lo.x, hi.x));
+            P[4 * q + 1] = mul2_rn(P[4 * q + 1], make_float2(lo.y, hi.y));
+            P[4 * q + 2] = mul2_rn(P[4 * q + 2], make_float2(lo.z, hi.z));
+            P[4 * q + 3] = mul2_rn(P[4 * q + 3], make_float2(lo.w, hi.w));
+        }
+    }
+    if constexpr (HAD) {
+#pragma unroll
+        for (int h = 1; h < 16; h <<= 1) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                if ((j & h) == 0) {
+                    const float2 a = P[j], b = P[j + h];
+                    P[j] = add2_rn(a, b);
+                    P[j + h] = sub2_rn(a, b);
                 }
-            } else {
-#pragma unroll
-                for (int i = 0; i < BLK; ++i) v[it][i] = 0.0f;
             }
         }
+        const float2 isq = make_float2(0x1.6a09e6p-3f, 0x1.6a09e6p-3f);   // binary32 nearest to 1/sqrt(32)
 #pragma unroll
-        for (int it = 0; it < BPT; ++it) {
-            const int bt = it * 256 + tid;
-            const int rt = bt >> 2, cb = bt & 3;
-            const int64_t row = row0 + rt;
-            const int64_t col = col0 + cb * BLK;
-            if (CHAN && valid[it]) {
-                const float4* cp = reinterpret_cast<const float4*>(p.chan + col);
+        for (int j = 0; j < 16; ++j) {
+            const float a = P[j].x, b = P[j].y;
+            P[j] = mul2_rn(make_float2(__fadd_rn(a, b), __fsub_rn(a, b)), isq);
+        }
+    }
+    float amax = 0.0f;
 #pragma unroll
-                for (int q = 0; q < BLK / 4; ++q) {
-                    const float4 c = __ldg(cp + q);
-                    v[it][4 * q] = __fmul_rn(v[it][4 * q], c.x);
-                    v[it][4 * q + 1] = __fmul_rn(v[it][4 * q + 1], c.y);
-                    v[it][4 * q + 2] = __fmul_rn(v[it][4 * q + 2], c.z);
-                    v[it][4 * q + 3] = __fmul_rn(v[it][4 * q + 3], c.w);
+    for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fmaxf(fabsf(P[j].x), fabsf(P[j].y)));
+    const int e = mx_exponent(amax, RU);
+    byte = (uint32_t)(e + 127);
+    const float m = exp2_int(-e);
+    const float2 mm = make_float2(m, m);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) P[j] = mul2_rn(P[j], mm);
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+        // codes of elements 8g..8g+7: P[8g..8g+7].x for g < 2, P[8(g-2)..].y otherwise
+        float q[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) q[i] = g < 2 ? P[8 * g + i].x : P[8 * (g - 2) + i].y;
+        w[g] = e2m1_pack8(q);
+    }
+}
+
+template <int BLK, bool BF16, bool TC, bool RU, bool HAD, bool CHAN>
+__global__ void __launch_bounds__(qz::THREADS, 1)
+    quantize_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmC, QuantParams p,
+                    int codes_tma) {
+    using G = QzGeom<BLK, BF16>;
+    using namespace qz;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* cbuf = smem + G::NSTAGE * G::STAGE;
+    uint8_t* sbuf = cbuf + NBUF * G::CODE_TILE;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + G::BAR_OFF);
+    uint64_t* empty = full + G::NSTAGE;
+    // consumer abort flags, indexed by tile-iteration parity: written before
+    // the per-tile consumer barrier, read after it, so every consumer takes
+    // the same decision
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + G::NSTAGE);
+    float* inv_tab = reinterpret_cast<float*>(smem + G::TAB_OFF);   // NVFP4: 1 / (s_b * s_t) per byte
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) {
+        for (int s = 0; s < G::NSTAGE; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], CONSUMER_WARPS);
+        }
+        abort_flag[0] = 0;
+        abort_flag[1] = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    const int64_t tiles_c = p.catoms;
+    const int64_t tiles = ((p.rows + G::ROWS - 1) / G::ROWS) * tiles_c;
+
+    if (warp == CONSUMER_WARPS) {
+        // ---- producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tmX);
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t last_phase[G::NSTAGE];
+            bool issued[G::NSTAGE];
+            for (int s = 0; s < G::NSTAGE; ++s) issued[s] = false, last_phase[s] = 0;
+            for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
+                // on time-out stop issuing: the consumers then time out on `full`
+                if (!mbar_wait(&empty[stage], phase ^ 1)) break;
+                mbar_arrive_expect_tx(&full[stage], G::STAGE);
+                const int64_t tr = t / tiles_c, tc = t % tiles_c;
+                uint8_t* dst = smem + stage * G::STAGE;
+#pragma unroll
+                for (int b = 0; b < G::NBOX; ++b)
+                    tma_load_2d(dst + b * (G::ROWS * 128), &tmX, &full[stage],
+                                (int32_t)(tc * 4 * BLK + b * (128 / G::ESZ)), (int32_t)(tr * G::ROWS));
+                issued[stage] = true;
+                last_phase[stage] = phase;
+                if (++stage == G::NSTAGE) { stage = 0; phase ^= 1; }
+            }
+            // no copy may still be landing in shared memory when the CTA exits
+            for (int s = 0; s < G::NSTAGE; ++s)
+                if (issued[s]) mbar_wait(&full[s], last_phase[s]);
+        }
+        return;
+    }
+
+    // ---- consumers
+    NvCtx sc;
+    if constexpr (BLK == 16) {
+        sc = nv_ctx(*p.gscale, inv_tab);
+        nv_fill_table(*p.gscale, inv_tab, tid, CONSUMERS);
+        named_barrier(1, CONSUMERS);
+    }
+    const int64_t bands = (p.rows + 127) / 128;
+    const int64_t crow = p.cols / 2;           // bytes of codes per row
+    int stage = 0, buf = 0;
+    uint32_t phase = 0, it = 0;
+    for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++it) {
+        const int64_t tr = t / tiles_c, tc = t % tiles_c;
+        const int64_t row0 = tr * G::ROWS, col0 = tc * 4 * BLK;
+        if (!mbar_wait(&full[stage], phase)) abort_flag[it & 1] = 1;
+
+        float v[G::BPT][BLK];
+        const uint8_t* sb = smem + stage * G::STAGE;
+#pragma unroll
+        for (int k = 0; k < G::BPT; ++k) {
+            const int b = tid + k * CONSUMERS;
+            const int j = b / G::ROWS, r = b % G::ROWS;
+            const int jo = j * BLK * G::ESZ;
+            const uint8_t* rowp = sb + (jo >> 7) * (G::ROWS * 128) + r * 128;
+            const int o16 = (jo & 127) >> 4;
+#pragma unroll
+            for (int c = 0; c < G::CHUNKS; ++c) {
+                const uint4 raw = *reinterpret_cast<const uint4*>(rowp + (((o16 + c) ^ (r & 7)) << 4));
+                float* d = &v[k][c * G::PER];
+                if (BF16) {
+                    d[0] = bf16_lo(raw.x); d[1] = bf16_hi(raw.x); d[2] = bf16_lo(raw.y); d[3] = bf16_hi(raw.y);
+                    d[4] = bf16_lo(raw.z); d[5] = bf16_hi(raw.z); d[6] = bf16_lo(raw.w); d[7] = bf16_hi(raw.w);
+                } else {
+                    d[0] = __uint_as_float(raw.x); d[1] = __uint_as_float(raw.y);
+                    d[2] = __uint_as_float(raw.z); d[3] = __uint_as_float(raw.w);
                 }
             }
-            if constexpr (HAD) {
-                fwht32_reg(*reinterpret_cast<float(*)[32]>(&v[it][0]));
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[stage]);
+        if (++stage == G::NSTAGE) { stage = 0; phase ^= 1; }
+
+        uint8_t* cb = cbuf + buf * G::CODE_TILE;
+        uint8_t* fb = sbuf + buf * G::SF_TILE;
 #pragma unroll
-                for (int i = 0; i < BLK; ++i) v[it][i] = __fmul_rn(v[it][i], inv_sqrt32);
-            }
-            float amax = 0.0f;
-#pragma unroll
-            for (int i = 0; i < BLK; ++i) amax = fmaxf(amax, fabsf(v[it][i]));
+        for (int k = 0; k < G::BPT; ++k) {
+            const int b = tid + k * CONSUMERS;
+            const int j = b / G::ROWS, r = b % G::ROWS;
+            const int64_t row = row0 + r, col = col0 + j * BLK;
             uint32_t byte;
-            if constexpr (BLK == 16) {
-                const NvScale sc = nv_scale_from_amax(amax, s_t, RU);
-                byte = sc.byte;
-#pragma unroll
-                for (int i = 0; i < BLK; ++i) v[it][i] = sc.degenerate ? 0.0f : __fmul_rn(v[it][i], sc.inv);
-            } else {
-                const int e = mx_exponent(amax, RU);
-                byte = (uint32_t)(e + 127);
-                const float mult = exp2_int(-e);
-#pragma unroll
-                for (int i = 0; i < BLK; ++i) v[it][i] = __fmul_rn(v[it][i], mult);
-            }
             uint32_t w[BLK / 8];
-#pragma unroll
-            for (int g = 0; g < BLK / 8; ++g) w[g] = e2m1_pack8(*reinterpret_cast<float(*)[8]>(&v[it][8 * g]));
-            if (valid[it]) {
-                uint8_t* dst = p.codes + row * (p.cols / 2) + col / 2;
+            if constexpr (BLK == 16) {
+                nv_block<RU>(v[k], sc, byte, w);
+            } else {
+                const float* chan = (CHAN && col < p.cols) ? p.chan + col : nullptr;
+                mx_block<RU, HAD>(v[k], chan, byte, w);
+            }
+            const bool inside = row < p.rows && col < p.cols;
+            if (codes_tma) {
+                uint8_t* dst = cb + r * (2 * BLK) + j * (BLK / 2);
+                if constexpr (BLK == 16) *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
+                else *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+            } else if (inside) {
+                uint8_t* dst = p.codes + row * crow + col / 2;
                 if constexpr (BLK == 16) *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
                 else *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
             }
-            if (TC) sf_atom[(rt & 31) * 16 + (rt >> 5) * 4 + cb] = (uint8_t)byte;
-            else if (valid[it]) p.scales[row * p.scols + tc * 4 + cb] = (uint8_t)byte;
+            if (TC) fb[(r >> 7) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + j] = (uint8_t)byte;
+            else if (inside) p.scales[row * p.scols + tc * 4 + j] = (uint8_t)byte;
         }
-        if (TC) {
-            __syncthreads();
-            if (tid < 32) {
-                const uint4 a = reinterpret_cast<const uint4*>(sf_atom)[tid];
-                reinterpret_cast<uint4*>(p.scales + (tr * p.catoms + tc) * 512)[tid] = a;
+        fence_proxy_async_smem();
+        named_barrier(1, CONSUMERS);
+        if (tid == 0) {
+            if (codes_tma) tma_store_2d(&tmC, cb, (int32_t)(col0 / 2), (int32_t)row0);
+            if (TC) {
+#pragma unroll
+                for (int a = 0; a < G::ROWS / 128; ++a) {
+                    const int64_t band = row0 / 128 + a;
+                    if (band < bands) bulk_store(p.scales + (band * p.catoms + tc) * 512, fb + a * 512, 512u);
+                }
             }
-            __syncthreads();
+            bulk_commit_group();
+            // the buffer the next-but-one tile writes is free once this returns
+            bulk_wait_read_1();
         }
+        if (abort_flag[it & 1]) break;
+        if (++buf == NBUF) buf = 0;
     }
+    if (tid == 0) bulk_wait_all();
 }
 
 // ------------------------------------------------------------------ sigma-delta
-// Elementwise over 8-weight chunks (grid-stride, two chunks per thread in
-// flight): it reads the fixed block scales and streams w, r in, r out, codes.
-template <int BLK, bool TC>
-__device__ __forceinline__ void sigma_delta_chunk(const SigmaDeltaParams& p, float s_t, int64_t row, int64_t col,
-                                                  const float4& w0, const float4& w1, const float4& r0,
-                                                  const float4& r1, uint32_t sb) {
-    float inv;
-    bool degenerate;
-    if (BLK == 16) {
-        const NvScale s = nv_scale_from_byte(sb, s_t);
-        inv = s.inv;
-        degenerate = s.degenerate;
-    } else {
-        inv = exp2_int(127 - (int)sb);
-        degenerate = false;
-    }
-    const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-    float rv[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
-    float v[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const float x = degenerate ? 0.0f : __fmul_rn(wv[i], inv);
-        v[i] = __fadd_rn(x, rv[i]);
-    }
-    const uint32_t codes = e2m1_pack8(v);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) rv[i] = __fsub_rn(v[i], e2m1_value((codes >> (4 * i)) & 15u));
-    const int64_t off = row * p.cols + col;
-    float4* rp = reinterpret_cast<float4*>(p.residue + off);
-    rp[0] = make_float4(rv[0], rv[1], rv[2], rv[3]);
-    rp[1] = make_float4(rv[4], rv[5], rv[6], rv[7]);
-    *reinterpret_cast<uint32_t*>(p.codes + row * (p.cols / 2) + col / 2) = codes;
+// Persistent, one CTA per SM, the same producer / consumer split as the
+// quantizer.  A tile is 32 rows x 128 weights; TMA brings the tile of w and of
+// the residue r into one shared-memory stage, together with the tile's scale
+// atoms when the scales are in the tensor-core layout (a bulk copy, so no
+// consumer waits on a global load), each consumer thread updates 4 weights
+// per row it owns (a warp covers one 512-byte row: conflict-free), writes the
+// new residue over the old one in the stage and its 4 codes into a staging
+// buffer, and one thread sends both tiles back with TMA stores.  The stage is
+// handed back to the producer once its residue store has read it.
+namespace sdk {
+constexpr int CONSUMER_WARPS = 16;
+constexpr int CONSUMERS = 32 * CONSUMER_WARPS;
+constexpr int THREADS = CONSUMERS + 32;
+constexpr int ROWS = 32;
+constexpr int COLS = 128;
+constexpr int HALF = ROWS * COLS * 4;            // w (or r) of one tile, 16 KB
+constexpr int SF_BYTES = 1024;                   // up to two scale atoms (tensor-core layout)
+constexpr int STAGE = 2 * HALF + SF_BYTES;
+constexpr int NSTAGE = 5;
+constexpr int CODE_TILE = ROWS * COLS / 2;       // 2 KB
+constexpr int NBUF = 3;
+constexpr int TAB_OFF = NSTAGE * STAGE + NBUF * CODE_TILE;   // 256-entry reciprocal table
+constexpr int BAR_OFF = TAB_OFF + 1024;
+constexpr int SMEM = BAR_OFF + 256 + 1024;
+constexpr int GPT = ROWS * COLS / 4 / CONSUMERS; // 4-weight groups per thread per tile
+}  // namespace sdk
+
+// Four E2M1 codes (element 0 in the low nibble) of four floats.
+__device__ __forceinline__ uint32_t e2m1_pack4(float a, float b, float c, float d) {
+    uint32_t out;
+    asm("{\n\t.reg .b8 b0, b1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "mov.b32 %0, {b0, b1, 0, 0};\n\t}"
+        : "=r"(out) : "f"(a), "f"(b), "f"(c), "f"(d));
+    return out;
 }
 
 template <int BLK, bool TC>
-__global__ void __launch_bounds__(256) sigma_delta_kernel(SigmaDeltaParams p) {
-    const int64_t cpr = p.cols / 8;
-    const int64_t total = p.rows * cpr;
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    const float s_t = (BLK == 16) ? *p.gscale : 0.0f;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += 2 * stride) {
-        const int64_t j = i + stride;
-        const bool has2 = j < total;
-        const int64_t row_a = i / cpr, col_a = (i % cpr) * 8;
-        const int64_t row_b = has2 ? j / cpr : row_a, col_b = has2 ? (j % cpr) * 8 : col_a;
-        const float4* wa = reinterpret_cast<const float4*>(p.w + row_a * p.cols + col_a);
-        const float4* ra = reinterpret_cast<const float4*>(p.residue + row_a * p.cols + col_a);
-        const float4* wb = reinterpret_cast<const float4*>(p.w + row_b * p.cols + col_b);
-        const float4* rb = reinterpret_cast<const float4*>(p.residue + row_b * p.cols + col_b);
-        const float4 wa0 = __ldcs(wa), wa1 = __ldcs(wa + 1), ra0 = __ldcs(ra), ra1 = __ldcs(ra + 1);
-        float4 wb0 = wa0, wb1 = wa1, rb0 = ra0, rb1 = ra1;
-        if (has2) { wb0 = __ldcs(wb); wb1 = __ldcs(wb + 1); rb0 = __ldcs(rb); rb1 = __ldcs(rb + 1); }
-        const int64_t ca = col_a / BLK, cbk = col_b / BLK;
-        const uint32_t sa = TC ? p.scales[tc_scale_offset(row_a, ca, p.catoms)] : p.scales[row_a * p.scols + ca];
-        const uint32_t sbb = TC ? p.scales[tc_scale_offset(row_b, cbk, p.catoms)] : p.scales[row_b * p.scols + cbk];
-        sigma_delta_chunk<BLK, TC>(p, s_t, row_a, col_a, wa0, wa1, ra0, ra1, sa);
-        if (has2) sigma_delta_chunk<BLK, TC>(p, s_t, row_b, col_b, wb0, wb1, rb0, rb1, sbb);
+__global__ void __launch_bounds__(sdk::THREADS, 1)
+    sigma_delta_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmR,
+                       const __grid_constant__ CUtensorMap tmC, SigmaDeltaParams p, int codes_tma) {
+    using namespace sdk;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* cbuf = smem + NSTAGE * STAGE;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
+    uint64_t* empty = full + NSTAGE;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + NSTAGE);   // [2], see quantize_kernel
+    float* inv_tab = reinterpret_cast<float*>(smem + TAB_OFF);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) {
+        for (int s = 0; s < NSTAGE; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        abort_flag[0] = 0;
+        abort_flag[1] = 0;
+        fence_mbar_init();
     }
+    __syncthreads();
+
+    const int64_t tiles_c = (p.cols + COLS - 1) / COLS;
+    const int64_t tiles = ((p.rows + ROWS - 1) / ROWS) * tiles_c;
+
+    if (warp == CONSUMER_WARPS) {
+        if (lane == 0) {
+            tma_prefetch_desc(&tmW);
+            tma_prefetch_desc(&tmR);
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t last_phase[NSTAGE];
+            bool issued[NSTAGE];
+            for (int s = 0; s < NSTAGE; ++s) issued[s] = false, last_phase[s] = 0;
+            constexpr int ATOMS = COLS / BLK / 4;          // atom columns per tile: 2 (NVFP4) or 1 (MXFP4)
+            for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
+                if (!mbar_wait(&empty[stage], phase ^ 1)) break;
+                const int64_t tc = t % tiles_c, tr = t / tiles_c;
+                const int32_t c0 = (int32_t)(tc * COLS), r0 = (int32_t)(tr * ROWS);
+                int64_t na = 0;
+                if (TC) {
+                    na = p.catoms - tc * ATOMS;
+                    na = na < ATOMS ? na : ATOMS;
+                }
+                mbar_arrive_expect_tx(&full[stage], 2 * HALF + (uint32_t)na * 512u);
+                tma_load_2d(smem + stage * STAGE, &tmW, &full[stage], c0, r0);
+                tma_load_2d(smem + stage * STAGE + HALF, &tmR, &full[stage], c0, r0);
+                if (TC)
+                    bulk_load(smem + stage * STAGE + 2 * HALF,
+                              p.scales + (((int64_t)r0 >> 7) * p.catoms + tc * ATOMS) * 512, (uint32_t)na * 512u,
+                              &full[stage]);
+                issued[stage] = true;
+                last_phase[stage] = phase;
+                if (++stage == NSTAGE) { stage = 0; phase ^= 1; }
+            }
+            for (int s = 0; s < NSTAGE; ++s)
+                if (issued[s]) mbar_wait(&full[s], last_phase[s]);
+        }
+        return;
+    }
+
+    // 1 / (s_b * s_t) (NVFP4) or 2^-e (MXFP4) for every scale byte; NaN marks
+    // a degenerate NVFP4 scale, whose weights normalise to +0
+    for (int bb = tid; bb < 256; bb += CONSUMERS) {
+        float inv;
+        if (BLK == 16) {
+            const NvScale r = nv_scale_from_byte((uint32_t)(bb & 0x7F), *p.gscale);
+            inv = r.degenerate ? __uint_as_float(0x7FC00000u) : r.inv;
+        } else {
+            inv = exp2_int(127 - bb);
+        }
+        inv_tab[bb] = inv;
+    }
+    named_barrier(1, CONSUMERS);
+    const int64_t crow = p.cols / 2;
+    int stage = 0, buf = 0, prev_stage = 0;
+    uint32_t phase = 0, it = 0;
+    for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++it) {
+        const int64_t row0 = (t / tiles_c) * ROWS, col0 = (t % tiles_c) * COLS;
+        if (!mbar_wait(&full[stage], phase)) abort_flag[it & 1] = 1;
+        uint8_t* sw = smem + stage * STAGE;
+        uint8_t* cb = cbuf + buf * CODE_TILE;
+#pragma unroll
+        for (int k = 0; k < GPT; ++k) {
+            const int g = tid + k * CONSUMERS;
+            const int r = g >> 5, q = g & 31;
+            const int64_t row = row0 + r, col = col0 + 4 * q;
+            const bool inside = row < p.rows && col < p.cols;
+            const float4 w4 = *reinterpret_cast<const float4*>(sw + r * 512 + q * 16);
+            float4* rp = reinterpret_cast<float4*>(sw + HALF + r * 512 + q * 16);
+            const float4 r4 = *rp;
+            uint32_t sb = 0;
+            if (inside) {
+                if (TC) {
+                    // atom q / (4 * BLK / 16) of the tile, byte (r0 + r) % 32 * 16 + (r0 / 32) % 4 * 4 + c % 4
+                    const int c = (4 * q) / BLK;
+                    sb = sw[2 * HALF + (c >> 2) * 512 + (int)(row & 31) * 16 + (int)((row >> 5) & 3) * 4 + (c & 3)];
+                } else {
+                    sb = __ldg(p.scales + row * p.scols + col / BLK);
+                }
+            }
+            const float inv = inv_tab[sb];
+            float2 x01, x23;
+            if (inv != inv) {
+                x01 = make_float2(0.0f, 0.0f);
+                x23 = x01;
+            } else {
+                x01 = mul2_rn(make_float2(w4.x, w4.y), make_float2(inv, inv));
+                x23 = mul2_rn(make_float2(w4.z, w4.w), make_float2(inv, inv));
+            }
+            const float2 v01 = add2_rn(x01, make_float2(r4.x, r4.y));
+            const float2 v23 = add2_rn(x23, make_float2(r4.z, r4.w));
+            const uint32_t codes = e2m1_pack4(v01.x, v01.y, v23.x, v23.y);
+            const float2 r01 = sub2_rn(v01, e2m1x2_value(codes & 0xFFu));
+            const float2 r23 = sub2_rn(v23, e2m1x2_value(codes >> 8));
+            *rp = make_float4(r01.x, r01.y, r23.x, r23.y);
+            if (codes_tma) *reinterpret_cast<uint16_t*>(cb + r * (COLS / 2) + q * 2) = (uint16_t)codes;
+            else if (inside) *reinterpret_cast<uint16_t*>(p.codes + row * crow + col / 2) = (uint16_t)codes;
+        }
+        fence_proxy_async_smem();
+        named_barrier(1, CONSUMERS);
+        if (tid == 0) {
+            tma_store_2d(&tmR, sw + HALF, (int32_t)col0, (int32_t)row0);
+            if (codes_tma) tma_store_2d(&tmC, cb, (int32_t)(col0 / 2), (int32_t)row0);
+            bulk_commit_group();
+            bulk_wait_read_1();
+            // the previous tile's residue store has read its stage: refill it
+            if (it > 0) mbar_arrive(&empty[prev_stage]);
+            prev_stage = stage;
+        }
+        if (abort_flag[it & 1]) break;
+        if (++stage == NSTAGE) { stage = 0; phase ^= 1; }
+        if (++buf == NBUF) buf = 0;
+    }
+    if (tid == 0) bulk_wait_all();
 }
 
 // ------------------------------------------------------------------ dequantize
@@ -319,69 +633,102 @@ static int grid_for(int64_t tiles, int num_sms, int per_sm) {
     return (int)(tiles < cap ? tiles : cap);
 }
 
-// Grid of exactly the CTAs that fit on the GPU at once (a persistent
-// grid-stride launch), so the last wave is never partial.
-template <typename K>
-static int resident_grid(K kernel, int64_t tiles, int num_sms) {
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, 256, 0) != cudaSuccess || per_sm < 1)
-        per_sm = 4;
-    return grid_for(tiles, num_sms, per_sm);
-}
+struct QuantMaps {
+    CUtensorMap x, codes;
+    int codes_tma;
+};
 
 template <int BLK, bool BF16, bool TC, bool RU, bool HAD, bool CHAN>
-static void launch_quant_one(const QuantParams& p, int64_t tiles, int num_sms, cudaStream_t st) {
+static cudaError_t launch_quant_one(const QuantParams& p, const QuantMaps& m, int num_sms, cudaStream_t st) {
+    using G = QzGeom<BLK, BF16>;
     auto k = quantize_kernel<BLK, BF16, TC, RU, HAD, CHAN>;
-    k<<<resident_grid(k, tiles, num_sms), 256, 0, st>>>(p);
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM);
+    if (e != cudaSuccess) return e;
+    const int64_t tiles = ((p.rows + G::ROWS - 1) / G::ROWS) * p.catoms;
+    const int grid = (int)(tiles < num_sms ? tiles : num_sms);
+    k<<<grid, qz::THREADS, G::SMEM, st>>>(m.x, m.codes, p, m.codes_tma);
+    return cudaGetLastError();
 }
 
 template <int BLK, bool BF16, bool TC, bool RU>
-static void launch_quant_mx_variants(const QuantParams& p, bool had, bool chan, int64_t tiles, int num_sms,
-                                     cudaStream_t st) {
-    if (had && chan) launch_quant_one<BLK, BF16, TC, RU, true, true>(p, tiles, num_sms, st);
-    else if (had) launch_quant_one<BLK, BF16, TC, RU, true, false>(p, tiles, num_sms, st);
-    else if (chan) launch_quant_one<BLK, BF16, TC, RU, false, true>(p, tiles, num_sms, st);
-    else launch_quant_one<BLK, BF16, TC, RU, false, false>(p, tiles, num_sms, st);
+static cudaError_t launch_quant_mx_variants(const QuantParams& p, const QuantMaps& m, bool had, bool chan,
+                                            int num_sms, cudaStream_t st) {
+    if (had && chan) return launch_quant_one<BLK, BF16, TC, RU, true, true>(p, m, num_sms, st);
+    if (had) return launch_quant_one<BLK, BF16, TC, RU, true, false>(p, m, num_sms, st);
+    if (chan) return launch_quant_one<BLK, BF16, TC, RU, false, true>(p, m, num_sms, st);
+    return launch_quant_one<BLK, BF16, TC, RU, false, false>(p, m, num_sms, st);
 }
 
 template <int BLK, bool BF16, bool TC>
-static void launch_quant_ru(const QuantParams& p, bool ru, bool had, bool chan, int64_t tiles, int num_sms,
-                            cudaStream_t st) {
+static cudaError_t launch_quant_ru(const QuantParams& p, const QuantMaps& m, bool ru, bool had, bool chan,
+                                   int num_sms, cudaStream_t st) {
     if constexpr (BLK == 16) {
-        if (ru) launch_quant_one<BLK, BF16, TC, true, false, false>(p, tiles, num_sms, st);
-        else launch_quant_one<BLK, BF16, TC, false, false, false>(p, tiles, num_sms, st);
+        if (ru) return launch_quant_one<BLK, BF16, TC, true, false, false>(p, m, num_sms, st);
+        return launch_quant_one<BLK, BF16, TC, false, false, false>(p, m, num_sms, st);
     } else {
-        if (ru) launch_quant_mx_variants<BLK, BF16, TC, true>(p, had, chan, tiles, num_sms, st);
-        else launch_quant_mx_variants<BLK, BF16, TC, false>(p, had, chan, tiles, num_sms, st);
+        if (ru) return launch_quant_mx_variants<BLK, BF16, TC, true>(p, m, had, chan, num_sms, st);
+        return launch_quant_mx_variants<BLK, BF16, TC, false>(p, m, had, chan, num_sms, st);
     }
 }
 
 template <int BLK>
-static void launch_quant_blk(const QuantParams& p, bool bf16, bool tc, bool ru, bool had, bool chan,
-                             int64_t tiles, int num_sms, cudaStream_t st) {
+static cudaError_t launch_quant_blk(const QuantParams& p, bool bf16, bool tc, bool ru, bool had, bool chan,
+                                    int num_sms, cudaStream_t st) {
+    QuantMaps m;
+    std::memset(&m, 0, sizeof(m));
+    const int esz = bf16 ? 2 : 4;
+    const int rows_tile = bf16 ? QzGeom<BLK, true>::ROWS : QzGeom<BLK, false>::ROWS;
+    if (!encode_map_2d(&m.x, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, p.x,
+                       (uint64_t)p.cols, (uint64_t)p.rows, (uint64_t)(p.ld * esz), (uint32_t)(128 / esz),
+                       (uint32_t)rows_tile, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    // codes leave by TMA when their row pitch allows it (a multiple of 16 bytes)
+    m.codes_tma = ((p.cols / 2) % 16 == 0) ? 1 : 0;
+    if (m.codes_tma &&
+        !encode_map_2d(&m.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.codes, (uint64_t)(p.cols / 2), (uint64_t)p.rows,
+                       (uint64_t)(p.cols / 2), (uint32_t)(2 * BLK), (uint32_t)rows_tile, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
     if (bf16) {
-        if (tc) launch_quant_ru<BLK, true, true>(p, ru, had, chan, tiles, num_sms, st);
-        else launch_quant_ru<BLK, true, false>(p, ru, had, chan, tiles, num_sms, st);
-    } else {
-        if (tc) launch_quant_ru<BLK, false, true>(p, ru, had, chan, tiles, num_sms, st);
-        else launch_quant_ru<BLK, false, false>(p, ru, had, chan, tiles, num_sms, st);
+        if (tc) return launch_quant_ru<BLK, true, true>(p, m, ru, had, chan, num_sms, st);
+        return launch_quant_ru<BLK, true, false>(p, m, ru, had, chan, num_sms, st);
     }
+    if (tc) return launch_quant_ru<BLK, false, true>(p, m, ru, had, chan, num_sms, st);
+    return launch_quant_ru<BLK, false, false>(p, m, ru, had, chan, num_sms, st);
 }
 
 cudaError_t launch_quantize(const QuantParams& p, int blk, bool bf16, bool tc, bool ru, bool had,
                             bool chan, cudaStream_t st, int num_sms) {
     if (p.rows == 0 || p.cols == 0) return cudaSuccess;
-    const int64_t tile_c = 4 * blk;
-    const int64_t tiles = ((p.rows + 127) / 128) * ((p.cols + tile_c - 1) / tile_c);
-    if (blk == 16) launch_quant_blk<16>(p, bf16, tc, ru, had, chan, tiles, num_sms, st);
-    else launch_quant_blk<32>(p, bf16, tc, ru, had, chan, tiles, num_sms, st);
-    return cudaGetLastError();
+    if (blk == 16) return launch_quant_blk<16>(p, bf16, tc, ru, had, chan, num_sms, st);
+    return launch_quant_blk<32>(p, bf16, tc, ru, had, chan, num_sms, st);
 }
 
+cudaError_t read_clear_quant_error(unsigned int* word) { return read_clear_module_error(word); }
+
 cudaError_t launch_sigma_delta(const SigmaDeltaParams& p, int blk, bool tc, cudaStream_t st, int num_sms) {
+    using namespace sdk;
     if (p.rows == 0 || p.cols == 0) return cudaSuccess;
-    const int64_t tiles = (p.rows * (p.cols / 8) + 511) / 512;   // CTAs of 256 threads, 2 chunks each
-#define Q4_SD(B, T) { auto k = sigma_delta_kernel<B, T>; k<<<resident_grid(k, tiles, num_sms), 256, 0, st>>>(p); }
+    CUtensorMap mw, mr, mc;
+    std::memset(&mc, 0, sizeof(mc));
+    if (!encode_map_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, p.w, (uint64_t)p.cols, (uint64_t)p.rows,
+                       (uint64_t)p.cols * 4, COLS, ROWS, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !encode_map_2d(&mr, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, p.residue, (uint64_t)p.cols, (uint64_t)p.rows,
+                       (uint64_t)p.cols * 4, COLS, ROWS, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    const int codes_tma = ((p.cols / 2) % 16 == 0) ? 1 : 0;
+    if (codes_tma && !encode_map_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.codes, (uint64_t)(p.cols / 2),
+                                    (uint64_t)p.rows, (uint64_t)(p.cols / 2), COLS / 2, ROWS,
+                                    CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    const int64_t tiles = ((p.rows + ROWS - 1) / ROWS) * ((p.cols + COLS - 1) / COLS);
+    const int grid = (int)(tiles < num_sms ? tiles : num_sms);
+#define Q4_SD(B, T)                                                                                  \
+    {                                                                                                \
+        auto k = sigma_delta_kernel<B, T>;                                                           \
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM); \
+        if (e != cudaSuccess) return e;                                                              \
+        k<<<grid, THREADS, SMEM, st>>>(mw, mr, mc, p, codes_tma);                                    \
+    }
     if (blk == 16) {
         if (tc) Q4_SD(16, true) else Q4_SD(16, false)
     } else {

@@ -55,7 +55,7 @@ def test_e2m1_decisions_exhaustive_near_grid():
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("ru", [False, True])
 @pytest.mark.parametrize("tc", [False, True])
-@pytest.mark.parametrize("shape", [(200, 336), (128, 64), (1, 16), (257, 1040)])
+@pytest.mark.parametrize("shape", [(200, 336), (128, 64), (1, 16), (257, 1040), (300, 1056), (513, 2080)])
 def test_nvfp4_quantize_parity(dtype, ru, tc, shape):
     rows, cols = shape
     x = synth.small_like("heavy", rows * 7 + cols, rows, cols)
@@ -68,6 +68,31 @@ def test_nvfp4_quantize_parity(dtype, ru, tc, shape):
         x_t = dev(x)
     s_t = oracle.tensor_scale(oracle.amax(x32), 1536.0 if ru else 2688.0)
     check_nvfp4(x32, x_t, s_t, ru, tc)
+
+
+@pytest.mark.parametrize("fmt", [q4.NVFP4, q4.MXFP4])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("rows,cols,ld", [(130, 320, 384), (257, 96, 1000), (64, 1024, 1032)])
+def test_quantize_strided_rows(fmt, dtype, rows, cols, ld):
+    """Rows `ld` elements apart (a column slice of a wider tensor)."""
+    full = synth.small_like("heavy", rows * 3 + ld, rows, ld)
+    if dtype == "bf16":
+        xt = synth.to_bf16(full)
+        x32 = np.ascontiguousarray(synth.bf16_to_f32(xt)[:, :cols])
+        x_t = dev(xt)[:, :cols]
+    else:
+        x32 = np.ascontiguousarray(full[:, :cols])
+        x_t = dev(full)[:, :cols]
+    assert x_t.stride(0) == ld
+    if fmt == q4.NVFP4:
+        s_t = oracle.tensor_scale(oracle.amax(x32), 2688.0)
+        gc, gs = q4.q4_quantize(fmt, x_t, gscale=gscale_dev(s_t), flags=q4.LAYOUT_TC)
+        oc, os_ = oracle.nvfp4_quantize(x32, s_t)
+    else:
+        gc, gs = q4.q4_quantize(fmt, x_t, flags=q4.LAYOUT_TC | q4.HADAMARD32)
+        oc, os_ = oracle.mxfp4_quantize(x32, hadamard=True)
+    assert np.array_equal(host(gc), oc)
+    assert np.array_equal(host(gs), oracle.scales_to_tc(os_))
 
 
 def test_nvfp4_degenerate_and_saturating_blocks():
@@ -85,7 +110,7 @@ def test_nvfp4_degenerate_and_saturating_blocks():
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("had,chan,ru", [(False, False, False), (True, False, False),
                                          (True, True, False), (False, True, True), (True, True, True)])
-@pytest.mark.parametrize("shape", [(200, 352), (128, 128), (3, 32)])
+@pytest.mark.parametrize("shape", [(200, 352), (128, 128), (3, 32), (390, 1312)])
 def test_mxfp4_quantize_parity(dtype, had, chan, ru, shape):
     rows, cols = shape
     x = synth.small_like("outlier", rows + 3 * cols, rows, cols)

@@ -29,9 +29,11 @@ def setup_scales(fmt, w32, tc=True):
 
 @pytest.mark.parametrize("fmt", [q4.NVFP4, q4.MXFP4])
 @pytest.mark.parametrize("tc", [True, False])
-@pytest.mark.parametrize("shape", [(200, 352), (512, 512), (1, 64)])
+@pytest.mark.parametrize("shape", [(200, 352), (512, 512), (1, 64), (70, 208), (33, 1040)])
 def test_sigma_delta_visits_bit_exact(fmt, tc, shape):
     rows, cols = shape
+    if fmt == q4.MXFP4 and cols % 32:
+        pytest.skip("MXFP4 needs whole 32-blocks")
     w = synth.small_like("weight", rows + cols, rows, cols)
     s_t, g_t, g_sc, o_sc = setup_scales(fmt, w, tc)
     r_gpu = torch.zeros((rows, cols), dtype=torch.float32, device=DEV)
