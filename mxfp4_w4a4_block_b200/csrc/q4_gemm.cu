@@ -824,30 +824,51 @@ cudaError_t launch_gemm(const GemmParams& p, cudaStream_t st, int num_sms) {
 }
 
 // ------------------------------------------------------------------ fused decode
-// Small-M GEMM with the activation quantization inside the kernel (no bf16
-// activation round trip, no workspace).  Operands are swapped so the weight
-// fills the MMA's 128-row side: D^T[n, m] = sum_k W[n, k] X[m, k].  Each CTA
-// owns 128 weight rows; warps 2..5 first quantize all of X (M <= 128 rows) into
-// shared memory -- codes in the 128-byte-swizzled K-major operand layout, scales
-// in tensor-core atoms -- while warp 0 already streams weight tiles by TMA.
-// The activation loads are batched (QBATCH per thread in flight) because the
-// quantize phase is a chain of L2 round trips.
+// Small-M GEMM (M <= 64) with the activation quantization inside the kernel:
+// no bf16 activation round trip and no workspace.  Operands are swapped so the
+// weight fills the MMA's 128-row side: D^T[n, m] = sum_k W[n, k] X[m, k], with
+// MMA N = np (M rounded up to 16).  Persistent CTAs over 128-row weight tiles:
+//   warp 0      TMA producer: per k-block of 256, the weight code tile
+//               (128 rows x 128 B, 128-byte swizzle) and its 4 scale atoms
+//               into a deep ring (the weight stream is the kernel's HBM
+//               traffic);
+//   warp 1      TMEM owner and MMA issuer: per k-block up to four
+//               128 x np x 64 block-scaled MMAs into four accumulators;
+//   warps 2..9  fetch the bf16 activations k-block by k-block (cp.async, a
+//               few k-blocks ahead) and quantize them in shared memory (codes
+//               into the swizzled K-major operand layout, scales into
+//               tensor-core atoms) while the weight tiles stream in;
+//   warps 10-13 stage each k-block's weight and activation scale atoms into
+//               TMEM (tcgen05.st, off the MMA thread: a tcgen05.cp there would
+//               queue with the MMAs), then run the epilogue: the summed
+//               accumulator lanes (= output columns), times alpha, to Y.
 namespace dec {
-constexpr int QUANT_WARPS = 8;           // warps 2..9 quantize X; warps 2..5 also run the epilogue
-constexpr int THREADS = 64 + 32 * QUANT_WARPS;
-constexpr int QBATCH = 8;                // 16-byte activation loads in flight per thread
-constexpr int W_STAGE = 128 * 128;       // 16 KB of weight codes per k-block
-constexpr int SFW_STAGE = 4 * 512;
+constexpr int QWARPS = 8;
+constexpr int EWARPS = 4;
+constexpr int FIRST_Q = 2;
+constexpr int FIRST_E = FIRST_Q + QWARPS;
+constexpr int THREADS = 32 * (FIRST_E + EWARPS);
+constexpr int W_STAGE = 128 * 128;       // weight codes of one k-block
+constexpr int SFW_STAGE = 4 * 512;       // their scale atoms
+constexpr int XSLOTS = 9;               // bf16 activation slabs (per-thread cp.async ring)
+constexpr int XDIST = 8;                // k-blocks fetched ahead (< XSLOTS): the fetch waits behind the weight stream
+constexpr int QSLOTS = 6;               // quantized activation k-blocks ahead of the MMAs
+constexpr int SFX = 4 * 512;             // activation scale atoms of one k-block
+constexpr int MAX_M = 16;
+constexpr int MAX_STAGES = 12;
 constexpr uint32_t TMEM_COLS = 256;
-constexpr uint32_t ACC_COL = 0;          // up to 128 fp32 columns
-constexpr uint32_t SFA_COL = 192;        // weight scales, 4 atoms x 4 columns
-constexpr uint32_t SFB_COL = 224;        // activation scales, 4 atoms x 4 columns
+constexpr int NACC = 4;                  // independent accumulators (MMA kk of a k-block -> accumulator kk)
+constexpr uint32_t ACC_COL = 0;          // NACC x np fp32 columns (np <= 32)
+constexpr uint32_t SF_COL = 128;         // SF_NBUF scale buffers of SF_BUF columns:
+constexpr uint32_t SF_BUF = 32;          //   weight atoms x 4 columns, then activation atoms x 4
+constexpr int SF_NBUF = 4;
 constexpr int MAX_SMEM = 232448;         // 227 KB opt-in limit per CTA
+constexpr int BAR_BYTES = 1024;       // barriers (< 512 B), then the 128-entry reciprocal table
 }  // namespace dec
 
 struct DecodeDev {
     int64_t M, N, K;
-    const uint16_t* x;
+    const uint16_t* x;       // bf16 activations [M, K]
     const float* a_gscale;
     const uint8_t* w_scales;
     const float* b_gscale;
@@ -864,34 +885,54 @@ __device__ __forceinline__ uint32_t sw128_offset(int row, int byte_in_row) {
                       (byte_in_row & 15));
 }
 
+struct DecodeLayout {
+    int xraw, xq, off_w, off_sfw, off_xraw, off_xq, off_sfx, off_bar, total;
+};
+
+__host__ __device__ inline DecodeLayout decode_layout(int np, int stages) {
+    DecodeLayout L;
+    L.xraw = np * 512;                    // bf16 slab: np rows x 256 elements
+    L.xq = np * 128;                      // codes: np rows x 128 bytes (1024-aligned: np % 16 == 0)
+    L.off_w = 0;
+    L.off_sfw = L.off_w + stages * dec::W_STAGE;
+    L.off_xq = L.off_sfw + stages * dec::SFW_STAGE;
+    L.off_xraw = L.off_xq + dec::QSLOTS * L.xq;
+    L.off_sfx = L.off_xraw + dec::XSLOTS * L.xraw;
+    L.off_bar = L.off_sfx + dec::QSLOTS * dec::SFX;
+    L.total = L.off_bar + dec::BAR_BYTES + 1024;
+    return L;
+}
+
 __global__ void __launch_bounds__(dec::THREADS, 1)
     fused_decode_kernel(const __grid_constant__ CUtensorMap tmW, DecodeDev p) {
     using namespace dec;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int np = p.np, nkb = p.nkb, S = p.stages;
-    const int xslab = np * 128;                              // bytes of X codes per k-block
-    uint8_t* sx = smem;                                      // nkb slabs
-    uint8_t* sxf = sx + (size_t)nkb * xslab;                 // nkb x 2 KB of X scale atoms
-    uint8_t* sw = sxf + (size_t)nkb * 2048;                  // S weight stages (1024-aligned)
-    uint8_t* swf = sw + (size_t)S * W_STAGE;                 // S x 2 KB weight scale atoms
-    uint64_t* full = reinterpret_cast<uint64_t*>(swf + (size_t)S * SFW_STAGE);
-    uint64_t* empty = full + S;
-    uint64_t* x_ready = empty + S;
-    uint64_t* tmem_full = x_ready + 1;
+    const DecodeLayout L = decode_layout(np, S);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.off_bar);   // [S] weight tile landed
+    uint64_t* empty = full + MAX_STAGES;                               // [S] its MMAs are done
+    uint64_t* xq_full = empty + MAX_STAGES;                            // [QSLOTS] quantized k-block ready
+    uint64_t* xq_empty = xq_full + QSLOTS;                             // [QSLOTS] its MMAs are done
+    uint64_t* sf_ready = xq_empty + QSLOTS;                            // [SF_NBUF] scales staged in TMEM buffer
+    uint64_t* sf_free = sf_ready + SF_NBUF;                            // [SF_NBUF] its MMAs are done
+    uint64_t* tmem_full = sf_free + SF_NBUF;
     uint64_t* tmem_empty = tmem_full + 1;
     uint64_t* mma_done = tmem_empty + 1;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+    float* inv_tab = reinterpret_cast<float*>(smem + L.off_bar + 512);   // 128 entries
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-        mbar_init(x_ready, 32 * QUANT_WARPS);
+        for (int x = 0; x < QSLOTS; ++x) {
+            mbar_init(&xq_full[x], QWARPS);
+            mbar_init(&xq_empty[x], 1);
+        }
+        for (int b = 0; b < SF_NBUF; ++b) { mbar_init(&sf_ready[b], EWARPS); mbar_init(&sf_free[b], 1); }
         mbar_init(tmem_full, 1);
-        mbar_init(tmem_empty, 128);
+        mbar_init(tmem_empty, EWARPS);
         mbar_init(mma_done, 1);
-        *abort_flag = 0;
         fence_mbar_init();
     }
     if (warp == 1) { tmem_alloc(tmem_holder, TMEM_COLS); tmem_relinquish(); }
@@ -906,130 +947,187 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
-            uint32_t last_phase[16];
-            bool issued[16];
-            for (int s = 0; s < S; ++s) issued[s] = false, last_phase[s] = 0;
-            for (int64_t t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x) {
+            uint32_t last_phase[MAX_STAGES];
+            bool issued[MAX_STAGES];
+            for (int s = 0; s < MAX_STAGES; ++s) issued[s] = false, last_phase[s] = 0;
+            bool ok = true;
+            for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
                 for (int kb = 0; kb < nkb; ++kb) {
-                    if (!mbar_wait(&empty[stage], phase ^ 1)) { *abort_flag = 1; break; }
+                    if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
                     const int64_t krem = p.K - (int64_t)kb * 256;
                     const int nmma = (krem < 256 ? (int)krem : 256) / 64;
                     mbar_arrive_expect_tx(&full[stage], W_STAGE + nmma * 512);
-                    tma_load_2d(sw + stage * W_STAGE, &tmW, &full[stage], kb * 128, (int32_t)(t * 128));
-                    bulk_load(swf + stage * SFW_STAGE, p.w_scales + (t * p.catoms + (int64_t)kb * 4) * 512,
+                    tma_load_2d(smem + L.off_w + stage * W_STAGE, &tmW, &full[stage], kb * 128, (int32_t)(t * 128));
+                    bulk_load(smem + L.off_sfw + stage * SFW_STAGE, p.w_scales + (t * p.catoms + (int64_t)kb * 4) * 512,
                               (uint32_t)nmma * 512u, &full[stage]);
                     issued[stage] = true;
                     last_phase[stage] = phase;
                     if (++stage == S) { stage = 0; phase ^= 1; }
                 }
             }
+            // no copy may still be landing in shared memory when the CTA exits
             for (int s = 0; s < S; ++s)
                 if (issued[s]) mbar_wait(&full[s], last_phase[s]);
         }
     } else if (warp == 1) {
         if (lane == 0) {
             const uint32_t idesc = idesc_mxf4(128, np, false);
-            int stage = 0;
-            uint32_t phase = 0, acc_phase = 0;
-            bool ok = mbar_wait(x_ready, 0);
-            if (!ok) *abort_flag = 1;
-            tc_fence_after();
-            for (int64_t t = blockIdx.x; ok && t < tiles && !*abort_flag; t += gridDim.x) {
-                if (!mbar_wait(tmem_empty, acc_phase ^ 1)) { *abort_flag = 1; break; }
+            int stage = 0, x = 0, b = 0;
+            uint32_t phase = 0, xphase = 0, bphase = 0, acc_phase = 0;
+            bool ok = true;
+            for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+                if (!mbar_wait(tmem_empty, acc_phase ^ 1)) { ok = false; break; }
                 tc_fence_after();
+                uint32_t started = 0;                    // bit j: accumulator j holds a partial sum
                 for (int kb = 0; kb < nkb; ++kb) {
-                    if (!mbar_wait(&full[stage], phase)) { *abort_flag = 1; break; }
+                    if (!mbar_wait(&full[stage], phase) || !mbar_wait(&xq_full[x], xphase) ||
+                        !mbar_wait(&sf_ready[b], bphase)) { ok = false; break; }
                     tc_fence_after();
                     const int64_t krem = p.K - (int64_t)kb * 256;
                     const int nmma = (krem < 256 ? (int)krem : 256) / 64;
-                    const uint32_t wf = smem_u32(swf + stage * SFW_STAGE);
-                    const uint32_t xf = smem_u32(sxf + kb * 2048);
-                    for (int a = 0; a < nmma; ++a) {
-                        tmem_cp_sf(tmem + SFA_COL + a * 4, smem_desc(wf + a * 512, 0, 128, 0));
-                        tmem_cp_sf(tmem + SFB_COL + a * 4, smem_desc(xf + a * 512, 0, 128, 0));
+                    const uint32_t sfa = tmem + SF_COL + b * SF_BUF, sfb = sfa + 16;
+                    const uint64_t adesc = smem_desc(smem_u32(smem + L.off_w + stage * W_STAGE), 16, 1024, 2);
+                    const uint64_t bdesc = smem_desc(smem_u32(smem + L.off_xq + x * L.xq), 16, 1024, 2);
+                    // four independent accumulation chains: tiny-N MMAs into one
+                    // accumulator would serialise on their latency
+                    for (int kk = 0; kk < nmma; ++kk) {
+                        mma_nvf4(tmem + ACC_COL + kk * np, adesc + 2 * kk, bdesc + 2 * kk, idesc, sfa + kk * 4,
+                                 sfb + kk * 4, (started >> kk) & 1u);
+                        started |= 1u << kk;
                     }
-                    const uint64_t adesc = smem_desc(smem_u32(sw + stage * W_STAGE), 16, 1024, 2);
-                    const uint64_t bdesc = smem_desc(smem_u32(sx + kb * xslab), 16, 1024, 2);
-                    for (int kk = 0; kk < nmma; ++kk)
-                        mma_nvf4(tmem + ACC_COL, adesc + 2 * kk, bdesc + 2 * kk, idesc, tmem + SFA_COL + kk * 4,
-                                 tmem + SFB_COL + kk * 4, (kb > 0 || kk > 0) ? 1u : 0u);
                     tc_commit(&empty[stage]);
+                    tc_commit(&xq_empty[x]);
+                    tc_commit(&sf_free[b]);
                     if (++stage == S) { stage = 0; phase ^= 1; }
+                    if (++x == QSLOTS) { x = 0; xphase ^= 1; }
+                    if (++b == SF_NBUF) { b = 0; bphase ^= 1; }
                 }
-                if (*abort_flag) break;
+                if (!ok) break;
                 tc_commit(tmem_full);
                 acc_phase ^= 1;
             }
+            // all MMAs of this thread are complete before TMEM is released
             tc_commit(mma_done);
             mbar_wait(mma_done, 0);
         }
-    } else {
-        // ---- quantize X into shared memory (warps 2..9)
-        const int qt = threadIdx.x - 64;
-        constexpr int QT = 32 * QUANT_WARPS;
-        const float s_t = *p.a_gscale;
-        for (int i = qt; i < nkb * 512; i += QT) reinterpret_cast<uint32_t*>(sxf)[i] = 0u;
-        asm volatile("bar.sync 1, %0;" ::"n"(QT) : "memory");
-        // thread -> (chunk ch of every row); the two halves of a 16-block are
-        // chunks ch and ch ^ 1, i.e. neighbouring lanes (cpr is a multiple of 8)
-        const int cpr = (int)(p.K / 8);
-        const int mrows = (int)p.M;
-        for (int ch = qt; ch < cpr; ch += QT) {
-            const unsigned mask = __activemask();
-            const int kb = ch >> 5;                        // 32 chunks of 8 per k-block
-            const int byte_in_row = (ch & 31) * 4;
-            for (int r0 = 0; r0 < np; r0 += QBATCH) {
-                uint4 raw[QBATCH];
-#pragma unroll
-                for (int j = 0; j < QBATCH; ++j) {
-                    const int r = r0 + j;
-                    raw[j] = make_uint4(0u, 0u, 0u, 0u);
-                    if (r < mrows) raw[j] = __ldg(reinterpret_cast<const uint4*>(p.x + (int64_t)r * p.K + ch * 8));
-                }
-#pragma unroll
-                for (int j = 0; j < QBATCH; ++j) {
-                    const int r = r0 + j;
-                    float v[8] = {bf16_lo(raw[j].x), bf16_hi(raw[j].x), bf16_lo(raw[j].y), bf16_hi(raw[j].y),
-                                  bf16_lo(raw[j].z), bf16_hi(raw[j].z), bf16_lo(raw[j].w), bf16_hi(raw[j].w)};
-                    float amax = 0.0f;
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
-                    amax = fmaxf(amax, __shfl_xor_sync(mask, amax, 1));
-                    const NvScale sc = nv_scale_from_amax(amax, s_t, false);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) v[i] = sc.degenerate ? 0.0f : __fmul_rn(v[i], sc.inv);
-                    *reinterpret_cast<uint32_t*>(sx + (size_t)kb * xslab + sw128_offset(r, byte_in_row)) =
-                        e2m1_pack8(v);
-                    if ((ch & 1) == 0) {
-                        const int cin = (ch >> 1) & 15;            // scale column within the k-block
-                        sxf[(size_t)kb * 2048 + (cin >> 2) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (cin & 3)] =
-                            (uint8_t)sc.byte;
-                    }
-                }
+    } else if (warp < FIRST_E) {
+        // ---- quantize activation slabs (warps 2..9)
+        const int qt = threadIdx.x - 32 * FIRST_Q;
+        constexpr int QT = 32 * QWARPS;
+        const NvCtx sc = nv_ctx(*p.a_gscale, inv_tab);
+        nv_fill_table(*p.a_gscale, inv_tab, qt, QT);
+        named_barrier(1, QT);
+        // Each quantizer thread fetches exactly the activation bytes it will
+        // quantize with cp.async, XDIST k-blocks ahead, into its own part of a
+        // ring of XSLOTS slabs.  These copies go through the load/store path,
+        // not the TMA queue the weight tiles fill, so they are not held up
+        // behind the weight stream; no thread reads another's bytes, so the
+        // copy groups alone order the ring.
+        const int64_t my_tiles = tiles > blockIdx.x ? (tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+        const int64_t total_kb = my_tiles * nkb;
+        const uint16_t* xg = p.x;
+        auto fetch = [&](int64_t i) {
+            uint8_t* raw = smem + L.off_xraw + (int)(i % XSLOTS) * L.xraw;
+            const int64_t k0 = (i % nkb) * 256;
+            for (int b = qt; b < np * 16; b += QT) {
+                const int m = b >> 4, j = b & 15;
+                const int64_t k = k0 + j * 16;
+                const bool in = m < p.M && k < p.K;     // outside X: zero fill
+                const uint16_t* src = in ? xg + m * p.K + k : xg;
+                cp_async16(raw + m * 512 + j * 32, src, in);
+                cp_async16(raw + m * 512 + j * 32 + 16, src + 8, in);
             }
+        };
+        for (int64_t i = 0; i < XDIST; ++i) {
+            if (i < total_kb) fetch(i);
+            cp_async_commit();
         }
-        fence_proxy_async_smem();
-        mbar_arrive(x_ready);
-        if (warp >= 6) goto decode_done;                     // warps 6..9 only quantize
-
-        // ---- epilogue: thread = one weight row = one output column
+        int y = 0;
+        uint32_t yphase = 0;
+        for (int64_t i = 0; i < total_kb; ++i) {
+            if (i + XDIST < total_kb) fetch(i + XDIST);
+            cp_async_commit();
+            cp_async_wait<XDIST>();                      // k-block i has landed
+            if (!mbar_wait(&xq_empty[y], yphase ^ 1)) break;
+            const uint8_t* raw = smem + L.off_xraw + (int)(i % XSLOTS) * L.xraw;
+            uint8_t* xq = smem + L.off_xq + y * L.xq;
+            uint8_t* sf = smem + L.off_sfx + y * SFX;
+            // block b = (row m = b / 16, block j = b % 16 of the 256-element k-block)
+            for (int b = qt; b < np * 16; b += QT) {
+                const int m = b >> 4, j = b & 15;
+                const uint4 c0 = *reinterpret_cast<const uint4*>(raw + m * 512 + j * 32);
+                const uint4 c1 = *reinterpret_cast<const uint4*>(raw + m * 512 + j * 32 + 16);
+                const float v[16] = {bf16_lo(c0.x), bf16_hi(c0.x), bf16_lo(c0.y), bf16_hi(c0.y),
+                                     bf16_lo(c0.z), bf16_hi(c0.z), bf16_lo(c0.w), bf16_hi(c0.w),
+                                     bf16_lo(c1.x), bf16_hi(c1.x), bf16_lo(c1.y), bf16_hi(c1.y),
+                                     bf16_lo(c1.z), bf16_hi(c1.z), bf16_lo(c1.w), bf16_hi(c1.w)};
+                uint32_t byte, w[2];
+                nv_block<false>(v, sc, byte, w);
+                *reinterpret_cast<uint2*>(xq + sw128_offset(m, j * 8)) = make_uint2(w[0], w[1]);
+                sf[(j >> 2) * 512 + (m & 31) * 16 + ((m >> 5) & 3) * 4 + (j & 3)] = (uint8_t)byte;
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&xq_full[y]);
+            if (++y == QSLOTS) { y = 0; yphase ^= 1; }
+        }
+        cp_async_wait<0>();                              // nothing still landing at exit
+    } else {
+        // ---- epilogue (warps 10..13): thread = one weight row = one output column
         const int quad = warp & 3;
         const float alpha = __fmul_rn(*p.a_gscale, *p.b_gscale);
+        const int nacc = p.K / 64 < NACC ? (int)(p.K / 64) : NACC;   // accumulators that received an MMA
+        const uint32_t qaddr = tmem + ((uint32_t)(quad * 32) << 16);
         uint32_t acc_phase = 0;
-        for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
-            if (!mbar_wait(tmem_full, acc_phase)) { *abort_flag = 1; break; }
+        int stage = 0, x = 0, b = 0;
+        uint32_t phase = 0, xphase = 0, bphase = 0;
+        bool ok = true;
+        for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+            // Stage every k-block's weight and activation scale atoms into a TMEM
+            // scale buffer with tcgen05.st (each warp fills its lane quarter
+            // with the whole atom), keeping these copies off the MMA thread.
+            for (int kb = 0; kb < nkb; ++kb) {
+                if (!mbar_wait(&full[stage], phase) || !mbar_wait(&xq_full[x], xphase) ||
+                    !mbar_wait(&sf_free[b], bphase ^ 1)) { ok = false; break; }
+                tc_fence_after();
+                const int64_t krem = p.K - (int64_t)kb * 256;
+                const int nmma = (krem < 256 ? (int)krem : 256) / 64;
+                const uint8_t* wf = smem + L.off_sfw + stage * SFW_STAGE;
+                const uint8_t* xf = smem + L.off_sfx + x * SFX;
+                const uint32_t dst = qaddr + SF_COL + b * SF_BUF;
+                for (int a = 0; a < nmma; ++a) {
+                    const uint4 va = *reinterpret_cast<const uint4*>(wf + a * 512 + lane * 16);
+                    const uint4 vb = *reinterpret_cast<const uint4*>(xf + a * 512 + lane * 16);
+                    tmem_st4(dst + a * 4, va.x, va.y, va.z, va.w);
+                    tmem_st4(dst + 16 + a * 4, vb.x, vb.y, vb.z, vb.w);
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sf_ready[b]);
+                if (++stage == S) { stage = 0; phase ^= 1; }
+                if (++x == QSLOTS) { x = 0; xphase ^= 1; }
+                if (++b == SF_NBUF) { b = 0; bphase ^= 1; }
+            }
+            if (!ok) break;
+            if (!mbar_wait(tmem_full, acc_phase)) break;
             tc_fence_after();
             const int64_t n = t * 128 + quad * 32 + lane;
-            for (int c0 = 0; c0 < np; c0 += 32) {
-                uint32_t r[32];
-                tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + ACC_COL + c0, r);
-                tmem_ld_wait();
+            for (int c0 = 0; c0 < np; c0 += 16) {
+                float acc[16];
+                for (int a = 0; a < nacc; ++a) {
+                    uint32_t r[16];
+                    tmem_ld16(tmem + ((uint32_t)(quad * 32) << 16) + ACC_COL + a * np + c0, r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) acc[j] = a == 0 ? __uint_as_float(r[j]) : __fadd_rn(acc[j], __uint_as_float(r[j]));
+                }
                 if (n < p.N) {
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
+                    for (int j = 0; j < 16; ++j) {
                         const int64_t m = c0 + j;
                         if (m < p.M) {
-                            const float val = __uint_as_float(r[j]) * alpha;
+                            const float val = acc[j] * alpha;
                             if (p.out_bf16)
                                 reinterpret_cast<__nv_bfloat16*>(p.y)[m * p.N + n] = __float2bfloat16_rn(val);
                             else
@@ -1039,27 +1137,22 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
                 }
             }
             tc_fence_before();
-            mbar_arrive(tmem_empty);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tmem_empty);
             acc_phase ^= 1;
         }
     }
-decode_done:
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
 }
 
-static int decode_smem_bytes(int np, int nkb, int stages) {
-    return 1024 + nkb * (np * 128 + 2048) + stages * (dec::W_STAGE + dec::SFW_STAGE) + (2 * stages + 8) * 8 + 64;
-}
-
 static int decode_stages(int64_t M, int64_t K) {
-    if (M <= 0 || M > 128 || K <= 0 || K > (1 << 20)) return 0;
+    if (M <= 0 || M > dec::MAX_M || K <= 0) return 0;
     const int np = (int)((M + 15) / 16 * 16);
-    const int nkb = (int)((K + 255) / 256);
-    int stages = 8;
-    while (stages >= 2 && decode_smem_bytes(np, nkb, stages) > dec::MAX_SMEM) --stages;
+    int stages = dec::MAX_STAGES;
+    while (stages >= 2 && decode_layout(np, stages).total > dec::MAX_SMEM) --stages;
     return stages >= 2 ? stages : 0;
 }
 
@@ -1079,7 +1172,7 @@ cudaError_t launch_fused_decode(const FusedDecodeParams& p, cudaStream_t st, int
     d.w_scales = p.b_scales; d.b_gscale = p.b_gscale; d.y = p.y;
     d.catoms = ((p.K / 16) + 3) / 4;
     d.np = np; d.nkb = nkb; d.stages = stages; d.out_bf16 = p.out_bf16 ? 1 : 0;
-    const int smem = decode_smem_bytes(np, nkb, stages);
+    const int smem = decode_layout(np, stages).total;
     cudaError_t e = cudaFuncSetAttribute(fused_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     const int64_t tiles = (p.N + 127) / 128;

@@ -138,63 +138,6 @@ struct QzGeom {
     static_assert(BPT >= 1 && ROWS % 128 == 0 && ROWS <= 256, "tile geometry");
 };
 
-// NVFP4 per-launch context: the tensor scale, 6 * s_t and its reciprocal,
-// whether the fast RN scale path applies, and the shared-memory table of
-// 1 / (dec(s_b) * s_t) for every E4M3 byte 0..127 (NaN marks a degenerate
-// scale: zero, or a reciprocal that is not finite).
-struct NvCtx {
-    float s_t, denom, rden;
-    bool st_ok, fast;
-    const float* tab;
-};
-
-__device__ __forceinline__ NvCtx nv_ctx(float s_t, const float* tab) {
-    NvCtx c;
-    c.s_t = s_t;
-    c.st_ok = st_valid(s_t);
-    c.denom = __fmul_rn(6.0f, s_t);
-    c.rden = __frcp_rn(c.denom);
-    c.fast = c.st_ok && isfinite(c.rden) && c.rden >= 0x1p-126f && c.denom >= 0x1p-126f;
-    c.tab = tab;
-    return c;
-}
-
-__device__ __forceinline__ void nv_fill_table(float s_t, float* tab, int tid, int nthreads) {
-    for (int b = tid; b < 128; b += nthreads) {
-        const NvScale r = nv_scale_from_byte((uint32_t)b, s_t);
-        tab[b] = r.degenerate ? __uint_as_float(0x7FC00000u) : r.inv;
-    }
-}
-
-// One NVFP4 block: amax, E4M3 scale byte (RN or RU of amax / (6 s_t)),
-// codes of x * inv (all zero for a degenerate scale).
-template <bool RU>
-__device__ __forceinline__ void nv_block(const float (&v)[16], const NvCtx& c, uint32_t& byte, uint32_t (&w)[2]) {
-    float amax = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
-    if (!c.st_ok) byte = 0;
-    else if (!RU && c.fast) byte = e4m3_rn_of_quotient(amax, c.denom, c.rden);
-    else byte = RU ? e4m3_ru(__fdiv_rn(amax, c.denom)) : e4m3_rn(__fdiv_rn(amax, c.denom));
-    const float inv = c.tab[byte];
-    if (inv != inv) {
-        w[0] = w[1] = 0u;
-        return;
-    }
-    const float2 iv = make_float2(inv, inv);
-#pragma unroll
-    for (int g = 0; g < 2; ++g) {
-        float q[8];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float2 m = mul2_rn(make_float2(v[8 * g + 2 * i], v[8 * g + 2 * i + 1]), iv);
-            q[2 * i] = m.x;
-            q[2 * i + 1] = m.y;
-        }
-        w[g] = e2m1_pack8(q);
-    }
-}
-
 // One MXFP4 block of 32 with the optional per-column multiplier and block
 // Hadamard-32.  Values are held as pairs P_j = (v_j, v_{j+16}), so the
 // butterflies of strides 1, 2, 4 and 8 (pairs j, j+h with both j, j+h < 16)

@@ -97,10 +97,12 @@ def test_gemm_closed_form_integer_case():
     assert np.all(y == K * 0.5)
 
 
-@pytest.mark.parametrize("M", [1, 16, 33, 128])
-def test_fused_activation_quant_decode_small(M):
-    """a_kind = A_BF16 for small M: the kernel quantizes the bf16 activations itself."""
-    N, K = 392, 1088
+@pytest.mark.parametrize("M,K", [(1, 1088), (16, 1088), (33, 1216), (64, 1152), (65, 1088), (128, 1088)])
+def test_fused_activation_quant_decode_small(M, K):
+    """a_kind = A_BF16 for small M: the kernel quantizes the bf16 activations
+    itself (M <= 64; larger M quantizes once into the workspace).  K leaves
+    partial last k-blocks of 64, 192 and 128 elements; N a partial tile."""
+    N = 392
     x = synth.to_bf16(synth.small_like("heavy", M, M, K))
     x32 = synth.bf16_to_f32(x)
     w = synth.small_like("weight", 9, N, K)
