@@ -76,6 +76,7 @@ def _load():
         "q4o_dequantize": (i32, [i32, P, P, f32, i64, i64, P]),
         "q4o_sigma_delta_step": (i32, [i32, P, i64, i64, P, f32, P, P]),
         "q4o_gemm": (i32, [i32, i64, i64, i64, P, P, f32, P, P, f32, P, i64, P]),
+        "q4o_gemm_w4a16": (i32, [i32, i64, i64, i64, P, P, P, f32, P, i64, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -250,6 +251,25 @@ def gemm(fmt: int, a_codes, a_scales, a_st, b_codes, b_scales, b_st, M, N, K, ro
                           None if idx is None else _ptr(idx), n_rows, _ptr(y))
     if rc != 0:
         raise ValueError("gemm: bad shape")
+    return y
+
+
+def gemm_w4a16(fmt: int, x, b_codes, b_scales, b_st, M, N, K, rows=None):
+    """Y = alpha * X dec(W)^T in binary64 with X given as float32 (bf16 values);
+    optionally only the listed rows."""
+    xa = _f32(x)
+    bc = np.ascontiguousarray(b_codes, dtype=np.uint8)
+    bsc = np.ascontiguousarray(b_scales, dtype=np.uint8)
+    if rows is None:
+        idx, n_rows = None, M
+    else:
+        idx = np.ascontiguousarray(rows, dtype=np.int64)
+        n_rows = idx.size
+    y = np.zeros((n_rows, N), np.float64)
+    rc = _load().q4o_gemm_w4a16(fmt, M, N, K, _ptr(xa), _ptr(bc), _ptr(bsc), float(np.float32(b_st)),
+                                None if idx is None else _ptr(idx), n_rows, _ptr(y))
+    if rc != 0:
+        raise ValueError("gemm_w4a16: bad shape")
     return y
 
 

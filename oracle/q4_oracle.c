@@ -430,3 +430,36 @@ int q4o_gemm(int format, int64_t M, int64_t N, int64_t K,
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* W4A16 GEMM Y = alpha * X dec(W)^T ([LT] introduction: weight            */
+/* Sigma-Delta evaluated in frozen-weight W4A16 forward passes; sec. 0.2:    */
+/* BF16 is the compute view of the weights).  X holds the activations as     */
+/* binary32 values (exact copies of their bf16 values); W is quantized       */
+/* (codes, row-major block scales); dec(W) = code * s_b and alpha = s_t for   */
+/* NVFP4, dec(W) = code * 2^e and alpha = 1 for MXFP4.  Triple loop in        */
+/* binary64.  If row_idx is non-NULL only those n_rows rows of Y are computed. */
+/* ------------------------------------------------------------------------ */
+int q4o_gemm_w4a16(int format, int64_t M, int64_t N, int64_t K, const float* x,
+                   const uint8_t* b_codes, const uint8_t* b_scales, float b_st,
+                   const int64_t* row_idx, int64_t n_rows, double* y)
+{
+    int blk = format == Q4O_NVFP4 ? 16 : 32;
+    if (K % blk != 0) return -1;
+    int64_t nb = K / blk;
+    double alpha = format == Q4O_NVFP4 ? (double)b_st : 1.0;
+    int64_t nr = row_idx ? n_rows : M;
+    for (int64_t ii = 0; ii < nr; ++ii) {
+        int64_t i = row_idx ? row_idx[ii] : ii;
+        for (int64_t j = 0; j < N; ++j) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                double b = q4o_e2m1_decode(code_at(b_codes, K, j, k))
+                         * block_scale_value(format, b_scales[j * nb + k / blk]);
+                acc += (double)x[i * K + k] * b;
+            }
+            y[ii * N + j] = alpha * acc;
+        }
+    }
+    return 0;
+}
