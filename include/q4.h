@@ -82,8 +82,10 @@ enum {
 /* Kinds of GEMM left operand. */
 enum {
     Q4_A_QUANTIZED = 0,  /* a = packed codes [M, K/2], a_scales in TC layout  */
-    Q4_A_BF16 = 1        /* a = bf16 [M, K]; quantized inside the call with
+    Q4_A_BF16 = 1,       /* a = bf16 [M, K]; quantized inside the call with
                             the tensor scale *d_a_gscale (NVFP4 only)         */
+    Q4_A_BF16_W4A16 = 2  /* a = bf16 [M, K] kept in bf16: W4A16, the weight is
+                            dequantized (exactly, to bf16) on the fly         */
 };
 
 /* Library version: major * 10000 + minor * 100 + patch. */
@@ -196,6 +198,16 @@ Q4_API q4_status q4_gemm(q4_format format, int block, int64_t M, int64_t N, int6
                   const float* d_b_gscale,
                   q4_dtype out_dt, void* y, void* workspace, size_t ws_bytes,
                   void* stream);
+
+/*
+ * a_kind = Q4_A_BF16_W4A16 ("Looped Transformer quantization", introduction
+ *   and sec. 0.2: the looped core runs weight-only 4-bit, W4A16, with BF16 as
+ *   the compute view):  Y = alpha * X dec(W)^T with X the bf16 activations
+ *   [M, K] (not quantized), dec(W) = code * s_b (NVFP4, exact in bf16) or
+ *   code * 2^e (MXFP4), alpha = s_tB (NVFP4) or 1; bf16 x bf16 products summed
+ *   in FP32 on the tensor cores.  a_scales and d_a_gscale must be NULL; no
+ *   workspace.  K % 64 == 0, N % 8 == 0.
+ */
 
 /* Scratch bytes q4_gemm needs for these arguments (0 when none). */
 Q4_API size_t q4_gemm_workspace_size(q4_format format, int64_t M, int64_t N, int64_t K,

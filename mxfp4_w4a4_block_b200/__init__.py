@@ -30,6 +30,7 @@ HADAMARD32 = 4
 
 A_QUANTIZED = 0
 A_BF16 = 1
+A_BF16_W4A16 = 2
 
 BLOCK = {NVFP4: 16, MXFP4: 32}
 

@@ -149,11 +149,13 @@ q4_status q4_gemm(q4_format format, int block, int64_t M, int64_t N, int64_t K, 
                   size_t ws_bytes, void* stream) {
     if (!valid_format(format) || !valid_dtype(out_dt) || M < 0 || N < 0 || K < 0) return Q4_ERR_ARG;
     if (block != block_of(format)) return Q4_ERR_UNSUPPORTED;
-    if (a_kind != Q4_A_QUANTIZED && a_kind != Q4_A_BF16) return Q4_ERR_ARG;
+    if (a_kind != Q4_A_QUANTIZED && a_kind != Q4_A_BF16 && a_kind != Q4_A_BF16_W4A16) return Q4_ERR_ARG;
     if (a_kind == Q4_A_BF16 && format != Q4_NVFP4) return Q4_ERR_UNSUPPORTED;
-    if (format == Q4_NVFP4 && (!d_a_gscale || !d_b_gscale)) return Q4_ERR_ARG;
+    const bool w4a16 = a_kind == Q4_A_BF16_W4A16;
+    if (format == Q4_NVFP4 && ((!w4a16 && !d_a_gscale) || !d_b_gscale)) return Q4_ERR_ARG;
     if (format == Q4_MXFP4 && (d_a_gscale || d_b_gscale)) return Q4_ERR_ARG;
-    if (a_kind == Q4_A_BF16 && a_scales) return Q4_ERR_ARG;
+    if (w4a16 && d_a_gscale) return Q4_ERR_ARG;
+    if (a_kind != Q4_A_QUANTIZED && a_scales) return Q4_ERR_ARG;
     if (K % 64 || N % 8) return Q4_ERR_SHAPE;
     if (K > ((int64_t)1 << 30) || M > ((int64_t)1 << 31) || N > ((int64_t)1 << 31)) return Q4_ERR_SHAPE;
     if (M == 0 || N == 0) return Q4_OK;
@@ -166,6 +168,12 @@ q4_status q4_gemm(q4_format format, int block, int64_t M, int64_t N, int64_t K, 
     if (!aligned16(a) || !aligned16(b_codes) || !aligned16(b_scales) || (a_scales && !aligned16(a_scales)))
         return Q4_ERR_ALIGN;
 
+    if (w4a16) {
+        q4::W4A16Params w;
+        w.M = M; w.N = N; w.K = K; w.x = a; w.b_codes = b_codes; w.b_scales = b_scales;
+        w.b_gscale = d_b_gscale; w.y = y; w.out_bf16 = out_dt == Q4_BF16; w.mxfp4 = format == Q4_MXFP4;
+        return cuda_status(q4::launch_w4a16(w, st, num_sms()));
+    }
     const uint8_t* a_codes = static_cast<const uint8_t*>(a);
     if (a_kind == Q4_A_BF16) {
         if (q4::fused_decode_supported(M, K)) {

@@ -823,6 +823,333 @@ cudaError_t launch_gemm(const GemmParams& p, cudaStream_t st, int num_sms) {
     return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ W4A16 GEMM
+// Y = alpha * X dec(W)^T with bf16 activations X [M, K] and a 4-bit weight W
+// [N, K] (codes + tensor-core scale atoms): the weight is dequantized in
+// shared memory to bf16 -- code * block scale is exact in bf16 (at most 6
+// significant bits, exponent in range) -- and multiplied on the tcgen05 tensor
+// cores (kind::f16, bf16 x bf16 -> fp32).  alpha = s_t (NVFP4) or 1 (MXFP4) is
+// applied in the epilogue.  Persistent CTAs over 128 x 256 output tiles:
+//   warp 0       TMA producer: per k-stage of 64 elements, the X tile
+//                (128 rows x 128 B, 128-byte swizzle), the weight code tile
+//                (256 rows x 32 B) and the two scale atoms of its row bands;
+//   warp 1       TMEM owner (two 256-column accumulators) and MMA issuer:
+//                four 128 x 256 x 16 MMAs per k-stage;
+//   warps 2..9   converters: thread r dequantizes weight row r of the stage
+//                (64 codes) into the bf16 operand tile in the swizzled K-major
+//                layout the MMA descriptors describe;
+//   warps 10..13 epilogue: drain an accumulator (one warp per TMEM lane
+//                quarter, 256 columns in two halves), release it to the MMAs
+//                of the next-but-one tile, scale, convert and store Y.
+namespace w16 {
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int KS = 64;                   // k elements per stage
+constexpr int STAGES = 3;
+constexpr int A_STAGE = BM * 128;        // bf16 X tile
+constexpr int B_STAGE = BN * 128;        // bf16 dequantized weight tile
+constexpr int C_STAGE = BN * 32;         // weight codes
+constexpr int S_STAGE = 1024;            // two scale atoms
+constexpr int OFF_B = A_STAGE;
+constexpr int OFF_C = OFF_B + B_STAGE;
+constexpr int OFF_S = OFF_C + C_STAGE;
+constexpr int STAGE = OFF_S + S_STAGE;   // 57 KB, a multiple of 1024
+constexpr int OFF_EPI = STAGES * STAGE;
+constexpr int EPI_WARPS = 4;
+constexpr int EPI_BYTES = 8192;          // per epilogue warp: 32 rows x 128 bf16
+constexpr int OFF_BAR = OFF_EPI + EPI_WARPS * EPI_BYTES;
+constexpr int SMEM_BYTES = OFF_BAR + 512 + 1024;
+constexpr int CONV_WARPS = 8;
+constexpr int FIRST_CONV = 2;
+constexpr int FIRST_EPI = FIRST_CONV + CONV_WARPS;
+constexpr int THREADS = 32 * (FIRST_EPI + EPI_WARPS);
+constexpr uint32_t TMEM_COLS = 512;      // two accumulators
+}  // namespace w16
+
+// Instruction descriptor of tcgen05.mma kind::f16: fp32 D (bits 4-5 = 1),
+// bf16 A and B (bits 7-9 and 10-12 = 1), both K-major, N >> 3 at bit 17,
+// M >> 4 at bit 24.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
+        : "memory");
+}
+
+// Two E2M1 codes (one byte, element 0 low) times a block scale, as a packed
+// bf16 pair (exact: the product has at most 6 significant bits).
+__device__ __forceinline__ uint32_t dequant2_bf16(uint32_t byte, float2 s) {
+    const float2 v = mul2_rn(e2m1x2_value(byte), s);
+    uint32_t out;
+    asm("cvt.rn.bf16x2.f32 %0, %2, %1;" : "=r"(out) : "f"(v.x), "f"(v.y));
+    return out;
+}
+
+struct W16Dev {
+    int64_t M, N, K;
+    const uint8_t* w_scales;
+    const float* b_gscale;
+    void* y;
+    int64_t catoms;
+    int out_bf16;
+};
+
+template <bool MX>
+__global__ void __launch_bounds__(w16::THREADS, 1)
+    w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmC,
+                      const __grid_constant__ CUtensorMap tmY, W16Dev p) {
+    using namespace w16;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);    // [STAGES] X, codes, scales landed
+    uint64_t* conv = full + STAGES;                                  // [STAGES] weight tile converted
+    uint64_t* empty = conv + STAGES;                                 // [STAGES] its MMAs are done
+    uint64_t* tmem_full = empty + STAGES;                            // [2]
+    uint64_t* tmem_empty = tmem_full + 2;                            // [2]
+    uint64_t* mma_done = tmem_empty + 2;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&conv[s], CONV_WARPS);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) { mbar_init(&tmem_full[b], 1); mbar_init(&tmem_empty[b], EPI_WARPS); }
+        mbar_init(mma_done, 1);
+        fence_mbar_init();
+    }
+    if (warp == 1) { tmem_alloc(tmem_holder, TMEM_COLS); tmem_relinquish(); }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmX);
+        tma_prefetch_desc(&tmC);
+        if (p.out_bf16) tma_prefetch_desc(&tmY);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    const int64_t tiles_m = (p.M + BM - 1) / BM;
+    const int64_t tiles = tiles_m * ((p.N + BN - 1) / BN);
+    const int nks = (int)(p.K / KS);
+    const int64_t bands = (p.N + 127) / 128;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t last_phase[STAGES];
+            bool issued[STAGES];
+            for (int s = 0; s < STAGES; ++s) issued[s] = false, last_phase[s] = 0;
+            bool ok = true;
+            for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+                const int64_t mt = t % tiles_m, nt = t / tiles_m;
+                const int nb = (nt * 2 + 1 < bands) ? 2 : 1;
+                for (int ks = 0; ks < nks; ++ks) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
+                    uint8_t* st = smem + stage * STAGE;
+                    mbar_arrive_expect_tx(&full[stage], (uint32_t)(A_STAGE + C_STAGE + nb * 512));
+                    tma_load_2d(st, &tmX, &full[stage], ks * KS, (int32_t)(mt * BM));
+                    tma_load_2d(st + OFF_C, &tmC, &full[stage], ks * (KS / 2), (int32_t)(nt * BN));
+                    // scale atom column of this stage: 64 elements = 4 NVFP4 blocks = one
+                    // atom column; 2 MXFP4 blocks = half of one
+                    const int64_t acol = MX ? ks / 2 : ks;
+                    for (int b = 0; b < nb; ++b)
+                        bulk_load(st + OFF_S + b * 512, p.w_scales + ((nt * 2 + b) * p.catoms + acol) * 512, 512u,
+                                  &full[stage]);
+                    issued[stage] = true;
+                    last_phase[stage] = phase;
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                }
+            }
+            for (int s = 0; s < STAGES; ++s)
+                if (issued[s]) mbar_wait(&full[s], last_phase[s]);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16(BM, BN);
+            int stage = 0;
+            uint32_t phase = 0, iter = 0;
+            bool ok = true;
+            for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++iter) {
+                const uint32_t ab = iter & 1;
+                if (!mbar_wait(&tmem_empty[ab], ((iter >> 1) & 1) ^ 1)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t acc = tmem + ab * 256;
+                for (int ks = 0; ks < nks; ++ks) {
+                    if (!mbar_wait(&full[stage], phase) || !mbar_wait(&conv[stage], phase)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint64_t ad = smem_desc(smem_u32(smem + stage * STAGE), 16, 1024, 2);
+                    const uint64_t bd = smem_desc(smem_u32(smem + stage * STAGE + OFF_B), 16, 1024, 2);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16(acc, ad + 2 * kk, bd + 2 * kk, idesc, (ks > 0 || kk > 0) ? 1u : 0u);
+                    tc_commit(&empty[stage]);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+                tc_commit(&tmem_full[ab]);
+            }
+            tc_commit(mma_done);
+            mbar_wait(mma_done, 0);
+        }
+    } else if (warp < FIRST_EPI) {
+        // ---- converters: thread r owns weight row r of every stage
+        const int r = threadIdx.x - 32 * FIRST_CONV;
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+            const int64_t nt = t / tiles_m;
+            const bool row_ok = nt * BN + r < p.N;
+            for (int ks = 0; ks < nks; ++ks) {
+                if (!mbar_wait(&full[stage], phase)) { ok = false; break; }
+                uint8_t* st = smem + stage * STAGE;
+                const uint4 c0 = *reinterpret_cast<const uint4*>(st + OFF_C + r * 32);
+                const uint4 c1 = *reinterpret_cast<const uint4*>(st + OFF_C + r * 32 + 16);
+                // the row's 4 scale bytes of this atom column: byte j = scale column j
+                const uint32_t sw = *reinterpret_cast<const uint32_t*>(st + OFF_S + (r >> 7) * 512 + (r & 31) * 16 +
+                                                                       ((r >> 5) & 3) * 4);
+                float sv[4];
+                if (MX) {
+                    const int j0 = (ks & 1) * 2;
+                    sv[0] = sv[1] = exp2_int((int)((sw >> (8 * j0)) & 0xFFu) - 127);
+                    sv[2] = sv[3] = exp2_int((int)((sw >> (8 * (j0 + 1))) & 0xFFu) - 127);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) sv[j] = e4m3_value((sw >> (8 * j)) & 0xFFu);
+                }
+                const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+                uint8_t* brow = st + OFF_B + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {          // 16-byte chunk c: elements 8c .. 8c + 7
+                    const float s = sv[c >> 1];
+                    const float2 s2 = make_float2(s, s);
+                    uint4 o;
+                    o.x = dequant2_bf16(cw[c] & 0xFFu, s2);
+                    o.y = dequant2_bf16((cw[c] >> 8) & 0xFFu, s2);
+                    o.z = dequant2_bf16((cw[c] >> 16) & 0xFFu, s2);
+                    o.w = dequant2_bf16(cw[c] >> 24, s2);
+                    if (!row_ok) o = make_uint4(0u, 0u, 0u, 0u);
+                    *reinterpret_cast<uint4*>(brow + ((c ^ (r & 7)) << 4)) = o;
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&conv[stage]);
+                if (++stage == STAGES) { stage = 0; phase ^= 1; }
+            }
+        }
+    } else {
+        // ---- epilogue: one warp per TMEM lane quarter, 256 columns in two halves,
+        // each half through the warp's own 8 KB buffer and two TMA stores
+        const int e = warp - FIRST_EPI;
+        const int quad = warp & 3;
+        const float alpha = MX ? 1.0f : *p.b_gscale;
+        const bool out_bf16 = p.out_bf16 != 0;
+        uint8_t* buf = smem + OFF_EPI + e * EPI_BYTES;
+        uint32_t iter = 0;
+        for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++iter) {
+            const uint32_t ab = iter & 1;
+            if (!mbar_wait(&tmem_full[ab], (iter >> 1) & 1)) break;
+            tc_fence_after();
+            const int64_t mt = t % tiles_m, nt = t / tiles_m;
+            const int64_t row = mt * BM + quad * 32 + lane;
+            for (int half = 0; half < 2; ++half) {
+                const int64_t col_base = nt * BN + half * 128;
+                const uint32_t taddr = tmem + ab * 256 + ((uint32_t)(quad * 32) << 16) + half * 128;
+                uint32_t pk[2][32];
+#pragma unroll
+                for (int round = 0; round < 4; ++round) {
+                    uint32_t v[32];
+                    tmem_ld32(taddr + round * 32, v);
+                    tmem_ld_wait();
+                    if (half == 1 && round == 3) {
+                        // the accumulator is drained: the MMAs of tile t + 2 may use it
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&tmem_empty[ab]);
+                    }
+                    if (out_bf16) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(v[2 * j]) * alpha,
+                                                                     __uint_as_float(v[2 * j + 1]) * alpha);
+                            pk[round >> 1][(round & 1) * 16 + j] = *reinterpret_cast<uint32_t*>(&h);
+                        }
+                    } else if (row < p.M) {
+                        store_row32(p.y, p.N, row, col_base + round * 32, v, alpha, false);
+                    }
+                }
+                if (out_bf16) {
+                    // the previous stores from this buffer have finished reading it
+                    if (lane == 0) bulk_wait_read_all();
+                    __syncwarp();
+#pragma unroll
+                    for (int b = 0; b < 2; ++b)
+#pragma unroll
+                        for (int c = 0; c < 8; ++c)
+                            *reinterpret_cast<uint4*>(buf + b * 4096 + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                                make_uint4(pk[b][4 * c], pk[b][4 * c + 1], pk[b][4 * c + 2], pk[b][4 * c + 3]);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        const int32_t r0 = (int32_t)(mt * BM + quad * 32);
+                        tma_store_2d(&tmY, buf, (int32_t)col_base, r0);
+                        tma_store_2d(&tmY, buf + 4096, (int32_t)(col_base + 64), r0);
+                        bulk_commit_group();
+                    }
+                    __syncwarp();
+                }
+            }
+        }
+        if (lane == 0) bulk_wait_all();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
+}
+
+cudaError_t launch_w4a16(const W4A16Params& p, cudaStream_t st, int num_sms) {
+    using namespace w16;
+    if (p.M == 0 || p.N == 0) return cudaSuccess;
+    CUtensorMap mx, mc, my;
+    std::memset(&my, 0, sizeof(my));
+    if (!encode_map_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.x, (uint64_t)p.K, (uint64_t)p.M, (uint64_t)p.K * 2,
+                       64u, (uint32_t)BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_map_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.b_codes, (uint64_t)(p.K / 2), (uint64_t)p.N,
+                       (uint64_t)(p.K / 2), 32u, (uint32_t)BN, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    if (p.out_bf16 && !make_out_map(&my, p.y, p.M, p.N)) return cudaErrorInvalidValue;
+    W16Dev d;
+    d.M = p.M; d.N = p.N; d.K = p.K;
+    d.w_scales = p.b_scales; d.b_gscale = p.b_gscale; d.y = p.y;
+    d.catoms = ((p.K / (p.mxfp4 ? 32 : 16)) + 3) / 4;
+    d.out_bf16 = p.out_bf16 ? 1 : 0;
+    const int64_t tiles = ((p.M + BM - 1) / BM) * ((p.N + BN - 1) / BN);
+    const int grid = (int)(tiles < num_sms ? tiles : num_sms);
+    cudaError_t e;
+    if (p.mxfp4) {
+        e = cudaFuncSetAttribute(w4a16_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        w4a16_gemm_kernel<true><<<grid, THREADS, SMEM_BYTES, st>>>(mx, mc, my, d);
+    } else {
+        e = cudaFuncSetAttribute(w4a16_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        w4a16_gemm_kernel<false><<<grid, THREADS, SMEM_BYTES, st>>>(mx, mc, my, d);
+    }
+    return cudaGetLastError();
+}
+
 // ------------------------------------------------------------------ fused decode
 // Small-M GEMM (M <= 64) with the activation quantization inside the kernel:
 // no bf16 activation round trip and no workspace.  Operands are swapped so the

@@ -61,6 +61,18 @@ struct FusedDecodeParams {
     bool out_bf16;
 };
 
+struct W4A16Params {
+    int64_t M, N, K;
+    const void* x;            // [M, K] bf16 activations
+    const uint8_t* b_codes;   // [N, K/2]
+    const uint8_t* b_scales;  // tensor-core layout
+    const float* b_gscale;    // NVFP4 s_t or nullptr
+    void* y;                  // [M, N]
+    bool out_bf16;
+    bool mxfp4;
+};
+
+cudaError_t launch_w4a16(const W4A16Params& p, cudaStream_t st, int num_sms);
 cudaError_t launch_amax(const void* x, int64_t n, bool bf16, float denom, float* d_out,
                         cudaStream_t st, int num_sms);
 cudaError_t launch_quantize(const QuantParams& p, int blk, bool bf16, bool tc, bool ru, bool had,

@@ -184,3 +184,45 @@ def test_gemm_k_zero_and_empty():
     assert float(y.abs().max()) == 0.0
     q4.q4_gemm(q4.NVFP4, 0, 64, 64, a, B.scales, B.g_t, B.codes, B.scales, B.g_t, out_dtype=torch.float32)
     assert q4.q4_get_device_error() == 0
+
+
+@pytest.mark.parametrize("fmt", [q4.NVFP4, q4.MXFP4])
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("mnk", [(128, 256, 64), (200, 392, 320), (300, 136, 1088), (64, 512, 192)])
+def test_w4a16_gemm_parity(fmt, out_dtype, mnk):
+    """a_kind = A_BF16_W4A16: bf16 activations times the weight dequantized to
+    bf16 on the fly; ragged M, partial weight tiles and bands, odd k-stage counts."""
+    M, N, K = mnk
+    x = synth.to_bf16(synth.small_like("heavy", M + K, M, K))
+    x32 = synth.bf16_to_f32(x)
+    B = Operand(fmt, synth.small_like("weight", N + 7, N, K), denom=1536.0)
+    y = q4.q4_gemm(fmt, M, N, K, dev(x), None, None, B.codes, B.scales, B.g_t, out_dtype=out_dtype,
+                   a_kind=q4.A_BF16_W4A16)
+    ref = oracle.gemm_w4a16(fmt, x32, B.o_codes, B.o_scales, B.s_t, M, N, K)
+    check(y, ref, out_dtype)
+
+
+def test_w4a16_looped_core_full_size_sampled_rows():
+    """Looped-core shape: X 4096 x 1024 bf16 times a 4096 x 1024 weight whose codes
+    come from three Sigma-Delta visits (RU scales, s_t = max|W| / 1536); the
+    oracle follows 96 sampled rows of Y with its own Sigma-Delta codes."""
+    d = synth.looped()
+    w = d["w"][-1]
+    N, K = w.shape
+    M = d["x"].shape[0]
+    x32 = synth.bf16_to_f32(d["x"])
+    s_t = oracle.tensor_scale(oracle.amax(w), 1536.0)
+    g_t = gscale_dev(s_t)
+    _, g_sc = q4.q4_quantize(q4.NVFP4, dev(w), gscale=g_t, flags=q4.SCALE_RU | q4.LAYOUT_TC)
+    _, o_sc = oracle.nvfp4_quantize(w, s_t, round_up=True)
+    r_gpu = torch.zeros((N, K), dtype=torch.float32, device=DEV)
+    r_orc = np.zeros((N, K), np.float32)
+    w_d = dev(w)
+    for _ in range(3):
+        g_codes = q4.q4_sigma_delta_step(q4.NVFP4, w_d, g_sc, r_gpu, gscale=g_t)
+        o_codes = oracle.sigma_delta_step(q4.NVFP4, w, o_sc, s_t, r_orc)
+    y = q4.q4_gemm(q4.NVFP4, M, N, K, dev(d["x"]), None, None, g_codes, g_sc, g_t, out_dtype=torch.float32,
+                   a_kind=q4.A_BF16_W4A16)
+    rows = np.sort(np.random.default_rng(1).choice(M, 96, replace=False))
+    ref = oracle.gemm_w4a16(q4.NVFP4, x32, o_codes, o_sc, s_t, M, N, K, rows=rows)
+    assert rel_fro(host(y)[rows], ref) <= GEMM_F32_TOL
