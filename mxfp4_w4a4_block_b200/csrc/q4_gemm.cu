@@ -832,12 +832,14 @@ cudaError_t launch_gemm(const GemmParams& p, cudaStream_t st, int num_sms) {
 // applied in the epilogue.  Persistent CTAs over 128 x 256 output tiles:
 //   warp 0       TMA producer: per k-stage of 64 elements, the X tile
 //                (128 rows x 128 B, 128-byte swizzle), the weight code tile
-//                (256 rows x 32 B) and the two scale atoms of its row bands;
+//                (256 rows x 32 B) and the two scale atoms of its row bands,
+//                into a 5-deep ring (a stage is free once the converters have
+//                read its codes and the MMAs its X tile);
 //   warp 1       TMEM owner (two 256-column accumulators) and MMA issuer:
 //                four 128 x 256 x 16 MMAs per k-stage;
 //   warps 2..9   converters: thread r dequantizes weight row r of the stage
-//                (64 codes) into the bf16 operand tile in the swizzled K-major
-//                layout the MMA descriptors describe;
+//                (64 codes) into one of two bf16 operand tiles, in the
+//                swizzled K-major layout the MMA descriptors describe;
 //   warps 10..13 epilogue: drain an accumulator (one warp per TMEM lane
 //                quarter, 256 columns in two halves), release it to the MMAs
 //                of the next-but-one tile, scale, convert and store Y.
@@ -845,16 +847,17 @@ namespace w16 {
 constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int KS = 64;                   // k elements per stage
-constexpr int STAGES = 3;
+constexpr int STAGES = 5;                // TMA ring: X tile, weight codes, scale atoms
 constexpr int A_STAGE = BM * 128;        // bf16 X tile
-constexpr int B_STAGE = BN * 128;        // bf16 dequantized weight tile
 constexpr int C_STAGE = BN * 32;         // weight codes
 constexpr int S_STAGE = 1024;            // two scale atoms
-constexpr int OFF_B = A_STAGE;
-constexpr int OFF_C = OFF_B + B_STAGE;
+constexpr int OFF_C = A_STAGE;
 constexpr int OFF_S = OFF_C + C_STAGE;
-constexpr int STAGE = OFF_S + S_STAGE;   // 57 KB, a multiple of 1024
-constexpr int OFF_EPI = STAGES * STAGE;
+constexpr int STAGE = OFF_S + S_STAGE;   // 25 KB, a multiple of 1024
+constexpr int BSLOTS = 2;                // converted bf16 weight tiles
+constexpr int B_SLOT = BN * 128;
+constexpr int OFF_B = STAGES * STAGE;
+constexpr int OFF_EPI = OFF_B + BSLOTS * B_SLOT;
 constexpr int EPI_WARPS = 4;
 constexpr int EPI_BYTES = 8192;          // per epilogue warp: 32 rows x 128 bf16
 constexpr int OFF_BAR = OFF_EPI + EPI_WARPS * EPI_BYTES;
@@ -882,13 +885,47 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64
         : "memory");
 }
 
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+// Eight E2M1 codes (element 0 in the low nibble) -> four packed bf16 pairs of
+// their values (element 2i in the low half of word i) with byte permutes
+// only, no conversion instructions (those run on a narrow pipe): the low and
+// high bytes of the bf16 patterns of the 8 magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6
+// are two 8-byte tables indexed by the code's low three bits, and each sign bit
+// is moved to bit 15 / 31 by a sign-replicating permute.
+__device__ __forceinline__ void e2m1x8_to_bf16(uint32_t w, uint32_t (&o)[4]) {
+    constexpr uint32_t LO0 = 0xC0800000u, LO1 = 0xC0804000u;   // low bytes: 0 0 80 C0 | 0 40 80 C0
+    constexpr uint32_t HI0 = 0x3F3F3F00u, HI1 = 0x40404040u;   // high bytes: 0 3F 3F 3F | 40 40 40 40
+    const uint32_t sel = w & 0x77777777u;
+    const uint32_t lo_a = prmt(LO0, LO1, sel), hi_a = prmt(HI0, HI1, sel);
+    const uint32_t lo_b = prmt(LO0, LO1, sel >> 16), hi_b = prmt(HI0, HI1, sel >> 16);
+    const uint32_t sg = w & 0x88888888u, sg4 = sg << 4;
+    o[0] = prmt(lo_a, hi_a, 0x5140u) | (prmt(sg4, sg, 0xC080u) & 0x80008000u);
+    o[1] = prmt(lo_a, hi_a, 0x7362u) | (prmt(sg4, sg, 0xD090u) & 0x80008000u);
+    o[2] = prmt(lo_b, hi_b, 0x5140u) | (prmt(sg4, sg, 0xE0A0u) & 0x80008000u);
+    o[3] = prmt(lo_b, hi_b, 0x7362u) | (prmt(sg4, sg, 0xF0B0u) & 0x80008000u);
+}
+
 // Two E2M1 codes (one byte, element 0 low) times a block scale, as a packed
-// bf16 pair (exact: the product has at most 6 significant bits).
+// bf16 pair, through the hardware E2M1 -> f16 conversion (the conversion
+// pipe; the byte-permute form above uses the integer pipe).
 __device__ __forceinline__ uint32_t dequant2_bf16(uint32_t byte, float2 s) {
     const float2 v = mul2_rn(e2m1x2_value(byte), s);
     uint32_t out;
     asm("cvt.rn.bf16x2.f32 %0, %2, %1;" : "=r"(out) : "f"(v.x), "f"(v.y));
     return out;
+}
+
+// a * b on packed bf16 pairs (exact here: code value times a block scale has
+// at most 6 significant bits).
+__device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
 }
 
 struct W16Dev {
@@ -908,9 +945,10 @@ __global__ void __launch_bounds__(w16::THREADS, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);    // [STAGES] X, codes, scales landed
-    uint64_t* conv = full + STAGES;                                  // [STAGES] weight tile converted
-    uint64_t* empty = conv + STAGES;                                 // [STAGES] its MMAs are done
-    uint64_t* tmem_full = empty + STAGES;                            // [2]
+    uint64_t* empty = full + STAGES;                                 // [STAGES] converters read it, MMAs done
+    uint64_t* b_full = empty + STAGES;                               // [BSLOTS] weight tile converted
+    uint64_t* b_empty = b_full + BSLOTS;                             // [BSLOTS] its MMAs are done
+    uint64_t* tmem_full = b_empty + BSLOTS;                          // [2]
     uint64_t* tmem_empty = tmem_full + 2;                            // [2]
     uint64_t* mma_done = tmem_empty + 2;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
@@ -919,9 +957,9 @@ __global__ void __launch_bounds__(w16::THREADS, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&conv[s], CONV_WARPS);
-            mbar_init(&empty[s], 1);
+            mbar_init(&empty[s], CONV_WARPS + 1);        // every converter warp + the MMA commit
         }
+        for (int b = 0; b < BSLOTS; ++b) { mbar_init(&b_full[b], CONV_WARPS); mbar_init(&b_empty[b], 1); }
         for (int b = 0; b < 2; ++b) { mbar_init(&tmem_full[b], 1); mbar_init(&tmem_empty[b], EPI_WARPS); }
         mbar_init(mma_done, 1);
         fence_mbar_init();
@@ -976,8 +1014,8 @@ __global__ void __launch_bounds__(w16::THREADS, 1)
     } else if (warp == 1) {
         if (lane == 0) {
             const uint32_t idesc = idesc_bf16(BM, BN);
-            int stage = 0;
-            uint32_t phase = 0, iter = 0;
+            int stage = 0, bs = 0;
+            uint32_t phase = 0, bphase = 0, iter = 0;
             bool ok = true;
             for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++iter) {
                 const uint32_t ab = iter & 1;
@@ -985,15 +1023,17 @@ __global__ void __launch_bounds__(w16::THREADS, 1)
                 tc_fence_after();
                 const uint32_t acc = tmem + ab * 256;
                 for (int ks = 0; ks < nks; ++ks) {
-                    if (!mbar_wait(&full[stage], phase) || !mbar_wait(&conv[stage], phase)) { ok = false; break; }
+                    if (!mbar_wait(&full[stage], phase) || !mbar_wait(&b_full[bs], bphase)) { ok = false; break; }
                     tc_fence_after();
                     const uint64_t ad = smem_desc(smem_u32(smem + stage * STAGE), 16, 1024, 2);
-                    const uint64_t bd = smem_desc(smem_u32(smem + stage * STAGE + OFF_B), 16, 1024, 2);
+                    const uint64_t bd = smem_desc(smem_u32(smem + OFF_B + bs * B_SLOT), 16, 1024, 2);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         mma_bf16(acc, ad + 2 * kk, bd + 2 * kk, idesc, (ks > 0 || kk > 0) ? 1u : 0u);
                     tc_commit(&empty[stage]);
+                    tc_commit(&b_empty[bs]);
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                    if (++bs == BSLOTS) { bs = 0; bphase ^= 1; }
                 }
                 if (!ok) break;
                 tc_commit(&tmem_full[ab]);
@@ -1004,47 +1044,66 @@ __global__ void __launch_bounds__(w16::THREADS, 1)
     } else if (warp < FIRST_EPI) {
         // ---- converters: thread r owns weight row r of every stage
         const int r = threadIdx.x - 32 * FIRST_CONV;
-        int stage = 0;
-        uint32_t phase = 0;
+        int stage = 0, bs = 0;
+        uint32_t phase = 0, bphase = 0;
         bool ok = true;
         for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
             const int64_t nt = t / tiles_m;
             const bool row_ok = nt * BN + r < p.N;
             for (int ks = 0; ks < nks; ++ks) {
-                if (!mbar_wait(&full[stage], phase)) { ok = false; break; }
+                if (!mbar_wait(&full[stage], phase) || !mbar_wait(&b_empty[bs], bphase ^ 1)) { ok = false; break; }
                 uint8_t* st = smem + stage * STAGE;
                 const uint4 c0 = *reinterpret_cast<const uint4*>(st + OFF_C + r * 32);
                 const uint4 c1 = *reinterpret_cast<const uint4*>(st + OFF_C + r * 32 + 16);
                 // the row's 4 scale bytes of this atom column: byte j = scale column j
                 const uint32_t sw = *reinterpret_cast<const uint32_t*>(st + OFF_S + (r >> 7) * 512 + (r & 31) * 16 +
                                                                        ((r >> 5) & 3) * 4);
-                float sv[4];
+                // block scales as packed bf16 pairs (exact: E4M3 has 4 significant
+                // bits, E8M0 is a power of two): sp[j] for elements 16j .. 16j + 15
+                uint32_t sp[4];
                 if (MX) {
                     const int j0 = (ks & 1) * 2;
-                    sv[0] = sv[1] = exp2_int((int)((sw >> (8 * j0)) & 0xFFu) - 127);
-                    sv[2] = sv[3] = exp2_int((int)((sw >> (8 * (j0 + 1))) & 0xFFu) - 127);
+                    const uint32_t a = __float_as_uint(exp2_int((int)((sw >> (8 * j0)) & 0xFFu) - 127)) >> 16;
+                    const uint32_t b = __float_as_uint(exp2_int((int)((sw >> (8 * (j0 + 1))) & 0xFFu) - 127)) >> 16;
+                    sp[0] = sp[1] = a | (a << 16);
+                    sp[2] = sp[3] = b | (b << 16);
                 } else {
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) sv[j] = e4m3_value((sw >> (8 * j)) & 0xFFu);
+                    for (int j = 0; j < 4; ++j) {
+                        const uint32_t h = __float_as_uint(e4m3_value((sw >> (8 * j)) & 0xFFu)) >> 16;
+                        sp[j] = h | (h << 16);
+                    }
                 }
                 const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-                uint8_t* brow = st + OFF_B + (r >> 3) * 1024 + (r & 7) * 128;
+                // the codes and scales are in registers: the stage may be refilled
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[stage]);
+                uint8_t* brow = smem + OFF_B + bs * B_SLOT + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {          // 16-byte chunk c: elements 8c .. 8c + 7
-                    const float s = sv[c >> 1];
-                    const float2 s2 = make_float2(s, s);
-                    uint4 o;
-                    o.x = dequant2_bf16(cw[c] & 0xFFu, s2);
-                    o.y = dequant2_bf16((cw[c] >> 8) & 0xFFu, s2);
-                    o.z = dequant2_bf16((cw[c] >> 16) & 0xFFu, s2);
-                    o.w = dequant2_bf16(cw[c] >> 24, s2);
-                    if (!row_ok) o = make_uint4(0u, 0u, 0u, 0u);
-                    *reinterpret_cast<uint4*>(brow + ((c ^ (r & 7)) << 4)) = o;
+                    const uint32_t sc = sp[c >> 1];
+                    uint4 v;
+                    if (c & 1) {
+                        // odd chunks through the conversion pipe, even ones through the
+                        // integer pipe: neither pipe alone sets the pace
+                        const float f = __uint_as_float(sc << 16);
+                        const float2 f2 = make_float2(f, f);
+                        v = make_uint4(dequant2_bf16(cw[c] & 0xFFu, f2), dequant2_bf16((cw[c] >> 8) & 0xFFu, f2),
+                                       dequant2_bf16((cw[c] >> 16) & 0xFFu, f2), dequant2_bf16(cw[c] >> 24, f2));
+                    } else {
+                        uint32_t o[4];
+                        e2m1x8_to_bf16(cw[c], o);
+                        v = make_uint4(mul_bf16x2(o[0], sc), mul_bf16x2(o[1], sc), mul_bf16x2(o[2], sc),
+                                       mul_bf16x2(o[3], sc));
+                    }
+                    if (!row_ok) v = make_uint4(0u, 0u, 0u, 0u);
+                    *reinterpret_cast<uint4*>(brow + ((c ^ (r & 7)) << 4)) = v;
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&conv[stage]);
+                if (lane == 0) mbar_arrive(&b_full[bs]);
                 if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                if (++bs == BSLOTS) { bs = 0; bphase ^= 1; }
             }
         }
     } else {
@@ -1065,7 +1124,11 @@ __global__ void __launch_bounds__(w16::THREADS, 1)
             for (int half = 0; half < 2; ++half) {
                 const int64_t col_base = nt * BN + half * 128;
                 const uint32_t taddr = tmem + ab * 256 + ((uint32_t)(quad * 32) << 16) + half * 128;
-                uint32_t pk[2][32];
+                if (out_bf16) {
+                    // the previous stores from this buffer have finished reading it
+                    if (lane == 0) bulk_wait_read_all();
+                    __syncwarp();
+                }
 #pragma unroll
                 for (int round = 0; round < 4; ++round) {
                     uint32_t v[32];
@@ -1078,26 +1141,26 @@ __global__ void __launch_bounds__(w16::THREADS, 1)
                         if (lane == 0) mbar_arrive(&tmem_empty[ab]);
                     }
                     if (out_bf16) {
+                        // columns 32*round .. +31 of this half: 16-byte chunks 4*(round&1) .. +3
+                        // of the 32 x 64 box round / 2, 128-byte swizzled
+                        uint32_t pk[16];
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
                             __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(v[2 * j]) * alpha,
                                                                      __uint_as_float(v[2 * j + 1]) * alpha);
-                            pk[round >> 1][(round & 1) * 16 + j] = *reinterpret_cast<uint32_t*>(&h);
+                            pk[j] = *reinterpret_cast<uint32_t*>(&h);
+                        }
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const int c = (round & 1) * 4 + q;
+                            *reinterpret_cast<uint4*>(buf + (round >> 1) * 4096 + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                                make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
                         }
                     } else if (row < p.M) {
                         store_row32(p.y, p.N, row, col_base + round * 32, v, alpha, false);
                     }
                 }
                 if (out_bf16) {
-                    // the previous stores from this buffer have finished reading it
-                    if (lane == 0) bulk_wait_read_all();
-                    __syncwarp();
-#pragma unroll
-                    for (int b = 0; b < 2; ++b)
-#pragma unroll
-                        for (int c = 0; c < 8; ++c)
-                            *reinterpret_cast<uint4*>(buf + b * 4096 + lane * 128 + ((c ^ (lane & 7)) << 4)) =
-                                make_uint4(pk[b][4 * c], pk[b][4 * c + 1], pk[b][4 * c + 2], pk[b][4 * c + 3]);
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) {
