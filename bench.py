@@ -46,6 +46,7 @@ WORKLOAD = ("prefill NVFP4 W4A4 linear: X 8192x5120 bf16 (0.02*Student-t(3), 20%
             "-> amax -> NVFP4 quantize -> GEMM with W 5120x5120 and 17408x5120 (N(0,0.02^2), pre-quantized), "
             "bf16 out")
 # algorithmic bytes per element (see the design notes)
+B_W4A16_GEMM_NOTE = "2*M*N*K FLOP on the bf16 tensor pipe"
 B_QUANT_BF16 = 2 + 0.5 + 1 / 16          # read bf16, write codes + E4M3 scale
 B_AMAX_BF16 = 2
 B_SIGMA_DELTA = 4 + 4 + 4 + 0.5 + 1 / 16  # w, r in, r out, codes, scale
@@ -61,6 +62,12 @@ def peaks():
                 "src": "measured"}
     return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sus": 1400.0, "src": "fallback"}
 
+
+# dram__bytes_read.sum + dram__bytes_write.sum of one launch of the roofline
+# kernel (gemm_kernel<NVFP4>, 8192 x 17408 x 5120) from the ncu capture
+# summarised in profiles/gemm_kernel_nvfp4_8192x17408x5120.md; to be re-taken
+# (or set to None) whenever that kernel changes
+GEMM_TRAFFIC_BYTES = 321.1e6
 
 # dense FP4 over dense bf16 on B200, nominal (9 / 2.25 PFLOP/s)
 FP4_OVER_BF16 = 4.0
@@ -217,25 +224,45 @@ def rows_bench(q4, dev, flush, pk, reps=30):
                          "online_transform_overhead": ms_q / ms_g}
     del xm, t, inv_t, wc, ws, xc, xs, ym
 
-    # a4: one Sigma-Delta visit over the 13 looped-core weights
+    # a4 + a7: one looped-core visit -- a Sigma-Delta requant of the 13 weights
+    # (41,943,040 weights) and the W4A16 GEMM of X (4096 x 1024 bf16) with each
     dl = synth.looped()
+    xl = dl["x"].to(dev)
+    Ml, Kl = xl.shape
     mats = []
     for w in dl["w"]:
         wt = torch.from_numpy(w).to(dev)
         g = q4.q4_amax(wt, 1536.0)
         _, sc = q4.q4_quantize(q4.NVFP4, wt, gscale=g[1:2], flags=q4.SCALE_RU | q4.LAYOUT_TC)
         mats.append((wt, sc, g[1:2].clone(), torch.zeros_like(wt),
-                     torch.empty((w.shape[0], w.shape[1] // 2), dtype=torch.uint8, device=dev)))
+                     torch.empty((w.shape[0], w.shape[1] // 2), dtype=torch.uint8, device=dev),
+                     torch.empty((Ml, w.shape[0]), dtype=torch.bfloat16, device=dev)))
     nw = sum(w.size for w in dl["w"])
+    w16_flops = sum(2.0 * Ml * w.shape[0] * Kl for w in dl["w"])
+
+    def sd_visit():
+        for wt, sc, g, r, c, _ in mats:
+            q4.q4_sigma_delta_step(q4.NVFP4, wt, sc, r, gscale=g, codes=c)
+
+    def w16_visit():
+        for wt, sc, g, r, c, y in mats:
+            q4.q4_gemm(q4.NVFP4, Ml, wt.shape[0], Kl, xl, None, None, c, sc, g, y=y, a_kind=q4.A_BF16_W4A16)
 
     def visit():
-        for wt, sc, g, r, c in mats:
-            q4.q4_sigma_delta_step(q4.NVFP4, wt, sc, r, gscale=g, codes=c)
-    ms_sd, _ = time_fn(visit, reps, flush)
+        sd_visit()
+        w16_visit()
+    ms_sd, _ = time_fn(sd_visit, reps, flush)
     gbs = nw * B_SIGMA_DELTA / (ms_sd * 1e-3) / 1e9
     out["sigma_delta_visit"] = {"weights": nw, "matrices": 13, "us": ms_sd * 1e3, "GB/s": gbs, "frac_hbm": gbs / hbm,
                                 "us_R32": ms_sd * 1e3 * 32}
-    del mats
+    ms_w, _ = time_fn(w16_visit, reps, flush)
+    tf = w16_flops / (ms_w * 1e-3) / 1e12
+    out["w4a16_visit"] = {"gemms": 13, "M": Ml, "K": Kl, "us": ms_w * 1e3, "TFLOP/s": tf,
+                          "frac_bf16": tf / pk["bf16"]}
+    ms_v, _ = time_fn(visit, max(5, reps // 3), flush)
+    out["looped_visit"] = {"us": ms_v * 1e3, "us_R32": ms_v * 1e3 * 32,
+                           "note": "Sigma-Delta requant of all 13 weights + 13 W4A16 GEMMs"}
+    del mats, xl
 
     # a6: decode-shaped GEMM with fused activation quantize
     dd = synth.decode()
@@ -276,9 +303,13 @@ def run_ours(args):
     hbm = pk["hbm_gbs"]
     fp4_burst = pk["bf16"] * FP4_OVER_BF16
     flush_buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    flush_rd = torch.ones(64 * 1024 * 1024, dtype=torch.float32, device=dev)
 
     def flush():
+        # write 256 MiB (evicts everything), then read another 256 MiB so that the
+        # L2 holds no dirty lines whose write-back the next kernel would pay for
         flush_buf.fill_(1)
+        flush_rd.sum()
 
     P = Prefill(q4, dev)
     for _ in range(max(args.warmup, 3)):
@@ -344,11 +375,18 @@ def run_ours(args):
 
     rows = None
     if not args.no_rows:
+        # the prefill activation quantize alone after a cold, clean L2
+        xq_ms, _ = time_fn(lambda: q4.q4_quantize(q4.NVFP4, P.x, gscale=P.amax[1:2], codes=P.xc, scales=P.xs), 30,
+                           flush)
+        xq_gbs = M * K * B_QUANT_BF16 / (xq_ms * 1e-3) / 1e9
+        iso_quant = {"shape": [M, K], "us": xq_ms * 1e3, "GB/s": xq_gbs, "frac_hbm": xq_gbs / hbm}
         del P
         torch.cuda.empty_cache()
         rows = rows_bench(q4, dev, flush, pk)
         rows["nvfp4_quantize_prefill_x"] = {"shape": [M, K], "us": k_ms[1] * 1e3, "GB/s": q_gbs,
-                                            "frac_hbm": q_gbs / hbm}
+                                            "frac_hbm": q_gbs / hbm,
+                                            "note": "inside the step, right after amax (X partly in L2)"}
+        rows["nvfp4_quantize_prefill_x_cold"] = iso_quant
         rows["amax_prefill_x"] = {"us": k_ms[0] * 1e3, "GB/s": a_gbs, "frac_hbm": a_gbs / hbm}
         rows["gemm_prefill_n5120"] = {"us": k_ms[2] * 1e3, "TFLOP/s": gemm1_tf, "frac_fp4": gemm1_tf / fp4_burst}
         rows["gemm_prefill_n17408"] = {"us": k_ms[3] * 1e3, "TFLOP/s": gemm2_tf, "frac_fp4": gemm2_tf / fp4_burst}
@@ -360,7 +398,7 @@ def run_ours(args):
         "warmup": max(args.warmup, 3), "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "e2m1 x e2m1 -> f32 (NVFP4 block-scaled)", "data": "synthetic",
         "config": {"workload": WORKLOAD, "M": M, "K": K, "N": [N1, N2], "quantize_GB/s": q_gbs,
-                   "quantize_frac_hbm": q_gbs / hbm, "l2": "flushed (256 MiB write) before every timed step",
+                   "quantize_frac_hbm": q_gbs / hbm, "l2": "flushed before every timed step: 256 MiB write, then a 256 MiB read (cold, clean L2)",
                    "parallelism": f"replicas x{world} (independent problems per GPU)"},
         "roofline": {"kernel": "gemm_kernel<NVFP4> 8192x17408x5120", "bound": "tensor", "achieved": gemm2_tf,
                      "peak": fp4_burst, "unit": "TFLOP/s", "frac": gemm2_tf / fp4_burst,
@@ -483,7 +521,7 @@ def main():
     ap.add_argument("--no-rows", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--traffic", type=float, default=None,
+    ap.add_argument("--traffic", type=float, default=GEMM_TRAFFIC_BYTES,
                     help="DRAM bytes per launch of the roofline kernel from an ncu capture")
     args = ap.parse_args()
     if args.impl == "reference":
