@@ -64,9 +64,9 @@ def peaks():
 
 
 # dram__bytes_read.sum + dram__bytes_write.sum of one launch of the roofline
-# kernel (gemm_kernel<NVFP4>, 8192 x 17408 x 5120) from the ncu capture
-# summarised in profiles/gemm_kernel_nvfp4_8192x17408x5120.md; to be re-taken
-# (or set to None) whenever that kernel changes
+# kernel (gemm_kernel<NVFP4>, 8192 x 17408 x 5120) from one ncu capture of
+# the bench's own prefill step; to be re-taken (or set to None) whenever that
+# kernel changes
 GEMM_TRAFFIC_BYTES = 321.1e6
 
 # dense FP4 over dense bf16 on B200, nominal (9 / 2.25 PFLOP/s)
