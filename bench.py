@@ -259,6 +259,18 @@ def rows_bench(q4, dev, flush, pk, reps=30):
     tf = w16_flops / (ms_w * 1e-3) / 1e12
     out["w4a16_visit"] = {"gemms": 13, "M": Ml, "K": Kl, "us": ms_w * 1e3, "TFLOP/s": tf,
                           "frac_bf16": tf / pk["bf16"]}
+    banks = [torch.empty((32, wt.shape[0], wt.shape[1] // 2), dtype=torch.uint8, device=dev)
+             for wt, *_ in mats]
+
+    def codebanks():
+        for (wt, sc, g, r, c, _), bk in zip(mats, banks):
+            q4.q4_sigma_delta_codebanks(q4.NVFP4, wt, sc, 32, gscale=g, codes=bk)
+    ms_cb, _ = time_fn(codebanks, max(5, reps // 3), flush)
+    gbs = nw * (4 + 32 * 0.5) / (ms_cb * 1e-3) / 1e9
+    out["sigma_delta_codebanks_K32"] = {"weights": nw, "visits": 32, "us": ms_cb * 1e3, "GB/s": gbs,
+                                        "frac_hbm": gbs / hbm, "B_per_weight": 4 + 32 * 0.5,
+                                        "vs_32_separate_visits": ms_sd * 32 / ms_cb}
+    del banks
     ms_v, _ = time_fn(visit, max(5, reps // 3), flush)
     out["looped_visit"] = {"us": ms_v * 1e3, "us_R32": ms_v * 1e3 * 32,
                            "note": "Sigma-Delta requant of all 13 weights + 13 W4A16 GEMMs"}
@@ -280,7 +292,13 @@ def rows_bench(q4, dev, flush, pk, reps=30):
     gbs = byts / (ms_d * 1e-3) / 1e9
     out["decode_fused_gemm"] = {"mnk": [Md, Nd, Kd], "us": ms_d * 1e3, "GB/s": gbs, "frac_hbm": gbs / hbm,
                                 "TFLOP/s": 2.0 * Md * Nd * Kd / (ms_d * 1e-3) / 1e12}
-    del xd, wc, ws, yd
+    # a8: dequantize (fake quant) of the decode weight, 17408 x 5120 -> bf16
+    dq = torch.empty((Nd, Kd), dtype=torch.bfloat16, device=dev)
+    ms_dq, _ = time_fn(lambda: q4.q4_dequantize(q4.NVFP4, wc, ws, Nd, Kd, gscale=gw, out_dtype=torch.bfloat16, out=dq),
+                       reps, flush)
+    gbs = Nd * Kd * B_DEQUANT_BF16 / (ms_dq * 1e-3) / 1e9
+    out["dequantize_bf16"] = {"shape": [Nd, Kd], "us": ms_dq * 1e3, "GB/s": gbs, "frac_hbm": gbs / hbm}
+    del xd, wc, ws, yd, dq
     torch.cuda.empty_cache()
     return out
 

@@ -175,6 +175,26 @@ Q4_API q4_status q4_sigma_delta_step(q4_format format, int block, const float* w
                               int flags, void* stream);
 
 /*
+ * q4_sigma_delta_codebanks -- the whole Sigma-Delta chain of `visits` loop
+ *   visits from r_0 = 0 in one pass, stored as codebanks ("Looped Transformer
+ *   quantization", sec. 2.3: for frozen-weight inference the last K visits
+ *   restart a chain of length K and use its codes in reverse order, tail visit
+ *   j taking the code of chain step K - j + 1; sec. 4: those K codes are
+ *   pre-generated as K codebanks, one bank read per visit).
+ *   Same arithmetic as `visits` calls of q4_sigma_delta_step on a zeroed
+ *   residue, but w and its scales are read once and the residue stays in
+ *   registers.  codes: device [visits, rows, cols/2]; bank k (0-based) holds
+ *   the codes of chain step k + 1, so tail visit j (1-based) of the reverse
+ *   schedule reads bank visits - j.  residue_out: NULL, or device float
+ *   [rows, cols] receiving r_visits.  visits in 1..4096.  Other arguments as
+ *   q4_sigma_delta_step.
+ */
+Q4_API q4_status q4_sigma_delta_codebanks(q4_format format, int block, const float* w,
+                                   int64_t rows, int64_t cols, const uint8_t* scales,
+                                   const float* d_gscale, int visits, uint8_t* codes,
+                                   float* residue_out, int flags, void* stream);
+
+/*
  * q4_gemm -- block-scaled FP4 GEMM  Y = alpha * dec(A) dec(B)^T  on the
  *   tcgen05 tensor cores ("Why Gated DeltaNet Survives 4-Bit Quantization",
  *   prerequisites: W4A4 runs the GEMM on native 4-bit tensor cores; "MACaQ",

@@ -9,8 +9,9 @@ there is no CPU fallback, and importing fails loudly if the library has not
 been built (``python -m mxfp4_w4a4_block_b200.build``).
 
 Function names mirror the C entry points: q4_amax, q4_quantize,
-q4_dequantize, q4_sigma_delta_step, q4_gemm, q4_gemm_workspace_size,
-q4_get_device_error, q4_scale_bytes.
+q4_dequantize, q4_sigma_delta_step, q4_sigma_delta_codebanks, q4_gemm,
+q4_gemm_workspace_size, q4_get_device_error, q4_scale_bytes (tail_bank is a
+pure indexing helper of the reverse-order codebank schedule).
 """
 from __future__ import annotations
 
@@ -54,6 +55,7 @@ SIGNATURES = {
     "q4_quantize": (_I, [_I, _I, _I, _P, _I64, _I64, _I64, _P, _P, _P, _P, _I, _P]),
     "q4_dequantize": (_I, [_I, _I, _P, _P, _P, _I64, _I64, _I, _I, _P, _P]),
     "q4_sigma_delta_step": (_I, [_I, _I, _P, _I64, _I64, _P, _P, _P, _P, _I, _P]),
+    "q4_sigma_delta_codebanks": (_I, [_I, _I, _P, _I64, _I64, _P, _P, _I, _P, _P, _I, _P]),
     "q4_gemm": (_I, [_I, _I, _I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _P, _I, _P, _P, _SZ, _P]),
     "q4_gemm_workspace_size": (_SZ, [_I, _I64, _I64, _I64, _I]),
     "q4_get_device_error": (_I, [_P]),
@@ -177,6 +179,30 @@ def q4_sigma_delta_step(fmt: int, w: torch.Tensor, scales: torch.Tensor, residue
                                    _ptr(residue), _ptr(codes), flags, _stream(stream))
     _check("q4_sigma_delta_step", st)
     return codes
+
+
+def q4_sigma_delta_codebanks(fmt: int, w: torch.Tensor, scales: torch.Tensor, visits: int,
+                             gscale: torch.Tensor | None = None, flags: int = LAYOUT_TC,
+                             codes: torch.Tensor | None = None, residue_out: torch.Tensor | None = None,
+                             stream=None) -> torch.Tensor:
+    """The Sigma-Delta chain of `visits` steps from a zero residue in one pass;
+    returns the codebanks [visits, rows, cols/2] (bank k = chain step k + 1)."""
+    rows, cols = w.shape
+    if codes is None:
+        codes = torch.empty((visits, rows, cols // 2), dtype=torch.uint8, device=w.device)
+    st = lib().q4_sigma_delta_codebanks(fmt, BLOCK[fmt], _ptr(w), rows, cols, _ptr(scales), _ptr(gscale), visits,
+                                        _ptr(codes), _ptr(residue_out), flags, _stream(stream))
+    _check("q4_sigma_delta_codebanks", st)
+    return codes
+
+
+def tail_bank(banks: torch.Tensor, j: int) -> torch.Tensor:
+    """The codes of tail visit j (1-based) in the reverse-order schedule: the
+    K-step chain's codes are used last-first, so visit j reads bank K - j."""
+    K = banks.shape[0]
+    if not 1 <= j <= K:
+        raise ValueError(f"tail visit {j} outside 1..{K}")
+    return banks[K - j]
 
 
 def q4_gemm(fmt: int, M: int, N: int, K: int, a: torch.Tensor, a_scales, a_gscale,

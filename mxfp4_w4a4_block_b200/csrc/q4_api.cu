@@ -114,6 +114,26 @@ q4_status q4_dequantize(q4_format format, int block, const uint8_t* codes, const
                                              (cudaStream_t)stream, num_sms()));
 }
 
+q4_status q4_sigma_delta_codebanks(q4_format format, int block, const float* w, int64_t rows, int64_t cols,
+                                   const uint8_t* scales, const float* d_gscale, int visits, uint8_t* codes,
+                                   float* residue_out, int flags, void* stream) {
+    if (!valid_format(format) || rows < 0 || cols < 0) return Q4_ERR_ARG;
+    if (block != block_of(format)) return Q4_ERR_UNSUPPORTED;
+    if (flags & ~(Q4_LAYOUT_TC)) return Q4_ERR_ARG;
+    if (visits < 1 || visits > 4096) return Q4_ERR_ARG;
+    if (format == Q4_NVFP4 && !d_gscale) return Q4_ERR_ARG;
+    if (format == Q4_MXFP4 && d_gscale) return Q4_ERR_ARG;
+    if (cols % block) return Q4_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return Q4_OK;
+    if (!w || !scales || !codes) return Q4_ERR_ARG;
+    if (!aligned16(w) || !aligned16(codes) || (residue_out && !aligned16(residue_out))) return Q4_ERR_ALIGN;
+    q4::SigmaDeltaParams p;
+    p.w = w; p.rows = rows; p.cols = cols; p.scales = scales; p.gscale = d_gscale;
+    p.residue = nullptr; p.codes = codes; p.scols = cols / block; p.catoms = catoms_of(cols, block);
+    return cuda_status(q4::launch_sigma_delta_banks(p, block, (flags & Q4_LAYOUT_TC) != 0, visits, residue_out,
+                                                    (cudaStream_t)stream, num_sms()));
+}
+
 q4_status q4_sigma_delta_step(q4_format format, int block, const float* w, int64_t rows, int64_t cols,
                               const uint8_t* scales, const float* d_gscale, float* residue, uint8_t* codes,
                               int flags, void* stream) {

@@ -529,6 +529,62 @@ __global__ void __launch_bounds__(sdk::THREADS, 1)
     if (tid == 0) bulk_wait_all();
 }
 
+// ------------------------------------------------------------------ sigma-delta codebanks
+// The K-visit Sigma-Delta chain from r_0 = 0 in one pass ("Looped Transformer
+// quantization", sec. 2.3: the tail visits restart a chain of length K and
+// use its codes in reverse order; sec. 4: the codes are stored as K
+// codebanks).  Each thread owns 8 consecutive weights: it reads them and their
+// block scale once, runs the K visits with the residue in registers, and
+// writes visit k's 4 code bytes into bank k (a warp writes 128 contiguous
+// bytes per bank).  Optionally the final residue r_K is stored.
+template <int BLK, bool TC>
+__global__ void __launch_bounds__(256) sigma_delta_banks_kernel(SigmaDeltaParams p, int visits, int64_t bank_bytes,
+                                                                float* r_out) {
+    const int64_t cpr = p.cols / 8;
+    const int64_t total = p.rows * cpr;
+    const float s_t = (BLK == 16) ? *p.gscale : 0.0f;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t row = i / cpr, col = (i % cpr) * 8;
+        const float4* wp = reinterpret_cast<const float4*>(p.w + row * p.cols + col);
+        const float4 w0 = __ldcs(wp), w1 = __ldcs(wp + 1);
+        const int64_t c = col / BLK;
+        const uint32_t sb = TC ? p.scales[tc_scale_offset(row, c, p.catoms)] : p.scales[row * p.scols + c];
+        float inv;
+        bool degenerate;
+        if (BLK == 16) {
+            const NvScale sc = nv_scale_from_byte(sb, s_t);
+            inv = sc.inv;
+            degenerate = sc.degenerate;
+        } else {
+            inv = exp2_int(127 - (int)sb);
+            degenerate = false;
+        }
+        const float2 iv = make_float2(inv, inv);
+        float2 x[4] = {mul2_rn(make_float2(w0.x, w0.y), iv), mul2_rn(make_float2(w0.z, w0.w), iv),
+                       mul2_rn(make_float2(w1.x, w1.y), iv), mul2_rn(make_float2(w1.z, w1.w), iv)};
+        if (degenerate)
+            for (int j = 0; j < 4; ++j) x[j] = make_float2(0.0f, 0.0f);
+        float2 r[4] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f),
+                       make_float2(0.0f, 0.0f)};
+        uint8_t* dst = p.codes + row * (p.cols / 2) + col / 2;
+        for (int k = 0; k < visits; ++k) {
+            float2 v[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) v[j] = add2_rn(x[j], r[j]);
+            const uint32_t codes = e2m1_pack4(v[0].x, v[0].y, v[1].x, v[1].y) |
+                                   (e2m1_pack4(v[2].x, v[2].y, v[3].x, v[3].y) << 16);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) r[j] = sub2_rn(v[j], e2m1x2_value((codes >> (8 * j)) & 0xFFu));
+            __stcs(reinterpret_cast<unsigned int*>(dst + (int64_t)k * bank_bytes), codes);
+        }
+        if (r_out != nullptr) {
+            float4* rp = reinterpret_cast<float4*>(r_out + row * p.cols + col);
+            rp[0] = make_float4(r[0].x, r[0].y, r[1].x, r[1].y);
+            rp[1] = make_float4(r[2].x, r[2].y, r[3].x, r[3].y);
+        }
+    }
+}
+
 // ------------------------------------------------------------------ dequantize
 template <int BLK, bool TC, bool OUT_BF16>
 __global__ void __launch_bounds__(256) dequantize_kernel(DequantParams p) {
@@ -695,6 +751,22 @@ cudaError_t launch_dequantize(const DequantParams& p, int blk, bool tc, bool out
         else { if (out_bf16) Q4_DQ(32, false, true); else Q4_DQ(32, false, false); }
     }
 #undef Q4_DQ
+    return cudaGetLastError();
+}
+
+cudaError_t launch_sigma_delta_banks(const SigmaDeltaParams& p, int blk, bool tc, int visits, float* r_out,
+                                     cudaStream_t st, int num_sms) {
+    if (p.rows == 0 || p.cols == 0) return cudaSuccess;
+    const int64_t chunks = p.rows * (p.cols / 8);
+    const int grid = grid_for((chunks + 255) / 256, num_sms, 8);
+    const int64_t bank = p.rows * (p.cols / 2);
+#define Q4_SDB(B, T) sigma_delta_banks_kernel<B, T><<<grid, 256, 0, st>>>(p, visits, bank, r_out)
+    if (blk == 16) {
+        if (tc) Q4_SDB(16, true); else Q4_SDB(16, false);
+    } else {
+        if (tc) Q4_SDB(32, true); else Q4_SDB(32, false);
+    }
+#undef Q4_SDB
     return cudaGetLastError();
 }
 

@@ -234,6 +234,17 @@ def sigma_delta_step(fmt: int, w, scales, s_t, r: np.ndarray) -> np.ndarray:
     return codes
 
 
+def sigma_delta_codebanks(fmt: int, w, scales, s_t, visits: int):
+    """The Sigma-Delta chain of `visits` steps from r_0 = 0 ("Looped Transformer
+    quantization", sec. 2.3 / sec. 4: the tail restarts a chain and stores its
+    codes as codebanks): `visits` applications of sigma_delta_step.  Returns
+    (banks [visits, rows, cols/2], r_visits)."""
+    a = _f32(w)
+    r = np.zeros(a.shape, np.float32)
+    banks = np.stack([sigma_delta_step(fmt, a, scales, s_t, r) for _ in range(visits)])
+    return banks, r
+
+
 def gemm(fmt: int, a_codes, a_scales, a_st, b_codes, b_scales, b_st, M, N, K, rows=None):
     """Y = alpha * dec(A) dec(B)^T in binary64; optionally only the listed rows."""
     ac = np.ascontiguousarray(a_codes, dtype=np.uint8)

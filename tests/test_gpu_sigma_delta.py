@@ -96,3 +96,37 @@ def test_looped_core_full_size_sampled_rows():
                 assert np.array_equal(host(gc)[sel], oc)
         assert np.array_equal(host(r_gpu)[sel].view(np.uint32), r_orc.view(np.uint32))
         assert float(r_gpu.abs().max()) <= 1.0 + 2 ** -20
+
+
+@pytest.mark.parametrize("fmt", [q4.NVFP4, q4.MXFP4])
+@pytest.mark.parametrize("tc", [True, False])
+@pytest.mark.parametrize("shape,K", [((200, 352), 1), ((64, 512), 5), ((33, 1024), 32)])
+def test_codebanks_bit_exact(fmt, tc, shape, K):
+    """The one-pass K-step chain: every bank and the final residue bit for bit
+    against the oracle (K successive steps from r_0 = 0)."""
+    rows, cols = shape
+    w = synth.small_like("weight", rows * 3 + K, rows, cols)
+    s_t, g_t, g_sc, o_sc = setup_scales(fmt, w, tc)
+    flags = q4.LAYOUT_TC if tc else 0
+    r_out = torch.empty((rows, cols), dtype=torch.float32, device=DEV)
+    banks = q4.q4_sigma_delta_codebanks(fmt, dev(w), g_sc, K, gscale=g_t, flags=flags, residue_out=r_out)
+    o_banks, o_r = oracle.sigma_delta_codebanks(fmt, w, o_sc, s_t, K)
+    assert np.array_equal(host(banks), o_banks)
+    assert np.array_equal(host(r_out).view(np.uint32), o_r.view(np.uint32))
+
+
+def test_codebanks_match_successive_steps_and_reverse_tail():
+    """On the GPU the one-pass banks equal K successive q4_sigma_delta_step
+    calls, and tail visit K (the last) of the reverse schedule reads the
+    round-to-nearest codes."""
+    w = synth.small_like("weight", 5, 256, 768)
+    s_t, g_t, g_sc, _ = setup_scales(q4.NVFP4, w)
+    K = 8
+    banks = q4.q4_sigma_delta_codebanks(q4.NVFP4, dev(w), g_sc, K, gscale=g_t)
+    r = torch.zeros((256, 768), dtype=torch.float32, device=DEV)
+    for k in range(K):
+        c = q4.q4_sigma_delta_step(q4.NVFP4, dev(w), g_sc, r, gscale=g_t)
+        assert torch.equal(c, banks[k])
+    rtn, _ = q4.q4_quantize(q4.NVFP4, dev(w), gscale=g_t, flags=q4.SCALE_RU | q4.LAYOUT_TC)
+    assert torch.equal(q4.tail_bank(banks, K), rtn)
+    assert torch.equal(q4.tail_bank(banks, 1), banks[K - 1])

@@ -145,3 +145,28 @@ def test_looped_weights_bound_telescoping_first_visit(orc, fmt):
         assert np.abs(cum + r).max() <= k * 2.0 ** -20 * 8
     # mean error after R visits is within d / (2R)
     assert np.abs(cum / R).max() <= 2.0 / (2 * R) * (1 + 1e-5)
+
+
+def test_codebanks_reverse_tail_schedule(orc):
+    """Codebanks of a K-step chain ("Looped Transformer quantization", sec. 2.3):
+    the chain starts from r_0 = 0, so bank 0 -- the code of the LAST tail visit
+    in the reverse schedule -- is the plain round-to-nearest code; every later
+    bank is the next Sigma-Delta step; the mean of the K decoded codes tracks x
+    within the first-order bound d / (2K) (largest gap d = 2 on E2M1)."""
+    import synth
+    w = synth.small_like("weight", 11, 48, 64)
+    s_t = orc.tensor_scale(orc.amax(w), 1536.0)
+    rtn, sc = orc.nvfp4_quantize(w, s_t, round_up=True)
+    K = 12
+    banks, rK = orc.sigma_delta_codebanks(orc.NVFP4, w, sc, s_t, K)
+    assert banks.shape == (K, 48, 32)
+    assert np.array_equal(banks[0], rtn)
+    r = np.zeros_like(w)
+    for k in range(K):
+        assert np.array_equal(orc.sigma_delta_step(orc.NVFP4, w, sc, s_t, r), banks[k])
+    assert np.array_equal(r.view(np.uint32), rK.view(np.uint32))
+    # mean decoded code vs the normalised weight x = w / S
+    S = orc.dequantize(orc.NVFP4, np.full_like(rtn, 0x22), sc, s_t, 48, 64)   # code 1.0 -> S per element
+    x = w.astype(np.float64) / S
+    mean = np.mean([orc.dequantize(orc.NVFP4, banks[k], sc, 1.0, 48, 64) / (S / s_t) for k in range(K)], axis=0)
+    assert np.max(np.abs(mean - x)) <= 2.0 / (2 * K) + 1e-6
