@@ -77,6 +77,8 @@ def _load():
         "q4o_sigma_delta_step": (i32, [i32, P, i64, i64, P, f32, P, P]),
         "q4o_gemm": (i32, [i32, i64, i64, i64, P, P, f32, P, P, f32, P, i64, P]),
         "q4o_gemm_w4a16": (i32, [i32, i64, i64, i64, P, P, P, f32, P, i64, P]),
+        "q4o_philox4x32_10": (None, [P, P, P]),
+        "q4o_sr_requant": (i32, [i32, P, i64, i64, P, f32, ctypes.c_uint64, ctypes.c_uint32, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -231,6 +233,29 @@ def sigma_delta_step(fmt: int, w, scales, s_t, r: np.ndarray) -> np.ndarray:
                                       float(np.float32(s_t)), _ptr(r), _ptr(codes))
     if rc != 0:
         raise ValueError("sigma_delta_step: bad shape")
+    return codes
+
+
+def philox4x32_10(ctr, key) -> np.ndarray:
+    """The Philox4x32-10 block function: 4 counter words, 2 key words -> 4 words."""
+    c = np.ascontiguousarray(ctr, dtype=np.uint32)
+    k = np.ascontiguousarray(key, dtype=np.uint32)
+    out = np.zeros(4, np.uint32)
+    _load().q4o_philox4x32_10(_ptr(c), _ptr(k), _ptr(out))
+    return out
+
+
+def sr_requant(fmt: int, w, scales, s_t, seed: int, visit: int) -> np.ndarray:
+    """Stochastic-rounding requant of W at one loop visit with fixed (row-major)
+    block scales; returns the codes [rows, cols/2]."""
+    a = _f32(w)
+    rows, cols = a.shape
+    s = np.ascontiguousarray(scales, dtype=np.uint8)
+    codes = np.zeros((rows, cols // 2), np.uint8)
+    rc = _load().q4o_sr_requant(fmt, _ptr(a), rows, cols, _ptr(s), float(np.float32(s_t)), int(seed), int(visit),
+                                _ptr(codes))
+    if rc != 0:
+        raise ValueError("sr_requant: bad shape")
     return codes
 
 

@@ -463,3 +463,100 @@ int q4o_gemm_w4a16(int format, int64_t M, int64_t N, int64_t K, const float* x,
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Philox4x32-10, the counter-based generator of Salmon, Moraes, Dror and    */
+/* Shaw, "Parallel Random Numbers: As Easy as 1, 2, 3" (SC 2011): ten rounds  */
+/* of two 32x32 -> 64-bit multiplies (multipliers 0xD2511F53, 0xCD9E8D57)     */
+/* mixing the four counter words with the two key words, the key bumped by    */
+/* the Weyl constants 0x9E3779B9, 0xBB67AE85 after every round.               */
+/* ------------------------------------------------------------------------ */
+void q4o_philox4x32_10(const uint32_t ctr_in[4], const uint32_t key_in[2], uint32_t out[4])
+{
+    uint32_t c0 = ctr_in[0], c1 = ctr_in[1], c2 = ctr_in[2], c3 = ctr_in[3];
+    uint32_t k0 = key_in[0], k1 = key_in[1];
+    for (int round = 0; round < 10; ++round) {
+        uint64_t p0 = (uint64_t)0xD2511F53u * c0;
+        uint64_t p1 = (uint64_t)0xCD9E8D57u * c2;
+        uint32_t n0 = (uint32_t)(p1 >> 32) ^ c1 ^ k0;
+        uint32_t n1 = (uint32_t)p1;
+        uint32_t n2 = (uint32_t)(p0 >> 32) ^ c3 ^ k1;
+        uint32_t n3 = (uint32_t)p0;
+        c0 = n0; c1 = n1; c2 = n2; c3 = n3;
+        k0 += 0x9E3779B9u;
+        k1 += 0xBB67AE85u;
+    }
+    out[0] = c0; out[1] = c1; out[2] = c2; out[3] = c3;
+}
+
+/* Uniform u in [0, 1) of element e at visit `visit`: Philox4x32-10 with     */
+/* counter (e/4 low word, e/4 high word, visit, 0) and key (seed low, seed    */
+/* high); element e takes output word e % 4, whose top 24 bits give          */
+/* u = (word >> 8) * 2^-24 (exact in binary32).                              */
+static float sr_uniform(uint64_t seed, uint32_t visit, int64_t e)
+{
+    uint64_t g = (uint64_t)e >> 2;
+    uint32_t ctr[4] = {(uint32_t)g, (uint32_t)(g >> 32), visit, 0u};
+    uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+    uint32_t out[4];
+    q4o_philox4x32_10(ctr, key, out);
+    return (float)(out[e & 3] >> 8) * 0x1p-24f;
+}
+
+/* Stochastic rounding onto the E2M1 grid ([LT] sec. 2.1: SR draws each code */
+/* so that its conditional expectation equals the weight).  For |x| between   */
+/* neighbouring magnitudes a <= |x| < b the magnitude is b when               */
+/* u < (|x| - a) / (b - a), else a (both operations exact: Sterbenz and a     */
+/* power-of-two gap); |x| >= 6 gives 6; the sign bit is x's (R1).            */
+static uint8_t sr_e2m1(float x, float u)
+{
+    float m = fabsf(x);
+    int idx;
+    if (m >= 6.0f) {
+        idx = 7;
+    } else {
+        int i = 0;
+        while (i < 7 && (float)E2M1_MAG[i + 1] <= m) ++i;
+        float a = (float)E2M1_MAG[i], b = (float)E2M1_MAG[i + 1];
+        float p = (m - a) / (b - a);
+        idx = u < p ? i + 1 : i;
+    }
+    return (uint8_t)((signbit(x) ? 0x8 : 0x0) | idx);
+}
+
+/* One stochastic-rounding requant of W at loop visit `visit` ([LT] sec. 2.1  */
+/* and sec. 3: the SR baseline of the looped-weight experiments, a fixed       */
+/* seed giving one weight trajectory): x = W * inv with the fixed block scale  */
+/* (R3, degenerate blocks give +0), code = SR(x).  Scales row-major.           */
+int q4o_sr_requant(int format, const float* w, int64_t rows, int64_t cols, const uint8_t* scales, float s_t,
+                   uint64_t seed, uint32_t visit, uint8_t* codes)
+{
+    int blk = format == Q4O_NVFP4 ? 16 : 32;
+    if (cols % blk != 0) return -1;
+    int64_t nb = cols / blk;
+    for (int64_t i = 0; i < rows; ++i) {
+        for (int64_t b = 0; b < nb; ++b) {
+            uint8_t sb = scales[i * nb + b];
+            float inv;
+            int degenerate;
+            if (format == Q4O_NVFP4) {
+                float S = (float)q4o_e4m3_decode(sb) * s_t;
+                inv = 1.0f / S;
+                degenerate = block_is_degenerate(S, inv, s_t);
+            } else {
+                inv = ldexpf(1.0f, 127 - (int)sb);
+                degenerate = 0;
+            }
+            for (int j = 0; j < blk; ++j) {
+                int64_t k = b * blk + j;
+                int64_t e = i * cols + k;
+                float x = degenerate ? 0.0f : w[e] * inv;
+                uint8_t c = sr_e2m1(x, sr_uniform(seed, visit, e));
+                uint8_t* dst = codes + i * (cols / 2) + k / 2;
+                if ((k & 1) == 0) *dst = (uint8_t)((*dst & 0xF0u) | c);
+                else *dst = (uint8_t)((*dst & 0x0Fu) | (uint8_t)(c << 4));
+            }
+        }
+    }
+    return 0;
+}
