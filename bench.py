@@ -50,6 +50,7 @@ B_W4A16_GEMM_NOTE = "2*M*N*K FLOP on the bf16 tensor pipe"
 B_QUANT_BF16 = 2 + 0.5 + 1 / 16          # read bf16, write codes + E4M3 scale
 B_AMAX_BF16 = 2
 B_SIGMA_DELTA = 4 + 4 + 4 + 0.5 + 1 / 16  # w, r in, r out, codes, scale
+B_SR = 4 + 0.5 + 1 / 16                   # w, codes, scale (the random numbers are computed)
 B_MX_QUANT_BF16 = 2 + 0.5 + 1 / 32       # read bf16, write codes + E8M0 scale
 B_DEQUANT_BF16 = 0.5 + 1 / 16 + 2
 
@@ -271,6 +272,13 @@ def rows_bench(q4, dev, flush, pk, reps=30):
                                         "frac_hbm": gbs / hbm, "B_per_weight": 4 + 32 * 0.5,
                                         "vs_32_separate_visits": ms_sd * 32 / ms_cb}
     del banks
+
+    def sr_visit():
+        for wt, sc, g, r, c, _ in mats:
+            q4.q4_sr_requant(q4.NVFP4, wt, sc, 42, 7, gscale=g, codes=c)
+    ms_sr, _ = time_fn(sr_visit, reps, flush)
+    gbs = nw * B_SR / (ms_sr * 1e-3) / 1e9
+    out["sr_requant_visit"] = {"weights": nw, "matrices": 13, "us": ms_sr * 1e3, "GB/s": gbs, "frac_hbm": gbs / hbm}
     ms_v, _ = time_fn(visit, max(5, reps // 3), flush)
     out["looped_visit"] = {"us": ms_v * 1e3, "us_R32": ms_v * 1e3 * 32,
                            "note": "Sigma-Delta requant of all 13 weights + 13 W4A16 GEMMs"}

@@ -175,6 +175,25 @@ Q4_API q4_status q4_sigma_delta_step(q4_format format, int block, const float* w
                               int flags, void* stream);
 
 /*
+ * q4_sr_requant -- one stochastic-rounding requant of a weight at a loop visit
+ *   ("Looped Transformer quantization", sec. 2.1: the stochastic-rounding
+ *   baseline draws every code so that its conditional expectation equals the
+ *   weight; sec. 3: a fixed seed gives one weight trajectory shared by all
+ *   inputs).  With the block scales fixed, x = w * inv (as in
+ *   q4_sigma_delta_step); for neighbouring E2M1 magnitudes a <= |x| < b the
+ *   code's magnitude is b when u < (|x| - a) / (b - a), else a; |x| >= 6 gives
+ *   6; the sign bit is x's.  u = (word >> 8) * 2^-24, where for element
+ *   e = row * cols + col the word is output e % 4 of Philox4x32-10 (Salmon et
+ *   al., SC 2011) with counter (e / 4 low, e / 4 high, visit, 0) and key
+ *   (seed low, seed high) -- any host or device implementation of that
+ *   generator reproduces the codes.
+ *   w, scales, d_gscale, codes, flags as q4_sigma_delta_step (no residue).
+ */
+Q4_API q4_status q4_sr_requant(q4_format format, int block, const float* w, int64_t rows,
+                        int64_t cols, const uint8_t* scales, const float* d_gscale,
+                        uint64_t seed, uint32_t visit, uint8_t* codes, int flags, void* stream);
+
+/*
  * q4_sigma_delta_codebanks -- the whole Sigma-Delta chain of `visits` loop
  *   visits from r_0 = 0 in one pass, stored as codebanks ("Looped Transformer
  *   quantization", sec. 2.3: for frozen-weight inference the last K visits

@@ -9,7 +9,7 @@ there is no CPU fallback, and importing fails loudly if the library has not
 been built (``python -m mxfp4_w4a4_block_b200.build``).
 
 Function names mirror the C entry points: q4_amax, q4_quantize,
-q4_dequantize, q4_sigma_delta_step, q4_sigma_delta_codebanks, q4_gemm,
+q4_dequantize, q4_sigma_delta_step, q4_sigma_delta_codebanks, q4_sr_requant, q4_gemm,
 q4_gemm_workspace_size, q4_get_device_error, q4_scale_bytes (tail_bank is a
 pure indexing helper of the reverse-order codebank schedule).
 """
@@ -56,6 +56,7 @@ SIGNATURES = {
     "q4_dequantize": (_I, [_I, _I, _P, _P, _P, _I64, _I64, _I, _I, _P, _P]),
     "q4_sigma_delta_step": (_I, [_I, _I, _P, _I64, _I64, _P, _P, _P, _P, _I, _P]),
     "q4_sigma_delta_codebanks": (_I, [_I, _I, _P, _I64, _I64, _P, _P, _I, _P, _P, _I, _P]),
+    "q4_sr_requant": (_I, [_I, _I, _P, _I64, _I64, _P, _P, ctypes.c_uint64, ctypes.c_uint32, _P, _I, _P]),
     "q4_gemm": (_I, [_I, _I, _I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _P, _I, _P, _P, _SZ, _P]),
     "q4_gemm_workspace_size": (_SZ, [_I, _I64, _I64, _I64, _I]),
     "q4_get_device_error": (_I, [_P]),
@@ -193,6 +194,19 @@ def q4_sigma_delta_codebanks(fmt: int, w: torch.Tensor, scales: torch.Tensor, vi
     st = lib().q4_sigma_delta_codebanks(fmt, BLOCK[fmt], _ptr(w), rows, cols, _ptr(scales), _ptr(gscale), visits,
                                         _ptr(codes), _ptr(residue_out), flags, _stream(stream))
     _check("q4_sigma_delta_codebanks", st)
+    return codes
+
+
+def q4_sr_requant(fmt: int, w: torch.Tensor, scales: torch.Tensor, seed: int, visit: int,
+                  gscale: torch.Tensor | None = None, flags: int = LAYOUT_TC, codes: torch.Tensor | None = None,
+                  stream=None) -> torch.Tensor:
+    """Stochastic-rounding requant of w at one loop visit; returns the codes."""
+    rows, cols = w.shape
+    if codes is None:
+        codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=w.device)
+    st = lib().q4_sr_requant(fmt, BLOCK[fmt], _ptr(w), rows, cols, _ptr(scales), _ptr(gscale), int(seed), int(visit),
+                             _ptr(codes), flags, _stream(stream))
+    _check("q4_sr_requant", st)
     return codes
 
 

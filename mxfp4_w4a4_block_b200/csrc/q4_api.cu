@@ -134,6 +134,25 @@ q4_status q4_sigma_delta_codebanks(q4_format format, int block, const float* w, 
                                                     (cudaStream_t)stream, num_sms()));
 }
 
+q4_status q4_sr_requant(q4_format format, int block, const float* w, int64_t rows, int64_t cols,
+                        const uint8_t* scales, const float* d_gscale, uint64_t seed, uint32_t visit, uint8_t* codes,
+                        int flags, void* stream) {
+    if (!valid_format(format) || rows < 0 || cols < 0) return Q4_ERR_ARG;
+    if (block != block_of(format)) return Q4_ERR_UNSUPPORTED;
+    if (flags & ~(Q4_LAYOUT_TC)) return Q4_ERR_ARG;
+    if (format == Q4_NVFP4 && !d_gscale) return Q4_ERR_ARG;
+    if (format == Q4_MXFP4 && d_gscale) return Q4_ERR_ARG;
+    if (cols % block) return Q4_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return Q4_OK;
+    if (!w || !scales || !codes) return Q4_ERR_ARG;
+    if (!aligned16(w) || !aligned16(codes)) return Q4_ERR_ALIGN;
+    q4::SigmaDeltaParams p;
+    p.w = w; p.rows = rows; p.cols = cols; p.scales = scales; p.gscale = d_gscale;
+    p.residue = nullptr; p.codes = codes; p.scols = cols / block; p.catoms = catoms_of(cols, block);
+    return cuda_status(q4::launch_sr_requant(p, block, (flags & Q4_LAYOUT_TC) != 0, seed, visit,
+                                             (cudaStream_t)stream, num_sms()));
+}
+
 q4_status q4_sigma_delta_step(q4_format format, int block, const float* w, int64_t rows, int64_t cols,
                               const uint8_t* scales, const float* d_gscale, float* residue, uint8_t* codes,
                               int flags, void* stream) {

@@ -80,6 +80,8 @@ cudaError_t launch_quantize(const QuantParams& p, int blk, bool bf16, bool tc, b
 cudaError_t launch_sigma_delta(const SigmaDeltaParams& p, int blk, bool tc, cudaStream_t st, int num_sms);
 cudaError_t launch_sigma_delta_banks(const SigmaDeltaParams& p, int blk, bool tc, int visits, float* r_out,
                                      cudaStream_t st, int num_sms);
+cudaError_t launch_sr_requant(const SigmaDeltaParams& p, int blk, bool tc, uint64_t seed, uint32_t visit,
+                              cudaStream_t st, int num_sms);
 cudaError_t launch_dequantize(const DequantParams& p, int blk, bool tc, bool out_bf16, cudaStream_t st,
                               int num_sms);
 cudaError_t launch_gemm(const GemmParams& p, cudaStream_t st, int num_sms);

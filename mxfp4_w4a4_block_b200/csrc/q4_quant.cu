@@ -585,6 +585,85 @@ __global__ void __launch_bounds__(256) sigma_delta_banks_kernel(SigmaDeltaParams
     }
 }
 
+// ------------------------------------------------------------------ stochastic-rounding requant
+// Philox4x32-10 (Salmon, Moraes, Dror and Shaw, "Parallel Random Numbers: As
+// Easy as 1, 2, 3", SC 2011): ten rounds of two 32 x 32 -> 64-bit multiplies
+// mixing the four counter words with the two key words; the key is bumped by
+// the Weyl constants after every round.
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint2 k) {
+#pragma unroll
+    for (int round = 0; round < 10; ++round) {
+        const uint32_t hi0 = __umulhi(0xD2511F53u, c.x), lo0 = 0xD2511F53u * c.x;
+        const uint32_t hi1 = __umulhi(0xCD9E8D57u, c.z), lo1 = 0xCD9E8D57u * c.z;
+        c = make_uint4(hi1 ^ c.y ^ k.x, lo1, hi0 ^ c.w ^ k.y, lo0);
+        k.x += 0x9E3779B9u;
+        k.y += 0xBB67AE85u;
+    }
+    return c;
+}
+
+// Stochastic rounding of a normalised value onto the E2M1 grid with the
+// uniform u in [0, 1): between neighbouring magnitudes a <= |x| < b the
+// magnitude is b when u < (|x| - a) / (b - a) (exact: the gap is 0.5, 1 or 2),
+// else a; |x| >= 6 gives 6; the sign bit is x's.
+__device__ __forceinline__ uint32_t sr_e2m1(float x, float u) {
+    const float m = fabsf(x);
+    uint32_t idx;
+    if (m >= 6.0f) {
+        idx = 7;
+    } else {
+        const uint32_t i = (m >= 0.5f) + (m >= 1.0f) + (m >= 1.5f) + (m >= 2.0f) + (m >= 3.0f) + (m >= 4.0f);
+        // twice the magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6, one nibble each
+        const uint32_t twice = 0xC8643210u;
+        const float a = (float)((twice >> (4 * i)) & 0xFu) * 0.5f;
+        // 1 / (b - a): gaps 0.5 below 2, 1 from 2 to 4, 2 from 4 to 6 (exact)
+        const float rgap = (i < 4) ? 2.0f : (i < 6 ? 1.0f : 0.5f);
+        idx = (u < __fmul_rn(__fsub_rn(m, a), rgap)) ? i + 1 : i;
+    }
+    return (signbit(x) ? 8u : 0u) | idx;
+}
+
+// One stochastic-rounding requant at a loop visit: each thread owns 8
+// consecutive weights e0 .. e0 + 7 (e0 = row * cols + col, a multiple of 8),
+// i.e. the two Philox blocks of counters (e0/4 + {0, 1}, visit), key = seed.
+template <int BLK, bool TC>
+__global__ void __launch_bounds__(256) sr_requant_kernel(SigmaDeltaParams p, uint64_t seed, uint32_t visit) {
+    const int64_t cpr = p.cols / 8;
+    const int64_t total = p.rows * cpr;
+    const float s_t = (BLK == 16) ? *p.gscale : 0.0f;
+    const uint2 key = make_uint2((uint32_t)seed, (uint32_t)(seed >> 32));
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t row = i / cpr, col = (i % cpr) * 8;
+        const float4* wp = reinterpret_cast<const float4*>(p.w + row * p.cols + col);
+        const float4 w0 = __ldcs(wp), w1 = __ldcs(wp + 1);
+        const int64_t c = col / BLK;
+        const uint32_t sb = TC ? p.scales[tc_scale_offset(row, c, p.catoms)] : p.scales[row * p.scols + c];
+        float inv;
+        bool degenerate;
+        if (BLK == 16) {
+            const NvScale sc = nv_scale_from_byte(sb, s_t);
+            inv = sc.inv;
+            degenerate = sc.degenerate;
+        } else {
+            inv = exp2_int(127 - (int)sb);
+            degenerate = false;
+        }
+        const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+        const uint64_t g = (uint64_t)(row * p.cols + col) >> 2;
+        const uint4 r0 = philox4x32_10(make_uint4((uint32_t)g, (uint32_t)(g >> 32), visit, 0u), key);
+        const uint4 r1 = philox4x32_10(make_uint4((uint32_t)(g + 1), (uint32_t)((g + 1) >> 32), visit, 0u), key);
+        const uint32_t rw[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+        uint32_t codes = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float x = degenerate ? 0.0f : __fmul_rn(wv[j], inv);
+            const float u = (float)(rw[j] >> 8) * 0x1p-24f;
+            codes |= sr_e2m1(x, u) << (4 * j);
+        }
+        *reinterpret_cast<uint32_t*>(p.codes + row * (p.cols / 2) + col / 2) = codes;
+    }
+}
+
 // ------------------------------------------------------------------ dequantize
 template <int BLK, bool TC, bool OUT_BF16>
 __global__ void __launch_bounds__(256) dequantize_kernel(DequantParams p) {
@@ -767,6 +846,21 @@ cudaError_t launch_sigma_delta_banks(const SigmaDeltaParams& p, int blk, bool tc
         if (tc) Q4_SDB(32, true); else Q4_SDB(32, false);
     }
 #undef Q4_SDB
+    return cudaGetLastError();
+}
+
+cudaError_t launch_sr_requant(const SigmaDeltaParams& p, int blk, bool tc, uint64_t seed, uint32_t visit,
+                              cudaStream_t st, int num_sms) {
+    if (p.rows == 0 || p.cols == 0) return cudaSuccess;
+    const int64_t chunks = p.rows * (p.cols / 8);
+    const int grid = grid_for((chunks + 255) / 256, num_sms, 8);
+#define Q4_SR(B, T) sr_requant_kernel<B, T><<<grid, 256, 0, st>>>(p, seed, visit)
+    if (blk == 16) {
+        if (tc) Q4_SR(16, true); else Q4_SR(16, false);
+    } else {
+        if (tc) Q4_SR(32, true); else Q4_SR(32, false);
+    }
+#undef Q4_SR
     return cudaGetLastError();
 }
 
