@@ -78,6 +78,7 @@ def _load():
         "q4o_gemm": (i32, [i32, i64, i64, i64, P, P, f32, P, P, f32, P, i64, P]),
         "q4o_gemm_w4a16": (i32, [i32, i64, i64, i64, P, P, P, f32, P, i64, P]),
         "q4o_philox4x32_10": (None, [P, P, P]),
+        "q4o_nvfp4_quantize46": (i32, [P, i64, i64, f32, P, P]),
         "q4o_sr_requant": (i32, [i32, P, i64, i64, P, f32, ctypes.c_uint64, ctypes.c_uint32, P]),
     }
     for name, (res, args) in sig.items():
@@ -144,6 +145,20 @@ def nvfp4_quantize(x, s_t, round_up: bool = False):
                                     int(round_up), _ptr(codes), _ptr(scales))
     if rc != 0:
         raise ValueError("nvfp4_quantize: cols must be a multiple of 16")
+    return codes, scales
+
+
+def nvfp4_quantize46(x, s_t):
+    """NVFP4 with 4/6 block scaling: per block the rounded-up E4M3 candidate
+    mapping the block max to 6 or to 4, whichever quantizes the block with the
+    smaller squared error (ties: 6).  Returns (codes, row-major scales)."""
+    a = _f32(x)
+    rows, cols = a.shape
+    codes = np.zeros((rows, cols // 2), np.uint8)
+    scales = np.zeros((rows, cols // 16), np.uint8)
+    rc = _load().q4o_nvfp4_quantize46(_ptr(a), rows, cols, float(np.float32(s_t)), _ptr(codes), _ptr(scales))
+    if rc != 0:
+        raise ValueError("nvfp4_quantize46: cols must be a multiple of 16")
     return codes, scales
 
 

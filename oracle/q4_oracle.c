@@ -560,3 +560,67 @@ int q4o_sr_requant(int format, const float* w, int64_t rows, int64_t cols, const
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* 4/6 block scaling ([LT] sec. 2.2 and the block_scale_46 call of sec. 2.5:  */
+/* each block's E4M3 scale is a rounded-up candidate that maps the block      */
+/* maximum to 6 or to 4; under s_t = max|W| / (6 * 256) either keeps |x| <= 6). */
+/* The choice between the two is not given on the page (reading R10): the      */
+/* candidate whose quantized block has the smaller sum of squared errors in   */
+/* the input's units, err = sum_j (x_j - dec(code_j) * S)^2 accumulated in     */
+/* binary64 in element order (x_j - dec * S is exact there); ties go to 6.     */
+/* ------------------------------------------------------------------------ */
+static void nv46_candidate(const float* xb, float amax, float s_t, float target, uint8_t* sb_out,
+                           uint8_t codes_out[16], double* err_out)
+{
+    uint8_t sb = 0;
+    if (s_t > 0.0f && isfinite(s_t)) {
+        float denom = target * s_t;
+        float sbf = amax / denom;
+        sb = q4o_e4m3_encode(sbf, 1);
+    }
+    float S = (float)q4o_e4m3_decode(sb) * s_t;
+    float inv = 1.0f / S;
+    int degenerate = block_is_degenerate(S, inv, s_t);
+    double err = 0.0;
+    for (int j = 0; j < 16; ++j) {
+        float v = degenerate ? 0.0f : xb[j] * inv;
+        uint8_t c = q4o_e2m1_encode(v);
+        codes_out[j] = c;
+        double d = (double)xb[j] - q4o_e2m1_decode(c) * (double)S;
+        err = err + d * d;
+    }
+    *sb_out = sb;
+    *err_out = err;
+}
+
+int q4o_nvfp4_quantize46(const float* x, int64_t rows, int64_t cols, float s_t, uint8_t* codes, uint8_t* scales)
+{
+    if (rows < 0 || cols < 0 || cols % 16 != 0) return -1;
+    const int64_t nb = cols / 16;
+    for (int64_t i = 0; i < rows; ++i) {
+        const float* xr = x + i * cols;
+        for (int64_t b = 0; b < nb; ++b) {
+            const float* xb = xr + b * 16;
+            float amax = 0.0f;
+            for (int j = 0; j < 16; ++j) {
+                float a = fabsf(xb[j]);
+                if (a > amax) amax = a;
+            }
+            uint8_t sb6, sb4, c6[16], c4[16];
+            double e6, e4;
+            nv46_candidate(xb, amax, s_t, 6.0f, &sb6, c6, &e6);
+            nv46_candidate(xb, amax, s_t, 4.0f, &sb4, c4, &e4);
+            const int four = e4 < e6;
+            scales[i * nb + b] = four ? sb4 : sb6;
+            for (int j = 0; j < 16; ++j) {
+                uint8_t c = four ? c4[j] : c6[j];
+                int64_t k = b * 16 + j;
+                uint8_t* dst = codes + i * (cols / 2) + k / 2;
+                if ((k & 1) == 0) *dst = (uint8_t)((*dst & 0xF0u) | c);
+                else *dst = (uint8_t)((*dst & 0x0Fu) | (uint8_t)(c << 4));
+            }
+        }
+    }
+    return 0;
+}

@@ -167,3 +167,45 @@ def test_tc_scale_layout_offsets(orc):
     tc = orc.scales_to_tc(s)
     assert np.array_equal(orc.scales_from_tc(tc, 130, 5), s)
     assert np.count_nonzero(tc) == s.size   # padding is zero, the map is injective
+
+
+def _block_sse(orc, x, codes, scales, s_t):
+    """Per-block sum of squared errors in the input's units, recomputed in numpy."""
+    deq = orc.dequantize(orc.NVFP4, codes, scales, s_t, *x.shape)
+    d = x.astype(np.float64) - deq
+    return (d * d).reshape(x.shape[0], -1, 16).sum(axis=2)
+
+
+def test_scale46_picks_the_better_rounded_up_candidate(orc):
+    """4/6 block scaling ("Looped Transformer quantization", sec. 2.2): every
+    block's scale is one of the two rounded-up E4M3 candidates (block max -> 6 or
+    -> 4), the choice never has a larger squared error than the other candidate
+    (numpy recomputation), and so it is never worse than plain round-up scaling."""
+    import synth
+    w = synth.small_like("weight", 21, 64, 256)
+    s_t = orc.tensor_scale(orc.amax(w), 1536.0)
+    c46, s46 = orc.nvfp4_quantize46(w, s_t)
+    c6, s6 = orc.nvfp4_quantize(w, s_t, round_up=True)
+    amax = np.abs(w.astype(np.float32)).reshape(64, -1, 16).max(axis=2)
+    cand4 = np.vectorize(lambda a: orc.e4m3_encode(float(np.float32(a) / np.float32(np.float32(4.0) * s_t)),
+                                                   round_up=True))(amax)
+    assert np.all((s46 == s6) | (s46 == cand4))
+    e46 = _block_sse(orc, w, c46, s46, s_t)
+    e6 = _block_sse(orc, w, c6, s6, s_t)
+    assert np.all(e46 <= e6)
+    assert np.any(s46 != s6)                     # the 4-candidate wins somewhere on real data
+    # where the 4-candidate was chosen it was strictly better
+    four = s46 != s6
+    assert np.all(e46[four] < e6[four])
+
+
+def test_scale46_keeps_normalised_weights_in_range(orc):
+    """With s_t = max|W| / (6 * 256) both rounded-up candidates keep |x| <= 6
+    (page fact), so no code of a 4/6-scaled weight saturates beyond the grid."""
+    import synth
+    w = synth.small_like("weight", 22, 32, 512)
+    s_t = orc.tensor_scale(orc.amax(w), 1536.0)
+    codes, scales = orc.nvfp4_quantize46(w, s_t)
+    S = orc.dequantize(orc.NVFP4, np.full_like(codes, 0x22), scales, s_t, 32, 512)
+    x = w.astype(np.float64) / S
+    assert np.abs(x).max() <= 6.0 * (1 + 2 ** -20)
