@@ -76,7 +76,8 @@ enum {
     Q4_SCALE_RU = 1,     /* round block scales up (NVFP4: E4M3 toward +inf;
                             MXFP4: smallest exponent with block max <= 6*2^e) */
     Q4_LAYOUT_TC = 2,    /* scales in the tensor-core layout (else row-major) */
-    Q4_HADAMARD32 = 4    /* MXFP4 only: block Hadamard-32 before quantizing   */
+    Q4_HADAMARD32 = 4,   /* MXFP4 only: block Hadamard-32 before quantizing   */
+    Q4_SCALE_46 = 8      /* NVFP4 only: 4/6 block scaling (see q4_quantize)    */
 };
 
 /* Kinds of GEMM left operand. */
@@ -135,7 +136,15 @@ Q4_API q4_status q4_amax(q4_dtype dt, const void* x, int64_t n, float denom, flo
  *   d_gscale: device pointer to s_t (NVFP4, required); must be NULL for MXFP4.
  *   d_chan: device float[cols] multipliers c (MXFP4 only, optional, NULL = 1).
  *   codes: device [rows, cols/2] bytes.  scales: device, q4_scale_bytes() bytes.
- *   flags: Q4_SCALE_RU | Q4_LAYOUT_TC | Q4_HADAMARD32.
+ *   flags: Q4_SCALE_RU | Q4_LAYOUT_TC | Q4_HADAMARD32 | Q4_SCALE_46.
+ *   Q4_SCALE_46 (NVFP4; "Looped Transformer quantization", sec. 2.2 and the
+ *     block_scale_46 of sec. 2.5): each block's scale is one of two rounded-up
+ *     candidates, E4M3_RU(amax / (6 * s_t)) or E4M3_RU(amax / (4 * s_t)); the
+ *     page gives no rule for the choice, so the block takes the candidate whose
+ *     codes have the smaller sum of squared errors sum_j (x_j - dec_j * S)^2,
+ *     formed in binary64 in element order (ties: the 6 candidate).  With
+ *     s_t = max|W| / (6 * 256) either candidate keeps |x| <= 6, as Sigma-Delta
+ *     requires.  Q4_SCALE_RU is implied.
  */
 Q4_API q4_status q4_quantize(q4_format format, int block, q4_dtype in_dt, const void* x,
                       int64_t rows, int64_t cols, int64_t ld,

@@ -28,6 +28,7 @@ BF16 = 1
 SCALE_RU = 1
 LAYOUT_TC = 2
 HADAMARD32 = 4
+SCALE_46 = 8
 
 A_QUANTIZED = 0
 A_BF16 = 1

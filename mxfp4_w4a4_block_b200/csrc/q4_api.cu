@@ -78,8 +78,9 @@ q4_status q4_quantize(q4_format format, int block, q4_dtype in_dt, const void* x
                       int flags, void* stream) {
     if (!valid_format(format) || !valid_dtype(in_dt) || rows < 0 || cols < 0 || ld < cols) return Q4_ERR_ARG;
     if (block != block_of(format)) return Q4_ERR_UNSUPPORTED;
-    if (flags & ~(Q4_SCALE_RU | Q4_LAYOUT_TC | Q4_HADAMARD32)) return Q4_ERR_ARG;
+    if (flags & ~(Q4_SCALE_RU | Q4_LAYOUT_TC | Q4_HADAMARD32 | Q4_SCALE_46)) return Q4_ERR_ARG;
     if (format == Q4_NVFP4 && ((flags & Q4_HADAMARD32) || d_chan)) return Q4_ERR_UNSUPPORTED;
+    if (format == Q4_MXFP4 && (flags & Q4_SCALE_46)) return Q4_ERR_UNSUPPORTED;
     if (format == Q4_NVFP4 && !d_gscale) return Q4_ERR_ARG;
     if (format == Q4_MXFP4 && d_gscale) return Q4_ERR_ARG;
     if (cols % block) return Q4_ERR_SHAPE;
@@ -94,7 +95,8 @@ q4_status q4_quantize(q4_format format, int block, q4_dtype in_dt, const void* x
     p.scols = cols / block; p.catoms = catoms_of(cols, block);
     return cuda_status(q4::launch_quantize(p, block, in_dt == Q4_BF16, (flags & Q4_LAYOUT_TC) != 0,
                                            (flags & Q4_SCALE_RU) != 0, (flags & Q4_HADAMARD32) != 0,
-                                           d_chan != nullptr, (cudaStream_t)stream, num_sms()));
+                                           d_chan != nullptr, (flags & Q4_SCALE_46) != 0, (cudaStream_t)stream,
+                                           num_sms()));
 }
 
 q4_status q4_dequantize(q4_format format, int block, const uint8_t* codes, const uint8_t* scales,
@@ -231,7 +233,7 @@ q4_status q4_gemm(q4_format format, int block, int64_t M, int64_t N, int64_t K, 
         q4::QuantParams qp;
         qp.x = a; qp.rows = M; qp.cols = K; qp.ld = K; qp.gscale = d_a_gscale; qp.chan = nullptr;
         qp.codes = ws; qp.scales = ws + codes_al; qp.scols = K / 16; qp.catoms = catoms_of(K, 16);
-        cudaError_t e = q4::launch_quantize(qp, 16, true, true, false, false, false, st, num_sms());
+        cudaError_t e = q4::launch_quantize(qp, 16, true, true, false, false, false, false, st, num_sms());
         if (e != cudaSuccess) return cuda_status(e);
         a_codes = ws;
         a_scales = ws + codes_al;

@@ -76,7 +76,7 @@ cudaError_t launch_w4a16(const W4A16Params& p, cudaStream_t st, int num_sms);
 cudaError_t launch_amax(const void* x, int64_t n, bool bf16, float denom, float* d_out,
                         cudaStream_t st, int num_sms);
 cudaError_t launch_quantize(const QuantParams& p, int blk, bool bf16, bool tc, bool ru, bool had,
-                            bool chan, cudaStream_t st, int num_sms);
+                            bool chan, bool s46, cudaStream_t st, int num_sms);
 cudaError_t launch_sigma_delta(const SigmaDeltaParams& p, int blk, bool tc, cudaStream_t st, int num_sms);
 cudaError_t launch_sigma_delta_banks(const SigmaDeltaParams& p, int blk, bool tc, int visits, float* r_out,
                                      cudaStream_t st, int num_sms);

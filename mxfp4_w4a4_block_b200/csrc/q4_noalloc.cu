@@ -77,7 +77,7 @@ extern "C" Q4_API q4_status q4_gemm_a_bf16_noalloc(int64_t M, int64_t N, int64_t
     q4::QuantParams qp;
     qp.x = a_bf16; qp.rows = M; qp.cols = K; qp.ld = K; qp.gscale = d_a_gscale; qp.chan = nullptr;
     qp.codes = scratch; qp.scales = scratch + codes_al; qp.scols = K / 16; qp.catoms = ((K / 16) + 3) / 4;
-    if (q4::launch_quantize(qp, 16, true, true, false, false, false, st, sms) != cudaSuccess) return Q4_ERR_CUDA;
+    if (q4::launch_quantize(qp, 16, true, true, false, false, false, false, st, sms) != cudaSuccess) return Q4_ERR_CUDA;
 
     q4::GemmParams p;
     p.M = M; p.N = N; p.K = K;

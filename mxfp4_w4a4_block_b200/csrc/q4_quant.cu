@@ -138,6 +138,62 @@ struct QzGeom {
     static_assert(BPT >= 1 && ROWS % 128 == 0 && ROWS <= 256, "tile geometry");
 };
 
+// One candidate of 4/6 block scaling: the rounded-up E4M3 scale mapping the
+// block max to `target` (6 or 4), the block's codes under it, and their sum of
+// squared errors in the input's units, accumulated in binary64 in element
+// order (x - dec(code) * S is exact there), explicitly rounded so that no
+// fused multiply-add changes it.
+__device__ __forceinline__ void nv46_candidate(const float (&v)[16], const NvCtx& c, float amax, float target,
+                                               uint32_t& byte, uint32_t (&w)[2], double& err) {
+    byte = c.st_ok ? e4m3_ru(__fdiv_rn(amax, __fmul_rn(target, c.s_t))) : 0u;
+    const float inv = c.tab[byte];
+    err = 0.0;
+    if (inv != inv) {                       // degenerate scale: every code is +0
+        w[0] = w[1] = 0u;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const double d = (double)v[i];
+            err = __dadd_rn(err, __dmul_rn(d, d));
+        }
+        return;
+    }
+    const double S = (double)__fmul_rn(e4m3_value(byte), c.s_t);
+    const float2 iv = make_float2(inv, inv);
+#pragma unroll
+    for (int g = 0; g < 2; ++g) {
+        float q[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 m = mul2_rn(make_float2(v[8 * g + 2 * i], v[8 * g + 2 * i + 1]), iv);
+            q[2 * i] = m.x;
+            q[2 * i + 1] = m.y;
+        }
+        w[g] = e2m1_pack8(q);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const double d = __dsub_rn((double)v[8 * g + i], __dmul_rn((double)e2m1_value((w[g] >> (4 * i)) & 15u), S));
+            err = __dadd_rn(err, __dmul_rn(d, d));
+        }
+    }
+}
+
+// 4/6 block scaling of one NVFP4 block: the rounded-up candidate mapping the
+// block max to 4 replaces the one mapping it to 6 when its squared error is
+// strictly smaller.
+__device__ __forceinline__ void nv_block46(const float (&v)[16], const NvCtx& c, uint32_t& byte, uint32_t (&w)[2]) {
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    uint32_t b6, b4, w6[2], w4[2];
+    double e6, e4;
+    nv46_candidate(v, c, amax, 6.0f, b6, w6, e6);
+    nv46_candidate(v, c, amax, 4.0f, b4, w4, e4);
+    const bool four = e4 < e6;
+    byte = four ? b4 : b6;
+    w[0] = four ? w4[0] : w6[0];
+    w[1] = four ? w4[1] : w6[1];
+}
+
 // One MXFP4 block of 32 with the optional per-column multiplier and block
 // Hadamard-32.  Values are held as pairs P_j = (v_j, v_{j+16}), so the
 // butterflies of strides 1, 2, 4 and 8 (pairs j, j+h with both j, j+h < 16)
@@ -196,7 +252,7 @@ __device__ __forceinline__ void mx_block(const float (&v)[32], const float* chan
     }
 }
 
-template <int BLK, bool BF16, bool TC, bool RU, bool HAD, bool CHAN>
+template <int BLK, bool BF16, bool TC, bool RU, bool HAD, bool CHAN, bool S46 = false>
 __global__ void __launch_bounds__(qz::THREADS, 1)
     quantize_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmC, QuantParams p,
                     int codes_tma) {
@@ -311,7 +367,8 @@ __global__ void __launch_bounds__(qz::THREADS, 1)
             uint32_t byte;
             uint32_t w[BLK / 8];
             if constexpr (BLK == 16) {
-                nv_block<RU>(v[k], sc, byte, w);
+                if constexpr (S46) nv_block46(v[k], sc, byte, w);
+                else nv_block<RU>(v[k], sc, byte, w);
             } else {
                 const float* chan = (CHAN && col < p.cols) ? p.chan + col : nullptr;
                 mx_block<RU, HAD>(v[k], chan, byte, w);
@@ -716,10 +773,10 @@ struct QuantMaps {
     int codes_tma;
 };
 
-template <int BLK, bool BF16, bool TC, bool RU, bool HAD, bool CHAN>
+template <int BLK, bool BF16, bool TC, bool RU, bool HAD, bool CHAN, bool S46 = false>
 static cudaError_t launch_quant_one(const QuantParams& p, const QuantMaps& m, int num_sms, cudaStream_t st) {
     using G = QzGeom<BLK, BF16>;
-    auto k = quantize_kernel<BLK, BF16, TC, RU, HAD, CHAN>;
+    auto k = quantize_kernel<BLK, BF16, TC, RU, HAD, CHAN, S46>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM);
     if (e != cudaSuccess) return e;
     const int64_t tiles = ((p.rows + G::ROWS - 1) / G::ROWS) * p.catoms;
@@ -739,8 +796,9 @@ static cudaError_t launch_quant_mx_variants(const QuantParams& p, const QuantMap
 
 template <int BLK, bool BF16, bool TC>
 static cudaError_t launch_quant_ru(const QuantParams& p, const QuantMaps& m, bool ru, bool had, bool chan,
-                                   int num_sms, cudaStream_t st) {
+                                   bool s46, int num_sms, cudaStream_t st) {
     if constexpr (BLK == 16) {
+        if (s46) return launch_quant_one<BLK, BF16, TC, true, false, false, true>(p, m, num_sms, st);
         if (ru) return launch_quant_one<BLK, BF16, TC, true, false, false>(p, m, num_sms, st);
         return launch_quant_one<BLK, BF16, TC, false, false, false>(p, m, num_sms, st);
     } else {
@@ -751,7 +809,7 @@ static cudaError_t launch_quant_ru(const QuantParams& p, const QuantMaps& m, boo
 
 template <int BLK>
 static cudaError_t launch_quant_blk(const QuantParams& p, bool bf16, bool tc, bool ru, bool had, bool chan,
-                                    int num_sms, cudaStream_t st) {
+                                    bool s46, int num_sms, cudaStream_t st) {
     QuantMaps m;
     std::memset(&m, 0, sizeof(m));
     const int esz = bf16 ? 2 : 4;
@@ -767,18 +825,18 @@ static cudaError_t launch_quant_blk(const QuantParams& p, bool bf16, bool tc, bo
                        (uint64_t)(p.cols / 2), (uint32_t)(2 * BLK), (uint32_t)rows_tile, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
     if (bf16) {
-        if (tc) return launch_quant_ru<BLK, true, true>(p, m, ru, had, chan, num_sms, st);
-        return launch_quant_ru<BLK, true, false>(p, m, ru, had, chan, num_sms, st);
+        if (tc) return launch_quant_ru<BLK, true, true>(p, m, ru, had, chan, s46, num_sms, st);
+        return launch_quant_ru<BLK, true, false>(p, m, ru, had, chan, s46, num_sms, st);
     }
-    if (tc) return launch_quant_ru<BLK, false, true>(p, m, ru, had, chan, num_sms, st);
-    return launch_quant_ru<BLK, false, false>(p, m, ru, had, chan, num_sms, st);
+    if (tc) return launch_quant_ru<BLK, false, true>(p, m, ru, had, chan, s46, num_sms, st);
+    return launch_quant_ru<BLK, false, false>(p, m, ru, had, chan, s46, num_sms, st);
 }
 
 cudaError_t launch_quantize(const QuantParams& p, int blk, bool bf16, bool tc, bool ru, bool had,
-                            bool chan, cudaStream_t st, int num_sms) {
+                            bool chan, bool s46, cudaStream_t st, int num_sms) {
     if (p.rows == 0 || p.cols == 0) return cudaSuccess;
-    if (blk == 16) return launch_quant_blk<16>(p, bf16, tc, ru, had, chan, num_sms, st);
-    return launch_quant_blk<32>(p, bf16, tc, ru, had, chan, num_sms, st);
+    if (blk == 16) return launch_quant_blk<16>(p, bf16, tc, ru, had, chan, s46, num_sms, st);
+    return launch_quant_blk<32>(p, bf16, tc, ru, had, chan, false, num_sms, st);
 }
 
 cudaError_t read_clear_quant_error(unsigned int* word) { return read_clear_module_error(word); }

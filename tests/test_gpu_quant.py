@@ -194,3 +194,47 @@ def test_mxfp4_activation_quantize_full_size():
     oc, os_ = oracle.mxfp4_quantize(x32, d["t"], hadamard=True)
     assert np.array_equal(host(gc), oc)
     assert np.array_equal(host(gs), oracle.scales_to_tc(os_))
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("tc", [False, True])
+@pytest.mark.parametrize("shape", [(200, 336), (128, 1024), (1, 16), (300, 1056)])
+def test_nvfp4_scale46_parity(dtype, tc, shape):
+    """4/6 block scaling: codes and the chosen scales bit for bit (the choice is
+    a binary64 squared-error comparison on both sides)."""
+    rows, cols = shape
+    x = synth.small_like("weight", rows * 5 + cols, rows, cols)
+    if dtype == "bf16":
+        xt = synth.to_bf16(x)
+        x32 = synth.bf16_to_f32(xt)
+        x_t = dev(xt)
+    else:
+        x32 = x
+        x_t = dev(x)
+    s_t = oracle.tensor_scale(oracle.amax(x32), 1536.0)
+    flags = q4.SCALE_46 | (q4.LAYOUT_TC if tc else 0)
+    gc, gs = q4.q4_quantize(q4.NVFP4, x_t, gscale=gscale_dev(s_t), flags=flags)
+    oc, os_ = oracle.nvfp4_quantize46(x32, s_t)
+    assert np.array_equal(host(gc), oc)
+    if tc:
+        assert np.array_equal(host(gs), oracle.scales_to_tc(os_))
+    else:
+        assert np.array_equal(host(gs).reshape(os_.shape), os_)
+
+
+def test_scale46_sigma_delta_chain():
+    """Sigma-Delta on 4/6 block scales (the page's block_scale_46(W) feeding the
+    loop): eight visits bit for bit, residues within |r| <= 1."""
+    w = synth.small_like("weight", 77, 256, 512)
+    s_t = oracle.tensor_scale(oracle.amax(w), 1536.0)
+    g_t = gscale_dev(s_t)
+    _, g_sc = q4.q4_quantize(q4.NVFP4, dev(w), gscale=g_t, flags=q4.SCALE_46 | q4.LAYOUT_TC)
+    _, o_sc = oracle.nvfp4_quantize46(w, s_t)
+    r_g = torch.zeros((256, 512), dtype=torch.float32, device=DEV)
+    r_o = np.zeros((256, 512), np.float32)
+    for _ in range(8):
+        gc = q4.q4_sigma_delta_step(q4.NVFP4, dev(w), g_sc, r_g, gscale=g_t)
+        oc = oracle.sigma_delta_step(q4.NVFP4, w, o_sc, s_t, r_o)
+        assert np.array_equal(host(gc), oc)
+    assert np.array_equal(host(r_g).view(np.uint32), r_o.view(np.uint32))
+    assert np.abs(r_o).max() <= 1.0 + 2 ** -20
