@@ -273,13 +273,16 @@ def rows_bench(q4, dev, flush, pk, reps=30):
                                         "vs_32_separate_visits": ms_sd * 32 / ms_cb}
     del banks
 
+    q46_out = [(torch.empty_like(c), torch.empty_like(sc)) for wt, sc, g, r, c, _ in mats]
+
     def q46():
-        for wt, sc, g, r, c, _ in mats:
-            q4.q4_quantize(q4.NVFP4, wt, gscale=g, flags=q4.SCALE_46 | q4.LAYOUT_TC, codes=c, scales=sc)
+        for (wt, sc, g, r, c, _), (c46, s46) in zip(mats, q46_out):
+            q4.q4_quantize(q4.NVFP4, wt, gscale=g, flags=q4.SCALE_46 | q4.LAYOUT_TC, codes=c46, scales=s46)
     ms_46, _ = time_fn(q46, reps, flush)
     gbs = nw * (4 + 0.5 + 1 / 16) / (ms_46 * 1e-3) / 1e9
     out["nvfp4_quantize46_looped_weights"] = {"weights": nw, "matrices": 13, "us": ms_46 * 1e3, "GB/s": gbs,
                                               "frac_hbm": gbs / hbm}
+    del q46_out
 
     def sr_visit():
         for wt, sc, g, r, c, _ in mats:
