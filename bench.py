@@ -290,6 +290,26 @@ def rows_bench(q4, dev, flush, pk, reps=30):
     ms_sr, _ = time_fn(sr_visit, reps, flush)
     gbs = nw * B_SR / (ms_sr * 1e-3) / 1e9
     out["sr_requant_visit"] = {"weights": nw, "matrices": 13, "us": ms_sr * 1e3, "GB/s": gbs, "frac_hbm": gbs / hbm}
+    # a decode-shaped visit (M = 16) with the Sigma-Delta codes generated inside the
+    # GEMM producer, against the same visit as a separate step + W4A16 GEMM
+    xd16 = xl[:16].contiguous()
+    yd16 = [torch.empty((16, wt.shape[0]), dtype=torch.bfloat16, device=dev) for wt, *_ in mats]
+
+    def fused16():
+        for (wt, sc, g, r, c, _), yy in zip(mats, yd16):
+            q4.q4_sigma_delta_gemm(q4.NVFP4, xd16, wt, sc, r, g, y=yy)
+
+    def unfused16():
+        for (wt, sc, g, r, c, _), yy in zip(mats, yd16):
+            q4.q4_sigma_delta_step(q4.NVFP4, wt, sc, r, gscale=g, codes=c)
+            q4.q4_gemm(q4.NVFP4, 16, wt.shape[0], Kl, xd16, None, None, c, sc, g, y=yy, a_kind=q4.A_BF16_W4A16)
+    ms_f, _ = time_fn(fused16, reps, flush)
+    ms_u, _ = time_fn(unfused16, reps, flush)
+    gbs = nw * 12.0 / (ms_f * 1e-3) / 1e9
+    out["sigma_delta_fused_gemm_m16"] = {"weights": nw, "matrices": 13, "M": 16, "us": ms_f * 1e3, "GB/s": gbs,
+                                         "frac_hbm": gbs / hbm, "B_per_weight": 12.0,
+                                         "unfused_us": ms_u * 1e3, "speedup_vs_unfused": ms_u / ms_f}
+    del xd16, yd16
     ms_v, _ = time_fn(visit, max(5, reps // 3), flush)
     out["looped_visit"] = {"us": ms_v * 1e3, "us_R32": ms_v * 1e3 * 32,
                            "note": "Sigma-Delta requant of all 13 weights + 13 W4A16 GEMMs"}

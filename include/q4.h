@@ -257,6 +257,25 @@ Q4_API q4_status q4_gemm(q4_format format, int block, int64_t M, int64_t N, int6
  *   workspace.  K % 64 == 0, N % 8 == 0.
  */
 
+/*
+ * q4_sigma_delta_gemm -- one loop visit with the Sigma-Delta code generation
+ *   fused into the GEMM's weight producer ("Looped Transformer quantization",
+ *   sec. 4: online code generation from the reference weight and the residue
+ *   state at every visit): with the NVFP4 block scales fixed,
+ *     q = E2M1(w * inv + r),  r <- (w * inv + r) - q   (as q4_sigma_delta_step)
+ *     Y = s_t * X (q * s_b)^T                          (as the W4A16 q4_gemm)
+ *   without writing the codes: each weight element and its residue are read
+ *   once and the residue is written back.  Decode shapes: M <= 16 (else
+ *   Q4_ERR_UNSUPPORTED).  NVFP4 only; scales must be in the tensor-core layout
+ *   (flags = Q4_LAYOUT_TC).  x: bf16 [M, K]; w: float [N, K]; residue: float
+ *   [N, K], read and written (zero = start of a chain); y: [M, N] of out_dt.
+ *   K % 64 == 0, N % 8 == 0.
+ */
+Q4_API q4_status q4_sigma_delta_gemm(q4_format format, int block, int64_t M, int64_t N, int64_t K,
+                              const void* x, const float* w, const uint8_t* scales,
+                              const float* d_gscale, float* residue, q4_dtype out_dt, void* y,
+                              int flags, void* stream);
+
 /* Scratch bytes q4_gemm needs for these arguments (0 when none). */
 Q4_API size_t q4_gemm_workspace_size(q4_format format, int64_t M, int64_t N, int64_t K,
                               int a_kind);

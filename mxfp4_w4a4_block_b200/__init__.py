@@ -9,7 +9,8 @@ there is no CPU fallback, and importing fails loudly if the library has not
 been built (``python -m mxfp4_w4a4_block_b200.build``).
 
 Function names mirror the C entry points: q4_amax, q4_quantize,
-q4_dequantize, q4_sigma_delta_step, q4_sigma_delta_codebanks, q4_sr_requant, q4_gemm,
+q4_dequantize, q4_sigma_delta_step, q4_sigma_delta_codebanks, q4_sr_requant,
+q4_sigma_delta_gemm, q4_gemm,
 q4_gemm_workspace_size, q4_get_device_error, q4_scale_bytes (tail_bank is a
 pure indexing helper of the reverse-order codebank schedule).
 """
@@ -57,6 +58,7 @@ SIGNATURES = {
     "q4_dequantize": (_I, [_I, _I, _P, _P, _P, _I64, _I64, _I, _I, _P, _P]),
     "q4_sigma_delta_step": (_I, [_I, _I, _P, _I64, _I64, _P, _P, _P, _P, _I, _P]),
     "q4_sigma_delta_codebanks": (_I, [_I, _I, _P, _I64, _I64, _P, _P, _I, _P, _P, _I, _P]),
+    "q4_sigma_delta_gemm": (_I, [_I, _I, _I64, _I64, _I64, _P, _P, _P, _P, _P, _I, _P, _I, _P]),
     "q4_sr_requant": (_I, [_I, _I, _P, _I64, _I64, _P, _P, ctypes.c_uint64, ctypes.c_uint32, _P, _I, _P]),
     "q4_gemm": (_I, [_I, _I, _I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _P, _I, _P, _P, _SZ, _P]),
     "q4_gemm_workspace_size": (_SZ, [_I, _I64, _I64, _I64, _I]),
@@ -209,6 +211,21 @@ def q4_sr_requant(fmt: int, w: torch.Tensor, scales: torch.Tensor, seed: int, vi
                              _ptr(codes), flags, _stream(stream))
     _check("q4_sr_requant", st)
     return codes
+
+
+def q4_sigma_delta_gemm(fmt: int, x: torch.Tensor, w: torch.Tensor, scales: torch.Tensor, residue: torch.Tensor,
+                        gscale: torch.Tensor, out_dtype=torch.bfloat16, y: torch.Tensor | None = None,
+                        flags: int = LAYOUT_TC, stream=None) -> torch.Tensor:
+    """One looped-core visit with the Sigma-Delta codes generated inside the
+    GEMM: updates `residue` in place and returns Y = s_t X (q s_b)^T."""
+    M, K = x.shape
+    N = w.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=out_dtype, device=x.device)
+    st = lib().q4_sigma_delta_gemm(fmt, BLOCK[fmt], M, N, K, _ptr(x), _ptr(w), _ptr(scales), _ptr(gscale),
+                                   _ptr(residue), _dtype_code(y), _ptr(y), flags, _stream(stream))
+    _check("q4_sigma_delta_gemm", st)
+    return y
 
 
 def tail_bank(banks: torch.Tensor, j: int) -> torch.Tensor:

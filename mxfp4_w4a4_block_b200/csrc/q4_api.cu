@@ -174,6 +174,25 @@ q4_status q4_sigma_delta_step(q4_format format, int block, const float* w, int64
                                               num_sms()));
 }
 
+q4_status q4_sigma_delta_gemm(q4_format format, int block, int64_t M, int64_t N, int64_t K, const void* x,
+                              const float* w, const uint8_t* scales, const float* d_gscale, float* residue,
+                              q4_dtype out_dt, void* y, int flags, void* stream) {
+    if (!valid_format(format) || !valid_dtype(out_dt) || M < 0 || N < 0 || K < 0) return Q4_ERR_ARG;
+    if (block != block_of(format)) return Q4_ERR_UNSUPPORTED;
+    if (format != Q4_NVFP4 || !(flags & Q4_LAYOUT_TC) || (flags & ~Q4_LAYOUT_TC)) return Q4_ERR_UNSUPPORTED;
+    if (!d_gscale) return Q4_ERR_ARG;
+    if (K % 64 || N % 8) return Q4_ERR_SHAPE;
+    if (M == 0 || N == 0 || K == 0) return M == 0 || N == 0 ? Q4_OK : Q4_ERR_SHAPE;
+    if (!q4::sd_gemm_supported(M, K)) return Q4_ERR_UNSUPPORTED;
+    if (!x || !w || !scales || !residue || !y) return Q4_ERR_ARG;
+    if (!aligned16(x) || !aligned16(w) || !aligned16(scales) || !aligned16(residue) || !aligned16(y))
+        return Q4_ERR_ALIGN;
+    q4::SdGemmParams p;
+    p.M = M; p.N = N; p.K = K; p.x = x; p.w = w; p.scales = scales; p.gscale = d_gscale; p.residue = residue;
+    p.y = y; p.out_bf16 = out_dt == Q4_BF16;
+    return cuda_status(q4::launch_sd_gemm(p, (cudaStream_t)stream, num_sms()));
+}
+
 size_t q4_gemm_workspace_size(q4_format format, int64_t M, int64_t N, int64_t K, int a_kind) {
     (void)N;
     if (a_kind != Q4_A_BF16 || format != Q4_NVFP4 || M <= 0 || K <= 0 || K % 64) return 0;

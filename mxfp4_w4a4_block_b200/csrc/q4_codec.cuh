@@ -26,6 +26,17 @@ __device__ __forceinline__ uint32_t e2m1_pack8(const float (&v)[8]) {
     return out;
 }
 
+// Four E2M1 codes (element 0 in the low nibble) of four floats.
+__device__ __forceinline__ uint32_t e2m1_pack4(float a, float b, float c, float d) {
+    uint32_t out;
+    asm("{\n\t.reg .b8 b0, b1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "mov.b32 %0, {b0, b1, 0, 0};\n\t}"
+        : "=r"(out) : "f"(a), "f"(b), "f"(c), "f"(d));
+    return out;
+}
+
 // Magnitude of an E2M1 code (low three bits) as float: 0, .5, 1, 1.5, 2, 3, 4, 6.
 __device__ __forceinline__ float e2m1_value(uint32_t code) {
     // twice the magnitudes, one nibble each: 0,1,2,3,4,6,8,12

@@ -1213,6 +1213,299 @@ cudaError_t launch_w4a16(const W4A16Params& p, cudaStream_t st, int num_sms) {
     return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ Sigma-Delta fused into the GEMM producer
+// One loop visit of the looped core with the code generation moved into the
+// GEMM ("Looped Transformer quantization", sec. 4: codes generated online from
+// the reference weight and the residue state at every visit): for a small
+// batch X (M <= 16 bf16 rows) and the FP32 master weight W [N, K] with fixed
+// NVFP4 block scales,
+//     q = E2M1(W * inv + r),  r <- (W * inv + r) - q,  Y = s_t * X (q * s_b)^T,
+// where the codes q never leave the chip: each weight element is read once
+// with its residue, the new residue is written back, and the dequantized
+// weight q * s_b (exact in bf16) is the tensor-core operand.  The product is
+// W4A16-style (bf16 activations) and operands are swapped so the weight fills
+// the MMA's 128-row side (tcgen05 kind::f16, 128 x 16 x 16).
+// A CTA owns 128 weight rows and one slice of K; the KS slices of a row band
+// form a thread-block cluster whose partial outputs are summed through
+// distributed shared memory by the cluster's first CTA:
+//   warp 0      TMA producer: per k-stage of 64 the W and r tiles (two
+//               128-row x 128-byte boxes each, 128-byte swizzle), the block
+//               scale atom and the X tile (np rows x 128 bytes, swizzled);
+//   warp 1      TMEM owner and MMA issuer;
+//   warps 2..5  Sigma-Delta: thread = weight row; the new residue replaces the
+//               old one in the stage (then one TMA store per box) and the
+//               dequantized bf16 row goes to the swizzled A operand tile;
+//   warps 6..9  epilogue: accumulator -> shared memory, cluster reduction,
+//               Y = s_t * sum by the cluster's first CTA.
+namespace sdg {
+constexpr int BM = 128;
+constexpr int KSTAGE = 64;
+constexpr int STAGES = 2;
+constexpr int OFF_W = 0;                 // 2 boxes x 16 KB fp32
+constexpr int OFF_R = 32768;             // 2 boxes x 16 KB fp32
+constexpr int OFF_A = 65536;             // 128 x 128 B bf16 operand
+constexpr int OFF_X = 81920;             // 16 x 128 B bf16 operand
+constexpr int OFF_SF = OFF_X + 2048;     // one scale atom
+constexpr int STAGE = 85 * 1024;
+constexpr int OFF_RED = STAGES * STAGE;  // fp32 partial tile [128][16]
+constexpr int OFF_BAR = OFF_RED + BM * 16 * 4;
+constexpr int SMEM_BYTES = OFF_BAR + 1024 + 1024;
+constexpr int CONV_WARPS = 4;
+constexpr int EPI_WARPS = 4;
+constexpr int THREADS = 32 * (2 + CONV_WARPS + EPI_WARPS);
+constexpr uint32_t TMEM_COLS = 32;
+constexpr int MAX_KS = 8;
+}  // namespace sdg
+
+struct SdgDev {
+    int64_t M, N, K;
+    const uint8_t* scales;   // tensor-core layout
+    const float* gscale;
+    void* y;
+    int64_t catoms;
+    int kslice;              // K elements per CTA (a multiple of 64)
+    int out_bf16;
+};
+
+__device__ __forceinline__ float ld_shared_cluster_f32(uint32_t addr) {
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+    return v;
+}
+
+__global__ void __launch_bounds__(sdg::THREADS, 1)
+    sd_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmR,
+                          const __grid_constant__ CUtensorMap tmX, SdgDev p) {
+    using namespace sdg;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);   // [STAGES] W, r, X, scales landed
+    uint64_t* conv = full + STAGES;                                 // [STAGES] residue + operand written
+    uint64_t* empty = conv + STAGES;                                // [STAGES] MMAs done + residue stored
+    uint64_t* tmem_full = empty + STAGES;
+    uint64_t* mma_done = tmem_full + 1;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
+    float* inv_tab = reinterpret_cast<float*>(smem + OFF_BAR + 512);   // 128 entries
+    float* red = reinterpret_cast<float*>(smem + OFF_RED);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();                        // K slice of this CTA
+    const int64_t row0 = (int64_t)blockIdx.y * BM;
+    const int64_t k_begin = (int64_t)rank * p.kslice;
+    const int nst = p.kslice / KSTAGE;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&conv[s], CONV_WARPS);
+            mbar_init(&empty[s], 2);                                // MMA commit + residue-store release
+        }
+        mbar_init(tmem_full, 1);
+        mbar_init(mma_done, 1);
+        fence_mbar_init();
+    }
+    if (warp == 1) { tmem_alloc(tmem_holder, TMEM_COLS); tmem_relinquish(); }
+    if (warp == 0 && lane == 0) { tma_prefetch_desc(&tmW); tma_prefetch_desc(&tmR); tma_prefetch_desc(&tmX); }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            uint32_t phase = 0;
+            int stage = 0;
+            uint32_t last_phase[STAGES];
+            bool issued[STAGES] = {false, false};
+            for (int i = 0; i < nst; ++i) {
+                if (!mbar_wait(&empty[stage], phase ^ 1)) break;
+                uint8_t* st = smem + stage * STAGE;
+                const int32_t k0 = (int32_t)(k_begin + (int64_t)i * KSTAGE);
+                mbar_arrive_expect_tx(&full[stage], 2 * 2 * 16384 + 2048 + 512);
+                for (int b = 0; b < 2; ++b) {
+                    tma_load_2d(st + OFF_W + b * 16384, &tmW, &full[stage], k0 + 32 * b, (int32_t)row0);
+                    tma_load_2d(st + OFF_R + b * 16384, &tmR, &full[stage], k0 + 32 * b, (int32_t)row0);
+                }
+                tma_load_2d(st + OFF_X, &tmX, &full[stage], k0, 0);
+                bulk_load(st + OFF_SF, p.scales + ((int64_t)blockIdx.y * p.catoms + k0 / 64) * 512, 512u,
+                          &full[stage]);
+                issued[stage] = true;
+                last_phase[stage] = phase;
+                if (++stage == STAGES) { stage = 0; phase ^= 1; }
+            }
+            for (int s = 0; s < STAGES; ++s)
+                if (issued[s]) mbar_wait(&full[s], last_phase[s]);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16(BM, 16);
+            uint32_t phase = 0;
+            int stage = 0;
+            bool ok = true;
+            for (int i = 0; i < nst; ++i) {
+                if (!mbar_wait(&full[stage], phase) || !mbar_wait(&conv[stage], phase)) { ok = false; break; }
+                tc_fence_after();
+                uint8_t* st = smem + stage * STAGE;
+                const uint64_t ad = smem_desc(smem_u32(st + OFF_A), 16, 1024, 2);
+                const uint64_t bd = smem_desc(smem_u32(st + OFF_X), 16, 1024, 2);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) mma_bf16(tmem, ad + 2 * kk, bd + 2 * kk, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+                tc_commit(&empty[stage]);
+                if (++stage == STAGES) { stage = 0; phase ^= 1; }
+            }
+            if (ok) tc_commit(tmem_full);
+            tc_commit(mma_done);
+            mbar_wait(mma_done, 0);
+        }
+    } else if (warp < 2 + CONV_WARPS) {
+        // ---- Sigma-Delta on weight row rr of each stage
+        const int rr = threadIdx.x - 64;
+        constexpr int CT = 32 * CONV_WARPS;
+        const float s_t = *p.gscale;
+        nv_fill_table(s_t, inv_tab, rr, CT);
+        named_barrier(1, CT);
+        const bool row_ok = row0 + rr < p.N;
+        uint32_t phase = 0;
+        int stage = 0;
+        for (int i = 0; i < nst; ++i) {
+            const bool got = mbar_wait(&full[stage], phase);
+            uint8_t* st = smem + stage * STAGE;
+            const uint32_t sw = *reinterpret_cast<const uint32_t*>(st + OFF_SF + (rr & 31) * 16 + ((rr >> 5) & 3) * 4);
+            uint8_t* arow = st + OFF_A + (rr >> 3) * 1024 + (rr & 7) * 128;
+#pragma unroll
+            for (int b = 0; b < 2; ++b) {
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    // elements e = 32b + 4c .. +3 of the stage, block j = e / 16
+                    const int j = 2 * b + (c >> 2);
+                    const uint32_t sb = (sw >> (8 * j)) & 0xFFu;
+                    const float inv = inv_tab[sb & 0x7Fu];
+                    const uint32_t off = (uint32_t)(b * 16384 + rr * 128 + ((c ^ (rr & 7)) << 4));
+                    const float4 w4 = *reinterpret_cast<const float4*>(st + OFF_W + off);
+                    float4* rp = reinterpret_cast<float4*>(st + OFF_R + off);
+                    const float4 r4 = *rp;
+                    float2 x01, x23;
+                    if (inv != inv) {
+                        x01 = make_float2(0.0f, 0.0f);
+                        x23 = x01;
+                    } else {
+                        x01 = mul2_rn(make_float2(w4.x, w4.y), make_float2(inv, inv));
+                        x23 = mul2_rn(make_float2(w4.z, w4.w), make_float2(inv, inv));
+                    }
+                    const float2 v01 = add2_rn(x01, make_float2(r4.x, r4.y));
+                    const float2 v23 = add2_rn(x23, make_float2(r4.z, r4.w));
+                    const uint32_t codes = e2m1_pack4(v01.x, v01.y, v23.x, v23.y);
+                    const float2 q01 = e2m1x2_value(codes & 0xFFu), q23 = e2m1x2_value(codes >> 8);
+                    const float2 n01 = sub2_rn(v01, q01), n23 = sub2_rn(v23, q23);
+                    *rp = make_float4(n01.x, n01.y, n23.x, n23.y);
+                    // dequantized weight q * s_b (exact in bf16), 4 elements = 8 bytes
+                    const float sv = e4m3_value(sb & 0x7Fu);
+                    uint32_t d0, d1;
+                    asm("cvt.rn.bf16x2.f32 %0, %2, %1;" : "=r"(d0) : "f"(q01.x * sv), "f"(q01.y * sv));
+                    asm("cvt.rn.bf16x2.f32 %0, %2, %1;" : "=r"(d1) : "f"(q23.x * sv), "f"(q23.y * sv));
+                    if (!row_ok) d0 = d1 = 0u;
+                    const int e2 = 64 * b + 8 * c;        // byte offset of the 4 bf16 in the 128-byte row
+                    *reinterpret_cast<uint2*>(arow + ((((e2 >> 4) ^ (rr & 7)) & 7) << 4) + (e2 & 15)) =
+                        make_uint2(d0, d1);
+                }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&conv[stage]);
+            // every row is done: store the new residue tile, release the stage once it is read
+            named_barrier(1, CT);
+            if (rr == 0) {
+                if (got) {
+                    const int32_t k0 = (int32_t)(k_begin + (int64_t)i * KSTAGE);
+                    for (int b = 0; b < 2; ++b) tma_store_2d(&tmR, st + OFF_R + b * 16384, k0 + 32 * b, (int32_t)row0);
+                    bulk_commit_group();
+                    bulk_wait_read_all();
+                }
+                mbar_arrive(&empty[stage]);
+            }
+            if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (rr == 0) bulk_wait_all();
+    } else {
+        // ---- epilogue: partial tile to shared memory, cluster reduction
+        const int quad = warp & 3;
+        const int rr = quad * 32 + lane;
+        const bool ok = mbar_wait(tmem_full, 0);
+        tc_fence_after();
+        uint32_t v[16];
+        tmem_ld16(tmem + ((uint32_t)(quad * 32) << 16), v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int m = 0; m < 16; ++m) red[rr * 16 + m] = ok ? __uint_as_float(v[m]) : 0.0f;
+    }
+    // every CTA's partial tile is in its shared memory
+    __syncthreads();
+    cluster_sync();
+    if (warp >= 2 + CONV_WARPS && rank == 0) {
+        const int quad = warp & 3;
+        const int rr = quad * 32 + lane;
+        const int64_t n = row0 + rr;
+        const float s_t = *p.gscale;
+        const uint32_t ks = (uint32_t)(p.K / p.kslice);
+        for (int m = 0; m < p.M; ++m) {
+            float acc = red[rr * 16 + m];
+            for (uint32_t q = 1; q < ks; ++q) acc += ld_shared_cluster_f32(mapa_shared(smem_u32(&red[rr * 16 + m]), q));
+            const float val = acc * s_t;
+            if (n < p.N) {
+                if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.y)[(int64_t)m * p.N + n] = __float2bfloat16_rn(val);
+                else reinterpret_cast<float*>(p.y)[(int64_t)m * p.N + n] = val;
+            }
+        }
+    }
+    // the first CTA has read every partial tile before any CTA leaves
+    __syncthreads();
+    cluster_sync();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
+}
+
+bool sd_gemm_supported(int64_t M, int64_t K) { return M >= 1 && M <= 16 && K % 64 == 0 && K > 0; }
+
+cudaError_t launch_sd_gemm(const SdGemmParams& p, cudaStream_t st, int num_sms) {
+    using namespace sdg;
+    if (p.M == 0 || p.N == 0) return cudaSuccess;
+    const int64_t tiles = (p.N + BM - 1) / BM;
+    // K slices per row band: enough CTAs to cover the GPU, at most 8 (a portable cluster)
+    int ks = 1;
+    while (ks < MAX_KS && tiles * ks * 2 <= num_sms && p.K % (64 * (ks * 2)) == 0) ks *= 2;
+    CUtensorMap mw, mr, mx;
+    if (!encode_map_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, p.w, (uint64_t)p.K, (uint64_t)p.N, (uint64_t)p.K * 4, 32u,
+                       (uint32_t)BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_map_2d(&mr, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, p.residue, (uint64_t)p.K, (uint64_t)p.N,
+                       (uint64_t)p.K * 4, 32u, (uint32_t)BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_map_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.x, (uint64_t)p.K, (uint64_t)p.M, (uint64_t)p.K * 2, 64u,
+                       16u, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    SdgDev d;
+    d.M = p.M; d.N = p.N; d.K = p.K; d.scales = p.scales; d.gscale = p.gscale; d.y = p.y;
+    d.catoms = ((p.K / 16) + 3) / 4;
+    d.kslice = (int)(p.K / ks);
+    d.out_bf16 = p.out_bf16 ? 1 : 0;
+    cudaError_t e = cudaFuncSetAttribute(sd_gemm_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)ks, (unsigned)tiles, 1);
+    cfg.blockDim = dim3(THREADS, 1, 1);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)ks;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, sd_gemm_decode_kernel, mw, mr, mx, d);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
 // ------------------------------------------------------------------ fused decode
 // Small-M GEMM (M <= 64) with the activation quantization inside the kernel:
 // no bf16 activation round trip and no workspace.  Operands are swapped so the

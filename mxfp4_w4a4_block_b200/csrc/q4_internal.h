@@ -73,6 +73,20 @@ struct W4A16Params {
 };
 
 cudaError_t launch_w4a16(const W4A16Params& p, cudaStream_t st, int num_sms);
+
+struct SdGemmParams {
+    int64_t M, N, K;
+    const void* x;            // [M, K] bf16 activations, M <= 16
+    const float* w;           // [N, K] fp32 master weight
+    const uint8_t* scales;    // NVFP4 block scales, tensor-core layout
+    const float* gscale;      // s_t
+    float* residue;           // [N, K] fp32, read and written
+    void* y;                  // [M, N]
+    bool out_bf16;
+};
+
+bool sd_gemm_supported(int64_t M, int64_t K);
+cudaError_t launch_sd_gemm(const SdGemmParams& p, cudaStream_t st, int num_sms);
 cudaError_t launch_amax(const void* x, int64_t n, bool bf16, float denom, float* d_out,
                         cudaStream_t st, int num_sms);
 cudaError_t launch_quantize(const QuantParams& p, int blk, bool bf16, bool tc, bool ru, bool had,

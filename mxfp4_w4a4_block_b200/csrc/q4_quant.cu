@@ -435,17 +435,6 @@ constexpr int SMEM = BAR_OFF + 256 + 1024;
 constexpr int GPT = ROWS * COLS / 4 / CONSUMERS; // 4-weight groups per thread per tile
 }  // namespace sdk
 
-// Four E2M1 codes (element 0 in the low nibble) of four floats.
-__device__ __forceinline__ uint32_t e2m1_pack4(float a, float b, float c, float d) {
-    uint32_t out;
-    asm("{\n\t.reg .b8 b0, b1;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
-        "mov.b32 %0, {b0, b1, 0, 0};\n\t}"
-        : "=r"(out) : "f"(a), "f"(b), "f"(c), "f"(d));
-    return out;
-}
-
 template <int BLK, bool TC>
 __global__ void __launch_bounds__(sdk::THREADS, 1)
     sigma_delta_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmR,

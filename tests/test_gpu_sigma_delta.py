@@ -7,7 +7,7 @@ import torch
 import oracle
 import synth
 import mxfp4_w4a4_block_b200 as q4
-from gpu_util import DEV, dev, gscale_dev, host
+from gpu_util import DEV, GEMM_F32_TOL, dev, gscale_dev, host, rel_fro
 
 pytestmark = pytest.mark.gpu
 
@@ -130,3 +130,42 @@ def test_codebanks_match_successive_steps_and_reverse_tail():
     rtn, _ = q4.q4_quantize(q4.NVFP4, dev(w), gscale=g_t, flags=q4.SCALE_RU | q4.LAYOUT_TC)
     assert torch.equal(q4.tail_bank(banks, K), rtn)
     assert torch.equal(q4.tail_bank(banks, 1), banks[K - 1])
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 392, 320), (16, 1024, 1024), (5, 4096, 1024), (16, 136, 64), (12, 256, 2048)])
+def test_sigma_delta_gemm_fused_producer(M, N, K):
+    """Sigma-Delta fused into the GEMM's weight producer: three visits; the
+    residue bit for bit against the oracle step, Y against the binary64 W4A16
+    oracle on the oracle's own codes of that visit."""
+    w = synth.small_like("weight", M + N + K, N, K)
+    x = synth.to_bf16(synth.small_like("gauss", 3 * M + K, M, K))
+    x32 = synth.bf16_to_f32(x)
+    s_t, g_t, g_sc, o_sc = setup_scales(q4.NVFP4, w)
+    r_gpu = torch.zeros((N, K), dtype=torch.float32, device=DEV)
+    r_orc = np.zeros((N, K), np.float32)
+    w_d, x_d = dev(w), dev(x)
+    for visit in range(3):
+        y = q4.q4_sigma_delta_gemm(q4.NVFP4, x_d, w_d, g_sc, r_gpu, g_t, out_dtype=torch.float32)
+        oc = oracle.sigma_delta_step(q4.NVFP4, w, o_sc, s_t, r_orc)
+        assert np.array_equal(host(r_gpu).view(np.uint32), r_orc.view(np.uint32)), f"residue, visit {visit + 1}"
+        ref = oracle.gemm_w4a16(q4.NVFP4, x32, oc, o_sc, s_t, M, N, K)
+        assert rel_fro(host(y), ref) <= GEMM_F32_TOL
+
+
+def test_sigma_delta_gemm_matches_unfused_path():
+    """The fused visit equals q4_sigma_delta_step followed by the W4A16 q4_gemm
+    (residue bit for bit, outputs to FP32 summation order)."""
+    M, N, K = 16, 4096, 1024
+    w = synth.looped()["w"][-1]
+    x = synth.to_bf16(synth.small_like("gauss", 9, M, K))
+    s_t, g_t, g_sc, _ = setup_scales(q4.NVFP4, w)
+    w_d, x_d = dev(w), dev(x)
+    r1 = torch.zeros((N, K), dtype=torch.float32, device=DEV)
+    r2 = torch.zeros((N, K), dtype=torch.float32, device=DEV)
+    for _ in range(2):
+        y1 = q4.q4_sigma_delta_gemm(q4.NVFP4, x_d, w_d, g_sc, r1, g_t, out_dtype=torch.float32)
+        c = q4.q4_sigma_delta_step(q4.NVFP4, w_d, g_sc, r2, gscale=g_t)
+        y2 = q4.q4_gemm(q4.NVFP4, M, N, K, x_d, None, None, c, g_sc, g_t, out_dtype=torch.float32,
+                        a_kind=q4.A_BF16_W4A16)
+        assert torch.equal(r1, r2)
+        assert rel_fro(host(y1), host(y2).astype(np.float64)) <= 1e-6
