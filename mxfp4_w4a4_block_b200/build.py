@@ -21,6 +21,12 @@ HEADERS = ["q4_internal.h", "q4_codec.cuh", "q4_ptx.cuh"]
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-O3", "-lineinfo", "-std=c++17",
+    # no contraction of a plain multiply and add into one fused operation:
+    # the codecs' decisions depend on every intermediate rounding (intended
+    # fused operations are written as explicit fma).  This does not stop
+    # ptxas from fusing a paired (f32x2) multiply into a paired add, so the
+    # kernels keep the product that feeds such an add scalar where it matters
+    "-fmad=false",
     "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
     "--expt-relaxed-constexpr",
     "-cudart", "static",
@@ -37,7 +43,7 @@ def _stale() -> bool:
     if not LIB.exists():
         return True
     t = LIB.stat().st_mtime
-    deps = [CSRC / s for s in SOURCES + HEADERS] + [INCLUDE / "q4.h"]
+    deps = [CSRC / s for s in SOURCES + HEADERS] + [INCLUDE / "q4.h", Path(__file__)]
     return any(d.stat().st_mtime > t for d in deps)
 
 
@@ -50,7 +56,7 @@ def build(force: bool = False, verbose: bool = False, extra=None) -> Path:
     objs = []
     for src in SOURCES:
         obj = objdir / (Path(src).stem + ".o")
-        cmd = [nvcc(), *NVCC_FLAGS, *(extra or []), "-I", str(INCLUDE), "-dc" if False else "-c",
+        cmd = [nvcc(), *NVCC_FLAGS, *(extra or []), "-I", str(INCLUDE), "-c",
                str(CSRC / src), "-o", str(obj)]
         if verbose:
             print(" ".join(cmd), file=sys.stderr)

@@ -157,6 +157,12 @@ __device__ __forceinline__ float2 mul2_rn(float2 a, float2 b) {
         : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
     return d;
 }
+// Two scalar products rounded to nearest, for a product that feeds an add:
+// ptxas fuses a paired multiply into the paired add that consumes it,
+// rounding modifier or not, while a scalar mul.rn is never contracted.
+__device__ __forceinline__ float2 mul2_sep_rn(float2 a, float2 b) {
+    return make_float2(__fmul_rn(a.x, b.x), __fmul_rn(a.y, b.y));
+}
 __device__ __forceinline__ float2 add2_rn(float2 a, float2 b) {
     float2 d;
     asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"

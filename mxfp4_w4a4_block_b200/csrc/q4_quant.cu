@@ -109,12 +109,14 @@ cudaError_t launch_amax(const void* x, int64_t n, bool bf16, float denom, float*
 // (the scale rule, the Hadamard rotation and the code packing stay in
 // registers), a warp taking 32 consecutive rows of one block column so its
 // swizzled shared-memory reads are conflict-free.  Codes and scale atoms are
-// staged in shared memory and leave by TMA / bulk stores (three staging
-// buffers, so the stores overlap the next tiles).
+// staged in shared memory (three staging buffers) and a store warp sends them
+// out by TMA / bulk stores; the consumer warps hand a finished buffer to it
+// through an mbarrier and go straight on to the next tile, so no consumer
+// ever waits on a CTA-wide barrier or on a store.
 namespace qz {
 constexpr int CONSUMER_WARPS = 16;
 constexpr int CONSUMERS = 32 * CONSUMER_WARPS;
-constexpr int THREADS = CONSUMERS + 32;          // + the producer warp
+constexpr int THREADS = CONSUMERS + 64;          // + the producer warp and the store warp
 constexpr int IN_BYTES = 160 * 1024;             // input stages
 constexpr int NBUF = 3;                          // output staging buffers
 }  // namespace qz
@@ -198,20 +200,24 @@ __device__ __forceinline__ void nv_block46(const float (&v)[16], const NvCtx& c,
 // Hadamard-32.  Values are held as pairs P_j = (v_j, v_{j+16}), so the
 // butterflies of strides 1, 2, 4 and 8 (pairs j, j+h with both j, j+h < 16)
 // are packed f32x2 operations; stride 16 pairs the two halves of each P_j.
-template <bool RU, bool HAD>
-__device__ __forceinline__ void mx_block(const float (&v)[32], const float* chan, uint32_t& byte, uint32_t (&w)[4]) {
+// Channel factors come preloaded in `cw` (PRE) or are read from `chan`
+// (nullptr: none).
+template <bool RU, bool HAD, bool CHAN, bool PRE>
+__device__ __forceinline__ void mx_block(const float (&v)[32], const float4 (&cw)[8], const float* chan, uint32_t& byte,
+                                         uint32_t (&w)[4]) {
     float2 P[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) P[j] = make_float2(v[j], v[j + 16]);
-    if (chan != nullptr) {
+    if (CHAN && (PRE || chan != nullptr)) {
         const float4* cp = reinterpret_cast<const float4*>(chan);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            const float4 lo = __ldg(cp + q), hi = __ldg(cp + 4 + q);
-            P[4 * q] = mul2_rn(P[4 * q], make_float2(lo.x, hi.x));
-            P[4 * q + 1] = mul2_rn(P[4 * q + 1], make_float2(lo.y, hi.y));
-            P[4 * q + 2] = mul2_rn(P[4 * q + 2], make_float2(lo.z, hi.z));
-            P[4 * q + 3] = mul2_rn(P[4 * q + 3], make_float2(lo.w, hi.w));
+            // the products feed the butterfly adds: scalar, never fused
+            const float4 lo = PRE ? cw[q] : __ldg(cp + q), hi = PRE ? cw[4 + q] : __ldg(cp + 4 + q);
+            P[4 * q] = mul2_sep_rn(P[4 * q], make_float2(lo.x, hi.x));
+            P[4 * q + 1] = mul2_sep_rn(P[4 * q + 1], make_float2(lo.y, hi.y));
+            P[4 * q + 2] = mul2_sep_rn(P[4 * q + 2], make_float2(lo.z, hi.z));
+            P[4 * q + 3] = mul2_sep_rn(P[4 * q + 3], make_float2(lo.w, hi.w));
         }
     }
     if constexpr (HAD) {
@@ -264,10 +270,8 @@ __global__ void __launch_bounds__(qz::THREADS, 1)
     uint8_t* sbuf = cbuf + NBUF * G::CODE_TILE;
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + G::BAR_OFF);
     uint64_t* empty = full + G::NSTAGE;
-    // consumer abort flags, indexed by tile-iteration parity: written before
-    // the per-tile consumer barrier, read after it, so every consumer takes
-    // the same decision
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + G::NSTAGE);
+    uint64_t* cfull = empty + G::NSTAGE;     // staging buffer written by every consumer warp
+    uint64_t* cfree = cfull + NBUF;          // staging buffer read out by its stores
     float* inv_tab = reinterpret_cast<float*>(smem + G::TAB_OFF);   // NVFP4: 1 / (s_b * s_t) per byte
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -276,8 +280,10 @@ __global__ void __launch_bounds__(qz::THREADS, 1)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], CONSUMER_WARPS);
         }
-        abort_flag[0] = 0;
-        abort_flag[1] = 0;
+        for (int b = 0; b < NBUF; ++b) {
+            mbar_init(&cfull[b], CONSUMER_WARPS);
+            mbar_init(&cfree[b], 1);
+        }
         fence_mbar_init();
     }
     __syncthreads();
@@ -314,6 +320,38 @@ __global__ void __launch_bounds__(qz::THREADS, 1)
         }
         return;
     }
+    if (warp == CONSUMER_WARPS + 1) {
+        // ---- store warp: sends each finished tile's codes and scale atoms
+        if (lane == 0) {
+            if (codes_tma) tma_prefetch_desc(&tmC);
+            const int64_t bands = (p.rows + 127) / 128;
+            int buf = 0;
+            uint32_t bphase = 0;
+            for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
+                // on time-out stop: nothing of this tile is complete
+                if (!mbar_wait(&cfull[buf], bphase)) break;
+                const int64_t tr = t / tiles_c, tc = t % tiles_c;
+                const int64_t row0 = tr * G::ROWS, col0 = tc * 4 * BLK;
+                uint8_t* cb = cbuf + buf * G::CODE_TILE;
+                uint8_t* fb = sbuf + buf * G::SF_TILE;
+                if (codes_tma) tma_store_2d(&tmC, cb, (int32_t)(col0 / 2), (int32_t)row0);
+                if (TC) {
+#pragma unroll
+                    for (int a = 0; a < G::ROWS / 128; ++a) {
+                        const int64_t band = row0 / 128 + a;
+                        if (band < bands) bulk_store(p.scales + (band * p.catoms + tc) * 512, fb + a * 512, 512u);
+                    }
+                }
+                bulk_commit_group();
+                // the consumers may overwrite the buffer once its stores have read it
+                bulk_wait_read_all();
+                mbar_arrive(&cfree[buf]);
+                if (++buf == NBUF) { buf = 0; bphase ^= 1; }
+            }
+            bulk_wait_all();
+        }
+        return;
+    }
 
     // ---- consumers
     NvCtx sc;
@@ -322,14 +360,31 @@ __global__ void __launch_bounds__(qz::THREADS, 1)
         nv_fill_table(*p.gscale, inv_tab, tid, CONSUMERS);
         named_barrier(1, CONSUMERS);
     }
-    const int64_t bands = (p.rows + 127) / 128;
     const int64_t crow = p.cols / 2;           // bytes of codes per row
     int stage = 0, buf = 0;
-    uint32_t phase = 0, it = 0;
-    for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++it) {
+    uint32_t phase = 0, bphase = 0;
+    // a consumer warp whose wait times out stops; every other role then
+    // times out in turn on the barriers that warp no longer arrives on
+    for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
         const int64_t tr = t / tiles_c, tc = t % tiles_c;
         const int64_t row0 = tr * G::ROWS, col0 = tc * 4 * BLK;
-        if (!mbar_wait(&full[stage], phase)) abort_flag[it & 1] = 1;
+        // MXFP4 channel factors of this thread's blocks (1 outside the
+        // tensor); for bf16 input they are loaded before the tile lands so
+        // their latency overlaps the wait (fp32 input has no registers to
+        // spare: there they are read inside the block step)
+        constexpr bool PRE = BLK == 32 && CHAN && BF16;
+        float4 cw[G::BPT][8];
+        if constexpr (PRE) {
+#pragma unroll
+            for (int k = 0; k < G::BPT; ++k) {
+                const int64_t col = col0 + ((tid + k * CONSUMERS) / G::ROWS) * BLK;
+                const float4* cp = reinterpret_cast<const float4*>(p.chan + col);
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    cw[k][q] = col < p.cols ? __ldg(cp + q) : make_float4(1.0f, 1.0f, 1.0f, 1.0f);
+            }
+        }
+        if (!mbar_wait(&full[stage], phase)) break;
 
         float v[G::BPT][BLK];
         const uint8_t* sb = smem + stage * G::STAGE;
@@ -356,6 +411,7 @@ __global__ void __launch_bounds__(qz::THREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[stage]);
         if (++stage == G::NSTAGE) { stage = 0; phase ^= 1; }
+        if (!mbar_wait(&cfree[buf], bphase ^ 1)) break;
 
         uint8_t* cb = cbuf + buf * G::CODE_TILE;
         uint8_t* fb = sbuf + buf * G::SF_TILE;
@@ -371,7 +427,7 @@ __global__ void __launch_bounds__(qz::THREADS, 1)
                 else nv_block<RU>(v[k], sc, byte, w);
             } else {
                 const float* chan = (CHAN && col < p.cols) ? p.chan + col : nullptr;
-                mx_block<RU, HAD>(v[k], chan, byte, w);
+                mx_block<RU, HAD, CHAN, PRE>(v[k], cw[k], chan, byte, w);
             }
             const bool inside = row < p.rows && col < p.cols;
             if (codes_tma) {
@@ -386,25 +442,12 @@ __global__ void __launch_bounds__(qz::THREADS, 1)
             if (TC) fb[(r >> 7) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + j] = (uint8_t)byte;
             else if (inside) p.scales[row * p.scols + tc * 4 + j] = (uint8_t)byte;
         }
+        // this warp's part of the staging buffer goes to the store warp
         fence_proxy_async_smem();
-        named_barrier(1, CONSUMERS);
-        if (tid == 0) {
-            if (codes_tma) tma_store_2d(&tmC, cb, (int32_t)(col0 / 2), (int32_t)row0);
-            if (TC) {
-#pragma unroll
-                for (int a = 0; a < G::ROWS / 128; ++a) {
-                    const int64_t band = row0 / 128 + a;
-                    if (band < bands) bulk_store(p.scales + (band * p.catoms + tc) * 512, fb + a * 512, 512u);
-                }
-            }
-            bulk_commit_group();
-            // the buffer the next-but-one tile writes is free once this returns
-            bulk_wait_read_1();
-        }
-        if (abort_flag[it & 1]) break;
-        if (++buf == NBUF) buf = 0;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&cfull[buf]);
+        if (++buf == NBUF) { buf = 0; bphase ^= 1; }
     }
-    if (tid == 0) bulk_wait_all();
 }
 
 // ------------------------------------------------------------------ sigma-delta
@@ -545,8 +588,8 @@ __global__ void __launch_bounds__(sdk::THREADS, 1)
                 x01 = make_float2(0.0f, 0.0f);
                 x23 = x01;
             } else {
-                x01 = mul2_rn(make_float2(w4.x, w4.y), make_float2(inv, inv));
-                x23 = mul2_rn(make_float2(w4.z, w4.w), make_float2(inv, inv));
+                x01 = mul2_sep_rn(make_float2(w4.x, w4.y), make_float2(inv, inv));   // feeds an add
+                x23 = mul2_sep_rn(make_float2(w4.z, w4.w), make_float2(inv, inv));
             }
             const float2 v01 = add2_rn(x01, make_float2(r4.x, r4.y));
             const float2 v23 = add2_rn(x23, make_float2(r4.z, r4.w));
@@ -606,8 +649,9 @@ __global__ void __launch_bounds__(256) sigma_delta_banks_kernel(SigmaDeltaParams
             degenerate = false;
         }
         const float2 iv = make_float2(inv, inv);
-        float2 x[4] = {mul2_rn(make_float2(w0.x, w0.y), iv), mul2_rn(make_float2(w0.z, w0.w), iv),
-                       mul2_rn(make_float2(w1.x, w1.y), iv), mul2_rn(make_float2(w1.z, w1.w), iv)};
+        // the products feed adds: scalar, never fused
+        float2 x[4] = {mul2_sep_rn(make_float2(w0.x, w0.y), iv), mul2_sep_rn(make_float2(w0.z, w0.w), iv),
+                       mul2_sep_rn(make_float2(w1.x, w1.y), iv), mul2_sep_rn(make_float2(w1.z, w1.w), iv)};
         if (degenerate)
             for (int j = 0; j < 4; ++j) x[j] = make_float2(0.0f, 0.0f);
         float2 r[4] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f),
