@@ -138,14 +138,36 @@ __device__ __forceinline__ NvScale nv_scale_from_byte(uint32_t byte, float s_t) 
 // is monotone, so when the bytes of q0 -/+ four steps agree that byte is the
 // answer; otherwise (next to an E4M3 rounding boundary) the quotient is
 // formed by the correctly rounded division.
-__device__ __forceinline__ uint32_t e4m3_rn_of_quotient(float amax, float denom, float rden) {
+// The fast half: true (byte set) when the bytes of q0 -/+ four steps agree.
+__device__ __forceinline__ bool e4m3_rn_of_quotient_fast(float amax, float rden, uint32_t& byte) {
     const uint32_t b = __float_as_uint(__fmul_rn(amax, rden));
     const float lo = __uint_as_float(b >= 4u ? b - 4u : 0u);
     const float hi = __uint_as_float(b + 4u);
     uint16_t pr;
     asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(pr) : "f"(fminf(hi, 448.0f)), "f"(fminf(lo, 448.0f)));
-    if ((pr & 0xFFu) == (uint32_t)(pr >> 8)) return pr & 0xFFu;
+    byte = pr & 0xFFu;
+    return byte == (uint32_t)(pr >> 8);
+}
+__device__ __forceinline__ uint32_t e4m3_rn_of_quotient(float amax, float denom, float rden) {
+    uint32_t byte;
+    if (e4m3_rn_of_quotient_fast(amax, rden, byte)) return byte;
     return e4m3_rn(__fdiv_rn(amax, denom));
+}
+
+// Largest magnitude of N values (0 if there is none that is not NaN) as a
+// balanced tree of maxima: depth log2 N instead of a chain of N; the maximum
+// does not depend on the order it is taken in.
+template <int N>
+__device__ __forceinline__ float amax_tree(const float* v) {
+    float m[N / 2];
+#pragma unroll
+    for (int i = 0; i < N / 2; ++i) m[i] = fmaxf(fabsf(v[2 * i]), fabsf(v[2 * i + 1]));
+#pragma unroll
+    for (int w = N / 4; w >= 1; w >>= 1) {
+#pragma unroll
+        for (int i = 0; i < w; ++i) m[i] = fmaxf(m[i], m[i + w]);
+    }
+    return fmaxf(0.0f, m[0]);
 }
 
 // ---- pairs of binary32 values on the f32x2 ALU: each lane is rounded to
@@ -218,33 +240,60 @@ __device__ __forceinline__ void nv_fill_table(float s_t, float* tab, int tid, in
     }
 }
 
-// One NVFP4 block: amax, E4M3 scale byte (RN or RU of amax / (6 s_t)),
-// codes of x * inv (all zero for a degenerate scale).
+// N NVFP4 blocks at once: amax, E4M3 scale byte (RN or RU of amax / (6 s_t)),
+// codes of x * inv (all zero for a degenerate scale).  Each step runs over
+// all N blocks before the next, with no branch that is not uniform across
+// the warp in between, so the blocks' dependency chains interleave.
+template <bool RU, int N>
+__device__ __forceinline__ void nv_blocks(const float (&v)[N][16], const NvCtx& c, uint32_t (&byte)[N],
+                                          uint32_t (&w)[N][2]) {
+    float amax[N];
+#pragma unroll
+    for (int k = 0; k < N; ++k) amax[k] = amax_tree<16>(v[k]);
+    if (!c.st_ok) {
+#pragma unroll
+        for (int k = 0; k < N; ++k) byte[k] = 0;
+    } else if (!RU && c.fast) {
+        bool ok[N];
+#pragma unroll
+        for (int k = 0; k < N; ++k) ok[k] = e4m3_rn_of_quotient_fast(amax[k], c.rden, byte[k]);
+        // next to an E4M3 rounding boundary: the correctly rounded division
+#pragma unroll
+        for (int k = 0; k < N; ++k)
+            if (!ok[k]) byte[k] = e4m3_rn(__fdiv_rn(amax[k], c.denom));
+    } else {
+#pragma unroll
+        for (int k = 0; k < N; ++k)
+            byte[k] = RU ? e4m3_ru(__fdiv_rn(amax[k], c.denom)) : e4m3_rn(__fdiv_rn(amax[k], c.denom));
+    }
+    float inv[N];
+#pragma unroll
+    for (int k = 0; k < N; ++k) inv[k] = c.tab[byte[k]];
+#pragma unroll
+    for (int k = 0; k < N; ++k) {
+        const float2 iv = make_float2(inv[k], inv[k]);
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+            float q[8];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 m = mul2_rn(make_float2(v[k][8 * g + 2 * i], v[k][8 * g + 2 * i + 1]), iv);
+                q[2 * i] = m.x;
+                q[2 * i + 1] = m.y;
+            }
+            // a degenerate scale (NaN entry) gives all-zero codes
+            w[k][g] = inv[k] != inv[k] ? 0u : e2m1_pack8(q);
+        }
+    }
+}
+
 template <bool RU>
 __device__ __forceinline__ void nv_block(const float (&v)[16], const NvCtx& c, uint32_t& byte, uint32_t (&w)[2]) {
-    float amax = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
-    if (!c.st_ok) byte = 0;
-    else if (!RU && c.fast) byte = e4m3_rn_of_quotient(amax, c.denom, c.rden);
-    else byte = RU ? e4m3_ru(__fdiv_rn(amax, c.denom)) : e4m3_rn(__fdiv_rn(amax, c.denom));
-    const float inv = c.tab[byte];
-    if (inv != inv) {
-        w[0] = w[1] = 0u;
-        return;
-    }
-    const float2 iv = make_float2(inv, inv);
-#pragma unroll
-    for (int g = 0; g < 2; ++g) {
-        float q[8];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float2 m = mul2_rn(make_float2(v[8 * g + 2 * i], v[8 * g + 2 * i + 1]), iv);
-            q[2 * i] = m.x;
-            q[2 * i + 1] = m.y;
-        }
-        w[g] = e2m1_pack8(q);
-    }
+    uint32_t b[1], ww[1][2];
+    nv_blocks<RU, 1>(reinterpret_cast<const float(&)[1][16]>(v), c, b, ww);
+    byte = b[0];
+    w[0] = ww[0][0];
+    w[1] = ww[0][1];
 }
 
 // Offset of scale (r, c) in the tensor-core scale layout (see q4.h).

@@ -183,9 +183,7 @@ __device__ __forceinline__ void nv46_candidate(const float (&v)[16], const NvCtx
 // block max to 4 replaces the one mapping it to 6 when its squared error is
 // strictly smaller.
 __device__ __forceinline__ void nv_block46(const float (&v)[16], const NvCtx& c, uint32_t& byte, uint32_t (&w)[2]) {
-    float amax = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    const float amax = amax_tree<16>(v);
     uint32_t b6, b4, w6[2], w4[2];
     double e6, e4;
     nv46_candidate(v, c, amax, 6.0f, b6, w6, e6);
@@ -239,9 +237,7 @@ __device__ __forceinline__ void mx_block(const float (&v)[32], const float4 (&cw
             P[j] = mul2_rn(make_float2(__fadd_rn(a, b), __fsub_rn(a, b)), isq);
         }
     }
-    float amax = 0.0f;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fmaxf(fabsf(P[j].x), fabsf(P[j].y)));
+    const float amax = amax_tree<32>(reinterpret_cast<const float*>(P));
     const int e = mx_exponent(amax, RU);
     byte = (uint32_t)(e + 127);
     const float m = exp2_int(-e);
@@ -415,6 +411,10 @@ __global__ void __launch_bounds__(qz::THREADS, 1)
 
         uint8_t* cb = cbuf + buf * G::CODE_TILE;
         uint8_t* fb = sbuf + buf * G::SF_TILE;
+        // NVFP4 (RN / RU): all of this thread's blocks at once
+        uint32_t nbyte[G::BPT], nw[G::BPT][2];
+        if constexpr (BLK == 16 && !S46) nv_blocks<RU, G::BPT>(reinterpret_cast<const float(&)[G::BPT][16]>(v), sc,
+                                                                 nbyte, nw);
 #pragma unroll
         for (int k = 0; k < G::BPT; ++k) {
             const int b = tid + k * CONSUMERS;
@@ -423,8 +423,13 @@ __global__ void __launch_bounds__(qz::THREADS, 1)
             uint32_t byte;
             uint32_t w[BLK / 8];
             if constexpr (BLK == 16) {
-                if constexpr (S46) nv_block46(v[k], sc, byte, w);
-                else nv_block<RU>(v[k], sc, byte, w);
+                if constexpr (S46) {
+                    nv_block46(v[k], sc, byte, w);
+                } else {
+                    byte = nbyte[k];
+                    w[0] = nw[k][0];
+                    w[1] = nw[k][1];
+                }
             } else {
                 const float* chan = (CHAN && col < p.cols) ? p.chan + col : nullptr;
                 mx_block<RU, HAD, CHAN, PRE>(v[k], cw[k], chan, byte, w);
