@@ -241,9 +241,15 @@ def rows_bench(q4, dev, flush, pk, reps=30):
     nw = sum(w.size for w in dl["w"])
     w16_flops = sum(2.0 * Ml * w.shape[0] * Kl for w in dl["w"])
 
+    # the per-visit requant steps run as one grouped launch over the 13 matrices
+    gW = [m[0] for m in mats]
+    gS = [m[1] for m in mats]
+    gG = [m[2] for m in mats]
+    gR = [m[3] for m in mats]
+    gC = [m[4] for m in mats]
+
     def sd_visit():
-        for wt, sc, g, r, c, _ in mats:
-            q4.q4_sigma_delta_step(q4.NVFP4, wt, sc, r, gscale=g, codes=c)
+        q4.q4_sigma_delta_step_grouped(q4.NVFP4, gW, gS, gR, gscales=gG, codes=gC)
 
     def w16_visit():
         for wt, sc, g, r, c, y in mats:
@@ -264,8 +270,7 @@ def rows_bench(q4, dev, flush, pk, reps=30):
              for wt, *_ in mats]
 
     def codebanks():
-        for (wt, sc, g, r, c, _), bk in zip(mats, banks):
-            q4.q4_sigma_delta_codebanks(q4.NVFP4, wt, sc, 32, gscale=g, codes=bk)
+        q4.q4_sigma_delta_codebanks_grouped(q4.NVFP4, gW, gS, 32, gscales=gG, codes=banks)
     ms_cb, _ = time_fn(codebanks, max(5, reps // 3), flush)
     gbs = nw * (4 + 32 * 0.5) / (ms_cb * 1e-3) / 1e9
     out["sigma_delta_codebanks_K32"] = {"weights": nw, "visits": 32, "us": ms_cb * 1e3, "GB/s": gbs,
@@ -273,20 +278,19 @@ def rows_bench(q4, dev, flush, pk, reps=30):
                                         "vs_32_separate_visits": ms_sd * 32 / ms_cb}
     del banks
 
-    q46_out = [(torch.empty_like(c), torch.empty_like(sc)) for wt, sc, g, r, c, _ in mats]
+    q46_c = [torch.empty_like(c) for c in gC]
+    q46_s = [torch.empty_like(sc) for sc in gS]
 
     def q46():
-        for (wt, sc, g, r, c, _), (c46, s46) in zip(mats, q46_out):
-            q4.q4_quantize(q4.NVFP4, wt, gscale=g, flags=q4.SCALE_46 | q4.LAYOUT_TC, codes=c46, scales=s46)
+        q4.q4_quantize_grouped(q4.NVFP4, gW, gscales=gG, flags=q4.SCALE_46 | q4.LAYOUT_TC, codes=q46_c, scales=q46_s)
     ms_46, _ = time_fn(q46, reps, flush)
     gbs = nw * (4 + 0.5 + 1 / 16) / (ms_46 * 1e-3) / 1e9
     out["nvfp4_quantize46_looped_weights"] = {"weights": nw, "matrices": 13, "us": ms_46 * 1e3, "GB/s": gbs,
                                               "frac_hbm": gbs / hbm}
-    del q46_out
+    del q46_c, q46_s
 
     def sr_visit():
-        for wt, sc, g, r, c, _ in mats:
-            q4.q4_sr_requant(q4.NVFP4, wt, sc, 42, 7, gscale=g, codes=c)
+        q4.q4_sr_requant_grouped(q4.NVFP4, gW, gS, 42, 7, gscales=gG, codes=gC)
     ms_sr, _ = time_fn(sr_visit, reps, flush)
     gbs = nw * B_SR / (ms_sr * 1e-3) / 1e9
     out["sr_requant_visit"] = {"weights": nw, "matrices": 13, "us": ms_sr * 1e3, "GB/s": gbs, "frac_hbm": gbs / hbm}
@@ -300,8 +304,8 @@ def rows_bench(q4, dev, flush, pk, reps=30):
             q4.q4_sigma_delta_gemm(q4.NVFP4, xd16, wt, sc, r, g, y=yy)
 
     def unfused16():
+        q4.q4_sigma_delta_step_grouped(q4.NVFP4, gW, gS, gR, gscales=gG, codes=gC)
         for (wt, sc, g, r, c, _), yy in zip(mats, yd16):
-            q4.q4_sigma_delta_step(q4.NVFP4, wt, sc, r, gscale=g, codes=c)
             q4.q4_gemm(q4.NVFP4, 16, wt.shape[0], Kl, xd16, None, None, c, sc, g, y=yy, a_kind=q4.A_BF16_W4A16)
     ms_f, _ = time_fn(fused16, reps, flush)
     ms_u, _ = time_fn(unfused16, reps, flush)

@@ -276,6 +276,49 @@ Q4_API q4_status q4_sigma_delta_gemm(q4_format format, int block, int64_t M, int
                               const float* d_gscale, float* residue, q4_dtype out_dt, void* y,
                               int flags, void* stream);
 
+/*
+ * Grouped calls -- one launch over a list of matrices.  The looped core of
+ * "Looped Transformer quantization" (sec. 2.1 and sec. 4) requantizes every
+ * weight of the core at each loop visit; the core has many matrices of a few
+ * million weights, where one launch per matrix costs more than the work.  Each
+ * grouped call is exactly the matching single-matrix call applied to every
+ * entry of `mats` (same arithmetic, same outputs byte for byte), in one kernel
+ * launch.  `mats` is a HOST array of `count` entries (0 <= count <=
+ * Q4_MAX_GROUP; 0 does nothing) read before the call returns; every pointer in
+ * it is device memory.  Matrices are dense (row stride = cols).  No output
+ * buffer of one entry may overlap any buffer of another entry.  format,
+ * block, flags apply to every entry.  An invalid entry fails the whole call
+ * before any launch (Q4_ERR_ARG / Q4_ERR_ALIGN / Q4_ERR_SHAPE).
+ */
+#define Q4_MAX_GROUP 32
+typedef struct q4_matrix {
+    const void* w;          /* weights [rows, cols]: float; q4_quantize_grouped: in_dt */
+    int64_t rows, cols;
+    uint8_t* scales;        /* block scales (layout per flags): read by the requant
+                               calls, written by q4_quantize_grouped (q4_scale_bytes) */
+    const float* d_gscale;  /* NVFP4 tensor scale s_t (one float); NULL for MXFP4 */
+    float* residue;         /* q4_sigma_delta_step_grouped: r [rows, cols], in/out;
+                               q4_sigma_delta_codebanks_grouped: NULL or r_visits out;
+                               ignored by the other calls */
+    uint8_t* codes;         /* codes [rows, cols/2]; codebanks: [visits, rows, cols/2] */
+} q4_matrix;
+
+/* q4_quantize on every entry (x = w, ld = cols, no channel multipliers). */
+Q4_API q4_status q4_quantize_grouped(q4_format format, int block, q4_dtype in_dt,
+                                     const q4_matrix* mats, int count, int flags, void* stream);
+/* q4_sigma_delta_step on every entry. */
+Q4_API q4_status q4_sigma_delta_step_grouped(q4_format format, int block, const q4_matrix* mats,
+                                             int count, int flags, void* stream);
+/* q4_sr_requant on every entry, all with the same seed and visit (each
+   matrix's elements are numbered from 0, as in the single call). */
+Q4_API q4_status q4_sr_requant_grouped(q4_format format, int block, const q4_matrix* mats,
+                                       int count, uint64_t seed, uint32_t visit, int flags,
+                                       void* stream);
+/* q4_sigma_delta_codebanks on every entry (residue = residue_out). */
+Q4_API q4_status q4_sigma_delta_codebanks_grouped(q4_format format, int block,
+                                                  const q4_matrix* mats, int count, int visits,
+                                                  int flags, void* stream);
+
 /* Scratch bytes q4_gemm needs for these arguments (0 when none). */
 Q4_API size_t q4_gemm_workspace_size(q4_format format, int64_t M, int64_t N, int64_t K,
                               int a_kind);

@@ -64,7 +64,19 @@ SIGNATURES = {
     "q4_gemm_workspace_size": (_SZ, [_I, _I64, _I64, _I64, _I]),
     "q4_get_device_error": (_I, [_P]),
     "q4_gemm_a_bf16_noalloc": (_I, [_I64, _I64, _I64, _P, _P, _P, _P, _P, _I, _P, _P]),
+    "q4_quantize_grouped": (_I, [_I, _I, _I, _P, _I, _I, _P]),
+    "q4_sigma_delta_step_grouped": (_I, [_I, _I, _P, _I, _I, _P]),
+    "q4_sr_requant_grouped": (_I, [_I, _I, _P, _I, ctypes.c_uint64, ctypes.c_uint32, _I, _P]),
+    "q4_sigma_delta_codebanks_grouped": (_I, [_I, _I, _P, _I, _I, _I, _P]),
 }
+
+MAX_GROUP = 32
+
+
+class Q4Matrix(ctypes.Structure):
+    """struct q4_matrix of include/q4.h (one entry of a grouped call)."""
+    _fields_ = [("w", _P), ("rows", _I64), ("cols", _I64), ("scales", _P), ("d_gscale", _P),
+                ("residue", _P), ("codes", _P)]
 
 _lib = None
 
@@ -210,6 +222,72 @@ def q4_sr_requant(fmt: int, w: torch.Tensor, scales: torch.Tensor, seed: int, vi
     st = lib().q4_sr_requant(fmt, BLOCK[fmt], _ptr(w), rows, cols, _ptr(scales), _ptr(gscale), int(seed), int(visit),
                              _ptr(codes), flags, _stream(stream))
     _check("q4_sr_requant", st)
+    return codes
+
+
+# ------------------------------------------------------------------ grouped calls
+def _group(ws, scales=None, gscales=None, residues=None, codes=None):
+    """The host array of q4_matrix entries for a grouped call."""
+    n = len(ws)
+    arr = (Q4Matrix * max(n, 1))()
+    for i, w in enumerate(ws):
+        rows, cols = w.shape
+        arr[i] = Q4Matrix(_ptr(w), rows, cols, _ptr(scales[i]) if scales is not None else None,
+                          _ptr(gscales[i]) if gscales is not None else None,
+                          _ptr(residues[i]) if residues is not None else None,
+                          _ptr(codes[i]) if codes is not None else None)
+    return arr, n
+
+
+def q4_quantize_grouped(fmt: int, ws, gscales=None, flags: int = LAYOUT_TC, codes=None, scales=None,
+                        stream=None):
+    """q4_quantize of every 2-D tensor in ws (one dtype) in one launch; returns (codes, scales) lists."""
+    if codes is None:
+        codes = [torch.empty((w.shape[0], w.shape[1] // 2), dtype=torch.uint8, device=w.device) for w in ws]
+    if scales is None:
+        scales = [torch.empty(max(q4_scale_bytes(fmt, w.shape[0], w.shape[1], flags), 1), dtype=torch.uint8,
+                              device=w.device) for w in ws]
+    arr, n = _group(ws, scales, gscales, None, codes)
+    dt = _dtype_code(ws[0]) if n else F32
+    st = lib().q4_quantize_grouped(fmt, BLOCK[fmt], dt, ctypes.addressof(arr), n, flags, _stream(stream))
+    _check("q4_quantize_grouped", st)
+    return codes, scales
+
+
+def q4_sigma_delta_step_grouped(fmt: int, ws, scales, residues, gscales=None, flags: int = LAYOUT_TC,
+                                codes=None, stream=None):
+    """q4_sigma_delta_step on every (w, scales, residue) in one launch; returns the codes list."""
+    if codes is None:
+        codes = [torch.empty((w.shape[0], w.shape[1] // 2), dtype=torch.uint8, device=w.device) for w in ws]
+    arr, n = _group(ws, scales, gscales, residues, codes)
+    st = lib().q4_sigma_delta_step_grouped(fmt, BLOCK[fmt], ctypes.addressof(arr), n, flags, _stream(stream))
+    _check("q4_sigma_delta_step_grouped", st)
+    return codes
+
+
+def q4_sr_requant_grouped(fmt: int, ws, scales, seed: int, visit: int, gscales=None, flags: int = LAYOUT_TC,
+                          codes=None, stream=None):
+    """q4_sr_requant on every (w, scales) in one launch; returns the codes list."""
+    if codes is None:
+        codes = [torch.empty((w.shape[0], w.shape[1] // 2), dtype=torch.uint8, device=w.device) for w in ws]
+    arr, n = _group(ws, scales, gscales, None, codes)
+    st = lib().q4_sr_requant_grouped(fmt, BLOCK[fmt], ctypes.addressof(arr), n, int(seed), int(visit), flags,
+                                     _stream(stream))
+    _check("q4_sr_requant_grouped", st)
+    return codes
+
+
+def q4_sigma_delta_codebanks_grouped(fmt: int, ws, scales, visits: int, gscales=None, flags: int = LAYOUT_TC,
+                                     codes=None, residue_out=None, stream=None):
+    """q4_sigma_delta_codebanks on every (w, scales) in one launch; returns the bank tensors
+    ([visits, rows, cols/2] each)."""
+    if codes is None:
+        codes = [torch.empty((visits, w.shape[0], w.shape[1] // 2), dtype=torch.uint8, device=w.device)
+                 for w in ws]
+    arr, n = _group(ws, scales, gscales, residue_out, codes)
+    st = lib().q4_sigma_delta_codebanks_grouped(fmt, BLOCK[fmt], ctypes.addressof(arr), n, int(visits), flags,
+                                                _stream(stream))
+    _check("q4_sigma_delta_codebanks_grouped", st)
     return codes
 
 

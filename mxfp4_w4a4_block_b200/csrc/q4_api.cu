@@ -35,6 +35,36 @@ bool valid_dtype(int d) { return d == Q4_F32 || d == Q4_BF16; }
 
 int64_t catoms_of(int64_t cols, int blk) { return ((cols / blk) + 3) / 4; }
 
+// Per-entry checks of a grouped call (the single-matrix call's checks) and
+// the launch table; entries with no elements are dropped.  need_res: the
+// residue must be present; res_io: a present residue must be aligned.
+q4_status group_from(q4_format format, int block, const q4_matrix* mats, int count, int flags, int allowed,
+                     bool need_res, bool res_io, bool scales_aligned, q4::GroupParams& g) {
+    if (!valid_format(format)) return Q4_ERR_ARG;
+    if (block != block_of(format)) return Q4_ERR_UNSUPPORTED;
+    if (flags & ~allowed) return Q4_ERR_ARG;
+    if (count < 0 || count > Q4_MAX_GROUP || (count > 0 && !mats)) return Q4_ERR_ARG;
+    g.count = 0;
+    g.total = 0;
+    for (int i = 0; i < count; ++i) {
+        const q4_matrix& m = mats[i];
+        if (m.rows < 0 || m.cols < 0) return Q4_ERR_ARG;
+        if (format == Q4_NVFP4 && !m.d_gscale) return Q4_ERR_ARG;
+        if (format == Q4_MXFP4 && m.d_gscale) return Q4_ERR_ARG;
+        if (m.cols % block) return Q4_ERR_SHAPE;
+        if (m.rows == 0 || m.cols == 0) continue;
+        if (!m.w || !m.scales || !m.codes || (need_res && !m.residue)) return Q4_ERR_ARG;
+        if (!aligned16(m.w) || !aligned16(m.codes) || (res_io && m.residue && !aligned16(m.residue)) ||
+            (scales_aligned && !aligned16(m.scales)))
+            return Q4_ERR_ALIGN;
+        q4::GroupItem& it = g.m[g.count++];
+        it.w = m.w; it.rows = m.rows; it.cols = m.cols; it.scales = m.scales; it.gscale = m.d_gscale;
+        it.residue = res_io ? m.residue : nullptr; it.codes = m.codes;
+        it.scols = m.cols / block; it.catoms = catoms_of(m.cols, block); it.start = 0;
+    }
+    return Q4_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -191,6 +221,48 @@ q4_status q4_sigma_delta_gemm(q4_format format, int block, int64_t M, int64_t N,
     p.M = M; p.N = N; p.K = K; p.x = x; p.w = w; p.scales = scales; p.gscale = d_gscale; p.residue = residue;
     p.y = y; p.out_bf16 = out_dt == Q4_BF16;
     return cuda_status(q4::launch_sd_gemm(p, (cudaStream_t)stream, num_sms()));
+}
+
+q4_status q4_quantize_grouped(q4_format format, int block, q4_dtype in_dt, const q4_matrix* mats, int count,
+                              int flags, void* stream) {
+    if (!valid_dtype(in_dt)) return Q4_ERR_ARG;
+    if (format == Q4_NVFP4 && (flags & Q4_HADAMARD32)) return Q4_ERR_UNSUPPORTED;
+    if (format == Q4_MXFP4 && (flags & Q4_SCALE_46)) return Q4_ERR_UNSUPPORTED;
+    q4::GroupParams g;
+    const q4_status s = group_from(format, block, mats, count, flags,
+                                   Q4_SCALE_RU | Q4_LAYOUT_TC | Q4_HADAMARD32 | Q4_SCALE_46, false, false, true, g);
+    if (s != Q4_OK || g.count == 0) return s;
+    return cuda_status(q4::launch_quantize_grouped(g, block, in_dt == Q4_BF16, (flags & Q4_LAYOUT_TC) != 0,
+                                                   (flags & Q4_SCALE_RU) != 0, (flags & Q4_HADAMARD32) != 0,
+                                                   (flags & Q4_SCALE_46) != 0, (cudaStream_t)stream, num_sms()));
+}
+
+q4_status q4_sigma_delta_step_grouped(q4_format format, int block, const q4_matrix* mats, int count, int flags,
+                                      void* stream) {
+    q4::GroupParams g;
+    const q4_status s = group_from(format, block, mats, count, flags, Q4_LAYOUT_TC, true, true, false, g);
+    if (s != Q4_OK || g.count == 0) return s;
+    return cuda_status(q4::launch_sigma_delta_grouped(g, block, (flags & Q4_LAYOUT_TC) != 0, (cudaStream_t)stream,
+                                                      num_sms()));
+}
+
+q4_status q4_sr_requant_grouped(q4_format format, int block, const q4_matrix* mats, int count, uint64_t seed,
+                                uint32_t visit, int flags, void* stream) {
+    q4::GroupParams g;
+    const q4_status s = group_from(format, block, mats, count, flags, Q4_LAYOUT_TC, false, false, false, g);
+    if (s != Q4_OK || g.count == 0) return s;
+    return cuda_status(q4::launch_sr_requant_grouped(g, block, (flags & Q4_LAYOUT_TC) != 0, seed, visit,
+                                                     (cudaStream_t)stream, num_sms()));
+}
+
+q4_status q4_sigma_delta_codebanks_grouped(q4_format format, int block, const q4_matrix* mats, int count,
+                                           int visits, int flags, void* stream) {
+    if (visits < 1 || visits > 4096) return Q4_ERR_ARG;
+    q4::GroupParams g;
+    const q4_status s = group_from(format, block, mats, count, flags, Q4_LAYOUT_TC, false, true, false, g);
+    if (s != Q4_OK || g.count == 0) return s;
+    return cuda_status(q4::launch_sigma_delta_banks_grouped(g, block, (flags & Q4_LAYOUT_TC) != 0, visits,
+                                                            (cudaStream_t)stream, num_sms()));
 }
 
 size_t q4_gemm_workspace_size(q4_format format, int64_t M, int64_t N, int64_t K, int a_kind) {

@@ -28,6 +28,28 @@ struct SigmaDeltaParams {
     int64_t scols, catoms;
 };
 
+// One matrix of a grouped launch, and the launch's table of them (passed
+// by value as a kernel parameter).  A work unit is 8 weights of a row for the
+// requant kernels and one block (padded grid in the tensor-core layout) for
+// the quantizer; `start` is the entry's first unit in the launch.
+constexpr int kMaxGroup = 32;
+struct GroupItem {
+    const void* w;        // [rows, cols], dense
+    int64_t rows, cols;
+    uint8_t* scales;
+    const float* gscale;
+    float* residue;
+    uint8_t* codes;
+    int64_t scols, catoms;
+    int64_t start;
+};
+struct GroupParams {
+    int count;
+    int64_t total;        // units over all entries
+    GroupItem m[kMaxGroup];
+};
+static_assert(sizeof(GroupParams) <= 4096, "a grouped launch's table must fit the kernel parameter space");
+
 struct DequantParams {
     const uint8_t* codes;
     const uint8_t* scales;
@@ -98,6 +120,15 @@ cudaError_t launch_sr_requant(const SigmaDeltaParams& p, int blk, bool tc, uint6
                               cudaStream_t st, int num_sms);
 cudaError_t launch_dequantize(const DequantParams& p, int blk, bool tc, bool out_bf16, cudaStream_t st,
                               int num_sms);
+// Grouped launches: every entry of g as the single-matrix launch above
+// (g.m[i].start and g.total are filled in by the launcher).
+cudaError_t launch_quantize_grouped(GroupParams& g, int blk, bool bf16, bool tc, bool ru, bool had, bool s46,
+                                    cudaStream_t st, int num_sms);
+cudaError_t launch_sigma_delta_grouped(GroupParams& g, int blk, bool tc, cudaStream_t st, int num_sms);
+cudaError_t launch_sr_requant_grouped(GroupParams& g, int blk, bool tc, uint64_t seed, uint32_t visit,
+                                      cudaStream_t st, int num_sms);
+cudaError_t launch_sigma_delta_banks_grouped(GroupParams& g, int blk, bool tc, int visits, cudaStream_t st,
+                                             int num_sms);
 cudaError_t launch_gemm(const GemmParams& p, cudaStream_t st, int num_sms);
 cudaError_t launch_fused_decode(const FusedDecodeParams& p, cudaStream_t st, int num_sms);
 

@@ -631,53 +631,68 @@ __global__ void __launch_bounds__(sdk::THREADS, 1)
 // block scale once, runs the K visits with the residue in registers, and
 // writes visit k's 4 code bytes into bank k (a warp writes 128 contiguous
 // bytes per bank).  Optionally the final residue r_K is stored.
+// Per-unit steps below are shared by the single-matrix and the grouped
+// launches.  A unit is 8 consecutive weights of a row: u = row * (cols / 8) +
+// col / 8.  P is SigmaDeltaParams or GroupItem.
+
+// Reciprocal block scale of weight (row, col): 1 / (dec(s_b) s_t) (NVFP4;
+// `degenerate` when that is not a usable scale: the codes are then 0) or
+// 2^-e (MXFP4).
+template <int BLK, bool TC, class P>
+__device__ __forceinline__ float unit_inv(const P& p, int64_t row, int64_t col, float s_t, bool& degenerate) {
+    const int64_t c = col / BLK;
+    const uint32_t sb = TC ? p.scales[tc_scale_offset(row, c, p.catoms)] : p.scales[row * p.scols + c];
+    if (BLK == 16) {
+        const NvScale sc = nv_scale_from_byte(sb, s_t);
+        degenerate = sc.degenerate;
+        return sc.inv;
+    }
+    degenerate = false;
+    return exp2_int(127 - (int)sb);
+}
+
+template <int BLK, bool TC, class P>
+__device__ __forceinline__ void banks_unit(const P& p, int64_t u, float s_t, int visits, int64_t bank_bytes,
+                                           float* r_out) {
+    const int64_t cpr = p.cols / 8;
+    const int64_t row = u / cpr, col = (u % cpr) * 8;
+    const float4* wp = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.w) + row * p.cols + col);
+    const float4 w0 = __ldcs(wp), w1 = __ldcs(wp + 1);
+    bool degenerate;
+    const float inv = unit_inv<BLK, TC>(p, row, col, s_t, degenerate);
+    const float2 iv = make_float2(inv, inv);
+    // the products feed adds: scalar, never fused
+    float2 x[4] = {mul2_sep_rn(make_float2(w0.x, w0.y), iv), mul2_sep_rn(make_float2(w0.z, w0.w), iv),
+                   mul2_sep_rn(make_float2(w1.x, w1.y), iv), mul2_sep_rn(make_float2(w1.z, w1.w), iv)};
+    if (degenerate)
+        for (int j = 0; j < 4; ++j) x[j] = make_float2(0.0f, 0.0f);
+    float2 r[4] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f),
+                   make_float2(0.0f, 0.0f)};
+    uint8_t* dst = p.codes + row * (p.cols / 2) + col / 2;
+    for (int k = 0; k < visits; ++k) {
+        float2 v[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) v[j] = add2_rn(x[j], r[j]);
+        const uint32_t codes = e2m1_pack4(v[0].x, v[0].y, v[1].x, v[1].y) |
+                               (e2m1_pack4(v[2].x, v[2].y, v[3].x, v[3].y) << 16);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) r[j] = sub2_rn(v[j], e2m1x2_value((codes >> (8 * j)) & 0xFFu));
+        __stcs(reinterpret_cast<unsigned int*>(dst + (int64_t)k * bank_bytes), codes);
+    }
+    if (r_out != nullptr) {
+        float4* rp = reinterpret_cast<float4*>(r_out + row * p.cols + col);
+        rp[0] = make_float4(r[0].x, r[0].y, r[1].x, r[1].y);
+        rp[1] = make_float4(r[2].x, r[2].y, r[3].x, r[3].y);
+    }
+}
+
 template <int BLK, bool TC>
 __global__ void __launch_bounds__(256) sigma_delta_banks_kernel(SigmaDeltaParams p, int visits, int64_t bank_bytes,
                                                                 float* r_out) {
-    const int64_t cpr = p.cols / 8;
-    const int64_t total = p.rows * cpr;
+    const int64_t total = p.rows * (p.cols / 8);
     const float s_t = (BLK == 16) ? *p.gscale : 0.0f;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t row = i / cpr, col = (i % cpr) * 8;
-        const float4* wp = reinterpret_cast<const float4*>(p.w + row * p.cols + col);
-        const float4 w0 = __ldcs(wp), w1 = __ldcs(wp + 1);
-        const int64_t c = col / BLK;
-        const uint32_t sb = TC ? p.scales[tc_scale_offset(row, c, p.catoms)] : p.scales[row * p.scols + c];
-        float inv;
-        bool degenerate;
-        if (BLK == 16) {
-            const NvScale sc = nv_scale_from_byte(sb, s_t);
-            inv = sc.inv;
-            degenerate = sc.degenerate;
-        } else {
-            inv = exp2_int(127 - (int)sb);
-            degenerate = false;
-        }
-        const float2 iv = make_float2(inv, inv);
-        // the products feed adds: scalar, never fused
-        float2 x[4] = {mul2_sep_rn(make_float2(w0.x, w0.y), iv), mul2_sep_rn(make_float2(w0.z, w0.w), iv),
-                       mul2_sep_rn(make_float2(w1.x, w1.y), iv), mul2_sep_rn(make_float2(w1.z, w1.w), iv)};
-        if (degenerate)
-            for (int j = 0; j < 4; ++j) x[j] = make_float2(0.0f, 0.0f);
-        float2 r[4] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f),
-                       make_float2(0.0f, 0.0f)};
-        uint8_t* dst = p.codes + row * (p.cols / 2) + col / 2;
-        for (int k = 0; k < visits; ++k) {
-            float2 v[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) v[j] = add2_rn(x[j], r[j]);
-            const uint32_t codes = e2m1_pack4(v[0].x, v[0].y, v[1].x, v[1].y) |
-                                   (e2m1_pack4(v[2].x, v[2].y, v[3].x, v[3].y) << 16);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) r[j] = sub2_rn(v[j], e2m1x2_value((codes >> (8 * j)) & 0xFFu));
-            __stcs(reinterpret_cast<unsigned int*>(dst + (int64_t)k * bank_bytes), codes);
-        }
-        if (r_out != nullptr) {
-            float4* rp = reinterpret_cast<float4*>(r_out + row * p.cols + col);
-            rp[0] = make_float4(r[0].x, r[0].y, r[1].x, r[1].y);
-            rp[1] = make_float4(r[2].x, r[2].y, r[3].x, r[3].y);
-        }
-    }
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x)
+        banks_unit<BLK, TC>(p, i, s_t, visits, bank_bytes, r_out);
 }
 
 // ------------------------------------------------------------------ stochastic-rounding requant
@@ -718,45 +733,71 @@ __device__ __forceinline__ uint32_t sr_e2m1(float x, float u) {
     return (signbit(x) ? 8u : 0u) | idx;
 }
 
-// One stochastic-rounding requant at a loop visit: each thread owns 8
-// consecutive weights e0 .. e0 + 7 (e0 = row * cols + col, a multiple of 8),
-// i.e. the two Philox blocks of counters (e0/4 + {0, 1}, visit), key = seed.
+// One stochastic-rounding requant at a loop visit of one unit: the 8
+// weights e0 .. e0 + 7 (e0 = row * cols + col, a multiple of 8) take the two
+// Philox blocks of counters (e0/4 + {0, 1}, visit), key = seed.
+template <int BLK, bool TC, class P>
+__device__ __forceinline__ void sr_unit(const P& p, int64_t u, float s_t, uint2 key, uint32_t visit) {
+    const int64_t cpr = p.cols / 8;
+    const int64_t row = u / cpr, col = (u % cpr) * 8;
+    const float4* wp = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.w) + row * p.cols + col);
+    const float4 w0 = __ldcs(wp), w1 = __ldcs(wp + 1);
+    bool degenerate;
+    const float inv = unit_inv<BLK, TC>(p, row, col, s_t, degenerate);
+    const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+    const uint64_t g = (uint64_t)(row * p.cols + col) >> 2;
+    const uint4 r0 = philox4x32_10(make_uint4((uint32_t)g, (uint32_t)(g >> 32), visit, 0u), key);
+    const uint4 r1 = philox4x32_10(make_uint4((uint32_t)(g + 1), (uint32_t)((g + 1) >> 32), visit, 0u), key);
+    const uint32_t rw[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+    uint32_t codes = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const float x = degenerate ? 0.0f : __fmul_rn(wv[j], inv);
+        const float uu = (float)(rw[j] >> 8) * 0x1p-24f;
+        codes |= sr_e2m1(x, uu) << (4 * j);
+    }
+    *reinterpret_cast<uint32_t*>(p.codes + row * (p.cols / 2) + col / 2) = codes;
+}
+
 template <int BLK, bool TC>
 __global__ void __launch_bounds__(256) sr_requant_kernel(SigmaDeltaParams p, uint64_t seed, uint32_t visit) {
-    const int64_t cpr = p.cols / 8;
-    const int64_t total = p.rows * cpr;
+    const int64_t total = p.rows * (p.cols / 8);
     const float s_t = (BLK == 16) ? *p.gscale : 0.0f;
     const uint2 key = make_uint2((uint32_t)seed, (uint32_t)(seed >> 32));
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t row = i / cpr, col = (i % cpr) * 8;
-        const float4* wp = reinterpret_cast<const float4*>(p.w + row * p.cols + col);
-        const float4 w0 = __ldcs(wp), w1 = __ldcs(wp + 1);
-        const int64_t c = col / BLK;
-        const uint32_t sb = TC ? p.scales[tc_scale_offset(row, c, p.catoms)] : p.scales[row * p.scols + c];
-        float inv;
-        bool degenerate;
-        if (BLK == 16) {
-            const NvScale sc = nv_scale_from_byte(sb, s_t);
-            inv = sc.inv;
-            degenerate = sc.degenerate;
-        } else {
-            inv = exp2_int(127 - (int)sb);
-            degenerate = false;
-        }
-        const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-        const uint64_t g = (uint64_t)(row * p.cols + col) >> 2;
-        const uint4 r0 = philox4x32_10(make_uint4((uint32_t)g, (uint32_t)(g >> 32), visit, 0u), key);
-        const uint4 r1 = philox4x32_10(make_uint4((uint32_t)(g + 1), (uint32_t)((g + 1) >> 32), visit, 0u), key);
-        const uint32_t rw[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
-        uint32_t codes = 0;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x)
+        sr_unit<BLK, TC>(p, i, s_t, key, visit);
+}
+
+// One Sigma-Delta step of one unit (as the tiled kernel above): x = w * inv,
+// v = x + r, q = E2M1(v), r <- v - q.
+template <int BLK, bool TC, class P>
+__device__ __forceinline__ void sd_unit(const P& p, int64_t u, float s_t) {
+    const int64_t cpr = p.cols / 8;
+    const int64_t row = u / cpr, col = (u % cpr) * 8;
+    const float4* wp = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.w) + row * p.cols + col);
+    float4* rp = reinterpret_cast<float4*>(p.residue + row * p.cols + col);
+    const float4 w0 = __ldcs(wp), w1 = __ldcs(wp + 1);
+    const float4 r0 = __ldcs(rp), r1 = __ldcs(rp + 1);
+    bool degenerate;
+    const float inv = unit_inv<BLK, TC>(p, row, col, s_t, degenerate);
+    const float2 iv = make_float2(inv, inv);
+    // the products feed adds: scalar, never fused
+    float2 x[4] = {mul2_sep_rn(make_float2(w0.x, w0.y), iv), mul2_sep_rn(make_float2(w0.z, w0.w), iv),
+                   mul2_sep_rn(make_float2(w1.x, w1.y), iv), mul2_sep_rn(make_float2(w1.z, w1.w), iv)};
+    if (degenerate)
+        for (int j = 0; j < 4; ++j) x[j] = make_float2(0.0f, 0.0f);
+    const float2 r[4] = {make_float2(r0.x, r0.y), make_float2(r0.z, r0.w), make_float2(r1.x, r1.y),
+                         make_float2(r1.z, r1.w)};
+    float2 v[4], n[4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const float x = degenerate ? 0.0f : __fmul_rn(wv[j], inv);
-            const float u = (float)(rw[j] >> 8) * 0x1p-24f;
-            codes |= sr_e2m1(x, u) << (4 * j);
-        }
-        *reinterpret_cast<uint32_t*>(p.codes + row * (p.cols / 2) + col / 2) = codes;
-    }
+    for (int j = 0; j < 4; ++j) v[j] = add2_rn(x[j], r[j]);
+    const uint32_t codes = e2m1_pack4(v[0].x, v[0].y, v[1].x, v[1].y) |
+                           (e2m1_pack4(v[2].x, v[2].y, v[3].x, v[3].y) << 16);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) n[j] = sub2_rn(v[j], e2m1x2_value((codes >> (8 * j)) & 0xFFu));
+    __stcs(rp, make_float4(n[0].x, n[0].y, n[1].x, n[1].y));
+    __stcs(rp + 1, make_float4(n[2].x, n[2].y, n[3].x, n[3].y));
+    __stcs(reinterpret_cast<unsigned int*>(p.codes + row * (p.cols / 2) + col / 2), codes);
 }
 
 // ------------------------------------------------------------------ dequantize
@@ -959,5 +1000,247 @@ cudaError_t launch_sr_requant(const SigmaDeltaParams& p, int blk, bool tc, uint6
 #undef Q4_SR
     return cudaGetLastError();
 }
+
+// ------------------------------------------------------------------ grouped launches
+// One launch over a list of matrices (the looped core requantizes all of its
+// weights at every loop visit; a matrix of a few million weights is too small
+// to amortise a launch of its own).  The units of all entries form one range
+// that the grid walks grid-stride; a unit's entry is the last one whose
+// `start` it has reached, and because entries are in unit order a thread's
+// entry index only moves forward along its walk.  Each unit runs exactly the
+// per-unit step of the single-matrix launch.
+__device__ __forceinline__ int group_entry(const GroupParams& g, int e, int64_t i) {
+    while (e + 1 < g.count && i >= g.m[e + 1].start) ++e;
+    return e;
+}
+
+template <int BLK, bool TC>
+__global__ void __launch_bounds__(256) sigma_delta_grouped_kernel(const __grid_constant__ GroupParams g) {
+    int e = -1;
+    GroupItem it;
+    float s_t = 0.0f;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < g.total; i += (int64_t)gridDim.x * blockDim.x) {
+        const int ne = group_entry(g, e < 0 ? 0 : e, i);
+        if (ne != e) {
+            e = ne;
+            it = g.m[e];
+            s_t = (BLK == 16) ? *it.gscale : 0.0f;
+        }
+        sd_unit<BLK, TC>(it, i - it.start, s_t);
+    }
+}
+
+template <int BLK, bool TC>
+__global__ void __launch_bounds__(256) sr_requant_grouped_kernel(const __grid_constant__ GroupParams g, uint64_t seed,
+                                                                 uint32_t visit) {
+    const uint2 key = make_uint2((uint32_t)seed, (uint32_t)(seed >> 32));
+    int e = -1;
+    GroupItem it;
+    float s_t = 0.0f;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < g.total; i += (int64_t)gridDim.x * blockDim.x) {
+        const int ne = group_entry(g, e < 0 ? 0 : e, i);
+        if (ne != e) {
+            e = ne;
+            it = g.m[e];
+            s_t = (BLK == 16) ? *it.gscale : 0.0f;
+        }
+        sr_unit<BLK, TC>(it, i - it.start, s_t, key, visit);
+    }
+}
+
+template <int BLK, bool TC>
+__global__ void __launch_bounds__(256) sigma_delta_banks_grouped_kernel(const __grid_constant__ GroupParams g,
+                                                                        int visits) {
+    int e = -1;
+    GroupItem it;
+    float s_t = 0.0f;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < g.total; i += (int64_t)gridDim.x * blockDim.x) {
+        const int ne = group_entry(g, e < 0 ? 0 : e, i);
+        if (ne != e) {
+            e = ne;
+            it = g.m[e];
+            s_t = (BLK == 16) ? *it.gscale : 0.0f;
+        }
+        banks_unit<BLK, TC>(it, i - it.start, s_t, visits, it.rows * (it.cols / 2), it.residue);
+    }
+}
+
+// Quantizer unit: one block, over the padded block grid in the tensor-core
+// layout (rows to a multiple of 128, blocks to a multiple of 4) so that the
+// padding scale bytes are written (0) as the tiled quantizer writes them.
+template <int BLK, bool BF16, bool TC, bool RU, bool HAD, bool S46>
+__device__ __forceinline__ void qz_unit(const GroupItem& p, int64_t u, const NvCtx& sc) {
+    const int64_t spad = TC ? p.catoms * 4 : p.scols;
+    const int64_t row = u / spad, b = u % spad;
+    if (row >= p.rows || b >= p.scols) {
+        if (TC) p.scales[tc_scale_offset(row, b, p.catoms)] = 0;
+        return;
+    }
+    float v[BLK];
+    if constexpr (BF16) {
+        const uint4* xp = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.w) + row * p.cols + b * BLK);
+#pragma unroll
+        for (int c = 0; c < BLK / 8; ++c) {
+            const uint4 raw = __ldg(xp + c);
+            float* d = v + 8 * c;
+            d[0] = bf16_lo(raw.x); d[1] = bf16_hi(raw.x); d[2] = bf16_lo(raw.y); d[3] = bf16_hi(raw.y);
+            d[4] = bf16_lo(raw.z); d[5] = bf16_hi(raw.z); d[6] = bf16_lo(raw.w); d[7] = bf16_hi(raw.w);
+        }
+    } else {
+        const float4* xp = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.w) + row * p.cols + b * BLK);
+#pragma unroll
+        for (int c = 0; c < BLK / 4; ++c) {
+            const float4 q = __ldg(xp + c);
+            v[4 * c] = q.x; v[4 * c + 1] = q.y; v[4 * c + 2] = q.z; v[4 * c + 3] = q.w;
+        }
+    }
+    uint32_t byte;
+    uint8_t* dst = p.codes + row * (p.cols / 2) + b * (BLK / 2);
+    if constexpr (BLK == 16) {
+        uint32_t w[2];
+        if constexpr (S46) {
+            nv_block46(v, sc, byte, w);
+        } else {
+            uint32_t bb[1], ww[1][2];
+            nv_blocks<RU, 1>(reinterpret_cast<const float(&)[1][16]>(v), sc, bb, ww);
+            byte = bb[0];
+            w[0] = ww[0][0];
+            w[1] = ww[0][1];
+        }
+        *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
+    } else {
+        uint32_t w[4];
+        const float4 cw[8] = {};
+        mx_block<RU, HAD, false, false>(v, cw, nullptr, byte, w);
+        *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    if (TC) p.scales[tc_scale_offset(row, b, p.catoms)] = (uint8_t)byte;
+    else p.scales[row * p.scols + b] = (uint8_t)byte;
+}
+
+template <int BLK, bool BF16, bool TC, bool RU, bool HAD, bool S46>
+__global__ void __launch_bounds__(256) quantize_grouped_kernel(const __grid_constant__ GroupParams g) {
+    // NVFP4: each entry's 128-entry table of 1 / (dec(s_b) s_t), as the tiled quantizer's
+    __shared__ float tabs[BLK == 16 ? kMaxGroup * 128 : 1];
+    if constexpr (BLK == 16) {
+        for (int k = threadIdx.x; k < g.count * 128; k += blockDim.x) {
+            const NvScale r = nv_scale_from_byte((uint32_t)(k & 127), *g.m[k >> 7].gscale);
+            tabs[k] = r.degenerate ? __uint_as_float(0x7FC00000u) : r.inv;
+        }
+        __syncthreads();
+    }
+    int e = -1;
+    GroupItem it;
+    NvCtx sc;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < g.total; i += (int64_t)gridDim.x * blockDim.x) {
+        const int ne = group_entry(g, e < 0 ? 0 : e, i);
+        if (ne != e) {
+            e = ne;
+            it = g.m[e];
+            if constexpr (BLK == 16) sc = nv_ctx(*it.gscale, tabs + e * 128);
+        }
+        qz_unit<BLK, BF16, TC, RU, HAD, S46>(it, i - it.start, sc);
+    }
+}
+
+// Entries' unit ranges; the grid is as many CTAs of 256 threads as are
+// resident on the GPU at once (persistent), fewer for a small launch.
+template <class K>
+static int fill_group(GroupParams& g, K kernel, int64_t (*units)(const GroupItem&), int num_sms) {
+    int64_t acc = 0;
+    for (int i = 0; i < g.count; ++i) {
+        g.m[i].start = acc;
+        acc += units(g.m[i]);
+    }
+    g.total = acc;
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, 256, 0) != cudaSuccess || occ < 1) occ = 1;
+    return grid_for((acc + 255) / 256, num_sms, occ);
+}
+
+static int64_t units8(const GroupItem& m) { return m.rows * (m.cols / 8); }
+static int64_t units_blocks_tc(const GroupItem& m) { return ((m.rows + 127) / 128) * 128 * m.catoms * 4; }
+static int64_t units_blocks_rm(const GroupItem& m) { return m.rows * m.scols; }
+
+template <int BLK, bool BF16, bool TC, bool RU, bool HAD, bool S46>
+static cudaError_t launch_qg(GroupParams& g, cudaStream_t st, int num_sms) {
+    auto k = quantize_grouped_kernel<BLK, BF16, TC, RU, HAD, S46>;
+    const int grid = fill_group(g, k, TC ? units_blocks_tc : units_blocks_rm, num_sms);
+    if (g.total == 0) return cudaSuccess;
+    k<<<grid, 256, 0, st>>>(g);
+    return cudaGetLastError();
+}
+
+template <int BLK, bool BF16, bool TC>
+static cudaError_t launch_qg_flags(GroupParams& g, bool ru, bool had, bool s46, cudaStream_t st, int num_sms) {
+    if constexpr (BLK == 16) {
+        if (s46) return launch_qg<16, BF16, TC, true, false, true>(g, st, num_sms);
+        if (ru) return launch_qg<16, BF16, TC, true, false, false>(g, st, num_sms);
+        return launch_qg<16, BF16, TC, false, false, false>(g, st, num_sms);
+    } else {
+        if (had) {
+            if (ru) return launch_qg<32, BF16, TC, true, true, false>(g, st, num_sms);
+            return launch_qg<32, BF16, TC, false, true, false>(g, st, num_sms);
+        }
+        if (ru) return launch_qg<32, BF16, TC, true, false, false>(g, st, num_sms);
+        return launch_qg<32, BF16, TC, false, false, false>(g, st, num_sms);
+    }
+}
+
+template <int BLK>
+static cudaError_t launch_qg_blk(GroupParams& g, bool bf16, bool tc, bool ru, bool had, bool s46, cudaStream_t st,
+                                 int num_sms) {
+    if (bf16) {
+        if (tc) return launch_qg_flags<BLK, true, true>(g, ru, had, s46, st, num_sms);
+        return launch_qg_flags<BLK, true, false>(g, ru, had, s46, st, num_sms);
+    }
+    if (tc) return launch_qg_flags<BLK, false, true>(g, ru, had, s46, st, num_sms);
+    return launch_qg_flags<BLK, false, false>(g, ru, had, s46, st, num_sms);
+}
+
+cudaError_t launch_quantize_grouped(GroupParams& g, int blk, bool bf16, bool tc, bool ru, bool had, bool s46,
+                                    cudaStream_t st, int num_sms) {
+    if (blk == 16) return launch_qg_blk<16>(g, bf16, tc, ru, had, s46, st, num_sms);
+    return launch_qg_blk<32>(g, bf16, tc, ru, had, s46, st, num_sms);
+}
+
+#define Q4_GROUP_LAUNCH(KERNEL, ...)                                  \
+    do {                                                              \
+        auto k = KERNEL;                                              \
+        const int grid = fill_group(g, k, units8, num_sms);           \
+        if (g.total == 0) return cudaSuccess;                         \
+        k<<<grid, 256, 0, st>>>(g __VA_OPT__(,) __VA_ARGS__);         \
+        return cudaGetLastError();                                    \
+    } while (0)
+
+cudaError_t launch_sigma_delta_grouped(GroupParams& g, int blk, bool tc, cudaStream_t st, int num_sms) {
+    if (blk == 16) {
+        if (tc) Q4_GROUP_LAUNCH((sigma_delta_grouped_kernel<16, true>));
+        Q4_GROUP_LAUNCH((sigma_delta_grouped_kernel<16, false>));
+    }
+    if (tc) Q4_GROUP_LAUNCH((sigma_delta_grouped_kernel<32, true>));
+    Q4_GROUP_LAUNCH((sigma_delta_grouped_kernel<32, false>));
+}
+
+cudaError_t launch_sr_requant_grouped(GroupParams& g, int blk, bool tc, uint64_t seed, uint32_t visit,
+                                      cudaStream_t st, int num_sms) {
+    if (blk == 16) {
+        if (tc) Q4_GROUP_LAUNCH((sr_requant_grouped_kernel<16, true>), seed, visit);
+        Q4_GROUP_LAUNCH((sr_requant_grouped_kernel<16, false>), seed, visit);
+    }
+    if (tc) Q4_GROUP_LAUNCH((sr_requant_grouped_kernel<32, true>), seed, visit);
+    Q4_GROUP_LAUNCH((sr_requant_grouped_kernel<32, false>), seed, visit);
+}
+
+cudaError_t launch_sigma_delta_banks_grouped(GroupParams& g, int blk, bool tc, int visits, cudaStream_t st,
+                                             int num_sms) {
+    if (blk == 16) {
+        if (tc) Q4_GROUP_LAUNCH((sigma_delta_banks_grouped_kernel<16, true>), visits);
+        Q4_GROUP_LAUNCH((sigma_delta_banks_grouped_kernel<16, false>), visits);
+    }
+    if (tc) Q4_GROUP_LAUNCH((sigma_delta_banks_grouped_kernel<32, true>), visits);
+    Q4_GROUP_LAUNCH((sigma_delta_banks_grouped_kernel<32, false>), visits);
+}
+#undef Q4_GROUP_LAUNCH
 
 }  // namespace q4

@@ -87,3 +87,40 @@ def test_host_validation_without_launch(lib):
                        None, 0, None) == 7
     # Sigma-Delta: NVFP4 needs s_t
     assert lib.q4_sigma_delta_step(q4.NVFP4, 16, P, 4, 64, P, None, P, P, 0, None) == 1
+
+
+def test_grouped_host_validation_without_launch(lib):
+    """Grouped calls check every entry as the single call would, before any launch."""
+    import mxfp4_w4a4_block_b200 as q4
+    P = 1 << 20
+    g = P + 4096
+
+    def mats(*entries):
+        arr = (q4.Q4Matrix * max(len(entries), 1))()
+        for i, e in enumerate(entries):
+            arr[i] = q4.Q4Matrix(*e)
+        return ctypes.addressof(arr), len(entries), arr
+
+    ok = (P, 4, 64, P, g, P, P)
+    a, n, keep = mats(ok, ok)
+    # more entries than Q4_MAX_GROUP, a negative count, a NULL array
+    assert lib.q4_sigma_delta_step_grouped(q4.NVFP4, 16, a, q4.MAX_GROUP + 1, 0, None) == 1
+    assert lib.q4_sigma_delta_step_grouped(q4.NVFP4, 16, a, -1, 0, None) == 1
+    assert lib.q4_sigma_delta_step_grouped(q4.NVFP4, 16, None, 2, 0, None) == 1
+    # nothing to do: no entries, or only empty matrices
+    assert lib.q4_sigma_delta_step_grouped(q4.NVFP4, 16, a, 0, 0, None) == 0
+    e, n, keep2 = mats((None, 0, 64, None, g, None, None), (None, 5, 0, None, g, None, None))
+    assert lib.q4_sr_requant_grouped(q4.NVFP4, 16, e, n, 1, 2, 0, None) == 0
+    # one bad entry fails the whole call: missing s_t, ragged columns, misaligned weights,
+    # missing residue for the step
+    for bad, want in [((P, 4, 64, P, None, P, P), 1), ((P, 4, 40, P, g, P, P), 3),
+                      ((P + 4, 4, 64, P, g, P, P), 2), ((P, 4, 64, P, g, None, P), 1)]:
+        b, n, keep3 = mats(ok, bad)
+        assert lib.q4_sigma_delta_step_grouped(q4.NVFP4, 16, b, n, 0, None) == want
+    # MXFP4 entries must not carry s_t; 4/6 scaling is NVFP4-only; codebank visit range
+    m, n, keep4 = mats((P, 4, 64, P, g, None, P))
+    assert lib.q4_quantize_grouped(q4.MXFP4, 32, q4.F32, m, n, 0, None) == 1
+    assert lib.q4_quantize_grouped(q4.MXFP4, 32, q4.F32, m, n, q4.SCALE_46, None) == 4
+    assert lib.q4_sigma_delta_codebanks_grouped(q4.NVFP4, 16, a, 2, 0, 0, None) == 1
+    # the block size must match the format
+    assert lib.q4_sr_requant_grouped(q4.NVFP4, 32, a, 2, 1, 2, 0, None) == 4
