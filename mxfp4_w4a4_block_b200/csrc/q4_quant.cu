@@ -633,15 +633,35 @@ __global__ void __launch_bounds__(sdk::THREADS, 1)
 // bytes per bank).  Optionally the final residue r_K is stored.
 // Per-unit steps below are shared by the single-matrix and the grouped
 // launches.  A unit is 8 consecutive weights of a row: u = row * (cols / 8) +
-// col / 8.  P is SigmaDeltaParams or GroupItem.
+// col / 8.  Each step is split into the unit's loads (`load8`) and its
+// arithmetic and stores (`*_finish`), so that a grouped launch can issue the
+// next unit's loads before the current unit's arithmetic.  P is
+// SigmaDeltaParams or GroupItem.
+struct In8 {
+    float4 w0, w1, r0, r1;   // weights; residue (Sigma-Delta step only)
+    uint32_t sb;             // the unit's block scale byte
+};
 
-// Reciprocal block scale of weight (row, col): 1 / (dec(s_b) s_t) (NVFP4;
-// `degenerate` when that is not a usable scale: the codes are then 0) or
-// 2^-e (MXFP4).
-template <int BLK, bool TC, class P>
-__device__ __forceinline__ float unit_inv(const P& p, int64_t row, int64_t col, float s_t, bool& degenerate) {
+template <int BLK, bool TC, bool RES, class P>
+__device__ __forceinline__ void load8(const P& p, int64_t u, In8& in) {
+    const int64_t cpr = p.cols / 8;
+    const int64_t row = u / cpr, col = (u % cpr) * 8;
+    const float4* wp = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.w) + row * p.cols + col);
+    in.w0 = __ldcs(wp);
+    in.w1 = __ldcs(wp + 1);
+    if constexpr (RES) {
+        const float4* rp = reinterpret_cast<const float4*>(p.residue + row * p.cols + col);
+        in.r0 = __ldcs(rp);
+        in.r1 = __ldcs(rp + 1);
+    }
     const int64_t c = col / BLK;
-    const uint32_t sb = TC ? p.scales[tc_scale_offset(row, c, p.catoms)] : p.scales[row * p.scols + c];
+    in.sb = TC ? p.scales[tc_scale_offset(row, c, p.catoms)] : p.scales[row * p.scols + c];
+}
+
+// Reciprocal block scale: 1 / (dec(s_b) s_t) (NVFP4; `degenerate` when that
+// is not a usable scale: the codes are then 0) or 2^-e (MXFP4).
+template <int BLK>
+__device__ __forceinline__ float inv_of(uint32_t sb, float s_t, bool& degenerate) {
     if (BLK == 16) {
         const NvScale sc = nv_scale_from_byte(sb, s_t);
         degenerate = sc.degenerate;
@@ -651,21 +671,28 @@ __device__ __forceinline__ float unit_inv(const P& p, int64_t row, int64_t col, 
     return exp2_int(127 - (int)sb);
 }
 
-template <int BLK, bool TC, class P>
-__device__ __forceinline__ void banks_unit(const P& p, int64_t u, float s_t, int visits, int64_t bank_bytes,
-                                           float* r_out) {
-    const int64_t cpr = p.cols / 8;
-    const int64_t row = u / cpr, col = (u % cpr) * 8;
-    const float4* wp = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.w) + row * p.cols + col);
-    const float4 w0 = __ldcs(wp), w1 = __ldcs(wp + 1);
+// x = w * inv for the unit's 8 weights (0 for a degenerate scale), as pairs.
+template <int BLK>
+__device__ __forceinline__ void scaled8(const In8& in, float s_t, float2 (&x)[4]) {
     bool degenerate;
-    const float inv = unit_inv<BLK, TC>(p, row, col, s_t, degenerate);
+    const float inv = inv_of<BLK>(in.sb, s_t, degenerate);
     const float2 iv = make_float2(inv, inv);
     // the products feed adds: scalar, never fused
-    float2 x[4] = {mul2_sep_rn(make_float2(w0.x, w0.y), iv), mul2_sep_rn(make_float2(w0.z, w0.w), iv),
-                   mul2_sep_rn(make_float2(w1.x, w1.y), iv), mul2_sep_rn(make_float2(w1.z, w1.w), iv)};
+    x[0] = mul2_sep_rn(make_float2(in.w0.x, in.w0.y), iv);
+    x[1] = mul2_sep_rn(make_float2(in.w0.z, in.w0.w), iv);
+    x[2] = mul2_sep_rn(make_float2(in.w1.x, in.w1.y), iv);
+    x[3] = mul2_sep_rn(make_float2(in.w1.z, in.w1.w), iv);
     if (degenerate)
         for (int j = 0; j < 4; ++j) x[j] = make_float2(0.0f, 0.0f);
+}
+
+template <int BLK, class P>
+__device__ __forceinline__ void banks_finish(const P& p, int64_t u, const In8& in, float s_t, int visits,
+                                             int64_t bank_bytes, float* r_out) {
+    const int64_t cpr = p.cols / 8;
+    const int64_t row = u / cpr, col = (u % cpr) * 8;
+    float2 x[4];
+    scaled8<BLK>(in, s_t, x);
     float2 r[4] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f),
                    make_float2(0.0f, 0.0f)};
     uint8_t* dst = p.codes + row * (p.cols / 2) + col / 2;
@@ -691,8 +718,12 @@ __global__ void __launch_bounds__(256) sigma_delta_banks_kernel(SigmaDeltaParams
                                                                 float* r_out) {
     const int64_t total = p.rows * (p.cols / 8);
     const float s_t = (BLK == 16) ? *p.gscale : 0.0f;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x)
-        banks_unit<BLK, TC>(p, i, s_t, visits, bank_bytes, r_out);
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        In8 in;
+        load8<BLK, TC, false>(p, i, in);
+        banks_finish<BLK>(p, i, in, s_t, visits, bank_bytes, r_out);
+    }
 }
 
 // ------------------------------------------------------------------ stochastic-rounding requant
@@ -703,8 +734,10 @@ __global__ void __launch_bounds__(256) sigma_delta_banks_kernel(SigmaDeltaParams
 __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint2 k) {
 #pragma unroll
     for (int round = 0; round < 10; ++round) {
-        const uint32_t hi0 = __umulhi(0xD2511F53u, c.x), lo0 = 0xD2511F53u * c.x;
-        const uint32_t hi1 = __umulhi(0xCD9E8D57u, c.z), lo1 = 0xCD9E8D57u * c.z;
+        // each 32 x 32 -> 64-bit product in one wide multiply
+        const uint64_t p0 = (uint64_t)0xD2511F53u * c.x, p1 = (uint64_t)0xCD9E8D57u * c.z;
+        const uint32_t hi0 = (uint32_t)(p0 >> 32), lo0 = (uint32_t)p0;
+        const uint32_t hi1 = (uint32_t)(p1 >> 32), lo1 = (uint32_t)p1;
         c = make_uint4(hi1 ^ c.y ^ k.x, lo1, hi0 ^ c.w ^ k.y, lo0);
         k.x += 0x9E3779B9u;
         k.y += 0xBB67AE85u;
@@ -714,37 +747,35 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint2 k) {
 
 // Stochastic rounding of a normalised value onto the E2M1 grid with the
 // uniform u in [0, 1): between neighbouring magnitudes a <= |x| < b the
-// magnitude is b when u < (|x| - a) / (b - a) (exact: the gap is 0.5, 1 or 2),
-// else a; |x| >= 6 gives 6; the sign bit is x's.
+// magnitude is b when u < (|x| - a) / (b - a), else a; |x| >= 6 gives 6; the
+// sign bit is x's.  The gap b - a is 0.5 below 2, 1 from 2 to 4 and 2 from 4
+// to 6, so with s = |x| / gap (exact: a power-of-two scaling) the lower
+// neighbour is floor(s) * gap and (|x| - a) / (b - a) = s - floor(s), both
+// exact; a's grid index is floor(s) + 0, 2 or 4 in the three ranges.
 __device__ __forceinline__ uint32_t sr_e2m1(float x, float u) {
     const float m = fabsf(x);
-    uint32_t idx;
-    if (m >= 6.0f) {
-        idx = 7;
-    } else {
-        const uint32_t i = (m >= 0.5f) + (m >= 1.0f) + (m >= 1.5f) + (m >= 2.0f) + (m >= 3.0f) + (m >= 4.0f);
-        // twice the magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6, one nibble each
-        const uint32_t twice = 0xC8643210u;
-        const float a = (float)((twice >> (4 * i)) & 0xFu) * 0.5f;
-        // 1 / (b - a): gaps 0.5 below 2, 1 from 2 to 4, 2 from 4 to 6 (exact)
-        const float rgap = (i < 4) ? 2.0f : (i < 6 ? 1.0f : 0.5f);
-        idx = (u < __fmul_rn(__fsub_rn(m, a), rgap)) ? i + 1 : i;
-    }
+    // NaN takes the first range and index 0, as the rule's comparisons give it
+    const bool lo = !(m >= 2.0f), mid = !(m >= 4.0f);
+    const float sgap = lo ? 2.0f : (mid ? 1.0f : 0.5f);
+    const float sv = __fmul_rn(m, sgap);
+    const float fl = floorf(sv);
+    const uint32_t i = (uint32_t)fl + (lo ? 0u : (mid ? 2u : 4u));
+    uint32_t idx = (u < __fsub_rn(sv, fl)) ? i + 1 : i;
+    if (m >= 6.0f) idx = 7;                 // also NaN-free saturation: |x| >= 6 takes 6
     return (signbit(x) ? 8u : 0u) | idx;
 }
 
 // One stochastic-rounding requant at a loop visit of one unit: the 8
 // weights e0 .. e0 + 7 (e0 = row * cols + col, a multiple of 8) take the two
 // Philox blocks of counters (e0/4 + {0, 1}, visit), key = seed.
-template <int BLK, bool TC, class P>
-__device__ __forceinline__ void sr_unit(const P& p, int64_t u, float s_t, uint2 key, uint32_t visit) {
+template <int BLK, class P>
+__device__ __forceinline__ void sr_finish(const P& p, int64_t u, const In8& in, float s_t, uint2 key,
+                                          uint32_t visit) {
     const int64_t cpr = p.cols / 8;
     const int64_t row = u / cpr, col = (u % cpr) * 8;
-    const float4* wp = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.w) + row * p.cols + col);
-    const float4 w0 = __ldcs(wp), w1 = __ldcs(wp + 1);
     bool degenerate;
-    const float inv = unit_inv<BLK, TC>(p, row, col, s_t, degenerate);
-    const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+    const float inv = inv_of<BLK>(in.sb, s_t, degenerate);
+    const float wv[8] = {in.w0.x, in.w0.y, in.w0.z, in.w0.w, in.w1.x, in.w1.y, in.w1.z, in.w1.w};
     const uint64_t g = (uint64_t)(row * p.cols + col) >> 2;
     const uint4 r0 = philox4x32_10(make_uint4((uint32_t)g, (uint32_t)(g >> 32), visit, 0u), key);
     const uint4 r1 = philox4x32_10(make_uint4((uint32_t)(g + 1), (uint32_t)((g + 1) >> 32), visit, 0u), key);
@@ -764,30 +795,24 @@ __global__ void __launch_bounds__(256) sr_requant_kernel(SigmaDeltaParams p, uin
     const int64_t total = p.rows * (p.cols / 8);
     const float s_t = (BLK == 16) ? *p.gscale : 0.0f;
     const uint2 key = make_uint2((uint32_t)seed, (uint32_t)(seed >> 32));
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x)
-        sr_unit<BLK, TC>(p, i, s_t, key, visit);
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        In8 in;
+        load8<BLK, TC, false>(p, i, in);
+        sr_finish<BLK>(p, i, in, s_t, key, visit);
+    }
 }
 
 // One Sigma-Delta step of one unit (as the tiled kernel above): x = w * inv,
 // v = x + r, q = E2M1(v), r <- v - q.
-template <int BLK, bool TC, class P>
-__device__ __forceinline__ void sd_unit(const P& p, int64_t u, float s_t) {
+template <int BLK, class P>
+__device__ __forceinline__ void sd_finish(const P& p, int64_t u, const In8& in, float s_t) {
     const int64_t cpr = p.cols / 8;
     const int64_t row = u / cpr, col = (u % cpr) * 8;
-    const float4* wp = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.w) + row * p.cols + col);
-    float4* rp = reinterpret_cast<float4*>(p.residue + row * p.cols + col);
-    const float4 w0 = __ldcs(wp), w1 = __ldcs(wp + 1);
-    const float4 r0 = __ldcs(rp), r1 = __ldcs(rp + 1);
-    bool degenerate;
-    const float inv = unit_inv<BLK, TC>(p, row, col, s_t, degenerate);
-    const float2 iv = make_float2(inv, inv);
-    // the products feed adds: scalar, never fused
-    float2 x[4] = {mul2_sep_rn(make_float2(w0.x, w0.y), iv), mul2_sep_rn(make_float2(w0.z, w0.w), iv),
-                   mul2_sep_rn(make_float2(w1.x, w1.y), iv), mul2_sep_rn(make_float2(w1.z, w1.w), iv)};
-    if (degenerate)
-        for (int j = 0; j < 4; ++j) x[j] = make_float2(0.0f, 0.0f);
-    const float2 r[4] = {make_float2(r0.x, r0.y), make_float2(r0.z, r0.w), make_float2(r1.x, r1.y),
-                         make_float2(r1.z, r1.w)};
+    float2 x[4];
+    scaled8<BLK>(in, s_t, x);
+    const float2 r[4] = {make_float2(in.r0.x, in.r0.y), make_float2(in.r0.z, in.r0.w),
+                         make_float2(in.r1.x, in.r1.y), make_float2(in.r1.z, in.r1.w)};
     float2 v[4], n[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) v[j] = add2_rn(x[j], r[j]);
@@ -795,6 +820,7 @@ __device__ __forceinline__ void sd_unit(const P& p, int64_t u, float s_t) {
                            (e2m1_pack4(v[2].x, v[2].y, v[3].x, v[3].y) << 16);
 #pragma unroll
     for (int j = 0; j < 4; ++j) n[j] = sub2_rn(v[j], e2m1x2_value((codes >> (8 * j)) & 0xFFu));
+    float4* rp = reinterpret_cast<float4*>(p.residue + row * p.cols + col);
     __stcs(rp, make_float4(n[0].x, n[0].y, n[1].x, n[1].y));
     __stcs(rp + 1, make_float4(n[2].x, n[2].y, n[3].x, n[3].y));
     __stcs(reinterpret_cast<unsigned int*>(p.codes + row * (p.cols / 2) + col / 2), codes);
@@ -1014,84 +1040,127 @@ __device__ __forceinline__ int group_entry(const GroupParams& g, int e, int64_t 
     return e;
 }
 
+// The grid-stride walk over a grouped launch's units.  With PIPE the loads of
+// a thread's next unit are issued before the arithmetic of its current one,
+// so every thread keeps one unit's loads in flight while it computes.
+template <bool PIPE, class In, class Load, class Finish>
+__device__ __forceinline__ void group_walk(const GroupParams& g, Load load, Finish finish) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= g.total) return;
+    int e = group_entry(g, 0, i);
+    if constexpr (!PIPE) {
+        for (; i < g.total; i += stride) {
+            e = group_entry(g, e, i);
+            In in;
+            load(e, i - g.m[e].start, in);
+            finish(e, i - g.m[e].start, in);
+        }
+    } else {
+        In cur;
+        load(e, i - g.m[e].start, cur);
+        for (;;) {
+            const int64_t n = i + stride;
+            const bool more = n < g.total;
+            int en = e;
+            In nxt;
+            if (more) {
+                en = group_entry(g, e, n);
+                load(en, n - g.m[en].start, nxt);
+            }
+            finish(e, i - g.m[e].start, cur);
+            if (!more) break;
+            i = n;
+            e = en;
+            cur = nxt;
+        }
+    }
+}
+
+// Each entry's tensor scale s_t (NVFP4), read once per CTA.
+template <int BLK>
+__device__ __forceinline__ void group_scales(const GroupParams& g, float* s_ts) {
+    if (BLK == 16)
+        for (int k = threadIdx.x; k < g.count; k += blockDim.x) s_ts[k] = *g.m[k].gscale;
+    __syncthreads();
+}
+
 template <int BLK, bool TC>
 __global__ void __launch_bounds__(256) sigma_delta_grouped_kernel(const __grid_constant__ GroupParams g) {
-    int e = -1;
-    GroupItem it;
-    float s_t = 0.0f;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < g.total; i += (int64_t)gridDim.x * blockDim.x) {
-        const int ne = group_entry(g, e < 0 ? 0 : e, i);
-        if (ne != e) {
-            e = ne;
-            it = g.m[e];
-            s_t = (BLK == 16) ? *it.gscale : 0.0f;
-        }
-        sd_unit<BLK, TC>(it, i - it.start, s_t);
-    }
+    __shared__ float s_ts[kMaxGroup];
+    group_scales<BLK>(g, s_ts);
+    group_walk<true, In8>(
+        g, [&](int e, int64_t u, In8& in) { load8<BLK, TC, true>(g.m[e], u, in); },
+        [&](int e, int64_t u, const In8& in) { sd_finish<BLK>(g.m[e], u, in, BLK == 16 ? s_ts[e] : 0.0f); });
 }
 
 template <int BLK, bool TC>
 __global__ void __launch_bounds__(256) sr_requant_grouped_kernel(const __grid_constant__ GroupParams g, uint64_t seed,
                                                                  uint32_t visit) {
+    __shared__ float s_ts[kMaxGroup];
+    group_scales<BLK>(g, s_ts);
     const uint2 key = make_uint2((uint32_t)seed, (uint32_t)(seed >> 32));
-    int e = -1;
-    GroupItem it;
-    float s_t = 0.0f;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < g.total; i += (int64_t)gridDim.x * blockDim.x) {
-        const int ne = group_entry(g, e < 0 ? 0 : e, i);
-        if (ne != e) {
-            e = ne;
-            it = g.m[e];
-            s_t = (BLK == 16) ? *it.gscale : 0.0f;
-        }
-        sr_unit<BLK, TC>(it, i - it.start, s_t, key, visit);
-    }
+    group_walk<true, In8>(
+        g, [&](int e, int64_t u, In8& in) { load8<BLK, TC, false>(g.m[e], u, in); },
+        [&](int e, int64_t u, const In8& in) {
+            sr_finish<BLK>(g.m[e], u, in, BLK == 16 ? s_ts[e] : 0.0f, key, visit);
+        });
 }
 
 template <int BLK, bool TC>
 __global__ void __launch_bounds__(256) sigma_delta_banks_grouped_kernel(const __grid_constant__ GroupParams g,
                                                                         int visits) {
-    int e = -1;
-    GroupItem it;
-    float s_t = 0.0f;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < g.total; i += (int64_t)gridDim.x * blockDim.x) {
-        const int ne = group_entry(g, e < 0 ? 0 : e, i);
-        if (ne != e) {
-            e = ne;
-            it = g.m[e];
-            s_t = (BLK == 16) ? *it.gscale : 0.0f;
-        }
-        banks_unit<BLK, TC>(it, i - it.start, s_t, visits, it.rows * (it.cols / 2), it.residue);
-    }
+    __shared__ float s_ts[kMaxGroup];
+    group_scales<BLK>(g, s_ts);
+    group_walk<true, In8>(
+        g, [&](int e, int64_t u, In8& in) { load8<BLK, TC, false>(g.m[e], u, in); },
+        [&](int e, int64_t u, const In8& in) {
+            const GroupItem& it = g.m[e];
+            banks_finish<BLK>(it, u, in, BLK == 16 ? s_ts[e] : 0.0f, visits, it.rows * (it.cols / 2), it.residue);
+        });
 }
 
 // Quantizer unit: one block, over the padded block grid in the tensor-core
 // layout (rows to a multiple of 128, blocks to a multiple of 4) so that the
 // padding scale bytes are written (0) as the tiled quantizer writes them.
-template <int BLK, bool BF16, bool TC, bool RU, bool HAD, bool S46>
-__device__ __forceinline__ void qz_unit(const GroupItem& p, int64_t u, const NvCtx& sc) {
+template <int BLK, bool BF16>
+struct QzIn {
+    uint4 raw[BLK * (BF16 ? 2 : 4) / 16];   // the block's input bytes
+    bool inside;
+};
+
+template <int BLK, bool BF16, bool TC>
+__device__ __forceinline__ void qz_load(const GroupItem& p, int64_t u, QzIn<BLK, BF16>& in) {
     const int64_t spad = TC ? p.catoms * 4 : p.scols;
     const int64_t row = u / spad, b = u % spad;
-    if (row >= p.rows || b >= p.scols) {
+    in.inside = row < p.rows && b < p.scols;
+    if (!in.inside) return;
+    const uint4* xp = reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(p.w) +
+                                                     (row * p.cols + b * BLK) * (BF16 ? 2 : 4));
+#pragma unroll
+    for (int c = 0; c < BLK * (BF16 ? 2 : 4) / 16; ++c) in.raw[c] = __ldcs(xp + c);
+}
+
+template <int BLK, bool BF16, bool TC, bool RU, bool HAD, bool S46>
+__device__ __forceinline__ void qz_finish(const GroupItem& p, int64_t u, const QzIn<BLK, BF16>& in,
+                                          const NvCtx& sc) {
+    const int64_t spad = TC ? p.catoms * 4 : p.scols;
+    const int64_t row = u / spad, b = u % spad;
+    if (!in.inside) {
         if (TC) p.scales[tc_scale_offset(row, b, p.catoms)] = 0;
         return;
     }
     float v[BLK];
-    if constexpr (BF16) {
-        const uint4* xp = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.w) + row * p.cols + b * BLK);
 #pragma unroll
-        for (int c = 0; c < BLK / 8; ++c) {
-            const uint4 raw = __ldg(xp + c);
+    for (int c = 0; c < BLK * (BF16 ? 2 : 4) / 16; ++c) {
+        const uint4 raw = in.raw[c];
+        if constexpr (BF16) {
             float* d = v + 8 * c;
             d[0] = bf16_lo(raw.x); d[1] = bf16_hi(raw.x); d[2] = bf16_lo(raw.y); d[3] = bf16_hi(raw.y);
             d[4] = bf16_lo(raw.z); d[5] = bf16_hi(raw.z); d[6] = bf16_lo(raw.w); d[7] = bf16_hi(raw.w);
-        }
-    } else {
-        const float4* xp = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.w) + row * p.cols + b * BLK);
-#pragma unroll
-        for (int c = 0; c < BLK / 4; ++c) {
-            const float4 q = __ldg(xp + c);
-            v[4 * c] = q.x; v[4 * c + 1] = q.y; v[4 * c + 2] = q.z; v[4 * c + 3] = q.w;
+        } else {
+            v[4 * c] = __uint_as_float(raw.x); v[4 * c + 1] = __uint_as_float(raw.y);
+            v[4 * c + 2] = __uint_as_float(raw.z); v[4 * c + 3] = __uint_as_float(raw.w);
         }
     }
     uint32_t byte;
@@ -1122,25 +1191,25 @@ template <int BLK, bool BF16, bool TC, bool RU, bool HAD, bool S46>
 __global__ void __launch_bounds__(256) quantize_grouped_kernel(const __grid_constant__ GroupParams g) {
     // NVFP4: each entry's 128-entry table of 1 / (dec(s_b) s_t), as the tiled quantizer's
     __shared__ float tabs[BLK == 16 ? kMaxGroup * 128 : 1];
+    __shared__ float s_ts[kMaxGroup];
     if constexpr (BLK == 16) {
         for (int k = threadIdx.x; k < g.count * 128; k += blockDim.x) {
             const NvScale r = nv_scale_from_byte((uint32_t)(k & 127), *g.m[k >> 7].gscale);
             tabs[k] = r.degenerate ? __uint_as_float(0x7FC00000u) : r.inv;
         }
+        for (int k = threadIdx.x; k < g.count; k += blockDim.x) s_ts[k] = *g.m[k].gscale;
         __syncthreads();
     }
-    int e = -1;
-    GroupItem it;
-    NvCtx sc;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < g.total; i += (int64_t)gridDim.x * blockDim.x) {
-        const int ne = group_entry(g, e < 0 ? 0 : e, i);
-        if (ne != e) {
-            e = ne;
-            it = g.m[e];
-            if constexpr (BLK == 16) sc = nv_ctx(*it.gscale, tabs + e * 128);
-        }
-        qz_unit<BLK, BF16, TC, RU, HAD, S46>(it, i - it.start, sc);
-    }
+    // a unit's loads in flight ahead of the current unit's arithmetic while that
+    // stays within 64 bytes (MXFP4 fp32 blocks are read just in time)
+    constexpr bool PIPE = BLK * (BF16 ? 2 : 4) <= 64;
+    group_walk<PIPE, QzIn<BLK, BF16>>(
+        g, [&](int e, int64_t u, QzIn<BLK, BF16>& in) { qz_load<BLK, BF16, TC>(g.m[e], u, in); },
+        [&](int e, int64_t u, const QzIn<BLK, BF16>& in) {
+            NvCtx sc;
+            if constexpr (BLK == 16) sc = nv_ctx(s_ts[e], tabs + e * 128);
+            qz_finish<BLK, BF16, TC, RU, HAD, S46>(g.m[e], u, in, sc);
+        });
 }
 
 // Entries' unit ranges; the grid is as many CTAs of 256 threads as are
