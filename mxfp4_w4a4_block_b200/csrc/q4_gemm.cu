@@ -885,31 +885,6 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64
         : "memory");
 }
 
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
-    uint32_t d;
-    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
-    return d;
-}
-
-// Eight E2M1 codes (element 0 in the low nibble) -> four packed bf16 pairs of
-// their values (element 2i in the low half of word i) with byte permutes
-// only, no conversion instructions (those run on a narrow pipe): the low and
-// high bytes of the bf16 patterns of the 8 magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6
-// are two 8-byte tables indexed by the code's low three bits, and each sign bit
-// is moved to bit 15 / 31 by a sign-replicating permute.
-__device__ __forceinline__ void e2m1x8_to_bf16(uint32_t w, uint32_t (&o)[4]) {
-    constexpr uint32_t LO0 = 0xC0800000u, LO1 = 0xC0804000u;   // low bytes: 0 0 80 C0 | 0 40 80 C0
-    constexpr uint32_t HI0 = 0x3F3F3F00u, HI1 = 0x40404040u;   // high bytes: 0 3F 3F 3F | 40 40 40 40
-    const uint32_t sel = w & 0x77777777u;
-    const uint32_t lo_a = prmt(LO0, LO1, sel), hi_a = prmt(HI0, HI1, sel);
-    const uint32_t lo_b = prmt(LO0, LO1, sel >> 16), hi_b = prmt(HI0, HI1, sel >> 16);
-    const uint32_t sg = w & 0x88888888u, sg4 = sg << 4;
-    o[0] = prmt(lo_a, hi_a, 0x5140u) | (prmt(sg4, sg, 0xC080u) & 0x80008000u);
-    o[1] = prmt(lo_a, hi_a, 0x7362u) | (prmt(sg4, sg, 0xD090u) & 0x80008000u);
-    o[2] = prmt(lo_b, hi_b, 0x5140u) | (prmt(sg4, sg, 0xE0A0u) & 0x80008000u);
-    o[3] = prmt(lo_b, hi_b, 0x7362u) | (prmt(sg4, sg, 0xF0B0u) & 0x80008000u);
-}
-
 // Two E2M1 codes (one byte, element 0 low) times a block scale, as a packed
 // bf16 pair, through the hardware E2M1 -> f16 conversion (the conversion
 // pipe; the byte-permute form above uses the integer pipe).

@@ -141,26 +141,20 @@ struct QzGeom {
 };
 
 // One candidate of 4/6 block scaling: the rounded-up E4M3 scale mapping the
-// block max to `target` (6 or 4), the block's codes under it, and their sum of
-// squared errors in the input's units, accumulated in binary64 in element
-// order (x - dec(code) * S is exact there), explicitly rounded so that no
-// fused multiply-add changes it.
-__device__ __forceinline__ void nv46_candidate(const float (&v)[16], const NvCtx& c, float amax, float target,
-                                               uint32_t& byte, uint32_t (&w)[2], double& err) {
-    byte = c.st_ok ? e4m3_ru(__fdiv_rn(amax, __fmul_rn(target, c.s_t))) : 0u;
-    const float inv = c.tab[byte];
-    err = 0.0;
-    if (inv != inv) {                       // degenerate scale: every code is +0
-        w[0] = w[1] = 0u;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const double d = (double)v[i];
-            err = __dadd_rn(err, __dmul_rn(d, d));
-        }
-        return;
-    }
-    const double S = (double)__fmul_rn(e4m3_value(byte), c.s_t);
-    const float2 iv = make_float2(inv, inv);
+// block max to `target` (6 or 4), its reciprocal from the table (NaN: a
+// degenerate scale, every code +0), S = dec(s_b) * s_t in binary32, and the
+// block's codes under it.
+struct Nv46Cand {
+    uint32_t byte, w[2];
+    float inv, S;
+};
+
+__device__ __forceinline__ Nv46Cand nv46_candidate(const float (&v)[16], const NvCtx& c, float amax, float target) {
+    Nv46Cand k;
+    k.byte = c.st_ok ? e4m3_ru(__fdiv_rn(amax, __fmul_rn(target, c.s_t))) : 0u;
+    k.inv = c.tab[k.byte];
+    k.S = __fmul_rn(e4m3_value(k.byte), c.s_t);
+    const float2 iv = make_float2(k.inv, k.inv);
 #pragma unroll
     for (int g = 0; g < 2; ++g) {
         float q[8];
@@ -170,28 +164,85 @@ __device__ __forceinline__ void nv46_candidate(const float (&v)[16], const NvCtx
             q[2 * i] = m.x;
             q[2 * i + 1] = m.y;
         }
-        w[g] = e2m1_pack8(q);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const double d = __dsub_rn((double)v[8 * g + i], __dmul_rn((double)e2m1_value((w[g] >> (4 * i)) & 15u), S));
-            err = __dadd_rn(err, __dmul_rn(d, d));
-        }
+        k.w[g] = k.inv != k.inv ? 0u : e2m1_pack8(q);
     }
+    return k;
 }
 
-// 4/6 block scaling of one NVFP4 block: the rounded-up candidate mapping the
-// block max to 4 replaces the one mapping it to 6 when its squared error is
-// strictly smaller.
+// The candidate's sum of squared errors sum_j (x_j - dec_j * S)^2 in the
+// input's units, accumulated in binary64 in element order (x - dec * S is
+// exact there), explicitly rounded so that no fused multiply-add changes it;
+// a degenerate scale gives sum_j x_j^2.
+__device__ __forceinline__ double nv46_sse_f64(const float (&v)[16], const Nv46Cand& k) {
+    double err = 0.0;
+    if (k.inv != k.inv) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const double d = (double)v[i];
+            err = __dadd_rn(err, __dmul_rn(d, d));
+        }
+        return err;
+    }
+    const double S = (double)k.S;
+#pragma unroll
+    for (int g = 0; g < 2; ++g)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const double d = __dsub_rn((double)v[8 * g + i], __dmul_rn((double)e2m1_value((k.w[g] >> (4 * i)) & 15u), S));
+            err = __dadd_rn(err, __dmul_rn(d, d));
+        }
+    return err;
+}
+
+// The same sum estimated in binary32: e_j = fma(-dec_j, S, x_j) is x_j -
+// dec_j * S correctly rounded, each square is added by one fma into one of
+// two partial sums.  While everything stays in the normal range the estimate
+// is within 20 * 2^-24 < 2^-19.6 of the exact sum, relatively (the square of
+// e_j adds at most 2^-23, each of the <= 9 additions into a partial sum and
+// the final one at most 2^-24 of what they add).  A non-finite scale gives a
+// NaN estimate.
+__device__ __forceinline__ float nv46_sse_f32(const float (&v)[16], const Nv46Cand& k) {
+    const float S = k.inv != k.inv ? 0.0f : k.S;
+    float acc0 = 0.0f, acc1 = 0.0f;
+#pragma unroll
+    for (int g = 0; g < 2; ++g) {
+        uint32_t o[4];
+        e2m1x8_to_bf16(k.w[g], o);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float d0 = __uint_as_float(o[i] << 16), d1 = __uint_as_float(o[i] & 0xFFFF0000u);
+            const float e0 = __fmaf_rn(-d0, S, v[8 * g + 2 * i]);
+            const float e1 = __fmaf_rn(-d1, S, v[8 * g + 2 * i + 1]);
+            acc0 = __fmaf_rn(e0, e0, acc0);
+            acc1 = __fmaf_rn(e1, e1, acc1);
+        }
+    }
+    return __fadd_rn(acc0, acc1);
+}
+
+// 4/6 block scaling of one NVFP4 block: the candidate with the smaller
+// binary64 squared error (ties: the 6 candidate).  Equal scale bytes give
+// equal codes, hence a tie.  Otherwise the binary32 estimates decide when
+// they differ by more than 2^-16 of their sum and both lie in [2^-100, inf):
+// each is within 2^-19.6 of its exact sum (the 2^-100 floor keeps the
+// subnormal parts of the squares below 2^-45 of the sum), so the exact sums,
+// and the binary64 sums (within 2^-48 of them), are ordered the same way.
+// Every other block takes the binary64 sums.
 __device__ __forceinline__ void nv_block46(const float (&v)[16], const NvCtx& c, uint32_t& byte, uint32_t (&w)[2]) {
     const float amax = amax_tree<16>(v);
-    uint32_t b6, b4, w6[2], w4[2];
-    double e6, e4;
-    nv46_candidate(v, c, amax, 6.0f, b6, w6, e6);
-    nv46_candidate(v, c, amax, 4.0f, b4, w4, e4);
-    const bool four = e4 < e6;
-    byte = four ? b4 : b6;
-    w[0] = four ? w4[0] : w6[0];
-    w[1] = four ? w4[1] : w6[1];
+    const Nv46Cand k6 = nv46_candidate(v, c, amax, 6.0f);
+    const Nv46Cand k4 = nv46_candidate(v, c, amax, 4.0f);
+    bool four = false;
+    if (k6.byte != k4.byte) {
+        const float e6 = nv46_sse_f32(v, k6), e4 = nv46_sse_f32(v, k4);
+        const float lo = fminf(e6, e4), hi = fmaxf(e6, e4);
+        const bool sure = e6 == e6 && e4 == e4 && hi < INFINITY && lo >= 0x1p-100f &&
+                          __fsub_rn(hi, lo) > __fmul_rn(0x1p-16f, __fadd_rn(hi, lo));
+        four = sure ? e4 < e6 : nv46_sse_f64(v, k4) < nv46_sse_f64(v, k6);
+    }
+    byte = four ? k4.byte : k6.byte;
+    w[0] = four ? k4.w[0] : k6.w[0];
+    w[1] = four ? k4.w[1] : k6.w[1];
 }
 
 // One MXFP4 block of 32 with the optional per-column multiplier and block

@@ -222,6 +222,41 @@ def test_nvfp4_scale46_parity(dtype, tc, shape):
         assert np.array_equal(host(gs).reshape(os_.shape), os_)
 
 
+def test_scale46_ties_and_near_ties():
+    """4/6 blocks whose two candidates tie or nearly tie (the kernels then take
+    the binary64 comparison): with s_t = 1 a block of values from {0, +-12, +-24}
+    with max 24 is exact under both scales (4 = 24/6 and 6 = 24/4), so both
+    squared errors are 0 and the 6 candidate wins; all-zero blocks give equal
+    scale bytes; blocks one ulp away from those give errors of nearly equal
+    size.  Random blocks fill the rest; single and grouped launches agree with
+    the oracle."""
+    rng = np.random.default_rng(46)
+    rows, cols = 256, 256
+    x = synth.small_like("weight", 461, rows, cols)
+    blocks = x.reshape(rows, cols // 16, 16)
+    exact = rng.choice(np.array([0, 12, -12, 24, -24], np.float32), size=(64, cols // 16, 16))
+    exact[:, :, 0] = 24.0
+    blocks[:64] = exact
+    blocks[64:96] = 0.0
+    near = rng.choice(np.array([0, 12, -12, 24, -24], np.float32), size=(32, cols // 16, 16))
+    near[:, :, 0] = 24.0
+    j = rng.integers(1, 16, size=(32, cols // 16))
+    sel = np.take_along_axis(near, j[..., None], axis=2)
+    np.put_along_axis(near, j[..., None], np.nextafter(sel, np.float32(np.inf)), axis=2)
+    blocks[96:128] = near
+    x = blocks.reshape(rows, cols).astype(np.float32)
+    s_t = np.float32(1.0)
+    oc, os_ = oracle.nvfp4_quantize46(x, s_t)
+    assert (os_[:64] == oracle.e4m3_encode(4.0)).all()       # the 6 candidate on exact ties
+    gc, gs = q4.q4_quantize(q4.NVFP4, dev(x), gscale=gscale_dev(s_t), flags=q4.SCALE_46 | q4.LAYOUT_TC)
+    assert np.array_equal(host(gc), oc)
+    assert np.array_equal(host(gs), oracle.scales_to_tc(os_))
+    gcs, gss = q4.q4_quantize_grouped(q4.NVFP4, [dev(x)], gscales=[gscale_dev(s_t)],
+                                      flags=q4.SCALE_46 | q4.LAYOUT_TC)
+    assert np.array_equal(host(gcs[0]), oc)
+    assert np.array_equal(host(gss[0]), oracle.scales_to_tc(os_))
+
+
 def test_scale46_sigma_delta_chain():
     """Sigma-Delta on 4/6 block scales (the page's block_scale_46(W) feeding the
     loop): eight visits bit for bit, residues within |r| <= 1."""
