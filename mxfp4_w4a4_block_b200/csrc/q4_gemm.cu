@@ -1050,9 +1050,6 @@ __global__ void __launch_bounds__(w16::THREADS, 1)
                     }
                 }
                 const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-                // the codes and scales are in registers: the stage may be refilled
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[stage]);
                 uint8_t* brow = smem + OFF_B + bs * B_SLOT + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {          // 16-byte chunk c: elements 8c .. 8c + 7
@@ -1076,7 +1073,12 @@ __global__ void __launch_bounds__(w16::THREADS, 1)
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&b_full[bs]);
+                // every code and scale of the stage has been used, so no lane's
+                // shared-memory load of it is still in flight: it may be refilled
+                if (lane == 0) {
+                    mbar_arrive(&empty[stage]);
+                    mbar_arrive(&b_full[bs]);
+                }
                 if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 if (++bs == BSLOTS) { bs = 0; bphase ^= 1; }
             }
@@ -1348,8 +1350,6 @@ __global__ void __launch_bounds__(w16p::THREADS, 1)
                         sp[q] = h | (h << 16);
                     }
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[stage]);
                 uint8_t* brow = smem + OFF_B + bs * B_SLOT + (r >> 3) * 1024 + (r & 7) * 128;
                 const uint32_t cw[4] = {cw4.x, cw4.y, cw4.z, cw4.w};
 #pragma unroll
@@ -1373,7 +1373,11 @@ __global__ void __launch_bounds__(w16p::THREADS, 1)
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(leader_b_full + 8u * (uint32_t)bs);
+                // the stage's codes and scales are all used: it may be refilled
+                if (lane == 0) {
+                    mbar_arrive(&empty[stage]);
+                    mbar_arrive_cluster(leader_b_full + 8u * (uint32_t)bs);
+                }
                 if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 if (++bs == BSLOTS) { bs = 0; bphase ^= 1; }
             }

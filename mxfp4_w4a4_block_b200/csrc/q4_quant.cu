@@ -455,8 +455,10 @@ __global__ void __launch_bounds__(qz::THREADS, 1)
                 }
             }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[stage]);
+        // the stage is handed back only once its values have been used (below):
+        // a lane's shared-memory loads may still be in flight after __syncwarp,
+        // and the refill must not overtake them
+        const int read_stage = stage;
         if (++stage == G::NSTAGE) { stage = 0; phase ^= 1; }
         if (!mbar_wait(&cfree[buf], bphase ^ 1)) break;
 
@@ -498,10 +500,14 @@ __global__ void __launch_bounds__(qz::THREADS, 1)
             if (TC) fb[(r >> 7) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + j] = (uint8_t)byte;
             else if (inside) p.scales[row * p.scols + tc * 4 + j] = (uint8_t)byte;
         }
-        // this warp's part of the staging buffer goes to the store warp
+        // this warp's part of the staging buffer goes to the store warp, and the
+        // input stage (every value of it now used) back to the producer
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&cfull[buf]);
+        if (lane == 0) {
+            mbar_arrive(&empty[read_stage]);
+            mbar_arrive(&cfull[buf]);
+        }
         if (++buf == NBUF) { buf = 0; bphase ^= 1; }
     }
 }
@@ -878,41 +884,112 @@ __device__ __forceinline__ void sd_finish(const P& p, int64_t u, const In8& in, 
 }
 
 // ------------------------------------------------------------------ dequantize
+// Eight elements from one word of codes: code * s_b (NVFP4) or code * 2^e
+// (MXFP4), exact, then one rounding for the NVFP4 tensor scale.  The code
+// values come from byte permutes (exact bf16 patterns, no conversions).
+template <int BLK>
+__device__ __forceinline__ void dq8(uint32_t codes, float sb, float s_t, float (&o)[8]) {
+    uint32_t q[4];
+    e2m1x8_to_bf16(codes, q);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        float2 v = mul2_rn(make_float2(__uint_as_float(q[j] << 16), __uint_as_float(q[j] & 0xFFFF0000u)),
+                           make_float2(sb, sb));
+        if (BLK == 16) v = mul2_rn(v, make_float2(s_t, s_t));
+        o[2 * j] = v.x;
+        o[2 * j + 1] = v.y;
+    }
+}
+
+__device__ __forceinline__ uint4 bf16x8(const float (&o)[8]) {
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(o[2 * j], o[2 * j + 1]);
+        w[j] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Two layouts of the work, each the faster one measured for its output type:
+// bf16 output: a thread owns whole blocks (its codes, BLK/2 bytes, and scale
+//   byte in one load each), and loads the next block before converting and
+//   storing the current one;
+// fp32 output: a unit is 8 elements (4 code bytes, two 16-byte stores); a warp
+//   takes 4 x 32 consecutive units, lane l the units l, l + 32, l + 64, l + 96,
+//   so every load and store instruction covers one contiguous range, and a
+//   thread issues its four units' loads before any of their arithmetic.
 template <int BLK, bool TC, bool OUT_BF16>
 __global__ void __launch_bounds__(256) dequantize_kernel(DequantParams p) {
-    const int64_t chunks_per_row = p.cols / 8;
-    const int64_t total = p.rows * chunks_per_row;
     const float s_t = (BLK == 16) ? *p.gscale : 1.0f;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t row = i / chunks_per_row;
-        const int64_t col = (i % chunks_per_row) * 8;
-        const uint32_t codes = *reinterpret_cast<const uint32_t*>(p.codes + row * (p.cols / 2) + col / 2);
-        const int64_t c = col / BLK;
-        const uint32_t byte = TC ? p.scales[tc_scale_offset(row, c, p.catoms)] : p.scales[row * p.scols + c];
-        float sc;
-        if (BLK == 16) sc = __fmul_rn(e4m3_value(byte), s_t);
-        else sc = exp2_int((int)byte - 127);
-        float o[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            float cv = e2m1_value((codes >> (4 * j)) & 15u);
-            // (code * s_b) is exact; one rounding for the tensor scale
-            o[j] = (BLK == 16) ? __fmul_rn(__fmul_rn(cv, e4m3_value(byte)), s_t) : __fmul_rn(cv, sc);
-        }
-        if (OUT_BF16) {
-            uint32_t w[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                __nv_bfloat162 h = __floats2bfloat162_rn(o[2 * j], o[2 * j + 1]);
-                w[j] = *reinterpret_cast<uint32_t*>(&h);
+    if constexpr (OUT_BF16) {
+        const int64_t total = p.rows * p.scols;
+        const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+        int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+        auto load = [&](int64_t u, uint32_t (&w)[BLK / 8], uint32_t& sb) {
+            const int64_t row = u / p.scols, b = u % p.scols;
+            const uint8_t* cp = p.codes + row * (p.cols / 2) + b * (BLK / 2);
+            if constexpr (BLK == 16) {
+                const uint2 c = __ldcs(reinterpret_cast<const uint2*>(cp));
+                w[0] = c.x; w[1] = c.y;
+            } else {
+                const uint4 c = __ldcs(reinterpret_cast<const uint4*>(cp));
+                w[0] = c.x; w[1] = c.y; w[2] = c.z; w[3] = c.w;
             }
-            *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.out) + row * p.cols + col) =
-                make_uint4(w[0], w[1], w[2], w[3]);
-        } else {
-            float4* op = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + row * p.cols + col);
-            op[0] = make_float4(o[0], o[1], o[2], o[3]);
-            op[1] = make_float4(o[4], o[5], o[6], o[7]);
+            sb = TC ? p.scales[tc_scale_offset(row, b, p.catoms)] : p.scales[row * p.scols + b];
+        };
+        if (i >= total) return;
+        uint32_t w[BLK / 8], sb;
+        load(i, w, sb);
+        for (;;) {
+            const int64_t n = i + stride;
+            uint32_t wn[BLK / 8], sbn = 0;
+            if (n < total) load(n, wn, sbn);
+            const int64_t row = i / p.scols, b = i % p.scols;
+            const float sv = (BLK == 16) ? e4m3_value(sb) : exp2_int((int)sb - 127);
+#pragma unroll
+            for (int g = 0; g < BLK / 8; ++g) {
+                float o[8];
+                dq8<BLK>(w[g], sv, s_t, o);
+                __stcs(reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.out) + row * p.cols + b * BLK + g * 8),
+                       bf16x8(o));
+            }
+            if (n >= total) break;
+            i = n;
+            sb = sbn;
+#pragma unroll
+            for (int g = 0; g < BLK / 8; ++g) w[g] = wn[g];
+        }
+    } else {
+        constexpr int U = 4;
+        const int64_t cpr = p.cols / 8;
+        const int64_t total = p.rows * cpr;
+        const int lane = threadIdx.x & 31;
+        const int64_t wid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+        const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+        for (int64_t base = wid * 32 * U; base < total; base += nw * 32 * U) {
+            uint32_t codes[U], byte[U];
+#pragma unroll
+            for (int k = 0; k < U; ++k) {
+                const int64_t u = base + k * 32 + lane;
+                if (u < total) {
+                    const int64_t row = u / cpr, col = (u % cpr) * 8;
+                    codes[k] = __ldcs(reinterpret_cast<const unsigned int*>(p.codes + row * (p.cols / 2) + col / 2));
+                    const int64_t c = col / BLK;
+                    byte[k] = TC ? p.scales[tc_scale_offset(row, c, p.catoms)] : p.scales[row * p.scols + c];
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < U; ++k) {
+                const int64_t u = base + k * 32 + lane;
+                if (u >= total) break;
+                const int64_t row = u / cpr, col = (u % cpr) * 8;
+                float o[8];
+                dq8<BLK>(codes[k], (BLK == 16) ? e4m3_value(byte[k]) : exp2_int((int)byte[k] - 127), s_t, o);
+                float4* op = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + row * p.cols + col);
+                __stcs(op, make_float4(o[0], o[1], o[2], o[3]));
+                __stcs(op + 1, make_float4(o[4], o[5], o[6], o[7]));
+            }
         }
     }
 }
@@ -922,6 +999,16 @@ static int grid_for(int64_t tiles, int num_sms, int per_sm) {
     int64_t cap = (int64_t)num_sms * per_sm;
     if (tiles < 1) return 1;
     return (int)(tiles < cap ? tiles : cap);
+}
+
+// CTAs of `threads` threads of `kernel` resident on one SM at once (>= 1): a
+// grid-stride kernel gets no more than that many per SM, since a partial
+// second wave would leave most SMs idle at the end.
+template <class K>
+static int resident_per_sm(K kernel, int threads) {
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, threads, 0) != cudaSuccess || occ < 1) occ = 1;
+    return occ;
 }
 
 struct QuantMaps {
@@ -1033,9 +1120,15 @@ cudaError_t launch_sigma_delta(const SigmaDeltaParams& p, int blk, bool tc, cuda
 cudaError_t launch_dequantize(const DequantParams& p, int blk, bool tc, bool out_bf16, cudaStream_t st,
                               int num_sms) {
     if (p.rows == 0 || p.cols == 0) return cudaSuccess;
-    const int64_t chunks = p.rows * (p.cols / 8);
-    const int grid = grid_for((chunks + 255) / 256, num_sms, 8);
-#define Q4_DQ(B, T, O) dequantize_kernel<B, T, O><<<grid, 256, 0, st>>>(p)
+    const int64_t units = p.rows * (p.cols / 8);
+    // as many CTAs as are resident at once (a second partial wave would idle most SMs)
+    // bf16 output: one block per thread-step; fp32: 4 units of 8 elements per thread-step
+    const int64_t steps = out_bf16 ? p.rows * p.scols : (units + 3) / 4;
+    auto launch = [&](auto kernel) {
+        const int grid = grid_for((steps + 255) / 256, num_sms, resident_per_sm(kernel, 256));
+        kernel<<<grid, 256, 0, st>>>(p);
+    };
+#define Q4_DQ(B, T, O) launch(dequantize_kernel<B, T, O>)
     if (blk == 16) {
         if (tc) { if (out_bf16) Q4_DQ(16, true, true); else Q4_DQ(16, true, false); }
         else { if (out_bf16) Q4_DQ(16, false, true); else Q4_DQ(16, false, false); }
@@ -1051,9 +1144,11 @@ cudaError_t launch_sigma_delta_banks(const SigmaDeltaParams& p, int blk, bool tc
                                      cudaStream_t st, int num_sms) {
     if (p.rows == 0 || p.cols == 0) return cudaSuccess;
     const int64_t chunks = p.rows * (p.cols / 8);
-    const int grid = grid_for((chunks + 255) / 256, num_sms, 8);
     const int64_t bank = p.rows * (p.cols / 2);
-#define Q4_SDB(B, T) sigma_delta_banks_kernel<B, T><<<grid, 256, 0, st>>>(p, visits, bank, r_out)
+#define Q4_SDB(B, T)                                                                                          \
+    sigma_delta_banks_kernel<B, T><<<grid_for((chunks + 255) / 256, num_sms,                                   \
+                                              resident_per_sm(sigma_delta_banks_kernel<B, T>, 256)),             \
+                                     256, 0, st>>>(p, visits, bank, r_out)
     if (blk == 16) {
         if (tc) Q4_SDB(16, true); else Q4_SDB(16, false);
     } else {
@@ -1067,8 +1162,9 @@ cudaError_t launch_sr_requant(const SigmaDeltaParams& p, int blk, bool tc, uint6
                               cudaStream_t st, int num_sms) {
     if (p.rows == 0 || p.cols == 0) return cudaSuccess;
     const int64_t chunks = p.rows * (p.cols / 8);
-    const int grid = grid_for((chunks + 255) / 256, num_sms, 8);
-#define Q4_SR(B, T) sr_requant_kernel<B, T><<<grid, 256, 0, st>>>(p, seed, visit)
+#define Q4_SR(B, T)                                                                                           \
+    sr_requant_kernel<B, T><<<grid_for((chunks + 255) / 256, num_sms, resident_per_sm(sr_requant_kernel<B, T>, 256)), \
+                              256, 0, st>>>(p, seed, visit)
     if (blk == 16) {
         if (tc) Q4_SR(16, true); else Q4_SR(16, false);
     } else {

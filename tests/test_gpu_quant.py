@@ -149,8 +149,11 @@ def test_amax_parity(dtype, n):
 @pytest.mark.parametrize("fmt", [q4.NVFP4, q4.MXFP4])
 @pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
 @pytest.mark.parametrize("tc", [False, True])
-def test_dequantize_parity(fmt, out_dtype, tc):
-    rows, cols = 130, 224
+@pytest.mark.parametrize("shape", [(130, 224), (4097, 4160)])
+def test_dequantize_parity(fmt, out_dtype, tc, shape):
+    """Bit for bit against the oracle; the larger ragged shape gives every thread
+    of the persistent grid several blocks / unit groups."""
+    rows, cols = shape
     x = synth.small_like("heavy", 5, rows, cols)
     flags = q4.LAYOUT_TC if tc else 0
     if fmt == q4.NVFP4:
@@ -220,6 +223,30 @@ def test_nvfp4_scale46_parity(dtype, tc, shape):
         assert np.array_equal(host(gs), oracle.scales_to_tc(os_))
     else:
         assert np.array_equal(host(gs).reshape(os_.shape), os_)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_quantize_repeated_launches_full_size(dtype):
+    """Ten launches of the tiled quantizer on 4097 x 4160 (ragged last row tile),
+    both scale layouts, each bit for bit against the oracle: consumer warps run
+    unsynchronised across tiles, so an input stage released before all of its
+    shared-memory reads completed would be refilled under them (seen as a few
+    wrong codes and scales in some launches)."""
+    rows, cols = 4097, 4160
+    x = synth.small_like("heavy", 5, rows, cols)
+    if dtype == "bf16":
+        xt = synth.to_bf16(x)
+        x = synth.bf16_to_f32(xt)
+        xd = dev(xt)
+    else:
+        xd = dev(x)
+    s_t = oracle.tensor_scale(oracle.amax(x), 2688.0)
+    oc, os_ = oracle.nvfp4_quantize(x, s_t)
+    for flags, o_sc in ((0, os_.reshape(-1)), (q4.LAYOUT_TC, oracle.scales_to_tc(os_))):
+        for k in range(10):
+            gc, gs = q4.q4_quantize(q4.NVFP4, xd, gscale=gscale_dev(s_t), flags=flags)
+            assert np.array_equal(host(gc), oc), f"codes, flags {flags}, launch {k}"
+            assert np.array_equal(host(gs).reshape(-1), o_sc), f"scales, flags {flags}, launch {k}"
 
 
 def test_scale46_ties_and_near_ties():
