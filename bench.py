@@ -300,8 +300,7 @@ def rows_bench(q4, dev, flush, pk, reps=30):
     yd16 = [torch.empty((16, wt.shape[0]), dtype=torch.bfloat16, device=dev) for wt, *_ in mats]
 
     def fused16():
-        for (wt, sc, g, r, c, _), yy in zip(mats, yd16):
-            q4.q4_sigma_delta_gemm(q4.NVFP4, xd16, wt, sc, r, g, y=yy)
+        q4.q4_sigma_delta_gemm_grouped(q4.NVFP4, [xd16] * len(mats), gW, gS, gR, gG, ys=yd16)
 
     def unfused16():
         q4.q4_sigma_delta_step_grouped(q4.NVFP4, gW, gS, gR, gscales=gG, codes=gC)

@@ -319,6 +319,27 @@ Q4_API q4_status q4_sigma_delta_codebanks_grouped(q4_format format, int block,
                                                   const q4_matrix* mats, int count, int visits,
                                                   int flags, void* stream);
 
+/* One matrix of q4_sigma_delta_gemm_grouped (all pointers device memory). */
+typedef struct q4_sd_gemm_entry {
+    const void* x;          /* bf16 activations [M, K] this weight multiplies */
+    const float* w;         /* FP32 master weight [N, K] */
+    const uint8_t* scales;  /* its NVFP4 block scales, tensor-core layout */
+    const float* d_gscale;  /* its tensor scale s_t (one float) */
+    float* residue;         /* its Sigma-Delta residue [N, K], read and written */
+    void* y;                /* output [M, N] of out_dt */
+    int64_t N;
+} q4_sd_gemm_entry;
+
+/* q4_sigma_delta_gemm on every entry in one launch: one loop visit of a looped
+   core whose matrices share M and K (sec. 4 of the looped page: the visit
+   requantizes and applies every weight of the core).  format = Q4_NVFP4,
+   flags = Q4_LAYOUT_TC, 1 <= M <= 16, K % 64 == 0, each N % 8 == 0;
+   0 <= count <= Q4_MAX_GROUP.  No buffer of one entry may overlap an output
+   (residue, y) of another. */
+Q4_API q4_status q4_sigma_delta_gemm_grouped(q4_format format, int block, int64_t M, int64_t K,
+                                             const q4_sd_gemm_entry* entries, int count,
+                                             q4_dtype out_dt, int flags, void* stream);
+
 /* Scratch bytes q4_gemm needs for these arguments (0 when none). */
 Q4_API size_t q4_gemm_workspace_size(q4_format format, int64_t M, int64_t N, int64_t K,
                               int a_kind);

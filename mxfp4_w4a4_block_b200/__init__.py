@@ -68,9 +68,16 @@ SIGNATURES = {
     "q4_sigma_delta_step_grouped": (_I, [_I, _I, _P, _I, _I, _P]),
     "q4_sr_requant_grouped": (_I, [_I, _I, _P, _I, ctypes.c_uint64, ctypes.c_uint32, _I, _P]),
     "q4_sigma_delta_codebanks_grouped": (_I, [_I, _I, _P, _I, _I, _I, _P]),
+    "q4_sigma_delta_gemm_grouped": (_I, [_I, _I, _I64, _I64, _P, _I, _I, _I, _P]),
 }
 
 MAX_GROUP = 32
+
+
+class Q4SdGemmEntry(ctypes.Structure):
+    """struct q4_sd_gemm_entry of include/q4.h."""
+    _fields_ = [("x", _P), ("w", _P), ("scales", _P), ("d_gscale", _P), ("residue", _P), ("y", _P),
+                ("N", _I64)]
 
 
 class Q4Matrix(ctypes.Structure):
@@ -289,6 +296,25 @@ def q4_sigma_delta_codebanks_grouped(fmt: int, ws, scales, visits: int, gscales=
                                                 _stream(stream))
     _check("q4_sigma_delta_codebanks_grouped", st)
     return codes
+
+
+def q4_sigma_delta_gemm_grouped(fmt: int, xs, ws, scales, residues, gscales, out_dtype=torch.bfloat16, ys=None,
+                                flags: int = LAYOUT_TC, stream=None):
+    """q4_sigma_delta_gemm on every (x, w, scales, residue, gscale) in one launch; the
+    entries share M and K.  Returns the list of outputs [M, N_i]."""
+    n = len(ws)
+    M, K = (xs[0].shape if n else (0, 0))
+    if ys is None:
+        ys = [torch.empty((M, w.shape[0]), dtype=out_dtype, device=w.device) for w in ws]
+    arr = (Q4SdGemmEntry * max(n, 1))()
+    for i in range(n):
+        arr[i] = Q4SdGemmEntry(_ptr(xs[i]), _ptr(ws[i]), _ptr(scales[i]), _ptr(gscales[i]), _ptr(residues[i]),
+                               _ptr(ys[i]), ws[i].shape[0])
+    dt = _dtype_code(ys[0]) if n else BF16
+    st = lib().q4_sigma_delta_gemm_grouped(fmt, BLOCK[fmt], M, K, ctypes.addressof(arr), n, dt, flags,
+                                           _stream(stream))
+    _check("q4_sigma_delta_gemm_grouped", st)
+    return ys
 
 
 def q4_sigma_delta_gemm(fmt: int, x: torch.Tensor, w: torch.Tensor, scales: torch.Tensor, residue: torch.Tensor,

@@ -265,6 +265,34 @@ q4_status q4_sigma_delta_codebanks_grouped(q4_format format, int block, const q4
                                                             (cudaStream_t)stream, num_sms()));
 }
 
+q4_status q4_sigma_delta_gemm_grouped(q4_format format, int block, int64_t M, int64_t K,
+                                      const q4_sd_gemm_entry* entries, int count, q4_dtype out_dt, int flags,
+                                      void* stream) {
+    if (!valid_format(format) || !valid_dtype(out_dt) || M < 0 || K < 0) return Q4_ERR_ARG;
+    if (block != block_of(format)) return Q4_ERR_UNSUPPORTED;
+    if (format != Q4_NVFP4 || !(flags & Q4_LAYOUT_TC) || (flags & ~Q4_LAYOUT_TC)) return Q4_ERR_UNSUPPORTED;
+    if (count < 0 || count > Q4_MAX_GROUP || (count > 0 && !entries)) return Q4_ERR_ARG;
+    if (K % 64) return Q4_ERR_SHAPE;
+    if (count == 0 || M == 0) return Q4_OK;
+    if (K == 0) return Q4_ERR_SHAPE;
+    if (!q4::sd_gemm_supported(M, K)) return Q4_ERR_UNSUPPORTED;
+    q4::SdGemmParams items[Q4_MAX_GROUP];
+    int n = 0;
+    for (int i = 0; i < count; ++i) {
+        const q4_sd_gemm_entry& e = entries[i];
+        if (e.N < 0) return Q4_ERR_ARG;
+        if (e.N % 8) return Q4_ERR_SHAPE;
+        if (e.N == 0) continue;
+        if (!e.x || !e.w || !e.scales || !e.d_gscale || !e.residue || !e.y) return Q4_ERR_ARG;
+        if (!aligned16(e.x) || !aligned16(e.w) || !aligned16(e.scales) || !aligned16(e.residue) || !aligned16(e.y))
+            return Q4_ERR_ALIGN;
+        q4::SdGemmParams& p = items[n++];
+        p.M = M; p.N = e.N; p.K = K; p.x = e.x; p.w = e.w; p.scales = e.scales; p.gscale = e.d_gscale;
+        p.residue = e.residue; p.y = e.y; p.out_bf16 = out_dt == Q4_BF16;
+    }
+    return cuda_status(q4::launch_sd_gemm_grouped(items, n, (cudaStream_t)stream, num_sms()));
+}
+
 size_t q4_gemm_workspace_size(q4_format format, int64_t M, int64_t N, int64_t K, int a_kind) {
     (void)N;
     if (a_kind != Q4_A_BF16 || format != Q4_NVFP4 || M <= 0 || K <= 0 || K % 64) return 0;

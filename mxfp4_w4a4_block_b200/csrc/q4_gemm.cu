@@ -21,6 +21,7 @@
 // scale columns in TMEM are double-buffered by k-block parity.
 // Every mbarrier wait is bounded; on time-out the kernel records an error and
 // winds down, waiting (bounded) for its own copies and MMAs before freeing TMEM.
+#include <cmath>
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
@@ -1585,9 +1586,10 @@ __device__ __forceinline__ float ld_shared_cluster_f32(uint32_t addr) {
     return v;
 }
 
-__global__ void __launch_bounds__(sdg::THREADS, 1)
-    sd_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmR,
-                          const __grid_constant__ CUtensorMap tmX, SdgDev p) {
+// One CTA of the fused step + GEMM: K slice `rank` of the 128-row band `band`
+// of the entry described by (tmW, tmR, tmX, p).
+__device__ __forceinline__ void sd_gemm_cta(const CUtensorMap& tmW, const CUtensorMap& tmR, const CUtensorMap& tmX,
+                                            const SdgDev& p, int64_t band) {
     using namespace sdg;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -1602,7 +1604,7 @@ __global__ void __launch_bounds__(sdg::THREADS, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();                        // K slice of this CTA
-    const int64_t row0 = (int64_t)blockIdx.y * BM;
+    const int64_t row0 = band * BM;
     const int64_t k_begin = (int64_t)rank * p.kslice;
     const int nst = p.kslice / KSTAGE;
     if (threadIdx.x == 0) {
@@ -1638,8 +1640,7 @@ __global__ void __launch_bounds__(sdg::THREADS, 1)
                     tma_load_2d(st + OFF_R + b * 16384, &tmR, &full[stage], k0 + 32 * b, (int32_t)row0);
                 }
                 tma_load_2d(st + OFF_X, &tmX, &full[stage], k0, 0);
-                bulk_load(st + OFF_SF, p.scales + ((int64_t)blockIdx.y * p.catoms + k0 / 64) * 512, 512u,
-                          &full[stage]);
+                bulk_load(st + OFF_SF, p.scales + (band * p.catoms + k0 / 64) * 512, 512u, &full[stage]);
                 issued[stage] = true;
                 last_phase[stage] = phase;
                 if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -1777,6 +1778,33 @@ __global__ void __launch_bounds__(sdg::THREADS, 1)
     if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
 }
 
+__global__ void __launch_bounds__(sdg::THREADS, 1)
+    sd_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmR,
+                          const __grid_constant__ CUtensorMap tmX, SdgDev p) {
+    sd_gemm_cta(tmW, tmR, tmX, p, (int64_t)blockIdx.y);
+}
+
+// Grouped: the row bands of all entries are the grid's y range, entry e
+// owning bands [band_start[e], band_start[e + 1]); every entry has the same K
+// and the same K split (the cluster shape is one per launch).
+struct SdgItem {
+    CUtensorMap w, r, x;
+    SdgDev d;
+};
+struct SdgGroup {
+    int count;
+    int band_start[kMaxGroup + 1];
+    SdgItem m[kMaxGroup];
+};
+static_assert(sizeof(SdgGroup) <= 32764, "kernel parameter space");
+
+__global__ void __launch_bounds__(sdg::THREADS, 1) sd_gemm_grouped_kernel(const __grid_constant__ SdgGroup g) {
+    int e = 0;
+    while (e + 1 < g.count && (int)blockIdx.y >= g.band_start[e + 1]) ++e;
+    const SdgItem& it = g.m[e];
+    sd_gemm_cta(it.w, it.r, it.x, it.d, (int64_t)blockIdx.y - g.band_start[e]);
+}
+
 bool sd_gemm_supported(int64_t M, int64_t K) { return M >= 1 && M <= 16 && K % 64 == 0 && K > 0; }
 
 cudaError_t launch_sd_gemm(const SdGemmParams& p, cudaStream_t st, int num_sms) {
@@ -1814,6 +1842,68 @@ cudaError_t launch_sd_gemm(const SdGemmParams& p, cudaStream_t st, int num_sms) 
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, sd_gemm_decode_kernel, mw, mr, mx, d);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+// Grouped launch: every entry has the same M, K and output type.  The K split
+// is the smallest of 1, 2, 4, 8 (dividing K into 64-element stages) whose
+// CTAs fill their last wave to at least 90 % (else the fullest): a small split
+// keeps the per-CTA fixed cost low, a ragged last wave idles most SMs.
+cudaError_t launch_sd_gemm_grouped(const SdGemmParams* items, int count, cudaStream_t st, int num_sms) {
+    using namespace sdg;
+    if (count <= 0) return cudaSuccess;
+    SdgGroup g;                         // the kernel parameter, staged on the host (14 KB)
+    std::memset(&g, 0, sizeof(g));
+    g.count = count;
+    int bands = 0;
+    for (int i = 0; i < count; ++i) {
+        g.band_start[i] = bands;
+        bands += (int)((items[i].N + BM - 1) / BM);
+    }
+    g.band_start[count] = bands;
+    const int64_t K = items[0].K;
+    int ks = 1;
+    double best = -1.0;
+    for (int c = 1; c <= MAX_KS; c *= 2) {
+        if (K % (64 * c)) break;
+        const double ctas = (double)bands * c;
+        const double waves = std::ceil(ctas / num_sms);
+        const double eff = ctas / (waves * num_sms);
+        if (eff > best + 1e-9) { best = eff; ks = c; }
+        if (eff >= 0.9) break;
+    }
+    for (int i = 0; i < count; ++i) {
+        const SdGemmParams& p = items[i];
+        SdgItem& it = g.m[i];
+        if (!encode_map_2d(&it.w, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, p.w, (uint64_t)p.K, (uint64_t)p.N,
+                           (uint64_t)p.K * 4, 32u, (uint32_t)BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !encode_map_2d(&it.r, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, p.residue, (uint64_t)p.K, (uint64_t)p.N,
+                           (uint64_t)p.K * 4, 32u, (uint32_t)BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !encode_map_2d(&it.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.x, (uint64_t)p.K, (uint64_t)p.M,
+                           (uint64_t)p.K * 2, 64u, 16u, CU_TENSOR_MAP_SWIZZLE_128B))
+            return cudaErrorInvalidValue;
+        SdgDev& d = it.d;
+        d.M = p.M; d.N = p.N; d.K = p.K; d.scales = p.scales; d.gscale = p.gscale; d.y = p.y;
+        d.catoms = ((p.K / 16) + 3) / 4;
+        d.kslice = (int)(p.K / ks);
+        d.out_bf16 = p.out_bf16 ? 1 : 0;
+    }
+    cudaError_t e = cudaFuncSetAttribute(sd_gemm_grouped_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)ks, (unsigned)bands, 1);
+    cfg.blockDim = dim3(THREADS, 1, 1);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)ks;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, sd_gemm_grouped_kernel, g);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

@@ -109,6 +109,9 @@ struct SdGemmParams {
 
 bool sd_gemm_supported(int64_t M, int64_t K);
 cudaError_t launch_sd_gemm(const SdGemmParams& p, cudaStream_t st, int num_sms);
+// Every entry as launch_sd_gemm, in one launch (entries share M, K, out_bf16;
+// count <= kMaxGroup).
+cudaError_t launch_sd_gemm_grouped(const SdGemmParams* items, int count, cudaStream_t st, int num_sms);
 cudaError_t launch_amax(const void* x, int64_t n, bool bf16, float denom, float* d_out,
                         cudaStream_t st, int num_sms);
 cudaError_t launch_quantize(const QuantParams& p, int blk, bool bf16, bool tc, bool ru, bool had,

@@ -169,3 +169,29 @@ def test_sigma_delta_gemm_matches_unfused_path():
                         a_kind=q4.A_BF16_W4A16)
         assert torch.equal(r1, r2)
         assert rel_fro(host(y1), host(y2).astype(np.float64)) <= 1e-6
+
+
+@pytest.mark.parametrize("M,K", [(16, 1024), (5, 320)])
+def test_sigma_delta_gemm_grouped(M, K):
+    """The fused step + GEMM over several weights in one launch (shared M and K,
+    each weight its own activations, N ragged against the 128-row bands): three
+    visits, every residue bit for bit against the oracle step and every Y against
+    the W4A16 oracle on the oracle's codes of that visit."""
+    Ns = [392, 1024, 136, 4096][: (4 if K == 1024 else 3)]
+    E = []
+    for i, N in enumerate(Ns):
+        w = synth.small_like("weight", 31 * i + N + K, N, K)
+        x = synth.to_bf16(synth.small_like("gauss", 7 * i + M + K, M, K))
+        s_t, g_t, g_sc, o_sc = setup_scales(q4.NVFP4, w)
+        E.append(dict(w=w, x32=synth.bf16_to_f32(x), wd=dev(w), xd=dev(x), s_t=s_t, g_t=g_t, g_sc=g_sc, o_sc=o_sc,
+                      r_gpu=torch.zeros((N, K), dtype=torch.float32, device=DEV), r_orc=np.zeros((N, K), np.float32)))
+    for visit in range(3):
+        ys = q4.q4_sigma_delta_gemm_grouped(q4.NVFP4, [e["xd"] for e in E], [e["wd"] for e in E],
+                                            [e["g_sc"] for e in E], [e["r_gpu"] for e in E], [e["g_t"] for e in E],
+                                            out_dtype=torch.float32)
+        for i, (e, N) in enumerate(zip(E, Ns)):
+            oc = oracle.sigma_delta_step(q4.NVFP4, e["w"], e["o_sc"], e["s_t"], e["r_orc"])
+            assert np.array_equal(host(e["r_gpu"]).view(np.uint32), e["r_orc"].view(np.uint32)), \
+                f"residue of entry {i}, visit {visit + 1}"
+            ref = oracle.gemm_w4a16(q4.NVFP4, e["x32"], oc, e["o_sc"], e["s_t"], M, N, K)
+            assert rel_fro(host(ys[i]), ref) <= GEMM_F32_TOL, f"Y of entry {i}, visit {visit + 1}"
