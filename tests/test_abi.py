@@ -124,3 +124,23 @@ def test_grouped_host_validation_without_launch(lib):
     assert lib.q4_sigma_delta_codebanks_grouped(q4.NVFP4, 16, a, 2, 0, 0, None) == 1
     # the block size must match the format
     assert lib.q4_sr_requant_grouped(q4.NVFP4, 32, a, 2, 1, 2, 0, None) == 4
+
+
+def test_grouped_sigma_delta_gemm_validation_without_launch(lib):
+    import mxfp4_w4a4_block_b200 as q4
+    P = 1 << 20
+    g = P + 4096
+    arr = (q4.Q4SdGemmEntry * 2)()
+    arr[0] = q4.Q4SdGemmEntry(P, P, P, g, P, P, 1024)
+    arr[1] = q4.Q4SdGemmEntry(P, P, P, g, P, P, 1020)          # N not a multiple of 8
+    a = ctypes.addressof(arr)
+    assert lib.q4_sigma_delta_gemm_grouped(q4.NVFP4, 16, 16, 1024, a, 2, q4.BF16, q4.LAYOUT_TC, None) == 3
+    assert lib.q4_sigma_delta_gemm_grouped(q4.NVFP4, 16, 16, 1000, a, 1, q4.BF16, q4.LAYOUT_TC, None) == 3
+    assert lib.q4_sigma_delta_gemm_grouped(q4.NVFP4, 16, 17, 1024, a, 1, q4.BF16, q4.LAYOUT_TC, None) == 4
+    assert lib.q4_sigma_delta_gemm_grouped(q4.MXFP4, 32, 16, 1024, a, 1, q4.BF16, q4.LAYOUT_TC, None) == 4
+    assert lib.q4_sigma_delta_gemm_grouped(q4.NVFP4, 16, 16, 1024, a, 1, q4.BF16, 0, None) == 4
+    assert lib.q4_sigma_delta_gemm_grouped(q4.NVFP4, 16, 16, 1024, a, q4.MAX_GROUP + 1, q4.BF16,
+                                           q4.LAYOUT_TC, None) == 1
+    assert lib.q4_sigma_delta_gemm_grouped(q4.NVFP4, 16, 16, 1024, a, 0, q4.BF16, q4.LAYOUT_TC, None) == 0
+    arr[0] = q4.Q4SdGemmEntry(P, P, P, None, P, P, 1024)         # missing s_t
+    assert lib.q4_sigma_delta_gemm_grouped(q4.NVFP4, 16, 16, 1024, a, 1, q4.BF16, q4.LAYOUT_TC, None) == 1
