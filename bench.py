@@ -442,7 +442,7 @@ def run_ours(args):
         iso_quant = {"shape": [M, K], "us": xq_ms * 1e3, "GB/s": xq_gbs, "frac_hbm": xq_gbs / hbm}
         del P
         torch.cuda.empty_cache()
-        rows = rows_bench(q4, dev, flush, pk)
+        rows = rows_bench(q4, dev, flush, pk, reps=args.rows_reps)
         rows["nvfp4_quantize_prefill_x"] = {"shape": [M, K], "us": k_ms[1] * 1e3, "GB/s": q_gbs,
                                             "frac_hbm": q_gbs / hbm,
                                             "note": "inside the step, right after amax (X partly in L2)"}
@@ -580,6 +580,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-rows", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--rows-reps", type=int, default=30,
+                    help="timed calls per kernel row (small values for profiler captures)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--traffic", type=float, default=GEMM_TRAFFIC_BYTES,
                     help="DRAM bytes per launch of the roofline kernel from an ncu capture")
