@@ -1,24 +1,31 @@
-// q4_gemm.cu -- block-scaled FP4 GEMM  Y = alpha * dec(A) dec(B)^T  on the
-// sm_100a tensor cores (tcgen05.mma kind::mxf4nvf4), persistent and warp
-// specialised:
+// q4_gemm.cu -- the GEMM kernels of the path, all on the sm_100a tensor cores
+// (tcgen05.mma, accumulators in TMEM), persistent and warp specialised.
+//
+// gemm_kernel: block-scaled FP4 W4A4  Y = alpha * dec(A) dec(B)^T
+// (kind::mxf4nvf4, block16 NVFP4 / block32 MXFP4):
 //   warp 0      TMA producer: A and B code tiles (128-byte swizzle) by tiled
 //               tensor copies, scale atoms by contiguous bulk copies, into a
 //               STAGES-deep ring guarded by full/empty mbarriers;
-//   warp 1      allocates TMEM, and one lane issues per k-block the copies of
-//               the A scale atoms shared memory -> TMEM (tcgen05.cp)
-//               interleaved with the block-scaled MMAs into an FP32
-//               accumulator in TMEM, from an unrolled loop over precomputed
-//               descriptors;
-//   warp 2      copies the B scale atoms into TMEM on its own, concurrently
-//               with the MMA stream (copies issued by the MMA thread would
-//               serialise with its MMAs), double-buffered by k-block parity
-//               and handed over through mbarriers;
-//   warps 3..10 epilogue: two warps per TMEM lane quarter each drain 128
-//               accumulator columns into registers (tcgen05.ld), release the
-//               accumulator to the next tile's MMAs, then scale, convert and
-//               store Y while those MMAs run.
-// CTA tile 128 x 256, k-block 256 elements (128 bytes of codes per row); the
-// scale columns in TMEM are double-buffered by k-block parity.
+//   warp 1      allocates TMEM; one lane issues each k-block's block-scaled
+//               MMAs into the FP32 accumulator from an unrolled loop over
+//               precomputed descriptors;
+//   warps 2..5  scale warps: copy each k-block's A and B scale atoms from
+//               shared memory into one of SF_NBUF TMEM scale buffers with
+//               tcgen05.st (each warp its TMEM lane quarter), off the tensor
+//               pipe that runs the MMAs, handed over through mbarriers;
+//   warps 6..13 epilogue: two warps per TMEM lane quarter drain 128
+//               accumulator columns each into registers (tcgen05.ld), release
+//               the accumulator to the next tile's MMAs, then scale, convert
+//               and store Y by TMA through a swizzled shared-memory buffer.
+// CTA tile 128 x 256, k-block 256 elements (128 bytes of codes per row).
+// gemm_pair_kernel is the same GEMM on CTA pairs (cta_group::2), off.
+//
+// w4a16_gemm_kernel: bf16 activations times the 4-bit weight dequantized
+// exactly to bf16 in shared memory by converter warps (kind::f16).
+// sd_gemm_decode_kernel / sd_gemm_grouped_kernel: the Sigma-Delta step fused
+// into that weight producer for decode shapes, K split over a cluster.
+// fused_decode_kernel: the W4A4 GEMM for M <= 16 with the activation
+// quantization fused into its producer.
 // Every mbarrier wait is bounded; on time-out the kernel records an error and
 // winds down, waiting (bounded) for its own copies and MMAs before freeing TMEM.
 #include <cmath>

@@ -1,12 +1,14 @@
 // q4_quant.cu -- memory-bound kernels of the path: tensor amax, NVFP4 / MXFP4
 // block quantization (with the optional per-channel scale and block
-// Hadamard-32 of MACaQ fused in), dequantization and the first-order
-// Sigma-Delta step of "Looped Transformer quantization", sec. 2.1.
+// Hadamard-32 of MACaQ fused in, and 4/6 block scaling), dequantization, the
+// first-order Sigma-Delta step of "Looped Transformer quantization", sec. 2.1,
+// its K-visit codebanks (sec. 2.3, 4) and the stochastic-rounding requant.
 //
 // The quantizer and the Sigma-Delta step are persistent producer/consumer
 // kernels: one thread streams tiles into shared memory by TMA, sixteen warps
-// compute, and the results leave by TMA stores (see each kernel).  amax and
-// dequantize are plain grid-stride streams.
+// compute, and the results leave by TMA stores (see each kernel).  amax,
+// dequantize, the codebanks and SR are grid-stride streams, and the grouped
+// launches walk the work units of a list of matrices grid-stride.
 #include <cstdint>
 #include <cstring>
 #include <cuda_runtime.h>
@@ -550,7 +552,10 @@ __global__ void __launch_bounds__(sdk::THREADS, 1)
     uint8_t* cbuf = smem + NSTAGE * STAGE;
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
     uint64_t* empty = full + NSTAGE;
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + NSTAGE);   // [2], see quantize_kernel
+    // consumer abort flags, indexed by tile-iteration parity: written before the
+    // per-tile consumer barrier, read after it, so every consumer takes the
+    // same decision
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + NSTAGE);
     float* inv_tab = reinterpret_cast<float*>(smem + TAB_OFF);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
