@@ -20,7 +20,9 @@
 namespace q4 {
 
 // ------------------------------------------------------------------ amax
-__global__ void __launch_bounds__(256) amax_kernel(const void* __restrict__ x, int64_t n, int bf16,
+// out[0] = max |x_i|; out[1] = out[0] / denom, written by the last CTA to
+// finish (out[1] counts the finished CTAs until then; both start at 0).
+__global__ void __launch_bounds__(256) amax_kernel(const void* __restrict__ x, int64_t n, int bf16, float denom,
                                                    unsigned int* __restrict__ out) {
     float m = 0.0f;
     const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -79,12 +81,17 @@ __global__ void __launch_bounds__(256) amax_kernel(const void* __restrict__ x, i
 #pragma unroll
         for (int o = 4; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         // magnitudes are non-negative, so their bit patterns order like integers
-        if (threadIdx.x == 0) atomicMax(out, __float_as_uint(m));
+        if (threadIdx.x == 0) {
+            atomicMax(out, __float_as_uint(m));
+            __threadfence();
+            if (atomicAdd(out + 1, 1u) == gridDim.x - 1) {
+                // every other CTA's maximum is in out[0]
+                __threadfence();
+                const float amax = __uint_as_float(atomicOr(out, 0u));
+                reinterpret_cast<float*>(out)[1] = __fdiv_rn(amax, denom);
+            }
+        }
     }
-}
-
-__global__ void amax_finalize_kernel(float* out, float denom) {
-    out[1] = __fdiv_rn(out[0], denom);
 }
 
 cudaError_t launch_amax(const void* x, int64_t n, bool bf16, float denom, float* d_out,
@@ -95,9 +102,9 @@ cudaError_t launch_amax(const void* x, int64_t n, bool bf16, float denom, float*
         int64_t vec = bf16 ? n / 8 : n / 4;
         int64_t blocks = (vec + 255) / 256;
         int grid = (int)(blocks < (int64_t)num_sms * 8 ? (blocks > 0 ? blocks : 1) : (int64_t)num_sms * 8);
-        amax_kernel<<<grid, 256, 0, st>>>(x, n, bf16 ? 1 : 0, reinterpret_cast<unsigned int*>(d_out));
+        amax_kernel<<<grid, 256, 0, st>>>(x, n, bf16 ? 1 : 0, denom, reinterpret_cast<unsigned int*>(d_out));
     }
-    amax_finalize_kernel<<<1, 1, 0, st>>>(d_out, denom);
+    // n = 0: both outputs stay 0 (= 0 / denom)
     return cudaGetLastError();
 }
 
