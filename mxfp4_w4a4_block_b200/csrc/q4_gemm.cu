@@ -1587,9 +1587,10 @@ struct SdgDev {
     int out_bf16;
 };
 
-__device__ __forceinline__ float ld_shared_cluster_f32(uint32_t addr) {
-    float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+__device__ __forceinline__ float4 ld_shared_cluster_v4(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr) : "memory");
     return v;
 }
 
@@ -1766,11 +1767,29 @@ __device__ __forceinline__ void sd_gemm_cta(const CUtensorMap& tmW, const CUtens
         const int64_t n = row0 + rr;
         const float s_t = *p.gscale;
         const uint32_t ks = (uint32_t)(p.K / p.kslice);
-        for (int m = 0; m < p.M; ++m) {
-            float acc = red[rr * 16 + m];
-            for (uint32_t q = 1; q < ks; ++q) acc += ld_shared_cluster_f32(mapa_shared(smem_u32(&red[rr * 16 + m]), q));
-            const float val = acc * s_t;
-            if (n < p.N) {
+        // this row's 16 partial sums, then each peer's 16 added in rank order;
+        // a peer's row comes as four independent 16-byte loads, not a chain of
+        // dependent scalar loads
+        float acc[16];
+#pragma unroll
+        for (int m = 0; m < 16; ++m) acc[m] = red[rr * 16 + m];
+        const uint32_t row_addr = smem_u32(&red[rr * 16]);
+        for (uint32_t q = 1; q < ks; ++q) {
+            const uint32_t peer = mapa_shared(row_addr, q);
+            float4 v[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) v[c] = ld_shared_cluster_v4(peer + 16u * c);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                acc[4 * c] += v[c].x;
+                acc[4 * c + 1] += v[c].y;
+                acc[4 * c + 2] += v[c].z;
+                acc[4 * c + 3] += v[c].w;
+            }
+        }
+        if (n < p.N) {
+            for (int m = 0; m < p.M; ++m) {
+                const float val = acc[m] * s_t;
                 if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.y)[(int64_t)m * p.N + n] = __float2bfloat16_rn(val);
                 else reinterpret_cast<float*>(p.y)[(int64_t)m * p.N + n] = val;
             }
