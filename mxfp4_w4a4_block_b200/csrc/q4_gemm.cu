@@ -1570,11 +1570,12 @@ constexpr int STAGE = 85 * 1024;
 constexpr int OFF_RED = STAGES * STAGE;  // fp32 partial tile [128][16]
 constexpr int OFF_BAR = OFF_RED + BM * 16 * 4;
 constexpr int SMEM_BYTES = OFF_BAR + 1024 + 1024;
-constexpr int CONV_WARPS = 4;
+constexpr int CONV_WARPS = 8;            // two threads per weight row, one per 32-element box
 constexpr int EPI_WARPS = 4;
 constexpr int THREADS = 32 * (2 + CONV_WARPS + EPI_WARPS);
 constexpr uint32_t TMEM_COLS = 32;
 constexpr int MAX_KS = 8;
+static_assert((32 * CONV_WARPS) % BM == 0 && 32 * CONV_WARPS / BM <= 2, "converter threads per weight row");
 }  // namespace sdg
 
 struct SdgDev {
@@ -1678,11 +1679,13 @@ __device__ __forceinline__ void sd_gemm_cta(const CUtensorMap& tmW, const CUtens
             mbar_wait(mma_done, 0);
         }
     } else if (warp < 2 + CONV_WARPS) {
-        // ---- Sigma-Delta on weight row rr of each stage
-        const int rr = threadIdx.x - 64;
+        // ---- Sigma-Delta on weight row rr of each stage, box(es) hb, hb + BPR, ...
+        const int ct = threadIdx.x - 64;
         constexpr int CT = 32 * CONV_WARPS;
+        constexpr int BPR = CT / BM;                 // threads per weight row
+        const int rr = ct % BM, hb = ct / BM;
         const float s_t = *p.gscale;
-        nv_fill_table(s_t, inv_tab, rr, CT);
+        nv_fill_table(s_t, inv_tab, ct, CT);
         named_barrier(1, CT);
         const bool row_ok = row0 + rr < p.N;
         uint32_t phase = 0;
@@ -1693,7 +1696,7 @@ __device__ __forceinline__ void sd_gemm_cta(const CUtensorMap& tmW, const CUtens
             const uint32_t sw = *reinterpret_cast<const uint32_t*>(st + OFF_SF + (rr & 31) * 16 + ((rr >> 5) & 3) * 4);
             uint8_t* arow = st + OFF_A + (rr >> 3) * 1024 + (rr & 7) * 128;
 #pragma unroll
-            for (int b = 0; b < 2; ++b) {
+            for (int b = hb; b < 2; b += BPR) {
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
                     // elements e = 32b + 4c .. +3 of the stage, block j = e / 16
@@ -1734,7 +1737,7 @@ __device__ __forceinline__ void sd_gemm_cta(const CUtensorMap& tmW, const CUtens
             if (lane == 0) mbar_arrive(&conv[stage]);
             // every row is done: store the new residue tile, release the stage once it is read
             named_barrier(1, CT);
-            if (rr == 0) {
+            if (ct == 0) {
                 if (got) {
                     const int32_t k0 = (int32_t)(k_begin + (int64_t)i * KSTAGE);
                     for (int b = 0; b < 2; ++b) tma_store_2d(&tmR, st + OFF_R + b * 16384, k0 + 32 * b, (int32_t)row0);
@@ -1745,7 +1748,7 @@ __device__ __forceinline__ void sd_gemm_cta(const CUtensorMap& tmW, const CUtens
             }
             if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
-        if (rr == 0) bulk_wait_all();
+        if (ct == 0) bulk_wait_all();
     } else {
         // ---- epilogue: partial tile to shared memory, cluster reduction
         const int quad = warp & 3;
@@ -1833,13 +1836,31 @@ __global__ void __launch_bounds__(sdg::THREADS, 1) sd_gemm_grouped_kernel(const 
 
 bool sd_gemm_supported(int64_t M, int64_t K) { return M >= 1 && M <= 16 && K % 64 == 0 && K > 0; }
 
+// K slices per row band (the cluster size, 1 to 8, dividing K into 64-element
+// stages) for `bands` row bands on `num_sms` SMs (one CTA per SM at a time):
+// the one with the least estimated time waves * (T0 + stages per CTA * TS),
+// T0 ~ 8 us the fixed cost of a CTA (set-up, first loads, cluster reduction)
+// and TS ~ 1.9 us a pipelined 64-element stage, both measured on the
+// looped-core shapes (K = 1024: splits 1 / 2 / 4 / 8 took 118 / 120 / 155 /
+// 261 us for 320 bands).
+static int choose_ksplit(int64_t bands, int64_t K, int num_sms) {
+    constexpr double T0 = 8.0, TS = 1.9;
+    int best_ks = 1;
+    double best_t = 1e300;
+    for (int ks = 1; ks <= sdg::MAX_KS; ks *= 2) {
+        if (K % (64 * ks)) break;
+        const double waves = std::ceil((double)(bands * ks) / num_sms);
+        const double t = waves * (T0 + (double)(K / ks / 64) * TS);
+        if (t < best_t) { best_t = t; best_ks = ks; }
+    }
+    return best_ks;
+}
+
 cudaError_t launch_sd_gemm(const SdGemmParams& p, cudaStream_t st, int num_sms) {
     using namespace sdg;
     if (p.M == 0 || p.N == 0) return cudaSuccess;
     const int64_t tiles = (p.N + BM - 1) / BM;
-    // K slices per row band: enough CTAs to cover the GPU, at most 8 (a portable cluster)
-    int ks = 1;
-    while (ks < MAX_KS && tiles * ks * 2 <= num_sms && p.K % (64 * (ks * 2)) == 0) ks *= 2;
+    const int ks = choose_ksplit(tiles, p.K, num_sms);
     CUtensorMap mw, mr, mx;
     if (!encode_map_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, p.w, (uint64_t)p.K, (uint64_t)p.N, (uint64_t)p.K * 4, 32u,
                        (uint32_t)BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -1872,10 +1893,8 @@ cudaError_t launch_sd_gemm(const SdGemmParams& p, cudaStream_t st, int num_sms) 
     return cudaGetLastError();
 }
 
-// Grouped launch: every entry has the same M, K and output type.  The K split
-// is the smallest of 1, 2, 4, 8 (dividing K into 64-element stages) whose
-// CTAs fill their last wave to at least 90 % (else the fullest): a small split
-// keeps the per-CTA fixed cost low, a ragged last wave idles most SMs.
+// Grouped launch: every entry has the same M, K and output type; the K split
+// comes from the same estimate over all entries' bands.
 cudaError_t launch_sd_gemm_grouped(const SdGemmParams* items, int count, cudaStream_t st, int num_sms) {
     using namespace sdg;
     if (count <= 0) return cudaSuccess;
@@ -1888,17 +1907,7 @@ cudaError_t launch_sd_gemm_grouped(const SdGemmParams* items, int count, cudaStr
         bands += (int)((items[i].N + BM - 1) / BM);
     }
     g.band_start[count] = bands;
-    const int64_t K = items[0].K;
-    int ks = 1;
-    double best = -1.0;
-    for (int c = 1; c <= MAX_KS; c *= 2) {
-        if (K % (64 * c)) break;
-        const double ctas = (double)bands * c;
-        const double waves = std::ceil(ctas / num_sms);
-        const double eff = ctas / (waves * num_sms);
-        if (eff > best + 1e-9) { best = eff; ks = c; }
-        if (eff >= 0.9) break;
-    }
+    const int ks = choose_ksplit(bands, items[0].K, num_sms);
     for (int i = 0; i < count; ++i) {
         const SdGemmParams& p = items[i];
         SdgItem& it = g.m[i];
