@@ -852,19 +852,24 @@ cudaError_t launch_gemm(const GemmParams& p, cudaStream_t st, int num_sms) {
 //                quarter, 256 columns in two halves), release it to the MMAs
 //                of the next-but-one tile, scale, convert and store Y.
 namespace w16 {
-constexpr int BM = 128;
+constexpr int BM = 128;                  // X rows of one MMA / one TMEM accumulator
+constexpr int SUBS = 2;                  // at most this many X row blocks per tile: every
+                                         // converted weight tile feeds one MMA per block
 constexpr int BN = 256;
 constexpr int KS = 64;                   // k elements per stage
-constexpr int STAGES = 5;                // TMA ring: X tile, weight codes, scale atoms
-constexpr int A_STAGE = BM * 128;        // bf16 X tile
+constexpr int A_STAGE = BM * 128;        // one bf16 X row block
 constexpr int C_STAGE = BN * 32;         // weight codes
 constexpr int S_STAGE = 1024;            // two scale atoms
-constexpr int OFF_C = A_STAGE;
-constexpr int OFF_S = OFF_C + C_STAGE;
-constexpr int STAGE = OFF_S + S_STAGE;   // 25 KB, a multiple of 1024
+// A stage holds `subs` X row blocks, the codes and the scale atoms (25 or 41 KB,
+// multiples of 1024); the ring is 5 stages deep with one block, 3 with two.
+constexpr int MAX_STAGES = 5;
+__host__ __device__ constexpr int stage_bytes(int subs) { return subs * A_STAGE + C_STAGE + S_STAGE; }
+__host__ __device__ constexpr int ring_stages(int subs) { return subs == 1 ? 5 : 3; }
+static_assert(stage_bytes(1) % 1024 == 0 && stage_bytes(2) % 1024 == 0, "stage alignment");
 constexpr int BSLOTS = 2;                // converted bf16 weight tiles
 constexpr int B_SLOT = BN * 128;
-constexpr int OFF_B = STAGES * STAGE;
+constexpr int OFF_B = ring_stages(1) * stage_bytes(1) > ring_stages(2) * stage_bytes(2)
+                          ? ring_stages(1) * stage_bytes(1) : ring_stages(2) * stage_bytes(2);
 constexpr int OFF_EPI = OFF_B + BSLOTS * B_SLOT;
 constexpr int EPI_WARPS = 4;
 constexpr int EPI_BYTES = 8192;          // per epilogue warp: 32 rows x 128 bf16
@@ -874,7 +879,8 @@ constexpr int CONV_WARPS = 8;
 constexpr int FIRST_CONV = 2;
 constexpr int FIRST_EPI = FIRST_CONV + CONV_WARPS;
 constexpr int THREADS = 32 * (FIRST_EPI + EPI_WARPS);
-constexpr uint32_t TMEM_COLS = 512;      // two accumulators
+constexpr uint32_t TMEM_COLS = 512;      // SUBS accumulators of BN columns
+static_assert(SUBS * BN <= (int)TMEM_COLS && SMEM_BYTES <= 232448, "W4A16 tile resources");
 }  // namespace w16
 
 // Instruction descriptor of tcgen05.mma kind::f16: fp32 D (bits 4-5 = 1),
@@ -918,6 +924,7 @@ struct W16Dev {
     void* y;
     int64_t catoms;
     int out_bf16;
+    int subs;                // X row blocks per tile (1 or 2)
 };
 
 template <bool MX>
@@ -927,9 +934,9 @@ __global__ void __launch_bounds__(w16::THREADS, 1)
     using namespace w16;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);    // [STAGES] X, codes, scales landed
-    uint64_t* empty = full + STAGES;                                 // [STAGES] converters read it, MMAs done
-    uint64_t* b_full = empty + STAGES;                               // [BSLOTS] weight tile converted
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);    // [stages] X, codes, scales landed
+    uint64_t* empty = full + MAX_STAGES;                             // [stages] converters read it, MMAs done
+    uint64_t* b_full = empty + MAX_STAGES;                           // [BSLOTS] weight tile converted
     uint64_t* b_empty = b_full + BSLOTS;                             // [BSLOTS] its MMAs are done
     uint64_t* tmem_full = b_empty + BSLOTS;                          // [2]
     uint64_t* tmem_empty = tmem_full + 2;                            // [2]
@@ -937,13 +944,16 @@ __global__ void __launch_bounds__(w16::THREADS, 1)
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int subs = p.subs;
+    const int STAGES = ring_stages(subs), STAGE = stage_bytes(subs);
+    const int OFF_C = subs * A_STAGE, OFF_S = OFF_C + C_STAGE;
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], CONV_WARPS + 1);        // every converter warp + the MMA commit
         }
         for (int b = 0; b < BSLOTS; ++b) { mbar_init(&b_full[b], CONV_WARPS); mbar_init(&b_empty[b], 1); }
-        for (int b = 0; b < 2; ++b) { mbar_init(&tmem_full[b], 1); mbar_init(&tmem_empty[b], EPI_WARPS); }
+        for (int b = 0; b < SUBS; ++b) { mbar_init(&tmem_full[b], 1); mbar_init(&tmem_empty[b], EPI_WARPS); }
         mbar_init(mma_done, 1);
         fence_mbar_init();
     }
@@ -958,7 +968,7 @@ __global__ void __launch_bounds__(w16::THREADS, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
 
-    const int64_t tiles_m = (p.M + BM - 1) / BM;
+    const int64_t tiles_m = (p.M + subs * BM - 1) / (subs * BM);
     const int64_t tiles = tiles_m * ((p.N + BN - 1) / BN);
     const int nks = (int)(p.K / KS);
     const int64_t bands = (p.N + 127) / 128;
@@ -967,8 +977,8 @@ __global__ void __launch_bounds__(w16::THREADS, 1)
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
-            uint32_t last_phase[STAGES];
-            bool issued[STAGES];
+            uint32_t last_phase[MAX_STAGES];
+            bool issued[MAX_STAGES];
             for (int s = 0; s < STAGES; ++s) issued[s] = false, last_phase[s] = 0;
             bool ok = true;
             for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
@@ -977,8 +987,11 @@ __global__ void __launch_bounds__(w16::THREADS, 1)
                 for (int ks = 0; ks < nks; ++ks) {
                     if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
                     uint8_t* st = smem + stage * STAGE;
-                    mbar_arrive_expect_tx(&full[stage], (uint32_t)(A_STAGE + C_STAGE + nb * 512));
-                    tma_load_2d(st, &tmX, &full[stage], ks * KS, (int32_t)(mt * BM));
+                    mbar_arrive_expect_tx(&full[stage], (uint32_t)(subs * A_STAGE + C_STAGE + nb * 512));
+                    // every X row block of the tile (rows past M read as zeros)
+                    for (int sb = 0; sb < subs; ++sb)
+                        tma_load_2d(st + sb * A_STAGE, &tmX, &full[stage], ks * KS,
+                                    (int32_t)(mt * subs * BM + sb * BM));
                     tma_load_2d(st + OFF_C, &tmC, &full[stage], ks * (KS / 2), (int32_t)(nt * BN));
                     // scale atom column of this stage: 64 elements = 4 NVFP4 blocks = one
                     // atom column; 2 MXFP4 blocks = half of one
@@ -998,28 +1011,37 @@ __global__ void __launch_bounds__(w16::THREADS, 1)
         if (lane == 0) {
             const uint32_t idesc = idesc_bf16(BM, BN);
             int stage = 0, bs = 0;
-            uint32_t phase = 0, bphase = 0, iter = 0;
+            uint32_t phase = 0, bphase = 0;
+            uint32_t uses[SUBS] = {};            // tiles each accumulator has served
             bool ok = true;
-            for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++iter) {
-                const uint32_t ab = iter & 1;
-                if (!mbar_wait(&tmem_empty[ab], ((iter >> 1) & 1) ^ 1)) { ok = false; break; }
-                tc_fence_after();
-                const uint32_t acc = tmem + ab * 256;
-                for (int ks = 0; ks < nks; ++ks) {
+            for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+                const int64_t mt = t % tiles_m;
+                // X row blocks of this tile that hold rows of X (a partial last tile skips the rest)
+                const int nsub = (int)min((int64_t)subs, (p.M - mt * subs * BM + BM - 1) / BM);
+                for (int ks = 0; ks < nks && ok; ++ks) {
                     if (!mbar_wait(&full[stage], phase) || !mbar_wait(&b_full[bs], bphase)) { ok = false; break; }
                     tc_fence_after();
-                    const uint64_t ad = smem_desc(smem_u32(smem + stage * STAGE), 16, 1024, 2);
                     const uint64_t bd = smem_desc(smem_u32(smem + OFF_B + bs * B_SLOT), 16, 1024, 2);
+                    for (int sb = 0; sb < nsub; ++sb) {
+                        if (ks == 0) {
+                            // accumulator sb drained by the epilogue of its previous tile
+                            if (!mbar_wait(&tmem_empty[sb], (uses[sb] & 1) ^ 1)) { ok = false; break; }
+                            tc_fence_after();
+                        }
+                        const uint64_t ad = smem_desc(smem_u32(smem + stage * STAGE + sb * A_STAGE), 16, 1024, 2);
+                        const uint32_t acc = tmem + sb * BN;
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16(acc, ad + 2 * kk, bd + 2 * kk, idesc, (ks > 0 || kk > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_bf16(acc, ad + 2 * kk, bd + 2 * kk, idesc, (ks > 0 || kk > 0) ? 1u : 0u);
+                        if (ks == nks - 1) tc_commit(&tmem_full[sb]);
+                    }
+                    if (!ok) break;
                     tc_commit(&empty[stage]);
                     tc_commit(&b_empty[bs]);
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                     if (++bs == BSLOTS) { bs = 0; bphase ^= 1; }
                 }
-                if (!ok) break;
-                tc_commit(&tmem_full[ab]);
+                for (int sb = 0; sb < nsub; ++sb) ++uses[sb];
             }
             tc_commit(mma_done);
             mbar_wait(mma_done, 0);
@@ -1099,16 +1121,20 @@ __global__ void __launch_bounds__(w16::THREADS, 1)
         const float alpha = MX ? 1.0f : *p.b_gscale;
         const bool out_bf16 = p.out_bf16 != 0;
         uint8_t* buf = smem + OFF_EPI + e * EPI_BYTES;
-        uint32_t iter = 0;
-        for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++iter) {
-            const uint32_t ab = iter & 1;
-            if (!mbar_wait(&tmem_full[ab], (iter >> 1) & 1)) break;
+        uint32_t uses[SUBS] = {};
+        bool ok = true;
+        for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+          const int64_t mt = t % tiles_m, nt = t / tiles_m;
+          const int nsub = (int)min((int64_t)subs, (p.M - mt * subs * BM + BM - 1) / BM);
+          for (int ab = 0; ab < nsub; ++ab) {
+            if (!mbar_wait(&tmem_full[ab], uses[ab] & 1)) { ok = false; break; }
+            ++uses[ab];
             tc_fence_after();
-            const int64_t mt = t % tiles_m, nt = t / tiles_m;
-            const int64_t row = mt * BM + quad * 32 + lane;
+            const int64_t row0 = mt * subs * BM + ab * BM;
+            const int64_t row = row0 + quad * 32 + lane;
             for (int half = 0; half < 2; ++half) {
                 const int64_t col_base = nt * BN + half * 128;
-                const uint32_t taddr = tmem + ab * 256 + ((uint32_t)(quad * 32) << 16) + half * 128;
+                const uint32_t taddr = tmem + ab * BN + ((uint32_t)(quad * 32) << 16) + half * 128;
                 if (out_bf16) {
                     // the previous stores from this buffer have finished reading it
                     if (lane == 0) bulk_wait_read_all();
@@ -1120,7 +1146,7 @@ __global__ void __launch_bounds__(w16::THREADS, 1)
                     tmem_ld32(taddr + round * 32, v);
                     tmem_ld_wait();
                     if (half == 1 && round == 3) {
-                        // the accumulator is drained: the MMAs of tile t + 2 may use it
+                        // the accumulator is drained: the next tile's MMAs may use it
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&tmem_empty[ab]);
@@ -1149,7 +1175,7 @@ __global__ void __launch_bounds__(w16::THREADS, 1)
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) {
-                        const int32_t r0 = (int32_t)(mt * BM + quad * 32);
+                        const int32_t r0 = (int32_t)(row0 + quad * 32);
                         tma_store_2d(&tmY, buf, (int32_t)col_base, r0);
                         tma_store_2d(&tmY, buf + 4096, (int32_t)(col_base + 64), r0);
                         bulk_commit_group();
@@ -1157,6 +1183,7 @@ __global__ void __launch_bounds__(w16::THREADS, 1)
                     __syncwarp();
                 }
             }
+          }
         }
         if (lane == 0) bulk_wait_all();
     }
@@ -1486,6 +1513,7 @@ cudaError_t launch_w4a16(const W4A16Params& p, cudaStream_t st, int num_sms) {
     d.w_scales = p.b_scales; d.b_gscale = p.b_gscale; d.y = p.y;
     d.catoms = ((p.K / (p.mxfp4 ? 32 : 16)) + 3) / 4;
     d.out_bf16 = p.out_bf16 ? 1 : 0;
+    d.subs = 1;
     if (pair) {
         // CTA pairs: each weight tile is dequantized once per 256 rows of X
         const int64_t ptiles = ((p.M + 2 * BM - 1) / (2 * BM)) * ((p.N + BN - 1) / BN);
@@ -1518,7 +1546,11 @@ cudaError_t launch_w4a16(const W4A16Params& p, cudaStream_t st, int num_sms) {
         if (e != cudaSuccess) return e;
         return cudaGetLastError();
     }
-    const int64_t tiles = ((p.M + BM - 1) / BM) * ((p.N + BN - 1) / BN);
+    // two X row blocks per tile (each converted weight tile feeds two MMAs) when
+    // the tiles still cover every SM, else one (more tiles, a deeper ring)
+    const int64_t tiles_n = (p.N + BN - 1) / BN;
+    d.subs = ((p.M + 2 * BM - 1) / (2 * BM)) * tiles_n >= num_sms ? 2 : 1;
+    const int64_t tiles = ((p.M + d.subs * BM - 1) / (d.subs * BM)) * tiles_n;
     const int grid = (int)(tiles < num_sms ? tiles : num_sms);
     cudaError_t e;
     if (p.mxfp4) {
