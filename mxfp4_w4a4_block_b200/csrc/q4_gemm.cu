@@ -941,7 +941,8 @@ __global__ void __launch_bounds__(w16::THREADS, 1)
     uint64_t* tmem_full = b_empty + BSLOTS;                          // [2]
     uint64_t* tmem_empty = tmem_full + 2;                            // [2]
     uint64_t* mma_done = tmem_empty + 2;
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
+    uint64_t* cfull = mma_done + 1;                                  // [stages] codes, scales landed
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(cfull + MAX_STAGES);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int subs = p.subs;
@@ -950,6 +951,7 @@ __global__ void __launch_bounds__(w16::THREADS, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
+            mbar_init(&cfull[s], 1);
             mbar_init(&empty[s], CONV_WARPS + 1);        // every converter warp + the MMA commit
         }
         for (int b = 0; b < BSLOTS; ++b) { mbar_init(&b_full[b], CONV_WARPS); mbar_init(&b_empty[b], 1); }
@@ -987,25 +989,31 @@ __global__ void __launch_bounds__(w16::THREADS, 1)
                 for (int ks = 0; ks < nks; ++ks) {
                     if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
                     uint8_t* st = smem + stage * STAGE;
-                    mbar_arrive_expect_tx(&full[stage], (uint32_t)(subs * A_STAGE + C_STAGE + nb * 512));
-                    // every X row block of the tile (rows past M read as zeros)
-                    for (int sb = 0; sb < subs; ++sb)
-                        tma_load_2d(st + sb * A_STAGE, &tmX, &full[stage], ks * KS,
-                                    (int32_t)(mt * subs * BM + sb * BM));
-                    tma_load_2d(st + OFF_C, &tmC, &full[stage], ks * (KS / 2), (int32_t)(nt * BN));
+                    // the weight codes and scale atoms first, on their own barrier: the
+                    // converters start while the X row blocks are still landing
+                    mbar_arrive_expect_tx(&cfull[stage], (uint32_t)(C_STAGE + nb * 512));
+                    tma_load_2d(st + OFF_C, &tmC, &cfull[stage], ks * (KS / 2), (int32_t)(nt * BN));
                     // scale atom column of this stage: 64 elements = 4 NVFP4 blocks = one
                     // atom column; 2 MXFP4 blocks = half of one
                     const int64_t acol = MX ? ks / 2 : ks;
                     for (int b = 0; b < nb; ++b)
                         bulk_load(st + OFF_S + b * 512, p.w_scales + ((nt * 2 + b) * p.catoms + acol) * 512, 512u,
-                                  &full[stage]);
+                                  &cfull[stage]);
+                    mbar_arrive_expect_tx(&full[stage], (uint32_t)(subs * A_STAGE));
+                    // every X row block of the tile (rows past M read as zeros)
+                    for (int sb = 0; sb < subs; ++sb)
+                        tma_load_2d(st + sb * A_STAGE, &tmX, &full[stage], ks * KS,
+                                    (int32_t)(mt * subs * BM + sb * BM));
                     issued[stage] = true;
                     last_phase[stage] = phase;
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
             }
             for (int s = 0; s < STAGES; ++s)
-                if (issued[s]) mbar_wait(&full[s], last_phase[s]);
+                if (issued[s]) {
+                    mbar_wait(&cfull[s], last_phase[s]);
+                    mbar_wait(&full[s], last_phase[s]);
+                }
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -1056,7 +1064,7 @@ __global__ void __launch_bounds__(w16::THREADS, 1)
             const int64_t nt = t / tiles_m;
             const bool row_ok = nt * BN + r < p.N;
             for (int ks = 0; ks < nks; ++ks) {
-                if (!mbar_wait(&full[stage], phase) || !mbar_wait(&b_empty[bs], bphase ^ 1)) { ok = false; break; }
+                if (!mbar_wait(&cfull[stage], phase) || !mbar_wait(&b_empty[bs], bphase ^ 1)) { ok = false; break; }
                 uint8_t* st = smem + stage * STAGE;
                 const uint4 c0 = *reinterpret_cast<const uint4*>(st + OFF_C + r * 32);
                 const uint4 c1 = *reinterpret_cast<const uint4*>(st + OFF_C + r * 32 + 16);
