@@ -99,9 +99,9 @@ def test_gemm_closed_form_integer_case():
 
 @pytest.mark.parametrize("M,K", [(1, 1088), (16, 1088), (33, 1216), (64, 1152), (65, 1088), (128, 1088)])
 def test_fused_activation_quant_decode_small(M, K):
-    """a_kind = A_BF16 for small M: the kernel quantizes the bf16 activations
-    itself (M <= 64; larger M quantizes once into the workspace).  K leaves
-    partial last k-blocks of 64, 192 and 128 elements; N a partial tile."""
+    """a_kind = A_BF16 for small M: the GEMM launch quantizes the bf16
+    activations itself (M <= 16; larger M quantizes once into the workspace).
+    K leaves partial last k-blocks of 64, 192 and 128 elements; N a partial tile."""
     N = 392
     x = synth.to_bf16(synth.small_like("heavy", M, M, K))
     x32 = synth.bf16_to_f32(x)
@@ -112,6 +112,24 @@ def test_fused_activation_quant_decode_small(M, K):
         y = q4.q4_gemm(q4.NVFP4, M, N, K, dev(x), None, A.g_t, B.codes, B.scales, B.g_t, out_dtype=od,
                        a_kind=q4.A_BF16)
         check(y, oracle_gemm(A, B), od)
+
+
+@pytest.mark.parametrize("M,K,many_tiles", [(3, 320, True), (16, 8256, False)])
+def test_fused_decode_more_tiles_than_sms_and_long_k(M, K, many_tiles):
+    """Fused decode with more 128-row weight tiles than SMs (CTAs take a second
+    tile and quantize the activations again for it), and with 33 k-blocks
+    (K = 8256, the activation ring wraps several times); called twice with new
+    activations on the second call."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    N = (sms + 4) * 128 + 64 if many_tiles else 392
+    w = synth.small_like("weight", 6, N, K)
+    B = Operand(q4.NVFP4, w)
+    for seed in (5, 7):
+        x = synth.to_bf16(synth.small_like("heavy", seed, M, K))
+        A = Operand(q4.NVFP4, synth.bf16_to_f32(x), x_t=dev(x))
+        y = q4.q4_gemm(q4.NVFP4, M, N, K, dev(x), None, A.g_t, B.codes, B.scales, B.g_t,
+                       out_dtype=torch.float32, a_kind=q4.A_BF16)
+        check(y, oracle_gemm(A, B), torch.float32)
 
 
 def test_fused_activation_quant_prefill_path():
