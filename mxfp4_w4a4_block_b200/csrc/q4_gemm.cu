@@ -2010,8 +2010,12 @@ constexpr int FIRST_E = FIRST_Q + QWARPS;
 constexpr int THREADS = 32 * (FIRST_E + EWARPS);
 constexpr int W_STAGE = 128 * 128;       // weight codes of one k-block
 constexpr int SFW_STAGE = 4 * 512;       // their scale atoms
-constexpr int XSLOTS = 9;               // bf16 activation slabs (per-thread cp.async ring)
-constexpr int XDIST = 8;                // k-blocks fetched ahead (< XSLOTS): the fetch waits behind the weight stream
+// The weight ring's depth sets the pace (a stage is refilled only after its
+// MMAs complete, so the bytes in flight per SM over the loaded round trip
+// bound the stream): the activation slabs are kept to 4 so that 9 weight
+// stages fit in shared memory rather than 7 (26.6 -> 24.6 us at 16 x 17408 x 5120).
+constexpr int XSLOTS = 4;               // bf16 activation slabs (per-thread cp.async ring)
+constexpr int XDIST = 3;                // k-blocks fetched ahead (< XSLOTS)
 constexpr int QSLOTS = 6;               // quantized activation k-blocks ahead of the MMAs
 constexpr int SFX = 4 * 512;             // activation scale atoms of one k-block
 constexpr int MAX_M = 16;
