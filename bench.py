@@ -377,8 +377,7 @@ def run_ours(args):
     torch.cuda.synchronize()
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
-    out_dir = ROOT / "gpurun_out"
-    clock_path = out_dir / "bench_clocks.csv" if out_dir.is_dir() else None
+    clock_path = Path(args.clocks_csv) if args.clocks_csv else None
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
@@ -580,6 +579,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-rows", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--clocks-csv", default=None,
+                    help="also write the clock samples taken during the timed steps to this CSV file")
     ap.add_argument("--rows-reps", type=int, default=30,
                     help="timed calls per kernel row (small values for profiler captures)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
