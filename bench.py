@@ -16,7 +16,8 @@ Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|referen
 N > 1 runs under torchrun, one process per GPU, each rank running the same
 workload on its own GPU (the problems are independent: weak scaling, no
 collective on the data path; NCCL only for the barrier and the max-over-ranks
-timing).  L2 is flushed (a 256 MiB write) between timed steps.
+timing).  L2 is flushed (a 256 MiB write, then a 256 MiB read, so that no
+dirty line is left) before every timed step.
 """
 from __future__ import annotations
 
@@ -345,11 +346,33 @@ def rows_bench(q4, dev, flush, pk, reps=30):
     return out
 
 
+def rank_env():
+    """(rank, world size, local rank) as the launcher sets them; a plain
+    single-process run is rank 0 of 1."""
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(x: float, dist, device) -> float:
+    """The slowest rank's figure.  Every rank calls this at the same point (the
+    collective order is the same on all ranks); `dist` None = one process."""
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(world: int, flops_per_rank_step: float, step_ms: float) -> float:
+    """Whole-job throughput: every rank runs its own copy of the step (weak
+    scaling), so the job does world x the step's FLOPs in the slowest rank's
+    step time."""
+    return world * flops_per_rank_step / (step_ms * 1e-3) / 1e12
+
+
 def run_ours(args):
     import mxfp4_w4a4_block_b200 as q4
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, world, local = rank_env()
     dist = None
     if world > 1:
         import datetime
@@ -391,18 +414,14 @@ def run_ours(args):
         dist.barrier()
     wall = time.perf_counter() - wall0
     seg = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)] for i in range(args.steps)])
-    step_ms = float(seg.sum(axis=1).mean())
-    if dist is not None:
-        t = torch.tensor([step_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        step_ms = float(t.item())
+    step_ms = max_over_ranks(float(seg.sum(axis=1).mean()), dist, dev)
     clocks = cs.summary()
     k_ms = seg.mean(axis=0)          # amax, quantize, gemm1, gemm2
     gemm2_tf = 2.0 * M * N2 * K / (k_ms[3] * 1e-3) / 1e12
     gemm1_tf = 2.0 * M * N1 * K / (k_ms[2] * 1e-3) / 1e12
     q_gbs = M * K * B_QUANT_BF16 / (k_ms[1] * 1e-3) / 1e9
     a_gbs = M * K * B_AMAX_BF16 / (k_ms[0] * 1e-3) / 1e9
-    value = world * GEMM_FLOPS / (step_ms * 1e-3) / 1e12
+    value = whole_job_tflops(world, GEMM_FLOPS, step_ms)
 
     # end to end through the C ABI with host buffers: pinned X in, both Y out
     e2e = None
@@ -423,12 +442,8 @@ def run_ours(args):
             e.synchronize()
             if i >= 2:
                 ts.append(s.elapsed_time(e))
-        e2e_ms = statistics.mean(ts)
-        if dist is not None:
-            t = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": world * GEMM_FLOPS / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+        e2e_ms = max_over_ranks(statistics.mean(ts), dist, dev)
+        e2e = {"value": whole_job_tflops(world, GEMM_FLOPS, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": int(P.x_host.numel() * 2),
                "d2h_bytes_per_step": int(sum(y.numel() * 2 for y in P.y)), "ms_per_step": e2e_ms}
 
@@ -534,7 +549,7 @@ def cpu_baseline(budget_s: float = 15.0):
 def run_reference(args):
     """The oracle arm: each step is a bounded sample of the prefill workload
     sized so that warm-up + timed steps take about two minutes in total."""
-    rank = int(os.environ.get("RANK", "0"))
+    rank, _, _ = rank_env()
     if rank != 0:
         return
     smp = OracleSample(rows=16, cols=64)
