@@ -1202,318 +1202,15 @@ __global__ void __launch_bounds__(w16::THREADS, 1)
     if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
 }
 
-// ------------------------------------------------------------------ W4A16 GEMM on CTA pairs
-// The same W4A16 GEMM on clusters of two CTAs sharing each MMA (cta_group::2):
-// a pair owns a 256 x 256 output tile, each CTA loads its own 128 rows of X
-// and dequantizes its own 128 rows of the 256-row weight tile, and the first
-// CTA issues 256 x 256 x 16 MMAs for both SMs -- so every weight tile is
-// dequantized once per 256 rows of X instead of once per 128, halving the
-// converters' work per MMA.  Both CTAs' X copies complete on the first CTA's
-// `xfull` barriers; both CTAs' converters release a converted slot to the
-// first CTA's `b_full`; the MMA commits are multicast to both CTAs' `empty`,
-// `b_empty` and `tmem_full`; both CTAs' epilogue warps release an
-// accumulator on the first CTA's `tmem_empty`.
-namespace w16p {
-constexpr int BM = 128;                  // rows of X per CTA (256 per pair)
-constexpr int BN = 256;                  // weight rows per pair tile (128 per CTA)
-constexpr int KS = 64;
-constexpr int STAGES = 6;
-constexpr int A_STAGE = BM * 128;        // 16 KB bf16 X tile
-constexpr int C_STAGE = 128 * 32;        // 4 KB: this CTA's weight-code rows
-constexpr int OFF_C = A_STAGE;
-constexpr int OFF_S = OFF_C + C_STAGE;   // one scale atom (this CTA's band)
-constexpr int STAGE = 21 * 1024;
-constexpr int BSLOTS = 2;
-constexpr int B_SLOT = 128 * 128;        // 16 KB: this CTA's half of the bf16 weight tile
-constexpr int OFF_B = STAGES * STAGE;
-constexpr int EPI_WARPS = 4;
-constexpr int EPI_BYTES = 8192;
-constexpr int OFF_EPI = OFF_B + BSLOTS * B_SLOT;
-constexpr int OFF_BAR = OFF_EPI + EPI_WARPS * EPI_BYTES;
-constexpr int SMEM_BYTES = OFF_BAR + 512 + 1024;
-constexpr int CONV_WARPS = 8;            // two threads per weight row
-constexpr int FIRST_CONV = 2;
-constexpr int FIRST_EPI = FIRST_CONV + CONV_WARPS;
-constexpr int THREADS = 32 * (FIRST_EPI + EPI_WARPS);
-constexpr uint32_t TMEM_COLS = 512;      // two accumulators
-}  // namespace w16p
-
-__device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                              uint32_t acc) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
-        : "memory");
-}
-
-template <bool MX>
-__global__ void __launch_bounds__(w16p::THREADS, 1)
-    w4a16_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmC,
-                      const __grid_constant__ CUtensorMap tmY, W16Dev p) {
-    using namespace w16p;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* xfull = reinterpret_cast<uint64_t*>(smem + OFF_BAR);  // [STAGES] (first CTA's) both X tiles landed
-    uint64_t* cfull = xfull + STAGES;                                // [STAGES] this CTA's codes + scales landed
-    uint64_t* empty = cfull + STAGES;                                // [STAGES] converters read it, MMAs done
-    uint64_t* b_full = empty + STAGES;                               // [BSLOTS] (first CTA's) both halves converted
-    uint64_t* b_empty = b_full + BSLOTS;                             // [BSLOTS] its MMAs are done
-    uint64_t* tmem_full = b_empty + BSLOTS;                          // [2]
-    uint64_t* tmem_empty = tmem_full + 2;                            // [2] (first CTA's) both epilogues drained
-    uint64_t* mma_done = tmem_empty + 2;
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint32_t rank = cluster_ctarank();
-    const bool leader = rank == 0;
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&xfull[s], 1);
-            mbar_init(&cfull[s], 1);
-            mbar_init(&empty[s], CONV_WARPS + 1);
-        }
-        for (int b = 0; b < BSLOTS; ++b) { mbar_init(&b_full[b], 2 * CONV_WARPS); mbar_init(&b_empty[b], 1); }
-        for (int b = 0; b < 2; ++b) { mbar_init(&tmem_full[b], 1); mbar_init(&tmem_empty[b], 2 * EPI_WARPS); }
-        mbar_init(mma_done, 1);
-        fence_mbar_init();
-    }
-    if (warp == 1) { tmem_alloc2(tmem_holder, TMEM_COLS); tmem_relinquish2(); }
-    if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(&tmX);
-        tma_prefetch_desc(&tmC);
-        if (p.out_bf16) tma_prefetch_desc(&tmY);
-    }
-    tc_fence_before();
-    __syncthreads();
-    cluster_sync();          // barriers and TMEM allocation are visible to the peer
-    tc_fence_after();
-    const uint32_t tmem = *tmem_holder;
-
-    const int64_t tiles_m = (p.M + 2 * BM - 1) / (2 * BM);
-    const int64_t tiles = tiles_m * ((p.N + BN - 1) / BN);
-    const int64_t pair_id = blockIdx.x / 2, npairs = gridDim.x / 2;
-    const int nks = (int)(p.K / KS);
-    const int64_t bands = (p.N + 127) / 128;
-
-    if (warp == 0) {
-        if (lane == 0) {
-            const uint32_t leader_xfull = mapa_shared(smem_u32(xfull), 0);
-            int stage = 0;
-            uint32_t phase = 0;
-            uint32_t last_phase[STAGES];
-            bool issued[STAGES];
-            for (int s = 0; s < STAGES; ++s) issued[s] = false, last_phase[s] = 0;
-            bool ok = true;
-            for (int64_t t = pair_id; t < tiles && ok; t += npairs) {
-                const int64_t mt = t % tiles_m, nt = t / tiles_m;
-                const int64_t band = nt * 2 + rank;                  // this CTA's 128 weight rows
-                for (int ks = 0; ks < nks; ++ks) {
-                    if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
-                    uint8_t* st = smem + stage * STAGE;
-                    if (leader) mbar_arrive_expect_tx(&xfull[stage], 2u * A_STAGE);
-                    tma_load_2d_pair(st, &tmX, leader_xfull + 8u * (uint32_t)stage, ks * KS,
-                                     (int32_t)(mt * 2 * BM + rank * BM));
-                    const bool has_band = band < bands;
-                    mbar_arrive_expect_tx(&cfull[stage], (uint32_t)(C_STAGE + (has_band ? 512 : 0)));
-                    tma_load_2d(st + OFF_C, &tmC, &cfull[stage], ks * (KS / 2), (int32_t)(band * 128));
-                    if (has_band)
-                        bulk_load(st + OFF_S, p.w_scales + (band * p.catoms + (MX ? ks / 2 : ks)) * 512, 512u,
-                                  &cfull[stage]);
-                    issued[stage] = true;
-                    last_phase[stage] = phase;
-                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
-                }
-            }
-            for (int s = 0; s < STAGES; ++s)
-                if (issued[s]) {
-                    mbar_wait(&cfull[s], last_phase[s]);
-                    if (leader) mbar_wait(&xfull[s], last_phase[s]);
-                }
-        }
-    } else if (warp == 1) {
-        if (lane == 0 && leader) {
-            const uint32_t idesc = idesc_bf16(2 * BM, BN);
-            int stage = 0, bs = 0;
-            uint32_t phase = 0, bphase = 0, iter = 0;
-            bool ok = true;
-            for (int64_t t = pair_id; t < tiles && ok; t += npairs, ++iter) {
-                const uint32_t ab = iter & 1;
-                if (!mbar_wait_cluster(&tmem_empty[ab], ((iter >> 1) & 1) ^ 1)) { ok = false; break; }
-                tc_fence_after();
-                const uint32_t acc = tmem + ab * 256;
-                for (int ks = 0; ks < nks; ++ks) {
-                    if (!mbar_wait(&xfull[stage], phase) || !mbar_wait_cluster(&b_full[bs], bphase)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint64_t ad = smem_desc(smem_u32(smem + stage * STAGE), 16, 1024, 2);
-                    const uint64_t bd = smem_desc(smem_u32(smem + OFF_B + bs * B_SLOT), 16, 1024, 2);
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16_pair(acc, ad + 2 * kk, bd + 2 * kk, idesc, (ks > 0 || kk > 0) ? 1u : 0u);
-                    tc_commit_pair_mc(&empty[stage], 0x3);
-                    tc_commit_pair_mc(&b_empty[bs], 0x3);
-                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
-                    if (++bs == BSLOTS) { bs = 0; bphase ^= 1; }
-                }
-                if (!ok) break;
-                tc_commit_pair_mc(&tmem_full[ab], 0x3);
-            }
-            tc_commit_pair(mma_done);
-            mbar_wait(mma_done, 0);
-        }
-    } else if (warp < FIRST_EPI) {
-        // ---- converters: two threads per weight row (32 codes each)
-        const int t = threadIdx.x - 32 * FIRST_CONV;
-        const int r = t >> 1, hf = t & 1;
-        const uint32_t leader_b_full = mapa_shared(smem_u32(b_full), 0);
-        int stage = 0, bs = 0;
-        uint32_t phase = 0, bphase = 0;
-        bool ok = true;
-        for (int64_t tile = pair_id; tile < tiles && ok; tile += npairs) {
-            const int64_t nt = tile / tiles_m;
-            const bool row_ok = (nt * 2 + rank) * 128 + r < p.N;
-            for (int ks = 0; ks < nks; ++ks) {
-                if (!mbar_wait(&cfull[stage], phase) || !mbar_wait(&b_empty[bs], bphase ^ 1)) { ok = false; break; }
-                uint8_t* st = smem + stage * STAGE;
-                const uint4 cw4 = *reinterpret_cast<const uint4*>(st + OFF_C + r * 32 + hf * 16);
-                const uint32_t sw = *reinterpret_cast<const uint32_t*>(st + OFF_S + (r & 31) * 16 + ((r >> 5) & 3) * 4);
-                // block scales of this thread's two 16-element blocks (NVFP4) or its one 32-block (MXFP4)
-                uint32_t sp[2];
-                if (MX) {
-                    const int j = (ks & 1) * 2 + hf;
-                    const uint32_t a = __float_as_uint(exp2_int((int)((sw >> (8 * j)) & 0xFFu) - 127)) >> 16;
-                    sp[0] = sp[1] = a | (a << 16);
-                } else {
-#pragma unroll
-                    for (int q = 0; q < 2; ++q) {
-                        const uint32_t h = __float_as_uint(e4m3_value((sw >> (8 * (2 * hf + q))) & 0xFFu)) >> 16;
-                        sp[q] = h | (h << 16);
-                    }
-                }
-                uint8_t* brow = smem + OFF_B + bs * B_SLOT + (r >> 3) * 1024 + (r & 7) * 128;
-                const uint32_t cw[4] = {cw4.x, cw4.y, cw4.z, cw4.w};
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {          // chunk c = 4 hf + q: elements 8c .. 8c + 7
-                    const int c = 4 * hf + q;
-                    const uint32_t sc = sp[q >> 1];
-                    uint4 v;
-                    if (q & 1) {
-                        const float f = __uint_as_float(sc << 16);
-                        const float2 f2 = make_float2(f, f);
-                        v = make_uint4(dequant2_bf16(cw[q] & 0xFFu, f2), dequant2_bf16((cw[q] >> 8) & 0xFFu, f2),
-                                       dequant2_bf16((cw[q] >> 16) & 0xFFu, f2), dequant2_bf16(cw[q] >> 24, f2));
-                    } else {
-                        uint32_t o[4];
-                        e2m1x8_to_bf16(cw[q], o);
-                        v = make_uint4(mul_bf16x2(o[0], sc), mul_bf16x2(o[1], sc), mul_bf16x2(o[2], sc),
-                                       mul_bf16x2(o[3], sc));
-                    }
-                    if (!row_ok) v = make_uint4(0u, 0u, 0u, 0u);
-                    *reinterpret_cast<uint4*>(brow + ((c ^ (r & 7)) << 4)) = v;
-                }
-                fence_proxy_async_smem();
-                __syncwarp();
-                // the stage's codes and scales are all used: it may be refilled
-                if (lane == 0) {
-                    mbar_arrive(&empty[stage]);
-                    mbar_arrive_cluster(leader_b_full + 8u * (uint32_t)bs);
-                }
-                if (++stage == STAGES) { stage = 0; phase ^= 1; }
-                if (++bs == BSLOTS) { bs = 0; bphase ^= 1; }
-            }
-        }
-    } else {
-        // ---- epilogue: one warp per TMEM lane quarter of this CTA's 128 rows
-        const int e = warp - FIRST_EPI;
-        const int quad = warp & 3;
-        const float alpha = MX ? 1.0f : *p.b_gscale;
-        const bool out_bf16 = p.out_bf16 != 0;
-        const uint32_t leader_tmem_empty = mapa_shared(smem_u32(tmem_empty), 0);
-        uint8_t* buf = smem + OFF_EPI + e * EPI_BYTES;
-        uint32_t iter = 0;
-        for (int64_t t = pair_id; t < tiles; t += npairs, ++iter) {
-            const uint32_t ab = iter & 1;
-            if (!mbar_wait(&tmem_full[ab], (iter >> 1) & 1)) break;
-            tc_fence_after();
-            const int64_t mt = t % tiles_m, nt = t / tiles_m;
-            const int64_t row = mt * 2 * BM + (int64_t)rank * BM + quad * 32 + lane;
-            for (int half = 0; half < 2; ++half) {
-                const int64_t col_base = nt * BN + half * 128;
-                const uint32_t taddr = tmem + ab * 256 + ((uint32_t)(quad * 32) << 16) + half * 128;
-                if (out_bf16) {
-                    if (lane == 0) bulk_wait_read_all();
-                    __syncwarp();
-                }
-#pragma unroll
-                for (int round = 0; round < 4; ++round) {
-                    uint32_t v[32];
-                    tmem_ld32(taddr + round * 32, v);
-                    tmem_ld_wait();
-                    if (half == 1 && round == 3) {
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive_cluster(leader_tmem_empty + 8u * ab);
-                    }
-                    if (out_bf16) {
-                        uint32_t pk[16];
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(v[2 * j]) * alpha,
-                                                                     __uint_as_float(v[2 * j + 1]) * alpha);
-                            pk[j] = *reinterpret_cast<uint32_t*>(&h);
-                        }
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const int c = (round & 1) * 4 + q;
-                            *reinterpret_cast<uint4*>(buf + (round >> 1) * 4096 + lane * 128 + ((c ^ (lane & 7)) << 4)) =
-                                make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-                        }
-                    } else if (row < p.M) {
-                        store_row32(p.y, p.N, row, col_base + round * 32, v, alpha, false);
-                    }
-                }
-                if (out_bf16) {
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        const int32_t r0 = (int32_t)(mt * 2 * BM + (int64_t)rank * BM + quad * 32);
-                        tma_store_2d(&tmY, buf, (int32_t)col_base, r0);
-                        tma_store_2d(&tmY, buf + 4096, (int32_t)(col_base + 64), r0);
-                        bulk_commit_group();
-                    }
-                    __syncwarp();
-                }
-            }
-        }
-        if (lane == 0) bulk_wait_all();
-    }
-
-    tc_fence_before();
-    __syncthreads();
-    cluster_sync();          // both CTAs are done with the pair's barriers and TMEM
-    tc_fence_after();
-    if (warp == 1) tmem_dealloc2(tmem, TMEM_COLS);
-    __syncthreads();
-    cluster_sync();
-}
-
-// CTA-pair W4A16 kernel for M > 128 (off: measured slower than the 1-CTA
-// kernel on the looped-core shapes, 81.7 vs 61 us on 4096 x 4096 x 1024).
-constexpr bool kUseW16Pair = false;
-
 cudaError_t launch_w4a16(const W4A16Params& p, cudaStream_t st, int num_sms) {
     using namespace w16;
     if (p.M == 0 || p.N == 0) return cudaSuccess;
     CUtensorMap mx, mc, my;
     std::memset(&my, 0, sizeof(my));
-    const bool pair = kUseW16Pair && p.M > BM && num_sms >= 2;
     if (!encode_map_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.x, (uint64_t)p.K, (uint64_t)p.M, (uint64_t)p.K * 2,
                        64u, (uint32_t)BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !encode_map_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.b_codes, (uint64_t)(p.K / 2), (uint64_t)p.N,
-                       (uint64_t)(p.K / 2), 32u, pair ? 128u : (uint32_t)BN, CU_TENSOR_MAP_SWIZZLE_NONE))
+                       (uint64_t)(p.K / 2), 32u, (uint32_t)BN, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
     if (p.out_bf16 && !make_out_map(&my, p.y, p.M, p.N)) return cudaErrorInvalidValue;
     W16Dev d;
@@ -1522,38 +1219,6 @@ cudaError_t launch_w4a16(const W4A16Params& p, cudaStream_t st, int num_sms) {
     d.catoms = ((p.K / (p.mxfp4 ? 32 : 16)) + 3) / 4;
     d.out_bf16 = p.out_bf16 ? 1 : 0;
     d.subs = 1;
-    if (pair) {
-        // CTA pairs: each weight tile is dequantized once per 256 rows of X
-        const int64_t ptiles = ((p.M + 2 * BM - 1) / (2 * BM)) * ((p.N + BN - 1) / BN);
-        int pairs = num_sms / 2;
-        if (ptiles < pairs) pairs = (int)ptiles;
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(2 * pairs, 1, 1);
-        cfg.blockDim = dim3(w16p::THREADS, 1, 1);
-        cfg.dynamicSmemBytes = w16p::SMEM_BYTES;
-        cfg.stream = st;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = 2;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        cudaError_t e;
-        if (p.mxfp4) {
-            e = cudaFuncSetAttribute(w4a16_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     w16p::SMEM_BYTES);
-            if (e != cudaSuccess) return e;
-            e = cudaLaunchKernelEx(&cfg, w4a16_pair_kernel<true>, mx, mc, my, d);
-        } else {
-            e = cudaFuncSetAttribute(w4a16_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     w16p::SMEM_BYTES);
-            if (e != cudaSuccess) return e;
-            e = cudaLaunchKernelEx(&cfg, w4a16_pair_kernel<false>, mx, mc, my, d);
-        }
-        if (e != cudaSuccess) return e;
-        return cudaGetLastError();
-    }
     // two X row blocks per tile (each converted weight tile feeds two MMAs) when
     // the tiles still cover every SM, else one (more tiles, a deeper ring)
     const int64_t tiles_n = (p.N + BN - 1) / BN;
