@@ -39,10 +39,12 @@
  *  R2 NVFP4 block scale: sbf = amax / (6 * s_t), two binary32 operations in
  *     that order, then E4M3 with round-to-nearest-even (mode RN) or round-up
  *     (mode RU, the "rounded up" candidate of [LT] sec. 2.2), saturating at 448.
- *  R3 Elements are normalised by one reciprocal per block: S = dec(sb) * s_t,
- *     inv = 1 / S, v = x * inv.  If S is 0, or inv is not finite, or s_t is not
- *     a positive finite number, the block is degenerate and its normalised
- *     values are taken as +0.
+ *  R3 Elements are normalised as [LT] sec. 2.5 writes it, x = W / s: the
+ *     block's decoded scale S = dec(sb) * s_t (one binary32 product), then one
+ *     correctly rounded binary32 division v = x / S per element.  If S is 0,
+ *     or its reciprocal 1 / S overflows binary32, or s_t is not a positive
+ *     finite number, the block is degenerate and its normalised values are
+ *     taken as +0.
  *  R4 MXFP4 shared exponent (mode RN): e = floor(log2(amax)) - 2, the OCP rule
  *     (emax of E2M1 is 2), clamped to [-127, 127]; mode RU takes the smallest e
  *     with amax <= 6 * 2^e, so that nothing saturates (needed by Sigma-Delta).
@@ -179,9 +181,9 @@ float q4o_tensor_scale(float amax, float denom)
 /* element 2i in the low nibble.  Scales are written row-major [rows, cols/16]. */
 /* Returns 0, or -1 for an invalid shape.                                    */
 /* ------------------------------------------------------------------------ */
-static int block_is_degenerate(float S, float inv, float s_t)
+static int block_is_degenerate(float S, float s_t)
 {
-    return !(s_t > 0.0f) || !isfinite(s_t) || S == 0.0f || !isfinite(inv);
+    return !(s_t > 0.0f) || !isfinite(s_t) || S == 0.0f || !isfinite(1.0f / S);
 }
 
 int q4o_nvfp4_quantize(const float* x, int64_t rows, int64_t cols, float s_t,
@@ -205,11 +207,10 @@ int q4o_nvfp4_quantize(const float* x, int64_t rows, int64_t cols, float s_t,
                 sb = q4o_e4m3_encode(sbf, round_up);
             }
             float S = (float)q4o_e4m3_decode(sb) * s_t;  /* R3 */
-            float inv = 1.0f / S;
-            int degenerate = block_is_degenerate(S, inv, s_t);
+            int degenerate = block_is_degenerate(S, s_t);
             scales[i * nb + b] = sb;
             for (int j = 0; j < 16; ++j) {
-                float v = degenerate ? 0.0f : xb[j] * inv;
+                float v = degenerate ? 0.0f : xb[j] / S;
                 uint8_t c = q4o_e2m1_encode(v);
                 int64_t k = b * 16 + j;
                 uint8_t* dst = codes + i * (cols / 2) + k / 2;
@@ -360,8 +361,8 @@ int q4o_dequantize(int format, const uint8_t* codes, const uint8_t* scales,
 /* One loop visit of first-order Sigma-Delta requantization ([LT] sec. 2.1  */
 /* and the code of sec. 2.5): with the block scale fixed, x = W / s,         */
 /* v_k = x + r_{k-1}, q_k = Q(v_k) (nearest E2M1, saturating), r_k = v_k - q_k.*/
-/* The caller zeroes r before the first visit (r_0 = 0).  x is formed with   */
-/* the per-block reciprocal of R3.  Scales row-major; s_t ignored for MXFP4. */
+/* The caller zeroes r before the first visit (r_0 = 0).  x = w / S, one     */
+/* binary32 division (R3).  Scales row-major; s_t ignored for MXFP4.         */
 /* ------------------------------------------------------------------------ */
 int q4o_sigma_delta_step(int format, const float* w, int64_t rows, int64_t cols,
                          const uint8_t* scales, float s_t, float* r, uint8_t* codes)
@@ -372,20 +373,19 @@ int q4o_sigma_delta_step(int format, const float* w, int64_t rows, int64_t cols,
     for (int64_t i = 0; i < rows; ++i) {
         for (int64_t b = 0; b < nb; ++b) {
             uint8_t sb = scales[i * nb + b];
-            float inv;
+            float S;
             int degenerate;
             if (format == Q4O_NVFP4) {
-                float S = (float)q4o_e4m3_decode(sb) * s_t;
-                inv = 1.0f / S;
-                degenerate = block_is_degenerate(S, inv, s_t);
+                S = (float)q4o_e4m3_decode(sb) * s_t;
+                degenerate = block_is_degenerate(S, s_t);
             } else {
-                inv = ldexpf(1.0f, 127 - (int)sb);   /* 2^-e, exact */
+                S = ldexpf(1.0f, (int)sb - 127);     /* 2^e, exact */
                 degenerate = 0;
             }
             for (int j = 0; j < blk; ++j) {
                 int64_t k = b * blk + j;
                 int64_t idx = i * cols + k;
-                float x = degenerate ? 0.0f : w[idx] * inv;
+                float x = degenerate ? 0.0f : w[idx] / S;
                 float v = x + r[idx];
                 uint8_t c = q4o_e2m1_encode(v);
                 r[idx] = v - (float)q4o_e2m1_decode(c);
@@ -526,7 +526,7 @@ static uint8_t sr_e2m1(float x, float u)
 
 /* One stochastic-rounding requant of W at loop visit `visit` ([LT] sec. 2.1  */
 /* and sec. 3: the SR baseline of the looped-weight experiments, a fixed       */
-/* seed giving one weight trajectory): x = W * inv with the fixed block scale  */
+/* seed giving one weight trajectory): x = W / S with the fixed block scale    */
 /* (R3, degenerate blocks give +0), code = SR(x).  Scales row-major.           */
 int q4o_sr_requant(int format, const float* w, int64_t rows, int64_t cols, const uint8_t* scales, float s_t,
                    uint64_t seed, uint32_t visit, uint8_t* codes)
@@ -537,20 +537,19 @@ int q4o_sr_requant(int format, const float* w, int64_t rows, int64_t cols, const
     for (int64_t i = 0; i < rows; ++i) {
         for (int64_t b = 0; b < nb; ++b) {
             uint8_t sb = scales[i * nb + b];
-            float inv;
+            float S;
             int degenerate;
             if (format == Q4O_NVFP4) {
-                float S = (float)q4o_e4m3_decode(sb) * s_t;
-                inv = 1.0f / S;
-                degenerate = block_is_degenerate(S, inv, s_t);
+                S = (float)q4o_e4m3_decode(sb) * s_t;
+                degenerate = block_is_degenerate(S, s_t);
             } else {
-                inv = ldexpf(1.0f, 127 - (int)sb);
+                S = ldexpf(1.0f, (int)sb - 127);     /* 2^e, exact */
                 degenerate = 0;
             }
             for (int j = 0; j < blk; ++j) {
                 int64_t k = b * blk + j;
                 int64_t e = i * cols + k;
-                float x = degenerate ? 0.0f : w[e] * inv;
+                float x = degenerate ? 0.0f : w[e] / S;
                 uint8_t c = sr_e2m1(x, sr_uniform(seed, visit, e));
                 uint8_t* dst = codes + i * (cols / 2) + k / 2;
                 if ((k & 1) == 0) *dst = (uint8_t)((*dst & 0xF0u) | c);
@@ -580,11 +579,10 @@ static void nv46_candidate(const float* xb, float amax, float s_t, float target,
         sb = q4o_e4m3_encode(sbf, 1);
     }
     float S = (float)q4o_e4m3_decode(sb) * s_t;
-    float inv = 1.0f / S;
-    int degenerate = block_is_degenerate(S, inv, s_t);
+    int degenerate = block_is_degenerate(S, s_t);
     double err = 0.0;
     for (int j = 0; j < 16; ++j) {
-        float v = degenerate ? 0.0f : xb[j] * inv;
+        float v = degenerate ? 0.0f : xb[j] / S;     /* R3 */
         uint8_t c = q4o_e2m1_encode(v);
         codes_out[j] = c;
         double d = (double)xb[j] - q4o_e2m1_decode(c) * (double)S;

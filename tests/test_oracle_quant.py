@@ -62,9 +62,9 @@ def test_nvfp4_codes_are_nearest(orc, kind, round_up):
     x = synth.small_like(kind, 7, 48, 160)
     s_t = np.float32(np.abs(x).max()) / np.float32(6 * 448)
     codes, scales = orc.nvfp4_quantize(x, s_t, round_up=round_up)
+    # x / S ("Looped Transformer quantization" sec. 2.5: x = W / s), numpy's binary32 division
     S = (e4m3_torch(scales).astype(np.float32) * np.float32(s_t)).astype(np.float32)
-    inv = (np.float32(1.0) / S).astype(np.float32)
-    v = (x.reshape(48, 10, 16) * inv[:, :, None]).astype(np.float32).reshape(-1)
+    v = (x.reshape(48, 10, 16) / S[:, :, None]).astype(np.float32).reshape(-1)
     check_nearest(v, unpack(codes).reshape(-1))
 
 
@@ -89,8 +89,7 @@ def test_nvfp4_round_up_scale_never_saturates(orc):
     s_t = np.float32(np.abs(w).max()) / np.float32(1536)
     codes, scales = orc.nvfp4_quantize(w, s_t, round_up=True)
     S = (e4m3_torch(scales).astype(np.float32) * s_t).astype(np.float32)
-    inv = (np.float32(1.0) / S).astype(np.float32)
-    v = (w.reshape(64, 32, 16) * inv[:, :, None]).astype(np.float32)
+    v = (w.reshape(64, 32, 16) / S[:, :, None]).astype(np.float32)
     assert np.abs(v).max() <= 6.0
 
 

@@ -125,13 +125,12 @@ def test_looped_weights_bound_telescoping_first_visit(orc, fmt):
         s_t = np.float32(np.abs(w).max()) / np.float32(1536)
         rtn_codes, scales = orc.nvfp4_quantize(w, s_t, round_up=True)
         S = np.repeat((e4m3_torch(scales).astype(np.float32) * s_t).astype(np.float32), 16, axis=1)
-        inv = (np.float32(1) / S).astype(np.float32)
     else:
         f = orc.MXFP4
         s_t = np.float32(0)
         rtn_codes, scales = orc.mxfp4_quantize(w, round_up=True)
-        inv = np.repeat((2.0 ** (127 - scales.astype(np.float64))).astype(np.float32), 32, axis=1)
-    x = (w * inv).astype(np.float32).astype(np.float64)
+        S = np.repeat((2.0 ** (scales.astype(np.float64) - 127)).astype(np.float32), 32, axis=1)
+    x = (w / S).astype(np.float32).astype(np.float64)       # sec. 2.5: x = W / s
     r = np.zeros_like(w)
     cum = np.zeros_like(x)
     for k in range(1, R + 1):

@@ -85,7 +85,7 @@ def test_sr_unbiased_and_visit_dependent(orc):
 
 
 def test_sr_uses_the_sigma_delta_normalisation(orc):
-    """x = W * inv with the fixed RU block scales, as the Sigma-Delta step: a
+    """x = W / S with the fixed RU block scales, as the Sigma-Delta step: a
     weight whose normalised value is on the grid is reproduced exactly."""
     w = synth.small_like("weight", 2, 8, 64)
     s_t = orc.tensor_scale(orc.amax(w), 1536.0)
