@@ -1,8 +1,8 @@
 """Benchmark of the 4-bit block-scaled W4A4 path on B200.
 
 One step = one pass of the prefill-shaped W4A4 linear over one batch:
-    tensor amax of X (8192 x 5120 bf16, heavy-tailed)      -> s_t
-    NVFP4 quantize of X (codes + tensor-core scales)       (the quantize GB/s)
+    tensor amax of X (8192 x 5120 bf16, heavy-tailed) -> s_t,
+    then NVFP4 quantize of X (codes + tensor-core scales),  one launch
     W4A4 GEMM with W1 (5120 x 5120) and W2 (17408 x 5120)  (the GEMM TFLOP/s)
 with the weights quantized once beforehand and resident in HBM.  `value` is
 the GEMM FLOPs of the step divided by the step's device time.  The other
@@ -151,7 +151,7 @@ class Prefill:
         d = synth.prefill()
         self.x_host = d["x"]                                  # bf16 CPU
         self.x = d["x"].to(dev)
-        self.amax = torch.zeros(2, dtype=torch.float32, device=dev)
+        self.amax = torch.zeros(4, dtype=torch.float32, device=dev)
         self.xc = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
         self.xs = torch.empty(q4.q4_scale_bytes(q4.NVFP4, M, K), dtype=torch.uint8, device=dev)
         self.w = []
@@ -168,18 +168,22 @@ class Prefill:
         q4 = self.q4
         if ev is not None:
             ev[0].record()
-        q4.q4_amax(self.x, 2688.0, out=self.amax)
+        q4.q4_amax_quantize(self.x, 2688.0, out=self.amax, codes=self.xc, scales=self.xs)
         if ev is not None:
             ev[1].record()
-        q4.q4_quantize(q4.NVFP4, self.x, gscale=self.amax[1:2], codes=self.xc, scales=self.xs)
-        if ev is not None:
-            ev[2].record()
         for i, (n, wc, ws, wg) in enumerate(self.w):
             q4.q4_gemm(q4.NVFP4, M, n, K, self.xc, self.xs, self.amax[1:2], wc, ws, wg, y=self.y[i])
             if ev is not None:
-                ev[3 + i].record()
+                ev[2 + i].record()
 
-    LAUNCHES_PER_STEP = 4   # amax (finishes with the tensor scale), quantize, two GEMMs
+    def two_launch_quantize(self):
+        """The same activation quantize as q4_amax then q4_quantize (for comparison)."""
+        q4 = self.q4
+        q4.q4_amax(self.x, 2688.0, out=self.amax)
+        q4.q4_quantize(q4.NVFP4, self.x, gscale=self.amax[1:2], codes=self.xc, scales=self.xs)
+
+    LAUNCHES_PER_STEP = 3   # amax + quantize (one cooperative launch), two GEMMs
+    SEGMENTS = 3
 
 
 def time_fn(fn, reps, flush, warm=3):
@@ -198,11 +202,112 @@ def time_fn(fn, reps, flush, warm=3):
     return statistics.mean(ts), min(ts)
 
 
+def sigma_delta_quality(q4, mats, visits=32):
+    """Weight representation error of R Sigma-Delta visits against static RTN
+    ("Looped Transformer quantization", sec. 2.1-2.2): per weight, the mean of
+    the R decoded codes against w, and the RTN code (the first visit from
+    r_0 = 0) against w, both from the GPU codes.  Also the largest mean error in
+    normalised units (|mean_k dec(q_k) / S - w / S|), which the page bounds by
+    d / (2R) = 1 / R on E2M1 (largest gap d = 2)."""
+    err_sd = err_rtn = 0.0
+    worst = 0.0
+    n = 0
+    for wt, sc, g, r, c, _ in mats:
+        rows, cols = wt.shape
+        r.zero_()
+        acc = torch.zeros_like(wt, dtype=torch.float64)
+        rtn = None
+        for k in range(visits):
+            q4.q4_sigma_delta_step(q4.NVFP4, wt, sc, r, gscale=g, codes=c)
+            dq = q4.q4_dequantize(q4.NVFP4, c, sc, rows, cols, gscale=g)
+            acc += dq
+            if k == 0:
+                rtn = dq.double()
+        one = torch.full_like(c, 0x22)                       # code 1.0 in both nibbles: dequantizes to S
+        S = q4.q4_dequantize(q4.NVFP4, one, sc, rows, cols, gscale=g).double()
+        w64 = wt.double()
+        mean = acc / visits
+        err_sd += float((mean - w64).abs().sum())
+        err_rtn += float((rtn - w64).abs().sum())
+        worst = max(worst, float(((mean - w64).abs() / S).max()))
+        n += wt.numel()
+        r.zero_()
+    return {"visits": visits, "weights": n, "mean_abs_err_sigma_delta": err_sd / n, "mean_abs_err_rtn": err_rtn / n,
+            "ratio_sigma_delta_over_rtn": err_sd / err_rtn, "max_normalised_mean_err": worst,
+            "bound_d_over_2R": 2.0 / (2 * visits)}
+
+
+def tiny_rows(q4, dev, reps=200):
+    """The tiny NVFP4 W4A4 linear (X 64 x 512, W 512 x 512 fp32, 1 % x50
+    outliers): amax and quantize of both operands + GEMM with bf16 out, and a
+    Sigma-Delta chain of W over R = 8 visits.  Latency-bound: microseconds per
+    call with warm L2, eager and as one CUDA graph replay."""
+    d = synth.tiny()
+    x = torch.from_numpy(d["x"]).to(dev)
+    w = torch.from_numpy(d["w"]).to(dev)
+    ax = torch.zeros(2, dtype=torch.float32, device=dev)
+    aw = torch.zeros(2, dtype=torch.float32, device=dev)
+    xc = torch.empty((64, 256), dtype=torch.uint8, device=dev)
+    xs = torch.empty(q4.q4_scale_bytes(q4.NVFP4, 64, 512), dtype=torch.uint8, device=dev)
+    wc = torch.empty((512, 256), dtype=torch.uint8, device=dev)
+    ws = torch.empty(q4.q4_scale_bytes(q4.NVFP4, 512, 512), dtype=torch.uint8, device=dev)
+    y = torch.empty((64, 512), dtype=torch.bfloat16, device=dev)
+    gw = q4.q4_amax(w, 1536.0)[1:2].clone()
+    _, sw = q4.q4_quantize(q4.NVFP4, w, gscale=gw, flags=q4.SCALE_RU | q4.LAYOUT_TC)
+    r = torch.zeros_like(w)
+    cw = torch.empty((512, 256), dtype=torch.uint8, device=dev)
+
+    def linear():
+        q4.q4_amax(x, 2688.0, out=ax)
+        q4.q4_quantize(q4.NVFP4, x, gscale=ax[1:2], codes=xc, scales=xs)
+        q4.q4_amax(w, 2688.0, out=aw)
+        q4.q4_quantize(q4.NVFP4, w, gscale=aw[1:2], codes=wc, scales=ws)
+        q4.q4_gemm(q4.NVFP4, 64, 512, 512, xc, xs, ax[1:2], wc, ws, aw[1:2], y=y)
+
+    def chain8():
+        r.zero_()
+        for _ in range(8):
+            q4.q4_sigma_delta_step(q4.NVFP4, w, sw, r, gscale=gw, codes=cw)
+
+    def per_call(fn):
+        for _ in range(10):
+            fn()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        s.record()
+        for _ in range(reps):
+            fn()
+        e.record()
+        e.synchronize()
+        return s.elapsed_time(e) * 1e3 / reps
+
+    out = {"linear_us": per_call(linear), "sigma_delta_R8_us": per_call(chain8),
+           "launches": {"linear": 5, "sigma_delta_R8": 9}, "l2": "warm (latency row)"}
+    for name, fn in (("linear", linear), ("sigma_delta_R8", chain8)):
+        try:
+            g = torch.cuda.CUDAGraph()
+            st = torch.cuda.Stream()
+            st.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(st):
+                fn()
+            torch.cuda.current_stream().wait_stream(st)
+            with torch.cuda.graph(g, capture_error_mode="relaxed"):
+                fn()
+            out[name + "_graph_us"] = per_call(g.replay)
+            del g
+        except Exception as ex:                  # report, do not hide, a capture that fails
+            out[name + "_graph_us"] = None
+            out[name + "_graph_error"] = str(ex)[:200]
+    out["gemm_TFLOP/s"] = 2.0 * 64 * 512 * 512 / (out["linear_us"] * 1e-6) / 1e12
+    return out
+
+
 def rows_bench(q4, dev, flush, pk, reps=30):
     """Per-row measurements on their own workloads (see module docstring)."""
     out = {}
     hbm = pk["hbm_gbs"]
     fp4 = pk["bf16"] * FP4_OVER_BF16
+    out["tiny_linear"] = tiny_rows(q4, dev)
 
     # a3 + a5 (MXFP4): quantize X with t and Hadamard-32, GEMM with pre-quantized W'
     d = synth.mxfp4()
@@ -317,6 +422,7 @@ def rows_bench(q4, dev, flush, pk, reps=30):
     ms_v, _ = time_fn(visit, max(5, reps // 3), flush)
     out["looped_visit"] = {"us": ms_v * 1e3, "us_R32": ms_v * 1e3 * 32,
                            "note": "Sigma-Delta requant of all 13 weights + 13 W4A16 GEMMs"}
+    out["sigma_delta_vs_rtn"] = sigma_delta_quality(q4, mats, visits=32)
     del mats, xl
 
     # a6: decode-shaped GEMM with fused activation quantize
@@ -395,11 +501,17 @@ def run_ours(args):
         flush_rd.sum()
 
     P = Prefill(q4, dev)
+    # the achieved heavy-tail statistic of the synthetic X: median over rows of max|x| / rms(x)
+    xf = P.x.float()
+    ratio = xf.abs().amax(dim=1) / xf.pow(2).mean(dim=1).sqrt()
+    x_stat = {"row_max_over_rms_median": float(ratio.median()),
+              "one_hot_block_fraction_recipe": 0.2}
+    del xf, ratio
     for _ in range(max(args.warmup, 3)):
         P.step()
     torch.cuda.synchronize()
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(Prefill.SEGMENTS + 1)] for _ in range(args.steps)]
     clock_path = Path(args.clocks_csv) if args.clocks_csv else None
     if dist is not None:
         dist.barrier()
@@ -413,14 +525,16 @@ def run_ours(args):
     if dist is not None:
         dist.barrier()
     wall = time.perf_counter() - wall0
-    seg = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)] for i in range(args.steps)])
+    seg = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(Prefill.SEGMENTS)]
+                    for i in range(args.steps)])
     step_ms = max_over_ranks(float(seg.sum(axis=1).mean()), dist, dev)
     clocks = cs.summary()
-    k_ms = seg.mean(axis=0)          # amax, quantize, gemm1, gemm2
-    gemm2_tf = 2.0 * M * N2 * K / (k_ms[3] * 1e-3) / 1e12
-    gemm1_tf = 2.0 * M * N1 * K / (k_ms[2] * 1e-3) / 1e12
-    q_gbs = M * K * B_QUANT_BF16 / (k_ms[1] * 1e-3) / 1e9
-    a_gbs = M * K * B_AMAX_BF16 / (k_ms[0] * 1e-3) / 1e9
+    k_ms = seg.mean(axis=0)          # amax + quantize, gemm1, gemm2
+    gemm2_tf = 2.0 * M * N2 * K / (k_ms[2] * 1e-3) / 1e12
+    gemm1_tf = 2.0 * M * N1 * K / (k_ms[1] * 1e-3) / 1e12
+    # the fused launch reads X from HBM once (the second pass mostly hits L2):
+    # its algorithmic bytes are those of the quantize alone
+    q_gbs = M * K * B_QUANT_BF16 / (k_ms[0] * 1e-3) / 1e9
     value = whole_job_tflops(world, GEMM_FLOPS, step_ms)
 
     # end to end through the C ABI with host buffers: pinned X in, both Y out
@@ -449,21 +563,31 @@ def run_ours(args):
 
     rows = None
     if not args.no_rows:
-        # the prefill activation quantize alone after a cold, clean L2
+        # the prefill activation quantize alone after a cold, clean L2, and the
+        # same work as two launches (amax, then quantize)
         xq_ms, _ = time_fn(lambda: q4.q4_quantize(q4.NVFP4, P.x, gscale=P.amax[1:2], codes=P.xc, scales=P.xs), 30,
                            flush)
         xq_gbs = M * K * B_QUANT_BF16 / (xq_ms * 1e-3) / 1e9
         iso_quant = {"shape": [M, K], "us": xq_ms * 1e3, "GB/s": xq_gbs, "frac_hbm": xq_gbs / hbm}
+        am_ms, _ = time_fn(lambda: q4.q4_amax(P.x, 2688.0, out=P.amax), 30, flush)
+        two_ms, _ = time_fn(P.two_launch_quantize, 30, flush)
+        fused_ms, _ = time_fn(lambda: q4.q4_amax_quantize(P.x, 2688.0, out=P.amax, codes=P.xc, scales=P.xs), 30,
+                              flush)
+        a_gbs = M * K * B_AMAX_BF16 / (am_ms * 1e-3) / 1e9
         del P
         torch.cuda.empty_cache()
         rows = rows_bench(q4, dev, flush, pk, reps=args.rows_reps)
-        rows["nvfp4_quantize_prefill_x"] = {"shape": [M, K], "us": k_ms[1] * 1e3, "GB/s": q_gbs,
-                                            "frac_hbm": q_gbs / hbm,
-                                            "note": "inside the step, right after amax (X partly in L2)"}
+        rows["amax_quantize_prefill_x"] = {"shape": [M, K], "us": k_ms[0] * 1e3, "GB/s": q_gbs,
+                                           "frac_hbm": q_gbs / hbm, "B_per_element": B_QUANT_BF16,
+                                           "note": "in the step: one cooperative launch, amax then quantize"}
+        fused_gbs = M * K * B_QUANT_BF16 / (fused_ms * 1e-3) / 1e9
+        rows["amax_quantize_prefill_x_cold"] = {"us": fused_ms * 1e3, "GB/s": fused_gbs, "frac_hbm": fused_gbs / hbm,
+                                                "two_launches_us": two_ms * 1e3,
+                                                "speedup_vs_two_launches": two_ms / fused_ms}
         rows["nvfp4_quantize_prefill_x_cold"] = iso_quant
-        rows["amax_prefill_x"] = {"us": k_ms[0] * 1e3, "GB/s": a_gbs, "frac_hbm": a_gbs / hbm}
-        rows["gemm_prefill_n5120"] = {"us": k_ms[2] * 1e3, "TFLOP/s": gemm1_tf, "frac_fp4": gemm1_tf / fp4_burst}
-        rows["gemm_prefill_n17408"] = {"us": k_ms[3] * 1e3, "TFLOP/s": gemm2_tf, "frac_fp4": gemm2_tf / fp4_burst}
+        rows["amax_prefill_x_cold"] = {"us": am_ms * 1e3, "GB/s": a_gbs, "frac_hbm": a_gbs / hbm}
+        rows["gemm_prefill_n5120"] = {"us": k_ms[1] * 1e3, "TFLOP/s": gemm1_tf, "frac_fp4": gemm1_tf / fp4_burst}
+        rows["gemm_prefill_n17408"] = {"us": k_ms[2] * 1e3, "TFLOP/s": gemm2_tf, "frac_fp4": gemm2_tf / fp4_burst}
 
     cpu = None if args.no_cpu_baseline or rank != 0 else cpu_baseline(budget_s=args.cpu_seconds)
 
@@ -471,7 +595,7 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": max(args.warmup, 3), "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "e2m1 x e2m1 -> f32 (NVFP4 block-scaled)", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "M": M, "K": K, "N": [N1, N2], "quantize_GB/s": q_gbs,
+        "config": {"workload": WORKLOAD, "M": M, "K": K, "N": [N1, N2], "x_stat": x_stat, "quantize_GB/s": q_gbs,
                    "quantize_frac_hbm": q_gbs / hbm, "l2": "flushed before every timed step: 256 MiB write, then a 256 MiB read (cold, clean L2)",
                    "parallelism": f"replicas x{world} (independent problems per GPU)"},
         "roofline": {"kernel": "gemm_kernel<NVFP4> 8192x17408x5120", "bound": "tensor", "achieved": gemm2_tf,
@@ -529,21 +653,92 @@ class OracleSample:
         return 2.0 * self.rows * self.cols * K, time.perf_counter() - t0
 
 
-def cpu_baseline(budget_s: float = 15.0):
-    """The CPU oracle as it stands, single-threaded, on a bounded sample of the
-    prefill workload (see OracleSample); GEMM FLOPs per second as TFLOP/s."""
+def _row_ranges(n: int, parts: int):
+    step = max(1, (n + parts - 1) // parts)
+    return [(i, min(n, i + step)) for i in range(0, n, step)]
+
+
+def _on_threads(fn, items, threads: int):
+    """fn over items on `threads` host threads.  The oracle's arithmetic runs
+    in C behind ctypes, which releases the GIL, so the calls run in parallel."""
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        return list(ex.map(fn, items))
+
+
+def cpu_baseline(budget_s: float = 10.0):
+    """The CPU oracle as it stands, on the machine's host cores: single-threaded and
+    row-parallel over every core the process may use (the same oracle calls on
+    row ranges, one host thread each).
+
+    * NVFP4 quantize of the full prefill X (8192 x 5120, amax included);
+    * one Sigma-Delta visit over all 13 looped-core weights (41,943,040);
+    * the binary64 GEMM on a sample: 64 rows of X against 256-row chunks of
+      W1 / W2 (K = 5120), for about budget_s / 2 seconds each way.
+    `value` is the all-core GEMM throughput in the line's unit."""
+    import oracle
+    threads = len(os.sched_getaffinity(0))
     smp = OracleSample()
-    xc, xs, tq = smp.quantize()
-    flops, tg, j = 0.0, 0.0, 0
-    while tg < budget_s:
+    x32 = synth.bf16_to_f32(synth.prefill(n_list=())["x"])
+
+    def quant(rng):
+        i0, i1 = rng
+        oracle.amax(x32[i0:i1])
+        oracle.nvfp4_quantize(x32[i0:i1], smp.s_t)
+    t0 = time.perf_counter()
+    quant((0, M))
+    q1 = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    _on_threads(quant, _row_ranges(M, 4 * threads), threads)
+    qn = time.perf_counter() - t0
+    qbytes = M * K * (B_QUANT_BF16 + B_AMAX_BF16)
+    del x32
+
+    dl = synth.looped(m=16)
+    mats = []
+
+    def prep(w):
+        s_t = oracle.tensor_scale(oracle.amax(w), 1536.0)
+        _, sc = oracle.nvfp4_quantize(w, s_t, round_up=True)
+        return w, sc, s_t, np.zeros_like(w)
+    mats = _on_threads(prep, dl["w"], threads)
+    nw = sum(w.size for w, *_ in mats)
+
+    def sd(item):
+        w, sc, s_t, r, (i0, i1) = item
+        oracle.sigma_delta_step(oracle.NVFP4, w[i0:i1], sc[i0:i1], s_t, r[i0:i1])
+    t0 = time.perf_counter()
+    for w, sc, s_t, r in mats:
+        sd((w, sc, s_t, r, (0, w.shape[0])))
+    s1 = time.perf_counter() - t0
+    items = [(w, sc, s_t, r, rr) for w, sc, s_t, r in mats for rr in _row_ranges(w.shape[0], threads)]
+    t0 = time.perf_counter()
+    _on_threads(sd, items, threads)
+    sn = time.perf_counter() - t0
+    del mats, dl
+
+    xc, xs, _ = smp.quantize()
+    f1, g1, j = 0.0, 0.0, 0
+    while g1 < budget_s / 2:
         f, t = smp.gemm_chunk(xc, xs, j % 2, j // 2)
-        flops += f
-        tg += t
-        j += 1
-    return {"value": flops / tg / 1e12, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"{smp.rows} rows of X (amax + NVFP4 quantize), then binary64 GEMMs of those rows "
-                      f"against {j} chunks of {smp.cols} weight rows (K = {K}), alternating W1/W2",
-            "quantize_GB/s": smp.rows * K * B_QUANT_BF16 / tq / 1e9, "gemm_seconds": tg}
+        f1, g1, j = f1 + f, g1 + t, j + 1
+    n_chunks = max(threads, 2 * threads)
+    t0 = time.perf_counter()
+    fn = 0.0
+    while time.perf_counter() - t0 < budget_s / 2:
+        res = _on_threads(lambda jj: smp.gemm_chunk(xc, xs, jj % 2, jj // 2)[0], range(n_chunks), threads)
+        fn += sum(res)
+    gn = time.perf_counter() - t0
+    return {"value": fn / gn / 1e12, "unit": UNIT, "cores": threads, "host_cpu_count": os.cpu_count(),
+            "kind": "oracle",
+            "sample": (f"GEMM: binary64 oracle on {smp.rows} rows of X against {smp.cols}-row chunks of W1/W2 "
+                       f"(K = {K}), ~{budget_s / 2:.0f} s single-threaded and ~{budget_s / 2:.0f} s on all "
+                       f"{threads} threads; quantize: the full 8192 x 5120 X (amax + NVFP4); Sigma-Delta: one "
+                       f"visit over the full looped core ({nw} weights)"),
+            "gemm_TFLOP/s_1thread": f1 / g1 / 1e12,
+            "quantize_GB/s_1thread": qbytes / q1 / 1e9, "quantize_GB/s_all": qbytes / qn / 1e9,
+            "sigma_delta_GB/s_1thread": nw * B_SIGMA_DELTA / s1 / 1e9,
+            "sigma_delta_GB/s_all": nw * B_SIGMA_DELTA / sn / 1e9}
 
 
 def run_reference(args):
@@ -598,7 +793,7 @@ def main():
                     help="also write the clock samples taken during the timed steps to this CSV file")
     ap.add_argument("--rows-reps", type=int, default=30,
                     help="timed calls per kernel row (small values for profiler captures)")
-    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--traffic", type=float, default=GEMM_TRAFFIC_BYTES,
                     help="DRAM bytes per launch of the roofline kernel from an ncu capture")
     args = ap.parse_args()

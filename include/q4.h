@@ -77,7 +77,12 @@ enum {
                             MXFP4: smallest exponent with block max <= 6*2^e) */
     Q4_LAYOUT_TC = 2,    /* scales in the tensor-core layout (else row-major) */
     Q4_HADAMARD32 = 4,   /* MXFP4 only: block Hadamard-32 before quantizing   */
-    Q4_SCALE_46 = 8      /* NVFP4 only: 4/6 block scaling (see q4_quantize)    */
+    Q4_SCALE_46 = 8,     /* NVFP4 only: 4/6 block scaling (see q4_quantize)    */
+    Q4_INJECT_STALL = 1 << 16  /* q4_quantize only, for failure-detection tests:
+                            every CTA's first input tile is never loaded, so a
+                            bounded wait inside the kernel runs out; the codes
+                            are then not valid and q4_get_device_error
+                            reports Q4_ERR_TIMEOUT (see q4_set_wait_limit)    */
 };
 
 /* Kinds of GEMM left operand. */
@@ -115,13 +120,35 @@ Q4_API q4_status q4_amax(q4_dtype dt, const void* x, int64_t n, float denom, flo
                   void* stream);
 
 /*
+ * q4_amax_quantize -- q4_amax followed by the NVFP4 q4_quantize, in one launch.
+ *   d_out[0] = amax = max|x| over the rows x cols matrix, d_out[1] = s_t =
+ *   amax / denom (one binary32 division), and codes/scales exactly as
+ *   q4_quantize(Q4_NVFP4, 16, ...) with that s_t ("Why Gated DeltaNet Survives
+ *   4-Bit Quantization", prerequisites: block scales under an FP32 per-tensor
+ *   scale taken from the tensor's maximum).  The launch is cooperative: every
+ *   CTA folds its share of |x| into out[0], waits (bounded) at a grid-wide
+ *   barrier counted in d_out[2], then quantizes; X is read a second time
+ *   while still largely in L2, so HBM sees it about once.
+ *   d_out: device, 4 floats (the last two are the launch's own scratch and
+ *   are cleared by it); 4-byte aligned.  flags: Q4_LAYOUT_TC, Q4_SCALE_RU.
+ *   Other arguments and requirements as q4_quantize.  rows or cols = 0 gives
+ *   d_out = {0, 0, 0, 0}.  A barrier wait that runs out is reported by
+ *   q4_get_device_error as Q4_ERR_TIMEOUT (codes then not valid).
+ */
+Q4_API q4_status q4_amax_quantize(q4_dtype in_dt, const void* x, int64_t rows, int64_t cols, int64_t ld,
+                                  float denom, float* d_out, uint8_t* codes, uint8_t* scales, int flags,
+                                  void* stream);
+
+/*
  * q4_quantize -- block quantization of a rows x cols matrix.
  *   NVFP4 ("Looped Transformer quantization", sec. 0.2; "Why Gated DeltaNet
  *   Survives 4-Bit Quantization", prerequisites): per 16-block,
  *     amax = max|x|,  s_b = E4M3(amax / (6 * s_t))   [RN, or RU with Q4_SCALE_RU],
- *     S = s_b * s_t,  inv = 1 / S,  code_i = E2M1(x_i * inv)  (nearest, ties to
+ *     S = s_b * s_t,  code_i = E2M1(x_i / S)  (one correctly rounded binary32
+ *     division, as "Looped Transformer quantization", sec. 2.5 writes x = W / s;
+ *     E2M1 rounding to nearest, ties to
  *     even mantissa, saturating at +-6, sign kept for values that round to 0);
- *     a block whose S is 0 or whose inv is not finite, and every block when s_t
+ *     a block whose S is 0 or whose reciprocal 1 / S overflows, and every block when s_t
  *     is not a positive finite number, gets code 0.
  *   MXFP4 ("MACaQ", prerequisites "MXFP4 microscaling format" and core method
  *   steps (i)-(ii), y = [(x . t) B]_MXFP4): per 32-block,
@@ -168,7 +195,8 @@ Q4_API q4_status q4_dequantize(q4_format format, int block, const uint8_t* codes
  * q4_sigma_delta_step -- one loop visit of first-order Sigma-Delta
  *   requantization ("Looped Transformer quantization", sec. 2.1, and the code
  *   of sec. 2.5): with the block scales fixed,
- *     x = w * inv (inv = 1/(s_b*s_t) per NVFP4 block, 2^-e per MXFP4 block),
+ *     x = w / S (one correctly rounded binary32 division; S = s_b*s_t per
+ *     NVFP4 block, 2^e per MXFP4 block),
  *     v = x + r,  q = E2M1(v),  r <- v - q,  codes <- q.
  *   Start a chain by zeroing r (r_0 = 0).  Scales normally come from
  *   q4_quantize with Q4_SCALE_RU and s_t = max|W| / (6*256), which keeps
@@ -188,7 +216,7 @@ Q4_API q4_status q4_sigma_delta_step(q4_format format, int block, const float* w
  *   ("Looped Transformer quantization", sec. 2.1: the stochastic-rounding
  *   baseline draws every code so that its conditional expectation equals the
  *   weight; sec. 3: a fixed seed gives one weight trajectory shared by all
- *   inputs).  With the block scales fixed, x = w * inv (as in
+ *   inputs).  With the block scales fixed, x = w / S (as in
  *   q4_sigma_delta_step); for neighbouring E2M1 magnitudes a <= |x| < b the
  *   code's magnitude is b when u < (|x| - a) / (b - a), else a; |x| >= 6 gives
  *   6; the sign bit is x's.  u = (word >> 8) * 2^-24, where for element
@@ -262,7 +290,7 @@ Q4_API q4_status q4_gemm(q4_format format, int block, int64_t M, int64_t N, int6
  *   fused into the GEMM's weight producer ("Looped Transformer quantization",
  *   sec. 4: online code generation from the reference weight and the residue
  *   state at every visit): with the NVFP4 block scales fixed,
- *     q = E2M1(w * inv + r),  r <- (w * inv + r) - q   (as q4_sigma_delta_step)
+ *     q = E2M1(w / S + r),  r <- (w / S + r) - q   (as q4_sigma_delta_step)
  *     Y = s_t * X (q * s_b)^T                          (as the W4A16 q4_gemm)
  *   without writing the codes: each weight element and its residue are read
  *   once and the residue is written back.  Decode shapes: M <= 16 (else
@@ -365,16 +393,36 @@ Q4_API size_t q4_gemm_workspace_size(q4_format format, int64_t M, int64_t N, int
  *   caller.  Each call overwrites every part of the array it reads, so nothing
  *   has to be cleared between calls.  The first call on a device looks up the
  *   array's device address (once per device, with that device current); make
- *   that first call before any stream capture.  A CUDA failure returns
- *   Q4_ERR_CUDA without updating q4_last_error().
- *   Arguments as q4_gemm: a_bf16 bf16 [M, K]; b_codes/b_scales/d_b_gscale the
- *   NVFP4 weight; y [M, N] of out_dt; K % 64 == 0, N % 8 == 0.
+ *   that first call before any stream capture.  The address stays cached for
+ *   the life of the process, so a cudaDeviceReset after the first call on a
+ *   device is not supported.
+ *   Arguments and results as q4_gemm with a_kind = Q4_A_BF16: a_bf16 bf16
+ *   [M, K]; b_codes/b_scales/d_b_gscale the NVFP4 weight (tensor-core scale
+ *   layout); y [M, N] of out_dt; K % 64 == 0, N % 8 == 0, K <= 2^30,
+ *   M, N <= 2^31 (else Q4_ERR_SHAPE); K == 0 zero-fills y.  It always takes the
+ *   quantize-then-GEMM route, also for M <= 16, where q4_gemm runs the fused
+ *   decode kernel instead (same codes and products, another summation order).
+ *   A CUDA failure returns Q4_ERR_CUDA with its text in q4_last_error().
  */
 #define Q4_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
 Q4_API q4_status q4_gemm_a_bf16_noalloc(int64_t M, int64_t N, int64_t K, const void* a_bf16,
                                         const float* d_a_gscale, const uint8_t* b_codes,
                                         const uint8_t* b_scales, const float* d_b_gscale,
                                         q4_dtype out_dt, void* y, void* stream);
+
+/*
+ * q4_set_wait_limit -- how long a bounded wait inside a kernel may spin before
+ *   it gives up: `cycles` SM clock cycles, 1000 <= cycles <= 2^40, or 0 for
+ *   the default Q4_DEFAULT_WAIT_CYCLES (about 1 s at B200 clocks).  A wait
+ *   that runs out records Q4_ERR_TIMEOUT for q4_get_device_error and the
+ *   kernel winds down (stops issuing, waits with the same limit for its own
+ *   copies in flight, frees what it allocated, exits).  Applies to launches
+ *   made after the call returns; the setting is per process and device and is
+ *   written with a synchronous copy, so do not call it during stream capture.
+ *   No counterpart on the source pages: failure detection of this library.
+ */
+#define Q4_DEFAULT_WAIT_CYCLES 2000000000ll
+Q4_API q4_status q4_set_wait_limit(int64_t cycles);
 
 /*
  * q4_get_device_error -- synchronises `stream`, then reads and clears the

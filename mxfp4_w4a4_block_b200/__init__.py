@@ -30,6 +30,7 @@ SCALE_RU = 1
 LAYOUT_TC = 2
 HADAMARD32 = 4
 SCALE_46 = 8
+INJECT_STALL = 1 << 16
 
 A_QUANTIZED = 0
 A_BF16 = 1
@@ -64,6 +65,8 @@ SIGNATURES = {
     "q4_gemm_workspace_size": (_SZ, [_I, _I64, _I64, _I64, _I]),
     "q4_get_device_error": (_I, [_P]),
     "q4_gemm_a_bf16_noalloc": (_I, [_I64, _I64, _I64, _P, _P, _P, _P, _P, _I, _P, _P]),
+    "q4_set_wait_limit": (_I, [_I64]),
+    "q4_amax_quantize": (_I, [_I, _P, _I64, _I64, _I64, ctypes.c_float, _P, _P, _P, _I, _P]),
     "q4_quantize_grouped": (_I, [_I, _I, _I, _P, _I, _I, _P]),
     "q4_sigma_delta_step_grouped": (_I, [_I, _I, _P, _I, _I, _P]),
     "q4_sr_requant_grouped": (_I, [_I, _I, _P, _I, ctypes.c_uint64, ctypes.c_uint32, _I, _P]),
@@ -159,6 +162,24 @@ def q4_amax(x: torch.Tensor, denom: float, out: torch.Tensor | None = None, stre
     _check("q4_amax", lib().q4_amax(_dtype_code(x), _ptr(x), x.numel(), float(denom), _ptr(out),
                                     _stream(stream)))
     return out
+
+
+def q4_amax_quantize(x: torch.Tensor, denom: float = 2688.0, out: torch.Tensor | None = None,
+                     flags: int = LAYOUT_TC, codes: torch.Tensor | None = None,
+                     scales: torch.Tensor | None = None, stream=None):
+    """Tensor amax, s_t = amax / denom and NVFP4 quantize in one launch;
+    returns (codes, scales, out) with out = [amax, s_t, scratch, scratch]."""
+    rows, cols = x.shape
+    ld = x.stride(0) if x.stride(1) == 1 else cols
+    if out is None:
+        out = torch.empty(4, dtype=torch.float32, device=x.device)
+    if codes is None:
+        codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(max(q4_scale_bytes(NVFP4, rows, cols, flags), 1), dtype=torch.uint8, device=x.device)
+    _check("q4_amax_quantize", lib().q4_amax_quantize(_dtype_code(x), _ptr(x), rows, cols, ld, float(denom), _ptr(out),
+                                                     _ptr(codes), _ptr(scales), flags, _stream(stream)))
+    return codes, scales, out
 
 
 def q4_quantize(fmt: int, x: torch.Tensor, gscale: torch.Tensor | None = None,
@@ -364,13 +385,21 @@ def q4_gemm_a_bf16_noalloc(M: int, N: int, K: int, a: torch.Tensor, a_gscale, b_
                            b_scales: torch.Tensor, b_gscale, out_dtype=torch.bfloat16,
                            y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """q4_gemm with bf16 activations using the library's fixed scratch array
-    instead of a workspace (for callers that cannot allocate at call time)."""
+    instead of a workspace (for callers that cannot allocate at call time).
+    The call runs with the operands' device current, since the library picks
+    the scratch array of the current device."""
     if y is None:
         y = torch.empty((M, N), dtype=out_dtype, device=b_codes.device)
-    st = lib().q4_gemm_a_bf16_noalloc(M, N, K, _ptr(a), _ptr(a_gscale), _ptr(b_codes), _ptr(b_scales),
-                                      _ptr(b_gscale), _dtype_code(y), _ptr(y), _stream(stream))
+    with torch.cuda.device(b_codes.device):
+        st = lib().q4_gemm_a_bf16_noalloc(M, N, K, _ptr(a), _ptr(a_gscale), _ptr(b_codes), _ptr(b_scales),
+                                          _ptr(b_gscale), _dtype_code(y), _ptr(y), _stream(stream))
     _check("q4_gemm_a_bf16_noalloc", st)
     return y
+
+
+def q4_set_wait_limit(cycles: int = 0) -> None:
+    """Bounded-wait limit of the kernels in SM clock cycles (0: the default)."""
+    _check("q4_set_wait_limit", lib().q4_set_wait_limit(int(cycles)))
 
 
 def q4_get_device_error(stream=None) -> int:

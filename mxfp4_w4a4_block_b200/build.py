@@ -53,15 +53,19 @@ def build(force: bool = False, verbose: bool = False, extra=None) -> Path:
         return LIB
     objdir = PKG / "_build"
     objdir.mkdir(exist_ok=True)
-    objs = []
+    objs, procs = [], []
+    # the sources compile independently: one nvcc process each, in parallel
     for src in SOURCES:
         obj = objdir / (Path(src).stem + ".o")
         cmd = [nvcc(), *NVCC_FLAGS, *(extra or []), "-I", str(INCLUDE), "-c",
                str(CSRC / src), "-o", str(obj)]
         if verbose:
             print(" ".join(cmd), file=sys.stderr)
-        subprocess.run(cmd, check=True)
+        procs.append((cmd, subprocess.Popen(cmd)))
         objs.append(str(obj))
+    for cmd, proc in procs:
+        if proc.wait() != 0:
+            raise subprocess.CalledProcessError(proc.returncode, cmd)
     tmp = LIB.with_suffix(f".{os.getpid()}.tmp")
     cmd = [nvcc(), "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-cudart", "static",
            "-Xcompiler", "-fPIC", *objs, "-o", str(tmp)]

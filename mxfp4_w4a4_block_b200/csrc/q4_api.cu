@@ -67,6 +67,10 @@ q4_status group_from(q4_format format, int block, const q4_matrix* mats, int cou
 
 }  // namespace
 
+namespace q4 {
+int status_of_cuda(cudaError_t e) { return (int)cuda_status(e); }
+}  // namespace q4
+
 extern "C" {
 
 int q4_version(void) { return 100; }
@@ -103,12 +107,34 @@ q4_status q4_amax(q4_dtype dt, const void* x, int64_t n, float denom, float* d_o
     return cuda_status(q4::launch_amax(x, n, dt == Q4_BF16, denom, d_out, (cudaStream_t)stream, num_sms()));
 }
 
+q4_status q4_amax_quantize(q4_dtype in_dt, const void* x, int64_t rows, int64_t cols, int64_t ld, float denom,
+                           float* d_out, uint8_t* codes, uint8_t* scales, int flags, void* stream) {
+    if (!valid_dtype(in_dt) || rows < 0 || cols < 0 || ld < cols || !d_out) return Q4_ERR_ARG;
+    if (!(denom > 0.0f) || !(denom < 3.0e38f)) return Q4_ERR_ARG;
+    if (flags & ~(Q4_SCALE_RU | Q4_LAYOUT_TC)) return Q4_ERR_ARG;
+    if (reinterpret_cast<uintptr_t>(d_out) & 3u) return Q4_ERR_ALIGN;
+    if (cols % 16) return Q4_ERR_SHAPE;
+    const int esz = in_dt == Q4_BF16 ? 2 : 4;
+    if (rows > 0 && cols > 0) {
+        if (!x || !codes || !scales) return Q4_ERR_ARG;
+        if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || (ld * esz) % 16) return Q4_ERR_ALIGN;
+    }
+    q4::QuantParams p;
+    p.x = x; p.rows = rows; p.cols = cols; p.ld = ld;
+    p.gscale = nullptr; p.chan = nullptr; p.codes = codes; p.scales = scales;
+    p.scols = cols / 16; p.catoms = catoms_of(cols, 16);
+    p.amax_out = reinterpret_cast<unsigned int*>(d_out);
+    p.denom = denom;
+    return cuda_status(q4::launch_amax_quantize(p, in_dt == Q4_BF16, (flags & Q4_LAYOUT_TC) != 0,
+                                                (flags & Q4_SCALE_RU) != 0, (cudaStream_t)stream, num_sms()));
+}
+
 q4_status q4_quantize(q4_format format, int block, q4_dtype in_dt, const void* x, int64_t rows, int64_t cols,
                       int64_t ld, const float* d_gscale, const float* d_chan, uint8_t* codes, uint8_t* scales,
                       int flags, void* stream) {
     if (!valid_format(format) || !valid_dtype(in_dt) || rows < 0 || cols < 0 || ld < cols) return Q4_ERR_ARG;
     if (block != block_of(format)) return Q4_ERR_UNSUPPORTED;
-    if (flags & ~(Q4_SCALE_RU | Q4_LAYOUT_TC | Q4_HADAMARD32 | Q4_SCALE_46)) return Q4_ERR_ARG;
+    if (flags & ~(Q4_SCALE_RU | Q4_LAYOUT_TC | Q4_HADAMARD32 | Q4_SCALE_46 | Q4_INJECT_STALL)) return Q4_ERR_ARG;
     if (format == Q4_NVFP4 && ((flags & Q4_HADAMARD32) || d_chan)) return Q4_ERR_UNSUPPORTED;
     if (format == Q4_MXFP4 && (flags & Q4_SCALE_46)) return Q4_ERR_UNSUPPORTED;
     if (format == Q4_NVFP4 && !d_gscale) return Q4_ERR_ARG;
@@ -123,6 +149,7 @@ q4_status q4_quantize(q4_format format, int block, q4_dtype in_dt, const void* x
     p.x = x; p.rows = rows; p.cols = cols; p.ld = ld;
     p.gscale = d_gscale; p.chan = d_chan; p.codes = codes; p.scales = scales;
     p.scols = cols / block; p.catoms = catoms_of(cols, block);
+    p.inject_stall = (flags & Q4_INJECT_STALL) ? 1 : 0;
     return cuda_status(q4::launch_quantize(p, block, in_dt == Q4_BF16, (flags & Q4_LAYOUT_TC) != 0,
                                            (flags & Q4_SCALE_RU) != 0, (flags & Q4_HADAMARD32) != 0,
                                            d_chan != nullptr, (flags & Q4_SCALE_46) != 0, (cudaStream_t)stream,
@@ -363,6 +390,12 @@ q4_status q4_gemm(q4_format format, int block, int64_t M, int64_t N, int64_t K, 
     p.b_codes = b_codes; p.b_scales = b_scales; p.b_gscale = d_b_gscale;
     p.y = y; p.out_bf16 = out_dt == Q4_BF16; p.mxfp4 = format == Q4_MXFP4;
     return cuda_status(q4::launch_gemm(p, st, num_sms()));
+}
+
+q4_status q4_set_wait_limit(int64_t cycles) {
+    if (cycles == 0) cycles = Q4_DEFAULT_WAIT_CYCLES;
+    if (cycles < 1000 || cycles > ((int64_t)1 << 40)) return Q4_ERR_ARG;
+    return cuda_status(q4::set_wait_limit((long long)cycles));
 }
 
 q4_status q4_get_device_error(void* stream) {

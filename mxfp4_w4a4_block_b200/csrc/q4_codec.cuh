@@ -120,11 +120,16 @@ __device__ __forceinline__ float exp2_int(int k) {
     return __uint_as_float(0x00400000u);
 }
 
-// Per-block normalisation factor of NVFP4 (see q4.h): inv = 1 / (s_b * s_t),
-// or 0 with *degenerate set when the block has no usable scale.
+// Per-block normalisation of NVFP4 (see q4.h): elements are divided by the
+// block's decoded scale S = dec(s_b) * s_t, one correctly rounded binary32
+// division per element ("Looped Transformer quantization", sec. 2.5: x = W / s).
+// y = RN(1 / S) feeds the quotient helpers below; it is NaN for a degenerate
+// block (S = 0, a reciprocal that overflows, or an unusable s_t: every
+// normalised value is +0) and 0 when S lies outside [2^-96, 2^29], where the
+// helpers take the correctly rounded division itself.
 struct NvScale {
     uint32_t byte;
-    float inv;
+    float S, y;
     bool degenerate;
 };
 
@@ -132,27 +137,121 @@ __device__ __forceinline__ bool st_valid(float s_t) {
     return s_t > 0.0f && isfinite(s_t);
 }
 
-__device__ __forceinline__ NvScale nv_scale_from_amax(float amax, float s_t, bool round_up) {
+__device__ __forceinline__ NvScale nv_scale_of(uint32_t byte, float s_t) {
     NvScale r;
-    r.byte = 0;
-    if (st_valid(s_t)) {
-        float denom = __fmul_rn(6.0f, s_t);
-        float sbf = __fdiv_rn(amax, denom);
-        r.byte = round_up ? e4m3_ru(sbf) : e4m3_rn(sbf);
-    }
-    float S = __fmul_rn(e4m3_value(r.byte), s_t);
-    r.inv = __frcp_rn(S);
-    r.degenerate = !st_valid(s_t) || S == 0.0f || !isfinite(r.inv);
+    r.byte = byte;
+    r.S = __fmul_rn(e4m3_value(byte), s_t);
+    const float y = __frcp_rn(r.S);
+    r.degenerate = !st_valid(s_t) || r.S == 0.0f || !isfinite(y);
+    r.y = r.degenerate ? __uint_as_float(0x7FC00000u) : ((r.S >= 0x1p-96f && r.S <= 0x1p29f) ? y : 0.0f);
     return r;
 }
 
-__device__ __forceinline__ NvScale nv_scale_from_byte(uint32_t byte, float s_t) {
-    NvScale r;
-    r.byte = byte;
-    float S = __fmul_rn(e4m3_value(byte), s_t);
-    r.inv = __frcp_rn(S);
-    r.degenerate = !st_valid(s_t) || S == 0.0f || !isfinite(r.inv);
-    return r;
+__device__ __forceinline__ NvScale nv_scale_from_amax(float amax, float s_t, bool round_up) {
+    uint32_t byte = 0;
+    if (st_valid(s_t)) {
+        float denom = __fmul_rn(6.0f, s_t);
+        float sbf = __fdiv_rn(amax, denom);
+        byte = round_up ? e4m3_ru(sbf) : e4m3_rn(sbf);
+    }
+    return nv_scale_of(byte, s_t);
+}
+
+__device__ __forceinline__ NvScale nv_scale_from_byte(uint32_t byte, float s_t) { return nv_scale_of(byte, s_t); }
+
+// ---- pairs of binary32 values on the f32x2 ALU: each lane is rounded to
+// nearest exactly as the scalar __fmul_rn / __fadd_rn / __fsub_rn.
+__device__ __forceinline__ float2 mul2_rn(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "mul.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+// Two scalar products rounded to nearest, for a product that feeds an add:
+// ptxas fuses a paired multiply into the paired add that consumes it,
+// rounding modifier or not, while a scalar mul.rn is never contracted.
+__device__ __forceinline__ float2 mul2_sep_rn(float2 a, float2 b) {
+    return make_float2(__fmul_rn(a.x, b.x), __fmul_rn(a.y, b.y));
+}
+__device__ __forceinline__ float2 add2_rn(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "add.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 sub2_rn(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "sub.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
+__device__ __forceinline__ float2 fma2_rn(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n\t.reg .b64 a, b, c, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\tmov.b64 c, {%6, %7};\n\t"
+        "fma.rn.f32x2 d, a, b, c;\n\tmov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+
+// ---- the correctly rounded quotient RN(w / S) from y = RN(1 / S)
+// One Markstein correction step (P. Markstein, "Computation of elementary
+// functions on the IBM RISC System/6000 processor", IBM J. Res. Develop. 34(1),
+// 1990): q0 = RN(w * y) is within one unit in the last place of w / S, so the
+// remainder r = w - q0 * S is a binary32 number that one fused multiply-add
+// forms exactly, and RN(q0 + r * y) is the correctly rounded quotient.  For
+// significands of w and S in [1, 2) the sequence was compared with the
+// correctly rounded division on every one of the 2^46 pairs; scaling w and S
+// by powers of two scales every step exactly while w, q0 and r stay on the
+// binary32 grid without overflow, which holds for S in [2^-96, 2^29] (y > 0)
+// and 2^-96 <= |w| <= 2^24 (then 2^-125 <= |q0| <= 2^120).
+__device__ __forceinline__ float quot_fast(float w, float S, float y) {
+    const float q0 = __fmul_rn(w, y);
+    const float r = __fmaf_rn(-q0, S, w);
+    return __fmaf_rn(r, y, q0);
+}
+
+__device__ __forceinline__ bool quot_domain(float w) { return fabsf(w) >= 0x1p-96f && fabsf(w) <= 0x1p24f; }
+
+// The correctly rounded division, out of line: taken only for values outside
+// the correction step's domain (zeros, subnormal-range or huge weights) or
+// scales outside its range.
+static __device__ __noinline__ float4 quot4_div(float4 w, float S) {
+    return make_float4(__fdiv_rn(w.x, S), __fdiv_rn(w.y, S), __fdiv_rn(w.z, S), __fdiv_rn(w.w, S));
+}
+
+// RN(w_j / S) for four finite values (S > 0 with its NvScale y, y not NaN):
+// the correction step on f32x2 pairs (the negated scale nS = -S is passed in,
+// so no operand needs negating), or the correctly rounded division for all
+// four when any of them lies outside the step's domain or y = 0.
+__device__ __forceinline__ float4 quot4_rn(float4 w, float S, float nS, float y) {
+    const float2 yy = make_float2(y, y), nn = make_float2(nS, nS);
+    const float2 wa = make_float2(w.x, w.y), wb = make_float2(w.z, w.w);
+    const float2 qa = mul2_rn(wa, yy), qb = mul2_rn(wb, yy);
+    const float2 ra = fma2_rn(qa, nn, wa), rb = fma2_rn(qb, nn, wb);
+    const float2 xa = fma2_rn(ra, yy, qa), xb = fma2_rn(rb, yy, qb);
+    const bool ok = y > 0.0f && quot_domain(w.x) && quot_domain(w.y) && quot_domain(w.z) && quot_domain(w.w);
+    if (__builtin_expect(!ok, 0)) return quot4_div(w, S);
+    return make_float4(xa.x, xa.y, xb.x, xb.y);
+}
+
+// RN(w / S) for one finite value, as quot4_rn.
+__device__ __forceinline__ float quot_rn(float w, float S, float y) {
+    if (y > 0.0f && quot_domain(w)) return quot_fast(w, S, y);
+    return __fdiv_rn(w, S);
+}
+
+// The code-decision form for a whole block whose guard `quot_block_fast`
+// holds: for every element whose quotient reaches 2^-3, |w| >= 2^-3 S >= 2^-99
+// keeps the remainder's bits above 2^-149 and q0 <= amax y <= 2^96, so the
+// quotient there is exact; smaller quotients may be off by a few units but stay
+// below 2^-3 with the sign of w, which is all the E2M1 code of such a value
+// (magnitude 0) depends on.
+__device__ __forceinline__ bool quot_block_fast(float amax, float y) {
+    return y > 0.0f && __fmul_rn(amax, y) <= 0x1p96f;
 }
 
 // E4M3 byte (round to nearest even, saturating) of the binary32 quotient
@@ -195,36 +294,6 @@ __device__ __forceinline__ float amax_tree(const float* v) {
     return fmaxf(0.0f, m[0]);
 }
 
-// ---- pairs of binary32 values on the f32x2 ALU: each lane is rounded to
-// nearest exactly as the scalar __fmul_rn / __fadd_rn / __fsub_rn.
-__device__ __forceinline__ float2 mul2_rn(float2 a, float2 b) {
-    float2 d;
-    asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
-        "mul.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
-        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-    return d;
-}
-// Two scalar products rounded to nearest, for a product that feeds an add:
-// ptxas fuses a paired multiply into the paired add that consumes it,
-// rounding modifier or not, while a scalar mul.rn is never contracted.
-__device__ __forceinline__ float2 mul2_sep_rn(float2 a, float2 b) {
-    return make_float2(__fmul_rn(a.x, b.x), __fmul_rn(a.y, b.y));
-}
-__device__ __forceinline__ float2 add2_rn(float2 a, float2 b) {
-    float2 d;
-    asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
-        "add.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
-        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-    return d;
-}
-__device__ __forceinline__ float2 sub2_rn(float2 a, float2 b) {
-    float2 d;
-    asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
-        "sub.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
-        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-    return d;
-}
-
 // Values of the two E2M1 codes in one byte (element 0 = low nibble -> .x),
 // through the hardware E2M1 -> f16 conversion (every E2M1 value is exact in
 // f16 and in binary32).
@@ -239,15 +308,15 @@ __device__ __forceinline__ float2 e2m1x2_value(uint32_t byte) {
 
 // NVFP4 per-launch context: the tensor scale, 6 * s_t and its reciprocal,
 // whether the fast RN scale path applies, and the shared-memory table of
-// 1 / (dec(s_b) * s_t) for every E4M3 byte 0..127 (NaN marks a degenerate
-// scale: zero, or a reciprocal that is not finite).
+// (S, y) = (dec(s_b) * s_t, RN(1 / S)) for every E4M3 byte 0..127, y as in
+// NvScale (NaN: degenerate; 0: S outside the correction step's range).
 struct NvCtx {
     float s_t, denom, rden;
     bool st_ok, fast;
-    const float* tab;
+    const float2* tab;
 };
 
-__device__ __forceinline__ NvCtx nv_ctx(float s_t, const float* tab) {
+__device__ __forceinline__ NvCtx nv_ctx(float s_t, const float2* tab) {
     NvCtx c;
     c.s_t = s_t;
     c.st_ok = st_valid(s_t);
@@ -258,17 +327,52 @@ __device__ __forceinline__ NvCtx nv_ctx(float s_t, const float* tab) {
     return c;
 }
 
-__device__ __forceinline__ void nv_fill_table(float s_t, float* tab, int tid, int nthreads) {
+__device__ __forceinline__ void nv_fill_table(float s_t, float2* tab, int tid, int nthreads) {
     for (int b = tid; b < 128; b += nthreads) {
-        const NvScale r = nv_scale_from_byte((uint32_t)b, s_t);
-        tab[b] = r.degenerate ? __uint_as_float(0x7FC00000u) : r.inv;
+        const NvScale r = nv_scale_of((uint32_t)b, s_t);
+        tab[b] = make_float2(r.S, r.y);
+    }
+}
+
+// E2M1 codes of the 16 values of a block divided by S (y = RN(1 / S) from the
+// table, amax the block's largest magnitude): 0 for a degenerate scale (y
+// NaN), the correction step on f32x2 pairs when the block guard holds, the
+// correctly rounded division otherwise.
+__device__ __forceinline__ void nv_codes16(const float (&v)[16], float2 sy, float amax, uint32_t (&w)[2]) {
+    const float S = sy.x, y = sy.y;
+    if (y != y) {
+        w[0] = w[1] = 0u;
+    } else if (quot_block_fast(amax, y)) {
+        const float2 yy = make_float2(y, y), SS = make_float2(S, S);
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+            float q[8];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 x = make_float2(v[8 * g + 2 * i], v[8 * g + 2 * i + 1]);
+                const float2 q0 = mul2_rn(x, yy);
+                const float2 t = fma2_rn(q0, SS, make_float2(-x.x, -x.y));
+                const float2 q1 = fma2_rn(make_float2(-t.x, -t.y), yy, q0);
+                q[2 * i] = q1.x;
+                q[2 * i + 1] = q1.y;
+            }
+            w[g] = e2m1_pack8(q);
+        }
+    } else {
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+            float q[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(v[8 * g + i], S);
+            w[g] = e2m1_pack8(q);
+        }
     }
 }
 
 // N NVFP4 blocks at once: amax, E4M3 scale byte (RN or RU of amax / (6 s_t)),
-// codes of x * inv (all zero for a degenerate scale).  Each step runs over
-// all N blocks before the next, with no branch that is not uniform across
-// the warp in between, so the blocks' dependency chains interleave.
+// codes of x / S (all zero for a degenerate scale).  Each step runs over all
+// N blocks before the next, with no branch that is not uniform across the
+// warp in between, so the blocks' dependency chains interleave.
 template <bool RU, int N>
 __device__ __forceinline__ void nv_blocks(const float (&v)[N][16], const NvCtx& c, uint32_t (&byte)[N],
                                           uint32_t (&w)[N][2]) {
@@ -291,25 +395,11 @@ __device__ __forceinline__ void nv_blocks(const float (&v)[N][16], const NvCtx& 
         for (int k = 0; k < N; ++k)
             byte[k] = RU ? e4m3_ru(__fdiv_rn(amax[k], c.denom)) : e4m3_rn(__fdiv_rn(amax[k], c.denom));
     }
-    float inv[N];
+    float2 sy[N];
 #pragma unroll
-    for (int k = 0; k < N; ++k) inv[k] = c.tab[byte[k]];
+    for (int k = 0; k < N; ++k) sy[k] = c.tab[byte[k]];
 #pragma unroll
-    for (int k = 0; k < N; ++k) {
-        const float2 iv = make_float2(inv[k], inv[k]);
-#pragma unroll
-        for (int g = 0; g < 2; ++g) {
-            float q[8];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float2 m = mul2_rn(make_float2(v[k][8 * g + 2 * i], v[k][8 * g + 2 * i + 1]), iv);
-                q[2 * i] = m.x;
-                q[2 * i + 1] = m.y;
-            }
-            // a degenerate scale (NaN entry) gives all-zero codes
-            w[k][g] = inv[k] != inv[k] ? 0u : e2m1_pack8(q);
-        }
-    }
+    for (int k = 0; k < N; ++k) nv_codes16(v[k], sy[k], amax[k], w[k]);
 }
 
 template <bool RU>

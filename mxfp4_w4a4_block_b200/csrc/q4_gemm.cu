@@ -1244,7 +1244,7 @@ cudaError_t launch_w4a16(const W4A16Params& p, cudaStream_t st, int num_sms) {
 // the reference weight and the residue state at every visit): for a small
 // batch X (M <= 16 bf16 rows) and the FP32 master weight W [N, K] with fixed
 // NVFP4 block scales,
-//     q = E2M1(W * inv + r),  r <- (W * inv + r) - q,  Y = s_t * X (q * s_b)^T,
+//     q = E2M1(W / S + r),  r <- (W / S + r) - q,  Y = s_t * X (q * s_b)^T,
 // where the codes q never leave the chip: each weight element is read once
 // with its residue, the new residue is written back, and the dequantized
 // weight q * s_b (exact in bf16) is the tensor-core operand.  The product is
@@ -1274,7 +1274,7 @@ constexpr int OFF_SF = OFF_X + 2048;     // one scale atom
 constexpr int STAGE = 85 * 1024;
 constexpr int OFF_RED = STAGES * STAGE;  // fp32 partial tile [128][16]
 constexpr int OFF_BAR = OFF_RED + BM * 16 * 4;
-constexpr int SMEM_BYTES = OFF_BAR + 1024 + 1024;
+constexpr int SMEM_BYTES = OFF_BAR + 512 + 1024 + 1024;   // barriers, (S, 1/S) table, alignment
 constexpr int CONV_WARPS = 8;            // two threads per weight row, one per 32-element box
 constexpr int EPI_WARPS = 4;
 constexpr int THREADS = 32 * (2 + CONV_WARPS + EPI_WARPS);
@@ -1313,7 +1313,7 @@ __device__ __forceinline__ void sd_gemm_cta(const CUtensorMap& tmW, const CUtens
     uint64_t* tmem_full = empty + STAGES;
     uint64_t* mma_done = tmem_full + 1;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
-    float* inv_tab = reinterpret_cast<float*>(smem + OFF_BAR + 512);   // 128 entries
+    float2* nv_tab = reinterpret_cast<float2*>(smem + OFF_BAR + 512);   // 128 (S, 1/S) entries
     float* red = reinterpret_cast<float*>(smem + OFF_RED);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1390,7 +1390,7 @@ __device__ __forceinline__ void sd_gemm_cta(const CUtensorMap& tmW, const CUtens
         constexpr int BPR = CT / BM;                 // threads per weight row
         const int rr = ct % BM, hb = ct / BM;
         const float s_t = *p.gscale;
-        nv_fill_table(s_t, inv_tab, ct, CT);
+        nv_fill_table(s_t, nv_tab, ct, CT);
         named_barrier(1, CT);
         const bool row_ok = row0 + rr < p.N;
         uint32_t phase = 0;
@@ -1407,18 +1407,19 @@ __device__ __forceinline__ void sd_gemm_cta(const CUtensorMap& tmW, const CUtens
                     // elements e = 32b + 4c .. +3 of the stage, block j = e / 16
                     const int j = 2 * b + (c >> 2);
                     const uint32_t sb = (sw >> (8 * j)) & 0xFFu;
-                    const float inv = inv_tab[sb & 0x7Fu];
+                    const float2 sy = nv_tab[sb & 0x7Fu];
                     const uint32_t off = (uint32_t)(b * 16384 + rr * 128 + ((c ^ (rr & 7)) << 4));
                     const float4 w4 = *reinterpret_cast<const float4*>(st + OFF_W + off);
                     float4* rp = reinterpret_cast<float4*>(st + OFF_R + off);
                     const float4 r4 = *rp;
                     float2 x01, x23;
-                    if (inv != inv) {
+                    if (sy.y != sy.y) {
                         x01 = make_float2(0.0f, 0.0f);
                         x23 = x01;
                     } else {
-                        x01 = mul2_sep_rn(make_float2(w4.x, w4.y), make_float2(inv, inv));   // feeds an add
-                        x23 = mul2_sep_rn(make_float2(w4.z, w4.w), make_float2(inv, inv));
+                        const float4 x = quot4_rn(w4, sy.x, -sy.x, sy.y);
+                        x01 = make_float2(x.x, x.y);
+                        x23 = make_float2(x.z, x.w);
                     }
                     const float2 v01 = add2_rn(x01, make_float2(r4.x, r4.y));
                     const float2 v23 = add2_rn(x23, make_float2(r4.z, r4.w));
@@ -1692,7 +1693,7 @@ constexpr uint32_t SF_COL = 128;         // SF_NBUF scale buffers of SF_BUF colu
 constexpr uint32_t SF_BUF = 32;          //   weight atoms x 4 columns, then activation atoms x 4
 constexpr int SF_NBUF = 4;
 constexpr int MAX_SMEM = 232448;         // 227 KB opt-in limit per CTA
-constexpr int BAR_BYTES = 1024;       // barriers (< 512 B), then the 128-entry reciprocal table
+constexpr int BAR_BYTES = 1536;       // barriers (< 512 B), then the 128-entry (S, 1/S) table
 }  // namespace dec
 
 struct DecodeDev {
@@ -1749,7 +1750,7 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
     uint64_t* tmem_empty = tmem_full + 1;
     uint64_t* mma_done = tmem_empty + 1;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
-    float* inv_tab = reinterpret_cast<float*>(smem + L.off_bar + 512);   // 128 entries
+    float2* nv_tab = reinterpret_cast<float2*>(smem + L.off_bar + 512);   // 128 (S, 1/S) entries
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -1843,8 +1844,8 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
         // ---- quantize activation slabs (warps 2..9)
         const int qt = threadIdx.x - 32 * FIRST_Q;
         constexpr int QT = 32 * QWARPS;
-        const NvCtx sc = nv_ctx(*p.a_gscale, inv_tab);
-        nv_fill_table(*p.a_gscale, inv_tab, qt, QT);
+        const NvCtx sc = nv_ctx(*p.a_gscale, nv_tab);
+        nv_fill_table(*p.a_gscale, nv_tab, qt, QT);
         named_barrier(1, QT);
         // Each quantizer thread fetches exactly the activation bytes it will
         // quantize with cp.async, XDIST k-blocks ahead, into its own part of a
@@ -2008,6 +2009,12 @@ cudaError_t launch_fused_decode(const FusedDecodeParams& p, cudaStream_t st, int
     const int grid = (int)(tiles < num_sms ? tiles : num_sms);
     fused_decode_kernel<<<grid, THREADS, smem, st>>>(mw, d);
     return cudaGetLastError();
+}
+
+cudaError_t set_wait_limit(long long cycles) {
+    cudaError_t e = set_module_wait_limit(cycles);
+    if (e == cudaSuccess) e = set_quant_wait_limit(cycles);
+    return e;
 }
 
 cudaError_t read_clear_device_error(unsigned int* word) {

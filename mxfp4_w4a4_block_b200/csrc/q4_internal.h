@@ -16,6 +16,12 @@ struct QuantParams {
     uint8_t* scales;      // tensor-core layout or row-major
     int64_t scols;        // cols / block
     int64_t catoms;       // ceil(scols / 4)
+    int inject_stall = 0; // failure-detection test: the tiled kernel loads nothing for its first tile
+    // amax + quantize in one launch: out[0] = amax, out[1] = amax / denom (the
+    // tensor scale used), out[2] = the grid barrier's arrival count (zeroed
+    // by the launcher)
+    unsigned int* amax_out = nullptr;
+    float denom = 0.0f;
 };
 
 struct SigmaDeltaParams {
@@ -116,6 +122,8 @@ cudaError_t launch_amax(const void* x, int64_t n, bool bf16, float denom, float*
                         cudaStream_t st, int num_sms);
 cudaError_t launch_quantize(const QuantParams& p, int blk, bool bf16, bool tc, bool ru, bool had,
                             bool chan, bool s46, cudaStream_t st, int num_sms);
+// NVFP4 tensor amax, tensor scale and block quantize in one cooperative launch.
+cudaError_t launch_amax_quantize(const QuantParams& p, bool bf16, bool tc, bool ru, cudaStream_t st, int num_sms);
 cudaError_t launch_sigma_delta(const SigmaDeltaParams& p, int blk, bool tc, cudaStream_t st, int num_sms);
 cudaError_t launch_sigma_delta_banks(const SigmaDeltaParams& p, int blk, bool tc, int visits, float* r_out,
                                      cudaStream_t st, int num_sms);
@@ -140,6 +148,10 @@ cudaError_t launch_fused_decode(const FusedDecodeParams& p, cudaStream_t st, int
 cudaError_t read_clear_device_error(unsigned int* word);
 cudaError_t read_clear_quant_error(unsigned int* word);
 
+// Sets the bounded-wait limit (SM clock cycles) of all kernel files.
+cudaError_t set_wait_limit(long long cycles);
+cudaError_t set_quant_wait_limit(long long cycles);
+
 // 2-D tiled tensor map over a row-major [outer, inner] array of `dt`
 // elements with rows `row_bytes` apart; out-of-range box parts read as zero
 // and are not written by stores.  False if the encoder rejects it.
@@ -149,5 +161,10 @@ bool encode_map_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, u
 // Whether the fused-activation small-M GEMM takes this shape (M <= 128 and
 // the quantized activations fit in shared memory next to >= 2 weight stages).
 bool fused_decode_supported(int64_t M, int64_t K);
+
+// Q4_OK for cudaSuccess; otherwise records the error's text for q4_last_error()
+// (per host thread) and returns Q4_ERR_CUDA (the value as an int: q4.h is not
+// included here).
+int status_of_cuda(cudaError_t e);
 
 }  // namespace q4

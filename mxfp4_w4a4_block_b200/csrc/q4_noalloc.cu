@@ -27,8 +27,10 @@ uint8_t* g_scratch_ptr[kMaxDevices] = {};
 
 // Device address of the scratch array on the current device.  In host code the
 // array's name is only a host-side stand-in, so the address is looked up once
-// per device (with that device current) and cached.
-cudaError_t scratch_on_current_device(uint8_t** out) {
+// per device (with that device current) and cached for the life of the
+// process: a cudaDeviceReset after the first call on a device is not supported
+// (the module may be loaded again elsewhere and the cached address goes stale).
+cudaError_t scratch_on_current_device(uint8_t** out, int* dev_out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -41,8 +43,11 @@ cudaError_t scratch_on_current_device(uint8_t** out) {
         g_scratch_ptr[dev] = static_cast<uint8_t*>(p);
     }
     *out = g_scratch_ptr[dev];
+    *dev_out = dev;
     return cudaSuccess;
 }
+
+q4_status status_of(cudaError_t e) { return (q4_status)q4::status_of_cuda(e); }
 
 }  // namespace
 
@@ -53,23 +58,28 @@ extern "C" Q4_API q4_status q4_gemm_a_bf16_noalloc(int64_t M, int64_t N, int64_t
     if (M < 0 || N < 0 || K < 0 || (out_dt != Q4_F32 && out_dt != Q4_BF16)) return Q4_ERR_ARG;
     if (!d_a_gscale || !d_b_gscale) return Q4_ERR_ARG;
     if (K % 64 || N % 8) return Q4_ERR_SHAPE;
+    if (K > ((int64_t)1 << 30) || M > ((int64_t)1 << 31) || N > ((int64_t)1 << 31)) return Q4_ERR_SHAPE;
     if (M == 0 || N == 0) return Q4_OK;
-    if (K == 0 || !a_bf16 || !b_codes || !b_scales || !y) return Q4_ERR_ARG;
+    if (!y) return Q4_ERR_ARG;
+    if (reinterpret_cast<uintptr_t>(y) & 15u) return Q4_ERR_ALIGN;
+    cudaStream_t st = (cudaStream_t)stream;
+    // K = 0: an empty sum, as q4_gemm gives it
+    if (K == 0) return status_of(cudaMemsetAsync(y, 0, (size_t)M * (size_t)N * (out_dt == Q4_BF16 ? 2 : 4), st));
+    if (!a_bf16 || !b_codes || !b_scales) return Q4_ERR_ARG;
     const uintptr_t mis = reinterpret_cast<uintptr_t>(a_bf16) | reinterpret_cast<uintptr_t>(b_codes) |
-                          reinterpret_cast<uintptr_t>(b_scales) | reinterpret_cast<uintptr_t>(y);
+                          reinterpret_cast<uintptr_t>(b_scales);
     if (mis & 15u) return Q4_ERR_ALIGN;
     // the activation codes and scales must fit in the fixed array
     const size_t codes = (size_t)M * (size_t)(K / 2);
     const size_t codes_al = (codes + 255) / 256 * 256;
     const size_t scales = q4_scale_bytes(Q4_NVFP4, M, K, Q4_LAYOUT_TC);
-    if (codes / (size_t)M != (size_t)(K / 2) || codes_al + scales > (size_t)Q4_NOALLOC_SCRATCH_BYTES)
-        return Q4_ERR_WORKSPACE;
+    if (codes_al + scales > (size_t)Q4_NOALLOC_SCRATCH_BYTES) return Q4_ERR_WORKSPACE;
 
     uint8_t* scratch = nullptr;
-    if (scratch_on_current_device(&scratch) != cudaSuccess) return Q4_ERR_CUDA;
-    cudaStream_t st = (cudaStream_t)stream;
     int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaError_t e = scratch_on_current_device(&scratch, &dev);
+    if (e != cudaSuccess) return status_of(e);
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1) sms = 148;
 
     // Every code byte the GEMM reads and every scale atom (padding included)
     // is written by the quantize launch, so nothing left from an earlier call
@@ -77,12 +87,13 @@ extern "C" Q4_API q4_status q4_gemm_a_bf16_noalloc(int64_t M, int64_t N, int64_t
     q4::QuantParams qp;
     qp.x = a_bf16; qp.rows = M; qp.cols = K; qp.ld = K; qp.gscale = d_a_gscale; qp.chan = nullptr;
     qp.codes = scratch; qp.scales = scratch + codes_al; qp.scols = K / 16; qp.catoms = ((K / 16) + 3) / 4;
-    if (q4::launch_quantize(qp, 16, true, true, false, false, false, false, st, sms) != cudaSuccess) return Q4_ERR_CUDA;
+    e = q4::launch_quantize(qp, 16, true, true, false, false, false, false, st, sms);
+    if (e != cudaSuccess) return status_of(e);
 
     q4::GemmParams p;
     p.M = M; p.N = N; p.K = K;
     p.a_codes = scratch; p.a_scales = scratch + codes_al; p.a_gscale = d_a_gscale;
     p.b_codes = b_codes; p.b_scales = b_scales; p.b_gscale = d_b_gscale;
     p.y = y; p.out_bf16 = out_dt == Q4_BF16; p.mxfp4 = false;
-    return q4::launch_gemm(p, st, sms) == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
+    return status_of(q4::launch_gemm(p, st, sms));
 }

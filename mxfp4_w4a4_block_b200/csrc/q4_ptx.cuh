@@ -23,9 +23,16 @@ static inline cudaError_t read_clear_module_error(unsigned int* word) {
     return cudaMemcpyToSymbol(g_device_error, &zero, sizeof(unsigned int));
 }
 
-// A bounded wait gives up after about this many SM clock cycles (~1 s at the
-// B200's clocks), records kErrTimeout and lets the kernel wind down.
+// A bounded wait gives up after g_wait_limit SM clock cycles (by default
+// kWaitCycles, about 1 s at the B200's clocks), records kErrTimeout and lets
+// the kernel wind down.  Like the error word, each kernel file has its own
+// copy; q4_set_wait_limit() sets all of them.
 constexpr long long kWaitCycles = 2000000000ll;
+static __device__ long long g_wait_limit = kWaitCycles;
+
+static inline cudaError_t set_module_wait_limit(long long cycles) {
+    return cudaMemcpyToSymbol(g_wait_limit, &cycles, sizeof(long long));
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -64,9 +71,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // records a timeout) if it has not completed within kWaitCycles.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
-    long long t0 = clock64();
+    const long long t0 = clock64(), limit = g_wait_limit;
     while (!mbar_try_wait(bar, parity)) {
-        if (clock64() - t0 > kWaitCycles) {
+        if (clock64() - t0 > limit) {
             atomicOr(&g_device_error, kErrTimeout);
             return false;
         }
@@ -87,14 +94,21 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
 }
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
-    long long t0 = clock64();
+    const long long t0 = clock64(), limit = g_wait_limit;
     while (!mbar_try_wait_cluster(bar, parity)) {
-        if (clock64() - t0 > kWaitCycles) {
+        if (clock64() - t0 > limit) {
             atomicOr(&g_device_error, kErrTimeout);
             return false;
         }
     }
     return true;
+}
+
+// ---------------------------------------------------------------- global flags
+__device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int* p) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
 }
 
 // ---------------------------------------------------------------- fences

@@ -144,37 +144,27 @@ struct QzGeom {
     static constexpr int CHUNKS = BLK * ESZ / 16;               // 16-byte chunks per block
     static constexpr int PER = 16 / ESZ;                        // values per chunk
     static constexpr int TAB_OFF = NSTAGE * STAGE + qz::NBUF * (CODE_TILE + SF_TILE);
-    static constexpr int BAR_OFF = TAB_OFF + 512;               // after the 128-entry reciprocal table
+    static constexpr int BAR_OFF = TAB_OFF + 1024;              // after the 128-entry (S, 1/S) table
     static constexpr int SMEM = BAR_OFF + 256 + 1024;           // + barriers, alignment slack
     static_assert(BPT >= 1 && ROWS % 128 == 0 && ROWS <= 256, "tile geometry");
 };
 
 // One candidate of 4/6 block scaling: the rounded-up E4M3 scale mapping the
-// block max to `target` (6 or 4), its reciprocal from the table (NaN: a
-// degenerate scale, every code +0), S = dec(s_b) * s_t in binary32, and the
-// block's codes under it.
+// block max to `target` (6 or 4), its table entry (S, y) with S = dec(s_b) *
+// s_t in binary32 (y NaN: a degenerate scale, every code +0), and the block's
+// codes of x / S.
 struct Nv46Cand {
     uint32_t byte, w[2];
-    float inv, S;
+    float S, y;
 };
 
 __device__ __forceinline__ Nv46Cand nv46_candidate(const float (&v)[16], const NvCtx& c, float amax, float target) {
     Nv46Cand k;
     k.byte = c.st_ok ? e4m3_ru(__fdiv_rn(amax, __fmul_rn(target, c.s_t))) : 0u;
-    k.inv = c.tab[k.byte];
-    k.S = __fmul_rn(e4m3_value(k.byte), c.s_t);
-    const float2 iv = make_float2(k.inv, k.inv);
-#pragma unroll
-    for (int g = 0; g < 2; ++g) {
-        float q[8];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float2 m = mul2_rn(make_float2(v[8 * g + 2 * i], v[8 * g + 2 * i + 1]), iv);
-            q[2 * i] = m.x;
-            q[2 * i + 1] = m.y;
-        }
-        k.w[g] = k.inv != k.inv ? 0u : e2m1_pack8(q);
-    }
+    const float2 sy = c.tab[k.byte];
+    k.S = sy.x;
+    k.y = sy.y;
+    nv_codes16(v, sy, amax, k.w);
     return k;
 }
 
@@ -184,7 +174,7 @@ __device__ __forceinline__ Nv46Cand nv46_candidate(const float (&v)[16], const N
 // a degenerate scale gives sum_j x_j^2.
 __device__ __forceinline__ double nv46_sse_f64(const float (&v)[16], const Nv46Cand& k) {
     double err = 0.0;
-    if (k.inv != k.inv) {
+    if (k.y != k.y) {
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             const double d = (double)v[i];
@@ -211,7 +201,7 @@ __device__ __forceinline__ double nv46_sse_f64(const float (&v)[16], const Nv46C
 // the final one at most 2^-24 of what they add).  A non-finite scale gives a
 // NaN estimate.
 __device__ __forceinline__ float nv46_sse_f32(const float (&v)[16], const Nv46Cand& k) {
-    const float S = k.inv != k.inv ? 0.0f : k.S;
+    const float S = k.y != k.y ? 0.0f : k.S;
     float acc0 = 0.0f, acc1 = 0.0f;
 #pragma unroll
     for (int g = 0; g < 2; ++g) {
@@ -314,7 +304,40 @@ __device__ __forceinline__ void mx_block(const float (&v)[32], const float4 (&cw
     }
 }
 
-template <int BLK, bool BF16, bool TC, bool RU, bool HAD, bool CHAN, bool S46 = false>
+// Largest |x| of the rows x cols tensor (row pitch ld elements) over this
+// thread's share: warp w of the grid takes rows w, w + warps, ..., its lanes
+// 16-byte chunks lane, lane + 32, ... of each row, four loads in flight.
+template <bool BF16>
+__device__ __forceinline__ float amax_share(const QuantParams& p, int gwarp, int nwarps, int lane) {
+    constexpr int ESZ = BF16 ? 2 : 4;
+    const int64_t cpr = p.cols * ESZ / 16;
+    float m = 0.0f;
+    auto fold = [&](const uint4& w) {
+        if (BF16) {
+            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) m = fmaxf(m, fmaxf(fabsf(bf16_lo(ws[j])), fabsf(bf16_hi(ws[j]))));
+        } else {
+            m = fmaxf(m, fmaxf(fmaxf(fabsf(__uint_as_float(w.x)), fabsf(__uint_as_float(w.y))),
+                               fmaxf(fabsf(__uint_as_float(w.z)), fabsf(__uint_as_float(w.w)))));
+        }
+    };
+    for (int64_t row = gwarp; row < p.rows; row += nwarps) {
+        const uint4* rp = reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(p.x) + row * p.ld * ESZ);
+        int64_t c = lane;
+        for (; c + 96 < cpr; c += 128) {
+            uint4 w[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) w[u] = __ldg(rp + c + 32 * u);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) fold(w[u]);
+        }
+        for (; c < cpr; c += 32) fold(__ldg(rp + c));
+    }
+    return m;
+}
+
+template <int BLK, bool BF16, bool TC, bool RU, bool HAD, bool CHAN, bool S46 = false, bool AMAX = false>
 __global__ void __launch_bounds__(qz::THREADS, 1)
     quantize_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmC, QuantParams p,
                     int codes_tma) {
@@ -328,7 +351,7 @@ __global__ void __launch_bounds__(qz::THREADS, 1)
     uint64_t* empty = full + G::NSTAGE;
     uint64_t* cfull = empty + G::NSTAGE;     // staging buffer written by every consumer warp
     uint64_t* cfree = cfull + NBUF;          // staging buffer read out by its stores
-    float* inv_tab = reinterpret_cast<float*>(smem + G::TAB_OFF);   // NVFP4: 1 / (s_b * s_t) per byte
+    float2* nv_tab = reinterpret_cast<float2*>(smem + G::TAB_OFF);  // NVFP4: (S, 1/S) per scale byte
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
@@ -343,6 +366,50 @@ __global__ void __launch_bounds__(qz::THREADS, 1)
         fence_mbar_init();
     }
     __syncthreads();
+
+    // With AMAX, the tensor scale comes first: every thread of the grid folds
+    // its share of |x| into a maximum, each CTA adds its maximum to out[0]
+    // (non-negative floats order like their bit patterns) and arrives on
+    // out[2]; once all CTAs have arrived (a bounded wait: the launch is
+    // cooperative, so they are all resident) each computes s_t = amax / denom
+    // itself, and CTA 0 stores it in out[1].  The quantization below then reads
+    // X a second time, mostly from L2.
+    float s_t_dyn = 0.0f;
+    if constexpr (AMAX) {
+        __shared__ float red[qz::THREADS / 32];
+        __shared__ float s_shared;
+        __shared__ int go;
+        float m = amax_share<BF16>(p, blockIdx.x * (qz::THREADS / 32) + warp, gridDim.x * (qz::THREADS / 32), lane);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (lane == 0) red[warp] = m;
+        __syncthreads();
+        if (tid == 0) {
+            float b = 0.0f;
+            for (int w = 0; w < qz::THREADS / 32; ++w) b = fmaxf(b, red[w]);
+            atomicMax(p.amax_out, __float_as_uint(b));
+            __threadfence();
+            atomicAdd(p.amax_out + 2, 1u);
+            bool ok = true;
+            const long long t0 = clock64(), limit = g_wait_limit;
+            while (ld_acquire_gpu(p.amax_out + 2) < gridDim.x) {
+                if (clock64() - t0 > limit) {
+                    atomicOr(&g_device_error, kErrTimeout);
+                    ok = false;
+                    break;
+                }
+            }
+            if (ok) {
+                const float amax = __uint_as_float(ld_acquire_gpu(p.amax_out));
+                s_shared = __fdiv_rn(amax, p.denom);
+                if (blockIdx.x == 0) reinterpret_cast<float*>(p.amax_out)[1] = s_shared;
+            }
+            go = ok ? 1 : 0;
+        }
+        __syncthreads();
+        if (!go) return;                  // nothing issued yet: the whole CTA leaves
+        s_t_dyn = s_shared;
+    }
 
     const int64_t tiles_c = p.catoms;
     const int64_t tiles = ((p.rows + G::ROWS - 1) / G::ROWS) * tiles_c;
@@ -359,15 +426,19 @@ __global__ void __launch_bounds__(qz::THREADS, 1)
             for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
                 // on time-out stop issuing: the consumers then time out on `full`
                 if (!mbar_wait(&empty[stage], phase ^ 1)) break;
-                mbar_arrive_expect_tx(&full[stage], G::STAGE);
-                const int64_t tr = t / tiles_c, tc = t % tiles_c;
-                uint8_t* dst = smem + stage * G::STAGE;
+                // failure-detection test (Q4_INJECT_STALL): the first tile's stage
+                // is never filled, so the consumers' bounded wait on it runs out
+                if (!(p.inject_stall && t == (int64_t)blockIdx.x)) {
+                    mbar_arrive_expect_tx(&full[stage], G::STAGE);
+                    const int64_t tr = t / tiles_c, tc = t % tiles_c;
+                    uint8_t* dst = smem + stage * G::STAGE;
 #pragma unroll
-                for (int b = 0; b < G::NBOX; ++b)
-                    tma_load_2d(dst + b * (G::ROWS * 128), &tmX, &full[stage],
-                                (int32_t)(tc * 4 * BLK + b * (128 / G::ESZ)), (int32_t)(tr * G::ROWS));
-                issued[stage] = true;
-                last_phase[stage] = phase;
+                    for (int b = 0; b < G::NBOX; ++b)
+                        tma_load_2d(dst + b * (G::ROWS * 128), &tmX, &full[stage],
+                                    (int32_t)(tc * 4 * BLK + b * (128 / G::ESZ)), (int32_t)(tr * G::ROWS));
+                    issued[stage] = true;
+                    last_phase[stage] = phase;
+                }
                 if (++stage == G::NSTAGE) { stage = 0; phase ^= 1; }
             }
             // no copy may still be landing in shared memory when the CTA exits
@@ -412,8 +483,9 @@ __global__ void __launch_bounds__(qz::THREADS, 1)
     // ---- consumers
     NvCtx sc;
     if constexpr (BLK == 16) {
-        sc = nv_ctx(*p.gscale, inv_tab);
-        nv_fill_table(*p.gscale, inv_tab, tid, CONSUMERS);
+        const float s_t = AMAX ? s_t_dyn : *p.gscale;
+        sc = nv_ctx(s_t, nv_tab);
+        nv_fill_table(s_t, nv_tab, tid, CONSUMERS);
         named_barrier(1, CONSUMERS);
     }
     const int64_t crow = p.cols / 2;           // bytes of codes per row
@@ -543,8 +615,8 @@ constexpr int STAGE = 2 * HALF + SF_BYTES;
 constexpr int NSTAGE = 5;
 constexpr int CODE_TILE = ROWS * COLS / 2;       // 2 KB
 constexpr int NBUF = 3;
-constexpr int TAB_OFF = NSTAGE * STAGE + NBUF * CODE_TILE;   // 256-entry reciprocal table
-constexpr int BAR_OFF = TAB_OFF + 1024;
+constexpr int TAB_OFF = NSTAGE * STAGE + NBUF * CODE_TILE;   // 256-entry (S, 1/S) table
+constexpr int BAR_OFF = TAB_OFF + 2048;
 constexpr int SMEM = BAR_OFF + 256 + 1024;
 constexpr int GPT = ROWS * COLS / 4 / CONSUMERS; // 4-weight groups per thread per tile
 }  // namespace sdk
@@ -563,7 +635,7 @@ __global__ void __launch_bounds__(sdk::THREADS, 1)
     // per-tile consumer barrier, read after it, so every consumer takes the
     // same decision
     volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + NSTAGE);
-    float* inv_tab = reinterpret_cast<float*>(smem + TAB_OFF);
+    float2* sc_tab = reinterpret_cast<float2*>(smem + TAB_OFF);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
@@ -616,17 +688,16 @@ __global__ void __launch_bounds__(sdk::THREADS, 1)
         return;
     }
 
-    // 1 / (s_b * s_t) (NVFP4) or 2^-e (MXFP4) for every scale byte; NaN marks
-    // a degenerate NVFP4 scale, whose weights normalise to +0
+    // per scale byte: (S, y) of NvScale (NVFP4; y NaN marks a degenerate scale,
+    // whose weights normalise to +0), or (2^e, 2^-e) (MXFP4: dividing by 2^e is
+    // the exact multiplication by 2^-e)
     for (int bb = tid; bb < 256; bb += CONSUMERS) {
-        float inv;
         if (BLK == 16) {
-            const NvScale r = nv_scale_from_byte((uint32_t)(bb & 0x7F), *p.gscale);
-            inv = r.degenerate ? __uint_as_float(0x7FC00000u) : r.inv;
+            const NvScale r = nv_scale_of((uint32_t)(bb & 0x7F), *p.gscale);
+            sc_tab[bb] = make_float2(r.S, r.y);
         } else {
-            inv = exp2_int(127 - bb);
+            sc_tab[bb] = make_float2(exp2_int(bb - 127), exp2_int(127 - bb));
         }
-        inv_tab[bb] = inv;
     }
     named_barrier(1, CONSUMERS);
     const int64_t crow = p.cols / 2;
@@ -656,14 +727,18 @@ __global__ void __launch_bounds__(sdk::THREADS, 1)
                     sb = __ldg(p.scales + row * p.scols + col / BLK);
                 }
             }
-            const float inv = inv_tab[sb];
+            const float2 sy = sc_tab[sb];
             float2 x01, x23;
-            if (inv != inv) {
+            if (BLK == 32) {
+                x01 = mul2_sep_rn(make_float2(w4.x, w4.y), make_float2(sy.y, sy.y));   // feeds an add
+                x23 = mul2_sep_rn(make_float2(w4.z, w4.w), make_float2(sy.y, sy.y));
+            } else if (sy.y != sy.y) {
                 x01 = make_float2(0.0f, 0.0f);
                 x23 = x01;
             } else {
-                x01 = mul2_sep_rn(make_float2(w4.x, w4.y), make_float2(inv, inv));   // feeds an add
-                x23 = mul2_sep_rn(make_float2(w4.z, w4.w), make_float2(inv, inv));
+                const float4 x = quot4_rn(w4, sy.x, -sy.x, sy.y);
+                x01 = make_float2(x.x, x.y);
+                x23 = make_float2(x.z, x.w);
             }
             const float2 v01 = add2_rn(x01, make_float2(r4.x, r4.y));
             const float2 v23 = add2_rn(x23, make_float2(r4.z, r4.w));
@@ -727,32 +802,31 @@ __device__ __forceinline__ void load8(const P& p, int64_t u, In8& in) {
     in.sb = TC ? p.scales[tc_scale_offset(row, c, p.catoms)] : p.scales[row * p.scols + c];
 }
 
-// Reciprocal block scale: 1 / (dec(s_b) s_t) (NVFP4; `degenerate` when that
-// is not a usable scale: the codes are then 0) or 2^-e (MXFP4).
-template <int BLK>
-__device__ __forceinline__ float inv_of(uint32_t sb, float s_t, bool& degenerate) {
-    if (BLK == 16) {
-        const NvScale sc = nv_scale_from_byte(sb, s_t);
-        degenerate = sc.degenerate;
-        return sc.inv;
-    }
-    degenerate = false;
-    return exp2_int(127 - (int)sb);
-}
-
-// x = w * inv for the unit's 8 weights (0 for a degenerate scale), as pairs.
+// The unit's 8 weights divided by their block scale, as pairs: x = w / S with
+// S = dec(s_b) s_t (NVFP4; all +0 for a degenerate scale), or w * 2^-e
+// (MXFP4, the exact quotient by 2^e).
 template <int BLK>
 __device__ __forceinline__ void scaled8(const In8& in, float s_t, float2 (&x)[4]) {
-    bool degenerate;
-    const float inv = inv_of<BLK>(in.sb, s_t, degenerate);
-    const float2 iv = make_float2(inv, inv);
-    // the products feed adds: scalar, never fused
-    x[0] = mul2_sep_rn(make_float2(in.w0.x, in.w0.y), iv);
-    x[1] = mul2_sep_rn(make_float2(in.w0.z, in.w0.w), iv);
-    x[2] = mul2_sep_rn(make_float2(in.w1.x, in.w1.y), iv);
-    x[3] = mul2_sep_rn(make_float2(in.w1.z, in.w1.w), iv);
-    if (degenerate)
-        for (int j = 0; j < 4; ++j) x[j] = make_float2(0.0f, 0.0f);
+    const float wv[8] = {in.w0.x, in.w0.y, in.w0.z, in.w0.w, in.w1.x, in.w1.y, in.w1.z, in.w1.w};
+    if (BLK == 16) {
+        const NvScale sc = nv_scale_of(in.sb, s_t);
+        if (sc.degenerate) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) x[j] = make_float2(0.0f, 0.0f);
+        } else {
+            const float4 a = quot4_rn(in.w0, sc.S, -sc.S, sc.y), b = quot4_rn(in.w1, sc.S, -sc.S, sc.y);
+            x[0] = make_float2(a.x, a.y);
+            x[1] = make_float2(a.z, a.w);
+            x[2] = make_float2(b.x, b.y);
+            x[3] = make_float2(b.z, b.w);
+        }
+    } else {
+        const float m = exp2_int(127 - (int)in.sb);
+        const float2 mm = make_float2(m, m);
+        // the products feed adds: scalar, never fused
+#pragma unroll
+        for (int j = 0; j < 4; ++j) x[j] = mul2_sep_rn(make_float2(wv[2 * j], wv[2 * j + 1]), mm);
+    }
 }
 
 template <int BLK, class P>
@@ -842,9 +916,8 @@ __device__ __forceinline__ void sr_finish(const P& p, int64_t u, const In8& in, 
                                           uint32_t visit) {
     const int64_t cpr = p.cols / 8;
     const int64_t row = u / cpr, col = (u % cpr) * 8;
-    bool degenerate;
-    const float inv = inv_of<BLK>(in.sb, s_t, degenerate);
-    const float wv[8] = {in.w0.x, in.w0.y, in.w0.z, in.w0.w, in.w1.x, in.w1.y, in.w1.z, in.w1.w};
+    float2 xs[4];
+    scaled8<BLK>(in, s_t, xs);
     const uint64_t g = (uint64_t)(row * p.cols + col) >> 2;
     const uint4 r0 = philox4x32_10(make_uint4((uint32_t)g, (uint32_t)(g >> 32), visit, 0u), key);
     const uint4 r1 = philox4x32_10(make_uint4((uint32_t)(g + 1), (uint32_t)((g + 1) >> 32), visit, 0u), key);
@@ -852,7 +925,7 @@ __device__ __forceinline__ void sr_finish(const P& p, int64_t u, const In8& in, 
     uint32_t codes = 0;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-        const float x = degenerate ? 0.0f : __fmul_rn(wv[j], inv);
+        const float x = (j & 1) ? xs[j >> 1].y : xs[j >> 1].x;
         const float uu = (float)(rw[j] >> 8) * 0x1p-24f;
         codes |= sr_e2m1(x, uu) << (4 * j);
     }
@@ -872,7 +945,7 @@ __global__ void __launch_bounds__(256) sr_requant_kernel(SigmaDeltaParams p, uin
     }
 }
 
-// One Sigma-Delta step of one unit (as the tiled kernel above): x = w * inv,
+// One Sigma-Delta step of one unit (as the tiled kernel above): x = w / S,
 // v = x + r, q = E2M1(v), r <- v - q.
 template <int BLK, class P>
 __device__ __forceinline__ void sd_finish(const P& p, int64_t u, const In8& in, float s_t) {
@@ -1094,7 +1167,65 @@ cudaError_t launch_quantize(const QuantParams& p, int blk, bool bf16, bool tc, b
     return launch_quant_blk<32>(p, bf16, tc, ru, had, chan, false, num_sms, st);
 }
 
+template <bool BF16, bool TC, bool RU>
+static cudaError_t launch_amax_quant_one(const QuantParams& p, const QuantMaps& m, int num_sms, cudaStream_t st) {
+    using G = QzGeom<16, BF16>;
+    auto k = quantize_kernel<16, BF16, TC, RU, false, false, false, true>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM);
+    if (e != cudaSuccess) return e;
+    int occ = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, qz::THREADS, G::SMEM);
+    if (e != cudaSuccess) return e;
+    if (occ < 1) return cudaErrorCooperativeLaunchTooLarge;
+    const int64_t tiles = ((p.rows + G::ROWS - 1) / G::ROWS) * p.catoms;
+    // every CTA must be resident at once for the grid-wide wait
+    const int64_t cap = (int64_t)num_sms * occ;
+    const int grid = (int)(tiles < num_sms ? tiles : (num_sms < cap ? num_sms : cap));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(qz::THREADS);
+    cfg.dynamicSmemBytes = G::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, k, m.x, m.codes, p, m.codes_tma);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+cudaError_t launch_amax_quantize(const QuantParams& p, bool bf16, bool tc, bool ru, cudaStream_t st, int num_sms) {
+    cudaError_t e = cudaMemsetAsync(p.amax_out, 0, 4 * sizeof(unsigned int), st);
+    if (e != cudaSuccess || p.rows == 0 || p.cols == 0) return e;
+    QuantMaps m;
+    std::memset(&m, 0, sizeof(m));
+    const int esz = bf16 ? 2 : 4;
+    const int rows_tile = bf16 ? QzGeom<16, true>::ROWS : QzGeom<16, false>::ROWS;
+    if (!encode_map_2d(&m.x, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, p.x,
+                       (uint64_t)p.cols, (uint64_t)p.rows, (uint64_t)(p.ld * esz), (uint32_t)(128 / esz),
+                       (uint32_t)rows_tile, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    m.codes_tma = ((p.cols / 2) % 16 == 0) ? 1 : 0;
+    if (m.codes_tma &&
+        !encode_map_2d(&m.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.codes, (uint64_t)(p.cols / 2), (uint64_t)p.rows,
+                       (uint64_t)(p.cols / 2), 32u, (uint32_t)rows_tile, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+#define Q4_AQ(B, T, R) return launch_amax_quant_one<B, T, R>(p, m, num_sms, st)
+    if (bf16) {
+        if (tc) { if (ru) Q4_AQ(true, true, true); Q4_AQ(true, true, false); }
+        if (ru) Q4_AQ(true, false, true);
+        Q4_AQ(true, false, false);
+    }
+    if (tc) { if (ru) Q4_AQ(false, true, true); Q4_AQ(false, true, false); }
+    if (ru) Q4_AQ(false, false, true);
+    Q4_AQ(false, false, false);
+#undef Q4_AQ
+}
+
 cudaError_t read_clear_quant_error(unsigned int* word) { return read_clear_module_error(word); }
+cudaError_t set_quant_wait_limit(long long cycles) { return set_module_wait_limit(cycles); }
 
 cudaError_t launch_sigma_delta(const SigmaDeltaParams& p, int blk, bool tc, cudaStream_t st, int num_sms) {
     using namespace sdk;
@@ -1348,13 +1479,13 @@ __device__ __forceinline__ void qz_finish(const GroupItem& p, int64_t u, const Q
 
 template <int BLK, bool BF16, bool TC, bool RU, bool HAD, bool S46>
 __global__ void __launch_bounds__(256) quantize_grouped_kernel(const __grid_constant__ GroupParams g) {
-    // NVFP4: each entry's 128-entry table of 1 / (dec(s_b) s_t), as the tiled quantizer's
-    __shared__ float tabs[BLK == 16 ? kMaxGroup * 128 : 1];
+    // NVFP4: each entry's 128-entry table of (S, 1/S), as the tiled quantizer's
+    __shared__ float2 tabs[BLK == 16 ? kMaxGroup * 128 : 1];
     __shared__ float s_ts[kMaxGroup];
     if constexpr (BLK == 16) {
         for (int k = threadIdx.x; k < g.count * 128; k += blockDim.x) {
-            const NvScale r = nv_scale_from_byte((uint32_t)(k & 127), *g.m[k >> 7].gscale);
-            tabs[k] = r.degenerate ? __uint_as_float(0x7FC00000u) : r.inv;
+            const NvScale r = nv_scale_of((uint32_t)(k & 127), *g.m[k >> 7].gscale);
+            tabs[k] = make_float2(r.S, r.y);
         }
         for (int k = threadIdx.x; k < g.count; k += blockDim.x) s_ts[k] = *g.m[k].gscale;
         __syncthreads();

@@ -87,6 +87,15 @@ def test_host_validation_without_launch(lib):
                        None, 0, None) == 7
     # Sigma-Delta: NVFP4 needs s_t
     assert lib.q4_sigma_delta_step(q4.NVFP4, 16, P, 4, 64, P, None, P, P, 0, None) == 1
+    # unknown flag bits are rejected; the stall injection is a quantize flag
+    assert lib.q4_quantize(q4.NVFP4, 16, q4.BF16, P, 4, 64, 64, g, None, P, P, 1 << 17, None) == 1
+    # wait limits outside [1000, 2^40] cycles
+    assert lib.q4_set_wait_limit(999) == 1
+    assert lib.q4_set_wait_limit((1 << 40) + 1) == 1
+    assert lib.q4_set_wait_limit(-5) == 1
+    # no-alloc GEMM: shape bounds before anything else happens
+    assert lib.q4_gemm_a_bf16_noalloc(4, (1 << 31) + 8, 64, P, g, P, P, g, q4.F32, P, None) == 3
+    assert lib.q4_gemm_a_bf16_noalloc(4, 16, 96, P, g, P, P, g, q4.F32, P, None) == 3
 
 
 def test_grouped_host_validation_without_launch(lib):

@@ -188,6 +188,62 @@ def test_prefill_activation_quantize_full_size():
     assert np.array_equal(host(gs), oracle.scales_to_tc(os_))
 
 
+def test_amax_quantize_prefill_full_size():
+    """amax, s_t and NVFP4 quantize of the prefill activation in one launch
+    (the benchmark's step): bit for bit against the oracle and equal to the two
+    separate launches, on two launches in a row."""
+    d = synth.prefill(n_list=())
+    x32 = synth.bf16_to_f32(d["x"])
+    x = dev(d["x"])
+    amax = oracle.amax(x32)
+    s_t = oracle.tensor_scale(amax, 2688.0)
+    oc, os_ = oracle.nvfp4_quantize(x32, s_t)
+    for _ in range(2):
+        gc, gs, out = q4.q4_amax_quantize(x, 2688.0)
+        o = host(out)
+        assert o[0] == amax and o[1] == s_t
+        assert np.array_equal(host(gc), oc)
+        assert np.array_equal(host(gs), oracle.scales_to_tc(os_))
+    assert q4.q4_get_device_error() == 0
+
+
+@pytest.mark.parametrize("rows,cols,ld,bf16,ru,tc", [
+    (300, 400, 400, False, False, False),
+    (300, 400, 416, True, True, True),
+    (1, 16, 16, True, False, True),
+    (4097, 160, 176, False, True, True),
+    (130, 5120, 5120, True, False, False)])
+def test_amax_quantize_parity(rows, cols, ld, bf16, ru, tc):
+    """Ragged, strided, fp32 and bf16, RN and RU scales, both layouts."""
+    full = synth.small_like("heavy", rows + cols, rows, ld)
+    if bf16:
+        xt = synth.to_bf16(full)
+        full = synth.bf16_to_f32(xt)
+        x = dev(xt)[:, :cols]
+    else:
+        x = dev(full)[:, :cols]
+    x32 = np.ascontiguousarray(full[:, :cols])
+    flags = (q4.SCALE_RU if ru else 0) | (q4.LAYOUT_TC if tc else 0)
+    gc, gs, out = q4.q4_amax_quantize(x, 2688.0, flags=flags)
+    amax = oracle.amax(x32)
+    s_t = oracle.tensor_scale(amax, 2688.0)
+    o = host(out)
+    assert o[0] == amax and o[1] == s_t
+    oc, os_ = oracle.nvfp4_quantize(x32, s_t, round_up=ru)
+    assert np.array_equal(host(gc), oc)
+    if tc:
+        assert np.array_equal(host(gs), oracle.scales_to_tc(os_))
+    else:
+        assert np.array_equal(host(gs).reshape(os_.shape), os_)
+
+
+def test_amax_quantize_empty():
+    x = torch.zeros((0, 64), dtype=torch.bfloat16, device=DEV)
+    out = torch.full((4,), 7.0, device=DEV)
+    q4.q4_amax_quantize(x, 2688.0, out=out)
+    assert np.array_equal(host(out), np.zeros(4, np.float32))
+
+
 def test_mxfp4_activation_quantize_full_size():
     """The MXFP4 activation (4096 x 4096 bf16) with t and Hadamard-32, bit for bit."""
     d = synth.mxfp4(n=256)
