@@ -137,13 +137,18 @@ __device__ __forceinline__ bool st_valid(float s_t) {
     return s_t > 0.0f && isfinite(s_t);
 }
 
+// y = RN(1 / S) for a scale S inside the correction step's range [2^-96, 2^29]
+// (see quot_fast below), 0 outside it (the quotient helpers then divide).
+__device__ __forceinline__ float quot_recip(float S) {
+    return (S >= 0x1p-96f && S <= 0x1p29f) ? __frcp_rn(S) : 0.0f;
+}
+
 __device__ __forceinline__ NvScale nv_scale_of(uint32_t byte, float s_t) {
     NvScale r;
     r.byte = byte;
     r.S = __fmul_rn(e4m3_value(byte), s_t);
-    const float y = __frcp_rn(r.S);
-    r.degenerate = !st_valid(s_t) || r.S == 0.0f || !isfinite(y);
-    r.y = r.degenerate ? __uint_as_float(0x7FC00000u) : ((r.S >= 0x1p-96f && r.S <= 0x1p29f) ? y : 0.0f);
+    r.degenerate = !st_valid(s_t) || r.S == 0.0f || !isfinite(__frcp_rn(r.S));
+    r.y = r.degenerate ? __uint_as_float(0x7FC00000u) : quot_recip(r.S);
     return r;
 }
 

@@ -36,14 +36,13 @@ __global__ void pairs_kernel(uint32_t b_lo, uint32_t b_count, uint32_t a_off, ui
     if (bad) atomicAdd(count, bad);
 }
 
-// Elementwise: out_rn[i] = quot_rn(w[i], S[i], y[i]), out_div[i] = __fdiv_rn(w[i], S[i]),
-// with y[i] the library's NvScale y of S (0 outside the fast range).
+// Elementwise: out_rn[i] = quot_rn(w[i], S[i], y), out_div[i] = __fdiv_rn(w[i], S[i]),
+// with y the library's reciprocal of S (0 outside the fast range).
 __global__ void elems_kernel(const float* w, const float* S, int64_t n, float* out_rn, float* out_div) {
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= n) return;
     const float s = S[i];
-    const float yr = __frcp_rn(s);
-    const float y = (s >= 0x1p-96f && s <= 0x1p96f) ? yr : 0.0f;
+    const float y = quot_recip(s);            // the library's rule: 0 outside the fast range
     out_rn[i] = quot_rn(w[i], s, y);
     out_div[i] = __fdiv_rn(w[i], s);
 }
@@ -56,8 +55,7 @@ __global__ void codes_kernel(const float* x, const float* S, int64_t nblocks, ui
     float v[16];
     for (int j = 0; j < 16; ++j) v[j] = x[blk * 16 + j];
     const float s = S[blk];
-    const float yr = __frcp_rn(s);
-    const float y = (s >= 0x1p-96f && s <= 0x1p96f) ? yr : 0.0f;
+    const float y = quot_recip(s);
     const float amax = amax_tree<16>(v);
     uint32_t w[2];
     nv_codes16(v, make_float2(s, y), amax, w);
