@@ -18,7 +18,6 @@
 //               the accumulator to the next tile's MMAs, then scale, convert
 //               and store Y by TMA through a swizzled shared-memory buffer.
 // CTA tile 128 x 256, k-block 256 elements (128 bytes of codes per row).
-// gemm_pair_kernel is the same GEMM on CTA pairs (cta_group::2), off.
 //
 // w4a16_gemm_kernel: bf16 activations times the 4-bit weight dequantized
 // exactly to bf16 in shared memory by converter warps (kind::f16).
@@ -452,353 +451,6 @@ static bool make_out_map(CUtensorMap* map, void* y, int64_t M, int64_t N) {
 }
 
 
-// ------------------------------------------------------------------ CTA-pair GEMM
-// The same GEMM on CTA pairs (clusters of two CTAs on two SMs) with the
-// 2-SM MMA: a pair owns a 256 x 256 output tile, each CTA stages its own 128
-// rows of A and its own 128 rows of the 256-row B tile; the leader CTA issues
-// one 256 x 256 x 64 MMA per K step for both SMs, which halves the per-SM
-// shared-memory and L2 traffic for B.  Both CTAs' A/B TMA loads complete on
-// the leader's `full` barriers; each CTA's scale warps stage its own A scales
-// and the whole B-scale tile into its own TMEM (its scale loads complete on a
-// local barrier) and release them to the leader's `sf_ready`; the leader's
-// commits are multicast to both CTAs' `empty`, `sf_free` and `tmem_full`;
-// both CTAs' epilogue warps release the accumulators on the leader's
-// `tmem_empty` and store their own 128 rows.
-namespace pair {
-constexpr int BM = 128;                  // rows of A per CTA (pair tile 256)
-constexpr int BN = 256;                  // columns per pair tile (128 rows of B per CTA)
-constexpr int KB_BYTES = 128;
-constexpr int KB_ELEMS = 256;
-constexpr int STAGES = 5;
-constexpr int A_STAGE = BM * KB_BYTES;          // 16 KB
-constexpr int B_STAGE = (BN / 2) * KB_BYTES;    // 16 KB
-constexpr int SFA_STAGE = 2048;
-constexpr int SFB_STAGE = 4096;                 // band 0 at +0, band 1 at +2048
-constexpr int OFF_B = STAGES * A_STAGE;
-constexpr int OFF_SFA = OFF_B + STAGES * B_STAGE;
-constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_STAGE;
-constexpr int OFF_EPI = OFF_SFB + STAGES * SFB_STAGE;
-constexpr int EPI_BYTES = 8192;
-constexpr int OFF_BAR = OFF_EPI + EPI_BYTES;
-constexpr int BAR_BYTES = 512;
-constexpr int SMEM_BYTES = OFF_BAR + BAR_BYTES + 1024;
-constexpr int SF_WARPS = 4;
-constexpr int EPI_WARPS = 8;
-constexpr int FIRST_EPI_WARP = 2 + SF_WARPS;
-constexpr int THREADS = 32 * FIRST_EPI_WARP + 32 * EPI_WARPS;
-constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t ACC_COL = 0;
-constexpr uint32_t SF_COL = 256;
-constexpr uint32_t SF_BUF = 48;
-constexpr uint32_t SFB_OFF = 16;
-constexpr int SF_NBUF = 4;               // scale buffers in TMEM (the hand-off crosses CTAs)
-}  // namespace pair
-
-template <bool MX>
-__global__ void __launch_bounds__(pair::THREADS, 1)
-    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
-                     const __grid_constant__ CUtensorMap tmY, GemmDev p) {
-    using namespace pair;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);   // [S] A/B of both CTAs (leader's)
-    uint64_t* sf_full = full + STAGES;                              // [S] this CTA's scale loads
-    uint64_t* empty = sf_full + STAGES;                             // [S]
-    uint64_t* tmem_full = empty + STAGES;
-    uint64_t* tmem_empty = tmem_full + 1;                           // leader's: both CTAs' epilogues
-    uint64_t* mma_done = tmem_empty + 1;
-    uint64_t* sf_ready = mma_done + 1;                              // [SF_NBUF] leader's: both CTAs' scale warps
-    uint64_t* sf_free = sf_ready + SF_NBUF;                         // [SF_NBUF]
-    uint64_t* epi_turn = sf_free + SF_NBUF;                         // [EPI_WARPS]
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(epi_turn + EPI_WARPS);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    const uint32_t rank = cluster_ctarank();
-    const bool leader = rank == 0;
-
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&sf_full[s], 1);
-            mbar_init(&empty[s], 1);
-        }
-        mbar_init(tmem_full, 1);
-        mbar_init(tmem_empty, 2 * EPI_WARPS);           // one arrival per epilogue warp of either CTA
-        mbar_init(mma_done, 1);
-        for (int b = 0; b < SF_NBUF; ++b) { mbar_init(&sf_ready[b], 2 * SF_WARPS); mbar_init(&sf_free[b], 1); }
-        for (int w = 0; w < EPI_WARPS; ++w) mbar_init(&epi_turn[w], 1);
-        *abort_flag = 0;
-        fence_mbar_init();
-    }
-    if (warp == 1) {
-        tmem_alloc2(tmem_holder, TMEM_COLS);
-        tmem_relinquish2();
-    }
-    if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(&tmA); tma_prefetch_desc(&tmB);
-        tma_prefetch_desc(&tmSA); tma_prefetch_desc(&tmSB);
-        if (p.out_bf16) tma_prefetch_desc(&tmY);
-    }
-    tc_fence_before();
-    __syncthreads();
-    cluster_sync();          // barriers and TMEM allocation are visible to the peer
-    tc_fence_after();
-    const uint32_t tmem = *tmem_holder;
-
-    const int64_t tiles_m = (p.M + 2 * BM - 1) / (2 * BM);
-    const int64_t tiles_n = (p.N + BN - 1) / BN;
-    const int64_t tiles = tiles_m * tiles_n;
-    const int64_t pair_id = blockIdx.x >> 1, npairs = gridDim.x >> 1;
-    const int nkb = (int)((p.K + KB_ELEMS - 1) / KB_ELEMS);
-    const int mma_per_atom = MX ? 2 : 1;
-    const int atoms_per_kb = 4 / mma_per_atom;
-    const uint32_t sf_bytes = 512u * (uint32_t)atoms_per_kb;       // one band's scales per k-block
-    const uint32_t ab_bytes = A_STAGE + B_STAGE;                    // one CTA's A/B loads per k-block
-
-    if (warp == 0) {
-        if (lane == 0) {
-            const uint32_t leader_full = mapa_shared(smem_u32(full), 0);
-            int stage = 0;
-            uint32_t phase = 0;
-            uint32_t last_phase[STAGES];
-            bool issued[STAGES];
-            for (int s = 0; s < STAGES; ++s) issued[s] = false, last_phase[s] = 0;
-            for (int64_t t = pair_id; t < tiles && !*abort_flag; t += npairs) {
-                const int64_t mt = t % tiles_m, nt = t / tiles_m;
-                for (int kb = 0; kb < nkb; ++kb) {
-                    if (!mbar_wait(&empty[stage], phase ^ 1)) { *abort_flag = 1; break; }
-                    if (leader) mbar_arrive_expect_tx(&full[stage], 2u * ab_bytes);
-                    mbar_arrive_expect_tx(&sf_full[stage], 3u * sf_bytes);
-                    const uint32_t fb = leader_full + 8u * (uint32_t)stage;
-                    const int32_t krow = (int32_t)(2 * kb * atoms_per_kb);
-                    tma_load_2d_pair(smem + stage * A_STAGE, &tmA, fb, kb * KB_BYTES, (int32_t)(mt * 2 * BM + rank * BM));
-                    tma_load_2d_pair(smem + OFF_B + stage * B_STAGE, &tmB, fb, kb * KB_BYTES,
-                                     (int32_t)(nt * BN + rank * (BN / 2)));
-                    tma_load_2d(smem + OFF_SFA + stage * SFA_STAGE, &tmSA, &sf_full[stage], 0,
-                                (int32_t)(2 * (mt * 2 + rank) * p.catoms) + krow);
-                    tma_load_2d(smem + OFF_SFB + stage * SFB_STAGE, &tmSB, &sf_full[stage], 0,
-                                (int32_t)(2 * (nt * 2) * p.catoms) + krow);
-                    tma_load_2d(smem + OFF_SFB + stage * SFB_STAGE + 2048, &tmSB, &sf_full[stage], 0,
-                                (int32_t)(2 * (nt * 2 + 1) * p.catoms) + krow);
-                    issued[stage] = true;
-                    last_phase[stage] = phase;
-                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
-                }
-            }
-            // never leave a copy in flight into shared memory we are about to release
-            for (int s = 0; s < STAGES; ++s)
-                if (issued[s]) {
-                    mbar_wait(&sf_full[s], last_phase[s]);
-                    if (leader) mbar_wait(&full[s], last_phase[s]);
-                }
-        }
-    } else if (warp == 1) {
-        if (lane == 0 && leader) {
-            const uint32_t idesc0 = idesc_mxf4(2 * BM, BN, MX);
-            const uint32_t idesc_hi = idesc_with_sf_id(idesc0, 2, 2);
-            const uint64_t adesc0 = smem_desc(smem_u32(smem), 16, 1024, 2);
-            const uint64_t bdesc0 = smem_desc(smem_u32(smem + OFF_B), 16, 1024, 2);
-            int stage = 0;
-            uint32_t phase = 0, acc_phase = 0, kpar = 0, kcount = 0;
-            for (int64_t t = pair_id; t < tiles && !*abort_flag; t += npairs) {
-                if (!mbar_wait(tmem_empty, acc_phase ^ 1)) { *abort_flag = 1; break; }
-                tc_fence_after();
-                for (int kb = 0; kb < nkb; ++kb) {
-                    if (!mbar_wait(&full[stage], phase)) { *abort_flag = 1; break; }
-                    if (!mbar_wait(&sf_ready[kpar], (kcount / SF_NBUF) & 1)) { *abort_flag = 1; break; }
-                    tc_fence_after();
-                    const int64_t krem = p.K - (int64_t)kb * KB_ELEMS;
-                    const int nmma = krem < KB_ELEMS ? (int)(krem / 64) : 4;
-                    const uint64_t ad = adesc0 + (uint64_t)(stage * (A_STAGE >> 4));
-                    const uint64_t bd = bdesc0 + (uint64_t)(stage * (B_STAGE >> 4));
-                    const uint32_t sfa = tmem + SF_COL + kpar * SF_BUF;
-                    const uint32_t sfb = sfa + SFB_OFF;
-                    uint32_t accf = kb > 0 ? 1u : 0u;
-                    for (int kk = 0; kk < nmma; ++kk) {
-                        const int atom = MX ? kk / 2 : kk;
-                        if (MX)
-                            mma_mxf4_pair(tmem + ACC_COL, ad + 2 * kk, bd + 2 * kk, (kk & 1) ? idesc_hi : idesc0,
-                                          sfa + atom * 4, sfb + atom * 8, accf);
-                        else
-                            mma_nvf4_pair(tmem + ACC_COL, ad + 2 * kk, bd + 2 * kk, idesc0, sfa + atom * 4,
-                                          sfb + atom * 8, accf);
-                        accf = 1u;
-                    }
-                    tc_commit_pair_mc(&empty[stage], 0x3);
-                    tc_commit_pair_mc(&sf_free[kpar], 0x3);
-                    ++kcount;
-                    kpar = kcount % SF_NBUF;
-                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
-                }
-                if (*abort_flag) break;
-                tc_commit_pair_mc(tmem_full, 0x3);
-                acc_phase ^= 1;
-            }
-            tc_commit_pair(mma_done);
-            mbar_wait(mma_done, 0);
-        }
-    } else if (warp < FIRST_EPI_WARP) {
-        const uint32_t quarter = (uint32_t)(warp & 3) * 32u;
-        const uint32_t leader_sf_ready = mapa_shared(smem_u32(sf_ready), 0);
-        int stage = 0;
-        uint32_t phase = 0, kpar = 0, kcount = 0;
-        for (int64_t t = pair_id; t < tiles && !*abort_flag; t += npairs) {
-            for (int kb = 0; kb < nkb; ++kb) {
-                if (!mbar_wait(&sf_full[stage], phase)) { *abort_flag = 1; break; }
-                if (!mbar_wait(&sf_free[kpar], ((kcount / SF_NBUF) & 1) ^ 1)) { *abort_flag = 1; break; }
-                tc_fence_after();
-                const int64_t krem = p.K - (int64_t)kb * KB_ELEMS;
-                const int nmma = krem < KB_ELEMS ? (int)(krem / 64) : 4;
-                const int na = (nmma + mma_per_atom - 1) / mma_per_atom;
-                stage_scales(tmem + (quarter << 16) + SF_COL + kpar * SF_BUF, smem + OFF_SFA + stage * SFA_STAGE,
-                             smem + OFF_SFB + stage * SFB_STAGE, na, lane);
-                tmem_st_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(leader_sf_ready + 8u * kpar);
-                ++kcount;
-                kpar = kcount % SF_NBUF;
-                if (++stage == STAGES) { stage = 0; phase ^= 1; }
-            }
-        }
-    } else {
-        const int quad = warp & 3;
-        const int half = (warp - FIRST_EPI_WARP) >> 2;
-        const int order = warp - FIRST_EPI_WARP;
-        const float alpha = MX ? 1.0f : __fmul_rn(*p.a_gscale, *p.b_gscale);
-        const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + ACC_COL + half * 128;
-        const uint32_t leader_tmem_empty = mapa_shared(smem_u32(tmem_empty), 0);
-        const bool out_bf16 = p.out_bf16 != 0;
-        uint8_t* buf = smem + OFF_EPI;
-        uint32_t acc_phase = 0, iter = 0;
-        for (int64_t t = pair_id; t < tiles; t += npairs, ++iter) {
-            if (!mbar_wait(tmem_full, acc_phase)) { *abort_flag = 1; break; }
-            tc_fence_after();
-            const int64_t mt = t % tiles_m, nt = t / tiles_m;
-            const int64_t row0 = mt * 2 * BM + (int64_t)rank * BM + quad * 32;
-            const int64_t row = row0 + lane;
-            const int64_t col_base = nt * BN + half * 128;
-            uint32_t pk[2][32];
-#pragma unroll
-            for (int round = 0; round < 4; ++round) {
-                uint32_t r[32];
-                tmem_ld32(taddr + round * 32, r);
-                tmem_ld_wait();
-                if (round == 3) {
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive_cluster(leader_tmem_empty);
-                }
-                if (out_bf16) {
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[2 * j]) * alpha,
-                                                                 __uint_as_float(r[2 * j + 1]) * alpha);
-                        pk[round >> 1][(round & 1) * 16 + j] = *reinterpret_cast<uint32_t*>(&h);
-                    }
-                } else if (row < p.M) {
-                    store_row32(p.y, p.N, row, col_base + round * 32, r, alpha, false);
-                }
-            }
-            if (out_bf16) {
-                const bool first = order == 0;
-                if (!mbar_wait(&epi_turn[order], first ? ((iter & 1) ^ 1) : (iter & 1))) { *abort_flag = 1; break; }
-#pragma unroll
-                for (int b = 0; b < 2; ++b)
-#pragma unroll
-                    for (int c = 0; c < 8; ++c)
-                        *reinterpret_cast<uint4*>(buf + b * 4096 + lane * 128 + ((c ^ (lane & 7)) << 4)) =
-                            make_uint4(pk[b][4 * c], pk[b][4 * c + 1], pk[b][4 * c + 2], pk[b][4 * c + 3]);
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    tma_store_2d(&tmY, buf, (int32_t)col_base, (int32_t)row0);
-                    tma_store_2d(&tmY, buf + 4096, (int32_t)(col_base + 64), (int32_t)row0);
-                    bulk_commit_group();
-                    bulk_wait_read_all();
-                    mbar_arrive(&epi_turn[(order + 1) % EPI_WARPS]);
-                }
-                __syncwarp();
-            }
-            acc_phase ^= 1;
-        }
-        if (lane == 0) bulk_wait_all();
-    }
-
-    tc_fence_before();
-    __syncthreads();
-    cluster_sync();          // both CTAs are done with the pair's barriers and TMEM
-    tc_fence_after();
-    if (warp == 1) tmem_dealloc2(tmem, TMEM_COLS);
-    __syncthreads();
-    cluster_sync();
-}
-
-// The scale tensor (tensor-core layout) as rows of 256 bytes: a k-block's
-// atoms of one 128-row band are 2 * atoms_per_kb consecutive rows.
-static bool make_scale_map(CUtensorMap* map, const void* base, int64_t bytes, int box_rows) {
-    auto enc = tensor_map_encoder();
-    if (!enc || bytes % 256) return false;
-    cuuint64_t dims[2] = {256u, (cuuint64_t)(bytes / 256)};
-    cuuint64_t strides[1] = {256u};
-    cuuint32_t box[2] = {256u, (cuuint32_t)box_rows};
-    cuuint32_t es[2] = {1u, 1u};
-    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
-// CTA-pair kernel for M >= 256 (off: the 1-CTA kernel with register-staged
-// scales is faster on the shapes measured so far).
-constexpr bool kUsePairKernel = false;
-
-static cudaError_t launch_gemm_pair(const GemmParams& p, const GemmDev& d, cudaStream_t st, int num_sms) {
-    using namespace pair;
-    CUtensorMap ma, mb, msa, msb, my;
-    const int blk = p.mxfp4 ? 32 : 16;
-    const int box_rows = 2 * (p.mxfp4 ? 2 : 4);
-    const int64_t sa_bytes = ((p.M + 127) / 128) * 128 * d.catoms * 4;
-    const int64_t sb_bytes = ((p.N + 127) / 128) * 128 * d.catoms * 4;
-    (void)blk;
-    if (!make_code_map(&ma, p.a_codes, p.M, p.K / 2, BM)) return cudaErrorInvalidValue;
-    if (!make_code_map(&mb, p.b_codes, p.N, p.K / 2, BN / 2)) return cudaErrorInvalidValue;
-    if (!make_scale_map(&msa, p.a_scales, sa_bytes, box_rows)) return cudaErrorInvalidValue;
-    if (!make_scale_map(&msb, p.b_scales, sb_bytes, box_rows)) return cudaErrorInvalidValue;
-    std::memset(&my, 0, sizeof(my));
-    if (p.out_bf16 && !make_out_map(&my, p.y, p.M, p.N)) return cudaErrorInvalidValue;
-    const int64_t tiles = ((p.M + 2 * BM - 1) / (2 * BM)) * ((p.N + BN - 1) / BN);
-    int pairs = num_sms / 2;
-    if (tiles < pairs) pairs = (int)tiles;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * pairs, 1, 1);
-    cfg.blockDim = dim3(THREADS, 1, 1);
-    cfg.dynamicSmemBytes = SMEM_BYTES;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cudaError_t e;
-    if (p.mxfp4) {
-        e = cudaFuncSetAttribute(gemm_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel<true>, ma, mb, msa, msb, my, d);
-    } else {
-        e = cudaFuncSetAttribute(gemm_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel<false>, ma, mb, msa, msb, my, d);
-    }
-    if (e != cudaSuccess) return e;
-    return cudaGetLastError();
-}
-
 cudaError_t launch_gemm(const GemmParams& p, cudaStream_t st, int num_sms) {
     using namespace gemm;
     if (p.M == 0 || p.N == 0) return cudaSuccess;
@@ -815,7 +467,6 @@ cudaError_t launch_gemm(const GemmParams& p, cudaStream_t st, int num_sms) {
     const int blk = p.mxfp4 ? 32 : 16;
     d.catoms = ((p.K / blk) + 3) / 4;
     d.out_bf16 = p.out_bf16 ? 1 : 0;
-    if (kUsePairKernel && p.M >= 2 * BM && num_sms >= 2) return launch_gemm_pair(p, d, st, num_sms);
     const int64_t tiles = ((p.M + BM - 1) / BM) * ((p.N + BN - 1) / BN);
     const int grid = (int)(tiles < num_sms ? tiles : num_sms);
     cudaError_t e;
