@@ -66,10 +66,27 @@ def peaks():
 
 
 # dram__bytes_read.sum + dram__bytes_write.sum of one launch of the roofline
-# kernel (gemm_kernel<NVFP4>, 8192 x 17408 x 5120) from one ncu capture of
-# the bench's own prefill step; to be re-taken (or set to None) whenever that
-# kernel changes
-GEMM_TRAFFIC_BYTES = 321.1e6
+# kernel (gemm_kernel<NVFP4>, 8192 x 17408 x 5120) from one ncu capture, with
+# the SHA-256 (first 16 hex digits) of the GEMM source file it was built from:
+# the bench reports the figure only while that file is unchanged.
+GEMM_TRAFFIC = {"bytes": None, "source_sha256_16": None}
+GEMM_SOURCE = ROOT / "mxfp4_w4a4_block_b200" / "csrc" / "q4_gemm.cu"
+
+
+def gemm_source_hash() -> str:
+    import hashlib
+    return hashlib.sha256(GEMM_SOURCE.read_bytes()).hexdigest()[:16]
+
+
+def roofline_traffic(override):
+    """(bytes or None, note): the captured DRAM traffic of the roofline kernel,
+    None once the GEMM source differs from the one the capture was made of."""
+    if override is not None:
+        return override, "given on the command line"
+    cur = gemm_source_hash()
+    if GEMM_TRAFFIC["bytes"] is not None and GEMM_TRAFFIC["source_sha256_16"] == cur:
+        return GEMM_TRAFFIC["bytes"], f"ncu capture of the kernel built from q4_gemm.cu sha256 {cur}"
+    return None, f"no capture of the current kernel (q4_gemm.cu sha256 {cur})"
 
 # dense FP4 over dense bf16 on B200, nominal (9 / 2.25 PFLOP/s)
 FP4_OVER_BF16 = 4.0
@@ -590,6 +607,7 @@ def run_ours(args):
         rows["gemm_prefill_n17408"] = {"us": k_ms[2] * 1e3, "TFLOP/s": gemm2_tf, "frac_fp4": gemm2_tf / fp4_burst}
 
     cpu = None if args.no_cpu_baseline or rank != 0 else cpu_baseline(budget_s=args.cpu_seconds)
+    traffic, traffic_note = roofline_traffic(args.traffic)
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -602,7 +620,8 @@ def run_ours(args):
                      "peak": fp4_burst, "unit": "TFLOP/s", "frac": gemm2_tf / fp4_burst,
                      "peak_note": f"dense FP4 = {pk['src']} bf16 burst {pk['bf16']} x 4 (nominal 9/2.25)",
                      "frac_vs_sustained": gemm2_tf / (pk["bf16_sus"] * FP4_OVER_BF16),
-                     "traffic": args.traffic},
+                     "traffic": traffic, "traffic_note": traffic_note,
+                     "algorithmic_bytes": M * K / 2 + M * K / 16 + N2 * K / 2 + N2 * K / 16 + 2 * M * N2},
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": Prefill.LAUNCHES_PER_STEP * args.steps,
@@ -779,6 +798,81 @@ def run_reference(args):
     }))
 
 
+PROFILE_ROWS = ("mxfp4_quantize", "amax_quantize", "nvfp4_quantize", "gemm_n5120", "gemm_n17408", "decode",
+                "sigma_delta_visit", "sd_gemm_m16", "w4a16_4096")
+
+
+def run_profile(row: str, launches: int):
+    """Launch one row's kernel `launches` times on its workload, untimed: the
+    program a profiler capture of that kernel runs."""
+    import mxfp4_w4a4_block_b200 as q4
+    dev = torch.device("cuda", 0)
+    if row == "mxfp4_quantize":
+        d = synth.mxfp4(n=256)
+        x, t = d["x"].to(dev), torch.from_numpy(d["t"]).to(dev)
+        c = torch.empty((4096, 2048), dtype=torch.uint8, device=dev)
+        sc = torch.empty(q4.q4_scale_bytes(q4.MXFP4, 4096, 4096), dtype=torch.uint8, device=dev)
+        fn = lambda: q4.q4_quantize(q4.MXFP4, x, chan=t, flags=q4.LAYOUT_TC | q4.HADAMARD32, codes=c, scales=sc)
+    elif row in ("amax_quantize", "nvfp4_quantize", "gemm_n5120", "gemm_n17408"):
+        n_list = {"gemm_n5120": (N1,), "gemm_n17408": (N2,)}.get(row, ())
+        d = synth.prefill(n_list=n_list)
+        x = d["x"].to(dev)
+        out = torch.zeros(4, dtype=torch.float32, device=dev)
+        c = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+        sc = torch.empty(q4.q4_scale_bytes(q4.NVFP4, M, K), dtype=torch.uint8, device=dev)
+        q4.q4_amax_quantize(x, 2688.0, out=out, codes=c, scales=sc)
+        if row == "amax_quantize":
+            fn = lambda: q4.q4_amax_quantize(x, 2688.0, out=out, codes=c, scales=sc)
+        elif row == "nvfp4_quantize":
+            fn = lambda: q4.q4_quantize(q4.NVFP4, x, gscale=out[1:2], codes=c, scales=sc)
+        else:
+            w = torch.from_numpy(d["w"][0]).to(dev)
+            g = q4.q4_amax(w, 2688.0)[1:2].clone()
+            wc, ws = q4.q4_quantize(q4.NVFP4, w, gscale=g)
+            del w
+            n = n_list[0]
+            y = torch.empty((M, n), dtype=torch.bfloat16, device=dev)
+            fn = lambda: q4.q4_gemm(q4.NVFP4, M, n, K, c, sc, out[1:2], wc, ws, g, y=y)
+    elif row == "decode":
+        dd = synth.decode()
+        xd = dd["x"].to(dev)
+        wt = torch.from_numpy(dd["w"]).to(dev)
+        gw = q4.q4_amax(wt, 2688.0)[1:2].clone()
+        wc, ws = q4.q4_quantize(q4.NVFP4, wt, gscale=gw)
+        del wt
+        gx = q4.q4_amax(xd, 2688.0)[1:2].clone()
+        yd = torch.empty((16, 17408), dtype=torch.bfloat16, device=dev)
+        fn = lambda: q4.q4_gemm(q4.NVFP4, 16, 17408, 5120, xd, None, gx, wc, ws, gw, y=yd, a_kind=q4.A_BF16)
+    else:
+        dl = synth.looped()
+        xl = dl["x"].to(dev)
+        mats = []
+        for w in dl["w"]:
+            wt = torch.from_numpy(w).to(dev)
+            g = q4.q4_amax(wt, 1536.0)[1:2].clone()
+            _, scl = q4.q4_quantize(q4.NVFP4, wt, gscale=g, flags=q4.SCALE_RU | q4.LAYOUT_TC)
+            mats.append((wt, scl, g, torch.zeros_like(wt),
+                         torch.empty((w.shape[0], w.shape[1] // 2), dtype=torch.uint8, device=dev)))
+        gW, gS, gG, gR, gC = ([m[i] for m in mats] for i in range(5))
+        if row == "sigma_delta_visit":
+            fn = lambda: q4.q4_sigma_delta_step_grouped(q4.NVFP4, gW, gS, gR, gscales=gG, codes=gC)
+        elif row == "sd_gemm_m16":
+            x16 = xl[:16].contiguous()
+            ys = [torch.empty((16, w.shape[0]), dtype=torch.bfloat16, device=dev) for w in gW]
+            fn = lambda: q4.q4_sigma_delta_gemm_grouped(q4.NVFP4, [x16] * len(gW), gW, gS, gR, gG, ys=ys)
+        else:
+            wt, scl, g, _, c = mats[4]                           # a 4096 x 1024 looped-core weight
+            q4.q4_sigma_delta_step(q4.NVFP4, wt, scl, torch.zeros_like(wt), gscale=g, codes=c)
+            y = torch.empty((xl.shape[0], wt.shape[0]), dtype=torch.bfloat16, device=dev)
+            fn = lambda: q4.q4_gemm(q4.NVFP4, xl.shape[0], wt.shape[0], xl.shape[1], xl, None, None, c, scl, g, y=y,
+                                    a_kind=q4.A_BF16_W4A16)
+    torch.cuda.synchronize()
+    for _ in range(launches):
+        fn()
+    torch.cuda.synchronize()
+    print(f"profiled row {row}: {launches} launches")
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -794,9 +888,15 @@ def main():
     ap.add_argument("--rows-reps", type=int, default=30,
                     help="timed calls per kernel row (small values for profiler captures)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--traffic", type=float, default=GEMM_TRAFFIC_BYTES,
-                    help="DRAM bytes per launch of the roofline kernel from an ncu capture")
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="DRAM bytes per launch of the roofline kernel from an ncu capture (overrides the stored one)")
+    ap.add_argument("--profile", choices=PROFILE_ROWS, default=None,
+                    help="only launch this row's kernel --profile-launches times, untimed (for profiler captures)")
+    ap.add_argument("--profile-launches", type=int, default=4)
     args = ap.parse_args()
+    if args.profile:
+        run_profile(args.profile, args.profile_launches)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

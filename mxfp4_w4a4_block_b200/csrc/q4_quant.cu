@@ -304,39 +304,6 @@ __device__ __forceinline__ void mx_block(const float (&v)[32], const float4 (&cw
     }
 }
 
-// Largest |x| of the rows x cols tensor (row pitch ld elements) over this
-// thread's share: warp w of the grid takes rows w, w + warps, ..., its lanes
-// 16-byte chunks lane, lane + 32, ... of each row, four loads in flight.
-template <bool BF16>
-__device__ __forceinline__ float amax_share(const QuantParams& p, int gwarp, int nwarps, int lane) {
-    constexpr int ESZ = BF16 ? 2 : 4;
-    const int64_t cpr = p.cols * ESZ / 16;
-    float m = 0.0f;
-    auto fold = [&](const uint4& w) {
-        if (BF16) {
-            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) m = fmaxf(m, fmaxf(fabsf(bf16_lo(ws[j])), fabsf(bf16_hi(ws[j]))));
-        } else {
-            m = fmaxf(m, fmaxf(fmaxf(fabsf(__uint_as_float(w.x)), fabsf(__uint_as_float(w.y))),
-                               fmaxf(fabsf(__uint_as_float(w.z)), fabsf(__uint_as_float(w.w)))));
-        }
-    };
-    for (int64_t row = gwarp; row < p.rows; row += nwarps) {
-        const uint4* rp = reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(p.x) + row * p.ld * ESZ);
-        int64_t c = lane;
-        for (; c + 96 < cpr; c += 128) {
-            uint4 w[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) w[u] = __ldg(rp + c + 32 * u);
-#pragma unroll
-            for (int u = 0; u < 4; ++u) fold(w[u]);
-        }
-        for (; c < cpr; c += 32) fold(__ldg(rp + c));
-    }
-    return m;
-}
-
 template <int BLK, bool BF16, bool TC, bool RU, bool HAD, bool CHAN, bool S46 = false, bool AMAX = false>
 __global__ void __launch_bounds__(qz::THREADS, 1)
     quantize_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmC, QuantParams p,
@@ -367,52 +334,16 @@ __global__ void __launch_bounds__(qz::THREADS, 1)
     }
     __syncthreads();
 
-    // With AMAX, the tensor scale comes first: every thread of the grid folds
-    // its share of |x| into a maximum, each CTA adds its maximum to out[0]
-    // (non-negative floats order like their bit patterns) and arrives on
-    // out[2]; once all CTAs have arrived (a bounded wait: the launch is
-    // cooperative, so they are all resident) each computes s_t = amax / denom
-    // itself, and CTA 0 stores it in out[1].  The quantization below then reads
-    // X a second time, mostly from L2.
-    float s_t_dyn = 0.0f;
-    if constexpr (AMAX) {
-        __shared__ float red[qz::THREADS / 32];
-        __shared__ float s_shared;
-        __shared__ int go;
-        float m = amax_share<BF16>(p, blockIdx.x * (qz::THREADS / 32) + warp, gridDim.x * (qz::THREADS / 32), lane);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        if (lane == 0) red[warp] = m;
-        __syncthreads();
-        if (tid == 0) {
-            float b = 0.0f;
-            for (int w = 0; w < qz::THREADS / 32; ++w) b = fmaxf(b, red[w]);
-            atomicMax(p.amax_out, __float_as_uint(b));
-            __threadfence();
-            atomicAdd(p.amax_out + 2, 1u);
-            bool ok = true;
-            const long long t0 = clock64(), limit = g_wait_limit;
-            while (ld_acquire_gpu(p.amax_out + 2) < gridDim.x) {
-                if (clock64() - t0 > limit) {
-                    atomicOr(&g_device_error, kErrTimeout);
-                    ok = false;
-                    break;
-                }
-            }
-            if (ok) {
-                const float amax = __uint_as_float(ld_acquire_gpu(p.amax_out));
-                s_shared = __fdiv_rn(amax, p.denom);
-                if (blockIdx.x == 0) reinterpret_cast<float*>(p.amax_out)[1] = s_shared;
-            }
-            go = ok ? 1 : 0;
-        }
-        __syncthreads();
-        if (!go) return;                  // nothing issued yet: the whole CTA leaves
-        s_t_dyn = s_shared;
-    }
-
     const int64_t tiles_c = p.catoms;
     const int64_t tiles = ((p.rows + G::ROWS - 1) / G::ROWS) * tiles_c;
+    // This CTA's tiles are blockIdx.x + i * gridDim.x, i < n_my.  With AMAX the
+    // launch makes two passes over them: the first only folds |x| into the
+    // tensor maximum, the second quantizes, in reverse order, so that the tiles
+    // read last (the likeliest to be still in L2) come first.
+    const int64_t n_my = tiles > blockIdx.x ? (tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    auto quant_tile = [&](int64_t i) -> int64_t {
+        return (int64_t)blockIdx.x + (AMAX ? (n_my - 1 - i) : i) * (int64_t)gridDim.x;
+    };
 
     if (warp == CONSUMER_WARPS) {
         // ---- producer
@@ -423,12 +354,17 @@ __global__ void __launch_bounds__(qz::THREADS, 1)
             uint32_t last_phase[G::NSTAGE];
             bool issued[G::NSTAGE];
             for (int s = 0; s < G::NSTAGE; ++s) issued[s] = false, last_phase[s] = 0;
-            for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
+            // the loads need no tensor scale, so with AMAX they run straight on
+            // from the first pass into the second while the grid meets
+            const int64_t iters = (AMAX ? 2 : 1) * n_my;
+            for (int64_t it = 0; it < iters; ++it) {
+                const int64_t t = (AMAX && it < n_my) ? (int64_t)blockIdx.x + it * (int64_t)gridDim.x
+                                                      : quant_tile(AMAX ? it - n_my : it);
                 // on time-out stop issuing: the consumers then time out on `full`
                 if (!mbar_wait(&empty[stage], phase ^ 1)) break;
                 // failure-detection test (Q4_INJECT_STALL): the first tile's stage
                 // is never filled, so the consumers' bounded wait on it runs out
-                if (!(p.inject_stall && t == (int64_t)blockIdx.x)) {
+                if (!(p.inject_stall && it == 0)) {
                     mbar_arrive_expect_tx(&full[stage], G::STAGE);
                     const int64_t tr = t / tiles_c, tc = t % tiles_c;
                     uint8_t* dst = smem + stage * G::STAGE;
@@ -454,7 +390,8 @@ __global__ void __launch_bounds__(qz::THREADS, 1)
             const int64_t bands = (p.rows + 127) / 128;
             int buf = 0;
             uint32_t bphase = 0;
-            for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
+            for (int64_t i = 0; i < n_my; ++i) {
+                const int64_t t = quant_tile(i);
                 // on time-out stop: nothing of this tile is complete
                 if (!mbar_wait(&cfull[buf], bphase)) break;
                 const int64_t tr = t / tiles_c, tc = t % tiles_c;
@@ -481,6 +418,108 @@ __global__ void __launch_bounds__(qz::THREADS, 1)
     }
 
     // ---- consumers
+    int stage = 0, buf = 0;
+    uint32_t phase = 0, bphase = 0;
+    // this thread's BPT blocks of a landed stage: the raw 16-byte chunks
+    // (shared-memory loads), then as floats
+    using Raw = uint4[G::BPT][G::CHUNKS];
+    auto load_raw = [&](const uint8_t* sb, Raw& raw) {
+#pragma unroll
+        for (int k = 0; k < G::BPT; ++k) {
+            const int b = tid + k * CONSUMERS;
+            const int j = b / G::ROWS, r = b % G::ROWS;
+            const int jo = j * BLK * G::ESZ;
+            const uint8_t* rowp = sb + (jo >> 7) * (G::ROWS * 128) + r * 128;
+            const int o16 = (jo & 127) >> 4;
+#pragma unroll
+            for (int c = 0; c < G::CHUNKS; ++c)
+                raw[k][c] = *reinterpret_cast<const uint4*>(rowp + (((o16 + c) ^ (r & 7)) << 4));
+        }
+    };
+    auto unpack = [&](const Raw& raw, float (&v)[G::BPT][BLK]) {
+#pragma unroll
+        for (int k = 0; k < G::BPT; ++k)
+#pragma unroll
+            for (int c = 0; c < G::CHUNKS; ++c) {
+                const uint4 w = raw[k][c];
+                float* d = &v[k][c * G::PER];
+                if (BF16) {
+                    d[0] = bf16_lo(w.x); d[1] = bf16_hi(w.x); d[2] = bf16_lo(w.y); d[3] = bf16_hi(w.y);
+                    d[4] = bf16_lo(w.z); d[5] = bf16_hi(w.z); d[6] = bf16_lo(w.w); d[7] = bf16_hi(w.w);
+                } else {
+                    d[0] = __uint_as_float(w.x); d[1] = __uint_as_float(w.y);
+                    d[2] = __uint_as_float(w.z); d[3] = __uint_as_float(w.w);
+                }
+            }
+    };
+    auto read_blocks = [&](const uint8_t* sb, float (&v)[G::BPT][BLK]) {
+        Raw raw;
+        load_raw(sb, raw);
+        unpack(raw, v);
+    };
+
+    // With AMAX the tensor scale comes first: the first pass folds every
+    // landed tile's |x| into this thread's maximum (zero-filled parts outside
+    // the tensor add nothing), each CTA adds its maximum to out[0] (non-negative
+    // floats order like their bit patterns) and arrives on out[2]; once all
+    // CTAs have arrived (a bounded wait: the launch is cooperative, so all are
+    // resident) each computes s_t = amax / denom itself and CTA 0 stores it in
+    // out[1].  The producer keeps the ring full meanwhile.
+    float s_t_dyn = 0.0f;
+    if constexpr (AMAX) {
+        __shared__ float red[CONSUMER_WARPS];
+        __shared__ float s_shared;
+        __shared__ int go;
+        float m = 0.0f;
+        bool ok = true;
+        for (int64_t i = 0; i < n_my; ++i) {
+            if (!mbar_wait(&full[stage], phase)) { ok = false; break; }
+            float v[G::BPT][BLK];
+            read_blocks(smem + stage * G::STAGE, v);
+#pragma unroll
+            for (int k = 0; k < G::BPT; ++k) m = fmaxf(m, amax_tree<BLK>(v[k]));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[stage]);
+            if (++stage == G::NSTAGE) { stage = 0; phase ^= 1; }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (lane == 0) red[warp] = ok ? m : -1.0f;
+        named_barrier(1, CONSUMERS);
+        if (tid == 0) {
+            float b = 0.0f;
+            bool all = true;
+            for (int w = 0; w < CONSUMER_WARPS; ++w) {
+                all = all && red[w] >= 0.0f;
+                b = fmaxf(b, red[w]);
+            }
+            if (all) {
+                atomicMax(p.amax_out, __float_as_uint(b));
+                __threadfence();
+                atomicAdd(p.amax_out + 2, 1u);
+                const long long t0 = clock64(), limit = g_wait_limit;
+                while (ld_acquire_gpu(p.amax_out + 2) < gridDim.x) {
+                    if (clock64() - t0 > limit) {
+                        atomicOr(&g_device_error, kErrTimeout);
+                        all = false;
+                        break;
+                    }
+                }
+            }
+            if (all) {
+                const float amax = __uint_as_float(ld_acquire_gpu(p.amax_out));
+                s_shared = __fdiv_rn(amax, p.denom);
+                if (blockIdx.x == 0) reinterpret_cast<float*>(p.amax_out)[1] = s_shared;
+            }
+            go = all ? 1 : 0;
+        }
+        named_barrier(1, CONSUMERS);
+        // without a tensor scale the consumers stop; the producer and the store
+        // warp then run out their bounded waits and leave
+        if (!go) return;
+        s_t_dyn = s_shared;
+    }
+
     NvCtx sc;
     if constexpr (BLK == 16) {
         const float s_t = AMAX ? s_t_dyn : *p.gscale;
@@ -489,11 +528,12 @@ __global__ void __launch_bounds__(qz::THREADS, 1)
         named_barrier(1, CONSUMERS);
     }
     const int64_t crow = p.cols / 2;           // bytes of codes per row
-    int stage = 0, buf = 0;
-    uint32_t phase = 0, bphase = 0;
+    Raw raw;
+    bool have_next = false;                    // raw holds the next tile's chunks already
     // a consumer warp whose wait times out stops; every other role then
     // times out in turn on the barriers that warp no longer arrives on
-    for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
+    for (int64_t i = 0; i < n_my; ++i) {
+        const int64_t t = quant_tile(i);
         const int64_t tr = t / tiles_c, tc = t % tiles_c;
         const int64_t row0 = tr * G::ROWS, col0 = tc * 4 * BLK;
         // MXFP4 channel factors of this thread's blocks (1 outside the
@@ -512,35 +552,23 @@ __global__ void __launch_bounds__(qz::THREADS, 1)
                     cw[k][q] = col < p.cols ? __ldg(cp + q) : make_float4(1.0f, 1.0f, 1.0f, 1.0f);
             }
         }
-        if (!mbar_wait(&full[stage], phase)) break;
-
-        float v[G::BPT][BLK];
-        const uint8_t* sb = smem + stage * G::STAGE;
-#pragma unroll
-        for (int k = 0; k < G::BPT; ++k) {
-            const int b = tid + k * CONSUMERS;
-            const int j = b / G::ROWS, r = b % G::ROWS;
-            const int jo = j * BLK * G::ESZ;
-            const uint8_t* rowp = sb + (jo >> 7) * (G::ROWS * 128) + r * 128;
-            const int o16 = (jo & 127) >> 4;
-#pragma unroll
-            for (int c = 0; c < G::CHUNKS; ++c) {
-                const uint4 raw = *reinterpret_cast<const uint4*>(rowp + (((o16 + c) ^ (r & 7)) << 4));
-                float* d = &v[k][c * G::PER];
-                if (BF16) {
-                    d[0] = bf16_lo(raw.x); d[1] = bf16_hi(raw.x); d[2] = bf16_lo(raw.y); d[3] = bf16_hi(raw.y);
-                    d[4] = bf16_lo(raw.z); d[5] = bf16_hi(raw.z); d[6] = bf16_lo(raw.w); d[7] = bf16_hi(raw.w);
-                } else {
-                    d[0] = __uint_as_float(raw.x); d[1] = __uint_as_float(raw.y);
-                    d[2] = __uint_as_float(raw.z); d[3] = __uint_as_float(raw.w);
-                }
-            }
+        if (!have_next) {
+            if (!mbar_wait(&full[stage], phase)) break;
+            load_raw(smem + stage * G::STAGE, raw);
         }
+        float v[G::BPT][BLK];
+        unpack(raw, v);
         // the stage is handed back only once its values have been used (below):
         // a lane's shared-memory loads may still be in flight after __syncwarp,
         // and the refill must not overtake them
         const int read_stage = stage;
         if (++stage == G::NSTAGE) { stage = 0; phase ^= 1; }
+        // the next tile's loads go out before this tile's arithmetic when its
+        // stage has already landed, so their latency hides behind the work
+        // (where a thread's chunks fit in 16 registers, so nothing spills)
+        constexpr bool PREFETCH = G::BPT * G::CHUNKS <= 4 && !S46;
+        have_next = PREFETCH && i + 1 < n_my && mbar_test_wait(&full[stage], phase);
+        if (have_next) load_raw(smem + stage * G::STAGE, raw);
         if (!mbar_wait(&cfree[buf], bphase ^ 1)) break;
 
         uint8_t* cb = cbuf + buf * G::CODE_TILE;
