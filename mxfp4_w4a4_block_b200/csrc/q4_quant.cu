@@ -528,8 +528,6 @@ __global__ void __launch_bounds__(qz::THREADS, 1)
         named_barrier(1, CONSUMERS);
     }
     const int64_t crow = p.cols / 2;           // bytes of codes per row
-    Raw raw;
-    bool have_next = false;                    // raw holds the next tile's chunks already
     // a consumer warp whose wait times out stops; every other role then
     // times out in turn on the barriers that warp no longer arrives on
     for (int64_t i = 0; i < n_my; ++i) {
@@ -552,23 +550,14 @@ __global__ void __launch_bounds__(qz::THREADS, 1)
                     cw[k][q] = col < p.cols ? __ldg(cp + q) : make_float4(1.0f, 1.0f, 1.0f, 1.0f);
             }
         }
-        if (!have_next) {
-            if (!mbar_wait(&full[stage], phase)) break;
-            load_raw(smem + stage * G::STAGE, raw);
-        }
+        if (!mbar_wait(&full[stage], phase)) break;
         float v[G::BPT][BLK];
-        unpack(raw, v);
+        read_blocks(smem + stage * G::STAGE, v);
         // the stage is handed back only once its values have been used (below):
         // a lane's shared-memory loads may still be in flight after __syncwarp,
         // and the refill must not overtake them
         const int read_stage = stage;
         if (++stage == G::NSTAGE) { stage = 0; phase ^= 1; }
-        // the next tile's loads go out before this tile's arithmetic when its
-        // stage has already landed, so their latency hides behind the work
-        // (where a thread's chunks fit in 16 registers, so nothing spills)
-        constexpr bool PREFETCH = G::BPT * G::CHUNKS <= 4 && !S46;
-        have_next = PREFETCH && i + 1 < n_my && mbar_test_wait(&full[stage], phase);
-        if (have_next) load_raw(smem + stage * G::STAGE, raw);
         if (!mbar_wait(&cfree[buf], bphase ^ 1)) break;
 
         uint8_t* cb = cbuf + buf * G::CODE_TILE;
