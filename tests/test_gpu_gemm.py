@@ -114,12 +114,14 @@ def test_fused_activation_quant_decode_small(M, K):
         check(y, oracle_gemm(A, B), od)
 
 
-@pytest.mark.parametrize("M,K,many_tiles", [(3, 320, True), (16, 8256, False)])
+@pytest.mark.parametrize("M,K,many_tiles", [(3, 320, True), (16, 8256, False), (16, 16384, False),
+                                             (16, 20480, False)])
 def test_fused_decode_more_tiles_than_sms_and_long_k(M, K, many_tiles):
     """Fused decode with more 128-row weight tiles than SMs (CTAs take a second
-    tile and quantize the activations again for it), and with 33 k-blocks
-    (K = 8256, the activation ring wraps several times); called twice with new
-    activations on the second call."""
+    tile and reuse their resident quantized activations for it), with 33 and 64
+    k-blocks (K = 16384: the resident activations leave room for 3 weight stages),
+    and K = 20480, past what fits, which takes the quantize-once workspace path;
+    called twice with new activations on the second call."""
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     N = (sms + 4) * 128 + 64 if many_tiles else 392
     w = synth.small_like("weight", 6, N, K)
