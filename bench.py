@@ -3,7 +3,8 @@
 One step = one pass of the prefill-shaped W4A4 linear over one batch:
     tensor amax of X (8192 x 5120 bf16, heavy-tailed) -> s_t,
     then NVFP4 quantize of X (codes + tensor-core scales),  one launch
-    W4A4 GEMM with W1 (5120 x 5120) and W2 (17408 x 5120)  (the GEMM TFLOP/s)
+    W4A4 GEMM of X with W1 (5120 x 5120) and W2 (17408 x 5120),
+    both weights in one launch                             (the GEMM TFLOP/s)
 with the weights quantized once beforehand and resident in HBM.  `value` is
 the GEMM FLOPs of the step divided by the step's device time.  The other
 rows of the path are timed on their own workloads under "rows": MXFP4
@@ -181,17 +182,19 @@ class Prefill:
         self.y = [torch.empty((M, n), dtype=torch.bfloat16, device=dev) for n, *_ in self.w]
         torch.cuda.synchronize()
 
-    def step(self, ev=None):
+    def step(self, ev=None, x=None, y=None):
         q4 = self.q4
+        x = self.x if x is None else x
+        y = self.y if y is None else y
         if ev is not None:
             ev[0].record()
-        q4.q4_amax_quantize(self.x, 2688.0, out=self.amax, codes=self.xc, scales=self.xs)
+        q4.q4_amax_quantize(x, 2688.0, out=self.amax, codes=self.xc, scales=self.xs)
         if ev is not None:
             ev[1].record()
-        for i, (n, wc, ws, wg) in enumerate(self.w):
-            q4.q4_gemm(q4.NVFP4, M, n, K, self.xc, self.xs, self.amax[1:2], wc, ws, wg, y=self.y[i])
-            if ev is not None:
-                ev[2 + i].record()
+        q4.q4_gemm_shared_a(q4.NVFP4, M, K, self.xc, self.xs, self.amax[1:2],
+                            [(wc, ws, wg, n) for n, wc, ws, wg in self.w], ys=y)
+        if ev is not None:
+            ev[2].record()
 
     def two_launch_quantize(self):
         """The same activation quantize as q4_amax then q4_quantize (for comparison)."""
@@ -199,8 +202,52 @@ class Prefill:
         q4.q4_amax(self.x, 2688.0, out=self.amax)
         q4.q4_quantize(q4.NVFP4, self.x, gscale=self.amax[1:2], codes=self.xc, scales=self.xs)
 
-    LAUNCHES_PER_STEP = 3   # amax + quantize (one cooperative launch), two GEMMs
-    SEGMENTS = 3
+    LAUNCHES_PER_STEP = 2   # amax + quantize (one cooperative launch), the two GEMMs (one launch)
+    SEGMENTS = 2
+
+
+def e2e_pipelined(P, steps: int):
+    """End to end through the public API with the host copies pipelined: every
+    step uploads its X from pinned host memory and reads both Y back to pinned
+    host memory, on three streams -- uploads, compute, downloads -- with the
+    device X and Y double-buffered, so the next step's upload and this step's
+    downloads overlap the compute.
+    Returns ms per step (device time from the first upload to the last download)."""
+    xh = P.x_host.pin_memory()
+    yh = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for y in P.y]
+    xd = [P.x, torch.empty_like(P.x)]
+    yd = [P.y, [torch.empty_like(y) for y in P.y]]
+    s_up, s_cmp, s_down = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    E = lambda: torch.cuda.Event()
+    up_done, cmp_done, down_done = [E(), E()], [E(), E()], [E(), E()]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    cur = torch.cuda.current_stream()
+    torch.cuda.synchronize()
+    start.record(cur)
+    for st in (s_up, s_cmp, s_down):
+        st.wait_stream(cur)
+    for i in range(steps):
+        b = i % 2
+        with torch.cuda.stream(s_up):
+            if i >= 2:
+                s_up.wait_event(cmp_done[b])          # step i - 2 has read X[b]
+            xd[b].copy_(xh, non_blocking=True)
+            up_done[b].record(s_up)
+        with torch.cuda.stream(s_cmp):
+            s_cmp.wait_event(up_done[b])
+            if i >= 2:
+                s_cmp.wait_event(down_done[b])        # step i - 2's results have left Y[b]
+            P.step(ev=[E(), E(), cmp_done[b]], x=xd[b], y=yd[b])
+        with torch.cuda.stream(s_down):
+            s_down.wait_event(cmp_done[b])
+            yh[0].copy_(yd[b][0], non_blocking=True)
+            yh[1].copy_(yd[b][1], non_blocking=True)
+            down_done[b].record(s_down)
+    for st in (s_up, s_cmp, s_down):
+        cur.wait_stream(st)
+    end.record(cur)
+    end.synchronize()
+    return start.elapsed_time(end) / steps
 
 
 def time_fn(fn, reps, flush, warm=3):
@@ -546,9 +593,8 @@ def run_ours(args):
                     for i in range(args.steps)])
     step_ms = max_over_ranks(float(seg.sum(axis=1).mean()), dist, dev)
     clocks = cs.summary()
-    k_ms = seg.mean(axis=0)          # amax + quantize, gemm1, gemm2
-    gemm2_tf = 2.0 * M * N2 * K / (k_ms[2] * 1e-3) / 1e12
-    gemm1_tf = 2.0 * M * N1 * K / (k_ms[1] * 1e-3) / 1e12
+    k_ms = seg.mean(axis=0)          # amax + quantize, the shared-A GEMM launch
+    gemm_tf = GEMM_FLOPS / (k_ms[1] * 1e-3) / 1e12
     # the fused launch reads X from HBM once (the second pass mostly hits L2):
     # its algorithmic bytes are those of the quantize alone
     q_gbs = M * K * B_QUANT_BF16 / (k_ms[0] * 1e-3) / 1e9
@@ -573,10 +619,21 @@ def run_ours(args):
             e.synchronize()
             if i >= 2:
                 ts.append(s.elapsed_time(e))
-        e2e_ms = max_over_ranks(statistics.mean(ts), dist, dev)
+        serial_ms = max_over_ranks(statistics.mean(ts), dist, dev)
+        pipe_err = None
+        try:
+            e2e_pipelined(P, 2)                              # warm-up of the streams and buffers
+            pipe_ms = e2e_pipelined(P, max(4, args.e2e_steps))
+        except Exception as ex:                              # report it; the serial figure stands
+            pipe_err, pipe_ms = str(ex)[:200], serial_ms
+        e2e_ms = max_over_ranks(pipe_ms, dist, dev)
         e2e = {"value": whole_job_tflops(world, GEMM_FLOPS, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": int(P.x_host.numel() * 2),
-               "d2h_bytes_per_step": int(sum(y.numel() * 2 for y in P.y)), "ms_per_step": e2e_ms}
+               "d2h_bytes_per_step": int(sum(y.numel() * 2 for y in P.y)), "ms_per_step": e2e_ms,
+               "note": ("copies pipelined over steps on three streams (uploads, compute, downloads)"
+                        if pipe_err is None else "pipelined run failed (" + pipe_err + "); serial figure"),
+               "serial": {"value": whole_job_tflops(world, GEMM_FLOPS, serial_ms), "ms_per_step": serial_ms,
+                          "note": "upload, step, downloads back to back, L2 flushed before each step"}}
 
     rows = None
     if not args.no_rows:
@@ -591,9 +648,7 @@ def run_ours(args):
         fused_ms, _ = time_fn(lambda: q4.q4_amax_quantize(P.x, 2688.0, out=P.amax, codes=P.xc, scales=P.xs), 30,
                               flush)
         a_gbs = M * K * B_AMAX_BF16 / (am_ms * 1e-3) / 1e9
-        del P
-        torch.cuda.empty_cache()
-        rows = rows_bench(q4, dev, flush, pk, reps=args.rows_reps)
+        rows = {}
         rows["amax_quantize_prefill_x"] = {"shape": [M, K], "us": k_ms[0] * 1e3, "GB/s": q_gbs,
                                            "frac_hbm": q_gbs / hbm, "B_per_element": B_QUANT_BF16,
                                            "note": "in the step: one cooperative launch, amax then quantize"}
@@ -603,8 +658,19 @@ def run_ours(args):
                                                 "speedup_vs_two_launches": two_ms / fused_ms}
         rows["nvfp4_quantize_prefill_x_cold"] = iso_quant
         rows["amax_prefill_x_cold"] = {"us": am_ms * 1e3, "GB/s": a_gbs, "frac_hbm": a_gbs / hbm}
-        rows["gemm_prefill_n5120"] = {"us": k_ms[1] * 1e3, "TFLOP/s": gemm1_tf, "frac_fp4": gemm1_tf / fp4_burst}
-        rows["gemm_prefill_n17408"] = {"us": k_ms[2] * 1e3, "TFLOP/s": gemm2_tf, "frac_fp4": gemm2_tf / fp4_burst}
+        rows["gemm_prefill_shared_a"] = {"us": k_ms[1] * 1e3, "TFLOP/s": gemm_tf, "frac_fp4": gemm_tf / fp4_burst,
+                                         "note": "in the step: both weights in one launch"}
+        for n, wc, ws, wg in P.w:
+            yy = torch.empty((M, n), dtype=torch.bfloat16, device=dev)
+            g_ms, _ = time_fn(lambda: q4.q4_gemm(q4.NVFP4, M, n, K, P.xc, P.xs, P.amax[1:2], wc, ws, wg, y=yy), 20,
+                              flush)
+            tf = 2.0 * M * n * K / (g_ms * 1e-3) / 1e12
+            rows[f"gemm_prefill_n{n}_cold"] = {"us": g_ms * 1e3, "TFLOP/s": tf, "frac_fp4": tf / fp4_burst,
+                                               "note": "the single-weight launch alone, after a cold, clean L2"}
+            del yy
+        del P
+        torch.cuda.empty_cache()
+        rows.update(rows_bench(q4, dev, flush, pk, reps=args.rows_reps))
 
     cpu = None if args.no_cpu_baseline or rank != 0 else cpu_baseline(budget_s=args.cpu_seconds)
     traffic, traffic_note = roofline_traffic(args.traffic)
@@ -616,12 +682,13 @@ def run_ours(args):
         "config": {"workload": WORKLOAD, "M": M, "K": K, "N": [N1, N2], "x_stat": x_stat, "quantize_GB/s": q_gbs,
                    "quantize_frac_hbm": q_gbs / hbm, "l2": "flushed before every timed step: 256 MiB write, then a 256 MiB read (cold, clean L2)",
                    "parallelism": f"replicas x{world} (independent problems per GPU)"},
-        "roofline": {"kernel": "gemm_kernel<NVFP4> 8192x17408x5120", "bound": "tensor", "achieved": gemm2_tf,
-                     "peak": fp4_burst, "unit": "TFLOP/s", "frac": gemm2_tf / fp4_burst,
+        "roofline": {"kernel": "gemm_kernel<NVFP4>, one launch over W1 and W2: 8192 x (5120 + 17408) x 5120",
+                     "bound": "tensor", "achieved": gemm_tf,
+                     "peak": fp4_burst, "unit": "TFLOP/s", "frac": gemm_tf / fp4_burst,
                      "peak_note": f"dense FP4 = {pk['src']} bf16 burst {pk['bf16']} x 4 (nominal 9/2.25)",
-                     "frac_vs_sustained": gemm2_tf / (pk["bf16_sus"] * FP4_OVER_BF16),
+                     "frac_vs_sustained": gemm_tf / (pk["bf16_sus"] * FP4_OVER_BF16),
                      "traffic": traffic, "traffic_note": traffic_note,
-                     "algorithmic_bytes": M * K / 2 + M * K / 16 + N2 * K / 2 + N2 * K / 16 + 2 * M * N2},
+                     "algorithmic_bytes": M * K / 2 + M * K / 16 + (N1 + N2) * K * (0.5 + 1 / 16) + 2 * M * (N1 + N2)},
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": Prefill.LAUNCHES_PER_STEP * args.steps,
@@ -798,7 +865,8 @@ def run_reference(args):
     }))
 
 
-PROFILE_ROWS = ("mxfp4_quantize", "amax_quantize", "nvfp4_quantize", "gemm_n5120", "gemm_n17408", "decode",
+PROFILE_ROWS = ("mxfp4_quantize", "amax_quantize", "nvfp4_quantize", "gemm_n5120", "gemm_n17408", "gemm_shared",
+                "decode",
                 "sigma_delta_visit", "sd_gemm_m16", "w4a16_4096")
 
 
@@ -813,8 +881,8 @@ def run_profile(row: str, launches: int):
         c = torch.empty((4096, 2048), dtype=torch.uint8, device=dev)
         sc = torch.empty(q4.q4_scale_bytes(q4.MXFP4, 4096, 4096), dtype=torch.uint8, device=dev)
         fn = lambda: q4.q4_quantize(q4.MXFP4, x, chan=t, flags=q4.LAYOUT_TC | q4.HADAMARD32, codes=c, scales=sc)
-    elif row in ("amax_quantize", "nvfp4_quantize", "gemm_n5120", "gemm_n17408"):
-        n_list = {"gemm_n5120": (N1,), "gemm_n17408": (N2,)}.get(row, ())
+    elif row in ("amax_quantize", "nvfp4_quantize", "gemm_n5120", "gemm_n17408", "gemm_shared"):
+        n_list = {"gemm_n5120": (N1,), "gemm_n17408": (N2,), "gemm_shared": (N1, N2)}.get(row, ())
         d = synth.prefill(n_list=n_list)
         x = d["x"].to(dev)
         out = torch.zeros(4, dtype=torch.float32, device=dev)
@@ -826,13 +894,19 @@ def run_profile(row: str, launches: int):
         elif row == "nvfp4_quantize":
             fn = lambda: q4.q4_quantize(q4.NVFP4, x, gscale=out[1:2], codes=c, scales=sc)
         else:
-            w = torch.from_numpy(d["w"][0]).to(dev)
-            g = q4.q4_amax(w, 2688.0)[1:2].clone()
-            wc, ws = q4.q4_quantize(q4.NVFP4, w, gscale=g)
-            del w
-            n = n_list[0]
-            y = torch.empty((M, n), dtype=torch.bfloat16, device=dev)
-            fn = lambda: q4.q4_gemm(q4.NVFP4, M, n, K, c, sc, out[1:2], wc, ws, g, y=y)
+            wts = []
+            for wn in d["w"]:
+                w = torch.from_numpy(wn).to(dev)
+                g = q4.q4_amax(w, 2688.0)[1:2].clone()
+                wc, ws = q4.q4_quantize(q4.NVFP4, w, gscale=g)
+                del w
+                wts.append((wc, ws, g, wn.shape[0]))
+            ys = [torch.empty((M, n), dtype=torch.bfloat16, device=dev) for n in n_list]
+            if row == "gemm_shared":
+                fn = lambda: q4.q4_gemm_shared_a(q4.NVFP4, M, K, c, sc, out[1:2], wts, ys=ys)
+            else:
+                wc, ws, g, n = wts[0]
+                fn = lambda: q4.q4_gemm(q4.NVFP4, M, n, K, c, sc, out[1:2], wc, ws, g, y=ys[0])
     elif row == "decode":
         dd = synth.decode()
         xd = dd["x"].to(dev)

@@ -368,6 +368,33 @@ Q4_API q4_status q4_sigma_delta_gemm_grouped(q4_format format, int block, int64_
                                              const q4_sd_gemm_entry* entries, int count,
                                              q4_dtype out_dt, int flags, void* stream);
 
+/* One weight of q4_gemm_shared_a. */
+typedef struct {
+    const uint8_t* b_codes;   /* [N, K/2] packed codes                              */
+    const uint8_t* b_scales;  /* tensor-core scale layout                           */
+    const float* d_b_gscale;  /* NVFP4: device s_t of the weight; MXFP4: NULL       */
+    void* y;                  /* [M, N] output of out_dt                            */
+    int64_t N;                /* N % 8 == 0; 0 skips the entry                      */
+} q4_gemm_weight;
+
+#define Q4_MAX_SHARED_A 4
+
+/*
+ * q4_gemm_shared_a -- one quantized A times several weights, Y_w = alpha_w *
+ *   dec(A) dec(B_w)^T for w < count, in one persistent launch: the output tiles
+ *   of every weight form one list walked by the same grid, so the launch pays
+ *   one ramp and one partial last wave instead of one per weight (the
+ *   projections of one layer input, as the W4A4 linear layers of the "Why
+ *   Gated DeltaNet Survives 4-Bit Quantization" page apply to a quantized
+ *   activation).  Each Y_w is, bit for bit, what q4_gemm with a_kind =
+ *   Q4_A_QUANTIZED gives for that weight.  a, a_scales, d_a_gscale, M, K and the
+ *   requirements as q4_gemm; 1 <= count <= Q4_MAX_SHARED_A; no y may overlap
+ *   another entry's y or any input.
+ */
+Q4_API q4_status q4_gemm_shared_a(q4_format format, int block, int64_t M, int64_t K, const uint8_t* a,
+                                  const uint8_t* a_scales, const float* d_a_gscale,
+                                  const q4_gemm_weight* weights, int count, q4_dtype out_dt, void* stream);
+
 /* Scratch bytes q4_gemm needs for these arguments (0 when none). */
 Q4_API size_t q4_gemm_workspace_size(q4_format format, int64_t M, int64_t N, int64_t K,
                               int a_kind);

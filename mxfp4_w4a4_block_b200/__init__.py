@@ -67,6 +67,7 @@ SIGNATURES = {
     "q4_gemm_a_bf16_noalloc": (_I, [_I64, _I64, _I64, _P, _P, _P, _P, _P, _I, _P, _P]),
     "q4_set_wait_limit": (_I, [_I64]),
     "q4_amax_quantize": (_I, [_I, _P, _I64, _I64, _I64, ctypes.c_float, _P, _P, _P, _I, _P]),
+    "q4_gemm_shared_a": (_I, [_I, _I, _I64, _I64, _P, _P, _P, _P, _I, _I, _P]),
     "q4_quantize_grouped": (_I, [_I, _I, _I, _P, _I, _I, _P]),
     "q4_sigma_delta_step_grouped": (_I, [_I, _I, _P, _I, _I, _P]),
     "q4_sr_requant_grouped": (_I, [_I, _I, _P, _I, ctypes.c_uint64, ctypes.c_uint32, _I, _P]),
@@ -81,6 +82,11 @@ class Q4SdGemmEntry(ctypes.Structure):
     """struct q4_sd_gemm_entry of include/q4.h."""
     _fields_ = [("x", _P), ("w", _P), ("scales", _P), ("d_gscale", _P), ("residue", _P), ("y", _P),
                 ("N", _I64)]
+
+
+class Q4GemmWeight(ctypes.Structure):
+    """struct q4_gemm_weight of include/q4.h (one weight of q4_gemm_shared_a)."""
+    _fields_ = [("b_codes", _P), ("b_scales", _P), ("d_b_gscale", _P), ("y", _P), ("N", _I64)]
 
 
 class Q4Matrix(ctypes.Structure):
@@ -379,6 +385,22 @@ def q4_gemm(fmt: int, M: int, N: int, K: int, a: torch.Tensor, a_scales, a_gscal
                        _ptr(workspace), ws_bytes, _stream(stream))
     _check("q4_gemm", st)
     return y
+
+
+def q4_gemm_shared_a(fmt: int, M: int, K: int, a: torch.Tensor, a_scales: torch.Tensor, a_gscale, weights,
+                     out_dtype=torch.bfloat16, ys=None, stream=None):
+    """Y_w = alpha_w dec(A) dec(B_w)^T for each weight (b_codes, b_scales, b_gscale, N) of
+    `weights`, in one launch; returns the list of Y_w."""
+    dev = a.device
+    if ys is None:
+        ys = [torch.empty((M, w[3]), dtype=out_dtype, device=dev) for w in weights]
+    arr = (Q4GemmWeight * len(weights))()
+    for i, (bc, bs, bg, n) in enumerate(weights):
+        arr[i] = Q4GemmWeight(_ptr(bc), _ptr(bs), _ptr(bg), _ptr(ys[i]), n)
+    st = lib().q4_gemm_shared_a(fmt, BLOCK[fmt], M, K, _ptr(a), _ptr(a_scales), _ptr(a_gscale),
+                                ctypes.cast(arr, ctypes.c_void_p), len(weights), _dtype_code(ys[0]), _stream(stream))
+    _check("q4_gemm_shared_a", st)
+    return ys
 
 
 def q4_gemm_a_bf16_noalloc(M: int, N: int, K: int, a: torch.Tensor, a_gscale, b_codes: torch.Tensor,

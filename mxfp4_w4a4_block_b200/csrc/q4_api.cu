@@ -398,6 +398,54 @@ q4_status q4_set_wait_limit(int64_t cycles) {
     return cuda_status(q4::set_wait_limit((long long)cycles));
 }
 
+q4_status q4_gemm_shared_a(q4_format format, int block, int64_t M, int64_t K, const uint8_t* a,
+                           const uint8_t* a_scales, const float* d_a_gscale, const q4_gemm_weight* weights,
+                           int count, q4_dtype out_dt, void* stream) {
+    if (!valid_format(format) || !valid_dtype(out_dt) || M < 0 || K < 0) return Q4_ERR_ARG;
+    if (block != block_of(format)) return Q4_ERR_UNSUPPORTED;
+    if (count < 1 || count > Q4_MAX_SHARED_A || !weights) return Q4_ERR_ARG;
+    if (format == Q4_NVFP4 && !d_a_gscale) return Q4_ERR_ARG;
+    if (format == Q4_MXFP4 && d_a_gscale) return Q4_ERR_ARG;
+    if (K % 64) return Q4_ERR_SHAPE;
+    if (K > ((int64_t)1 << 30) || M > ((int64_t)1 << 31)) return Q4_ERR_SHAPE;
+    for (int i = 0; i < count; ++i) {
+        const q4_gemm_weight& w = weights[i];
+        if (w.N < 0) return Q4_ERR_ARG;
+        if (w.N % 8 || w.N > ((int64_t)1 << 31)) return Q4_ERR_SHAPE;
+        if (format == Q4_NVFP4 && !w.d_b_gscale) return Q4_ERR_ARG;
+        if (format == Q4_MXFP4 && w.d_b_gscale) return Q4_ERR_ARG;
+        if (M == 0 || w.N == 0) continue;
+        if (!w.y) return Q4_ERR_ARG;
+        if (!aligned16(w.y)) return Q4_ERR_ALIGN;
+        if (K == 0) continue;
+        if (!w.b_codes || !w.b_scales) return Q4_ERR_ARG;
+        if (!aligned16(w.b_codes) || !aligned16(w.b_scales)) return Q4_ERR_ALIGN;
+    }
+    if (M == 0) return Q4_OK;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (K == 0) {
+        for (int i = 0; i < count; ++i)
+            if (weights[i].N > 0) {
+                const size_t ysz = (size_t)M * (size_t)weights[i].N * (out_dt == Q4_BF16 ? 2 : 4);
+                const q4_status s = cuda_status(cudaMemsetAsync(weights[i].y, 0, ysz, st));
+                if (s != Q4_OK) return s;
+            }
+        return Q4_OK;
+    }
+    if (!a || !a_scales) return Q4_ERR_ARG;
+    if (!aligned16(a) || !aligned16(a_scales)) return Q4_ERR_ALIGN;
+    q4::GemmParams ps[Q4_MAX_SHARED_A];
+    for (int i = 0; i < count; ++i) {
+        q4::GemmParams& p = ps[i];
+        const q4_gemm_weight& w = weights[i];
+        p.M = M; p.N = w.N; p.K = K;
+        p.a_codes = a; p.a_scales = a_scales; p.a_gscale = d_a_gscale;
+        p.b_codes = w.b_codes; p.b_scales = w.b_scales; p.b_gscale = w.d_b_gscale;
+        p.y = w.y; p.out_bf16 = out_dt == Q4_BF16; p.mxfp4 = format == Q4_MXFP4;
+    }
+    return cuda_status(q4::launch_gemm_multi(ps, count, st, num_sms()));
+}
+
 q4_status q4_get_device_error(void* stream) {
     cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_status(e);

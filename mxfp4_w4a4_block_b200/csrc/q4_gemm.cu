@@ -69,18 +69,40 @@ constexpr uint32_t SF_COL = 256;         // SF_NBUF buffers of 48 columns, one p
 constexpr int SF_NBUF = 4;
 constexpr uint32_t SF_BUF = 48;          // per buffer: SFA 4 atoms x 4 columns, then SFB 4 atoms x 8
 constexpr uint32_t SFB_OFF = 16;
+constexpr int MAX_W = 4;                 // weights that share one A in a launch
 }  // namespace gemm
 
+// One A [M, K] times up to MAX_W weights B_w [N_w, K] into Y_w [M, N_w]: the
+// tiles of all weights form one list (weight w's tiles from tile_start[w]),
+// walked by the persistent CTAs as one grid.
 struct GemmDev {
-    int64_t M, N, K;
+    int64_t M, K;
+    int nw;
+    int64_t N[gemm::MAX_W];
+    int64_t tile_start[gemm::MAX_W + 1];
     const uint8_t* a_scales;
-    const uint8_t* b_scales;
+    const uint8_t* b_scales[gemm::MAX_W];
     const float* a_gscale;
-    const float* b_gscale;
-    void* y;
+    const float* b_gscale[gemm::MAX_W];
+    void* y[gemm::MAX_W];
     int64_t catoms;      // scale atom-columns per 128-row band (same for A and B)
     int out_bf16;
 };
+
+// The launch's tensor maps: A, and each weight's B and (bf16 output) Y.
+struct GemmMaps {
+    CUtensorMap a;
+    CUtensorMap b[gemm::MAX_W];
+    CUtensorMap y[gemm::MAX_W];
+};
+
+// Weight of tile t: the last w whose tiles start at or before t.
+__device__ __forceinline__ int gemm_weight_of(const GemmDev& p, int64_t t) {
+    int w = 0;
+#pragma unroll
+    for (int i = 1; i < gemm::MAX_W; ++i) w += (i < p.nw && t >= p.tile_start[i]) ? 1 : 0;
+    return w;
+}
 
 // Store 32 consecutive fp32 results of one output row (columns col0..col0+31,
 // only those < N), scaled by alpha.
@@ -145,8 +167,7 @@ __device__ __forceinline__ void store_row32_bf16(void* y, int64_t N, int64_t row
 
 template <bool MX>
 __global__ void __launch_bounds__(gemm::THREADS, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const __grid_constant__ CUtensorMap tmY, GemmDev p) {
+    gemm_kernel(const __grid_constant__ GemmMaps maps, const __grid_constant__ GemmDev p) {
     using namespace gemm;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -182,9 +203,11 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
         tmem_relinquish();
     }
     if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(&tmA);
-        tma_prefetch_desc(&tmB);
-        if (p.out_bf16) tma_prefetch_desc(&tmY);
+        tma_prefetch_desc(&maps.a);
+        for (int w = 0; w < p.nw; ++w) {
+            tma_prefetch_desc(&maps.b[w]);
+            if (p.out_bf16) tma_prefetch_desc(&maps.y[w]);
+        }
     }
     tc_fence_before();
     __syncthreads();
@@ -192,12 +215,10 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
     const uint32_t tmem = *tmem_holder;
 
     const int64_t tiles_m = (p.M + BM - 1) / BM;
-    const int64_t tiles_n = (p.N + BN - 1) / BN;
-    const int64_t tiles = tiles_m * tiles_n;
+    const int64_t tiles = p.tile_start[p.nw];
     const int nkb = (int)((p.K + KB_ELEMS - 1) / KB_ELEMS);
     const int mma_per_atom = MX ? 2 : 1;
     const int atoms_per_kb = 4 / mma_per_atom;
-    const int64_t bands_n = (p.N + 127) / 128;
 
     if (warp == 0) {
         if (lane == 0) {
@@ -207,7 +228,10 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
             bool issued[STAGES];
             for (int s = 0; s < STAGES; ++s) issued[s] = false, last_phase[s] = 0;
             for (int64_t t = blockIdx.x; t < tiles && !*abort_flag; t += gridDim.x) {
-                const int64_t mt = t % tiles_m, nt = t / tiles_m;
+                const int w = gemm_weight_of(p, t);
+                const int64_t lt = t - p.tile_start[w];
+                const int64_t mt = lt % tiles_m, nt = lt / tiles_m;
+                const int64_t bands_n = (p.N[w] + 127) / 128;
                 const int nbands = (nt * 2 + 1 < bands_n) ? 2 : 1;
                 for (int kb = 0; kb < nkb; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1)) { *abort_flag = 1; break; }
@@ -217,14 +241,15 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
                     const int na = (nmma + mma_per_atom - 1) / mma_per_atom;
                     const uint32_t bytes = A_STAGE + B_STAGE + (uint32_t)na * 512u * (1u + (uint32_t)nbands);
                     mbar_arrive_expect_tx(&full[stage], bytes);
-                    tma_load_2d(smem + stage * A_STAGE, &tmA, &full[stage], kb * KB_BYTES, (int32_t)(mt * BM));
-                    tma_load_2d(smem + OFF_B + stage * B_STAGE, &tmB, &full[stage], kb * KB_BYTES, (int32_t)(nt * BN));
+                    tma_load_2d(smem + stage * A_STAGE, &maps.a, &full[stage], kb * KB_BYTES, (int32_t)(mt * BM));
+                    tma_load_2d(smem + OFF_B + stage * B_STAGE, &maps.b[w], &full[stage], kb * KB_BYTES,
+                                (int32_t)(nt * BN));
                     const int64_t acol = (int64_t)kb * atoms_per_kb;
                     bulk_load(smem + OFF_SFA + stage * SFA_STAGE, p.a_scales + (mt * p.catoms + acol) * 512,
                               (uint32_t)na * 512u, &full[stage]);
                     for (int b = 0; b < nbands; ++b)
                         bulk_load(smem + OFF_SFB + stage * SFB_STAGE + b * 2048,
-                                  p.b_scales + ((nt * 2 + b) * p.catoms + acol) * 512, (uint32_t)na * 512u,
+                                  p.b_scales[w] + ((nt * 2 + b) * p.catoms + acol) * 512, (uint32_t)na * 512u,
                                   &full[stage]);
                     issued[stage] = true;
                     last_phase[stage] = phase;
@@ -324,7 +349,7 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
         const int quad = warp & 3;                 // TMEM lane quarter this warp may access
         const int half = (warp - FIRST_EPI_WARP) >> 2;   // which 128 accumulator columns
         const int row_in_tile = quad * 32 + lane;
-        const float alpha = MX ? 1.0f : __fmul_rn(*p.a_gscale, *p.b_gscale);
+        const float a_st = MX ? 1.0f : *p.a_gscale;
         const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + ACC_COL + half * 128;
         const bool out_bf16 = p.out_bf16 != 0;
         const int order = warp - FIRST_EPI_WARP;          // position in the store-buffer turn chain
@@ -333,9 +358,12 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
         for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++iter) {
             if (!mbar_wait(tmem_full, acc_phase)) { *abort_flag = 1; break; }
             tc_fence_after();
-            const int64_t mt = t % tiles_m, nt = t / tiles_m;
+            const int w = gemm_weight_of(p, t);
+            const int64_t lt = t - p.tile_start[w];
+            const int64_t mt = lt % tiles_m, nt = lt / tiles_m;
             const int64_t row = mt * BM + row_in_tile;
             const int64_t col_base = nt * BN + half * 128;
+            const float alpha = MX ? 1.0f : __fmul_rn(a_st, *p.b_gscale[w]);
             uint32_t pk[2][32];          // bf16 pairs: [0] columns 0..63, [1] columns 64..127
 #pragma unroll
             for (int round = 0; round < 4; ++round) {
@@ -356,7 +384,7 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
                         pk[round >> 1][(round & 1) * 16 + j] = *reinterpret_cast<uint32_t*>(&h);
                     }
                 } else if (row < p.M) {
-                    store_row32(p.y, p.N, row, col_base + round * 32, r, alpha, false);
+                    store_row32(p.y[w], p.N[w], row, col_base + round * 32, r, alpha, false);
                 }
             }
             if (out_bf16) {
@@ -376,8 +404,8 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
                 __syncwarp();
                 if (lane == 0) {
                     const int32_t r0 = (int32_t)(mt * BM + quad * 32);
-                    tma_store_2d(&tmY, buf, (int32_t)col_base, r0);
-                    tma_store_2d(&tmY, buf + 4096, (int32_t)(col_base + 64), r0);
+                    tma_store_2d(&maps.y[w], buf, (int32_t)col_base, r0);
+                    tma_store_2d(&maps.y[w], buf + 4096, (int32_t)(col_base + 64), r0);
                     bulk_commit_group();
                     bulk_wait_read_all();
                     mbar_arrive(&epi_turn[(order + 1) % EPI_WARPS]);
@@ -451,35 +479,58 @@ static bool make_out_map(CUtensorMap* map, void* y, int64_t M, int64_t N) {
 }
 
 
-cudaError_t launch_gemm(const GemmParams& p, cudaStream_t st, int num_sms) {
+// One quantized A times nw weights in one persistent launch (nw = 1: q4_gemm).
+cudaError_t launch_gemm_multi(const GemmParams* ps, int nw, cudaStream_t st, int num_sms) {
     using namespace gemm;
-    if (p.M == 0 || p.N == 0) return cudaSuccess;
-    CUtensorMap ma, mb, my;
-    if (!make_code_map(&ma, p.a_codes, p.M, p.K / 2, BM)) return cudaErrorInvalidValue;
-    if (!make_code_map(&mb, p.b_codes, p.N, p.K / 2, BN)) return cudaErrorInvalidValue;
-    std::memset(&my, 0, sizeof(my));
-    if (p.out_bf16 && !make_out_map(&my, p.y, p.M, p.N)) return cudaErrorInvalidValue;
+    if (nw < 1 || nw > MAX_W) return cudaErrorInvalidValue;
+    const GemmParams& p0 = ps[0];
+    if (p0.M == 0) return cudaSuccess;
+    GemmMaps maps;
+    std::memset(&maps, 0, sizeof(maps));
     GemmDev d;
-    d.M = p.M; d.N = p.N; d.K = p.K;
-    d.a_scales = p.a_scales; d.b_scales = p.b_scales;
-    d.a_gscale = p.a_gscale; d.b_gscale = p.b_gscale;
-    d.y = p.y;
-    const int blk = p.mxfp4 ? 32 : 16;
-    d.catoms = ((p.K / blk) + 3) / 4;
-    d.out_bf16 = p.out_bf16 ? 1 : 0;
-    const int64_t tiles = ((p.M + BM - 1) / BM) * ((p.N + BN - 1) / BN);
+    std::memset(&d, 0, sizeof(d));
+    if (!make_code_map(&maps.a, p0.a_codes, p0.M, p0.K / 2, BM)) return cudaErrorInvalidValue;
+    d.M = p0.M; d.K = p0.K;
+    d.a_scales = p0.a_scales; d.a_gscale = p0.a_gscale;
+    const int blk = p0.mxfp4 ? 32 : 16;
+    d.catoms = ((p0.K / blk) + 3) / 4;
+    d.out_bf16 = p0.out_bf16 ? 1 : 0;
+    const int64_t tiles_m = (p0.M + BM - 1) / BM;
+    int n = 0;
+    int64_t tiles = 0;
+    for (int i = 0; i < nw; ++i) {
+        const GemmParams& p = ps[i];
+        if (p.N == 0) continue;               // nothing to compute for this weight
+        if (!make_code_map(&maps.b[n], p.b_codes, p.N, p.K / 2, BN)) return cudaErrorInvalidValue;
+        if (p.out_bf16 && !make_out_map(&maps.y[n], p.y, p.M, p.N)) return cudaErrorInvalidValue;
+        d.N[n] = p.N;
+        d.b_scales[n] = p.b_scales;
+        d.b_gscale[n] = p.b_gscale;
+        d.y[n] = p.y;
+        d.tile_start[n] = tiles;
+        tiles += tiles_m * ((p.N + BN - 1) / BN);
+        ++n;
+    }
+    if (n == 0) return cudaSuccess;
+    d.nw = n;
+    for (int i = n; i <= MAX_W; ++i) d.tile_start[i] = tiles;
     const int grid = (int)(tiles < num_sms ? tiles : num_sms);
     cudaError_t e;
-    if (p.mxfp4) {
+    if (p0.mxfp4) {
         e = cudaFuncSetAttribute(gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
         if (e != cudaSuccess) return e;
-        gemm_kernel<true><<<grid, THREADS, SMEM_BYTES, st>>>(ma, mb, my, d);
+        gemm_kernel<true><<<grid, THREADS, SMEM_BYTES, st>>>(maps, d);
     } else {
         e = cudaFuncSetAttribute(gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
         if (e != cudaSuccess) return e;
-        gemm_kernel<false><<<grid, THREADS, SMEM_BYTES, st>>>(ma, mb, my, d);
+        gemm_kernel<false><<<grid, THREADS, SMEM_BYTES, st>>>(maps, d);
     }
     return cudaGetLastError();
+}
+
+cudaError_t launch_gemm(const GemmParams& p, cudaStream_t st, int num_sms) {
+    if (p.M == 0 || p.N == 0) return cudaSuccess;
+    return launch_gemm_multi(&p, 1, st, num_sms);
 }
 
 // ------------------------------------------------------------------ W4A16 GEMM
@@ -1327,14 +1378,12 @@ constexpr int FIRST_E = FIRST_Q + QWARPS;
 constexpr int THREADS = 32 * (FIRST_E + EWARPS);
 constexpr int W_STAGE = 128 * 128;       // weight codes of one k-block
 constexpr int SFW_STAGE = 4 * 512;       // their scale atoms
-// The weight ring's depth sets the pace (a stage is refilled only after its
-// MMAs complete, so the bytes in flight per SM over the loaded round trip
-// bound the stream): the activation slabs are kept to 4 so that 9 weight
-// stages fit in shared memory rather than 7 (26.6 -> 24.6 us at 16 x 17408 x 5120).
-constexpr int XSLOTS = 4;               // bf16 activation slabs (per-thread cp.async ring)
-constexpr int XDIST = 3;                // k-blocks fetched ahead (< XSLOTS)
-constexpr int QSLOTS = 6;               // quantized activation k-blocks ahead of the MMAs
-constexpr int SFX = 4 * 512;             // activation scale atoms of one k-block
+// The activations are quantized once per CTA into a resident buffer (codes in
+// the swizzled K-major operand layout, one 16-row x 128-byte tile per k-block,
+// and the block scales packed per k-block), so the activation path never waits
+// on the MMAs and CTAs with more than one weight tile reuse it; the rest of
+// shared memory is the weight ring.
+constexpr int XDIST = 4;                // k-blocks of activations loaded ahead, in registers
 constexpr int MAX_M = 16;
 constexpr int MAX_STAGES = 12;
 constexpr uint32_t TMEM_COLS = 256;
@@ -1344,7 +1393,7 @@ constexpr uint32_t SF_COL = 128;         // SF_NBUF scale buffers of SF_BUF colu
 constexpr uint32_t SF_BUF = 32;          //   weight atoms x 4 columns, then activation atoms x 4
 constexpr int SF_NBUF = 4;
 constexpr int MAX_SMEM = 232448;         // 227 KB opt-in limit per CTA
-constexpr int BAR_BYTES = 1536;       // barriers (< 512 B), then the 128-entry (S, 1/S) table
+constexpr int FIXED_BARS = 40;        // ring, scale-buffer, TMEM and done barriers (<= 40)
 }  // namespace dec
 
 struct DecodeDev {
@@ -1367,20 +1416,22 @@ __device__ __forceinline__ uint32_t sw128_offset(int row, int byte_in_row) {
 }
 
 struct DecodeLayout {
-    int xraw, xq, off_w, off_sfw, off_xraw, off_xq, off_sfx, off_bar, total;
+    int off_w, off_sfw, off_xq, off_xs, off_bar, off_tab, total;
 };
 
-__host__ __device__ inline DecodeLayout decode_layout(int np, int stages) {
+// Weight ring (S stages of codes and scale atoms), the resident activation codes
+// (nkb tiles of np x 128 bytes) and scales (nkb x 4 atoms x np rows x 4 bytes),
+// the barriers (the fixed ones, then one per k-block of activations) and the
+// 128-entry (S, 1/S) table.
+__host__ __device__ inline DecodeLayout decode_layout(int np, int nkb, int stages) {
     DecodeLayout L;
-    L.xraw = np * 512;                    // bf16 slab: np rows x 256 elements
-    L.xq = np * 128;                      // codes: np rows x 128 bytes (1024-aligned: np % 16 == 0)
     L.off_w = 0;
     L.off_sfw = L.off_w + stages * dec::W_STAGE;
-    L.off_xq = L.off_sfw + stages * dec::SFW_STAGE;
-    L.off_xraw = L.off_xq + dec::QSLOTS * L.xq;
-    L.off_sfx = L.off_xraw + dec::XSLOTS * L.xraw;
-    L.off_bar = L.off_sfx + dec::QSLOTS * dec::SFX;
-    L.total = L.off_bar + dec::BAR_BYTES + 1024;
+    L.off_xq = L.off_sfw + stages * dec::SFW_STAGE;        // 1024-aligned: both stage sizes are
+    L.off_xs = L.off_xq + nkb * np * 128;
+    L.off_bar = L.off_xs + nkb * 16 * np;
+    L.off_tab = (L.off_bar + 8 * (dec::FIXED_BARS + nkb) + 15) / 16 * 16;
+    L.total = L.off_tab + 128 * 8 + 1024;                   // + alignment slack
     return L;
 }
 
@@ -1390,26 +1441,23 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int np = p.np, nkb = p.nkb, S = p.stages;
-    const DecodeLayout L = decode_layout(np, S);
+    const DecodeLayout L = decode_layout(np, nkb, S);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.off_bar);   // [S] weight tile landed
     uint64_t* empty = full + MAX_STAGES;                               // [S] its MMAs are done
-    uint64_t* xq_full = empty + MAX_STAGES;                            // [QSLOTS] quantized k-block ready
-    uint64_t* xq_empty = xq_full + QSLOTS;                             // [QSLOTS] its MMAs are done
-    uint64_t* sf_ready = xq_empty + QSLOTS;                            // [SF_NBUF] scales staged in TMEM buffer
+    uint64_t* sf_ready = empty + MAX_STAGES;                           // [SF_NBUF] scales staged in TMEM buffer
     uint64_t* sf_free = sf_ready + SF_NBUF;                            // [SF_NBUF] its MMAs are done
     uint64_t* tmem_full = sf_free + SF_NBUF;
     uint64_t* tmem_empty = tmem_full + 1;
     uint64_t* mma_done = tmem_empty + 1;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
-    float2* nv_tab = reinterpret_cast<float2*>(smem + L.off_bar + 512);   // 128 (S, 1/S) entries
+    uint64_t* xres = reinterpret_cast<uint64_t*>(smem + L.off_bar) + FIXED_BARS;   // [nkb] activations ready
+    float2* nv_tab = reinterpret_cast<float2*>(smem + L.off_tab);      // 128 (S, 1/S) entries
+    const uint8_t* xs_res = smem + L.off_xs;                           // packed activation scales
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-        for (int x = 0; x < QSLOTS; ++x) {
-            mbar_init(&xq_full[x], QWARPS);
-            mbar_init(&xq_empty[x], 1);
-        }
+        for (int kb = 0; kb < nkb; ++kb) mbar_init(&xres[kb], QWARPS);
         for (int b = 0; b < SF_NBUF; ++b) { mbar_init(&sf_ready[b], EWARPS); mbar_init(&sf_free[b], 1); }
         mbar_init(tmem_full, 1);
         mbar_init(tmem_empty, EWARPS);
@@ -1453,22 +1501,22 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
     } else if (warp == 1) {
         if (lane == 0) {
             const uint32_t idesc = idesc_mxf4(128, np, false);
-            int stage = 0, x = 0, b = 0;
-            uint32_t phase = 0, xphase = 0, bphase = 0, acc_phase = 0;
+            int stage = 0, b = 0;
+            uint32_t phase = 0, bphase = 0, acc_phase = 0;
             bool ok = true;
             for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
                 if (!mbar_wait(tmem_empty, acc_phase ^ 1)) { ok = false; break; }
                 tc_fence_after();
                 uint32_t started = 0;                    // bit j: accumulator j holds a partial sum
                 for (int kb = 0; kb < nkb; ++kb) {
-                    if (!mbar_wait(&full[stage], phase) || !mbar_wait(&xq_full[x], xphase) ||
+                    if (!mbar_wait(&full[stage], phase) || !mbar_wait(&xres[kb], 0) ||
                         !mbar_wait(&sf_ready[b], bphase)) { ok = false; break; }
                     tc_fence_after();
                     const int64_t krem = p.K - (int64_t)kb * 256;
                     const int nmma = (krem < 256 ? (int)krem : 256) / 64;
                     const uint32_t sfa = tmem + SF_COL + b * SF_BUF, sfb = sfa + 16;
                     const uint64_t adesc = smem_desc(smem_u32(smem + L.off_w + stage * W_STAGE), 16, 1024, 2);
-                    const uint64_t bdesc = smem_desc(smem_u32(smem + L.off_xq + x * L.xq), 16, 1024, 2);
+                    const uint64_t bdesc = smem_desc(smem_u32(smem + L.off_xq + kb * np * 128), 16, 1024, 2);
                     // four independent accumulation chains: tiny-N MMAs into one
                     // accumulator would serialise on their latency
                     for (int kk = 0; kk < nmma; ++kk) {
@@ -1477,10 +1525,8 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
                         started |= 1u << kk;
                     }
                     tc_commit(&empty[stage]);
-                    tc_commit(&xq_empty[x]);
                     tc_commit(&sf_free[b]);
                     if (++stage == S) { stage = 0; phase ^= 1; }
-                    if (++x == QSLOTS) { x = 0; xphase ^= 1; }
                     if (++b == SF_NBUF) { b = 0; bphase ^= 1; }
                 }
                 if (!ok) break;
@@ -1492,67 +1538,55 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
             mbar_wait(mma_done, 0);
         }
     } else if (warp < FIRST_E) {
-        // ---- quantize activation slabs (warps 2..9)
+        // ---- quantize the activations (warps 2..9), once per CTA
         const int qt = threadIdx.x - 32 * FIRST_Q;
         constexpr int QT = 32 * QWARPS;
         const NvCtx sc = nv_ctx(*p.a_gscale, nv_tab);
         nv_fill_table(*p.a_gscale, nv_tab, qt, QT);
         named_barrier(1, QT);
-        // Each quantizer thread fetches exactly the activation bytes it will
-        // quantize with cp.async, XDIST k-blocks ahead, into its own part of a
-        // ring of XSLOTS slabs.  These copies go through the load/store path,
-        // not the TMA queue the weight tiles fill, so they are not held up
-        // behind the weight stream; no thread reads another's bytes, so the
-        // copy groups alone order the ring.
-        const int64_t my_tiles = tiles > blockIdx.x ? (tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-        const int64_t total_kb = my_tiles * nkb;
-        const uint16_t* xg = p.x;
-        auto fetch = [&](int64_t i) {
-            uint8_t* raw = smem + L.off_xraw + (int)(i % XSLOTS) * L.xraw;
-            const int64_t k0 = (i % nkb) * 256;
-            for (int b = qt; b < np * 16; b += QT) {
-                const int m = b >> 4, j = b & 15;
-                const int64_t k = k0 + j * 16;
-                const bool in = m < p.M && k < p.K;     // outside X: zero fill
-                const uint16_t* src = in ? xg + m * p.K + k : xg;
-                cp_async16(raw + m * 512 + j * 32, src, in);
-                cp_async16(raw + m * 512 + j * 32 + 16, src + 8, in);
+        // Thread qt owns block (row m = qt / 16, block j = qt % 16) of every
+        // k-block (np * 16 <= QT blocks per k-block); its 32 input bytes are
+        // loaded XDIST k-blocks ahead into registers (rows and columns outside X
+        // read as zero), then quantized into the resident codes and scales.
+        const int m = qt >> 4, j = qt & 15;
+        const bool active = qt < np * 16;
+        const uint16_t* xrow = p.x + (int64_t)m * p.K;
+        auto load = [&](int kb, uint4 (&r)[2]) {
+            const int64_t k = (int64_t)kb * 256 + j * 16;
+            if (active && m < p.M && k < p.K) {
+                r[0] = __ldg(reinterpret_cast<const uint4*>(xrow + k));
+                r[1] = __ldg(reinterpret_cast<const uint4*>(xrow + k + 8));
+            } else {
+                r[0] = r[1] = make_uint4(0u, 0u, 0u, 0u);
             }
         };
-        for (int64_t i = 0; i < XDIST; ++i) {
-            if (i < total_kb) fetch(i);
-            cp_async_commit();
-        }
-        int y = 0;
-        uint32_t yphase = 0;
-        for (int64_t i = 0; i < total_kb; ++i) {
-            if (i + XDIST < total_kb) fetch(i + XDIST);
-            cp_async_commit();
-            cp_async_wait<XDIST>();                      // k-block i has landed
-            if (!mbar_wait(&xq_empty[y], yphase ^ 1)) break;
-            const uint8_t* raw = smem + L.off_xraw + (int)(i % XSLOTS) * L.xraw;
-            uint8_t* xq = smem + L.off_xq + y * L.xq;
-            uint8_t* sf = smem + L.off_sfx + y * SFX;
-            // block b = (row m = b / 16, block j = b % 16 of the 256-element k-block)
-            for (int b = qt; b < np * 16; b += QT) {
-                const int m = b >> 4, j = b & 15;
-                const uint4 c0 = *reinterpret_cast<const uint4*>(raw + m * 512 + j * 32);
-                const uint4 c1 = *reinterpret_cast<const uint4*>(raw + m * 512 + j * 32 + 16);
-                const float v[16] = {bf16_lo(c0.x), bf16_hi(c0.x), bf16_lo(c0.y), bf16_hi(c0.y),
-                                     bf16_lo(c0.z), bf16_hi(c0.z), bf16_lo(c0.w), bf16_hi(c0.w),
-                                     bf16_lo(c1.x), bf16_hi(c1.x), bf16_lo(c1.y), bf16_hi(c1.y),
-                                     bf16_lo(c1.z), bf16_hi(c1.z), bf16_lo(c1.w), bf16_hi(c1.w)};
-                uint32_t byte, w[2];
-                nv_block<false>(v, sc, byte, w);
-                *reinterpret_cast<uint2*>(xq + sw128_offset(m, j * 8)) = make_uint2(w[0], w[1]);
-                sf[(j >> 2) * 512 + (m & 31) * 16 + ((m >> 5) & 3) * 4 + (j & 3)] = (uint8_t)byte;
+        uint4 ring[XDIST][2];
+#pragma unroll
+        for (int u = 0; u < XDIST; ++u) load(u, ring[u]);   // beyond nkb: zero, never used
+        uint8_t* xq_res = smem + L.off_xq;
+        uint8_t* xs_w = smem + L.off_xs;
+        for (int kb0 = 0; kb0 < nkb; kb0 += XDIST) {
+#pragma unroll
+            for (int u = 0; u < XDIST; ++u) {
+                const int kb = kb0 + u;
+                if (kb >= nkb) break;
+                const uint4 c0 = ring[u][0], c1 = ring[u][1];
+                if (kb + XDIST < nkb) load(kb + XDIST, ring[u]);
+                if (active) {
+                    const float v[16] = {bf16_lo(c0.x), bf16_hi(c0.x), bf16_lo(c0.y), bf16_hi(c0.y),
+                                         bf16_lo(c0.z), bf16_hi(c0.z), bf16_lo(c0.w), bf16_hi(c0.w),
+                                         bf16_lo(c1.x), bf16_hi(c1.x), bf16_lo(c1.y), bf16_hi(c1.y),
+                                         bf16_lo(c1.z), bf16_hi(c1.z), bf16_lo(c1.w), bf16_hi(c1.w)};
+                    uint32_t byte, w[2];
+                    nv_block<false>(v, sc, byte, w);
+                    *reinterpret_cast<uint2*>(xq_res + kb * np * 128 + sw128_offset(m, j * 8)) = make_uint2(w[0], w[1]);
+                    xs_w[((kb * 4 + (j >> 2)) * np + m) * 4 + (j & 3)] = (uint8_t)byte;
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&xres[kb]);
             }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&xq_full[y]);
-            if (++y == QSLOTS) { y = 0; yphase ^= 1; }
         }
-        cp_async_wait<0>();                              // nothing still landing at exit
     } else {
         // ---- epilogue (warps 10..13): thread = one weight row = one output column
         const int quad = warp & 3;
@@ -1560,34 +1594,35 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
         const int nacc = p.K / 64 < NACC ? (int)(p.K / 64) : NACC;   // accumulators that received an MMA
         const uint32_t qaddr = tmem + ((uint32_t)(quad * 32) << 16);
         uint32_t acc_phase = 0;
-        int stage = 0, x = 0, b = 0;
-        uint32_t phase = 0, xphase = 0, bphase = 0;
+        int stage = 0, b = 0;
+        uint32_t phase = 0, bphase = 0;
         bool ok = true;
         for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
             // Stage every k-block's weight and activation scale atoms into a TMEM
             // scale buffer with tcgen05.st (each warp fills its lane quarter
             // with the whole atom), keeping these copies off the MMA thread.
             for (int kb = 0; kb < nkb; ++kb) {
-                if (!mbar_wait(&full[stage], phase) || !mbar_wait(&xq_full[x], xphase) ||
+                if (!mbar_wait(&full[stage], phase) || !mbar_wait(&xres[kb], 0) ||
                     !mbar_wait(&sf_free[b], bphase ^ 1)) { ok = false; break; }
                 tc_fence_after();
                 const int64_t krem = p.K - (int64_t)kb * 256;
                 const int nmma = (krem < 256 ? (int)krem : 256) / 64;
                 const uint8_t* wf = smem + L.off_sfw + stage * SFW_STAGE;
-                const uint8_t* xf = smem + L.off_sfx + x * SFX;
                 const uint32_t dst = qaddr + SF_COL + b * SF_BUF;
                 for (int a = 0; a < nmma; ++a) {
+                    // the activation atom in the tensor-core layout: lane l holds rows
+                    // l, l + 32, l + 64, l + 96, of which only row l < np exists
                     const uint4 va = *reinterpret_cast<const uint4*>(wf + a * 512 + lane * 16);
-                    const uint4 vb = *reinterpret_cast<const uint4*>(xf + a * 512 + lane * 16);
+                    const uint32_t xb =
+                        lane < np ? *reinterpret_cast<const uint32_t*>(xs_res + ((kb * 4 + a) * np + lane) * 4) : 0u;
                     tmem_st4(dst + a * 4, va.x, va.y, va.z, va.w);
-                    tmem_st4(dst + 16 + a * 4, vb.x, vb.y, vb.z, vb.w);
+                    tmem_st4(dst + 16 + a * 4, xb, 0u, 0u, 0u);
                 }
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sf_ready[b]);
                 if (++stage == S) { stage = 0; phase ^= 1; }
-                if (++x == QSLOTS) { x = 0; xphase ^= 1; }
                 if (++b == SF_NBUF) { b = 0; bphase ^= 1; }
             }
             if (!ok) break;
@@ -1629,12 +1664,15 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
     if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
 }
 
+// Weight stages that fit beside the resident activations (0: the shape is not
+// taken by the fused kernel; at least 3 stages are required).
 static int decode_stages(int64_t M, int64_t K) {
-    if (M <= 0 || M > dec::MAX_M || K <= 0) return 0;
+    if (M <= 0 || M > dec::MAX_M || K <= 0 || K > (1 << 20)) return 0;
     const int np = (int)((M + 15) / 16 * 16);
+    const int nkb = (int)((K + 255) / 256);
     int stages = dec::MAX_STAGES;
-    while (stages >= 2 && decode_layout(np, stages).total > dec::MAX_SMEM) --stages;
-    return stages >= 2 ? stages : 0;
+    while (stages >= 3 && decode_layout(np, nkb, stages).total > dec::MAX_SMEM) --stages;
+    return stages >= 3 ? stages : 0;
 }
 
 bool fused_decode_supported(int64_t M, int64_t K) { return decode_stages(M, K) > 0; }
@@ -1653,7 +1691,7 @@ cudaError_t launch_fused_decode(const FusedDecodeParams& p, cudaStream_t st, int
     d.w_scales = p.b_scales; d.b_gscale = p.b_gscale; d.y = p.y;
     d.catoms = ((p.K / 16) + 3) / 4;
     d.np = np; d.nkb = nkb; d.stages = stages; d.out_bf16 = p.out_bf16 ? 1 : 0;
-    const int smem = decode_layout(np, stages).total;
+    const int smem = decode_layout(np, nkb, stages).total;
     cudaError_t e = cudaFuncSetAttribute(fused_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     const int64_t tiles = (p.N + 127) / 128;

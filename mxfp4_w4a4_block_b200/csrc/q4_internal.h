@@ -141,6 +141,8 @@ cudaError_t launch_sr_requant_grouped(GroupParams& g, int blk, bool tc, uint64_t
 cudaError_t launch_sigma_delta_banks_grouped(GroupParams& g, int blk, bool tc, int visits, cudaStream_t st,
                                              int num_sms);
 cudaError_t launch_gemm(const GemmParams& p, cudaStream_t st, int num_sms);
+// One quantized A (ps[i].M, K, a_* equal for all i) times 1..4 weights in one launch.
+cudaError_t launch_gemm_multi(const GemmParams* ps, int nw, cudaStream_t st, int num_sms);
 cudaError_t launch_fused_decode(const FusedDecodeParams& p, cudaStream_t st, int num_sms);
 
 // Reads and clears the device error words of all kernel files (bit 0: a

@@ -93,6 +93,20 @@ def test_host_validation_without_launch(lib):
     assert lib.q4_set_wait_limit(999) == 1
     assert lib.q4_set_wait_limit((1 << 40) + 1) == 1
     assert lib.q4_set_wait_limit(-5) == 1
+    # shared-A GEMM: 1..4 weights, each validated like q4_gemm
+    W = q4.Q4GemmWeight
+    one = (W * 1)(W(P, P, g, P, 64))
+    five = (W * 5)(*[W(P, P, g, P, 64) for _ in range(5)])
+    assert lib.q4_gemm_shared_a(q4.NVFP4, 16, 128, 128, P, P, g, one, 0, q4.BF16, None) == 1
+    assert lib.q4_gemm_shared_a(q4.NVFP4, 16, 128, 128, P, P, g, five, 5, q4.BF16, None) == 1
+    assert lib.q4_gemm_shared_a(q4.NVFP4, 16, 128, 128, P, P, None, one, 1, q4.BF16, None) == 1
+    bad_n = (W * 1)(W(P, P, g, P, 12))
+    assert lib.q4_gemm_shared_a(q4.NVFP4, 16, 128, 128, P, P, g, bad_n, 1, q4.BF16, None) == 3
+    no_gs = (W * 1)(W(P, P, None, P, 64))
+    assert lib.q4_gemm_shared_a(q4.NVFP4, 16, 128, 128, P, P, g, no_gs, 1, q4.BF16, None) == 1
+    mis = (W * 1)(W(P + 8, P, g, P, 64))
+    assert lib.q4_gemm_shared_a(q4.NVFP4, 16, 128, 128, P, P, g, mis, 1, q4.BF16, None) == 2
+    assert lib.q4_gemm_shared_a(q4.NVFP4, 16, 128, 96, P, P, g, one, 1, q4.BF16, None) == 3
     # no-alloc GEMM: shape bounds before anything else happens
     assert lib.q4_gemm_a_bf16_noalloc(4, (1 << 31) + 8, 64, P, g, P, P, g, q4.F32, P, None) == 3
     assert lib.q4_gemm_a_bf16_noalloc(4, 16, 96, P, g, P, P, g, q4.F32, P, None) == 3

@@ -274,3 +274,37 @@ def test_w4a16_repeatable_full_size():
     rows = np.sort(np.random.default_rng(2).choice(M, 64, replace=False))
     ref = oracle.gemm_w4a16(q4.NVFP4, synth.bf16_to_f32(d["x"]), B.o_codes, B.o_scales, B.s_t, M, N, K, rows=rows)
     assert rel_fro(ys[0][rows], ref) <= GEMM_F32_TOL
+
+
+@pytest.mark.parametrize("fmt", [q4.NVFP4, q4.MXFP4])
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_shared_a_equals_separate_gemms(fmt, out_dtype):
+    """q4_gemm_shared_a: every Y_w is bit for bit the single-weight q4_gemm
+    (same tiles, same arithmetic), with ragged M and N, a skipped N = 0 entry,
+    and the first weight also checked against the oracle."""
+    M, K = 300, 640
+    A = Operand(fmt, synth.small_like("heavy", 41, M, K))
+    Bs = [Operand(fmt, synth.small_like("weight", 50 + i, n, K)) for i, n in enumerate((264, 392, 136))]
+    ws = [(B.codes, B.scales, B.g_t, B.rows) for B in Bs]
+    ws.insert(1, (Bs[0].codes, Bs[0].scales, Bs[0].g_t, 0))
+    ys = q4.q4_gemm_shared_a(fmt, M, K, A.codes, A.scales, A.g_t, ws, out_dtype=out_dtype)
+    view = torch.int16 if out_dtype == torch.bfloat16 else torch.int32
+    for y, B in zip([ys[0]] + ys[2:], Bs):
+        ref = run_gemm(A, B, out_dtype)
+        assert torch.equal(y.view(view), ref.view(view))
+    check(ys[0], oracle_gemm(A, Bs[0]), out_dtype)
+
+
+def test_shared_a_prefill_pair_bitwise():
+    """The benchmark's step: the prefill activation (8192 x 5120) times both
+    prefill weights (N = 5120 and 17408) in one launch equals the two q4_gemm
+    calls bit for bit (each of those is held to the oracle above)."""
+    d = synth.prefill()
+    x32 = synth.bf16_to_f32(d["x"])
+    A = Operand(q4.NVFP4, x32, x_t=dev(d["x"]))
+    Bs = [Operand(q4.NVFP4, w) for w in d["w"]]
+    ys = q4.q4_gemm_shared_a(q4.NVFP4, 8192, 5120, A.codes, A.scales, A.g_t,
+                             [(B.codes, B.scales, B.g_t, B.rows) for B in Bs])
+    for y, B in zip(ys, Bs):
+        assert torch.equal(y.view(torch.int16), run_gemm(A, B, torch.bfloat16).view(torch.int16))
+    assert q4.q4_get_device_error() == 0
