@@ -90,6 +90,35 @@ def roofline_traffic(override):
         return GEMM_TRAFFIC["bytes"], f"ncu capture of the kernel built from q4_gemm.cu sha256 {cur}"
     return None, f"no capture of the current kernel (q4_gemm.cu sha256 {cur})"
 
+# Warp instructions executed by one launch of the three issue-bound grouped
+# kernels (smsp__inst_executed.sum from one ncu capture each), with the
+# SHA-256 (first 16 hex digits) of the quantizer sources they were built from;
+# a row reports its issue bound only while those files are unchanged.
+ISSUE_COUNTS = {"sources_sha256_16": "2f0ecddb833cf9bf",
+                "sr_requant_visit": 96292792, "nvfp4_quantize46_looped_weights": 50849394,
+                "sigma_delta_codebanks_K32": 239890479}
+ISSUE_SOURCES = [ROOT / "mxfp4_w4a4_block_b200" / "csrc" / n for n in ("q4_quant.cu", "q4_codec.cuh", "q4_ptx.cuh")]
+SM_CLOCK_MAX_MHZ = 1965.0      # clocks.max.sm of this B200
+ISSUE_PER_SM_CYCLE = 4         # schedulers per SM, one warp instruction each per cycle
+
+
+def issue_sources_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in ISSUE_SOURCES:
+        h.update(f.read_bytes())
+    return h.hexdigest()[:16]
+
+
+def issue_bound(row: str, us: float, n_sms: int):
+    """Issue-rate bound of an instruction-bound row: the captured warp
+    instructions over 4 per SM per cycle at the maximum SM clock."""
+    if ISSUE_COUNTS.get("sources_sha256_16") != issue_sources_hash() or row not in ISSUE_COUNTS:
+        return {"bound": "alu", "note": "no capture of the current build"}
+    t = ISSUE_COUNTS[row] / (n_sms * ISSUE_PER_SM_CYCLE * SM_CLOCK_MAX_MHZ * 1e6) * 1e6
+    return {"bound": "alu", "warp_instructions": ISSUE_COUNTS[row], "issue_bound_us": t, "frac": t / us}
+
+
 # dense FP4 over dense bf16 on B200, nominal (9 / 2.25 PFLOP/s)
 FP4_OVER_BF16 = 4.0
 
@@ -377,6 +406,7 @@ def rows_bench(q4, dev, flush, pk, reps=30):
     out = {}
     hbm = pk["hbm_gbs"]
     fp4 = pk["bf16"] * FP4_OVER_BF16
+    n_sms = torch.cuda.get_device_properties(dev).multi_processor_count
     out["tiny_linear"] = tiny_rows(q4, dev)
 
     # a3 + a5 (MXFP4): quantize X with t and Hadamard-32, GEMM with pre-quantized W'
@@ -452,6 +482,7 @@ def rows_bench(q4, dev, flush, pk, reps=30):
     out["sigma_delta_codebanks_K32"] = {"weights": nw, "visits": 32, "us": ms_cb * 1e3, "GB/s": gbs,
                                         "frac_hbm": gbs / hbm, "B_per_weight": 4 + 32 * 0.5,
                                         "vs_32_separate_visits": ms_sd * 32 / ms_cb}
+    out["sigma_delta_codebanks_K32"]["issue"] = issue_bound("sigma_delta_codebanks_K32", ms_cb * 1e3, n_sms)
     del banks
 
     q46_c = [torch.empty_like(c) for c in gC]
@@ -463,6 +494,7 @@ def rows_bench(q4, dev, flush, pk, reps=30):
     gbs = nw * (4 + 0.5 + 1 / 16) / (ms_46 * 1e-3) / 1e9
     out["nvfp4_quantize46_looped_weights"] = {"weights": nw, "matrices": 13, "us": ms_46 * 1e3, "GB/s": gbs,
                                               "frac_hbm": gbs / hbm}
+    out["nvfp4_quantize46_looped_weights"]["issue"] = issue_bound("nvfp4_quantize46_looped_weights", ms_46 * 1e3, n_sms)
     del q46_c, q46_s
 
     def sr_visit():
@@ -470,6 +502,7 @@ def rows_bench(q4, dev, flush, pk, reps=30):
     ms_sr, _ = time_fn(sr_visit, reps, flush)
     gbs = nw * B_SR / (ms_sr * 1e-3) / 1e9
     out["sr_requant_visit"] = {"weights": nw, "matrices": 13, "us": ms_sr * 1e3, "GB/s": gbs, "frac_hbm": gbs / hbm}
+    out["sr_requant_visit"]["issue"] = issue_bound("sr_requant_visit", ms_sr * 1e3, n_sms)
     # a decode-shaped visit (M = 16) with the Sigma-Delta codes generated inside the
     # GEMM producer, against the same visit as a separate step + W4A16 GEMM
     xd16 = xl[:16].contiguous()

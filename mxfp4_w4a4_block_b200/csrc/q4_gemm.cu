@@ -1362,18 +1362,23 @@ cudaError_t launch_sd_gemm_grouped(const SdGemmParams* items, int count, cudaStr
 //               traffic);
 //   warp 1      TMEM owner and MMA issuer: per k-block up to four
 //               128 x np x 64 block-scaled MMAs into four accumulators;
-//   warps 2..9  fetch the bf16 activations k-block by k-block (cp.async, a
-//               few k-blocks ahead) and quantize them in shared memory (codes
-//               into the swizzled K-major operand layout, scales into
-//               tensor-core atoms) while the weight tiles stream in;
-//   warps 10-13 stage each k-block's weight and activation scale atoms into
+//   warp 2      TMA producer of the bf16 activations: one 2-D tile of M rows
+//               x 256 elements per k-block into a ring of its own, as deep as
+//               shared memory allows, so their loads never queue behind one
+//               another (a register-staged load a few k-blocks ahead waited
+//               out the latency of the weight stream in flight at each step);
+//   warps 3..10 quantize the landed activation tiles once per CTA into a
+//               resident buffer (codes in the swizzled K-major operand layout,
+//               scales packed per k-block) while the weight tiles stream in;
+//   warps 11-14 stage each k-block's weight and activation scale atoms into
 //               TMEM (tcgen05.st, off the MMA thread: a tcgen05.cp there would
 //               queue with the MMAs), then run the epilogue: the summed
 //               accumulator lanes (= output columns), times alpha, to Y.
 namespace dec {
 constexpr int QWARPS = 8;
 constexpr int EWARPS = 4;
-constexpr int FIRST_Q = 2;
+constexpr int XWARP = 2;                 // TMA producer of the bf16 activation tiles
+constexpr int FIRST_Q = 3;
 constexpr int FIRST_E = FIRST_Q + QWARPS;
 constexpr int THREADS = 32 * (FIRST_E + EWARPS);
 constexpr int W_STAGE = 128 * 128;       // weight codes of one k-block
@@ -1381,10 +1386,13 @@ constexpr int SFW_STAGE = 4 * 512;       // their scale atoms
 // The activations are quantized once per CTA into a resident buffer (codes in
 // the swizzled K-major operand layout, one 16-row x 128-byte tile per k-block,
 // and the block scales packed per k-block), so the activation path never waits
-// on the MMAs and CTAs with more than one weight tile reuse it; the rest of
-// shared memory is the weight ring.
-constexpr int XDIST = 4;                // k-blocks of activations loaded ahead, in registers
+// on the MMAs and CTAs with more than one weight tile reuse it.  The bf16 tiles
+// it is made from land by TMA in a ring of XS stages; the rest of shared memory
+// is the weight ring.
 constexpr int MAX_M = 16;
+constexpr int X_ROW = 512;               // bytes of one activation row of a k-block (256 bf16)
+constexpr int X_STAGE = MAX_M * X_ROW;   // one k-block of activations
+constexpr int MAX_XS = 8;
 constexpr int MAX_STAGES = 12;
 constexpr uint32_t TMEM_COLS = 256;
 constexpr int NACC = 4;                  // independent accumulators (MMA kk of a k-block -> accumulator kk)
@@ -1393,7 +1401,8 @@ constexpr uint32_t SF_COL = 128;         // SF_NBUF scale buffers of SF_BUF colu
 constexpr uint32_t SF_BUF = 32;          //   weight atoms x 4 columns, then activation atoms x 4
 constexpr int SF_NBUF = 4;
 constexpr int MAX_SMEM = 232448;         // 227 KB opt-in limit per CTA
-constexpr int FIXED_BARS = 40;        // ring, scale-buffer, TMEM and done barriers (<= 40)
+constexpr int FIXED_BARS = 56;           // weight ring 2 x 12, scale buffers 2 x 4, TMEM and done 3,
+                                         // the TMEM holder's slot, activation ring 2 x 8 (<= 56)
 }  // namespace dec
 
 struct DecodeDev {
@@ -1406,7 +1415,8 @@ struct DecodeDev {
     int64_t catoms;
     int np;           // MMA N: M rounded up to 16
     int nkb;          // k-blocks of 256
-    int stages;
+    int stages;       // weight ring depth
+    int xs;           // activation ring depth
     int out_bf16;
 };
 
@@ -1416,19 +1426,21 @@ __device__ __forceinline__ uint32_t sw128_offset(int row, int byte_in_row) {
 }
 
 struct DecodeLayout {
-    int off_w, off_sfw, off_xq, off_xs, off_bar, off_tab, total;
+    int off_w, off_sfw, off_xq, off_x, off_xs, off_bar, off_tab, total;
 };
 
 // Weight ring (S stages of codes and scale atoms), the resident activation codes
-// (nkb tiles of np x 128 bytes) and scales (nkb x 4 atoms x np rows x 4 bytes),
-// the barriers (the fixed ones, then one per k-block of activations) and the
-// 128-entry (S, 1/S) table.
-__host__ __device__ inline DecodeLayout decode_layout(int np, int nkb, int stages) {
+// (nkb tiles of np x 128 bytes), the activation ring (XS bf16 tiles), the
+// resident activation scales (nkb x 4 atoms x np rows x 4 bytes), the barriers
+// (the fixed ones, then one per k-block of activations) and the 128-entry
+// (S, 1/S) table.
+__host__ __device__ inline DecodeLayout decode_layout(int np, int nkb, int stages, int xs) {
     DecodeLayout L;
     L.off_w = 0;
     L.off_sfw = L.off_w + stages * dec::W_STAGE;
     L.off_xq = L.off_sfw + stages * dec::SFW_STAGE;        // 1024-aligned: both stage sizes are
-    L.off_xs = L.off_xq + nkb * np * 128;
+    L.off_x = L.off_xq + nkb * np * 128;                   // 1024-aligned: np * 128 = 2048
+    L.off_xs = L.off_x + xs * dec::X_STAGE;
     L.off_bar = L.off_xs + nkb * 16 * np;
     L.off_tab = (L.off_bar + 8 * (dec::FIXED_BARS + nkb) + 15) / 16 * 16;
     L.total = L.off_tab + 128 * 8 + 1024;                   // + alignment slack
@@ -1436,12 +1448,13 @@ __host__ __device__ inline DecodeLayout decode_layout(int np, int nkb, int stage
 }
 
 __global__ void __launch_bounds__(dec::THREADS, 1)
-    fused_decode_kernel(const __grid_constant__ CUtensorMap tmW, DecodeDev p) {
+    fused_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                        DecodeDev p) {
     using namespace dec;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int np = p.np, nkb = p.nkb, S = p.stages;
-    const DecodeLayout L = decode_layout(np, nkb, S);
+    const int np = p.np, nkb = p.nkb, S = p.stages, XS = p.xs;
+    const DecodeLayout L = decode_layout(np, nkb, S, XS);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.off_bar);   // [S] weight tile landed
     uint64_t* empty = full + MAX_STAGES;                               // [S] its MMAs are done
     uint64_t* sf_ready = empty + MAX_STAGES;                           // [SF_NBUF] scales staged in TMEM buffer
@@ -1450,6 +1463,8 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
     uint64_t* tmem_empty = tmem_full + 1;
     uint64_t* mma_done = tmem_empty + 1;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
+    uint64_t* xfull = mma_done + 2;                                    // [XS] activation tile landed
+    uint64_t* xempty = xfull + MAX_XS;                                 // [XS] its values are quantized
     uint64_t* xres = reinterpret_cast<uint64_t*>(smem + L.off_bar) + FIXED_BARS;   // [nkb] activations ready
     float2* nv_tab = reinterpret_cast<float2*>(smem + L.off_tab);      // 128 (S, 1/S) entries
     const uint8_t* xs_res = smem + L.off_xs;                           // packed activation scales
@@ -1458,6 +1473,7 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
         for (int kb = 0; kb < nkb; ++kb) mbar_init(&xres[kb], QWARPS);
+        for (int s = 0; s < XS; ++s) { mbar_init(&xfull[s], 1); mbar_init(&xempty[s], QWARPS); }
         for (int b = 0; b < SF_NBUF; ++b) { mbar_init(&sf_ready[b], EWARPS); mbar_init(&sf_free[b], 1); }
         mbar_init(tmem_full, 1);
         mbar_init(tmem_empty, EWARPS);
@@ -1466,6 +1482,7 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
     }
     if (warp == 1) { tmem_alloc(tmem_holder, TMEM_COLS); tmem_relinquish(); }
     if (warp == 0 && lane == 0) tma_prefetch_desc(&tmW);
+    if (warp == XWARP && lane == 0) tma_prefetch_desc(&tmX);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -1537,58 +1554,73 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
             tc_commit(mma_done);
             mbar_wait(mma_done, 0);
         }
+    } else if (warp == XWARP) {
+        // ---- activation tiles (M rows x 256 bf16 per k-block), once per CTA
+        if (lane == 0) {
+            const uint32_t xbytes = (uint32_t)p.M * (uint32_t)X_ROW;   // the box: M rows x 256 elements
+            int s = 0;
+            uint32_t ph = 0;
+            uint32_t last_phase[MAX_XS];
+            bool issued[MAX_XS];
+            for (int i = 0; i < MAX_XS; ++i) issued[i] = false, last_phase[i] = 0;
+            for (int kb = 0; kb < nkb; ++kb) {
+                if (!mbar_wait(&xempty[s], ph ^ 1)) break;
+                mbar_arrive_expect_tx(&xfull[s], xbytes);
+                tma_load_2d(smem + L.off_x + s * X_STAGE, &tmX, &xfull[s], kb * 256, 0);
+                issued[s] = true;
+                last_phase[s] = ph;
+                if (++s == XS) { s = 0; ph ^= 1; }
+            }
+            // no copy may still be landing in shared memory when the CTA exits
+            for (int i = 0; i < XS; ++i)
+                if (issued[i]) mbar_wait(&xfull[i], last_phase[i]);
+        }
     } else if (warp < FIRST_E) {
-        // ---- quantize the activations (warps 2..9), once per CTA
+        // ---- quantize the activations (warps 3..10), once per CTA
         const int qt = threadIdx.x - 32 * FIRST_Q;
         constexpr int QT = 32 * QWARPS;
         const NvCtx sc = nv_ctx(*p.a_gscale, nv_tab);
         nv_fill_table(*p.a_gscale, nv_tab, qt, QT);
         named_barrier(1, QT);
         // Thread qt owns block (row m = qt / 16, block j = qt % 16) of every
-        // k-block (np * 16 <= QT blocks per k-block); its 32 input bytes are
-        // loaded XDIST k-blocks ahead into registers (rows and columns outside X
-        // read as zero), then quantized into the resident codes and scales.
+        // k-block (np * 16 <= QT blocks per k-block): its 32 bytes of the landed
+        // tile (rows at or beyond M and columns beyond K are zero) are quantized
+        // into the resident codes and scales; the tile goes back to the producer
+        // once every warp has used what it read (and the k-block is ready).
         const int m = qt >> 4, j = qt & 15;
         const bool active = qt < np * 16;
-        const uint16_t* xrow = p.x + (int64_t)m * p.K;
-        auto load = [&](int kb, uint4 (&r)[2]) {
-            const int64_t k = (int64_t)kb * 256 + j * 16;
-            if (active && m < p.M && k < p.K) {
-                r[0] = __ldg(reinterpret_cast<const uint4*>(xrow + k));
-                r[1] = __ldg(reinterpret_cast<const uint4*>(xrow + k + 8));
-            } else {
-                r[0] = r[1] = make_uint4(0u, 0u, 0u, 0u);
-            }
-        };
-        uint4 ring[XDIST][2];
-#pragma unroll
-        for (int u = 0; u < XDIST; ++u) load(u, ring[u]);   // beyond nkb: zero, never used
         uint8_t* xq_res = smem + L.off_xq;
         uint8_t* xs_w = smem + L.off_xs;
-        for (int kb0 = 0; kb0 < nkb; kb0 += XDIST) {
-#pragma unroll
-            for (int u = 0; u < XDIST; ++u) {
-                const int kb = kb0 + u;
-                if (kb >= nkb) break;
-                const uint4 c0 = ring[u][0], c1 = ring[u][1];
-                if (kb + XDIST < nkb) load(kb + XDIST, ring[u]);
-                if (active) {
-                    const float v[16] = {bf16_lo(c0.x), bf16_hi(c0.x), bf16_lo(c0.y), bf16_hi(c0.y),
-                                         bf16_lo(c0.z), bf16_hi(c0.z), bf16_lo(c0.w), bf16_hi(c0.w),
-                                         bf16_lo(c1.x), bf16_hi(c1.x), bf16_lo(c1.y), bf16_hi(c1.y),
-                                         bf16_lo(c1.z), bf16_hi(c1.z), bf16_lo(c1.w), bf16_hi(c1.w)};
-                    uint32_t byte, w[2];
-                    nv_block<false>(v, sc, byte, w);
-                    *reinterpret_cast<uint2*>(xq_res + kb * np * 128 + sw128_offset(m, j * 8)) = make_uint2(w[0], w[1]);
-                    xs_w[((kb * 4 + (j >> 2)) * np + m) * 4 + (j & 3)] = (uint8_t)byte;
+        int s = 0;
+        uint32_t ph = 0;
+        for (int kb = 0; kb < nkb; ++kb) {
+            if (!mbar_wait(&xfull[s], ph)) break;
+            if (active) {
+                uint4 c0 = make_uint4(0u, 0u, 0u, 0u), c1 = c0;
+                if (m < p.M) {
+                    const uint8_t* src = smem + L.off_x + s * X_STAGE + m * X_ROW + j * 32;
+                    c0 = *reinterpret_cast<const uint4*>(src);
+                    c1 = *reinterpret_cast<const uint4*>(src + 16);
                 }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&xres[kb]);
+                const float v[16] = {bf16_lo(c0.x), bf16_hi(c0.x), bf16_lo(c0.y), bf16_hi(c0.y),
+                                     bf16_lo(c0.z), bf16_hi(c0.z), bf16_lo(c0.w), bf16_hi(c0.w),
+                                     bf16_lo(c1.x), bf16_hi(c1.x), bf16_lo(c1.y), bf16_hi(c1.y),
+                                     bf16_lo(c1.z), bf16_hi(c1.z), bf16_lo(c1.w), bf16_hi(c1.w)};
+                uint32_t byte, w[2];
+                nv_block<false>(v, sc, byte, w);
+                *reinterpret_cast<uint2*>(xq_res + kb * np * 128 + sw128_offset(m, j * 8)) = make_uint2(w[0], w[1]);
+                xs_w[((kb * 4 + (j >> 2)) * np + m) * 4 + (j & 3)] = (uint8_t)byte;
             }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&xempty[s]);
+                mbar_arrive(&xres[kb]);
+            }
+            if (++s == XS) { s = 0; ph ^= 1; }
         }
     } else {
-        // ---- epilogue (warps 10..13): thread = one weight row = one output column
+        // ---- epilogue (warps 11..14): thread = one weight row = one output column
         const int quad = warp & 3;
         const float alpha = __fmul_rn(*p.a_gscale, *p.b_gscale);
         const int nacc = p.K / 64 < NACC ? (int)(p.K / 64) : NACC;   // accumulators that received an MMA
@@ -1664,39 +1696,68 @@ __global__ void __launch_bounds__(dec::THREADS, 1)
     if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
 }
 
-// Weight stages that fit beside the resident activations (0: the shape is not
-// taken by the fused kernel; at least 3 stages are required).
-static int decode_stages(int64_t M, int64_t K) {
-    if (M <= 0 || M > dec::MAX_M || K <= 0 || K > (1 << 20)) return 0;
+// Ring depths that fit beside the resident activations: the deepest activation
+// ring of 8, 4 or 2 tiles that leaves at least 4 (8) or 3 (4, 2) weight stages,
+// with as many weight stages as then fit.  False: the shape is not taken by the
+// fused kernel (K below one k-block of 256, M above 16, or K so long that the
+// resident activations leave no room).
+static bool decode_config(int64_t M, int64_t K, int* stages, int* xs) {
+    if (M <= 0 || M > dec::MAX_M || K < 256 || K > (1 << 20)) return false;
     const int np = (int)((M + 15) / 16 * 16);
     const int nkb = (int)((K + 255) / 256);
-    int stages = dec::MAX_STAGES;
-    while (stages >= 3 && decode_layout(np, nkb, stages).total > dec::MAX_SMEM) --stages;
-    return stages >= 3 ? stages : 0;
+    const int cand[3][2] = {{8, 4}, {4, 3}, {2, 3}};
+    for (const auto& c : cand) {
+        int st = dec::MAX_STAGES;
+        while (st >= c[1] && decode_layout(np, nkb, st, c[0]).total > dec::MAX_SMEM) --st;
+        if (st >= c[1]) {
+            *stages = st;
+            *xs = c[0];
+            return true;
+        }
+    }
+    return false;
 }
 
-bool fused_decode_supported(int64_t M, int64_t K) { return decode_stages(M, K) > 0; }
+bool fused_decode_supported(int64_t M, int64_t K) {
+    int st, xs;
+    return decode_config(M, K, &st, &xs);
+}
+
+// bf16 activations [M, K] for TMA tiles of M rows x 256 elements (no swizzle).
+static bool make_act_map(CUtensorMap* map, const void* x, int64_t M, int64_t K) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+    cuuint64_t strides[1] = {(cuuint64_t)(K * 2)};
+    cuuint32_t box[2] = {256u, (cuuint32_t)M};
+    cuuint32_t es[2] = {1u, 1u};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
 
 cudaError_t launch_fused_decode(const FusedDecodeParams& p, cudaStream_t st, int num_sms) {
     using namespace dec;
     if (p.M == 0 || p.N == 0) return cudaSuccess;
     const int np = (int)((p.M + 15) / 16 * 16);
     const int nkb = (int)((p.K + 255) / 256);
-    const int stages = decode_stages(p.M, p.K);
-    if (stages == 0) return cudaErrorNotSupported;
-    CUtensorMap mw;
+    int stages = 0, xs = 0;
+    if (!decode_config(p.M, p.K, &stages, &xs)) return cudaErrorNotSupported;
+    CUtensorMap mw, mx;
     if (!make_code_map(&mw, p.b_codes, p.N, p.K / 2, 128)) return cudaErrorInvalidValue;
+    if (!make_act_map(&mx, p.a_bf16, p.M, p.K)) return cudaErrorInvalidValue;
     DecodeDev d;
     d.M = p.M; d.N = p.N; d.K = p.K; d.x = p.a_bf16; d.a_gscale = p.a_gscale;
     d.w_scales = p.b_scales; d.b_gscale = p.b_gscale; d.y = p.y;
     d.catoms = ((p.K / 16) + 3) / 4;
-    d.np = np; d.nkb = nkb; d.stages = stages; d.out_bf16 = p.out_bf16 ? 1 : 0;
-    const int smem = decode_layout(np, nkb, stages).total;
+    d.np = np; d.nkb = nkb; d.stages = stages; d.xs = xs; d.out_bf16 = p.out_bf16 ? 1 : 0;
+    const int smem = decode_layout(np, nkb, stages, xs).total;
     cudaError_t e = cudaFuncSetAttribute(fused_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     const int64_t tiles = (p.N + 127) / 128;
     const int grid = (int)(tiles < num_sms ? tiles : num_sms);
-    fused_decode_kernel<<<grid, THREADS, smem, st>>>(mw, d);
+    fused_decode_kernel<<<grid, THREADS, smem, st>>>(mw, mx, d);
     return cudaGetLastError();
 }
 
