@@ -71,7 +71,7 @@ def peaks():
 # 17408) x 5120) from one ncu capture, with
 # the SHA-256 (first 16 hex digits) of the GEMM source file it was built from:
 # the bench reports the figure only while that file is unchanged.
-GEMM_TRAFFIC = {"bytes": 92746496 + 327137024, "source_sha256_16": "a379a113f7001dc6"}
+GEMM_TRAFFIC = {"bytes": 92923136 + 325975808, "source_sha256_16": "ae6a7400766f27ac"}
 GEMM_SOURCE = ROOT / "mxfp4_w4a4_block_b200" / "csrc" / "q4_gemm.cu"
 
 
@@ -713,6 +713,14 @@ def run_ours(args):
 
     cpu = None if args.no_cpu_baseline or rank != 0 else cpu_baseline(budget_s=args.cpu_seconds)
     traffic, traffic_note = roofline_traffic(args.traffic)
+    # a timed region of a second or more runs the GEMM under the power cap: its
+    # peak is then the sustained (seconds-long loop) figure, else the burst one
+    fp4_sus = pk["bf16_sus"] * FP4_OVER_BF16
+    sustained = wall >= 1.0
+    fp4_peak = fp4_sus if sustained else fp4_burst
+    peak_note = (f"dense FP4 = {pk['src']} bf16 {'sustained' if sustained else 'burst'} "
+                 f"{pk['bf16_sus'] if sustained else pk['bf16']} x 4 (nominal 9/2.25); "
+                 f"{'sustained' if sustained else 'burst'}: the timed region lasted {wall:.2f} s")
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -723,9 +731,10 @@ def run_ours(args):
                    "parallelism": f"replicas x{world} (independent problems per GPU)"},
         "roofline": {"kernel": "gemm_kernel<NVFP4>, one launch over W1 and W2: 8192 x (5120 + 17408) x 5120",
                      "bound": "tensor", "achieved": gemm_tf,
-                     "peak": fp4_burst, "unit": "TFLOP/s", "frac": gemm_tf / fp4_burst,
-                     "peak_note": f"dense FP4 = {pk['src']} bf16 burst {pk['bf16']} x 4 (nominal 9/2.25)",
-                     "frac_vs_sustained": gemm_tf / (pk["bf16_sus"] * FP4_OVER_BF16),
+                     "peak": fp4_peak, "unit": "TFLOP/s", "frac": gemm_tf / fp4_peak,
+                     "peak_note": peak_note,
+                     "frac_vs_burst": gemm_tf / fp4_burst,
+                     "frac_vs_sustained": gemm_tf / fp4_sus,
                      "traffic": traffic, "traffic_note": traffic_note,
                      "algorithmic_bytes": M * K / 2 + M * K / 16 + (N1 + N2) * K * (0.5 + 1 / 16) + 2 * M * (N1 + N2)},
         "cpu_baseline": cpu,
