@@ -71,13 +71,20 @@ def peaks():
 # 17408) x 5120) from one ncu capture, with
 # the SHA-256 (first 16 hex digits) of the GEMM source file it was built from:
 # the bench reports the figure only while that file is unchanged.
-GEMM_TRAFFIC = {"bytes": 92923136 + 325975808, "source_sha256_16": "ae6a7400766f27ac"}
+GEMM_TRAFFIC = {"bytes": 92923136 + 325975808, "source_sha256_16": "4aa354952cce7c86"}
 GEMM_SOURCE = ROOT / "mxfp4_w4a4_block_b200" / "csrc" / "q4_gemm.cu"
 
 
 def gemm_source_hash() -> str:
+    """SHA-256 (16 hex digits) of what the roofline GEMM is built from: the W4A4
+    GEMM section of q4_gemm.cu (from its namespace to the W4A16 section) and the
+    PTX wrapper header."""
     import hashlib
-    return hashlib.sha256(GEMM_SOURCE.read_bytes()).hexdigest()[:16]
+    text = GEMM_SOURCE.read_text()
+    a, b = text.index("namespace gemm {"), text.index("// ------------------------------------------------------------------ W4A16")
+    h = hashlib.sha256(text[a:b].encode())
+    h.update((GEMM_SOURCE.parent / "q4_ptx.cuh").read_bytes())
+    return h.hexdigest()[:16]
 
 
 def roofline_traffic(override):
@@ -87,8 +94,8 @@ def roofline_traffic(override):
         return override, "given on the command line"
     cur = gemm_source_hash()
     if GEMM_TRAFFIC["bytes"] is not None and GEMM_TRAFFIC["source_sha256_16"] == cur:
-        return GEMM_TRAFFIC["bytes"], f"ncu capture of the kernel built from q4_gemm.cu sha256 {cur}"
-    return None, f"no capture of the current kernel (q4_gemm.cu sha256 {cur})"
+        return GEMM_TRAFFIC["bytes"], f"ncu capture of the kernel built from the GEMM source with sha256 {cur}"
+    return None, f"no capture of the current kernel (GEMM source sha256 {cur})"
 
 # Warp instructions executed by one launch of the three issue-bound grouped
 # kernels (smsp__inst_executed.sum from one ncu capture each), with the
@@ -355,6 +362,9 @@ def tiny_rows(q4, dev, reps=200):
     _, sw = q4.q4_quantize(q4.NVFP4, w, gscale=gw, flags=q4.SCALE_RU | q4.LAYOUT_TC)
     r = torch.zeros_like(w)
     cw = torch.empty((512, 256), dtype=torch.uint8, device=dev)
+    ax4 = torch.zeros(4, dtype=torch.float32, device=dev)
+    aw4 = torch.zeros(4, dtype=torch.float32, device=dev)
+    banks8 = torch.empty((8, 512, 256), dtype=torch.uint8, device=dev)
 
     def linear():
         q4.q4_amax(x, 2688.0, out=ax)
@@ -363,10 +373,18 @@ def tiny_rows(q4, dev, reps=200):
         q4.q4_quantize(q4.NVFP4, w, gscale=aw[1:2], codes=wc, scales=ws)
         q4.q4_gemm(q4.NVFP4, 64, 512, 512, xc, xs, ax[1:2], wc, ws, aw[1:2], y=y)
 
+    def linear_fused():
+        q4.q4_amax_quantize(x, 2688.0, out=ax4, codes=xc, scales=xs)
+        q4.q4_amax_quantize(w, 2688.0, out=aw4, codes=wc, scales=ws)
+        q4.q4_gemm(q4.NVFP4, 64, 512, 512, xc, xs, ax4[1:2], wc, ws, aw4[1:2], y=y)
+
     def chain8():
         r.zero_()
         for _ in range(8):
             q4.q4_sigma_delta_step(q4.NVFP4, w, sw, r, gscale=gw, codes=cw)
+
+    def chain8_banks():
+        q4.q4_sigma_delta_codebanks(q4.NVFP4, w, sw, 8, gscale=gw, codes=banks8)
 
     def per_call(fn):
         for _ in range(10):
@@ -381,8 +399,13 @@ def tiny_rows(q4, dev, reps=200):
         return s.elapsed_time(e) * 1e3 / reps
 
     out = {"linear_us": per_call(linear), "sigma_delta_R8_us": per_call(chain8),
-           "launches": {"linear": 5, "sigma_delta_R8": 9}, "l2": "warm (latency row)"}
-    for name, fn in (("linear", linear), ("sigma_delta_R8", chain8)):
+           "linear_fused_us": per_call(linear_fused), "sigma_delta_R8_banks_us": per_call(chain8_banks),
+           "launches": {"linear": 5, "linear_fused": 3, "sigma_delta_R8": 9, "sigma_delta_R8_banks": 1},
+           "note": "linear_fused: amax and quantize of each operand in one cooperative launch; "
+                   "sigma_delta_R8_banks: the 8-visit chain as one codebank launch (same codes)",
+           "l2": "warm (latency row)"}
+    for name, fn in (("linear", linear), ("sigma_delta_R8", chain8), ("linear_fused", linear_fused),
+                     ("sigma_delta_R8_banks", chain8_banks)):
         try:
             g = torch.cuda.CUDAGraph()
             st = torch.cuda.Stream()

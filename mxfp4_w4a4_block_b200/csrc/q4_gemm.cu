@@ -954,7 +954,9 @@ cudaError_t launch_w4a16(const W4A16Params& p, cudaStream_t st, int num_sms) {
 // the MMA's 128-row side (tcgen05 kind::f16, 128 x 16 x 16).
 // A CTA owns 128 weight rows and one slice of K; the KS slices of a row band
 // form a thread-block cluster whose partial outputs are summed through
-// distributed shared memory by the cluster's first CTA:
+// distributed shared memory by the cluster's first CTA.  A CTA holds one
+// 85 KB stage, so two CTAs share an SM and one's set-up, first loads and
+// reduction overlap the other's stream:
 //   warp 0      TMA producer: per k-stage of 64 the W and r tiles (two
 //               128-row x 128-byte boxes each, 128-byte swizzle), the block
 //               scale atom and the X tile (np rows x 128 bytes, swizzled);
@@ -967,7 +969,7 @@ cudaError_t launch_w4a16(const W4A16Params& p, cudaStream_t st, int num_sms) {
 namespace sdg {
 constexpr int BM = 128;
 constexpr int KSTAGE = 64;
-constexpr int STAGES = 2;
+constexpr int STAGES = 1;                // per CTA; two CTAs share an SM
 constexpr int OFF_W = 0;                 // 2 boxes x 16 KB fp32
 constexpr int OFF_R = 32768;             // 2 boxes x 16 KB fp32
 constexpr int OFF_A = 65536;             // 128 x 128 B bf16 operand
@@ -1045,7 +1047,7 @@ __device__ __forceinline__ void sd_gemm_cta(const CUtensorMap& tmW, const CUtens
             uint32_t phase = 0;
             int stage = 0;
             uint32_t last_phase[STAGES];
-            bool issued[STAGES] = {false, false};
+            bool issued[STAGES] = {};
             for (int i = 0; i < nst; ++i) {
                 if (!mbar_wait(&empty[stage], phase ^ 1)) break;
                 uint8_t* st = smem + stage * STAGE;
@@ -1215,7 +1217,7 @@ __device__ __forceinline__ void sd_gemm_cta(const CUtensorMap& tmW, const CUtens
     if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
 }
 
-__global__ void __launch_bounds__(sdg::THREADS, 1)
+__global__ void __launch_bounds__(sdg::THREADS, 2)
     sd_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmR,
                           const __grid_constant__ CUtensorMap tmX, SdgDev p) {
     sd_gemm_cta(tmW, tmR, tmX, p, (int64_t)blockIdx.y);
@@ -1235,7 +1237,7 @@ struct SdgGroup {
 };
 static_assert(sizeof(SdgGroup) <= 32764, "kernel parameter space");
 
-__global__ void __launch_bounds__(sdg::THREADS, 1) sd_gemm_grouped_kernel(const __grid_constant__ SdgGroup g) {
+__global__ void __launch_bounds__(sdg::THREADS, 2) sd_gemm_grouped_kernel(const __grid_constant__ SdgGroup g) {
     int e = 0;
     while (e + 1 < g.count && (int)blockIdx.y >= g.band_start[e + 1]) ++e;
     const SdgItem& it = g.m[e];
@@ -1245,19 +1247,20 @@ __global__ void __launch_bounds__(sdg::THREADS, 1) sd_gemm_grouped_kernel(const 
 bool sd_gemm_supported(int64_t M, int64_t K) { return M >= 1 && M <= 16 && K % 64 == 0 && K > 0; }
 
 // K slices per row band (the cluster size, 1 to 8, dividing K into 64-element
-// stages) for `bands` row bands on `num_sms` SMs (one CTA per SM at a time):
+// stages) for `bands` row bands on `num_sms` SMs (two CTAs per SM at a time):
 // the one with the least estimated time waves * (T0 + stages per CTA * TS),
 // T0 ~ 8 us the fixed cost of a CTA (set-up, first loads, cluster reduction)
-// and TS ~ 1.9 us a pipelined 64-element stage, both measured on the
-// looped-core shapes (K = 1024: splits 1 / 2 / 4 / 8 took 118 / 120 / 155 /
-// 261 us for 320 bands).
+// and TS ~ 1.9 us a 64-element stage, both measured on the looped-core shapes
+// with one two-stage CTA per SM (K = 1024: splits 1 / 2 / 4 / 8 took 118 /
+// 120 / 155 / 261 us for 320 bands).  One single-stage CTA beside another on
+// the same SM overlaps one CTA's set-up and reduction with the other's stream.
 static int choose_ksplit(int64_t bands, int64_t K, int num_sms) {
     constexpr double T0 = 8.0, TS = 1.9;
     int best_ks = 1;
     double best_t = 1e300;
     for (int ks = 1; ks <= sdg::MAX_KS; ks *= 2) {
         if (K % (64 * ks)) break;
-        const double waves = std::ceil((double)(bands * ks) / num_sms);
+        const double waves = std::ceil((double)(bands * ks) / (2 * num_sms));
         const double t = waves * (T0 + (double)(K / ks / 64) * TS);
         if (t < best_t) { best_t = t; best_ks = ks; }
     }
