@@ -1355,7 +1355,7 @@ cudaError_t launch_sd_gemm_grouped(const SdGemmParams* items, int count, cudaStr
 }
 
 // ------------------------------------------------------------------ fused decode
-// Small-M GEMM (M <= 64) with the activation quantization inside the kernel:
+// Small-M GEMM (M <= 16) with the activation quantization inside the kernel:
 // no bf16 activation round trip and no workspace.  Operands are swapped so the
 // weight fills the MMA's 128-row side: D^T[n, m] = sum_k W[n, k] X[m, k], with
 // MMA N = np (M rounded up to 16).  Persistent CTAs over 128-row weight tiles:
@@ -1410,7 +1410,6 @@ constexpr int FIXED_BARS = 56;           // weight ring 2 x 12, scale buffers 2 
 
 struct DecodeDev {
     int64_t M, N, K;
-    const uint16_t* x;       // bf16 activations [M, K]
     const float* a_gscale;
     const uint8_t* w_scales;
     const float* b_gscale;
@@ -1751,7 +1750,7 @@ cudaError_t launch_fused_decode(const FusedDecodeParams& p, cudaStream_t st, int
     if (!make_code_map(&mw, p.b_codes, p.N, p.K / 2, 128)) return cudaErrorInvalidValue;
     if (!make_act_map(&mx, p.a_bf16, p.M, p.K)) return cudaErrorInvalidValue;
     DecodeDev d;
-    d.M = p.M; d.N = p.N; d.K = p.K; d.x = p.a_bf16; d.a_gscale = p.a_gscale;
+    d.M = p.M; d.N = p.N; d.K = p.K; d.a_gscale = p.a_gscale;
     d.w_scales = p.b_scales; d.b_gscale = p.b_gscale; d.y = p.y;
     d.catoms = ((p.K / 16) + 3) / 4;
     d.np = np; d.nkb = nkb; d.stages = stages; d.xs = xs; d.out_bf16 = p.out_bf16 ? 1 : 0;
