@@ -56,6 +56,9 @@ def test_scale_bytes(lib):
 def test_workspace_size(lib):
     import mxfp4_w4a4_block_b200 as q4
     assert q4.q4_gemm_workspace_size(q4.NVFP4, 16, 17408, 5120, q4.A_BF16) == 0
+    # below one 256-element k-block the activations are quantized once into the workspace
+    # (codes 5 x 96 bytes rounded up to 256, then one 128-row band of three 512-byte scale atoms)
+    assert q4.q4_gemm_workspace_size(q4.NVFP4, 5, 392, 192, q4.A_BF16) == 512 + 3 * 512
     assert q4.q4_gemm_workspace_size(q4.NVFP4, 8192, 5120, 5120, q4.A_QUANTIZED) == 0
     ws = q4.q4_gemm_workspace_size(q4.NVFP4, 8192, 5120, 5120, q4.A_BF16)
     assert ws == 8192 * 2560 + 8192 * 320

@@ -97,11 +97,12 @@ def test_gemm_closed_form_integer_case():
     assert np.all(y == K * 0.5)
 
 
-@pytest.mark.parametrize("M,K", [(1, 1088), (16, 1088), (33, 1216), (64, 1152), (65, 1088), (128, 1088)])
+@pytest.mark.parametrize("M,K", [(1, 1088), (16, 1088), (33, 1216), (64, 1152), (65, 1088), (128, 1088), (5, 192)])
 def test_fused_activation_quant_decode_small(M, K):
     """a_kind = A_BF16 for small M: the GEMM launch quantizes the bf16
-    activations itself (M <= 16; larger M quantizes once into the workspace).
-    K leaves partial last k-blocks of 64, 192 and 128 elements; N a partial tile."""
+    activations itself (M <= 16 and K of at least one 256-element k-block;
+    larger M, or K = 192, quantizes once into the workspace).  K leaves partial
+    last k-blocks of 64, 192 and 128 elements; N a partial tile."""
     N = 392
     x = synth.to_bf16(synth.small_like("heavy", M, M, K))
     x32 = synth.bf16_to_f32(x)
