@@ -266,6 +266,9 @@ Q4_API q4_status q4_sigma_delta_codebanks(q4_format format, int block, const flo
  *   K % 64 == 0 (K = 0 writes zeros); N % 8 == 0; M, N >= 0 arbitrary otherwise.
  *   workspace: device scratch of ws_bytes >= q4_gemm_workspace_size(...)
  *     (0 bytes for Q4_A_QUANTIZED); its contents on entry do not matter.
+ *     Q4_A_BF16 with M <= 16 and 256 <= K (up to about 16k: the quantized
+ *     activations stay resident in shared memory) runs the fused decode kernel
+ *     and needs none; other shapes quantize A once into the workspace.
  */
 Q4_API q4_status q4_gemm(q4_format format, int block, int64_t M, int64_t N, int64_t K,
                   int a_kind, const void* a, const uint8_t* a_scales,
